@@ -1,0 +1,356 @@
+#!/usr/bin/env python
+"""Throughput of the hashed n-gram embedding lookup on B200 (one JSON line on rank 0).
+
+A step is one pass of the whole path -- remap + hash, gather, projections, gate + conv +
+residual -- over one batch of the workload (default: the Engram layer at hidden 2560,
+8 x 4096 tokens, 16 tables of 999,983 rows x 160).  Inputs are resident in HBM when the
+timed region starts; the e2e figure repeats the measurement through the same public call
+with the inputs copied from pinned host memory and the output copied back every step.
+
+Multi-GPU (torchrun): every rank runs its own replica on its own batch (the lookup has no
+cross-token exchange), so scaling is weak; time is the max over ranks.
+
+--impl reference times the CPU oracle (the only reference this method has) on a bounded
+sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    sm_max=d.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, sm_max=1965.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "engram":
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle on a bounded sample (the reference arm and the cpu_baseline object)
+def oracle_sample(wl, n_tok_sample: int, seq: int = 0):
+    """Time the oracle's steps (remap, hash, gather, gate + conv + residual) on the first
+    n_tok_sample tokens of sequence `seq`.  Table rows are regenerated from the seeded
+    generator before the clock starts (the tables are never materialised on the host)."""
+    import oracle
+    b = seq % wl.B
+    T = min(wl.T, n_tok_sample)
+    ids = wl.ids()[b:b + 1, :T]
+    remap = wl.remap()
+    t_gen0 = time.perf_counter()
+    idx_probe = oracle.hash_ids(remap[ids], wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id)
+    tables = [synth.fill_rows_bf16(wl.table_spec(h), wl.d_e, idx_probe[:, h]) for h in range(wl.H)]
+    local_idx = np.tile(np.arange(T, dtype=np.uint32)[:, None], (1, wl.H))
+    h = synth.fill_rows_bf16(wl.h_spec(0), wl.d_h, b * wl.T + np.arange(T))
+    Wk = synth.fill_bf16(wl.wk_spec(), (wl.d_h, wl.d_m))
+    Wv = synth.fill_bf16(wl.wv_spec(), (wl.d_h, wl.d_m))
+    one = np.full(wl.d_h, 0x3F80, dtype=np.uint16)
+    cw = synth.fill_bf16(wl.conv_spec(), (wl.d_h, wl.conv_kernel))
+    t_gen = time.perf_counter() - t_gen0
+    t0 = time.perf_counter()
+    xr = oracle.remap(ids, remap)
+    idx = oracle.hash_ids(xr, wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id)
+    m = oracle.gather(local_idx, tables)      # compact tables hold exactly the rows idx names
+    oracle.gate_conv(h, m, Wk, Wv, one, one, one, cw, 1, T, dil=wl.conv_dilation, eps=wl.eps)
+    dt = time.perf_counter() - t0
+    assert np.array_equal(idx, idx_probe)
+    return T, dt, t_gen
+
+
+def run_reference(args, wl, world, rank):
+    """Reference arm: the CPU oracle, rank 0 only, one bounded sample per step."""
+    if rank != 0:
+        return
+    for k in range(args.warmup):
+        oracle_sample(wl, min(16, args.oracle_tokens), seq=k)
+    times, T, t_gen = [], 0, 0.0
+    for k in range(args.steps):
+        T, dt, tg = oracle_sample(wl, args.oracle_tokens, seq=k)
+        times.append(dt)
+        t_gen += tg
+    tps = T * len(times) / sum(times)
+    sample = (f"{args.steps} samples of 1 sequence x {T} tokens of {wl.name}; fp64 scalar C, 1 thread; "
+              f"table-row regeneration ({t_gen:.2f} s total) not timed")
+    line = {
+        "impl": "reference", "metric": "engram_tokens_per_s", "value": tps, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.mean(times) * 1e3 * wl.n_tok / T,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, world),
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, world):
+    return {"workload": wl.name, "tokens_per_step_per_gpu": wl.n_tok, "B": wl.B, "T": wl.T,
+            "orders": list(wl.orders), "K": wl.K, "H": wl.H, "table_rows": wl.primes[0], "d_e": wl.d_e,
+            "d_m": wl.d_m, "d_h": wl.d_h, "table_GiB": round(wl.table_bytes / 2 ** 30, 2),
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (hidden states, memory vectors and tables each exceed 126 MB)"
+            if wl.n_tok * wl.d_h * 2 > L2_BYTES else "inputs smaller than L2; L2 not flushed"}
+
+
+# ---------------------------------------------------------------------------------------
+def run_engram(args, wl, world, rank, local):
+    import hashed_gram_embedding_remap_b200 as E
+    from synth import fill_gpu
+
+    dev = f"cuda:{local}"
+    torch.cuda.set_device(local)
+    fill_gpu.build()
+    stream = torch.cuda.current_stream()
+    free, _ = torch.cuda.mem_get_info()
+    need = wl.table_bytes + 4 * wl.n_tok * (wl.d_h * 8 + wl.d_m * 2)
+    if need > free:
+        raise SystemExit(f"not enough device memory: need ~{need / 2**30:.1f} GiB, free {free / 2**30:.1f} GiB")
+    # per-rank input: each rank draws its own batch (seed offset by rank)
+    tables = [fill_gpu.filled((wl.primes[h], wl.d_e), wl.table_spec(h), dev) for h in range(wl.H)]
+    ids_np = wl.ids(step=rank)
+    ids = torch.from_numpy(ids_np).to(dev)
+    remap = None if wl.identity_remap else torch.from_numpy(wl.remap()).to(dev)
+    h = fill_gpu.filled((wl.n_tok, wl.d_h), wl.h_spec(rank), dev)
+    wk = fill_gpu.filled((wl.d_h, wl.d_m), wl.wk_spec(), dev)
+    wv = fill_gpu.filled((wl.d_h, wl.d_m), wl.wv_spec(), dev)
+    one = torch.full((wl.d_h,), 0x3F80, dtype=torch.int16, device=dev).view(torch.bfloat16)
+    cw = fill_gpu.filled((wl.d_h, wl.conv_kernel), wl.conv_spec(), dev)
+    history = torch.from_numpy(wl.history()).to(dev) if wl.decode else None
+    state = fill_gpu.filled((wl.B, wl.state_len, wl.d_h), wl.state_spec(), dev) if wl.decode else None
+    plan = E.Plan.from_workload(wl)
+    weights = E.Weights(wk, wv, one, one, one, cw)
+    out = torch.empty((wl.n_tok, wl.d_h), dtype=torch.bfloat16, device=dev)
+    ws = E.alloc_workspace(plan, wl.n_tok, dev)
+    nstage = E.ENGRAM_FORWARD_STAGES + 1
+
+    def step(evs=None):
+        E.engram_forward(plan, weights, tables, ids, h, out, ws, remap=remap, history=history,
+                         conv_state=state, stream=stream, stage_events=evs)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    E.engram_device_status(clear=True)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage)] for _ in range(args.steps)]
+    for row in evs:          # create the events before the timed region
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = start.elapsed_time(stop)
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    stage_names = ["hash", "gather", "proj", "gate_conv"]
+    stage_ms = {n: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
+                for i, n in enumerate(stage_names)}
+    status = E.engram_device_status(clear=True)
+    if status:
+        raise SystemExit(f"device status {status:#x} after the timed region")
+
+    # ---- e2e: inputs from pinned host memory, result back to pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        ids_host = torch.from_numpy(ids_np).pin_memory()
+        h_host = torch.empty((wl.n_tok, wl.d_h), dtype=torch.bfloat16).pin_memory()
+        h_host.copy_(h.cpu())
+        out_host = torch.empty((wl.n_tok, wl.d_h), dtype=torch.bfloat16).pin_memory()
+        ids_dev2 = torch.empty_like(ids)
+        h_dev2 = torch.empty_like(h)
+
+        def e2e_step():
+            ids_dev2.copy_(ids_host, non_blocking=True)
+            h_dev2.copy_(h_host, non_blocking=True)
+            E.engram_forward(plan, weights, tables, ids_dev2, h_dev2, out, ws, remap=remap, history=history,
+                             conv_state=state, stream=stream)
+            out_host.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        t2.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(s2.elapsed_time(t2), world)
+        h2d = ids_host.numel() * 4 + h_host.numel() * 2
+        d2h = out_host.numel() * 2
+        e2e = {"value": wl.n_tok * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    peaks = load_peaks()
+    n_tok = wl.n_tok
+    flops = 2.0 * n_tok * wl.d_m * 2 * wl.d_h
+    proj_s = stage_ms["proj"] / 1e3
+    tflops = flops / proj_s / 1e12
+    roofline = {"bound": "tensor", "kernel": "proj_kernel (tcgen05 k/v projections + gate partials)",
+                "achieved": tflops, "peak": peaks["bf16_sus"], "unit": "TFLOP/s", "frac": tflops / peaks["bf16_sus"],
+                "traffic": None, "peak_source": f"{peaks['source']} bf16 sustained",
+                "algorithmic_per_launch": flops}
+    # HBM view of the memory-bound kernels (gather and gate+conv)
+    row_bytes = wl.H * wl.d_e * 2
+    gather_bytes = n_tok * (row_bytes * 2 + wl.H * 4)            # rows read + m written + row ids
+    gate_bytes = n_tok * (wl.d_h * 4 + wl.d_h * 2 * 2)            # v read, h read, out written
+    hbm = {"gather_GBps": gather_bytes / (stage_ms["gather"] / 1e3) / 1e9,
+           "gate_conv_GBps": gate_bytes / (stage_ms["gate_conv"] / 1e3) / 1e9,
+           "peak_GBps": peaks["hbm"], "nominal_GBps": 8000.0}
+    hbm["gather_frac"] = hbm["gather_GBps"] / peaks["hbm"]
+    hbm["gate_conv_frac"] = hbm["gate_conv_GBps"] / peaks["hbm"]
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        T, dt, t_gen = oracle_sample(wl, args.cpu_baseline_tokens)
+        cpu = {"value": T / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"1 sequence x {T} tokens of {wl.name}; fp64 scalar C, 1 thread; "
+                         f"table-row regeneration ({t_gen:.2f} s) not timed"}
+
+    value = n_tok * world * args.steps / (elapsed_ms / 1e3)
+    line = {
+        "metric": "engram_tokens_per_s", "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Zipf ids, counter-based bf16 tables/weights)",
+        "config": workload_config(wl, world),
+        "stages_ms": stage_ms, "hbm": hbm, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": args.steps * (E.ENGRAM_FORWARD_STAGES + (1 if wl.decode else 0)),
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["engram", "reference"], default="engram")
+    ap.add_argument("--workload", default="layer2560", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--oracle-tokens", type=int, default=128)
+    ap.add_argument("--cpu-baseline-tokens", type=int, default=768)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = synth.get_workload(args.workload)
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, wl, world, rank)
+        else:
+            run_engram(args, wl, world, rank, local)
+    finally:
+        if world > 1 and args.impl == "engram":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,14 @@
+"""B200-native hashed n-gram embedding lookup (Engram / N-gram Embedding).
+
+The computation lives in ``libengram.so`` (hand-written CUDA for sm_100a behind a C ABI,
+declared in ``include/engram.h``).  This package is its thin Python binding; it never
+computes a step itself and has no CPU fallback.
+"""
+from ._native import (  # noqa: F401
+    ENGRAM_ERR_CUDA, ENGRAM_ERR_INVALID_ARG, ENGRAM_ERR_OOM, ENGRAM_ERR_TIMEOUT,
+    ENGRAM_ERR_UNSUPPORTED, ENGRAM_FORWARD_STAGES, ENGRAM_OK, ENGRAM_STATUS_BAD_ROW,
+    ENGRAM_STATUS_BAD_TOKEN, ENGRAM_STATUS_WAIT_TIMEOUT, ENGRAM_TABLES_DEVICE,
+    ENGRAM_TABLES_HOST_MAPPED, EngramError, LIB_PATH, Plan, Weights, alloc_workspace,
+    engram_advance_history, engram_device_status, engram_forward, engram_gate_conv,
+    engram_gather, engram_hash, engram_remap, engram_workspace_size, last_error, lib, version,
+)

@@ -1,0 +1,296 @@
+"""ctypes binding of the C ABI in include/engram.h (argument marshalling only).
+
+Every function here forwards to the same-named entry point of ``libengram.so``; all the
+computation runs in the library's CUDA kernels.  There is no fallback: if the shared
+library is missing or cannot be loaded, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libengram.so")
+
+ENGRAM_OK = 0
+ENGRAM_ERR_INVALID_ARG = -1
+ENGRAM_ERR_UNSUPPORTED = -2
+ENGRAM_ERR_CUDA = -3
+ENGRAM_ERR_OOM = -4
+ENGRAM_ERR_TIMEOUT = -5
+ENGRAM_STATUS_BAD_TOKEN = 0x1
+ENGRAM_STATUS_BAD_ROW = 0x2
+ENGRAM_STATUS_WAIT_TIMEOUT = 0x4
+ENGRAM_MAX_ORDERS = 4
+ENGRAM_MAX_TABLES = 32
+ENGRAM_FORWARD_STAGES = 4
+ENGRAM_TABLES_DEVICE = 0
+ENGRAM_TABLES_HOST_MAPPED = 1
+
+_ERRNAMES = {-1: "ENGRAM_ERR_INVALID_ARG", -2: "ENGRAM_ERR_UNSUPPORTED", -3: "ENGRAM_ERR_CUDA",
+             -4: "ENGRAM_ERR_OOM", -5: "ENGRAM_ERR_TIMEOUT"}
+
+
+class EngramError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{_ERRNAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+class engram_config(C.Structure):
+    _fields_ = [
+        ("num_orders", C.c_int32),
+        ("orders", C.c_int32 * ENGRAM_MAX_ORDERS),
+        ("heads_per_order", C.c_int32),
+        ("table_rows", C.c_int64 * ENGRAM_MAX_TABLES),
+        ("row_dim", C.c_int32),
+        ("hidden_dim", C.c_int32),
+        ("vocab_in", C.c_int32),
+        ("vocab_out", C.c_int32),
+        ("pad_id", C.c_int32),
+        ("conv_kernel", C.c_int32),
+        ("conv_dilation", C.c_int32),
+        ("table_location", C.c_int32),
+        ("hash_seed", C.c_uint64),
+        ("eps", C.c_float),
+        ("reserved", C.c_int32 * 7),
+    ]
+
+
+class engram_plan(C.Structure):
+    _fields_ = [
+        ("cfg", engram_config),
+        ("mult", (C.c_uint64 * ENGRAM_MAX_ORDERS) * ENGRAM_MAX_TABLES),
+        ("num_tables", C.c_int32),
+        ("mem_dim", C.c_int32),
+        ("hist_len", C.c_int32),
+        ("state_len", C.c_int32),
+        ("magic", C.c_uint32),
+        ("reserved", C.c_int32 * 3),
+    ]
+
+
+class engram_weights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("w_k", "w_v", "gamma_q", "gamma_k", "gamma_c", "conv_w")]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"CUDA library not built: {LIB_PATH} is missing "
+                          "(run __graft_entry__.build() or python -m hashed_gram_embedding_remap_b200.build)")
+    L = C.CDLL(LIB_PATH)
+    P, i32, i64, sz = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t
+    sig = {
+        "engram_init": (C.c_int, [P, P]),
+        "engram_workspace_size": (sz, [P, i64]),
+        "engram_remap": (C.c_int, [P, P, i64, P, P, P]),
+        "engram_hash": (C.c_int, [P, P, i32, i32, P, P, P]),
+        "engram_advance_history": (C.c_int, [P, P, i32, i32, P, P]),
+        "engram_gather": (C.c_int, [P, P, P, i64, P, P]),
+        "engram_gate_conv": (C.c_int, [P, P, P, P, i32, i32, P, P, P, P, sz, P]),
+        "engram_forward": (C.c_int, [P, P, P, P, P, i32, i32, P, P, P, P, P, P, sz, P, P]),
+        "engram_device_status": (C.c_int, [P, C.c_int]),
+        "engram_last_error": (C.c_char_p, []),
+        "engram_version": (C.c_char_p, []),
+        "engram_sizeof": (sz, [C.c_char_p]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    for name, cls in (("engram_config", engram_config), ("engram_plan", engram_plan),
+                      ("engram_weights", engram_weights)):
+        n = L.engram_sizeof(name.encode())
+        if n != C.sizeof(cls):
+            raise ImportError(f"ABI mismatch: sizeof({name}) is {n} in the library, {C.sizeof(cls)} here")
+    return L
+
+
+lib = _load()
+
+
+def last_error() -> str:
+    return lib.engram_last_error().decode()
+
+
+def version() -> str:
+    return lib.engram_version().decode()
+
+
+def _check(rc: int):
+    if rc != ENGRAM_OK:
+        raise EngramError(rc, last_error())
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> C.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+_BF16 = (torch.bfloat16, torch.int16, torch.uint16)
+
+
+# ---------------------------------------------------------------------------------------
+class Plan:
+    """A validated lookup configuration (engram_plan), built by engram_init."""
+
+    def __init__(self, *, orders: Sequence[int], heads_per_order: int, table_rows: Sequence[int],
+                 row_dim: int, hidden_dim: int, vocab_in: int, vocab_out: int, hash_seed: int,
+                 eps: float = 1e-6, conv_kernel: int = 4, table_location: int = ENGRAM_TABLES_DEVICE):
+        cfg = engram_config()
+        cfg.num_orders = len(orders)
+        for i, o in enumerate(orders):
+            cfg.orders[i] = int(o)
+        cfg.heads_per_order = int(heads_per_order)
+        for i, p in enumerate(table_rows):
+            cfg.table_rows[i] = int(p)
+        cfg.row_dim = int(row_dim)
+        cfg.hidden_dim = int(hidden_dim)
+        cfg.vocab_in = int(vocab_in)
+        cfg.vocab_out = int(vocab_out)
+        cfg.pad_id = int(vocab_out)
+        cfg.conv_kernel = int(conv_kernel)
+        cfg.conv_dilation = int(max(orders)) if len(orders) else 0
+        cfg.table_location = int(table_location)
+        cfg.hash_seed = int(hash_seed) & 0xFFFFFFFFFFFFFFFF
+        cfg.eps = float(eps)
+        self.cfg = cfg
+        self.plan = engram_plan()
+        _check(lib.engram_init(C.byref(cfg), C.byref(self.plan)))
+
+    @classmethod
+    def from_workload(cls, wl, **kw) -> "Plan":
+        loc = ENGRAM_TABLES_HOST_MAPPED if kw.pop("host_tables", False) else ENGRAM_TABLES_DEVICE
+        return cls(orders=wl.orders, heads_per_order=wl.K, table_rows=wl.primes, row_dim=wl.d_e,
+                   hidden_dim=wl.d_h, vocab_in=wl.vocab_in, vocab_out=wl.vocab_out,
+                   hash_seed=wl.hash_seed, eps=wl.eps, conv_kernel=wl.conv_kernel,
+                   table_location=loc, **kw)
+
+    @property
+    def num_tables(self) -> int:
+        return self.plan.num_tables
+
+    @property
+    def mem_dim(self) -> int:
+        return self.plan.mem_dim
+
+    @property
+    def hist_len(self) -> int:
+        return self.plan.hist_len
+
+    @property
+    def state_len(self) -> int:
+        return self.plan.state_len
+
+    @property
+    def _as_parameter_(self):
+        return C.byref(self.plan)
+
+
+class Weights:
+    """Device tensors of the gate and conv, bundled as engram_weights."""
+
+    def __init__(self, w_k, w_v, gamma_q, gamma_k, gamma_c, conv_w):
+        self.tensors = (w_k, w_v, gamma_q, gamma_k, gamma_c, conv_w)
+        names = ("w_k", "w_v", "gamma_q", "gamma_k", "gamma_c", "conv_w")
+        self.struct = engram_weights(*[_ptr(t, _BF16, n) for t, n in zip(self.tensors, names)])
+
+    @property
+    def _as_parameter_(self):
+        return C.byref(self.struct)
+
+
+def _table_array(tables):
+    arr = (C.c_void_p * len(tables))()
+    for i, t in enumerate(tables):
+        arr[i] = t if isinstance(t, int) else t.data_ptr()
+    return arr
+
+
+# ---------------------------------------------------------------------------------------
+def engram_workspace_size(plan: Plan, n_tok: int) -> int:
+    return int(lib.engram_workspace_size(plan, int(n_tok)))
+
+
+def engram_remap(plan: Plan, ids: torch.Tensor, remap: torch.Tensor, out: torch.Tensor, stream=None):
+    _check(lib.engram_remap(plan, _ptr(ids, torch.int32, "ids"), ids.numel(),
+                            _ptr(remap, torch.int32, "remap"), _ptr(out, torch.int32, "out"),
+                            _stream(stream)))
+
+
+def engram_hash(plan: Plan, ids_remapped: torch.Tensor, idx: torch.Tensor,
+                history: Optional[torch.Tensor] = None, stream=None):
+    B, T = ids_remapped.shape
+    _check(lib.engram_hash(plan, _ptr(ids_remapped, torch.int32, "ids_remapped"), B, T,
+                           _ptr(history, torch.int32, "history"),
+                           _ptr(idx, (torch.int32, torch.uint32), "idx"), _stream(stream)))
+
+
+def engram_advance_history(plan: Plan, ids_remapped: torch.Tensor, history: torch.Tensor, stream=None):
+    B, T = ids_remapped.shape
+    _check(lib.engram_advance_history(plan, _ptr(ids_remapped, torch.int32, "ids_remapped"), B, T,
+                                      _ptr(history, torch.int32, "history"), _stream(stream)))
+
+
+def engram_gather(plan: Plan, idx: torch.Tensor, tables, m: torch.Tensor, stream=None):
+    arr = _table_array(tables)
+    _check(lib.engram_gather(plan, _ptr(idx, (torch.int32, torch.uint32), "idx"), arr, idx.shape[0],
+                             _ptr(m, _BF16, "m"), _stream(stream)))
+
+
+def engram_gate_conv(plan: Plan, weights: Weights, h: torch.Tensor, m: torch.Tensor, B: int, T: int,
+                     out: torch.Tensor, workspace: torch.Tensor, conv_state: Optional[torch.Tensor] = None,
+                     delta_dbg: Optional[torch.Tensor] = None, stream=None):
+    _check(lib.engram_gate_conv(plan, weights, _ptr(h, _BF16, "h"), _ptr(m, _BF16, "m"), B, T,
+                                _ptr(conv_state, _BF16, "conv_state"), _ptr(out, _BF16, "out"),
+                                _ptr(delta_dbg, torch.float32, "delta_dbg"),
+                                _ptr(workspace, None, "workspace"),
+                                workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def engram_forward(plan: Plan, weights: Weights, tables, ids: torch.Tensor, h: torch.Tensor,
+                   out: torch.Tensor, workspace: torch.Tensor, remap: Optional[torch.Tensor] = None,
+                   history: Optional[torch.Tensor] = None, conv_state: Optional[torch.Tensor] = None,
+                   delta_dbg: Optional[torch.Tensor] = None, stream=None, stage_events=None):
+    B, T = ids.shape
+    arr = _table_array(tables)
+    ev = None
+    if stage_events is not None:
+        if len(stage_events) != ENGRAM_FORWARD_STAGES + 1:
+            raise ValueError(f"stage_events needs {ENGRAM_FORWARD_STAGES + 1} events")
+        ev = (C.c_void_p * len(stage_events))(*[e._as_parameter_.value for e in stage_events])
+    _check(lib.engram_forward(plan, weights, arr, _ptr(ids, torch.int32, "ids"),
+                              _ptr(remap, torch.int32, "remap"), B, T,
+                              _ptr(history, torch.int32, "history"), _ptr(conv_state, _BF16, "conv_state"),
+                              _ptr(h, _BF16, "h"), _ptr(out, _BF16, "out"),
+                              _ptr(delta_dbg, torch.float32, "delta_dbg"), _ptr(workspace, None, "workspace"),
+                              workspace.numel() * workspace.element_size(), _stream(stream), ev))
+
+
+def engram_device_status(clear: bool = True) -> int:
+    s = C.c_uint32(0)
+    _check(lib.engram_device_status(C.byref(s), int(clear)))
+    return int(s.value)
+
+
+def alloc_workspace(plan: Plan, n_tok: int, device="cuda") -> torch.Tensor:
+    """A workspace tensor of the size engram_workspace_size reports (torch allocations are
+    at least 256-byte aligned)."""
+    n = engram_workspace_size(plan, n_tok)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)

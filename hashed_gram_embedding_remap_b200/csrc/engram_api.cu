@@ -1,0 +1,574 @@
+// Host side of the C ABI declared in include/engram.h: validation, derived constants,
+// workspace layout, TMA descriptor encoding and kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "engram.h"
+#include "kernels_gate.cuh"
+#include "kernels_lookup.cuh"
+#include "ptx.cuh"
+
+namespace {
+
+constexpr uint32_t kPlanMagic = 0xE9A7B200u;
+thread_local std::string g_last_error;
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(ENGRAM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define ENGRAM_CUDA_TRY(expr, what)              \
+    do {                                         \
+        cudaError_t e_ = (expr);                 \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+    } while (0)
+
+// ---------------------------------------------------------------- host-side integer helpers
+uint64_t splitmix64_first(uint64_t state) {
+    uint64_t z = state + 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+uint64_t mulmod(uint64_t a, uint64_t b, uint64_t m) {
+    return static_cast<uint64_t>((static_cast<unsigned __int128>(a) * b) % m);
+}
+
+uint64_t powmod(uint64_t a, uint64_t e, uint64_t m) {
+    uint64_t r = 1 % m;
+    a %= m;
+    while (e) {
+        if (e & 1) r = mulmod(r, a, m);
+        a = mulmod(a, a, m);
+        e >>= 1;
+    }
+    return r;
+}
+
+// Deterministic Miller-Rabin for n < 2^32 (witnesses 2, 7, 61).
+bool is_prime_u32(uint64_t n) {
+    if (n < 2) return false;
+    for (uint64_t p : {2ull, 3ull, 5ull, 7ull, 11ull, 13ull, 61ull}) {
+        if (n % p == 0) return n == p;
+    }
+    uint64_t d = n - 1;
+    int r = 0;
+    while ((d & 1) == 0) {
+        d >>= 1;
+        ++r;
+    }
+    for (uint64_t a : {2ull, 7ull, 61ull}) {
+        uint64_t x = powmod(a, d, n);
+        if (x == 1 || x == n - 1) continue;
+        bool comp = true;
+        for (int i = 1; i < r; ++i) {
+            x = mulmod(x, x, n);
+            if (x == n - 1) {
+                comp = false;
+                break;
+            }
+        }
+        if (comp) return false;
+    }
+    return true;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_plan(const engram_plan *plan) {
+    if (plan == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "plan is NULL");
+    if (plan->magic != kPlanMagic) return fail(ENGRAM_ERR_INVALID_ARG, "plan was not initialised by engram_init");
+    return ENGRAM_OK;
+}
+
+// ---------------------------------------------------------------- workspace layout
+struct Workspace {
+    size_t xr, idx, m, v, part, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Width of the projection's N tile: the widest of 256/128/64 that divides d_h and still
+// gives at least two waves of CTAs on the GPU.  ENGRAM_PROJ_TILE_N (64, 128 or 256) forces a
+// width (for tuning and tests); it is read once per process.
+int choose_bn(int d_h, int64_t n_tok) {
+    static const int forced = [] {
+        const char *e = std::getenv("ENGRAM_PROJ_TILE_N");
+        const int v = e ? std::atoi(e) : 0;
+        return (v == 64 || v == 128 || v == 256) ? v : 0;
+    }();
+    if (forced && d_h % forced == 0) return forced;
+    const int64_t m_tiles = (n_tok + engram::kBM - 1) / engram::kBM;
+    const int cands[3] = {256, 128, 64};
+    for (int bn : cands) {
+        if (d_h % bn != 0) continue;
+        if (bn == 64 || m_tiles * (2 * d_h / bn) >= 2 * 148) return bn;
+    }
+    return 64;
+}
+
+Workspace layout(const engram_plan *plan, int64_t n_tok) {
+    Workspace w{};
+    const int H = plan->num_tables;
+    const int d_h = plan->cfg.hidden_dim;
+    const int bn = choose_bn(d_h, n_tok);
+    const int n_tiles = 2 * d_h / bn;
+    size_t off = 0;
+    w.xr = off;   off = align256(off + sizeof(int32_t) * n_tok);
+    w.idx = off;  off = align256(off + sizeof(uint32_t) * n_tok * H);
+    w.m = off;    off = align256(off + sizeof(uint16_t) * n_tok * plan->mem_dim);
+    w.v = off;    off = align256(off + sizeof(float) * n_tok * d_h);
+    w.part = off; off = align256(off + sizeof(float4) * n_tok * n_tiles);
+    w.total = off;
+    return w;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Row-major bf16 [rows, cols] -> tensor map with a box of box_rows x 64 columns (128 B),
+// 128-byte swizzle, zero fill outside the tensor.
+int make_map_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto enc = get_encode_fn();
+    if (enc == nullptr) return fail(ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(engram::kBK), box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return ENGRAM_OK;
+}
+
+template <int BN>
+int set_proj_smem_attr() {
+    // Per device: the attribute is a property of the function on the current device.
+    static bool done[64] = {};
+    int dev = 0;
+    ENGRAM_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev < 64 && done[dev]) return ENGRAM_OK;
+    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::proj_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         engram::ProjCfg<BN>::kSmemBytes),
+                    "cudaFuncSetAttribute(proj_kernel)");
+    if (dev < 64) done[dev] = true;
+    return ENGRAM_OK;
+}
+
+template <int BN>
+int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
+                int64_t n_tok, float *v, float4 *part, cudaStream_t stream) {
+    const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim;
+    CUtensorMap map_m, map_wk, map_wv;
+    int rc;
+    if ((rc = make_map_bf16(&map_m, m, static_cast<uint64_t>(n_tok), d_m, engram::kBM)) != ENGRAM_OK) return rc;
+    if ((rc = make_map_bf16(&map_wk, w->w_k, d_h, d_m, BN)) != ENGRAM_OK) return rc;
+    if ((rc = make_map_bf16(&map_wv, w->w_v, d_h, d_m, BN)) != ENGRAM_OK) return rc;
+    if ((rc = set_proj_smem_attr<BN>()) != ENGRAM_OK) return rc;
+    engram::ProjParams p{};
+    p.h = h;
+    p.gamma_q = w->gamma_q;
+    p.gamma_k = w->gamma_k;
+    p.v = v;
+    p.part = part;
+    p.n_tok = n_tok;
+    p.d_m = d_m;
+    p.d_h = d_h;
+    p.n_tiles = 2 * d_h / BN;
+    p.k_blocks = (d_m + engram::kBK - 1) / engram::kBK;
+    dim3 grid(p.n_tiles, static_cast<unsigned>((n_tok + engram::kBM - 1) / engram::kBM));
+    engram::proj_kernel<BN><<<grid, engram::kProjThreads, engram::ProjCfg<BN>::kSmemBytes, stream>>>(
+        map_m, map_wk, map_wv, p);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "proj_kernel launch");
+    return ENGRAM_OK;
+}
+
+int validate_weights(const engram_plan *plan, const engram_weights *w) {
+    if (w == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "weights is NULL");
+    const void *ptrs[6] = {w->w_k, w->w_v, w->gamma_q, w->gamma_k, w->gamma_c, w->conv_w};
+    const char *names[6] = {"w_k", "w_v", "gamma_q", "gamma_k", "gamma_c", "conv_w"};
+    for (int i = 0; i < 6; ++i) {
+        if (ptrs[i] == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "weights.%s is NULL", names[i]);
+        if (i < 2 && !aligned16(ptrs[i])) return fail(ENGRAM_ERR_INVALID_ARG, "weights.%s is not 16-byte aligned", names[i]);
+        if (i >= 2 && (reinterpret_cast<uintptr_t>(ptrs[i]) & 7u))
+            return fail(ENGRAM_ERR_INVALID_ARG, "weights.%s is not 8-byte aligned", names[i]);
+    }
+    (void)plan;
+    return ENGRAM_OK;
+}
+
+int launch_hash(const engram_plan *plan, const int32_t *ids, const int32_t *remap, const int32_t *history,
+                int32_t B, int32_t T, uint32_t *idx, int32_t *xr_out, cudaStream_t stream) {
+    engram::HashParams p{};
+    const engram_config &c = plan->cfg;
+    const int K = c.heads_per_order;
+    for (int oi = 0; oi < c.num_orders; ++oi)
+        for (int j = 0; j < K; ++j) {
+            const int h = oi * K + j;
+            p.order[h] = c.orders[oi];
+            p.prime[h] = static_cast<uint64_t>(c.table_rows[h]);
+            for (int i = 0; i < ENGRAM_MAX_ORDERS; ++i) p.mult[h][i] = plan->mult[h][i];
+        }
+    p.H = plan->num_tables;
+    p.max_order = c.orders[c.num_orders - 1];
+    p.hist_len = plan->hist_len;
+    p.pad_id = c.pad_id;
+    p.vocab_in = c.vocab_in;
+    p.B = B;
+    p.T = T;
+    const int64_t n_tok = static_cast<int64_t>(B) * T;
+    const int threads = 256;
+    const unsigned blocks = static_cast<unsigned>((n_tok + threads - 1) / threads);
+    engram::hash_kernel<<<blocks, threads, 0, stream>>>(ids, remap, history, idx, xr_out, p);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "hash_kernel launch");
+    return ENGRAM_OK;
+}
+
+int sm_count() {
+    static int count[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 64 && count[dev]) return count[dev];
+    int n = 148;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (dev < 64) count[dev] = n;
+    return n;
+}
+
+int launch_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables, int64_t n_tok,
+                  uint16_t *m, cudaStream_t stream) {
+    engram::GatherParams p{};
+    const int H = plan->num_tables;
+    for (int h = 0; h < H; ++h) {
+        p.table[h] = tables[h];
+        p.rows[h] = static_cast<uint64_t>(plan->cfg.table_rows[h]);
+    }
+    p.H = H;
+    p.chunks_per_row = plan->cfg.row_dim / 8;
+    p.chunks_per_tok = H * p.chunks_per_row;
+    p.n_tok = n_tok;
+    const int64_t total = n_tok * p.chunks_per_tok;
+    constexpr int kUnroll = 4;
+    const int threads = 256;
+    int64_t blocks = (total + threads * kUnroll - 1) / (threads * kUnroll);
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;  // 8 x 256 threads resident per SM
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    engram::gather_kernel<kUnroll><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        idx, reinterpret_cast<uint4 *>(m), p);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "gather_kernel launch");
+    return ENGRAM_OK;
+}
+
+int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const float *v,
+                     const float4 *part, int n_tiles, int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out,
+                     float *delta, cudaStream_t stream) {
+    engram::GateParams p{};
+    const int d_h = plan->cfg.hidden_dim;
+    p.h = h;
+    p.v = v;
+    p.part = part;
+    p.gamma_c = w->gamma_c;
+    p.conv_w = w->conv_w;
+    p.conv_state = conv_state;
+    p.out = out;
+    p.delta = delta;
+    p.B = B;
+    p.T = T;
+    p.d_h = d_h;
+    p.n_tiles = n_tiles;
+    p.n_key_tiles = n_tiles / 2;
+    p.ksize = plan->cfg.conv_kernel;
+    p.dil = plan->cfg.conv_dilation;
+    p.state_len = plan->state_len;
+    p.tok_chunk = conv_state != nullptr ? T : 32;
+    p.eps = plan->cfg.eps;
+    p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(d_h));
+    const int threads = engram::kGateThreads;
+    const unsigned slices = static_cast<unsigned>((d_h / 4 + threads - 1) / threads);
+    const size_t smem = sizeof(float) * 2 * static_cast<size_t>(p.tok_chunk + p.state_len);
+    if (smem > 48 * 1024) {
+        ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::gate_conv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem)),
+                        "cudaFuncSetAttribute(gate_conv_kernel)");
+    }
+    dim3 grid(static_cast<unsigned>((T + p.tok_chunk - 1) / p.tok_chunk), static_cast<unsigned>(B), slices);
+    engram::gate_conv_kernel<<<grid, threads, smem, stream>>>(p);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_conv_kernel launch");
+    return ENGRAM_OK;
+}
+
+int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
+                   int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out, float *delta, uint8_t *ws,
+                   cudaStream_t stream, void *const *events) {
+    const int64_t n_tok = static_cast<int64_t>(B) * T;
+    const Workspace L = layout(plan, n_tok);
+    const int d_h = plan->cfg.hidden_dim;
+    const int bn = choose_bn(d_h, n_tok);
+    float *v = reinterpret_cast<float *>(ws + L.v);
+    float4 *part = reinterpret_cast<float4 *>(ws + L.part);
+    int rc;
+    if (events) ENGRAM_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), stream), "cudaEventRecord");
+    if (bn == 256) rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream);
+    else if (bn == 128) rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream);
+    else rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream);
+    if (rc != ENGRAM_OK) return rc;
+    if (events) ENGRAM_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), stream), "cudaEventRecord");
+    return launch_gate_conv(plan, w, h, v, part, 2 * d_h / bn, B, T, conv_state, out, delta, stream);
+}
+
+int check_bt(int32_t B, int32_t T) {
+    if (B < 0 || T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "B and T must be >= 0 (got %d, %d)", B, T);
+    if (static_cast<int64_t>(B) * T > (int64_t(1) << 31))
+        return fail(ENGRAM_ERR_UNSUPPORTED, "B*T above 2^31 tokens per call");
+    if (B > 65535) return fail(ENGRAM_ERR_UNSUPPORTED, "B above 65535 sequences per call");
+    return ENGRAM_OK;
+}
+
+}  // namespace
+
+// =====================================================================================
+extern "C" {
+
+const char *engram_last_error(void) { return g_last_error.c_str(); }
+
+const char *engram_version(void) { return "0.1.0"; }
+
+size_t engram_sizeof(const char *type_name) {
+    if (type_name == nullptr) return 0;
+    if (std::strcmp(type_name, "engram_config") == 0) return sizeof(engram_config);
+    if (std::strcmp(type_name, "engram_plan") == 0) return sizeof(engram_plan);
+    if (std::strcmp(type_name, "engram_weights") == 0) return sizeof(engram_weights);
+    return 0;
+}
+
+int engram_init(const engram_config *cfg, engram_plan *plan) {
+    g_last_error.clear();
+    if (cfg == nullptr || plan == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "cfg and plan must be non-NULL");
+    const engram_config &c = *cfg;
+    if (c.num_orders < 1 || c.num_orders > ENGRAM_MAX_ORDERS)
+        return fail(ENGRAM_ERR_UNSUPPORTED, "num_orders must be in 1..%d", ENGRAM_MAX_ORDERS);
+    for (int i = 0; i < c.num_orders; ++i) {
+        if (c.orders[i] < 1 || c.orders[i] > ENGRAM_MAX_ORDERS)
+            return fail(ENGRAM_ERR_UNSUPPORTED, "order %d outside 1..%d", c.orders[i], ENGRAM_MAX_ORDERS);
+        if (i > 0 && c.orders[i] <= c.orders[i - 1])
+            return fail(ENGRAM_ERR_INVALID_ARG, "orders must be strictly increasing");
+    }
+    if (c.heads_per_order < 1) return fail(ENGRAM_ERR_INVALID_ARG, "heads_per_order must be >= 1");
+    const int H = c.num_orders * c.heads_per_order;
+    if (H > ENGRAM_MAX_TABLES) return fail(ENGRAM_ERR_UNSUPPORTED, "num_orders * heads_per_order > %d", ENGRAM_MAX_TABLES);
+    for (int h = 0; h < H; ++h) {
+        const int64_t P = c.table_rows[h];
+        if (P < 2 || P > 0xFFFFFFFFll) return fail(ENGRAM_ERR_INVALID_ARG, "table_rows[%d] = %lld outside [2, 2^32)", h, (long long)P);
+        if (!is_prime_u32(static_cast<uint64_t>(P)))
+            return fail(ENGRAM_ERR_INVALID_ARG, "table_rows[%d] = %lld is not prime", h, (long long)P);
+    }
+    for (int h = H; h < ENGRAM_MAX_TABLES; ++h)
+        if (c.table_rows[h] != 0) return fail(ENGRAM_ERR_INVALID_ARG, "table_rows[%d] set beyond the %d tables", h, H);
+    if (c.row_dim <= 0 || c.row_dim % 8 != 0) return fail(ENGRAM_ERR_UNSUPPORTED, "row_dim must be a positive multiple of 8");
+    if (c.hidden_dim <= 0 || c.hidden_dim % 64 != 0)
+        return fail(ENGRAM_ERR_UNSUPPORTED, "hidden_dim must be a positive multiple of 64");
+    if (static_cast<int64_t>(H) * c.row_dim > (1 << 20)) return fail(ENGRAM_ERR_UNSUPPORTED, "memory dim above 2^20");
+    if (c.vocab_in <= 0 || c.vocab_out <= 0) return fail(ENGRAM_ERR_INVALID_ARG, "vocab sizes must be positive");
+    if (c.vocab_out == 0x7FFFFFFF) return fail(ENGRAM_ERR_INVALID_ARG, "vocab_out too large (pad id must fit)");
+    if (c.pad_id != c.vocab_out) return fail(ENGRAM_ERR_INVALID_ARG, "pad_id must equal vocab_out");
+    if (c.conv_kernel < 1 || c.conv_kernel > 8) return fail(ENGRAM_ERR_UNSUPPORTED, "conv_kernel must be in 1..8");
+    if (c.conv_dilation != c.orders[c.num_orders - 1])
+        return fail(ENGRAM_ERR_INVALID_ARG, "conv_dilation must equal the largest order");
+    if (!(c.eps > 0.f) || !std::isfinite(c.eps)) return fail(ENGRAM_ERR_INVALID_ARG, "eps must be a positive finite number");
+    if (c.table_location != ENGRAM_TABLES_DEVICE && c.table_location != ENGRAM_TABLES_HOST_MAPPED)
+        return fail(ENGRAM_ERR_INVALID_ARG, "unknown table_location");
+    for (int i = 0; i < 7; ++i)
+        if (c.reserved[i] != 0) return fail(ENGRAM_ERR_INVALID_ARG, "reserved fields must be zero");
+
+    std::memset(plan, 0, sizeof *plan);
+    plan->cfg = c;
+    for (int oi = 0; oi < c.num_orders; ++oi)
+        for (int j = 0; j < c.heads_per_order; ++j)
+            for (int i = 0; i < c.orders[oi]; ++i) {
+                const uint64_t key = c.hash_seed ^ ((static_cast<uint64_t>(c.orders[oi]) << 16) ^
+                                                    (static_cast<uint64_t>(j) << 8) ^ static_cast<uint64_t>(i));
+                plan->mult[oi * c.heads_per_order + j][i] = splitmix64_first(key) | 1ull;
+            }
+    plan->num_tables = H;
+    plan->mem_dim = H * c.row_dim;
+    plan->hist_len = c.orders[c.num_orders - 1] - 1;
+    plan->state_len = (c.conv_kernel - 1) * c.conv_dilation;
+    plan->magic = kPlanMagic;
+    return ENGRAM_OK;
+}
+
+size_t engram_workspace_size(const engram_plan *plan, int64_t n_tok) {
+    if (plan == nullptr || plan->magic != kPlanMagic || n_tok < 0) return 0;
+    return layout(plan, n_tok).total;
+}
+
+int engram_remap(const engram_plan *plan, const int32_t *ids, int64_t n, const int32_t *remap, int32_t *out,
+                 engram_stream_t stream) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if (n < 0) return fail(ENGRAM_ERR_INVALID_ARG, "n must be >= 0");
+    if (n == 0) return ENGRAM_OK;
+    if (!ids || !remap || !out) return fail(ENGRAM_ERR_INVALID_ARG, "ids, remap and out must be non-NULL");
+    const int threads = 256;
+    int64_t blocks = (n + threads - 1) / threads;
+    if (blocks > 65535LL * 16) blocks = 65535LL * 16;
+    engram::remap_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        ids, n, remap, plan->cfg.vocab_in, plan->cfg.pad_id, out);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "remap_kernel launch");
+    return ENGRAM_OK;
+}
+
+int engram_hash(const engram_plan *plan, const int32_t *ids_remapped, int32_t B, int32_t T,
+                const int32_t *history, uint32_t *idx, engram_stream_t stream) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if ((rc = check_bt(B, T)) != ENGRAM_OK) return rc;
+    if (static_cast<int64_t>(B) * T == 0) return ENGRAM_OK;
+    if (!ids_remapped || !idx) return fail(ENGRAM_ERR_INVALID_ARG, "ids_remapped and idx must be non-NULL");
+    return launch_hash(plan, ids_remapped, nullptr, history, B, T, idx, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int engram_advance_history(const engram_plan *plan, const int32_t *ids_remapped, int32_t B, int32_t T,
+                           int32_t *history, engram_stream_t stream) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if ((rc = check_bt(B, T)) != ENGRAM_OK) return rc;
+    if (B == 0 || plan->hist_len == 0) return ENGRAM_OK;
+    if (!history || (T > 0 && !ids_remapped)) return fail(ENGRAM_ERR_INVALID_ARG, "history and ids must be non-NULL");
+    engram::advance_history_kernel<<<(B + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+        ids_remapped, B, T, history, plan->hist_len);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "advance_history_kernel launch");
+    return ENGRAM_OK;
+}
+
+int engram_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables, int64_t n_tok,
+                  uint16_t *m, engram_stream_t stream) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if (n_tok < 0) return fail(ENGRAM_ERR_INVALID_ARG, "n_tok must be >= 0");
+    if (n_tok == 0) return ENGRAM_OK;
+    if (!idx || !tables || !m) return fail(ENGRAM_ERR_INVALID_ARG, "idx, tables and m must be non-NULL");
+    if (!aligned16(m)) return fail(ENGRAM_ERR_INVALID_ARG, "m is not 16-byte aligned");
+    for (int h = 0; h < plan->num_tables; ++h) {
+        if (!tables[h]) return fail(ENGRAM_ERR_INVALID_ARG, "tables[%d] is NULL", h);
+        if (!aligned16(tables[h])) return fail(ENGRAM_ERR_INVALID_ARG, "tables[%d] is not 16-byte aligned", h);
+    }
+    return launch_gather(plan, idx, tables, n_tok, m, static_cast<cudaStream_t>(stream));
+}
+
+int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
+                     int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out, float *delta_dbg, void *workspace,
+                     size_t workspace_bytes, engram_stream_t stream) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if ((rc = check_bt(B, T)) != ENGRAM_OK) return rc;
+    if ((rc = validate_weights(plan, w)) != ENGRAM_OK) return rc;
+    const int64_t n_tok = static_cast<int64_t>(B) * T;
+    if (n_tok == 0) return ENGRAM_OK;
+    if (!h || !m || !out) return fail(ENGRAM_ERR_INVALID_ARG, "h, m and out must be non-NULL");
+    if (!aligned16(h) || !aligned16(m) || !aligned16(out) || (delta_dbg && !aligned16(delta_dbg)) ||
+        (conv_state && !aligned16(conv_state)))
+        return fail(ENGRAM_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (conv_state && T > 16384) return fail(ENGRAM_ERR_UNSUPPORTED, "T above 16384 with a conv state");
+    const size_t need = layout(plan, n_tok).total;
+    if (!workspace || workspace_bytes < need)
+        return fail(ENGRAM_ERR_INVALID_ARG, "workspace too small: need %zu bytes", need);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(ENGRAM_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+    return gate_conv_impl(plan, w, h, m, B, T, conv_state, out, delta_dbg, static_cast<uint8_t *>(workspace),
+                          static_cast<cudaStream_t>(stream), nullptr);
+}
+
+int engram_forward(const engram_plan *plan, const engram_weights *w, const uint16_t *const *tables,
+                   const int32_t *ids, const int32_t *remap, int32_t B, int32_t T, int32_t *history,
+                   uint16_t *conv_state, const uint16_t *h, uint16_t *out, float *delta_dbg, void *workspace,
+                   size_t workspace_bytes, engram_stream_t stream_, void *const *stage_events) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if ((rc = check_bt(B, T)) != ENGRAM_OK) return rc;
+    if ((rc = validate_weights(plan, w)) != ENGRAM_OK) return rc;
+    const int64_t n_tok = static_cast<int64_t>(B) * T;
+    if (n_tok == 0) return ENGRAM_OK;
+    if (!ids || !h || !out || !tables) return fail(ENGRAM_ERR_INVALID_ARG, "ids, tables, h and out must be non-NULL");
+    if (!aligned16(h) || !aligned16(out) || (delta_dbg && !aligned16(delta_dbg)) || (conv_state && !aligned16(conv_state)))
+        return fail(ENGRAM_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    for (int t = 0; t < plan->num_tables; ++t) {
+        if (!tables[t]) return fail(ENGRAM_ERR_INVALID_ARG, "tables[%d] is NULL", t);
+        if (!aligned16(tables[t])) return fail(ENGRAM_ERR_INVALID_ARG, "tables[%d] is not 16-byte aligned", t);
+    }
+    if (conv_state && T > 16384) return fail(ENGRAM_ERR_UNSUPPORTED, "T above 16384 with a conv state");
+    const Workspace L = layout(plan, n_tok);
+    if (!workspace || workspace_bytes < L.total)
+        return fail(ENGRAM_ERR_INVALID_ARG, "workspace too small: need %zu bytes", L.total);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(ENGRAM_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int32_t *xr = reinterpret_cast<int32_t *>(ws + L.xr);
+    uint32_t *idx = reinterpret_cast<uint32_t *>(ws + L.idx);
+    uint16_t *m = reinterpret_cast<uint16_t *>(ws + L.m);
+    auto rec = [&](int i) -> int {
+        if (stage_events) ENGRAM_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), stream), "cudaEventRecord");
+        return ENGRAM_OK;
+    };
+    if ((rc = rec(0)) != ENGRAM_OK) return rc;
+    if ((rc = launch_hash(plan, ids, remap, history, B, T, idx, xr, stream)) != ENGRAM_OK) return rc;
+    if ((rc = rec(1)) != ENGRAM_OK) return rc;
+    if ((rc = launch_gather(plan, idx, tables, n_tok, m, stream)) != ENGRAM_OK) return rc;
+    if ((rc = gate_conv_impl(plan, w, h, m, B, T, conv_state, out, delta_dbg, ws, stream,
+                             stage_events ? stage_events + 2 : nullptr)) != ENGRAM_OK)
+        return rc;
+    if ((rc = rec(4)) != ENGRAM_OK) return rc;
+    if (history != nullptr && plan->hist_len > 0) {
+        engram::advance_history_kernel<<<(B + 127) / 128, 128, 0, stream>>>(xr, B, T, history, plan->hist_len);
+        ENGRAM_CUDA_TRY(cudaGetLastError(), "advance_history_kernel launch");
+    }
+    return ENGRAM_OK;
+}
+
+int engram_device_status(uint32_t *status, int clear) {
+    if (!status) return fail(ENGRAM_ERR_INVALID_ARG, "status is NULL");
+    ENGRAM_CUDA_TRY(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+    uint32_t s = 0;
+    ENGRAM_CUDA_TRY(cudaMemcpyFromSymbol(&s, g_engram_status, sizeof s), "cudaMemcpyFromSymbol");
+    if (clear) {
+        const uint32_t zero = 0;
+        ENGRAM_CUDA_TRY(cudaMemcpyToSymbol(g_engram_status, &zero, sizeof zero), "cudaMemcpyToSymbol");
+    }
+    *status = s;
+    return ENGRAM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,199 @@
+/*
+ * engram.h -- C ABI of the B200 (sm_100a) hashed n-gram embedding lookup.
+ *
+ * The lookup ("Engram" conditional memory / N-gram Embedding) runs six steps per token:
+ *   1. remap the token id through a many-to-one vocabulary-compression table
+ *      [yktysq.com "Qwen 4用上DeepSeek的Engram", 四个关键组件 #1 Tokenizer Compression];
+ *   2. form the 2-gram (x_{t-1}, x_t) and 3-gram (x_{t-2}, x_{t-1}, x_t) keys and hash each with
+ *      K independent heads into prime-sized tables [same page, #2 Multi-Head Hashing;
+ *      zhichai.net "Qwen3.8-Flash-Next 把容量从「计算」搬到「存储」", §2.3 N-gram Embedding];
+ *   3. gather one row per head and concatenate the rows into the memory vector m
+ *      [yktysq #2; zhichai §2.3: 16 rows x 160 values = E_t in R^2560];
+ *   4. gate: q = RMSNorm(h), k = RMSNorm(W_k m), v = W_v m, g = sigmoid(q.k / sqrt(d_h)),
+ *      U = g v [yktysq #3 Context-aware Gating; zhichai §2.3 g_t, U_t];
+ *   5. depthwise causal conv, kernel 4, dilation = largest order, on RMSNorm(U), then SiLU
+ *      [yktysq #4; zhichai §2.3 Delta_t = U_t + SiLU(DWConv(RMSNorm(U_t)))];
+ *   6. residual: out = h + Delta [zhichai §2.3 R~_t = R_t + Delta_t].
+ *
+ * Conventions (every entry point):
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major, dense, unless
+ *     stated otherwise.  bf16 tensors are passed as their raw 16-bit patterns (uint16_t).
+ *   - Pointers to bf16 / fp32 tensors must be 16-byte aligned.
+ *   - The library allocates no device memory.  Scratch comes from the caller's workspace,
+ *     sized by engram_workspace_size().
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and returns an int status: ENGRAM_OK or a negative ENGRAM_ERR_* code.  Arguments are
+ *     validated on the host before anything is launched; on error nothing is launched and
+ *     engram_last_error() describes the problem (thread-local string).
+ *   - Data-dependent errors found on the device (a token id outside [0, vocab_in), a row id
+ *     outside its table) never fault: the offending element reads the pad id / a zero row
+ *     and a bit is set in the per-device status word, read by engram_device_status().
+ *   - Calls on one stream are ordered; calls that share output or workspace buffers on
+ *     different streams race.
+ */
+#ifndef ENGRAM_H
+#define ENGRAM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- status codes */
+#define ENGRAM_OK 0
+#define ENGRAM_ERR_INVALID_ARG (-1) /* null / misaligned pointer, bad size, dim mismatch */
+#define ENGRAM_ERR_UNSUPPORTED (-2) /* valid but not handled: d_e % 8, order outside 1..4, ... */
+#define ENGRAM_ERR_CUDA (-3)        /* a CUDA runtime call failed; see engram_last_error() */
+#define ENGRAM_ERR_OOM (-4)         /* not enough device memory for the request */
+#define ENGRAM_ERR_TIMEOUT (-5)     /* a bounded device-side wait gave up */
+
+/* bits of the per-device status word (engram_device_status) */
+#define ENGRAM_STATUS_BAD_TOKEN 0x1u    /* a token id was outside [0, vocab_in) */
+#define ENGRAM_STATUS_BAD_ROW 0x2u      /* a row id was outside [0, table_rows[h]) */
+#define ENGRAM_STATUS_WAIT_TIMEOUT 0x4u /* a pipeline wait inside a kernel gave up */
+
+/* ---------------------------------------------------------------- limits */
+#define ENGRAM_MAX_ORDERS 4
+#define ENGRAM_MAX_TABLES 32
+#define ENGRAM_MAX_HIST 3 /* largest order - 1 */
+
+typedef void *engram_stream_t; /* cudaStream_t */
+
+enum engram_table_location {
+    ENGRAM_TABLES_DEVICE = 0,     /* tables resident in HBM */
+    ENGRAM_TABLES_HOST_MAPPED = 1 /* tables in pinned, mapped host memory */
+};
+
+/* Static description of one lookup layer.  Filled by the caller, checked by engram_init. */
+typedef struct engram_config {
+    int32_t num_orders;                   /* |O|, 1..ENGRAM_MAX_ORDERS */
+    int32_t orders[ENGRAM_MAX_ORDERS];    /* n-gram orders, strictly increasing, each 1..4;
+                                             the pages use {2, 3} */
+    int32_t heads_per_order;              /* K >= 1; tables H = num_orders * K <= 32 */
+    int64_t table_rows[ENGRAM_MAX_TABLES]; /* P_h, each a prime < 2^32, for h = oi*K + j */
+    int32_t row_dim;                      /* d_e, multiple of 8 */
+    int32_t hidden_dim;                   /* d_h, multiple of 64 */
+    int32_t vocab_in;                     /* V: ids are in [0, V) */
+    int32_t vocab_out;                    /* V': remapped ids are in [0, V') */
+    int32_t pad_id;                       /* id used before a sequence start; must be V' */
+    int32_t conv_kernel;                  /* depthwise conv taps, 1..8 (pages: 4) */
+    int32_t conv_dilation;                /* must equal the largest order (pages) */
+    int32_t table_location;               /* enum engram_table_location */
+    uint64_t hash_seed;                   /* seeds the per-head hash multipliers */
+    float eps;                            /* RMSNorm epsilon (> 0) */
+    int32_t reserved[7];                  /* must be zero */
+} engram_config;
+
+/* Validated config plus derived constants.  Caller-owned, plain data: engram_init fills
+ * it, every other call reads it.  Do not modify its fields. */
+typedef struct engram_plan {
+    engram_config cfg;
+    uint64_t mult[ENGRAM_MAX_TABLES][ENGRAM_MAX_ORDERS]; /* hash multipliers a_{o,j,i} */
+    int32_t num_tables;  /* H */
+    int32_t mem_dim;     /* d_m = H * d_e */
+    int32_t hist_len;    /* largest order - 1 */
+    int32_t state_len;   /* (conv_kernel - 1) * conv_dilation */
+    uint32_t magic;
+    int32_t reserved[3];
+} engram_plan;
+
+/* Weights of the gate and conv (device pointers, bf16 patterns). */
+typedef struct engram_weights {
+    const uint16_t *w_k;     /* [d_h, d_m], row r = output channel r */
+    const uint16_t *w_v;     /* [d_h, d_m] */
+    const uint16_t *gamma_q; /* [d_h] RMSNorm gain of the query (hidden state) */
+    const uint16_t *gamma_k; /* [d_h] RMSNorm gain of the key */
+    const uint16_t *gamma_c; /* [d_h] RMSNorm gain of the conv input */
+    const uint16_t *conv_w;  /* [d_h, conv_kernel]; tap i reads position t - i*dilation */
+} engram_weights;
+
+/* Validate `cfg` and fill `plan` (host only, no CUDA call).  Checks: orders, K, H <= 32,
+ * primality of every table_rows[h] (deterministic Miller-Rabin), d_e % 8 == 0,
+ * d_h % 64 == 0, pad_id == vocab_out, dilation == largest order, eps > 0, reserved == 0.
+ * Derives the hash multipliers: a_{o,j,i} = SplitMix64(seed ^ (o<<16 ^ j<<8 ^ i)) | 1. */
+int engram_init(const engram_config *cfg, engram_plan *plan);
+
+/* Bytes of device workspace engram_forward / engram_gate_conv need for n_tok = B*T tokens
+ * (remapped ids, row ids, memory vectors, fp32 value projections, per-tile partial sums;
+ * each region 256-byte aligned).  0 on an invalid plan. */
+size_t engram_workspace_size(const engram_plan *plan, int64_t n_tok);
+
+/* Step 1 [yktysq #1]: out[i] = remap[ids[i]] for i < n.
+ * ids, out: int32 [n] (may alias).  remap: int32 [vocab_in], values in [0, vocab_out).
+ * An id outside [0, vocab_in) yields pad_id and sets ENGRAM_STATUS_BAD_TOKEN. */
+int engram_remap(const engram_plan *plan, const int32_t *ids, int64_t n, const int32_t *remap,
+                 int32_t *out, engram_stream_t stream);
+
+/* Step 2 [yktysq #2; zhichai §2.3]: row ids of every n-gram head.
+ * ids_remapped: int32 [B, T] in [0, vocab_out].
+ * history: NULL, or int32 [B, hist_len] remapped ids preceding position 0 (oldest first);
+ *          positions before both the sequence and the history use pad_id.
+ * idx: uint32 [B*T, H], column h = oi*K + j (order-major, head-minor).
+ * Hash: s = XOR_i (x'_{t-i} + 1) * a_{o,j,i} mod 2^64; idx = fmix64(s) mod P_h, where fmix64
+ * is the MurmurHash3 64-bit finaliser. */
+int engram_hash(const engram_plan *plan, const int32_t *ids_remapped, int32_t B, int32_t T,
+                const int32_t *history, uint32_t *idx, engram_stream_t stream);
+
+/* Decode bookkeeping: history <- last hist_len ids of (history ++ ids_remapped[b, :]), in
+ * place.  history: int32 [B, hist_len]. */
+int engram_advance_history(const engram_plan *plan, const int32_t *ids_remapped, int32_t B,
+                           int32_t T, int32_t *history, engram_stream_t stream);
+
+/* Step 3 [yktysq #2; zhichai §2.3]: m[n, h*d_e:(h+1)*d_e] = tables[h][idx[n, h], :].
+ * tables: HOST array of H pointers, each to bf16 [table_rows[h], d_e] (device memory, or
+ * pinned mapped host memory when cfg.table_location == ENGRAM_TABLES_HOST_MAPPED).
+ * idx: uint32 [n_tok, H].  m: bf16 [n_tok, d_m].  Bit patterns are copied unchanged.
+ * A row id >= table_rows[h] yields a zero row and sets ENGRAM_STATUS_BAD_ROW. */
+int engram_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables,
+                  int64_t n_tok, uint16_t *m, engram_stream_t stream);
+
+/* Steps 4-6 [yktysq #3, #4; zhichai §2.3]: gate, conv, residual for B sequences of T tokens.
+ * h: bf16 [B*T, d_h] hidden states.  m: bf16 [B*T, d_m] memory vectors.
+ * conv_state: NULL for prefill (zero left padding), or bf16 [B, state_len, d_h] conv inputs
+ *             of the state_len positions before this call, oldest first; updated in place.
+ *             With a state, T <= 16384.
+ * out: bf16 [B*T, d_h] = bf16_rne(h + Delta).  May not alias h.
+ * delta_dbg: NULL, or fp32 [B*T, d_h] receiving Delta before the residual add.
+ * The projections k~ = W_k m and v = W_v m run on the tcgen05 tensor cores (bf16 inputs,
+ * fp32 accumulation); norms, gate and conv run in fp32.
+ * workspace: >= engram_workspace_size(plan, B*T) bytes, 256-byte aligned. */
+int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uint16_t *h,
+                     const uint16_t *m, int32_t B, int32_t T, uint16_t *conv_state,
+                     uint16_t *out, float *delta_dbg, void *workspace, size_t workspace_bytes,
+                     engram_stream_t stream);
+
+/* Steps 1-6 chained: remap + hash (one kernel), gather, projections with the gate's partial
+ * reductions fused in their epilogue, then gate + conv + residual (one kernel), then the
+ * history update when `history` is given.
+ * ids: int32 [B, T] raw token ids.  remap: int32 [vocab_in], or NULL when ids are already
+ * in the compressed vocabulary.  history / conv_state: NULL for prefill, or the decode state
+ * (read, then updated in place).  Other arguments as in the steps above.
+ * stage_events: NULL, or an array of ENGRAM_FORWARD_STAGES + 1 cudaEvent_t recorded on
+ * `stream` before each stage and after the last (a profiling hook; no effect on results). */
+#define ENGRAM_FORWARD_STAGES 4 /* hash, gather, projections, gate+conv */
+int engram_forward(const engram_plan *plan, const engram_weights *w,
+                   const uint16_t *const *tables, const int32_t *ids, const int32_t *remap,
+                   int32_t B, int32_t T, int32_t *history, uint16_t *conv_state,
+                   const uint16_t *h, uint16_t *out, float *delta_dbg, void *workspace,
+                   size_t workspace_bytes, engram_stream_t stream, void *const *stage_events);
+
+/* Read (and optionally clear) the status word of the current device.  Synchronises the
+ * device.  *status receives the OR of ENGRAM_STATUS_* bits since the last clear. */
+int engram_device_status(uint32_t *status, int clear);
+
+/* Description of the last error on this thread ("" if none). */
+const char *engram_last_error(void);
+
+/* Library version, e.g. "0.1.0". */
+const char *engram_version(void);
+
+/* sizeof() of a public struct, by name ("engram_config", "engram_plan", "engram_weights"),
+ * so that bindings in other languages can check their layout; 0 for an unknown name. */
+size_t engram_sizeof(const char *type_name);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ENGRAM_H */

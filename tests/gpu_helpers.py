@@ -1,0 +1,91 @@
+"""Device-side input construction for the GPU tests (same seeds and bits as the host side)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import hashed_gram_embedding_remap_b200 as E
+import synth
+from synth import fill_gpu
+
+ONE = 0x3F80
+
+# Tolerances on Delta (fp32 debug output) and on out (bf16): the benchmark spec's bound is
+# max-abs 1e-2 / mean-abs 1e-3 for gated outputs (bf16 storage, fp32 accumulation).  On out
+# an element may also differ by one bf16 ulp of the oracle's value: at |out| >= 4 one ulp
+# (2^-5) exceeds 1e-2, and any fp32-vs-fp64 difference can move a value across a rounding
+# boundary.
+DELTA_MAX_ABS = 1e-2
+DELTA_MEAN_ABS = 1e-3
+
+
+def to_dev(a: np.ndarray, device="cuda") -> torch.Tensor:
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(a).to(device)
+
+
+def to_host_u16(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+class DeviceInputs:
+    """All tensors of one workload on the device; tables filled on the GPU."""
+
+    def __init__(self, wl: synth.Workload, step: int = 0, device="cuda", tables=None):
+        fill_gpu.build()
+        self.wl = wl
+        self.ids_np = wl.ids(step)
+        self.remap_np = wl.remap()
+        self.ids = to_dev(self.ids_np, device)
+        self.remap = to_dev(self.remap_np, device)
+        if tables is None:
+            tables = [fill_gpu.filled((wl.primes[h], wl.d_e), wl.table_spec(h), device) for h in range(wl.H)]
+        self.tables = tables
+        self.h = fill_gpu.filled((wl.n_tok, wl.d_h), wl.h_spec(step), device)
+        self.w_k = fill_gpu.filled((wl.d_h, wl.d_m), wl.wk_spec(), device)
+        self.w_v = fill_gpu.filled((wl.d_h, wl.d_m), wl.wv_spec(), device)
+        ones = torch.full((wl.d_h,), ONE, dtype=torch.int16, device=device).view(torch.bfloat16)
+        self.gamma_q, self.gamma_k, self.gamma_c = ones.clone(), ones.clone(), ones.clone()
+        self.conv_w = fill_gpu.filled((wl.d_h, wl.conv_kernel), wl.conv_spec(), device)
+        self.history = to_dev(wl.history(), device) if wl.decode else None
+        self.conv_state = (fill_gpu.filled((wl.B, wl.state_len, wl.d_h), wl.state_spec(), device)
+                           if wl.decode else None)
+        self.plan = E.Plan.from_workload(wl)
+        self.weights = E.Weights(self.w_k, self.w_v, self.gamma_q, self.gamma_k, self.gamma_c, self.conv_w)
+        self.out = torch.empty((wl.n_tok, wl.d_h), dtype=torch.bfloat16, device=device)
+        self.delta = torch.empty((wl.n_tok, wl.d_h), dtype=torch.float32, device=device)
+        self.ws = E.alloc_workspace(self.plan, wl.n_tok, device)
+
+    def forward(self, delta=True, **kw):
+        E.engram_forward(self.plan, self.weights, self.tables, self.ids, self.h, self.out, self.ws,
+                         remap=None if self.wl.identity_remap else self.remap,
+                         history=self.history, conv_state=self.conv_state,
+                         delta_dbg=self.delta if delta else None, **kw)
+        return self
+
+    def host_weights(self):
+        return dict(Wk=to_host_u16(self.w_k), Wv=to_host_u16(self.w_v), gamma_q=to_host_u16(self.gamma_q),
+                    gamma_k=to_host_u16(self.gamma_k), gamma_c=to_host_u16(self.gamma_c),
+                    conv_w=to_host_u16(self.conv_w))
+
+
+def assert_delta_close(got: np.ndarray, ref: np.ndarray, max_abs=DELTA_MAX_ABS, mean_abs=DELTA_MEAN_ABS):
+    d = np.abs(got.astype(np.float64) - ref.astype(np.float64))
+    assert np.isfinite(got).all()
+    assert d.max() <= max_abs, f"Delta max-abs {d.max():.3e} > {max_abs}"
+    assert d.mean() <= mean_abs, f"Delta mean-abs {d.mean():.3e} > {mean_abs}"
+    return float(d.max()), float(d.mean())
+
+
+def assert_out_close(got_bits: np.ndarray, ref_bits: np.ndarray):
+    g = synth.bf16_to_float(got_bits).astype(np.float64)
+    r = synth.bf16_to_float(ref_bits).astype(np.float64)
+    v = np.abs(r)
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(v, 2.0 ** -126))) - 7)
+    d = np.abs(g - r)
+    bad = d > np.maximum(DELTA_MAX_ABS, ulp)
+    assert not bad.any(), f"{bad.sum()} outputs beyond max(1e-2, 1 ulp); worst {d.max():.3e}"
+    assert d.mean() <= DELTA_MEAN_ABS, f"out mean-abs {d.mean():.3e}"
+    return float((d > ulp).mean())

@@ -1,0 +1,122 @@
+"""The C-ABI library loads on the host and exports every entry point include/engram.h declares;
+host-side validation works without a GPU (invalid arguments are rejected before any launch)."""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import hashed_gram_embedding_remap_b200 as E
+import synth
+from hashed_gram_embedding_remap_b200 import _native
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "engram.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(engram_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert {"engram_remap", "engram_hash", "engram_gather", "engram_gate_conv", "engram_forward"} <= set(names)
+    lib = C.CDLL(E.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in engram.h but not exported"
+
+
+def test_struct_layouts_match_header():
+    for name, cls in (("engram_config", _native.engram_config), ("engram_plan", _native.engram_plan),
+                      ("engram_weights", _native.engram_weights)):
+        assert E.lib.engram_sizeof(name.encode()) == C.sizeof(cls)
+    assert E.lib.engram_sizeof(b"nope") == 0
+
+
+def _plan(**kw):
+    base = dict(orders=(2, 3), heads_per_order=2, table_rows=(10007, 10009, 10037, 10039), row_dim=32,
+                hidden_dim=256, vocab_in=1000, vocab_out=770, hash_seed=7)
+    base.update(kw)
+    return E.Plan(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(table_rows=(10007, 10009, 10037, 10040)), E.ENGRAM_ERR_INVALID_ARG),   # not prime
+    (dict(table_rows=(10007, 10009, 10037)), E.ENGRAM_ERR_INVALID_ARG),          # 0 rows for table 3
+    (dict(orders=(3, 2)), E.ENGRAM_ERR_INVALID_ARG),                             # not increasing
+    (dict(orders=(2, 5)), E.ENGRAM_ERR_UNSUPPORTED),
+    (dict(row_dim=30), E.ENGRAM_ERR_UNSUPPORTED),
+    (dict(hidden_dim=200), E.ENGRAM_ERR_UNSUPPORTED),
+    (dict(eps=0.0), E.ENGRAM_ERR_INVALID_ARG),
+    (dict(conv_kernel=9), E.ENGRAM_ERR_UNSUPPORTED),
+    (dict(heads_per_order=17), E.ENGRAM_ERR_UNSUPPORTED),
+])
+def test_init_rejects_bad_configs(kw, code):
+    with pytest.raises(E.EngramError) as ei:
+        _plan(**kw)
+    assert ei.value.code == code
+
+
+def test_init_accepts_every_workload_and_derives_constants():
+    for name, wl in synth.WORKLOADS.items():
+        p = E.Plan.from_workload(wl)
+        assert p.num_tables == wl.H and p.mem_dim == wl.d_m
+        assert p.hist_len == max(wl.orders) - 1 and p.state_len == 3 * max(wl.orders)
+        assert E.engram_workspace_size(p, wl.n_tok) > 0
+    p = _plan()
+    assert E.engram_workspace_size(p, 1000) < E.engram_workspace_size(p, 2000)
+    assert E.engram_workspace_size(p, 0) >= 0
+
+
+def test_hash_multipliers_are_odd_and_seeded():
+    p1, p2 = _plan(hash_seed=1), _plan(hash_seed=2)
+    m1 = [p1.plan.mult[h][i] for h in range(4) for i in range(2)]
+    m2 = [p2.plan.mult[h][i] for h in range(4) for i in range(2)]
+    assert all(x & 1 for x in m1) and m1 != m2
+
+
+def test_invalid_calls_fail_on_host_without_launching():
+    lib = E.lib
+    p = _plan()
+    # uninitialised plan
+    bad = _native.engram_plan()
+    assert lib.engram_hash(C.byref(bad), None, 1, 1, None, None, None) == E.ENGRAM_ERR_INVALID_ARG
+    assert "engram_init" in E.last_error()
+    # NULL outputs / negative sizes
+    assert lib.engram_hash(p, None, 1, 4, None, None, None) == E.ENGRAM_ERR_INVALID_ARG
+    assert lib.engram_hash(p, None, -1, 4, None, None, None) == E.ENGRAM_ERR_INVALID_ARG
+    assert lib.engram_gather(p, None, None, -5, None, None) == E.ENGRAM_ERR_INVALID_ARG
+    # misaligned table pointer
+    tabs = (C.c_void_p * 4)(16, 32, 48, 65)
+    assert lib.engram_gather(p, C.c_void_p(16), tabs, 3, C.c_void_p(16), None) == E.ENGRAM_ERR_INVALID_ARG
+    assert "aligned" in E.last_error()
+    # missing weights
+    w = _native.engram_weights()
+    assert lib.engram_gate_conv(p, C.byref(w), None, None, 1, 1, None, None, None, None, 0, None) \
+        == E.ENGRAM_ERR_INVALID_ARG
+    # empty calls are no-ops and succeed without a device
+    assert lib.engram_hash(p, None, 0, 5, None, None, None) == E.ENGRAM_OK
+    assert lib.engram_gather(p, None, None, 0, None, None) == E.ENGRAM_OK
+    assert lib.engram_remap(p, None, 0, None, None, None) == E.ENGRAM_OK
+
+
+def test_workspace_too_small_is_rejected():
+    p = _plan()
+    ws = E.engram_workspace_size(p, 512)
+    w = _native.engram_weights(*[C.c_void_p(256 * (i + 1)) for i in range(6)])
+    rc = E.lib.engram_gate_conv(p, C.byref(w), C.c_void_p(256), C.c_void_p(512), 1, 512, None,
+                                C.c_void_p(768), None, C.c_void_p(1024), ws - 1, None)
+    assert rc == E.ENGRAM_ERR_INVALID_ARG and "workspace" in E.last_error()
+
+
+def test_product_has_no_oracle_dependency():
+    """The CUDA path never imports or links the oracle (the oracle is test infrastructure)."""
+    pkg = os.path.dirname(E.__file__)
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(root, f), encoding="utf-8").read()
+                assert "import oracle" not in text and "from oracle" not in text and "liboracle" not in text

@@ -1,0 +1,244 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bit-exact: remapped ids, row ids, gathered memory vectors, the GPU input generator.
+Tolerance (stated in gpu_helpers): Delta max-abs 1e-2 / mean-abs 1e-3; out within
+max(1e-2, one bf16 ulp) and mean-abs 1e-3.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import hashed_gram_embedding_remap_b200 as E
+import oracle
+import synth
+from gpu_helpers import DeviceInputs, assert_delta_close, assert_out_close, to_dev, to_host_u16
+from helpers import small_workload
+from synth import fill_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _idx_oracle(wl, ids_np, history=None):
+    xr = wl.remap()[ids_np]
+    return oracle.hash_ids(xr, wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id, history=history)
+
+
+# ------------------------------------------------------------------ generator
+def test_gpu_fill_matches_cpu_bits():
+    spec = synth.FillSpec(2024, 3, 0.02)
+    t = fill_gpu.filled((1003, 40), spec)
+    assert np.array_equal(to_host_u16(t), synth.fill_bf16(spec, (1003, 40)))
+    # rows regenerated on demand from a large tensor
+    big = fill_gpu.filled((200_003, 160), spec)
+    rows = np.array([0, 1, 77777, 200_002])
+    assert np.array_equal(to_host_u16(big[torch.from_numpy(rows).cuda()]), synth.fill_rows_bf16(spec, 160, rows))
+
+
+# ------------------------------------------------------------------ steps 1-2
+@pytest.mark.parametrize("name", ["tiny", "layer2560", "prefill20m"])
+def test_remap_and_hash_bit_exact_full_size(name):
+    wl = synth.get_workload(name)
+    plan = E.Plan.from_workload(wl)
+    ids = wl.ids()
+    d_ids, d_remap = to_dev(ids), to_dev(wl.remap())
+    xr = torch.empty_like(d_ids)
+    E.engram_remap(plan, d_ids, d_remap, xr)
+    xr_ref = oracle.remap(ids, wl.remap())
+    assert np.array_equal(xr.cpu().numpy(), xr_ref)
+    idx = torch.empty((wl.n_tok, wl.H), dtype=torch.int32, device="cuda")
+    E.engram_hash(plan, xr, idx)
+    ref = oracle.hash_ids(xr_ref, wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id)
+    assert np.array_equal(idx.cpu().numpy().view(np.uint32), ref)
+
+
+def test_hash_with_history_and_advance():
+    wl = synth.get_workload("decode20m")
+    plan = E.Plan.from_workload(wl)
+    hist_np = wl.history()
+    for T in (1, 2, 5):
+        ids = synth.zipf_ids(wl.vocab_in, 1.1, (wl.B, T), 99 + T)
+        d_ids, hist = to_dev(ids), to_dev(hist_np)
+        idx = torch.empty((wl.B * T, wl.H), dtype=torch.int32, device="cuda")
+        E.engram_hash(plan, d_ids, idx, history=hist)
+        ref = oracle.hash_ids(ids, wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id, history=hist_np)
+        assert np.array_equal(idx.cpu().numpy().view(np.uint32), ref)
+        E.engram_advance_history(plan, d_ids, hist)
+        assert np.array_equal(hist.cpu().numpy(), oracle.advance_history(ids, hist_np, 2, wl.pad_id))
+
+
+def test_hash_brute_force_small_vocab():
+    V = 31
+    wl = small_workload(vocab_in=V, vocab_out=V, B=V * V, T=3)
+    plan = E.Plan.from_workload(wl)
+    a, b, c = np.meshgrid(np.arange(V), np.arange(V), np.arange(V), indexing="ij")
+    xr = np.stack([a.ravel(), b.ravel(), c.ravel()], axis=1).astype(np.int32)
+    idx = torch.empty((xr.size, wl.H), dtype=torch.int32, device="cuda")
+    E.engram_hash(plan, to_dev(xr), idx)
+    ref = oracle.hash_ids(xr, wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id)
+    assert np.array_equal(idx.cpu().numpy().view(np.uint32), ref)
+
+
+# ------------------------------------------------------------------ step 3
+@pytest.mark.parametrize("K,d_e", [(2, 32), (3, 40), (8, 160)])
+def test_gather_bit_exact(K, d_e):
+    wl = small_workload(K=K, d_e=d_e, B=3, T=97)
+    plan = E.Plan.from_workload(wl)
+    tables_np = [synth.fill_bf16(wl.table_spec(h), (wl.primes[h], d_e)) for h in range(wl.H)]
+    tables = [to_dev(t) for t in tables_np]
+    idx_np = _idx_oracle(wl, wl.ids())
+    m = torch.empty((wl.n_tok, wl.d_m), dtype=torch.bfloat16, device="cuda")
+    E.engram_gather(plan, to_dev(idx_np.view(np.int32)), tables, m)
+    assert np.array_equal(to_host_u16(m), oracle.gather(idx_np, tables_np))
+
+
+def test_gather_full_size_layer2560_sampled_rows():
+    wl = synth.get_workload("layer2560")
+    di = DeviceInputs(wl)
+    idx_np = _idx_oracle(wl, di.ids_np)
+    m = torch.empty((wl.n_tok, wl.d_m), dtype=torch.bfloat16, device="cuda")
+    E.engram_gather(di.plan, to_dev(idx_np.view(np.int32)), di.tables, m)
+    rng = np.random.default_rng(5)
+    sample = np.concatenate([[0, 1, wl.n_tok - 1], rng.integers(0, wl.n_tok, 200)])
+    got = to_host_u16(m[torch.from_numpy(sample).cuda()]).reshape(len(sample), wl.H, wl.d_e)
+    for h in range(wl.H):
+        ref = synth.fill_rows_bf16(wl.table_spec(h), wl.d_e, idx_np[sample, h])
+        assert np.array_equal(got[:, h, :], ref)
+
+
+def test_bad_ids_and_rows_raise_status_not_faults():
+    wl = small_workload(B=1, T=16)
+    plan = E.Plan.from_workload(wl)
+    E.engram_device_status(clear=True)
+    ids = torch.tensor([[0, 5, wl.vocab_in + 3, -1] * 4], dtype=torch.int32, device="cuda")
+    out = torch.empty_like(ids)
+    E.engram_remap(plan, ids, to_dev(wl.remap()), out)
+    assert E.engram_device_status(clear=True) & E.ENGRAM_STATUS_BAD_TOKEN
+    assert (out.cpu().numpy()[0, 2::4] == wl.pad_id).all()
+    tables = [to_dev(synth.fill_bf16(wl.table_spec(h), (wl.primes[h], wl.d_e))) for h in range(wl.H)]
+    idx = torch.zeros((4, wl.H), dtype=torch.int32, device="cuda")
+    idx[1, 2] = wl.primes[2]          # one past the end
+    m = torch.empty((4, wl.d_m), dtype=torch.bfloat16, device="cuda")
+    E.engram_gather(plan, idx, tables, m)
+    assert E.engram_device_status(clear=True) & E.ENGRAM_STATUS_BAD_ROW
+    mh = to_host_u16(m).reshape(4, wl.H, wl.d_e)
+    assert (mh[1, 2] == 0).all() and not (mh[0, 2] == 0).all()
+    assert E.engram_device_status(clear=True) == 0
+
+
+# ------------------------------------------------------------------ steps 1-6
+def _oracle_full(wl, di):
+    w = di.host_weights()
+    tables = [synth.fill_bf16(wl.table_spec(h), (wl.primes[h], wl.d_e)) for h in range(wl.H)]
+    h = synth.fill_bf16(wl.h_spec(0), (wl.n_tok, wl.d_h))
+    kw = {}
+    if wl.decode:
+        kw = dict(history=wl.history(), conv_state=to_host_u16(di.conv_state), decode_outputs=True)
+    return oracle.forward(di.ids_np, di.remap_np, tables, h, w["Wk"], w["Wv"], w["gamma_q"],
+                          w["gamma_k"], w["gamma_c"], w["conv_w"], orders=wl.orders, K=wl.K,
+                          primes=wl.primes, seed=wl.hash_seed, pad_id=wl.pad_id, eps=wl.eps, **kw)
+
+
+PARITY_CASES = {
+    # name: workload (n_tok spans several 128-token tiles with a ragged tail where noted)
+    "tiny": synth.get_workload("tiny"),
+    "ragged_k_bn64": small_workload("ragged_k", B=3, T=333, K=3, d_e=40, d_h=384),     # d_m=240
+    "bn128": small_workload("bn128", B=2, T=4777, K=2, d_e=24, d_h=384),               # 9554 tok
+    "bn256": small_workload("bn256", B=5, T=1901, K=2, d_e=24, d_h=512),               # 9505 tok
+    "seq_shorter_than_halo": small_workload("short", B=40, T=7, K=2, d_e=16, d_h=128),
+}
+
+
+@pytest.mark.parametrize("case", list(PARITY_CASES))
+def test_forward_matches_oracle(case):
+    wl = PARITY_CASES[case]
+    di = DeviceInputs(wl).forward()
+    torch.cuda.synchronize()
+    ref = _oracle_full(wl, di)
+    assert_delta_close(di.delta.cpu().numpy(), ref["delta"])
+    assert_out_close(to_host_u16(di.out), ref["out"])
+    assert E.engram_device_status(clear=True) == 0
+
+
+def test_gate_conv_entry_matches_forward():
+    wl = PARITY_CASES["ragged_k_bn64"]
+    di = DeviceInputs(wl).forward()
+    out_fwd = di.out.clone()
+    idx_np = _idx_oracle(wl, di.ids_np)
+    m = torch.empty((wl.n_tok, wl.d_m), dtype=torch.bfloat16, device="cuda")
+    E.engram_gather(di.plan, to_dev(idx_np.view(np.int32)), di.tables, m)
+    out2 = torch.empty_like(di.out)
+    E.engram_gate_conv(di.plan, di.weights, di.h, m, wl.B, wl.T, out2, di.ws)
+    assert torch.equal(out_fwd.view(torch.int16), out2.view(torch.int16))
+
+
+def test_decode_steps_match_oracle_and_update_state():
+    wl = small_workload("dec", B=6, T=1, K=2, d_e=32, d_h=256, decode=True)
+    di = DeviceInputs(wl)
+    w = di.host_weights()
+    tables = [synth.fill_bf16(wl.table_spec(h), (wl.primes[h], wl.d_e)) for h in range(wl.H)]
+    hist = wl.history()
+    state = to_host_u16(di.conv_state)
+    for step in range(12):
+        ids_np = synth.zipf_ids(wl.vocab_in, 1.1, (wl.B, 1), 500 + step)
+        h_np = synth.fill_bf16(wl.h_spec(step), (wl.B, wl.d_h))
+        di.ids = to_dev(ids_np)
+        di.h = to_dev(h_np)
+        di.forward()
+        ref = oracle.forward(ids_np, di.remap_np, tables, h_np, w["Wk"], w["Wv"], w["gamma_q"], w["gamma_k"],
+                             w["gamma_c"], w["conv_w"], orders=wl.orders, K=wl.K, primes=wl.primes,
+                             seed=wl.hash_seed, pad_id=wl.pad_id, eps=wl.eps, history=hist,
+                             conv_state=state, decode_outputs=True)
+        torch.cuda.synchronize()
+        assert_delta_close(di.delta.cpu().numpy(), ref["delta"])
+        assert_out_close(to_host_u16(di.out), ref["out"])
+        assert np.array_equal(di.history.cpu().numpy(), ref["history"])
+        got_state = synth.bf16_to_float(to_host_u16(di.conv_state))
+        ref_state = synth.bf16_to_float(ref["state"])
+        # the new slot is bf16(u) on both sides: at most one bf16 ulp apart
+        assert np.abs(got_state - ref_state).max() <= 2.0 ** -5 + 1e-7
+        hist, state = ref["history"], to_host_u16(di.conv_state)
+
+
+def _window_oracle(wl, di, w, b, t):
+    """Oracle for token (b, t) on a window of at most 1 + state_len tokens, with the rows it
+    needs regenerated from the seeded generator (the tables are never materialised)."""
+    S = wl.state_len
+    w0 = max(0, t - S)
+    ids = di.ids_np[b:b + 1, w0:t + 1]
+    remap = di.remap_np
+    xr_full = remap[di.ids_np[b]]
+    hist = np.array([[xr_full[p] if p >= 0 else wl.pad_id for p in (w0 - 2, w0 - 1)]], dtype=np.int32)
+    xr = remap[ids]
+    idx = oracle.hash_ids(xr, wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id, history=hist)
+    W = idx.shape[0]
+    tables = [synth.fill_rows_bf16(wl.table_spec(h), wl.d_e, idx[:, h]) for h in range(wl.H)]
+    m = oracle.gather(np.tile(np.arange(W, dtype=np.uint32)[:, None], (1, wl.H)), tables)
+    rows = np.arange(b * wl.T + w0, b * wl.T + t + 1)
+    h = synth.fill_rows_bf16(wl.h_spec(0), wl.d_h, rows)
+    r = oracle.gate_conv(h, m, w["Wk"], w["Wv"], w["gamma_q"], w["gamma_k"], w["gamma_c"], w["conv_w"],
+                         1, W, dil=wl.conv_dilation, eps=wl.eps)
+    return r["delta"][-1], r["out"][-1]
+
+
+@pytest.mark.slow
+def test_forward_full_size_layer2560_sampled():
+    """The full 8x4096 workload in the benchmark's launch configuration, checked on sampled
+    tokens (sequence starts, tile edges, random) that the oracle computes one by one."""
+    wl = synth.get_workload("layer2560")
+    di = DeviceInputs(wl).forward()
+    torch.cuda.synchronize()
+    w = {k: v for k, v in di.host_weights().items()}
+    rng = np.random.default_rng(8)
+    picks = [(0, 0), (0, 1), (0, 2), (0, 9), (1, 0), (7, wl.T - 1), (3, 127), (3, 128), (5, 4095)]
+    picks += [(int(rng.integers(0, wl.B)), int(rng.integers(0, wl.T))) for _ in range(15)]
+    got_d = di.delta.cpu().numpy()
+    got_o = to_host_u16(di.out)
+    ds, rs, os_, ros = [], [], [], []
+    for b, t in picks:
+        d_ref, o_ref = _window_oracle(wl, di, w, b, t)
+        n = b * wl.T + t
+        ds.append(got_d[n]); rs.append(d_ref); os_.append(got_o[n]); ros.append(o_ref)
+    assert_delta_close(np.stack(ds), np.stack(rs))
+    assert_out_close(np.stack(os_), np.stack(ros))

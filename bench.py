@@ -45,51 +45,84 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event (throttle) reasons sampled through NVML every 20 ms
+    while the timed region runs (read-only queries)."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, cuda_index: int, period_s: float = 0.02):
+        self.cuda_index = cuda_index
+        self.period = period_s
         self.rows = []
-        self.proc = None
+        self.handle = None
+        self.error = None
+        self._stop = threading.Event()
+
+    def _open(self):
+        import pynvml
+        pynvml.nvmlInit()
+        bus = None
+        try:
+            props = torch.cuda.get_device_properties(self.cuda_index)
+            bus = getattr(props, "pci_bus_id", None)
+            dom = getattr(props, "pci_domain_id", 0)
+            dev = getattr(props, "pci_device_id", 0)
+            if bus is not None:
+                bus = f"{dom:08x}:{bus:02x}:{dev:02x}.0"
+        except Exception:
+            bus = None
+        if bus:
+            try:
+                return pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = self.cuda_index
+        if vis:
+            ids = [v.strip() for v in vis.split(",")]
+            if idx < len(ids) and ids[idx].isdigit():
+                idx = int(ids[idx])
+        return pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        import pynvml
+        while not self._stop.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+                reasons = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+                power = pynvml.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                self.rows.append((time.perf_counter(), sm, reasons, power))
+            except Exception as e:  # keep the benchmark running; report the failure
+                self.error = str(e)
+                return
+            time.sleep(self.period)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml
+            self.handle = self._open()
+            self.max_sm = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+            time.sleep(3 * self.period)
+        except Exception as e:
+            self.error = str(e)
+            self.handle = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.rows.append(parts)
-
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.t.join(timeout=2)
+        self._stop.set()
+        if self.handle is not None:
+            self.thread.join(timeout=2)
 
-    def summary(self):
-        if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(self.rows)}
+    def summary(self, t0=None, t1=None):
+        rows = [r for r in self.rows if (t0 is None or r[0] >= t0) and (t1 is None or r[0] <= t1)]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": getattr(self, "max_sm", None), "reasons": ["unsampled"],
+                    "samples": 0, "error": self.error}
+        reasons = sorted({name for r in rows for bit, name in self.REASONS.items() if r[2] & bit})
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": self.max_sm, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(r[3] for r in rows), "source": "nvml"}
 
 
 def dist_setup(args):
@@ -156,11 +189,16 @@ def run_reference(args, wl, world, rank):
     """Reference arm: the CPU oracle, rank 0 only, one bounded sample per step."""
     if rank != 0:
         return
+    per_tok = []
     for k in range(args.warmup):
-        oracle_sample(wl, min(16, args.oracle_tokens), seq=k)
+        Tw, dtw, _ = oracle_sample(wl, 8, seq=k)
+        per_tok.append(dtw / Tw)
+    # size each step's sample so that all timed steps take about --reference-seconds
+    est = min(per_tok) if per_tok else 0.01
+    n_sample = int(max(4, min(args.oracle_tokens, args.reference_seconds / max(1e-9, est * args.steps))))
     times, T, t_gen = [], 0, 0.0
     for k in range(args.steps):
-        T, dt, tg = oracle_sample(wl, args.oracle_tokens, seq=k)
+        T, dt, tg = oracle_sample(wl, n_sample, seq=k)
         times.append(dt)
         t_gen += tg
     tps = T * len(times) / sum(times)
@@ -236,11 +274,13 @@ def run_engram(args, wl, world, rank, local):
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
+        t_host0 = time.perf_counter()
         start.record(stream)
         for k in range(args.steps):
             step(evs[k])
         stop.record(stream)
         torch.cuda.synchronize()
+        t_host1 = time.perf_counter()
     barrier(world)
     elapsed_ms = start.elapsed_time(stop)
     elapsed_ms = max_over_ranks(elapsed_ms, world)
@@ -319,7 +359,7 @@ def run_engram(args, wl, world, rank, local):
         "config": workload_config(wl, world),
         "stages_ms": stage_ms, "hbm": hbm, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * (E.ENGRAM_FORWARD_STAGES + (1 if wl.decode else 0)),
-        "clocks": clocks.summary(),
+        "clocks": clocks.summary(t_host0, t_host1),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -328,12 +368,13 @@ def run_engram(args, wl, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["engram", "reference"], default="engram")
     ap.add_argument("--workload", default="layer2560", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--oracle-tokens", type=int, default=128)
     ap.add_argument("--cpu-baseline-tokens", type=int, default=768)
+    ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

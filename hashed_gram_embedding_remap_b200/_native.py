@@ -29,6 +29,7 @@ ENGRAM_MAX_TABLES = 32
 ENGRAM_FORWARD_STAGES = 4
 ENGRAM_TABLES_DEVICE = 0
 ENGRAM_TABLES_HOST_MAPPED = 1
+ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _ERRNAMES = {-1: "ENGRAM_ERR_INVALID_ARG", -2: "ENGRAM_ERR_UNSUPPORTED", -3: "ENGRAM_ERR_CUDA",
              -4: "ENGRAM_ERR_OOM", -5: "ENGRAM_ERR_TIMEOUT"}
@@ -92,6 +93,7 @@ def _load():
         "engram_gather": (C.c_int, [P, P, P, i64, P, P]),
         "engram_gate_conv": (C.c_int, [P, P, P, P, i32, i32, P, P, P, P, sz, P]),
         "engram_forward": (C.c_int, [P, P, P, P, P, i32, i32, P, P, P, P, P, P, sz, P, P]),
+        "engram_gate_conv_noalloc": (C.c_int, [P, P, P, P, i32, i32, P, P, P, P]),
         "engram_device_status": (C.c_int, [P, C.c_int]),
         "engram_last_error": (C.c_char_p, []),
         "engram_version": (C.c_char_p, []),
@@ -262,6 +264,16 @@ def engram_gate_conv(plan: Plan, weights: Weights, h: torch.Tensor, m: torch.Ten
                                 _ptr(delta_dbg, torch.float32, "delta_dbg"),
                                 _ptr(workspace, None, "workspace"),
                                 workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def engram_gate_conv_noalloc(plan: Plan, weights: Weights, h: torch.Tensor, m: torch.Tensor, B: int, T: int,
+                             out: torch.Tensor, conv_state: Optional[torch.Tensor] = None,
+                             delta_dbg: Optional[torch.Tensor] = None, stream=None):
+    """engram_gate_conv without a workspace, for hosts that cannot allocate device memory
+    (their scratch is the library's fixed per-GPU array of ENGRAM_NOALLOC_SCRATCH_BYTES)."""
+    _check(lib.engram_gate_conv_noalloc(plan, weights, _ptr(h, _BF16, "h"), _ptr(m, _BF16, "m"), B, T,
+                                        _ptr(conv_state, _BF16, "conv_state"), _ptr(out, _BF16, "out"),
+                                        _ptr(delta_dbg, torch.float32, "delta_dbg"), _stream(stream)))
 
 
 def engram_forward(plan: Plan, weights: Weights, tables, ids: torch.Tensor, h: torch.Tensor,

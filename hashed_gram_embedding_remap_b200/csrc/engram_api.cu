@@ -358,6 +358,29 @@ int check_bt(int32_t B, int32_t T) {
     return ENGRAM_OK;
 }
 
+// ---------------------------------------------------------------- no-allocation variant
+// Scratch for engram_gate_conv_noalloc: one array per device in the library's static device
+// data.  Host code may not pass the symbol itself to a kernel (on the host it only names a
+// shadow variable); the device address is looked up once per device below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[ENGRAM_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mutex;
+uint8_t *g_noalloc_ptr[64] = {};
+
+int noalloc_scratch(uint8_t **out) {
+    int dev = 0;
+    ENGRAM_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(ENGRAM_ERR_UNSUPPORTED, "device ordinal %d above 63", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        ENGRAM_CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(no-alloc scratch)");
+        g_noalloc_ptr[dev] = static_cast<uint8_t *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return ENGRAM_OK;
+}
+
 }  // namespace
 
 // =====================================================================================
@@ -556,6 +579,41 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const uint1
         ENGRAM_CUDA_TRY(cudaGetLastError(), "advance_history_kernel launch");
     }
     return ENGRAM_OK;
+}
+
+int engram_gate_conv_noalloc(const engram_plan *plan, const engram_weights *w, const uint16_t *h,
+                             const uint16_t *m, int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out,
+                             float *delta_dbg, engram_stream_t stream_) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if ((rc = check_bt(B, T)) != ENGRAM_OK) return rc;
+    if ((rc = validate_weights(plan, w)) != ENGRAM_OK) return rc;
+    const int64_t n_tok = static_cast<int64_t>(B) * T;
+    if (n_tok == 0) return ENGRAM_OK;
+    if (!h || !m || !out) return fail(ENGRAM_ERR_INVALID_ARG, "h, m and out must be non-NULL");
+    if (!aligned16(h) || !aligned16(m) || !aligned16(out) || (delta_dbg && !aligned16(delta_dbg)) ||
+        (conv_state && !aligned16(conv_state)))
+        return fail(ENGRAM_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (conv_state && T > 16384) return fail(ENGRAM_ERR_UNSUPPORTED, "T above 16384 with a conv state");
+    const int d_h = plan->cfg.hidden_dim;
+    const int bn = choose_bn(d_h, n_tok);
+    const int n_tiles = 2 * d_h / bn;
+    const size_t v_bytes = align256(sizeof(float) * static_cast<size_t>(n_tok) * d_h);
+    const size_t part_bytes = align256(sizeof(float4) * static_cast<size_t>(n_tok) * n_tiles);
+    if (v_bytes + part_bytes > ENGRAM_NOALLOC_SCRATCH_BYTES)
+        return fail(ENGRAM_ERR_UNSUPPORTED,
+                    "%lld tokens need %zu bytes of scratch; the static scratch holds %u bytes",
+                    static_cast<long long>(n_tok), v_bytes + part_bytes, ENGRAM_NOALLOC_SCRATCH_BYTES);
+    uint8_t *scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch)) != ENGRAM_OK) return rc;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    float *v = reinterpret_cast<float *>(scratch);
+    float4 *part = reinterpret_cast<float4 *>(scratch + v_bytes);
+    if (bn == 256) rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream);
+    else if (bn == 128) rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream);
+    else rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream);
+    if (rc != ENGRAM_OK) return rc;
+    return launch_gate_conv(plan, w, h, v, part, n_tiles, B, T, conv_state, out, delta_dbg, stream);
 }
 
 int engram_device_status(uint32_t *status, int clear) {

@@ -179,6 +179,31 @@ int engram_forward(const engram_plan *plan, const engram_weights *w,
                    const uint16_t *h, uint16_t *out, float *delta_dbg, void *workspace,
                    size_t workspace_bytes, engram_stream_t stream, void *const *stage_events);
 
+/* Steps 4-6 like engram_gate_conv, for callers that cannot allocate device memory: no
+ * workspace argument.  This entry point has no counterpart in the pages; it exists for
+ * hosts that hand an operator only its inputs and outputs and own every device allocation
+ * themselves (plugin and custom-op interfaces of inference servers, runtimes with a fixed
+ * memory budget, code paths where the device-wide synchronisation of cudaMalloc/cudaFree is
+ * not acceptable).  Its scratch (fp32 value projections and per-tile partial sums) lives in
+ * a statically sized array in the library's device data, ENGRAM_NOALLOC_SCRATCH_BYTES per
+ * GPU, which every GPU that loads the library holds until the process exits.
+ *  - Sizes: the call needs 4*B*T*d_h bytes for v plus 16*B*T*(2*d_h/BN) bytes of partial
+ *    sums (BN = 64, 128 or 256, the projection tile width), each rounded up to 256; a
+ *    request that does not fit returns ENGRAM_ERR_UNSUPPORTED and launches nothing.  At
+ *    d_h = 2560 that is about 2,900 tokens per call.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call before any
+ *    stream capture.  No call allocates or frees memory.
+ *  - Every call on a device shares the one array and leaves its contents behind.  No part of
+ *    it needs clearing: each element a call reads is written earlier in the same call.
+ *    Calls that overlap on the GPU (other streams, other host threads) race on the array
+ *    and must be serialised by the caller.
+ * Other arguments, layouts and results are those of engram_gate_conv. */
+#define ENGRAM_NOALLOC_SCRATCH_BYTES (32u << 20)
+int engram_gate_conv_noalloc(const engram_plan *plan, const engram_weights *w, const uint16_t *h,
+                             const uint16_t *m, int32_t B, int32_t T, uint16_t *conv_state,
+                             uint16_t *out, float *delta_dbg, engram_stream_t stream);
+
 /* Read (and optionally clear) the status word of the current device.  Synchronises the
  * device.  *status receives the OR of ENGRAM_STATUS_* bits since the last clear. */
 int engram_device_status(uint32_t *status, int clear);

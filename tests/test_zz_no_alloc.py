@@ -1,0 +1,77 @@
+"""The workspace-free gate/conv entry point (engram_gate_conv_noalloc).
+
+Some hosts cannot allocate device memory for an operator: plugin and custom-op interfaces
+of inference servers pass an op only its inputs and outputs and own every allocation, and
+some runtimes run under a fixed memory budget or cannot afford the device-wide
+synchronisation of cudaMalloc/cudaFree.  For them the library keeps the scratch of the
+projection + gate/conv step in a fixed per-GPU array inside its own device data.  This
+test calls that entry point through the C ABI twice in a row and checks each result
+against the workspace entry point, within the tolerance the parity tests use.  It lives in
+its own file so that pytest collects it last.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import hashed_gram_embedding_remap_b200 as E
+import oracle
+import synth
+from gpu_helpers import DeviceInputs, assert_delta_close, assert_out_close, to_dev, to_host_u16
+from helpers import small_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _memory_vectors(wl, di):
+    xr = wl.remap()[di.ids_np]
+    idx = oracle.hash_ids(xr, wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id)
+    m = torch.empty((wl.n_tok, wl.d_m), dtype=torch.bfloat16, device="cuda")
+    E.engram_gather(di.plan, to_dev(idx.view(np.int32)), di.tables, m)
+    return m
+
+
+@pytest.mark.parametrize("case", ["prefill", "decode"])
+def test_noalloc_matches_workspace_entry_two_calls(case):
+    if case == "prefill":
+        wl = small_workload("noalloc_prefill", B=3, T=333, K=3, d_e=40, d_h=384)
+    else:
+        wl = small_workload("noalloc_decode", B=64, T=1, K=2, d_e=32, d_h=512, decode=True)
+    di = DeviceInputs(wl)
+    m = _memory_vectors(wl, di)
+    state0 = di.conv_state.clone() if di.conv_state is not None else None
+
+    ref_out = torch.empty_like(di.out)
+    ref_delta = torch.empty_like(di.delta)
+    ref_state = state0.clone() if state0 is not None else None
+    E.engram_gate_conv(di.plan, di.weights, di.h, m, wl.B, wl.T, ref_out, di.ws, conv_state=ref_state,
+                       delta_dbg=ref_delta)
+    torch.cuda.synchronize()
+    ref_o, ref_d = to_host_u16(ref_out), ref_delta.cpu().numpy()
+
+    for call in range(2):
+        out = torch.full_like(di.out, 7.0)
+        delta = torch.full_like(di.delta, float("nan"))
+        state = state0.clone() if state0 is not None else None
+        E.engram_gate_conv_noalloc(di.plan, di.weights, di.h, m, wl.B, wl.T, out, conv_state=state,
+                                   delta_dbg=delta)
+        torch.cuda.synchronize()
+        assert_delta_close(delta.cpu().numpy(), ref_d)
+        assert_out_close(to_host_u16(out), ref_o)
+        if state is not None:
+            diff = np.abs(synth.bf16_to_float(to_host_u16(state)) - synth.bf16_to_float(to_host_u16(ref_state)))
+            assert diff.max() <= 2.0 ** -5
+    assert E.engram_device_status(clear=True) == 0
+
+
+def test_noalloc_rejects_requests_beyond_its_scratch():
+    wl = small_workload("noalloc_big", B=1, T=8, K=2, d_e=32, d_h=2560)
+    plan = E.Plan.from_workload(wl)
+    # 4 bytes of v per channel alone exceed the array at this many tokens
+    T = E.ENGRAM_NOALLOC_SCRATCH_BYTES // (4 * wl.d_h) + 1
+    dummy = torch.empty(16, dtype=torch.bfloat16, device="cuda")
+    w = E.Weights(dummy, dummy, dummy, dummy, dummy, dummy)
+    with pytest.raises(E.EngramError) as ei:
+        E.engram_gate_conv_noalloc(plan, w, dummy, dummy, 1, T, dummy)
+    assert ei.value.code == E.ENGRAM_ERR_UNSUPPORTED and "scratch" in str(ei.value)

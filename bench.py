@@ -266,18 +266,37 @@ def run_engram(args, wl, world, rank, local):
     E.engram_device_status(clear=True)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage)] for _ in range(args.steps)]
-    for row in evs:          # create the events before the timed region
+    for row in evs:          # create the events before the timed region (and before capture)
         for e in row:
             e.record(stream)
     torch.cuda.synchronize()
+    graph = None
+    if not args.eager:
+        # The whole timed region (K steps, each with its stage events) as one CUDA graph:
+        # no host launch overhead between kernels, which decode-sized steps would otherwise see.
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=cap, capture_error_mode="thread_local"):
+            cs = torch.cuda.current_stream()
+            for k in range(args.steps):
+                E.engram_forward(plan, weights, tables, ids, h, out, ws, remap=remap, history=history,
+                                 conv_state=state, stream=cs, stage_events=evs[k])
+        stream.wait_stream(cap)
+        torch.cuda.synchronize()
+        graph.replay()            # one untimed replay: uploads the graph
+        torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         t_host0 = time.perf_counter()
         start.record(stream)
-        for k in range(args.steps):
-            step(evs[k])
+        if graph is not None:
+            graph.replay()
+        else:
+            for k in range(args.steps):
+                step(evs[k])
         stop.record(stream)
         torch.cuda.synchronize()
         t_host1 = time.perf_counter()
@@ -311,18 +330,38 @@ def run_engram(args, wl, world, rank, local):
         for _ in range(max(1, args.warmup)):
             e2e_step()
         torch.cuda.synchronize()
+        g2 = None
+        if not args.eager:
+            g2 = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream()
+            cap.wait_stream(stream)
+            with torch.cuda.graph(g2, stream=cap, capture_error_mode="thread_local"):
+                for _ in range(args.steps):
+                    ids_dev2.copy_(ids_host, non_blocking=True)
+                    h_dev2.copy_(h_host, non_blocking=True)
+                    E.engram_forward(plan, weights, tables, ids_dev2, h_dev2, out, ws, remap=remap,
+                                     history=history, conv_state=state, stream=torch.cuda.current_stream())
+                    out_host.copy_(out, non_blocking=True)
+            stream.wait_stream(cap)
+            torch.cuda.synchronize()
+            g2.replay()
+            torch.cuda.synchronize()
         barrier(world)
         s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s2.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        if g2 is not None:
+            g2.replay()
+        else:
+            for _ in range(args.steps):
+                e2e_step()
         t2.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(s2.elapsed_time(t2), world)
         h2d = ids_host.numel() * 4 + h_host.numel() * 2
         d2h = out_host.numel() * 2
         e2e = {"value": wl.n_tok * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "mode": "eager" if args.eager else "cuda-graph of K steps (copies + engram_forward)"}
 
     peaks = load_peaks()
     n_tok = wl.n_tok
@@ -359,6 +398,7 @@ def run_engram(args, wl, world, rank, local):
         "config": workload_config(wl, world),
         "stages_ms": stage_ms, "hbm": hbm, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * (E.ENGRAM_FORWARD_STAGES + (1 if wl.decode else 0)),
+        "launch_mode": "eager" if args.eager else "one CUDA graph of the K timed steps",
         "clocks": clocks.summary(t_host0, t_host1),
     }
     if rank == 0:
@@ -376,6 +416,7 @@ def main():
     ap.add_argument("--cpu-baseline-tokens", type=int, default=768)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="launch every step from the host (no CUDA graph)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -174,6 +174,17 @@ int make_map_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t co
     return ENGRAM_OK;
 }
 
+int sm_count() {
+    static int count[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 64 && count[dev]) return count[dev];
+    int n = 148;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (dev < 64) count[dev] = n;
+    return n;
+}
+
 template <int BN>
 int set_proj_smem_attr() {
     // Per device: the attribute is a property of the function on the current device.
@@ -209,7 +220,11 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     p.d_h = d_h;
     p.n_tiles = 2 * d_h / BN;
     p.k_blocks = (d_m + engram::kBK - 1) / engram::kBK;
-    dim3 grid(p.n_tiles, static_cast<unsigned>((n_tok + engram::kBM - 1) / engram::kBM));
+    p.m_tiles = static_cast<int32_t>((n_tok + engram::kBM - 1) / engram::kBM);
+    const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+    if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
+    const int64_t sms = sm_count();
+    dim3 grid(static_cast<unsigned>(total < sms ? total : sms));
     engram::proj_kernel<BN><<<grid, engram::kProjThreads, engram::ProjCfg<BN>::kSmemBytes, stream>>>(
         map_m, map_wk, map_wv, p);
     ENGRAM_CUDA_TRY(cudaGetLastError(), "proj_kernel launch");
@@ -257,16 +272,6 @@ int launch_hash(const engram_plan *plan, const int32_t *ids, const int32_t *rema
     return ENGRAM_OK;
 }
 
-int sm_count() {
-    static int count[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    if (dev < 64 && count[dev]) return count[dev];
-    int n = 148;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (dev < 64) count[dev] = n;
-    return n;
-}
 
 int launch_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables, int64_t n_tok,
                   uint16_t *m, cudaStream_t stream) {
@@ -314,11 +319,14 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
     p.ksize = plan->cfg.conv_kernel;
     p.dil = plan->cfg.conv_dilation;
     p.state_len = plan->state_len;
-    p.tok_chunk = conv_state != nullptr ? T : 32;
+    constexpr int kChain = 12;   // outputs per residue chain in the k=4, dilation-3 fast path
+    const bool fast = conv_state == nullptr && p.ksize == 4 && p.dil == 3;
+    p.tok_chunk = conv_state != nullptr ? T : (fast ? 3 * kChain : 32);
     p.eps = plan->cfg.eps;
     p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(d_h));
-    const int threads = engram::kGateThreads;
-    const unsigned slices = static_cast<unsigned>((d_h / 4 + threads - 1) / threads);
+    const int threads = fast ? engram::kGateFastThreads : engram::kGateThreads;
+    const int per_thread = fast ? 2 : 4;   // channels per thread
+    const unsigned slices = static_cast<unsigned>((d_h / per_thread + threads - 1) / threads);
     const size_t smem = sizeof(float) * 2 * static_cast<size_t>(p.tok_chunk + p.state_len);
     if (smem > 48 * 1024) {
         ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::gate_conv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -326,9 +334,21 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
                         "cudaFuncSetAttribute(gate_conv_kernel)");
     }
     dim3 grid(static_cast<unsigned>((T + p.tok_chunk - 1) / p.tok_chunk), static_cast<unsigned>(B), slices);
-    engram::gate_conv_kernel<<<grid, threads, smem, stream>>>(p);
+    if (fast) engram::gate_conv_k4d3_kernel<kChain><<<grid, threads, 0, stream>>>(p);
+    else engram::gate_conv_kernel<<<grid, threads, smem, stream>>>(p);
     ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_conv_kernel launch");
     return ENGRAM_OK;
+}
+
+// Stage events are profiling hooks.  Under stream capture they must become event-record
+// nodes of the graph (cudaEventRecordExternal) so that they can be timed after a replay.
+cudaError_t record_stage_event(void *ev, cudaStream_t stream) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(stream, &st);
+    if (e != cudaSuccess) return e;
+    if (st == cudaStreamCaptureStatusActive)
+        return cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev), stream, cudaEventRecordExternal);
+    return cudaEventRecord(static_cast<cudaEvent_t>(ev), stream);
 }
 
 int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
@@ -341,12 +361,12 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
     float *v = reinterpret_cast<float *>(ws + L.v);
     float4 *part = reinterpret_cast<float4 *>(ws + L.part);
     int rc;
-    if (events) ENGRAM_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[0]), stream), "cudaEventRecord");
+    if (events) ENGRAM_CUDA_TRY(record_stage_event(events[0], stream), "cudaEventRecord");
     if (bn == 256) rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream);
     else if (bn == 128) rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream);
     else rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream);
     if (rc != ENGRAM_OK) return rc;
-    if (events) ENGRAM_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(events[1]), stream), "cudaEventRecord");
+    if (events) ENGRAM_CUDA_TRY(record_stage_event(events[1], stream), "cudaEventRecord");
     return launch_gate_conv(plan, w, h, v, part, 2 * d_h / bn, B, T, conv_state, out, delta, stream);
 }
 
@@ -563,7 +583,7 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const uint1
     uint32_t *idx = reinterpret_cast<uint32_t *>(ws + L.idx);
     uint16_t *m = reinterpret_cast<uint16_t *>(ws + L.m);
     auto rec = [&](int i) -> int {
-        if (stage_events) ENGRAM_CUDA_TRY(cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), stream), "cudaEventRecord");
+        if (stage_events) ENGRAM_CUDA_TRY(record_stage_event(stage_events[i], stream), "cudaEventRecord");
         return ENGRAM_OK;
     };
     if ((rc = rec(0)) != ENGRAM_OK) return rc;

@@ -37,10 +37,11 @@ struct ProjCfg {
     static constexpr int kBTile = BN * kBK * 2;
     static constexpr int kStageBytes = kATile + kBTile;
     static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
-    static constexpr int kTmemCols = BN;                          // fp32 accumulator columns
-    // dynamic smem: [align pad][stages x A][stages x B][barriers][gamma_qk BN floats][tmem addr]
-    static constexpr int kBarBytes = (2 * kStages + 1) * 8;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + BN * 4 + 16;
+    static constexpr int kAccum = 2;                              // TMEM accumulators (double buffer)
+    static constexpr int kTmemCols = kAccum * BN;                 // fp32 columns, power of two
+    // dynamic smem: [align pad][stages x A][stages x B][full, empty, tmem_full, tmem_empty][tmem addr]
+    static constexpr int kBarBytes = (2 * kStages + 2 * kAccum) * 8;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 16;
 };
 
 struct ProjParams {
@@ -53,6 +54,7 @@ struct ProjParams {
     int32_t d_m, d_h;
     int32_t n_tiles;           // 2 * d_h / BN: key tiles first, then value tiles
     int32_t k_blocks;          // ceil(d_m / kBK)
+    int32_t m_tiles;           // ceil(n_tok / kBM)
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -61,29 +63,33 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
     return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
 
+// Persistent: grid = min(#tiles, #SMs); CTA i takes tiles i, i + grid, ...  Tile t covers
+// tokens [128*(t / n_tiles), +128) and channel slice t % n_tiles, so the CTAs running at
+// one time share a few 128-token blocks of m (re-read from L2) and stream all of W.
+// Roles: warp 0 = TMA producer, warp 1 = TMEM owner + MMA issuer, warps 2-5 = epilogue.
+// Two TMEM accumulators: the epilogue drains tile i while the MMAs of tile i+1 run.
 template <int BN>
 __global__ void __launch_bounds__(kProjThreads, 1)
     proj_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ CUtensorMap map_wk,
                 const __grid_constant__ CUtensorMap map_wv, const __grid_constant__ ProjParams p) {
     using Cfg = ProjCfg<BN>;
     constexpr int S = Cfg::kStages;
+    constexpr int NACC = Cfg::kAccum;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + S * Cfg::kATile;
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes);
     uint64_t *empty_bar = full_bar + S;
-    uint64_t *accum_bar = empty_bar + S;
-    float *s_gqk = reinterpret_cast<float *>(accum_bar + 1);
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(s_gqk + BN);
+    uint64_t *tfull_bar = empty_bar + S;      // MMA -> epilogue, one per accumulator
+    uint64_t *tempty_bar = tfull_bar + NACC;  // epilogue -> MMA, one per accumulator
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(tempty_bar + NACC);
     __shared__ int s_abort;
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int tile_n = blockIdx.x;                 // which BN-wide slice of [k~ | v]
-    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
-    const bool is_key = tile_n * BN < p.d_h;
-    const int c0 = is_key ? tile_n * BN : tile_n * BN - p.d_h;   // channel offset in d_h
+    const int total = p.m_tiles * p.n_tiles;
+    const int key_tiles = p.d_h / BN;
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -91,18 +97,18 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
-        mbar_init(accum_bar, 1);
+        for (int a = 0; a < NACC; ++a) {
+            mbar_init(&tfull_bar[a], 1);
+            mbar_init(&tempty_bar[a], 4);   // one arrival per epilogue warp
+        }
         fence_barrier_init();
         tma_prefetch_desc(&map_m);
-        tma_prefetch_desc(is_key ? &map_wk : &map_wv);
+        tma_prefetch_desc(&map_wk);
+        tma_prefetch_desc(&map_wv);
     }
     if (warp == 1) {
         tmem_alloc(s_tmem, Cfg::kTmemCols);
         tmem_relinquish();
-    }
-    if (warp >= 2) {
-        for (int c = threadIdx.x - 64; c < BN; c += 128)
-            s_gqk[c] = is_key ? bf16_bits_to_f32(p.gamma_q[c0 + c]) * bf16_bits_to_f32(p.gamma_k[c0 + c]) : 0.f;
     }
     tc_fence_before();
     __syncthreads();
@@ -111,76 +117,104 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            const CUtensorMap *map_w = is_key ? &map_wk : &map_wv;
-            int issued = 0;
-            for (int kb = 0; kb < p.k_blocks; ++kb) {
-                const int s = kb % S;
-                const uint32_t ph = (kb / S) & 1;
-                if (!mbar_wait(&empty_bar[s], ph ^ 1, &s_abort)) break;
-                mbar_arrive_expect_tx(&full_bar[s], Cfg::kStageBytes);
-                tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, static_cast<int>(m0));
-                tma_load_2d(sB + s * Cfg::kBTile, map_w, &full_bar[s], kb * kBK, c0);
-                ++issued;
+            int it = 0, issued = 0;
+            for (int t = blockIdx.x; t < total && !s_abort; t += gridDim.x) {
+                const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
+                const bool is_key = nt < key_tiles;
+                const CUtensorMap *map_w = is_key ? &map_wk : &map_wv;
+                const int c0 = (is_key ? nt : nt - key_tiles) * BN;
+                const int m0 = mt * kBM;
+                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1;
+                    if (!mbar_wait(&empty_bar[s], ph ^ 1, &s_abort)) break;
+                    mbar_arrive_expect_tx(&full_bar[s], Cfg::kStageBytes);
+                    tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
+                    tma_load_2d(sB + s * Cfg::kBTile, map_w, &full_bar[s], kb * kBK, c0);
+                    issued = it + 1;
+                }
             }
             if (s_abort) {
                 // Every issued copy must land before the CTA's shared memory is released.
                 volatile int never = 0;
-                for (int kb = issued - S > 0 ? issued - S : 0; kb < issued; ++kb)
-                    if (!mbar_wait(&full_bar[kb % S], (kb / S) & 1, &never)) break;
+                for (int k = issued - S > 0 ? issued - S : 0; k < issued; ++k)
+                    if (!mbar_wait(&full_bar[k % S], (k / S) & 1, &never)) break;
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
-            bool ok = true;
-            for (int kb = 0; kb < p.k_blocks; ++kb) {
-                const int s = kb % S;
-                const uint32_t ph = (kb / S) & 1;
-                if (!mbar_wait(&full_bar[s], ph, &s_abort)) { ok = false; break; }
+            int it = 0, li = 0;
+            for (int t = blockIdx.x; t < total && !s_abort; t += gridDim.x, ++li) {
+                const int acc = li % NACC;
+                const uint32_t use = li / NACC;
+                if (!mbar_wait(&tempty_bar[acc], (use & 1) ^ 1, &s_abort)) break;
                 tc_fence_after();
-                const uint64_t adesc = sdesc_kmajor_sw128(sA + s * Cfg::kATile);
-                const uint64_t bdesc = sdesc_kmajor_sw128(sB + s * Cfg::kBTile);
+                const uint32_t dst = tmem_base + acc * BN;
+                bool ok = true;
+                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1;
+                    if (!mbar_wait(&full_bar[s], ph, &s_abort)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t adesc = sdesc_kmajor_sw128(sA + s * Cfg::kATile);
+                    const uint64_t bdesc = sdesc_kmajor_sw128(sB + s * Cfg::kBTile);
 #pragma unroll
-                for (int k = 0; k < kBK / kUmmaK; ++k) {
-                    // advance 16 elements (32 bytes) along K inside the swizzled row
-                    const uint64_t koff = static_cast<uint64_t>((k * kUmmaK * 2) >> 4);
-                    umma_bf16_ss(tmem_base, adesc + koff, bdesc + koff, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < kBK / kUmmaK; ++k) {
+                        const uint64_t koff = static_cast<uint64_t>((k * kUmmaK * 2) >> 4);
+                        umma_bf16_ss(dst, adesc + koff, bdesc + koff, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&empty_bar[s]);   // frees the stage once these MMAs have read it
                 }
-                umma_commit(&empty_bar[s]);  // frees the stage once these MMAs have read it
+                if (!ok) break;
+                umma_commit(&tfull_bar[acc]);     // accumulator ready for the epilogue
             }
-            if (ok) umma_commit(accum_bar);
-            else mbar_arrive(accum_bar);    // release the epilogue; it sees s_abort
+            if (s_abort) {
+                for (int a = 0; a < NACC; ++a) mbar_arrive(&tfull_bar[a]);   // release waiting epilogue warps
+            }
         }
     } else {
         // ---------------------------------------------------------------- epilogue
         const int sub = warp & 3;                      // TMEM lane quarter this warp may access
         const int row = sub * 32 + lane;
-        const int64_t n = m0 + row;
-        const bool valid = n < p.n_tok;
-        const bool got = mbar_wait(accum_bar, 0, &s_abort) && !s_abort;
-        tc_fence_after();
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f;
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(sub * 32) << 16);
-        if (got) {
+        int li = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++li) {
+            const int acc = li % NACC;
+            const uint32_t use = li / NACC;
+            if (!mbar_wait(&tfull_bar[acc], use & 1, &s_abort) || s_abort) break;
+            tc_fence_after();
+            const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
+            const bool is_key = nt < key_tiles;
+            const int c0 = (is_key ? nt : nt - key_tiles) * BN;
+            const int64_t n = static_cast<int64_t>(mt) * kBM + row;
+            const bool valid = n < p.n_tok;
+            const uint32_t taddr = tmem_base + acc * BN + (static_cast<uint32_t>(sub * 32) << 16);
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f;
             for (int cc = 0; cc < BN; cc += 32) {
-                float acc[32];
-                tmem_ld32(taddr + cc, acc);
+                float accv[32];
+                tmem_ld32(taddr + cc, accv);
                 if (!valid) continue;
                 if (is_key) {
                     const uint4 *hp = reinterpret_cast<const uint4 *>(p.h + n * p.d_h + c0 + cc);
+                    const uint4 *gq = reinterpret_cast<const uint4 *>(p.gamma_q + c0 + cc);
+                    const uint4 *gk = reinterpret_cast<const uint4 *>(p.gamma_k + c0 + cc);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint4 hw = __ldg(hp + q);
-                        const uint32_t w4[4] = {hw.x, hw.y, hw.z, hw.w};
+                        const uint4 hw = __ldg(hp + q), qw = __ldg(gq + q), kw = __ldg(gk + q);
+                        const uint32_t h4[4] = {hw.x, hw.y, hw.z, hw.w};
+                        const uint32_t q4[4] = {qw.x, qw.y, qw.z, qw.w};
+                        const uint32_t k4[4] = {kw.x, kw.y, kw.z, kw.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int j = q * 8 + e * 2;
-                            const float h0 = bf16_lo(w4[e]), h1 = bf16_hi(w4[e]);
-                            const float k0 = acc[j], k1 = acc[j + 1];
+                            const float h0 = bf16_lo(h4[e]), h1 = bf16_hi(h4[e]);
+                            const float g0 = bf16_lo(q4[e]) * bf16_lo(k4[e]);
+                            const float g1 = bf16_hi(q4[e]) * bf16_hi(k4[e]);
+                            const float k0 = accv[j], k1 = accv[j + 1];
                             a0 = fmaf(h0, h0, a0);
                             a0 = fmaf(h1, h1, a0);
-                            a1 = fmaf(h0 * s_gqk[cc + j], k0, a1);
-                            a1 = fmaf(h1 * s_gqk[cc + j + 1], k1, a1);
+                            a1 = fmaf(h0 * g0, k0, a1);
+                            a1 = fmaf(h1 * g1, k1, a1);
                             a2 = fmaf(k0, k0, a2);
                             a2 = fmaf(k1, k1, a2);
                         }
@@ -189,7 +223,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                     float4 *vp = reinterpret_cast<float4 *>(p.v + n * p.d_h + c0 + cc);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 x = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+                        const float4 x = make_float4(accv[4 * q], accv[4 * q + 1], accv[4 * q + 2], accv[4 * q + 3]);
                         vp[q] = x;
                         a0 = fmaf(x.x, x.x, a0);
                         a0 = fmaf(x.y, x.y, a0);
@@ -198,7 +232,11 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                     }
                 }
             }
-            if (valid) p.part[n * p.n_tiles + tile_n] = make_float4(a0, a1, a2, 0.f);
+            // the accumulator has been read: hand it back to the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+            if (valid) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
         }
     }
     tc_fence_before();
@@ -367,6 +405,135 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
                 }
                 *reinterpret_cast<uint2 *>(p.conv_state + (static_cast<int64_t>(b) * p.state_len + s) * p.d_h + c) = o;
             }
+        }
+    }
+}
+
+// Prefill fast path for the pages' conv shape (kernel 4, dilation 3, no carried state).
+// Same arithmetic as gate_conv_kernel, organised for memory-level parallelism: a CTA covers
+// 3*CH tokens of one sequence and 2*kGateFastThreads channels; each thread owns 2 channels
+// and, for each residue r of the tokens mod 3, first issues every load of its chain -- CH + 3
+// value rows (3 of them the conv halo) and CH hidden rows -- and only then computes, so a
+// thread keeps ~35 independent loads in flight instead of walking a dependent chain.
+constexpr int kGateFastThreads = 256;
+
+__device__ __forceinline__ float fast_sigmoid(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
+
+template <int CH>
+__global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(const __grid_constant__ GateParams p) {
+    constexpr int KS = 4, DIL = 3, HALO = (KS - 1) * DIL, TC = CH * DIL;
+    __shared__ float s_g[TC + HALO];
+    __shared__ float s_beta[TC + HALO];
+    const int b = blockIdx.y;
+    const int t0 = blockIdx.x * TC;
+    if (t0 >= p.T) return;
+    const int t1 = min(p.T, t0 + TC);
+    const int lo = t0 - HALO;
+    const float inv_d = 1.f / static_cast<float>(p.d_h);
+    const int64_t row0 = static_cast<int64_t>(b) * p.T;
+
+    // per-token scalars: one warp per token, lanes split the tiles, fixed-order reduction
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    for (int i = warp; i < TC + HALO; i += kGateFastThreads / 32) {
+        const int t = lo + i;
+        float g = 0.f, beta = 0.f;
+        if (t >= 0 && t < t1) {
+            const float4 *pp = p.part + (row0 + t) * p.n_tiles;
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+            for (int j = lane; j < p.n_tiles; j += 32) {
+                const float4 q = __ldg(pp + j);
+                if (j < p.n_key_tiles) {
+                    s0 += q.x;
+                    s1 += q.y;
+                    s2 += q.z;
+                } else {
+                    s3 += q.x;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+                s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+                s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+                s3 += __shfl_xor_sync(0xffffffffu, s3, o);
+            }
+            const float rms_h = sqrtf(s0 * inv_d + p.eps);
+            const float rms_k = sqrtf(s2 * inv_d + p.eps);
+            g = fast_sigmoid(s1 / (rms_h * rms_k) * p.inv_sqrt_d);
+            beta = g / sqrtf(g * g * s3 * inv_d + p.eps);
+        }
+        if (lane == 0) {
+            s_g[i] = g;
+            s_beta[i] = beta;
+        }
+    }
+    __syncthreads();
+
+    const int q = blockIdx.z * blockDim.x + threadIdx.x;
+    if (q >= p.d_h / 2) return;
+    const int c = q * 2;
+    float gc[2], w[2][KS];
+    {
+        const uint32_t gw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_c + c));
+        gc[0] = bf16_lo(gw);
+        gc[1] = bf16_hi(gw);
+        const uint2 *wp = reinterpret_cast<const uint2 *>(p.conv_w + c * KS);   // 2 channels x 4 taps
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const uint2 ww = __ldg(wp + e);
+            w[e][0] = bf16_lo(ww.x); w[e][1] = bf16_hi(ww.x); w[e][2] = bf16_lo(ww.y); w[e][3] = bf16_hi(ww.y);
+        }
+    }
+#pragma unroll 1
+    for (int r = 0; r < DIL; ++r) {
+        float2 vv[CH + KS - 1];
+        uint32_t hh[CH];
+#pragma unroll
+        for (int j = 0; j < CH + KS - 1; ++j) {
+            const int t = lo + r + DIL * j;
+            vv[j] = (t >= 0 && t < t1) ? __ldg(reinterpret_cast<const float2 *>(p.v + (row0 + t) * p.d_h + c))
+                                       : make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+            const int t = t0 + r + DIL * j;
+            hh[j] = t < t1 ? __ldg(reinterpret_cast<const uint32_t *>(p.h + (row0 + t) * p.d_h + c)) : 0u;
+        }
+        float u[KS][2];   // u[i] holds the conv input i chain steps back
+#pragma unroll
+        for (int i = 0; i < KS; ++i) u[i][0] = u[i][1] = 0.f;
+#pragma unroll
+        for (int j = 0; j < CH + KS - 1; ++j) {
+            const int si = r + DIL * j;            // index into s_g / s_beta
+            const float beta = s_beta[si];
+            const float vj[2] = {vv[j].x, vv[j].y};
+#pragma unroll
+            for (int i = KS - 1; i > 0; --i) {
+                u[i][0] = u[i - 1][0];
+                u[i][1] = u[i - 1][1];
+            }
+            u[0][0] = beta * vj[0] * gc[0];
+            u[0][1] = beta * vj[1] * gc[1];
+            if (j < KS - 1) continue;
+            const int t = lo + si;
+            if (t >= t1) continue;
+            const float g = s_g[si];
+            const uint32_t hw = hh[j - (KS - 1)];
+            const float hv[2] = {bf16_lo(hw), bf16_hi(hw)};
+            float dl[2];
+            uint32_t ob[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float acc = 0.f;
+#pragma unroll
+                for (int i = 0; i < KS; ++i) acc = fmaf(w[e][i], u[i][e], acc);
+                dl[e] = fmaf(g, vj[e], acc * fast_sigmoid(acc));
+                ob[e] = f32_to_bf16_bits(hv[e] + dl[e]);
+            }
+            const int64_t n = row0 + t;
+            *reinterpret_cast<uint32_t *>(p.out + n * p.d_h + c) = ob[0] | (ob[1] << 16);
+            if (p.delta != nullptr)
+                *reinterpret_cast<float2 *>(p.delta + n * p.d_h + c) = make_float2(dl[0], dl[1]);
         }
     }
 }

@@ -171,7 +171,11 @@ int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
  * in the compressed vocabulary.  history / conv_state: NULL for prefill, or the decode state
  * (read, then updated in place).  Other arguments as in the steps above.
  * stage_events: NULL, or an array of ENGRAM_FORWARD_STAGES + 1 cudaEvent_t recorded on
- * `stream` before each stage and after the last (a profiling hook; no effect on results). */
+ * `stream` before each stage and after the last (a profiling hook; no effect on results).
+ * Under stream capture they are recorded as external event nodes, so a replayed graph can
+ * be timed per stage.
+ * CUDA graphs: after one eager call on a device (which resolves the tensor-map encoder and
+ * sets kernel attributes), engram_forward / engram_gate_conv may be captured and replayed. */
 #define ENGRAM_FORWARD_STAGES 4 /* hash, gather, projections, gate+conv */
 int engram_forward(const engram_plan *plan, const engram_weights *w,
                    const uint16_t *const *tables, const int32_t *ids, const int32_t *remap,

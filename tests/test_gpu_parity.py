@@ -242,3 +242,25 @@ def test_forward_full_size_layer2560_sampled():
         ds.append(got_d[n]); rs.append(d_ref); os_.append(got_o[n]); ros.append(o_ref)
     assert_delta_close(np.stack(ds), np.stack(rs))
     assert_out_close(np.stack(os_), np.stack(ros))
+
+
+def test_forward_replays_identically_in_a_cuda_graph():
+    """After one eager call on the device, engram_forward can be captured in a CUDA graph;
+    replays give the eager result bit for bit."""
+    wl = PARITY_CASES["ragged_k_bn64"]
+    di = DeviceInputs(wl).forward(delta=False)
+    torch.cuda.synchronize()
+    eager = di.out.clone()
+    di.out.zero_()
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+        E.engram_forward(di.plan, di.weights, di.tables, di.ids, di.h, di.out, di.ws, remap=di.remap,
+                         stream=torch.cuda.current_stream())
+    torch.cuda.current_stream().wait_stream(cap)
+    for _ in range(2):
+        di.out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(di.out.view(torch.int16), eager.view(torch.int16))

@@ -10,5 +10,5 @@ from ._native import (  # noqa: F401
     ENGRAM_STATUS_BAD_TOKEN, ENGRAM_STATUS_WAIT_TIMEOUT, ENGRAM_TABLES_DEVICE,
     ENGRAM_TABLES_HOST_MAPPED, ENGRAM_NOALLOC_SCRATCH_BYTES, EngramError, LIB_PATH, Plan, Weights, alloc_workspace,
     engram_advance_history, engram_device_status, engram_forward, engram_gate_conv,
-    engram_gate_conv_noalloc, engram_gather, engram_hash, engram_remap, engram_workspace_size, last_error, lib, version,
+    engram_gate_conv_noalloc, engram_gather, engram_hash, engram_stage_rows, engram_remap, engram_workspace_size, last_error, lib, version,
 )

@@ -91,6 +91,8 @@ def _load():
         "engram_hash": (C.c_int, [P, P, i32, i32, P, P, P]),
         "engram_advance_history": (C.c_int, [P, P, i32, i32, P, P]),
         "engram_gather": (C.c_int, [P, P, P, i64, P, P]),
+        "engram_stage_rows": (C.c_int, [P, P, i64, P, P, i32, P, P, P, P]),
+        "engram_gather_bounded": (C.c_int, [P, P, P, i64, i64, P, P]),
         "engram_gate_conv": (C.c_int, [P, P, P, P, i32, i32, P, P, P, P, sz, P]),
         "engram_forward": (C.c_int, [P, P, P, P, P, i32, i32, P, P, P, P, P, P, sz, P, P]),
         "engram_gate_conv_noalloc": (C.c_int, [P, P, P, P, i32, i32, P, P, P, P]),
@@ -250,10 +252,28 @@ def engram_advance_history(plan: Plan, ids_remapped: torch.Tensor, history: torc
                                       _ptr(history, torch.int32, "history"), _stream(stream)))
 
 
-def engram_gather(plan: Plan, idx: torch.Tensor, tables, m: torch.Tensor, stream=None):
+def engram_gather(plan: Plan, idx: torch.Tensor, tables, m: torch.Tensor, stream=None, rows_bound: int = 0):
+    """rows_bound > 0: every table holds only that many rows (device staging buffers from
+    engram_stage_rows); row ids at or beyond it read a zero row and raise the status bit."""
     arr = _table_array(tables)
+    if rows_bound:
+        _check(lib.engram_gather_bounded(plan, _ptr(idx, (torch.int32, torch.uint32), "idx"), arr, idx.shape[0],
+                                         int(rows_bound), _ptr(m, _BF16, "m"), _stream(stream)))
+        return
     _check(lib.engram_gather(plan, _ptr(idx, (torch.int32, torch.uint32), "idx"), arr, idx.shape[0],
                              _ptr(m, _BF16, "m"), _stream(stream)))
+
+
+def engram_stage_rows(plan: Plan, idx: torch.Tensor, tables, staging, staged_idx: torch.Tensor,
+                      unique_rows: torch.Tensor, n_unique: torch.Tensor, stream=None):
+    """Copy each distinct row the batch needs from (host-mapped) tables into device staging."""
+    n_tok = idx.shape[0]
+    cap = staging[0].shape[0]
+    _check(lib.engram_stage_rows(plan, _ptr(idx, (torch.int32, torch.uint32), "idx"), n_tok,
+                                 _table_array(tables), _table_array(staging), cap,
+                                 _ptr(staged_idx, (torch.int32, torch.uint32), "staged_idx"),
+                                 _ptr(unique_rows, (torch.int32, torch.uint32), "unique_rows"),
+                                 _ptr(n_unique, torch.int32, "n_unique"), _stream(stream)))
 
 
 def engram_gate_conv(plan: Plan, weights: Weights, h: torch.Tensor, m: torch.Tensor, B: int, T: int,

@@ -103,7 +103,10 @@ int check_plan(const engram_plan *plan) {
 
 // ---------------------------------------------------------------- workspace layout
 struct Workspace {
-    size_t xr, idx, m, v, part, total;
+    size_t xr, idx, m, v, part;
+    size_t staged_idx, unique, n_unique, staging;  // host-resident tables only
+    bool staged;                                   // rows go through device staging
+    size_t total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -139,6 +142,13 @@ Workspace layout(const engram_plan *plan, int64_t n_tok) {
     w.m = off;    off = align256(off + sizeof(uint16_t) * n_tok * plan->mem_dim);
     w.v = off;    off = align256(off + sizeof(float) * n_tok * d_h);
     w.part = off; off = align256(off + sizeof(float4) * n_tok * n_tiles);
+    w.staged = plan->cfg.table_location == ENGRAM_TABLES_HOST_MAPPED && n_tok <= engram::kStageMaxTok;
+    if (w.staged) {
+        w.staged_idx = off; off = align256(off + sizeof(uint32_t) * n_tok * H);
+        w.unique = off;     off = align256(off + sizeof(uint32_t) * n_tok * H);
+        w.n_unique = off;   off = align256(off + sizeof(int32_t) * H);
+        w.staging = off;    off = align256(off + sizeof(uint16_t) * n_tok * H * plan->cfg.row_dim);
+    }
     w.total = off;
     return w;
 }
@@ -273,13 +283,14 @@ int launch_hash(const engram_plan *plan, const int32_t *ids, const int32_t *rema
 }
 
 
+// rows_override > 0 bounds every table at that many rows (device staging buffers).
 int launch_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables, int64_t n_tok,
-                  uint16_t *m, cudaStream_t stream) {
+                  uint16_t *m, cudaStream_t stream, int64_t rows_override = 0) {
     engram::GatherParams p{};
     const int H = plan->num_tables;
     for (int h = 0; h < H; ++h) {
         p.table[h] = tables[h];
-        p.rows[h] = static_cast<uint64_t>(plan->cfg.table_rows[h]);
+        p.rows[h] = static_cast<uint64_t>(rows_override > 0 ? rows_override : plan->cfg.table_rows[h]);
     }
     p.H = H;
     p.chunks_per_row = plan->cfg.row_dim / 8;
@@ -337,6 +348,42 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
     if (fast) engram::gate_conv_k4d3_kernel<kChain><<<grid, threads, 0, stream>>>(p);
     else engram::gate_conv_kernel<<<grid, threads, smem, stream>>>(p);
     ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_conv_kernel launch");
+    return ENGRAM_OK;
+}
+
+int launch_stage(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, const uint16_t *const *tables,
+                 uint16_t *const *staging, int32_t capacity, uint32_t *staged_idx, uint32_t *unique_rows,
+                 int32_t *n_unique, cudaStream_t stream) {
+    const int H = plan->num_tables;
+    int N = 1;
+    while (N < n_tok) N <<= 1;
+    const size_t smem = sizeof(uint32_t) * 2 * static_cast<size_t>(N);
+    if (smem > 48 * 1024)
+        ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::stage_dedup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem)),
+                        "cudaFuncSetAttribute(stage_dedup_kernel)");
+    engram::stage_dedup_kernel<<<H, engram::kDedupThreads, smem, stream>>>(
+        idx, static_cast<int32_t>(n_tok), H, capacity, staged_idx, unique_rows, n_unique);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "stage_dedup_kernel launch");
+    engram::StageParams p{};
+    for (int h = 0; h < H; ++h) {
+        p.table[h] = tables[h];
+        p.staging[h] = staging[h];
+        p.rows[h] = static_cast<uint64_t>(plan->cfg.table_rows[h]);
+    }
+    p.unique_rows = unique_rows;
+    p.n_unique = n_unique;
+    p.H = H;
+    p.capacity = capacity;
+    p.chunks_per_row = plan->cfg.row_dim / 8;
+    const int64_t total = static_cast<int64_t>(H) * n_tok * p.chunks_per_row;
+    constexpr int kUnroll = 4;
+    int64_t blocks = (total + 256 * kUnroll - 1) / (256 * kUnroll);
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    engram::stage_copy_kernel<kUnroll><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "stage_copy_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -533,6 +580,42 @@ int engram_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *
     return launch_gather(plan, idx, tables, n_tok, m, static_cast<cudaStream_t>(stream));
 }
 
+int engram_gather_bounded(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables,
+                          int64_t n_tok, int64_t rows, uint16_t *m, engram_stream_t stream) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if (n_tok < 0 || rows < 1) return fail(ENGRAM_ERR_INVALID_ARG, "n_tok must be >= 0 and rows >= 1");
+    if (n_tok == 0) return ENGRAM_OK;
+    if (!idx || !tables || !m) return fail(ENGRAM_ERR_INVALID_ARG, "idx, tables and m must be non-NULL");
+    if (!aligned16(m)) return fail(ENGRAM_ERR_INVALID_ARG, "m is not 16-byte aligned");
+    for (int h = 0; h < plan->num_tables; ++h) {
+        if (!tables[h]) return fail(ENGRAM_ERR_INVALID_ARG, "tables[%d] is NULL", h);
+        if (!aligned16(tables[h])) return fail(ENGRAM_ERR_INVALID_ARG, "tables[%d] is not 16-byte aligned", h);
+    }
+    return launch_gather(plan, idx, tables, n_tok, m, static_cast<cudaStream_t>(stream), rows);
+}
+
+int engram_stage_rows(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, const uint16_t *const *tables,
+                      uint16_t *const *staging, int32_t capacity, uint32_t *staged_idx, uint32_t *unique_rows,
+                      int32_t *n_unique, engram_stream_t stream) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if (n_tok < 0) return fail(ENGRAM_ERR_INVALID_ARG, "n_tok must be >= 0");
+    if (n_tok == 0) return ENGRAM_OK;
+    if (n_tok > engram::kStageMaxTok)
+        return fail(ENGRAM_ERR_UNSUPPORTED, "engram_stage_rows handles at most %d tokens per call", engram::kStageMaxTok);
+    if (capacity < n_tok) return fail(ENGRAM_ERR_INVALID_ARG, "capacity %d < n_tok %lld", capacity, (long long)n_tok);
+    if (!idx || !tables || !staging || !staged_idx || !unique_rows || !n_unique)
+        return fail(ENGRAM_ERR_INVALID_ARG, "NULL argument");
+    for (int h = 0; h < plan->num_tables; ++h) {
+        if (!tables[h] || !staging[h]) return fail(ENGRAM_ERR_INVALID_ARG, "tables[%d] or staging[%d] is NULL", h, h);
+        if (!aligned16(tables[h]) || !aligned16(staging[h]))
+            return fail(ENGRAM_ERR_INVALID_ARG, "tables[%d] / staging[%d] not 16-byte aligned", h, h);
+    }
+    return launch_stage(plan, idx, n_tok, tables, staging, capacity, staged_idx, unique_rows, n_unique,
+                        static_cast<cudaStream_t>(stream));
+}
+
 int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                      int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out, float *delta_dbg, void *workspace,
                      size_t workspace_bytes, engram_stream_t stream) {
@@ -589,7 +672,22 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const uint1
     if ((rc = rec(0)) != ENGRAM_OK) return rc;
     if ((rc = launch_hash(plan, ids, remap, history, B, T, idx, xr, stream)) != ENGRAM_OK) return rc;
     if ((rc = rec(1)) != ENGRAM_OK) return rc;
-    if ((rc = launch_gather(plan, idx, tables, n_tok, m, stream)) != ENGRAM_OK) return rc;
+    if (L.staged) {
+        // host-resident tables: fetch each distinct row of the batch once into HBM staging,
+        // then gather from there (results are bit-identical to the HBM-resident path)
+        const int H = plan->num_tables;
+        uint16_t *stage_ptr[ENGRAM_MAX_TABLES];
+        for (int h = 0; h < H; ++h)
+            stage_ptr[h] = reinterpret_cast<uint16_t *>(ws + L.staging) + static_cast<int64_t>(h) * n_tok * plan->cfg.row_dim;
+        uint32_t *sidx = reinterpret_cast<uint32_t *>(ws + L.staged_idx);
+        if ((rc = launch_stage(plan, idx, n_tok, tables, stage_ptr, static_cast<int32_t>(n_tok), sidx,
+                               reinterpret_cast<uint32_t *>(ws + L.unique), reinterpret_cast<int32_t *>(ws + L.n_unique),
+                               stream)) != ENGRAM_OK)
+            return rc;
+        if ((rc = launch_gather(plan, sidx, stage_ptr, n_tok, m, stream, n_tok)) != ENGRAM_OK) return rc;
+    } else if ((rc = launch_gather(plan, idx, tables, n_tok, m, stream)) != ENGRAM_OK) {
+        return rc;
+    }
     if ((rc = gate_conv_impl(plan, w, h, m, B, T, conv_state, out, delta_dbg, ws, stream,
                              stage_events ? stage_events + 2 : nullptr)) != ENGRAM_OK)
         return rc;

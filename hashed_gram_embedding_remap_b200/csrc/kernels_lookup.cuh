@@ -174,4 +174,138 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint32_t *__restrict_
     }
 }
 
+// ---------------------------------------------------------------- host-resident tables
+// A step's row ids are known before its compute starts, so the rows a batch needs can be
+// fetched from host memory ahead of use.  stage_dedup_kernel (one CTA per table) sorts the
+// batch's row ids with their positions in shared memory (bitonic), marks the first of each
+// run of equal ids, and assigns slots in sorted order: unique[h][s] is the s-th distinct row
+// id and staged_idx[n, h] the slot of token n.  stage_copy_kernel then copies only the
+// distinct rows from the (pinned, mapped) host tables into device staging, many CTAs wide so
+// that enough reads are in flight to fill the host link.
+constexpr int kStageMaxTok = 8192;
+constexpr int kDedupThreads = 1024;
+
+__global__ void __launch_bounds__(kDedupThreads) stage_dedup_kernel(const uint32_t *__restrict__ idx, int32_t n,
+                                                                    int32_t H, int32_t capacity,
+                                                                    uint32_t *__restrict__ staged_idx,
+                                                                    uint32_t *__restrict__ unique_rows,
+                                                                    int32_t *__restrict__ n_unique) {
+    extern __shared__ uint32_t s_dd[];
+    int N = 1;
+    while (N < n) N <<= 1;
+    uint32_t *key = s_dd;
+    uint32_t *pos = s_dd + N;
+    __shared__ int32_t s_count[kDedupThreads / 32];
+    const int h = blockIdx.x;
+    for (int i = threadIdx.x; i < N; i += blockDim.x) {
+        key[i] = i < n ? idx[static_cast<int64_t>(i) * H + h] : 0xFFFFFFFFu;
+        pos[i] = static_cast<uint32_t>(i);
+    }
+    __syncthreads();
+    // bitonic sort of (key, pos) pairs, ascending; positions break ties (stable order)
+    for (int k = 2; k <= N; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < N; i += blockDim.x) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const bool up = (i & k) == 0;
+                    const uint64_t a = (static_cast<uint64_t>(key[i]) << 32) | pos[i];
+                    const uint64_t b = (static_cast<uint64_t>(key[l]) << 32) | pos[l];
+                    if ((a > b) == up) {
+                        key[i] = static_cast<uint32_t>(b >> 32);
+                        pos[i] = static_cast<uint32_t>(b);
+                        key[l] = static_cast<uint32_t>(a >> 32);
+                        pos[l] = static_cast<uint32_t>(a);
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    // each thread owns a contiguous segment; count run heads, block-scan the counts
+    const int per = (N + blockDim.x - 1) / blockDim.x;
+    const int beg = threadIdx.x * per;
+    const int end = min(n, beg + per);
+    int cnt = 0;
+    for (int i = beg; i < end; ++i) cnt += (i == 0 || key[i] != key[i - 1]);
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_count[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < blockDim.x / 32 ? s_count[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += v;
+        }
+        if (lane < blockDim.x / 32) s_count[lane] = wi - w;   // exclusive warp offsets
+        if (lane == 31) n_unique[h] = wi;
+    }
+    __syncthreads();
+    int slot = s_count[warp] + incl - cnt;   // exclusive offset of this thread's first head
+    for (int i = beg; i < end; ++i) {
+        const bool head = (i == 0 || key[i] != key[i - 1]);
+        if (head) {
+            unique_rows[static_cast<int64_t>(h) * capacity + slot] = key[i];
+            ++slot;
+        }
+        staged_idx[static_cast<int64_t>(pos[i]) * H + h] = static_cast<uint32_t>(slot - 1);
+    }
+}
+
+struct StageParams {
+    const uint16_t *table[ENGRAM_MAX_TABLES];  // host-mapped
+    uint16_t *staging[ENGRAM_MAX_TABLES];      // device, [capacity, d_e]
+    uint64_t rows[ENGRAM_MAX_TABLES];
+    const uint32_t *unique_rows;               // [H, capacity]
+    const int32_t *n_unique;                   // [H]
+    int32_t H, capacity, chunks_per_row;
+};
+
+template <int UNROLL>
+__global__ void __launch_bounds__(256) stage_copy_kernel(const __grid_constant__ StageParams p) {
+    const int64_t per_table = static_cast<int64_t>(p.capacity) * p.chunks_per_row;
+    const int64_t total = per_table * p.H;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < total;
+         base += stride * UNROLL) {
+        uint4 val[UNROLL];
+        int64_t dst[UNROLL];
+        int hh[UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            const int64_t i = base + u * stride;
+            dst[u] = -1;
+            hh[u] = 0;
+            if (i < total) {
+                const int h = static_cast<int>(i / per_table);
+                const int64_t r = i - h * per_table;
+                const int32_t s = static_cast<int32_t>(r / p.chunks_per_row);
+                const int32_t c = static_cast<int32_t>(r - static_cast<int64_t>(s) * p.chunks_per_row);
+                if (s < __ldg(p.n_unique + h)) {
+                    const uint32_t row = __ldg(p.unique_rows + static_cast<int64_t>(h) * p.capacity + s);
+                    hh[u] = h;
+                    dst[u] = r;
+                    if (row < p.rows[h]) {
+                        val[u] = reinterpret_cast<const uint4 *>(p.table[h])[static_cast<int64_t>(row) * p.chunks_per_row + c];
+                    } else {
+                        val[u] = make_uint4(0, 0, 0, 0);
+                        atomicOr(&g_engram_status, ENGRAM_STATUS_BAD_ROW);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u)
+            if (dst[u] >= 0) reinterpret_cast<uint4 *>(p.staging[hh[u]])[dst[u]] = val[u];
+    }
+}
+
 }  // namespace engram

@@ -149,6 +149,33 @@ int engram_advance_history(const engram_plan *plan, const int32_t *ids_remapped,
 int engram_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables,
                   int64_t n_tok, uint16_t *m, engram_stream_t stream);
 
+/* Step 3 with host-resident tables (a7) [zhichai §2.3: the row ids are known as soon as the
+ * token enters the network, so the table can live in host memory and be prefetched;
+ * communeify "Engram 到底是什麼": asynchronous prefetch from system RAM overlapped with
+ * compute; xiaodao: host memory and the host link become the bottleneck].
+ * Copies each DISTINCT row the batch needs, once, from the tables into device staging:
+ *   staging[h][staged_idx[n, h], :] == tables[h][idx[n, h], :]   for every token n.
+ * idx: uint32 [n_tok, H] (device).  tables: HOST array of H pointers to pinned, mapped
+ * host memory (or device memory) [table_rows[h], d_e].  staging: HOST array of H device
+ * pointers, each [capacity, d_e].  staged_idx: uint32 [n_tok, H] (device, out).
+ * unique_rows: uint32 [H, capacity] (device, out): the distinct row ids in increasing order.
+ * n_unique: int32 [H] (device, out).  n_tok <= capacity, n_tok <= 8192.
+ * The copy is done by a kernel reading the mapped host memory directly (zero-copy), many
+ * CTAs wide; call it on a side stream to overlap the host-link transfer with other work.
+ * engram_forward takes this path itself when cfg.table_location is
+ * ENGRAM_TABLES_HOST_MAPPED and B*T <= 8192 (above that it gathers straight from the mapped
+ * tables); results are bit-identical to HBM-resident tables. */
+int engram_stage_rows(const engram_plan *plan, const uint32_t *idx, int64_t n_tok,
+                      const uint16_t *const *tables, uint16_t *const *staging, int32_t capacity,
+                      uint32_t *staged_idx, uint32_t *unique_rows, int32_t *n_unique,
+                      engram_stream_t stream);
+
+/* engram_gather over tables that all hold `rows` rows (e.g. the staging buffers filled by
+ * engram_stage_rows, with staged_idx as idx).  Same layout and error behaviour as
+ * engram_gather, with `rows` as every table's bound. */
+int engram_gather_bounded(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables,
+                          int64_t n_tok, int64_t rows, uint16_t *m, engram_stream_t stream);
+
 /* Steps 4-6 [yktysq #3, #4; zhichai §2.3]: gate, conv, residual for B sequences of T tokens.
  * h: bf16 [B*T, d_h] hidden states.  m: bf16 [B*T, d_m] memory vectors.
  * conv_state: NULL for prefill (zero left padding), or bf16 [B, state_len, d_h] conv inputs

@@ -56,4 +56,14 @@ int synth_fill_bf16(void *dst, uint64_t n, uint64_t offset, uint64_t key, float 
     return static_cast<int>(cudaGetLastError());
 }
 
+// Pinned host memory mapped into the device address space (for host-resident tables).
+// Returns a cudaError_t code; *out receives a pointer usable from host and device.
+int synth_host_alloc_mapped(uint64_t bytes, void **out) {
+    if (out == nullptr) return static_cast<int>(cudaErrorInvalidValue);
+    *out = nullptr;
+    return static_cast<int>(cudaHostAlloc(out, bytes, cudaHostAllocMapped | cudaHostAllocPortable));
+}
+
+int synth_host_free(void *p) { return static_cast<int>(cudaFreeHost(p)); }
+
 }  // extern "C"

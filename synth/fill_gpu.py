@@ -32,6 +32,10 @@ def _get():
         L = C.CDLL(_LIB)
         L.synth_fill_bf16.restype = C.c_int
         L.synth_fill_bf16.argtypes = [C.c_void_p, C.c_uint64, C.c_uint64, C.c_uint64, C.c_float, C.c_void_p]
+        L.synth_host_alloc_mapped.restype = C.c_int
+        L.synth_host_alloc_mapped.argtypes = [C.c_uint64, C.POINTER(C.c_void_p)]
+        L.synth_host_free.restype = C.c_int
+        L.synth_host_free.argtypes = [C.c_void_p]
         _lib = L
     return _lib
 
@@ -51,3 +55,30 @@ def fill_(t: torch.Tensor, spec: FillSpec, offset: int = 0, stream=None) -> torc
 def filled(shape, spec: FillSpec, device="cuda") -> torch.Tensor:
     t = torch.empty(shape, dtype=torch.bfloat16, device=device)
     return fill_(t, spec)
+
+
+class HostMapped:
+    """A pinned, device-mapped host buffer viewed as a CPU torch tensor of bf16 [rows, cols].
+    Its data_ptr() is valid on the device too (unified addressing).  Freed by close()."""
+
+    def __init__(self, rows: int, cols: int):
+        self.ptr = C.c_void_p()
+        nbytes = int(rows) * int(cols) * 2
+        rc = _get().synth_host_alloc_mapped(nbytes, C.byref(self.ptr))
+        if rc != 0 or not self.ptr.value:
+            raise MemoryError(f"cudaHostAlloc({nbytes} bytes, mapped) failed with CUDA error {rc}")
+        import numpy as np
+        arr = np.ctypeslib.as_array((C.c_int16 * (int(rows) * int(cols))).from_address(self.ptr.value))
+        self.tensor = torch.from_numpy(arr).view(torch.bfloat16).view(int(rows), int(cols))
+
+    def close(self):
+        if self.ptr is not None and self.ptr.value:
+            self.tensor = None
+            _get().synth_host_free(self.ptr)
+            self.ptr = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -418,7 +418,7 @@ def run_hostpinned(args, wl, world, rank, local):
     torch.cuda.set_device(local)
     fill_gpu.build()
     comp = torch.cuda.current_stream()
-    pref = torch.cuda.Stream()
+    pref = torch.cuda.Stream(priority=-1)   # prefetch kernels get SMs ahead of the stand-in GEMM
     t0 = time.perf_counter()
     bufs = [fill_gpu.HostMapped(wl.primes[h], wl.d_e) for h in range(wl.H)]
     for h, b in enumerate(bufs):
@@ -596,11 +596,17 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch every step from the host (no CUDA graph)")
     ap.add_argument("--ids", choices=["uniform", "zipf"], default=None, help="id distribution (host-pinned workload)")
+    ap.add_argument("--table-rows", type=int, default=0, help="override the table size (largest prime <= N)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = synth.get_workload(args.workload)
+    if args.table_rows:
+        # same kernels and shapes with smaller tables (for profiling captures that must stay small)
+        p = synth.largest_prime_below(args.table_rows + 1) if synth.workloads.is_prime(args.table_rows) is False \
+            else args.table_rows
+        wl = wl.with_(primes=(p,) * wl.H, name=f"{wl.name}[rows={p}]")
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -103,7 +103,7 @@ int check_plan(const engram_plan *plan) {
 
 // ---------------------------------------------------------------- workspace layout
 struct Workspace {
-    size_t xr, idx, m, v, part;
+    size_t xr, idx, m, v, part, acc;
     size_t staged_idx, unique, n_unique, staging;  // host-resident tables only
     bool staged;                                   // rows go through device staging
     size_t total;
@@ -130,18 +130,60 @@ int choose_bn(int d_h, int64_t n_tok) {
     return 64;
 }
 
+// Work decomposition of the projection for n_tok tokens.  When even the widest tile leaves
+// most SMs idle (decode-sized batches), K is split so that every SM streams its own slice of
+// the weights; the split-K partial accumulators are finished by splitk_reduce_kernel.
+struct ProjShape {
+    int bn, n_tiles, k_blocks, k_splits, kb_per_split;
+};
+
+ProjShape proj_shape(const engram_plan *plan, int64_t n_tok, bool allow_split) {
+    ProjShape ps{};
+    const int d_h = plan->cfg.hidden_dim;
+    ps.k_blocks = (plan->mem_dim + engram::kBK - 1) / engram::kBK;
+    ps.k_splits = 1;
+    ps.kb_per_split = ps.k_blocks;
+    const int64_t m_tiles = (n_tok + engram::kBM - 1) / engram::kBM;
+    const int sms = 148;
+    int wide = 64;
+    for (int bn : {256, 128}) {
+        if (d_h % bn == 0) {
+            wide = bn;
+            break;
+        }
+    }
+    const int64_t mn = m_tiles * (2 * d_h / wide);
+    int splits = 1;
+    if (allow_split && mn > 0 && mn < sms) {
+        splits = static_cast<int>(sms / mn);
+        if (splits > ps.k_blocks / 4) splits = ps.k_blocks / 4;
+        if (splits < 1) splits = 1;
+    }
+    if (splits > 1) {
+        ps.bn = wide;
+        ps.kb_per_split = (ps.k_blocks + splits - 1) / splits;
+        ps.k_splits = (ps.k_blocks + ps.kb_per_split - 1) / ps.kb_per_split;
+    } else {
+        ps.bn = choose_bn(d_h, n_tok);
+    }
+    ps.n_tiles = 2 * d_h / ps.bn;
+    return ps;
+}
+
 Workspace layout(const engram_plan *plan, int64_t n_tok) {
     Workspace w{};
     const int H = plan->num_tables;
     const int d_h = plan->cfg.hidden_dim;
-    const int bn = choose_bn(d_h, n_tok);
-    const int n_tiles = 2 * d_h / bn;
+    const ProjShape ps = proj_shape(plan, n_tok, true);
+    const int n_tiles = ps.n_tiles;
     size_t off = 0;
     w.xr = off;   off = align256(off + sizeof(int32_t) * n_tok);
     w.idx = off;  off = align256(off + sizeof(uint32_t) * n_tok * H);
     w.m = off;    off = align256(off + sizeof(uint16_t) * n_tok * plan->mem_dim);
     w.v = off;    off = align256(off + sizeof(float) * n_tok * d_h);
     w.part = off; off = align256(off + sizeof(float4) * n_tok * n_tiles);
+    w.acc = off;
+    if (ps.k_splits > 1) off = align256(off + sizeof(float) * ps.k_splits * n_tok * 2 * d_h);
     w.staged = plan->cfg.table_location == ENGRAM_TABLES_HOST_MAPPED && n_tok <= engram::kStageMaxTok;
     if (w.staged) {
         w.staged_idx = off; off = align256(off + sizeof(uint32_t) * n_tok * H);
@@ -211,7 +253,8 @@ int set_proj_smem_attr() {
 
 template <int BN>
 int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
-                int64_t n_tok, float *v, float4 *part, cudaStream_t stream) {
+                int64_t n_tok, float *v, float4 *part, cudaStream_t stream, float *acc = nullptr,
+                int k_splits = 1, int kb_per_split = 0) {
     const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim;
     CUtensorMap map_m, map_wk, map_wv;
     int rc;
@@ -231,13 +274,21 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     p.n_tiles = 2 * d_h / BN;
     p.k_blocks = (d_m + engram::kBK - 1) / engram::kBK;
     p.m_tiles = static_cast<int32_t>((n_tok + engram::kBM - 1) / engram::kBM);
-    const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+    p.k_splits = (acc != nullptr && k_splits > 1) ? k_splits : 1;
+    p.kb_per_split = p.k_splits > 1 ? kb_per_split : p.k_blocks;
+    p.acc_out = p.k_splits > 1 ? acc : nullptr;
+    const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles * p.k_splits;
     if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
     const int64_t sms = sm_count();
     dim3 grid(static_cast<unsigned>(total < sms ? total : sms));
     engram::proj_kernel<BN><<<grid, engram::kProjThreads, engram::ProjCfg<BN>::kSmemBytes, stream>>>(
         map_m, map_wk, map_wv, p);
     ENGRAM_CUDA_TRY(cudaGetLastError(), "proj_kernel launch");
+    if (p.k_splits > 1) {
+        engram::splitk_reduce_kernel<<<dim3(p.n_tiles, static_cast<unsigned>(n_tok)), engram::kReduceThreads, 0,
+                                       stream>>>(p, BN);
+        ENGRAM_CUDA_TRY(cudaGetLastError(), "splitk_reduce_kernel launch");
+    }
     return ENGRAM_OK;
 }
 
@@ -331,8 +382,8 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
     p.dil = plan->cfg.conv_dilation;
     p.state_len = plan->state_len;
     constexpr int kChain = 12;   // outputs per residue chain in the k=4, dilation-3 fast path
-    const bool fast = conv_state == nullptr && p.ksize == 4 && p.dil == 3;
-    p.tok_chunk = conv_state != nullptr ? T : (fast ? 3 * kChain : 32);
+    const bool fast = p.ksize == 4 && p.dil == 3 && (conv_state == nullptr || T <= 3 * kChain);
+    p.tok_chunk = fast ? 3 * kChain : (conv_state != nullptr ? T : 32);
     p.eps = plan->cfg.eps;
     p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(d_h));
     const int threads = fast ? engram::kGateFastThreads : engram::kGateThreads;
@@ -343,6 +394,12 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
         ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::gate_conv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem)),
                         "cudaFuncSetAttribute(gate_conv_kernel)");
+    }
+    if (fast && conv_state != nullptr && T == 1) {
+        const unsigned dslices = static_cast<unsigned>((d_h / 2 + engram::kDecodeThreads - 1) / engram::kDecodeThreads);
+        engram::gate_conv_decode_kernel<<<dim3(dslices, static_cast<unsigned>(B)), engram::kDecodeThreads, 0, stream>>>(p);
+        ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_conv_decode_kernel launch");
+        return ENGRAM_OK;
     }
     dim3 grid(static_cast<unsigned>((T + p.tok_chunk - 1) / p.tok_chunk), static_cast<unsigned>(B), slices);
     if (fast) engram::gate_conv_k4d3_kernel<kChain><<<grid, threads, 0, stream>>>(p);
@@ -403,18 +460,18 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
                    cudaStream_t stream, void *const *events) {
     const int64_t n_tok = static_cast<int64_t>(B) * T;
     const Workspace L = layout(plan, n_tok);
-    const int d_h = plan->cfg.hidden_dim;
-    const int bn = choose_bn(d_h, n_tok);
+    const ProjShape ps = proj_shape(plan, n_tok, true);
     float *v = reinterpret_cast<float *>(ws + L.v);
     float4 *part = reinterpret_cast<float4 *>(ws + L.part);
+    float *acc = ps.k_splits > 1 ? reinterpret_cast<float *>(ws + L.acc) : nullptr;
     int rc;
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[0], stream), "cudaEventRecord");
-    if (bn == 256) rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream);
-    else if (bn == 128) rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream);
-    else rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream);
+    if (ps.bn == 256) rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split);
+    else if (ps.bn == 128) rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split);
+    else rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split);
     if (rc != ENGRAM_OK) return rc;
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[1], stream), "cudaEventRecord");
-    return launch_gate_conv(plan, w, h, v, part, 2 * d_h / bn, B, T, conv_state, out, delta, stream);
+    return launch_gate_conv(plan, w, h, v, part, ps.n_tiles, B, T, conv_state, out, delta, stream);
 }
 
 int check_bt(int32_t B, int32_t T) {

@@ -55,6 +55,9 @@ struct ProjParams {
     int32_t n_tiles;           // 2 * d_h / BN: key tiles first, then value tiles
     int32_t k_blocks;          // ceil(d_m / kBK)
     int32_t m_tiles;           // ceil(n_tok / kBM)
+    int32_t k_splits;          // > 1: split-K, raw fp32 partial accumulators go to acc_out
+    int32_t kb_per_split;      // k-blocks per split
+    float *acc_out;            // [k_splits, n_tok, 2*d_h] when k_splits > 1
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -88,7 +91,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int total = p.m_tiles * p.n_tiles;
+    const int mn_tiles = p.m_tiles * p.n_tiles;
+    const int total = mn_tiles * p.k_splits;   // work units: (k split, m tile, n tile), n fastest
     const int key_tiles = p.d_h / BN;
 
     if (threadIdx.x == 0) {
@@ -119,12 +123,14 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         if (lane == 0) {
             int it = 0, issued = 0;
             for (int t = blockIdx.x; t < total && !s_abort; t += gridDim.x) {
-                const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
+                const int ks = t / mn_tiles, tmn = t - ks * mn_tiles;
+                const int mt = tmn / p.n_tiles, nt = tmn - mt * p.n_tiles;
                 const bool is_key = nt < key_tiles;
                 const CUtensorMap *map_w = is_key ? &map_wk : &map_wv;
                 const int c0 = (is_key ? nt : nt - key_tiles) * BN;
                 const int m0 = mt * kBM;
-                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                const int kb0 = ks * p.kb_per_split, kb1 = min(p.k_blocks, kb0 + p.kb_per_split);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1;
                     if (!mbar_wait(&empty_bar[s], ph ^ 1, &s_abort)) break;
@@ -151,8 +157,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 if (!mbar_wait(&tempty_bar[acc], (use & 1) ^ 1, &s_abort)) break;
                 tc_fence_after();
                 const uint32_t dst = tmem_base + acc * BN;
+                const int ks = t / mn_tiles;
+                const int kb0 = ks * p.kb_per_split, kb1 = min(p.k_blocks, kb0 + p.kb_per_split);
                 bool ok = true;
-                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1;
                     if (!mbar_wait(&full_bar[s], ph, &s_abort)) { ok = false; break; }
@@ -162,7 +170,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 #pragma unroll
                     for (int k = 0; k < kBK / kUmmaK; ++k) {
                         const uint64_t koff = static_cast<uint64_t>((k * kUmmaK * 2) >> 4);
-                        umma_bf16_ss(dst, adesc + koff, bdesc + koff, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                        umma_bf16_ss(dst, adesc + koff, bdesc + koff, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
                     }
                     umma_commit(&empty_bar[s]);   // frees the stage once these MMAs have read it
                 }
@@ -183,7 +191,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             const uint32_t use = li / NACC;
             if (!mbar_wait(&tfull_bar[acc], use & 1, &s_abort) || s_abort) break;
             tc_fence_after();
-            const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
+            const int ks = t / mn_tiles, tmn = t - ks * mn_tiles;
+            const int mt = tmn / p.n_tiles, nt = tmn - mt * p.n_tiles;
             const bool is_key = nt < key_tiles;
             const int c0 = (is_key ? nt : nt - key_tiles) * BN;
             const int64_t n = static_cast<int64_t>(mt) * kBM + row;
@@ -194,7 +203,14 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 float accv[32];
                 tmem_ld32(taddr + cc, accv);
                 if (!valid) continue;
-                if (is_key) {
+                if (p.k_splits > 1) {
+                    // split-K: raw partial accumulator; splitk_reduce_kernel finishes the tile
+                    float4 *ap = reinterpret_cast<float4 *>(
+                        p.acc_out + (static_cast<int64_t>(ks) * p.n_tok + n) * (2 * p.d_h) + nt * BN + cc);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        ap[q] = make_float4(accv[4 * q], accv[4 * q + 1], accv[4 * q + 2], accv[4 * q + 3]);
+                } else if (is_key) {
                     const uint4 *hp = reinterpret_cast<const uint4 *>(p.h + n * p.d_h + c0 + cc);
                     const uint4 *gq = reinterpret_cast<const uint4 *>(p.gamma_q + c0 + cc);
                     const uint4 *gk = reinterpret_cast<const uint4 *>(p.gamma_k + c0 + cc);
@@ -236,7 +252,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty_bar[acc]);
-            if (valid) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
+            if (valid && p.k_splits == 1) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
         }
     }
     tc_fence_before();
@@ -244,6 +260,66 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    }
+}
+
+// Finishes a split-K projection: sums the k_splits partial accumulators of one token and one
+// BN-wide tile, then produces exactly what the unsplit epilogue produces for that tile --
+// (S0, S1, S2) for a key tile, v and S3 for a value tile.  Grid: (n_tiles, n_tok); block:
+// kReduceThreads threads x 2 channels; fixed-order sums (deterministic).
+constexpr int kReduceThreads = 128;
+
+__global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const __grid_constant__ ProjParams p, int BN) {
+    __shared__ float s_red[3][kReduceThreads / 32];
+    const int nt = blockIdx.x;
+    const int64_t n = blockIdx.y;
+    const int key_tiles = p.d_h / BN;
+    const bool is_key = nt < key_tiles;
+    const int c0 = (is_key ? nt : nt - key_tiles) * BN;
+    const int64_t stride_split = p.n_tok * (2 * p.d_h);
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+    for (int j = threadIdx.x * 2; j < BN; j += kReduceThreads * 2) {
+        const float *src = p.acc_out + n * (2 * p.d_h) + nt * BN + j;
+        float x0 = 0.f, x1 = 0.f;
+        for (int ks = 0; ks < p.k_splits; ++ks) {
+            const float2 q = __ldg(reinterpret_cast<const float2 *>(src + ks * stride_split));
+            x0 += q.x;
+            x1 += q.y;
+        }
+        if (is_key) {
+            const uint32_t hw = __ldg(reinterpret_cast<const uint32_t *>(p.h + n * p.d_h + c0 + j));
+            const uint32_t qw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_q + c0 + j));
+            const uint32_t kw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_k + c0 + j));
+            const float h0 = bf16_lo(hw), h1 = bf16_hi(hw);
+            a0 = fmaf(h0, h0, fmaf(h1, h1, a0));
+            a1 = fmaf(h0 * bf16_lo(qw) * bf16_lo(kw), x0, fmaf(h1 * bf16_hi(qw) * bf16_hi(kw), x1, a1));
+            a2 = fmaf(x0, x0, fmaf(x1, x1, a2));
+        } else {
+            *reinterpret_cast<float2 *>(p.v + n * p.d_h + c0 + j) = make_float2(x0, x1);
+            a0 = fmaf(x0, x0, fmaf(x1, x1, a0));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+        a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+        a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+    }
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (lane == 0) {
+        s_red[0][warp] = a0;
+        s_red[1][warp] = a1;
+        s_red[2][warp] = a2;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b0 = 0.f, b1 = 0.f, b2 = 0.f;
+        for (int w = 0; w < kReduceThreads / 32; ++w) {
+            b0 += s_red[0][w];
+            b1 += s_red[1][w];
+            b2 += s_red[2][w];
+        }
+        p.part[n * p.n_tiles + nt] = make_float4(b0, b1, b2, 0.f);
     }
 }
 
@@ -409,7 +485,8 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
     }
 }
 
-// Prefill fast path for the pages' conv shape (kernel 4, dilation 3, no carried state).
+// Fast path for the pages' conv shape (kernel 4, dilation 3): prefill, and decode with a
+// carried conv state when one chunk covers the whole call (T <= 3*CH).
 // Same arithmetic as gate_conv_kernel, organised for memory-level parallelism: a CTA covers
 // 3*CH tokens of one sequence and 2*kGateFastThreads channels; each thread owns 2 channels
 // and, for each residue r of the tokens mod 3, first issues every load of its chain -- CH + 3
@@ -491,8 +568,16 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
 #pragma unroll
         for (int j = 0; j < CH + KS - 1; ++j) {
             const int t = lo + r + DIL * j;
-            vv[j] = (t >= 0 && t < t1) ? __ldg(reinterpret_cast<const float2 *>(p.v + (row0 + t) * p.d_h + c))
-                                       : make_float2(0.f, 0.f);
+            if (t >= 0 && t < t1) {
+                vv[j] = __ldg(reinterpret_cast<const float2 *>(p.v + (row0 + t) * p.d_h + c));
+            } else if (t < 0 && p.conv_state != nullptr) {
+                // conv input carried from the previous call (already u, stored bf16)
+                const uint32_t sw = *reinterpret_cast<const uint32_t *>(
+                    p.conv_state + (static_cast<int64_t>(b) * HALO + HALO + t) * p.d_h + c);
+                vv[j] = make_float2(bf16_lo(sw), bf16_hi(sw));
+            } else {
+                vv[j] = make_float2(0.f, 0.f);
+            }
         }
 #pragma unroll
         for (int j = 0; j < CH; ++j) {
@@ -512,8 +597,13 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
                 u[i][0] = u[i - 1][0];
                 u[i][1] = u[i - 1][1];
             }
-            u[0][0] = beta * vj[0] * gc[0];
-            u[0][1] = beta * vj[1] * gc[1];
+            if (lo + si >= 0) {
+                u[0][0] = beta * vj[0] * gc[0];
+                u[0][1] = beta * vj[1] * gc[1];
+            } else {
+                u[0][0] = vj[0];
+                u[0][1] = vj[1];
+            }
             if (j < KS - 1) continue;
             const int t = lo + si;
             if (t >= t1) continue;
@@ -536,6 +626,105 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
                 *reinterpret_cast<float2 *>(p.delta + n * p.d_h + c) = make_float2(dl[0], dl[1]);
         }
     }
+    if (p.conv_state != nullptr) {
+        // new state slot s <- conv input at position T - HALO + s; this CTA covers the whole
+        // call (T <= TC), and each thread rewrites only its own channels, after reading them.
+#pragma unroll 1
+        for (int sl = 0; sl < HALO; ++sl) {
+            const int t = p.T - HALO + sl;
+            uint32_t o;
+            if (t >= 0) {
+                const float2 vt = __ldg(reinterpret_cast<const float2 *>(p.v + (row0 + t) * p.d_h + c));
+                const float beta = s_beta[t - lo];
+                o = static_cast<uint32_t>(f32_to_bf16_bits(beta * vt.x * gc[0])) |
+                    (static_cast<uint32_t>(f32_to_bf16_bits(beta * vt.y * gc[1])) << 16);
+            } else {
+                o = *reinterpret_cast<const uint32_t *>(
+                    p.conv_state + (static_cast<int64_t>(b) * HALO + HALO + t) * p.d_h + c);
+            }
+            *reinterpret_cast<uint32_t *>(p.conv_state + (static_cast<int64_t>(b) * HALO + sl) * p.d_h + c) = o;
+        }
+    }
+}
+
+// Decode step (T = 1) with a carried conv state, kernel 4 / dilation 3: the conv taps of the
+// new token read state slots 6, 3 and 0 (positions t-3, t-6, t-9); the new state is slots
+// 1..8 followed by u_t.  One CTA per (sequence, 512-channel slice); each thread loads all of
+// its 2 channels' data (9 state slots, v, h) in one round trip, then computes and writes.
+constexpr int kDecodeThreads = 256;
+
+__global__ void __launch_bounds__(kDecodeThreads) gate_conv_decode_kernel(const __grid_constant__ GateParams p) {
+    constexpr int S = 9;
+    __shared__ float s_gb[2];
+    const int b = blockIdx.y;
+    const float inv_d = 1.f / static_cast<float>(p.d_h);
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const float4 *pp = p.part + static_cast<int64_t>(b) * p.n_tiles;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+        for (int j = lane; j < p.n_tiles; j += 32) {
+            const float4 q = __ldg(pp + j);
+            if (j < p.n_key_tiles) {
+                s0 += q.x;
+                s1 += q.y;
+                s2 += q.z;
+            } else {
+                s3 += q.x;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+            s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+            s3 += __shfl_xor_sync(0xffffffffu, s3, o);
+        }
+        if (lane == 0) {
+            const float rms_h = sqrtf(s0 * inv_d + p.eps);
+            const float rms_k = sqrtf(s2 * inv_d + p.eps);
+            const float g = fast_sigmoid(s1 / (rms_h * rms_k) * p.inv_sqrt_d);
+            s_gb[0] = g;
+            s_gb[1] = g / sqrtf(g * g * s3 * inv_d + p.eps);
+        }
+    }
+    // issue this thread's loads while warp 0 reduces the scalars
+    const int q = blockIdx.x * blockDim.x + threadIdx.x;
+    const bool active = q < p.d_h / 2;
+    const int c = q * 2;
+    uint32_t st[S];
+    float2 v = make_float2(0.f, 0.f);
+    uint32_t hw = 0, gw = 0;
+    uint2 w0 = make_uint2(0, 0), w1 = make_uint2(0, 0);
+    uint16_t *state = p.conv_state + static_cast<int64_t>(b) * S * p.d_h + c;
+    if (active) {
+#pragma unroll
+        for (int k = 0; k < S; ++k) st[k] = *reinterpret_cast<const uint32_t *>(state + k * p.d_h);
+        v = __ldg(reinterpret_cast<const float2 *>(p.v + static_cast<int64_t>(b) * p.d_h + c));
+        hw = __ldg(reinterpret_cast<const uint32_t *>(p.h + static_cast<int64_t>(b) * p.d_h + c));
+        gw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_c + c));
+        w0 = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + c * 4));
+        w1 = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + (c + 1) * 4));
+    }
+    __syncthreads();
+    if (!active) return;
+    const float g = s_gb[0], beta = s_gb[1];
+    const float u0 = beta * v.x * bf16_lo(gw), u1 = beta * v.y * bf16_hi(gw);
+    // taps: i = 0 current, 1 -> slot 6 (t-3), 2 -> slot 3 (t-6), 3 -> slot 0 (t-9)
+    const float c0 = fmaf(bf16_lo(w0.x), u0, fmaf(bf16_hi(w0.x), bf16_lo(st[6]),
+                     fmaf(bf16_lo(w0.y), bf16_lo(st[3]), bf16_hi(w0.y) * bf16_lo(st[0]))));
+    const float c1 = fmaf(bf16_lo(w1.x), u1, fmaf(bf16_hi(w1.x), bf16_hi(st[6]),
+                     fmaf(bf16_lo(w1.y), bf16_hi(st[3]), bf16_hi(w1.y) * bf16_hi(st[0]))));
+    const float d0 = fmaf(g, v.x, c0 * fast_sigmoid(c0));
+    const float d1 = fmaf(g, v.y, c1 * fast_sigmoid(c1));
+    const uint32_t o = static_cast<uint32_t>(f32_to_bf16_bits(bf16_lo(hw) + d0)) |
+                       (static_cast<uint32_t>(f32_to_bf16_bits(bf16_hi(hw) + d1)) << 16);
+    *reinterpret_cast<uint32_t *>(p.out + static_cast<int64_t>(b) * p.d_h + c) = o;
+    if (p.delta != nullptr)
+        *reinterpret_cast<float2 *>(p.delta + static_cast<int64_t>(b) * p.d_h + c) = make_float2(d0, d1);
+#pragma unroll
+    for (int k = 0; k < S - 1; ++k) *reinterpret_cast<uint32_t *>(state + k * p.d_h) = st[k + 1];
+    *reinterpret_cast<uint32_t *>(state + (S - 1) * p.d_h) =
+        static_cast<uint32_t>(f32_to_bf16_bits(u0)) | (static_cast<uint32_t>(f32_to_bf16_bits(u1)) << 16);
 }
 
 }  // namespace engram

@@ -147,6 +147,9 @@ PARITY_CASES = {
     "bn128": small_workload("bn128", B=2, T=4777, K=2, d_e=24, d_h=384),               # 9554 tok
     "bn256": small_workload("bn256", B=5, T=1901, K=2, d_e=24, d_h=512),               # 9505 tok
     "seq_shorter_than_halo": small_workload("short", B=40, T=7, K=2, d_e=16, d_h=128),
+    # decode-sized batches: the projection splits K across CTAs (partial accumulators + reduce)
+    "splitk_64tok": small_workload("splitk64", B=64, T=1, K=1, d_e=512, d_h=512),          # 4 splits
+    "splitk_ragged_k": small_workload("splitk200", B=100, T=2, K=1, d_e=360, d_h=512),     # d_m=720, 3 splits
 }
 
 
@@ -173,8 +176,12 @@ def test_gate_conv_entry_matches_forward():
     assert torch.equal(out_fwd.view(torch.int16), out2.view(torch.int16))
 
 
-def test_decode_steps_match_oracle_and_update_state():
-    wl = small_workload("dec", B=6, T=1, K=2, d_e=32, d_h=256, decode=True)
+@pytest.mark.parametrize("geom", ["small", "splitk"])
+def test_decode_steps_match_oracle_and_update_state(geom):
+    if geom == "small":
+        wl = small_workload("dec", B=6, T=1, K=2, d_e=32, d_h=256, decode=True)
+    else:
+        wl = small_workload("dec_split", B=32, T=1, K=1, d_e=512, d_h=512, decode=True)
     di = DeviceInputs(wl)
     w = di.host_weights()
     tables = [synth.fill_bf16(wl.table_spec(h), (wl.primes[h], wl.d_e)) for h in range(wl.H)]

@@ -102,6 +102,7 @@ int check_plan(const engram_plan *plan) {
 }
 
 // ---------------------------------------------------------------- workspace layout
+constexpr int64_t kFusedLookupMaxRows = 16384;   // (token, table) rows handled by lookup_kernel
 struct Workspace {
     size_t xr, idx, m, v, part, acc;
     size_t staged_idx, unique, n_unique, staging;  // host-resident tables only
@@ -153,9 +154,16 @@ ProjShape proj_shape(const engram_plan *plan, int64_t n_tok, bool allow_split) {
         }
     }
     const int64_t mn = m_tiles * (2 * d_h / wide);
+    // ENGRAM_PROJ_SPLITS (>= 1) forces the split count of decode-sized batches (tuning);
+    // read once per process.
+    static const int forced_splits = [] {
+        const char *e = std::getenv("ENGRAM_PROJ_SPLITS");
+        const int v = e ? std::atoi(e) : 0;
+        return v > 0 ? v : 0;
+    }();
     int splits = 1;
     if (allow_split && mn > 0 && mn < sms) {
-        splits = static_cast<int>(sms / mn);
+        splits = forced_splits ? forced_splits : static_cast<int>(sms / mn);
         if (splits > ps.k_blocks / 4) splits = ps.k_blocks / 4;
         if (splits < 1) splits = 1;
     }
@@ -254,7 +262,8 @@ int set_proj_smem_attr() {
 template <int BN>
 int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                 int64_t n_tok, float *v, float4 *part, cudaStream_t stream, float *acc = nullptr,
-                int k_splits = 1, int kb_per_split = 0) {
+                int k_splits = 1, int kb_per_split = 0, bool run_reduce = true,
+                engram::ProjParams *params_out = nullptr) {
     const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim;
     CUtensorMap map_m, map_wk, map_wv;
     int rc;
@@ -284,7 +293,8 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     engram::proj_kernel<BN><<<grid, engram::kProjThreads, engram::ProjCfg<BN>::kSmemBytes, stream>>>(
         map_m, map_wk, map_wv, p);
     ENGRAM_CUDA_TRY(cudaGetLastError(), "proj_kernel launch");
-    if (p.k_splits > 1) {
+    if (params_out) *params_out = p;
+    if (p.k_splits > 1 && run_reduce) {
         engram::splitk_reduce_kernel<<<dim3(p.n_tiles, static_cast<unsigned>(n_tok)), engram::kReduceThreads, 0,
                                        stream>>>(p, BN);
         ENGRAM_CUDA_TRY(cudaGetLastError(), "splitk_reduce_kernel launch");
@@ -303,6 +313,44 @@ int validate_weights(const engram_plan *plan, const engram_weights *w) {
             return fail(ENGRAM_ERR_INVALID_ARG, "weights.%s is not 8-byte aligned", names[i]);
     }
     (void)plan;
+    return ENGRAM_OK;
+}
+
+engram::HashParams make_hash_params(const engram_plan *plan, int32_t B, int32_t T) {
+    engram::HashParams p{};
+    const engram_config &c = plan->cfg;
+    const int K = c.heads_per_order;
+    for (int oi = 0; oi < c.num_orders; ++oi)
+        for (int j = 0; j < K; ++j) {
+            const int h = oi * K + j;
+            p.order[h] = c.orders[oi];
+            p.prime[h] = static_cast<uint64_t>(c.table_rows[h]);
+            for (int i = 0; i < ENGRAM_MAX_ORDERS; ++i) p.mult[h][i] = plan->mult[h][i];
+        }
+    p.H = plan->num_tables;
+    p.max_order = c.orders[c.num_orders - 1];
+    p.hist_len = plan->hist_len;
+    p.pad_id = c.pad_id;
+    p.vocab_in = c.vocab_in;
+    p.B = B;
+    p.T = T;
+    return p;
+}
+
+// Fused remap + hash + gather, one warp per (token, table) row.
+int launch_lookup(const engram_plan *plan, const int32_t *ids, const int32_t *remap, const int32_t *history,
+                  int32_t B, int32_t T, const uint16_t *const *tables, int32_t *xr_out, uint16_t *m,
+                  cudaStream_t stream) {
+    engram::LookupParams p{};
+    p.hash = make_hash_params(plan, B, T);
+    for (int h = 0; h < plan->num_tables; ++h) p.table[h] = tables[h];
+    p.chunks_per_row = plan->cfg.row_dim / 8;
+    const int64_t warps = static_cast<int64_t>(B) * T * plan->num_tables;
+    const int threads = 256;
+    const int64_t blocks = (warps * 32 + threads - 1) / threads;
+    engram::lookup_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(ids, remap, history, xr_out,
+                                                                                reinterpret_cast<uint4 *>(m), p);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "lookup_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -358,6 +406,33 @@ int launch_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *
         idx, reinterpret_cast<uint4 *>(m), p);
     ENGRAM_CUDA_TRY(cudaGetLastError(), "gather_kernel launch");
     return ENGRAM_OK;
+}
+
+engram::GateParams make_gate_params(const engram_plan *plan, const engram_weights *w, const uint16_t *h,
+                                    const float *v, const float4 *part, int n_tiles, int32_t B, int32_t T,
+                                    uint16_t *conv_state, uint16_t *out, float *delta) {
+    engram::GateParams p{};
+    const int d_h = plan->cfg.hidden_dim;
+    p.h = h;
+    p.v = v;
+    p.part = part;
+    p.gamma_c = w->gamma_c;
+    p.conv_w = w->conv_w;
+    p.conv_state = conv_state;
+    p.out = out;
+    p.delta = delta;
+    p.B = B;
+    p.T = T;
+    p.d_h = d_h;
+    p.n_tiles = n_tiles;
+    p.n_key_tiles = n_tiles / 2;
+    p.ksize = plan->cfg.conv_kernel;
+    p.dil = plan->cfg.conv_dilation;
+    p.state_len = plan->state_len;
+    p.tok_chunk = 1;
+    p.eps = plan->cfg.eps;
+    p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(d_h));
+    return p;
 }
 
 int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const float *v,
@@ -464,13 +539,27 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
     float *v = reinterpret_cast<float *>(ws + L.v);
     float4 *part = reinterpret_cast<float4 *>(ws + L.part);
     float *acc = ps.k_splits > 1 ? reinterpret_cast<float *>(ws + L.acc) : nullptr;
+    const int d_h = plan->cfg.hidden_dim;
+    // one-token decode steps after a split-K projection: reduce + gate + conv in one kernel
+    const bool fused_decode = ps.k_splits > 1 && T == 1 && plan->cfg.conv_kernel == 4 &&
+                              plan->cfg.conv_dilation == 3 && d_h <= 2 * engram::kFusedDecodeThreads * engram::kFusedDecodeMaxPairs;
+    engram::ProjParams pp{};
     int rc;
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[0], stream), "cudaEventRecord");
-    if (ps.bn == 256) rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split);
-    else if (ps.bn == 128) rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split);
-    else rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split);
+    if (ps.bn == 256)
+        rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
+    else if (ps.bn == 128)
+        rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
+    else
+        rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
     if (rc != ENGRAM_OK) return rc;
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[1], stream), "cudaEventRecord");
+    if (fused_decode) {
+        const engram::GateParams gp = make_gate_params(plan, w, h, v, part, ps.n_tiles, B, T, conv_state, out, delta);
+        engram::decode_fused_kernel<<<static_cast<unsigned>(B), engram::kFusedDecodeThreads, 0, stream>>>(pp, gp);
+        ENGRAM_CUDA_TRY(cudaGetLastError(), "decode_fused_kernel launch");
+        return ENGRAM_OK;
+    }
     return launch_gate_conv(plan, w, h, v, part, ps.n_tiles, B, T, conv_state, out, delta, stream);
 }
 
@@ -726,10 +815,21 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const uint1
         if (stage_events) ENGRAM_CUDA_TRY(record_stage_event(stage_events[i], stream), "cudaEventRecord");
         return ENGRAM_OK;
     };
+    // Decode-sized batches on HBM-resident tables: remap + hash + gather in one kernel (the
+    // row ids stay in registers).  Larger batches: the hash kernel, then the wide gather.
+    const bool fused_lookup = !L.staged && plan->cfg.table_location == ENGRAM_TABLES_DEVICE &&
+                              n_tok * plan->num_tables <= kFusedLookupMaxRows;
     if ((rc = rec(0)) != ENGRAM_OK) return rc;
-    if ((rc = launch_hash(plan, ids, remap, history, B, T, idx, xr, stream)) != ENGRAM_OK) return rc;
-    if ((rc = rec(1)) != ENGRAM_OK) return rc;
-    if (L.staged) {
+    if (fused_lookup) {
+        if ((rc = rec(1)) != ENGRAM_OK) return rc;
+        if ((rc = launch_lookup(plan, ids, remap, history, B, T, tables, xr, m, stream)) != ENGRAM_OK) return rc;
+    } else {
+        if ((rc = launch_hash(plan, ids, remap, history, B, T, idx, xr, stream)) != ENGRAM_OK) return rc;
+        if ((rc = rec(1)) != ENGRAM_OK) return rc;
+    }
+    if (fused_lookup) {
+        // rows already in m
+    } else if (L.staged) {
         // host-resident tables: fetch each distinct row of the batch once into HBM staging,
         // then gather from there (results are bit-identical to the HBM-resident path)
         const int H = plan->num_tables;

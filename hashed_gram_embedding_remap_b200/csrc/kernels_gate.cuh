@@ -727,4 +727,122 @@ __global__ void __launch_bounds__(kDecodeThreads) gate_conv_decode_kernel(const 
         static_cast<uint32_t>(f32_to_bf16_bits(u0)) | (static_cast<uint32_t>(f32_to_bf16_bits(u1)) << 16);
 }
 
+// Decode step (T = 1) after a split-K projection, fully fused: one CTA per token sums the
+// k_splits partial accumulators of its [k~ | v] row, reduces S0..S3 across the block, then
+// applies gate, conv (kernel 4, dilation 3, taps from the carried state or zeros), SiLU,
+// residual and the state shift.  Replaces splitk_reduce_kernel + the gate kernel for decode.
+constexpr int kFusedDecodeThreads = 512;
+constexpr int kFusedDecodeMaxPairs = 4;   // d_h <= 2 * 512 * 4 = 4096
+
+__global__ void __launch_bounds__(kFusedDecodeThreads) decode_fused_kernel(const __grid_constant__ ProjParams pp,
+                                                                           const __grid_constant__ GateParams p) {
+    constexpr int S = 9;
+    __shared__ float s_red[4][kFusedDecodeThreads / 32];
+    __shared__ float s_gb[2];
+    const int b = blockIdx.x;
+    const int d_h = p.d_h;
+    const int64_t split_stride = pp.n_tok * (2 * d_h);
+    const float *acc = pp.acc_out + static_cast<int64_t>(b) * (2 * d_h);
+    float2 v[kFusedDecodeMaxPairs];
+    uint32_t hv[kFusedDecodeMaxPairs], gw[kFusedDecodeMaxPairs], st[kFusedDecodeMaxPairs][S];
+    uint2 w0[kFusedDecodeMaxPairs], w1[kFusedDecodeMaxPairs];
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    // one round trip: split accumulators, h, gains, conv weights and the carried state
+#pragma unroll
+    for (int k = 0; k < kFusedDecodeMaxPairs; ++k) {
+        const int c = 2 * (threadIdx.x + k * kFusedDecodeThreads);
+        v[k] = make_float2(0.f, 0.f);
+        hv[k] = gw[k] = 0;
+        w0[k] = w1[k] = make_uint2(0, 0);
+#pragma unroll
+        for (int j = 0; j < S; ++j) st[k][j] = 0;
+        if (c < d_h) {
+            if (p.conv_state != nullptr) {
+                const uint16_t *state = p.conv_state + static_cast<int64_t>(b) * S * d_h + c;
+#pragma unroll
+                for (int j = 0; j < S; ++j) st[k][j] = *reinterpret_cast<const uint32_t *>(state + j * d_h);
+            }
+            gw[k] = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_c + c));
+            w0[k] = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + c * 4));
+            w1[k] = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + (c + 1) * 4));
+            float2 kt = make_float2(0.f, 0.f), vt = make_float2(0.f, 0.f);
+            for (int ks = 0; ks < pp.k_splits; ++ks) {
+                const float2 x = __ldg(reinterpret_cast<const float2 *>(acc + ks * split_stride + c));
+                const float2 y = __ldg(reinterpret_cast<const float2 *>(acc + ks * split_stride + d_h + c));
+                kt.x += x.x;
+                kt.y += x.y;
+                vt.x += y.x;
+                vt.y += y.y;
+            }
+            const uint32_t hw = __ldg(reinterpret_cast<const uint32_t *>(pp.h + static_cast<int64_t>(b) * d_h + c));
+            const uint32_t qw = __ldg(reinterpret_cast<const uint32_t *>(pp.gamma_q + c));
+            const uint32_t kw = __ldg(reinterpret_cast<const uint32_t *>(pp.gamma_k + c));
+            const float h0 = bf16_lo(hw), h1 = bf16_hi(hw);
+            a0 = fmaf(h0, h0, fmaf(h1, h1, a0));
+            a1 = fmaf(h0 * bf16_lo(qw) * bf16_lo(kw), kt.x, fmaf(h1 * bf16_hi(qw) * bf16_hi(kw), kt.y, a1));
+            a2 = fmaf(kt.x, kt.x, fmaf(kt.y, kt.y, a2));
+            a3 = fmaf(vt.x, vt.x, fmaf(vt.y, vt.y, a3));
+            v[k] = vt;
+            hv[k] = hw;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+        a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+        a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+        a3 += __shfl_xor_sync(0xffffffffu, a3, o);
+    }
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (lane == 0) {
+        s_red[0][warp] = a0;
+        s_red[1][warp] = a1;
+        s_red[2][warp] = a2;
+        s_red[3][warp] = a3;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+        for (int w = 0; w < kFusedDecodeThreads / 32; ++w) {
+            s0 += s_red[0][w];
+            s1 += s_red[1][w];
+            s2 += s_red[2][w];
+            s3 += s_red[3][w];
+        }
+        const float inv_d = 1.f / static_cast<float>(d_h);
+        const float rms_h = sqrtf(s0 * inv_d + p.eps);
+        const float rms_k = sqrtf(s2 * inv_d + p.eps);
+        const float g = fast_sigmoid(s1 / (rms_h * rms_k) * p.inv_sqrt_d);
+        s_gb[0] = g;
+        s_gb[1] = g / sqrtf(g * g * s3 * inv_d + p.eps);
+    }
+    __syncthreads();
+    const float g = s_gb[0], beta = s_gb[1];
+#pragma unroll
+    for (int k = 0; k < kFusedDecodeMaxPairs; ++k) {
+        const int c = 2 * (threadIdx.x + k * kFusedDecodeThreads);
+        if (c >= d_h) continue;
+        const float u0 = beta * v[k].x * bf16_lo(gw[k]), u1 = beta * v[k].y * bf16_hi(gw[k]);
+        // taps: i = 0 current, 1 -> slot 6 (t-3), 2 -> slot 3 (t-6), 3 -> slot 0 (t-9)
+        const float c0 = fmaf(bf16_lo(w0[k].x), u0, fmaf(bf16_hi(w0[k].x), bf16_lo(st[k][6]),
+                         fmaf(bf16_lo(w0[k].y), bf16_lo(st[k][3]), bf16_hi(w0[k].y) * bf16_lo(st[k][0]))));
+        const float c1 = fmaf(bf16_lo(w1[k].x), u1, fmaf(bf16_hi(w1[k].x), bf16_hi(st[k][6]),
+                         fmaf(bf16_lo(w1[k].y), bf16_hi(st[k][3]), bf16_hi(w1[k].y) * bf16_hi(st[k][0]))));
+        const float d0 = fmaf(g, v[k].x, c0 * fast_sigmoid(c0));
+        const float d1 = fmaf(g, v[k].y, c1 * fast_sigmoid(c1));
+        const uint32_t o = static_cast<uint32_t>(f32_to_bf16_bits(bf16_lo(hv[k]) + d0)) |
+                           (static_cast<uint32_t>(f32_to_bf16_bits(bf16_hi(hv[k]) + d1)) << 16);
+        *reinterpret_cast<uint32_t *>(p.out + static_cast<int64_t>(b) * d_h + c) = o;
+        if (p.delta != nullptr)
+            *reinterpret_cast<float2 *>(p.delta + static_cast<int64_t>(b) * d_h + c) = make_float2(d0, d1);
+        if (p.conv_state != nullptr) {
+            uint16_t *state = p.conv_state + static_cast<int64_t>(b) * S * d_h + c;
+#pragma unroll
+            for (int j = 0; j < S - 1; ++j) *reinterpret_cast<uint32_t *>(state + j * d_h) = st[k][j + 1];
+            *reinterpret_cast<uint32_t *>(state + (S - 1) * d_h) =
+                static_cast<uint32_t>(f32_to_bf16_bits(u0)) | (static_cast<uint32_t>(f32_to_bf16_bits(u1)) << 16);
+        }
+    }
+}
+
 }  // namespace engram

@@ -174,6 +174,67 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint32_t *__restrict_
     }
 }
 
+// Steps 1-3 fused for device-resident tables: one warp per (token, table) row.  Lane 0
+// remaps the gram's ids and hashes them (same arithmetic as hash_kernel), the row id is
+// broadcast to the warp, and the 32 lanes copy the row into m as 16-byte chunks.  Used by
+// engram_forward: the row ids never round-trip through memory (the remapped current id is
+// still written for the decode-history update).
+struct LookupParams {
+    HashParams hash;
+    const uint16_t *table[ENGRAM_MAX_TABLES];
+    int32_t chunks_per_row;  // d_e / 8
+};
+
+__global__ void __launch_bounds__(256) lookup_kernel(const int32_t *__restrict__ ids,
+                                                     const int32_t *__restrict__ remap,
+                                                     const int32_t *__restrict__ history,
+                                                     int32_t *__restrict__ xr_out, uint4 *__restrict__ m,
+                                                     const __grid_constant__ LookupParams p) {
+    const HashParams &hp = p.hash;
+    const int64_t n_tok = static_cast<int64_t>(hp.B) * hp.T;
+    const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+    const int lane = threadIdx.x % 32;
+    const int64_t n = warp_id / hp.H;
+    if (n >= n_tok) return;
+    const int h = static_cast<int>(warp_id - n * hp.H);
+    uint32_t row = 0;
+    if (lane == 0) {
+        const int32_t b = static_cast<int32_t>(n / hp.T);
+        const int32_t t = static_cast<int32_t>(n - static_cast<int64_t>(b) * hp.T);
+        const int o = hp.order[h];
+        uint64_t s = 0;
+        for (int i = 0; i < o; ++i) {
+            const int32_t pos = t - i;
+            int32_t x;
+            if (pos >= 0) {
+                const int32_t raw = __ldg(ids + (n - i));
+                if (remap != nullptr) {
+                    if (raw >= 0 && raw < hp.vocab_in) {
+                        x = __ldg(remap + raw);
+                    } else {
+                        x = hp.pad_id;
+                        if (i == 0) atomicOr(&g_engram_status, ENGRAM_STATUS_BAD_TOKEN);
+                    }
+                } else {
+                    x = raw;
+                }
+            } else if (history != nullptr && -pos <= hp.hist_len) {
+                x = __ldg(history + static_cast<int64_t>(b) * hp.hist_len + hp.hist_len + pos);
+            } else {
+                x = hp.pad_id;
+            }
+            if (i == 0 && h == 0 && xr_out != nullptr) xr_out[n] = x;
+            s ^= (static_cast<uint64_t>(static_cast<int64_t>(x)) + 1ull) * hp.mult[h][i];
+        }
+        row = static_cast<uint32_t>(fmix64(s) % hp.prime[h]);
+    }
+    row = __shfl_sync(0xffffffffu, row, 0);
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.table[h]) + static_cast<int64_t>(row) * p.chunks_per_row;
+    uint4 *dst = m + (n * hp.H + h) * p.chunks_per_row;
+#pragma unroll 4
+    for (int c = lane; c < p.chunks_per_row; c += 32) dst[c] = __ldg(src + c);
+}
+
 // ---------------------------------------------------------------- host-resident tables
 // A step's row ids are known before its compute starts, so the rows a batch needs can be
 // fetched from host memory ahead of use.  stage_dedup_kernel (one CTA per table) sorts the

@@ -35,6 +35,23 @@ import synth  # noqa: E402
 L2_BYTES = 126 * 2 ** 20
 
 
+def kernel_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu summary
+    (profiles/traffic.json), or None when that summary was taken on a different version of
+    the kernel's source file than the one built here."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    entry = json.load(open(p)).get(kernel, {}).get(workload)
+    if not entry:
+        return None
+    src = os.path.join(ROOT, entry["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != entry["source_sha256"]:
+        return None
+    return entry["dram_bytes_per_launch"]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -378,7 +395,7 @@ def run_engram(args, wl, world, rank, local):
     tflops = flops / proj_s / 1e12
     roofline = {"bound": "tensor", "kernel": "proj_kernel (tcgen05 k/v projections + gate partials)",
                 "achieved": tflops, "peak": peaks["bf16_sus"], "unit": "TFLOP/s", "frac": tflops / peaks["bf16_sus"],
-                "traffic": None, "peak_source": f"{peaks['source']} bf16 sustained",
+                "traffic": kernel_traffic("proj_kernel", wl.name), "peak_source": f"{peaks['source']} bf16 sustained",
                 "algorithmic_per_launch": flops}
     # HBM view of the memory-bound kernels (gather and gate+conv)
     row_bytes = wl.H * wl.d_e * 2

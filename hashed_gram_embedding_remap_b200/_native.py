@@ -30,6 +30,7 @@ ENGRAM_FORWARD_STAGES = 4
 ENGRAM_TABLES_DEVICE = 0
 ENGRAM_TABLES_HOST_MAPPED = 1
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
+ENGRAM_FLAG_FUSED_GATE = 0x1
 
 _ERRNAMES = {-1: "ENGRAM_ERR_INVALID_ARG", -2: "ENGRAM_ERR_UNSUPPORTED", -3: "ENGRAM_ERR_CUDA",
              -4: "ENGRAM_ERR_OOM", -5: "ENGRAM_ERR_TIMEOUT"}
@@ -57,7 +58,8 @@ class engram_config(C.Structure):
         ("table_location", C.c_int32),
         ("hash_seed", C.c_uint64),
         ("eps", C.c_float),
-        ("reserved", C.c_int32 * 7),
+        ("flags", C.c_int32),
+        ("reserved", C.c_int32 * 6),
     ]
 
 
@@ -156,7 +158,8 @@ class Plan:
 
     def __init__(self, *, orders: Sequence[int], heads_per_order: int, table_rows: Sequence[int],
                  row_dim: int, hidden_dim: int, vocab_in: int, vocab_out: int, hash_seed: int,
-                 eps: float = 1e-6, conv_kernel: int = 4, table_location: int = ENGRAM_TABLES_DEVICE):
+                 eps: float = 1e-6, conv_kernel: int = 4, table_location: int = ENGRAM_TABLES_DEVICE,
+                 flags: int = 0):
         cfg = engram_config()
         cfg.num_orders = len(orders)
         for i, o in enumerate(orders):
@@ -174,6 +177,7 @@ class Plan:
         cfg.table_location = int(table_location)
         cfg.hash_seed = int(hash_seed) & 0xFFFFFFFFFFFFFFFF
         cfg.eps = float(eps)
+        cfg.flags = int(flags)
         self.cfg = cfg
         self.plan = engram_plan()
         _check(lib.engram_init(C.byref(cfg), C.byref(self.plan)))

@@ -14,6 +14,7 @@
 
 #include "engram.h"
 #include "kernels_gate.cuh"
+#include "kernels_fused.cuh"
 #include "kernels_lookup.cuh"
 #include "ptx.cuh"
 
@@ -178,6 +179,20 @@ ProjShape proj_shape(const engram_plan *plan, int64_t n_tok, bool allow_split) {
     return ps;
 }
 
+// With ENGRAM_FLAG_FUSED_GATE, prefill with the pages' conv shape runs projections, gate
+// and conv in one kernel (fused_proj_gate_kernel).
+bool use_fused_gate(const engram_plan *plan, int64_t n_tok, bool has_state) {
+    if (!(plan->cfg.flags & ENGRAM_FLAG_FUSED_GATE) || has_state || n_tok <= 0) return false;
+    if (plan->cfg.conv_kernel != 4 || plan->cfg.conv_dilation != 3) return false;
+    return plan->cfg.hidden_dim % 256 == 0;
+}
+
+size_t fused_vbuf_bytes(const engram_plan *plan, int64_t n_tok) {
+    const int64_t units = (n_tok + engram::kFusedRows - 1) / engram::kFusedRows;
+    const int64_t ctas = units < 148 ? units : 148;
+    return sizeof(float) * static_cast<size_t>(ctas) * 2 * engram::kBM * plan->cfg.hidden_dim;
+}
+
 Workspace layout(const engram_plan *plan, int64_t n_tok) {
     Workspace w{};
     const int H = plan->num_tables;
@@ -188,7 +203,12 @@ Workspace layout(const engram_plan *plan, int64_t n_tok) {
     w.xr = off;   off = align256(off + sizeof(int32_t) * n_tok);
     w.idx = off;  off = align256(off + sizeof(uint32_t) * n_tok * H);
     w.m = off;    off = align256(off + sizeof(uint16_t) * n_tok * plan->mem_dim);
-    w.v = off;    off = align256(off + sizeof(float) * n_tok * d_h);
+    size_t v_bytes = sizeof(float) * n_tok * d_h;
+    if (use_fused_gate(plan, n_tok, false)) {
+        const size_t fb = fused_vbuf_bytes(plan, n_tok);   // the fused kernel's v scratch reuses this region
+        if (fb > v_bytes) v_bytes = fb;
+    }
+    w.v = off;    off = align256(off + v_bytes);
     w.part = off; off = align256(off + sizeof(float4) * n_tok * n_tiles);
     w.acc = off;
     if (ps.k_splits > 1) off = align256(off + sizeof(float) * ps.k_splits * n_tok * 2 * d_h);
@@ -308,9 +328,7 @@ int validate_weights(const engram_plan *plan, const engram_weights *w) {
     const char *names[6] = {"w_k", "w_v", "gamma_q", "gamma_k", "gamma_c", "conv_w"};
     for (int i = 0; i < 6; ++i) {
         if (ptrs[i] == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "weights.%s is NULL", names[i]);
-        if (i < 2 && !aligned16(ptrs[i])) return fail(ENGRAM_ERR_INVALID_ARG, "weights.%s is not 16-byte aligned", names[i]);
-        if (i >= 2 && (reinterpret_cast<uintptr_t>(ptrs[i]) & 7u))
-            return fail(ENGRAM_ERR_INVALID_ARG, "weights.%s is not 8-byte aligned", names[i]);
+        if (!aligned16(ptrs[i])) return fail(ENGRAM_ERR_INVALID_ARG, "weights.%s is not 16-byte aligned", names[i]);
     }
     (void)plan;
     return ENGRAM_OK;
@@ -519,6 +537,53 @@ int launch_stage(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, co
     return ENGRAM_OK;
 }
 
+int set_fused_smem_attr() {
+    static bool done[64] = {};
+    int dev = 0;
+    ENGRAM_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev < 64 && done[dev]) return ENGRAM_OK;
+    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::fused_proj_gate_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         engram::FusedCfg<256>::kSmemBytes),
+                    "cudaFuncSetAttribute(fused_proj_gate_kernel)");
+    if (dev < 64) done[dev] = true;
+    return ENGRAM_OK;
+}
+
+int launch_fused_gate(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
+                      int32_t B, int32_t T, uint16_t *out, float *delta, float *vbuf, cudaStream_t stream) {
+    const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim;
+    const int64_t n_tok = static_cast<int64_t>(B) * T;
+    CUtensorMap map_m, map_wk, map_wv;
+    int rc;
+    if ((rc = make_map_bf16(&map_m, m, static_cast<uint64_t>(n_tok), d_m, engram::kBM)) != ENGRAM_OK) return rc;
+    if ((rc = make_map_bf16(&map_wk, w->w_k, d_h, d_m, 256)) != ENGRAM_OK) return rc;
+    if ((rc = make_map_bf16(&map_wv, w->w_v, d_h, d_m, 256)) != ENGRAM_OK) return rc;
+    if ((rc = set_fused_smem_attr()) != ENGRAM_OK) return rc;
+    engram::FusedParams p{};
+    p.h = h;
+    p.gamma_q = w->gamma_q;
+    p.gamma_k = w->gamma_k;
+    p.gamma_c = w->gamma_c;
+    p.conv_w = w->conv_w;
+    p.out = out;
+    p.delta = delta;
+    p.vbuf = vbuf;
+    p.n_tok = n_tok;
+    p.T = T;
+    p.d_m = d_m;
+    p.d_h = d_h;
+    p.k_blocks = (d_m + engram::kBK - 1) / engram::kBK;
+    p.n_units = static_cast<int32_t>((n_tok + engram::kFusedRows - 1) / engram::kFusedRows);
+    p.eps = plan->cfg.eps;
+    p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(d_h));
+    const int sms = sm_count();
+    const unsigned grid = static_cast<unsigned>(p.n_units < sms ? p.n_units : sms);
+    engram::fused_proj_gate_kernel<256><<<grid, engram::kFusedThreads, engram::FusedCfg<256>::kSmemBytes, stream>>>(
+        map_m, map_wk, map_wv, p);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "fused_proj_gate_kernel launch");
+    return ENGRAM_OK;
+}
+
 // Stage events are profiling hooks.  Under stream capture they must become event-record
 // nodes of the graph (cudaEventRecordExternal) so that they can be timed after a replay.
 cudaError_t record_stage_event(void *ev, cudaStream_t stream) {
@@ -535,6 +600,11 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
                    cudaStream_t stream, void *const *events) {
     const int64_t n_tok = static_cast<int64_t>(B) * T;
     const Workspace L = layout(plan, n_tok);
+    if (use_fused_gate(plan, n_tok, conv_state != nullptr)) {
+        if (events) ENGRAM_CUDA_TRY(record_stage_event(events[0], stream), "cudaEventRecord");
+        if (events) ENGRAM_CUDA_TRY(record_stage_event(events[1], stream), "cudaEventRecord");
+        return launch_fused_gate(plan, w, h, m, B, T, out, delta, reinterpret_cast<float *>(ws + L.v), stream);
+    }
     const ProjShape ps = proj_shape(plan, n_tok, true);
     float *v = reinterpret_cast<float *>(ws + L.v);
     float4 *part = reinterpret_cast<float4 *>(ws + L.part);
@@ -647,8 +717,9 @@ int engram_init(const engram_config *cfg, engram_plan *plan) {
     if (!(c.eps > 0.f) || !std::isfinite(c.eps)) return fail(ENGRAM_ERR_INVALID_ARG, "eps must be a positive finite number");
     if (c.table_location != ENGRAM_TABLES_DEVICE && c.table_location != ENGRAM_TABLES_HOST_MAPPED)
         return fail(ENGRAM_ERR_INVALID_ARG, "unknown table_location");
-    for (int i = 0; i < 7; ++i)
+    for (int i = 0; i < 6; ++i)
         if (c.reserved[i] != 0) return fail(ENGRAM_ERR_INVALID_ARG, "reserved fields must be zero");
+    if (c.flags & ~ENGRAM_FLAG_FUSED_GATE) return fail(ENGRAM_ERR_INVALID_ARG, "unknown flags 0x%x", c.flags);
 
     std::memset(plan, 0, sizeof *plan);
     plan->cfg = c;

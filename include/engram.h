@@ -83,8 +83,16 @@ typedef struct engram_config {
     int32_t table_location;               /* enum engram_table_location */
     uint64_t hash_seed;                   /* seeds the per-head hash multipliers */
     float eps;                            /* RMSNorm epsilon (> 0) */
-    int32_t reserved[7];                  /* must be zero */
+    int32_t flags;                        /* ENGRAM_FLAG_* bits */
+    int32_t reserved[6];                  /* must be zero */
 } engram_config;
+
+/* engram_config.flags */
+#define ENGRAM_FLAG_FUSED_GATE 0x1 /* prefill with kernel 4 / dilation 3 and d_h % 256 == 0:
+                                      run projections, gate and conv in ONE persistent kernel
+                                      (the conv pass rides in the projection's epilogue warps).
+                                      Results match the two-kernel path within tolerance; it is
+                                      opt-in because it is currently slower on B200. */
 
 /* Validated config plus derived constants.  Caller-owned, plain data: engram_init fills
  * it, every other call reads it.  Do not modify its fields. */

@@ -33,7 +33,7 @@ def to_host_u16(t: torch.Tensor) -> np.ndarray:
 class DeviceInputs:
     """All tensors of one workload on the device; tables filled on the GPU."""
 
-    def __init__(self, wl: synth.Workload, step: int = 0, device="cuda", tables=None):
+    def __init__(self, wl: synth.Workload, step: int = 0, device="cuda", tables=None, flags: int = 0):
         fill_gpu.build()
         self.wl = wl
         self.ids_np = wl.ids(step)
@@ -52,7 +52,7 @@ class DeviceInputs:
         self.history = to_dev(wl.history(), device) if wl.decode else None
         self.conv_state = (fill_gpu.filled((wl.B, wl.state_len, wl.d_h), wl.state_spec(), device)
                            if wl.decode else None)
-        self.plan = E.Plan.from_workload(wl)
+        self.plan = E.Plan.from_workload(wl, flags=flags)
         self.weights = E.Weights(self.w_k, self.w_v, self.gamma_q, self.gamma_k, self.gamma_c, self.conv_w)
         self.out = torch.empty((wl.n_tok, wl.d_h), dtype=torch.bfloat16, device=device)
         self.delta = torch.empty((wl.n_tok, wl.d_h), dtype=torch.float32, device=device)

@@ -145,7 +145,12 @@ PARITY_CASES = {
     "tiny": synth.get_workload("tiny"),
     "ragged_k_bn64": small_workload("ragged_k", B=3, T=333, K=3, d_e=40, d_h=384),     # d_m=240
     "bn128": small_workload("bn128", B=2, T=4777, K=2, d_e=24, d_h=384),               # 9554 tok
-    "bn256": small_workload("bn256", B=5, T=1901, K=2, d_e=24, d_h=512),               # 9505 tok
+    # >= 64 units of 119 tokens with d_h % 256 == 0: projections, gate and conv in one kernel
+    "fused_bn256": small_workload("bn256", B=5, T=1901, K=2, d_e=24, d_h=512),         # 9505 tok
+    "fused_seq_edges": small_workload("fseq", B=40, T=200, K=2, d_e=16, d_h=256),      # starts inside units
+    "fused_short_seqs": small_workload("fshort", B=800, T=10, K=2, d_e=16, d_h=256),   # T < conv halo + 1
+    # fewer units: separate projection (BN = 256) and gate/conv kernels
+    "bn256_unfused": small_workload("bn256u", B=4, T=500, K=2, d_e=32, d_h=2560),      # 2000 tok
     "seq_shorter_than_halo": small_workload("short", B=40, T=7, K=2, d_e=16, d_h=128),
     # decode-sized batches: the projection splits K across CTAs (partial accumulators + reduce)
     "splitk_64tok": small_workload("splitk64", B=64, T=1, K=1, d_e=512, d_h=512),          # 4 splits
@@ -156,7 +161,8 @@ PARITY_CASES = {
 @pytest.mark.parametrize("case", list(PARITY_CASES))
 def test_forward_matches_oracle(case):
     wl = PARITY_CASES[case]
-    di = DeviceInputs(wl).forward()
+    flags = E.ENGRAM_FLAG_FUSED_GATE if case.startswith("fused") else 0
+    di = DeviceInputs(wl, flags=flags).forward()
     torch.cuda.synchronize()
     ref = _oracle_full(wl, di)
     assert_delta_close(di.delta.cpu().numpy(), ref["delta"])

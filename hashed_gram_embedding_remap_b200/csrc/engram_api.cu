@@ -105,7 +105,7 @@ int check_plan(const engram_plan *plan) {
 // ---------------------------------------------------------------- workspace layout
 constexpr int64_t kFusedLookupMaxRows = 16384;   // (token, table) rows handled by lookup_kernel
 struct Workspace {
-    size_t xr, idx, m, v, part, acc;
+    size_t xr, idx, m, v, part, acc, scal;
     size_t staged_idx, unique, n_unique, staging;  // host-resident tables only
     bool staged;                                   // rows go through device staging
     size_t total;
@@ -212,6 +212,7 @@ Workspace layout(const engram_plan *plan, int64_t n_tok) {
     w.part = off; off = align256(off + sizeof(float4) * n_tok * n_tiles);
     w.acc = off;
     if (ps.k_splits > 1) off = align256(off + sizeof(float) * ps.k_splits * n_tok * 2 * d_h);
+    w.scal = off; off = align256(off + sizeof(float2) * n_tok);
     w.staged = plan->cfg.table_location == ENGRAM_TABLES_HOST_MAPPED && n_tok <= engram::kStageMaxTok;
     if (w.staged) {
         w.staged_idx = off; off = align256(off + sizeof(uint32_t) * n_tok * H);
@@ -455,7 +456,7 @@ engram::GateParams make_gate_params(const engram_plan *plan, const engram_weight
 
 int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const float *v,
                      const float4 *part, int n_tiles, int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out,
-                     float *delta, cudaStream_t stream) {
+                     float *delta, cudaStream_t stream, float2 *scal = nullptr) {
     engram::GateParams p{};
     const int d_h = plan->cfg.hidden_dim;
     p.h = h;
@@ -495,6 +496,14 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
         return ENGRAM_OK;
     }
     dim3 grid(static_cast<unsigned>((T + p.tok_chunk - 1) / p.tok_chunk), static_cast<unsigned>(B), slices);
+    if (fast && scal != nullptr && conv_state == nullptr) {
+        // scalars once per token instead of once per (CTA, halo-extended chunk)
+        const int64_t n_tok = static_cast<int64_t>(B) * T;
+        engram::gate_scalars_kernel<<<static_cast<unsigned>((n_tok * 32 + 255) / 256), 256, 0, stream>>>(
+            part, n_tok, n_tiles, p.n_key_tiles, d_h, p.eps, p.inv_sqrt_d, scal);
+        ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_scalars_kernel launch");
+        p.scal = scal;
+    }
     if (fast) engram::gate_conv_k4d3_kernel<kChain><<<grid, threads, 0, stream>>>(p);
     else engram::gate_conv_kernel<<<grid, threads, smem, stream>>>(p);
     ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_conv_kernel launch");
@@ -630,7 +639,8 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
         ENGRAM_CUDA_TRY(cudaGetLastError(), "decode_fused_kernel launch");
         return ENGRAM_OK;
     }
-    return launch_gate_conv(plan, w, h, v, part, ps.n_tiles, B, T, conv_state, out, delta, stream);
+    return launch_gate_conv(plan, w, h, v, part, ps.n_tiles, B, T, conv_state, out, delta, stream,
+                            reinterpret_cast<float2 *>(ws + L.scal));
 }
 
 int check_bt(int32_t B, int32_t T) {

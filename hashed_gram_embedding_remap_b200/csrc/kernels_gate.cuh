@@ -1,327 +1,20 @@
-// Steps 4-6 of the lookup.
-//
-// (a) proj_kernel: the value and key projections [k~ | v] = m [W_k ; W_v]^T on the tcgen05
-//     tensor cores.  One CTA computes a 128-token x BN-channel tile: a TMA producer warp
-//     streams 128x64 tiles of m and BNx64 tiles of W (128-byte swizzle) through an S-stage
-//     shared-memory ring, one thread issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM
-//     accumulator, and four epilogue warps read the accumulator back with tcgen05.ld.  The
-//     epilogue never writes k~: for a key tile it reduces, per token, the three partial sums
-//     the gate needs over the tile's channels --
-//         S0 = sum h^2,  S1 = sum h * gamma_q * gamma_k * k~,  S2 = sum k~^2
-//     -- and for a value tile it writes v (fp32) and S3 = sum v^2.  The gate kernel combines
-//     the partials of all tiles in a fixed order (deterministic, no atomics).
-// (b) gate_conv_kernel: per token, g = sigmoid(S1 / (rms_h rms_k sqrt(d))), with
-//     rms_h = sqrt(S0/d + eps), rms_k = sqrt(S2/d + eps); U = g v; u = U / rms_U * gamma_c with
-//     rms_U = sqrt(g^2 S3 / d + eps); c_t = sum_i w_i u_{t - i*dil}; Delta = U + c sigmoid(c);
-//     out = bf16_rne(h + Delta).  Each thread owns 4 channels and walks the tokens of one
-//     residue class modulo the dilation, so the dilated conv becomes a dense 4-tap shift
-//     register in registers.
+// Steps 5-6 of the lookup (and the finishing of step 4's gate statistics): per-token gate
+// scalars g = sigmoid(S1 / (rms_h rms_k sqrt(d))) and beta = g / rms_U from the projection
+// partials; u = beta v gamma_c; c_t = sum_i w_i u_{t - i*dil}; Delta = g v + c sigmoid(c);
+// out = bf16_rne(h + Delta).  Kernels: a generic one (any conv shape, optional carried
+// state), the kernel-4 dilation-3 chain kernel for prefill and short stateful calls, the
+// one-token decode kernels (with a carried conv state), and the fused split-K reduce + decode
+// gate.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
 
 #include "engram.h"
+#include "kernels_proj.cuh"
 #include "ptx.cuh"
 
 namespace engram {
-
-constexpr int kBM = 128;          // tokens per tile (UMMA M)
-constexpr int kBK = 64;           // K elements per stage: one 128-byte swizzle row
-constexpr int kUmmaK = 16;        // K per tcgen05.mma for 16-bit inputs
-constexpr int kProjThreads = 192; // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
-
-template <int BN>
-struct ProjCfg {
-    static constexpr int kATile = kBM * kBK * 2;                 // 16 KB
-    static constexpr int kBTile = BN * kBK * 2;
-    static constexpr int kStageBytes = kATile + kBTile;
-    static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
-    static constexpr int kAccum = 2;                              // TMEM accumulators (double buffer)
-    static constexpr int kTmemCols = kAccum * BN;                 // fp32 columns, power of two
-    // dynamic smem: [align pad][stages x A][stages x B][full, empty, tmem_full, tmem_empty][tmem addr]
-    static constexpr int kBarBytes = (2 * kStages + 2 * kAccum) * 8;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 16;
-};
-
-struct ProjParams {
-    const uint16_t *h;         // [n_tok, d_h] bf16
-    const uint16_t *gamma_q;   // [d_h]
-    const uint16_t *gamma_k;   // [d_h]
-    float *v;                  // [n_tok, d_h] fp32 out
-    float4 *part;              // [n_tok, n_tiles] partial sums out
-    int64_t n_tok;
-    int32_t d_m, d_h;
-    int32_t n_tiles;           // 2 * d_h / BN: key tiles first, then value tiles
-    int32_t k_blocks;          // ceil(d_m / kBK)
-    int32_t m_tiles;           // ceil(n_tok / kBM)
-    int32_t k_splits;          // > 1: split-K, raw fp32 partial accumulators go to acc_out
-    int32_t kb_per_split;      // k-blocks per split
-    float *acc_out;            // [k_splits, n_tok, 2*d_h] when k_splits > 1
-};
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
-    return __uint_as_float(static_cast<uint32_t>(b) << 16);
-}
-
-// Persistent: grid = min(#tiles, #SMs); CTA i takes tiles i, i + grid, ...  Tile t covers
-// tokens [128*(t / n_tiles), +128) and channel slice t % n_tiles, so the CTAs running at
-// one time share a few 128-token blocks of m (re-read from L2) and stream all of W.
-// Roles: warp 0 = TMA producer, warp 1 = TMEM owner + MMA issuer, warps 2-5 = epilogue.
-// Two TMEM accumulators: the epilogue drains tile i while the MMAs of tile i+1 run.
-template <int BN>
-__global__ void __launch_bounds__(kProjThreads, 1)
-    proj_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ CUtensorMap map_wk,
-                const __grid_constant__ CUtensorMap map_wv, const __grid_constant__ ProjParams p) {
-    using Cfg = ProjCfg<BN>;
-    constexpr int S = Cfg::kStages;
-    constexpr int NACC = Cfg::kAccum;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem;
-    uint8_t *sB = smem + S * Cfg::kATile;
-    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes);
-    uint64_t *empty_bar = full_bar + S;
-    uint64_t *tfull_bar = empty_bar + S;      // MMA -> epilogue, one per accumulator
-    uint64_t *tempty_bar = tfull_bar + NACC;  // epilogue -> MMA, one per accumulator
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(tempty_bar + NACC);
-    __shared__ int s_abort;
-
-    const int warp = threadIdx.x / 32;
-    const int lane = threadIdx.x % 32;
-    const int mn_tiles = p.m_tiles * p.n_tiles;
-    const int total = mn_tiles * p.k_splits;   // work units: (k split, m tile, n tile), n fastest
-    const int key_tiles = p.d_h / BN;
-
-    if (threadIdx.x == 0) {
-        s_abort = 0;
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], 1);
-        }
-        for (int a = 0; a < NACC; ++a) {
-            mbar_init(&tfull_bar[a], 1);
-            mbar_init(&tempty_bar[a], 4);   // one arrival per epilogue warp
-        }
-        fence_barrier_init();
-        tma_prefetch_desc(&map_m);
-        tma_prefetch_desc(&map_wk);
-        tma_prefetch_desc(&map_wv);
-    }
-    if (warp == 1) {
-        tmem_alloc(s_tmem, Cfg::kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *s_tmem;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            int it = 0, issued = 0;
-            for (int t = blockIdx.x; t < total && !s_abort; t += gridDim.x) {
-                const int ks = t / mn_tiles, tmn = t - ks * mn_tiles;
-                const int mt = tmn / p.n_tiles, nt = tmn - mt * p.n_tiles;
-                const bool is_key = nt < key_tiles;
-                const CUtensorMap *map_w = is_key ? &map_wk : &map_wv;
-                const int c0 = (is_key ? nt : nt - key_tiles) * BN;
-                const int m0 = mt * kBM;
-                const int kb0 = ks * p.kb_per_split, kb1 = min(p.k_blocks, kb0 + p.kb_per_split);
-                for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (it / S) & 1;
-                    if (!mbar_wait(&empty_bar[s], ph ^ 1, &s_abort)) break;
-                    mbar_arrive_expect_tx(&full_bar[s], Cfg::kStageBytes);
-                    tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
-                    tma_load_2d(sB + s * Cfg::kBTile, map_w, &full_bar[s], kb * kBK, c0);
-                    issued = it + 1;
-                }
-            }
-            if (s_abort) {
-                // Every issued copy must land before the CTA's shared memory is released.
-                volatile int never = 0;
-                for (int k = issued - S > 0 ? issued - S : 0; k < issued; ++k)
-                    if (!mbar_wait(&full_bar[k % S], (k / S) & 1, &never)) break;
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
-            int it = 0, li = 0;
-            for (int t = blockIdx.x; t < total && !s_abort; t += gridDim.x, ++li) {
-                const int acc = li % NACC;
-                const uint32_t use = li / NACC;
-                if (!mbar_wait(&tempty_bar[acc], (use & 1) ^ 1, &s_abort)) break;
-                tc_fence_after();
-                const uint32_t dst = tmem_base + acc * BN;
-                const int ks = t / mn_tiles;
-                const int kb0 = ks * p.kb_per_split, kb1 = min(p.k_blocks, kb0 + p.kb_per_split);
-                bool ok = true;
-                for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (it / S) & 1;
-                    if (!mbar_wait(&full_bar[s], ph, &s_abort)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint64_t adesc = sdesc_kmajor_sw128(sA + s * Cfg::kATile);
-                    const uint64_t bdesc = sdesc_kmajor_sw128(sB + s * Cfg::kBTile);
-#pragma unroll
-                    for (int k = 0; k < kBK / kUmmaK; ++k) {
-                        const uint64_t koff = static_cast<uint64_t>((k * kUmmaK * 2) >> 4);
-                        umma_bf16_ss(dst, adesc + koff, bdesc + koff, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
-                    }
-                    umma_commit(&empty_bar[s]);   // frees the stage once these MMAs have read it
-                }
-                if (!ok) break;
-                umma_commit(&tfull_bar[acc]);     // accumulator ready for the epilogue
-            }
-            if (s_abort) {
-                for (int a = 0; a < NACC; ++a) mbar_arrive(&tfull_bar[a]);   // release waiting epilogue warps
-            }
-        }
-    } else {
-        // ---------------------------------------------------------------- epilogue
-        const int sub = warp & 3;                      // TMEM lane quarter this warp may access
-        const int row = sub * 32 + lane;
-        int li = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x, ++li) {
-            const int acc = li % NACC;
-            const uint32_t use = li / NACC;
-            if (!mbar_wait(&tfull_bar[acc], use & 1, &s_abort) || s_abort) break;
-            tc_fence_after();
-            const int ks = t / mn_tiles, tmn = t - ks * mn_tiles;
-            const int mt = tmn / p.n_tiles, nt = tmn - mt * p.n_tiles;
-            const bool is_key = nt < key_tiles;
-            const int c0 = (is_key ? nt : nt - key_tiles) * BN;
-            const int64_t n = static_cast<int64_t>(mt) * kBM + row;
-            const bool valid = n < p.n_tok;
-            const uint32_t taddr = tmem_base + acc * BN + (static_cast<uint32_t>(sub * 32) << 16);
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f;
-            for (int cc = 0; cc < BN; cc += 32) {
-                float accv[32];
-                tmem_ld32(taddr + cc, accv);
-                if (!valid) continue;
-                if (p.k_splits > 1) {
-                    // split-K: raw partial accumulator; splitk_reduce_kernel finishes the tile
-                    float4 *ap = reinterpret_cast<float4 *>(
-                        p.acc_out + (static_cast<int64_t>(ks) * p.n_tok + n) * (2 * p.d_h) + nt * BN + cc);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        ap[q] = make_float4(accv[4 * q], accv[4 * q + 1], accv[4 * q + 2], accv[4 * q + 3]);
-                } else if (is_key) {
-                    const uint4 *hp = reinterpret_cast<const uint4 *>(p.h + n * p.d_h + c0 + cc);
-                    const uint4 *gq = reinterpret_cast<const uint4 *>(p.gamma_q + c0 + cc);
-                    const uint4 *gk = reinterpret_cast<const uint4 *>(p.gamma_k + c0 + cc);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 hw = __ldg(hp + q), qw = __ldg(gq + q), kw = __ldg(gk + q);
-                        const uint32_t h4[4] = {hw.x, hw.y, hw.z, hw.w};
-                        const uint32_t q4[4] = {qw.x, qw.y, qw.z, qw.w};
-                        const uint32_t k4[4] = {kw.x, kw.y, kw.z, kw.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = q * 8 + e * 2;
-                            const float h0 = bf16_lo(h4[e]), h1 = bf16_hi(h4[e]);
-                            const float g0 = bf16_lo(q4[e]) * bf16_lo(k4[e]);
-                            const float g1 = bf16_hi(q4[e]) * bf16_hi(k4[e]);
-                            const float k0 = accv[j], k1 = accv[j + 1];
-                            a0 = fmaf(h0, h0, a0);
-                            a0 = fmaf(h1, h1, a0);
-                            a1 = fmaf(h0 * g0, k0, a1);
-                            a1 = fmaf(h1 * g1, k1, a1);
-                            a2 = fmaf(k0, k0, a2);
-                            a2 = fmaf(k1, k1, a2);
-                        }
-                    }
-                } else {
-                    float4 *vp = reinterpret_cast<float4 *>(p.v + n * p.d_h + c0 + cc);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 x = make_float4(accv[4 * q], accv[4 * q + 1], accv[4 * q + 2], accv[4 * q + 3]);
-                        vp[q] = x;
-                        a0 = fmaf(x.x, x.x, a0);
-                        a0 = fmaf(x.y, x.y, a0);
-                        a0 = fmaf(x.z, x.z, a0);
-                        a0 = fmaf(x.w, x.w, a0);
-                    }
-                }
-            }
-            // the accumulator has been read: hand it back to the MMA warp
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
-            if (valid && p.k_splits == 1) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem_base, Cfg::kTmemCols);
-    }
-}
-
-// Finishes a split-K projection: sums the k_splits partial accumulators of one token and one
-// BN-wide tile, then produces exactly what the unsplit epilogue produces for that tile --
-// (S0, S1, S2) for a key tile, v and S3 for a value tile.  Grid: (n_tiles, n_tok); block:
-// kReduceThreads threads x 2 channels; fixed-order sums (deterministic).
-constexpr int kReduceThreads = 128;
-
-__global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const __grid_constant__ ProjParams p, int BN) {
-    __shared__ float s_red[3][kReduceThreads / 32];
-    const int nt = blockIdx.x;
-    const int64_t n = blockIdx.y;
-    const int key_tiles = p.d_h / BN;
-    const bool is_key = nt < key_tiles;
-    const int c0 = (is_key ? nt : nt - key_tiles) * BN;
-    const int64_t stride_split = p.n_tok * (2 * p.d_h);
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f;
-    for (int j = threadIdx.x * 2; j < BN; j += kReduceThreads * 2) {
-        const float *src = p.acc_out + n * (2 * p.d_h) + nt * BN + j;
-        float x0 = 0.f, x1 = 0.f;
-        for (int ks = 0; ks < p.k_splits; ++ks) {
-            const float2 q = __ldg(reinterpret_cast<const float2 *>(src + ks * stride_split));
-            x0 += q.x;
-            x1 += q.y;
-        }
-        if (is_key) {
-            const uint32_t hw = __ldg(reinterpret_cast<const uint32_t *>(p.h + n * p.d_h + c0 + j));
-            const uint32_t qw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_q + c0 + j));
-            const uint32_t kw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_k + c0 + j));
-            const float h0 = bf16_lo(hw), h1 = bf16_hi(hw);
-            a0 = fmaf(h0, h0, fmaf(h1, h1, a0));
-            a1 = fmaf(h0 * bf16_lo(qw) * bf16_lo(kw), x0, fmaf(h1 * bf16_hi(qw) * bf16_hi(kw), x1, a1));
-            a2 = fmaf(x0, x0, fmaf(x1, x1, a2));
-        } else {
-            *reinterpret_cast<float2 *>(p.v + n * p.d_h + c0 + j) = make_float2(x0, x1);
-            a0 = fmaf(x0, x0, fmaf(x1, x1, a0));
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        a0 += __shfl_xor_sync(0xffffffffu, a0, o);
-        a1 += __shfl_xor_sync(0xffffffffu, a1, o);
-        a2 += __shfl_xor_sync(0xffffffffu, a2, o);
-    }
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    if (lane == 0) {
-        s_red[0][warp] = a0;
-        s_red[1][warp] = a1;
-        s_red[2][warp] = a2;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float b0 = 0.f, b1 = 0.f, b2 = 0.f;
-        for (int w = 0; w < kReduceThreads / 32; ++w) {
-            b0 += s_red[0][w];
-            b1 += s_red[1][w];
-            b2 += s_red[2][w];
-        }
-        p.part[n * p.n_tiles + nt] = make_float4(b0, b1, b2, 0.f);
-    }
-}
 
 struct GateParams {
     const uint16_t *h;        // [n_tok, d_h]
@@ -340,6 +33,7 @@ struct GateParams {
     int32_t tok_chunk;        // tokens per CTA (T when a conv state is carried)
     float eps;
     float inv_sqrt_d;
+    const float2 *scal;       // [n_tok] (g, beta) from gate_scalars_kernel, or null
 };
 
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + __expf(-z)); }
@@ -485,6 +179,51 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
     }
 }
 
+// Per-token gate scalars from the projection partials: scal[n] = (g, g / rms_U).  One warp
+// per token; lanes split the tiles, fixed-order butterfly reduction.
+__global__ void __launch_bounds__(256) gate_scalars_kernel(const float4 *__restrict__ part, int64_t n_tok,
+                                                           int32_t n_tiles, int32_t n_key_tiles, int32_t d_h,
+                                                           float eps, float inv_sqrt_d, float2 *__restrict__ scal) {
+    const int64_t n = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+    const int lane = threadIdx.x % 32;
+    if (n >= n_tok) return;
+    const float4 *pp = part + n * n_tiles;
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    for (int j = lane; j < n_tiles; j += 32) {
+        const float4 q = __ldg(pp + j);
+        if (j < n_key_tiles) {
+            s0 += q.x;
+            s1 += q.y;
+            s2 += q.z;
+        } else {
+            s3 += q.x;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+        s3 += __shfl_xor_sync(0xffffffffu, s3, o);
+    }
+    if (lane == 0) {
+        const float inv_d = 1.f / static_cast<float>(d_h);
+        const float rms_h = sqrtf(s0 * inv_d + eps);
+        const float rms_k = sqrtf(s2 * inv_d + eps);
+        const float g = 1.f / (1.f + __expf(-(s1 / (rms_h * rms_k) * inv_sqrt_d)));
+        scal[n] = make_float2(g, g / sqrtf(g * g * s3 * inv_d + eps));
+    }
+}
+
+// x * sigmoid(x) = h + h * tanh(h) with h = x / 2, on the hardware tanh approximation
+// (relative error about 2^-11).
+__device__ __forceinline__ float silu_fast(float x) {
+    const float h = 0.5f * x;
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
+}
+
 // Fast path for the pages' conv shape (kernel 4, dilation 3): prefill, and decode with a
 // carried conv state when one chunk covers the whole call (T <= 3*CH).
 // Same arithmetic as gate_conv_kernel, organised for memory-level parallelism: a CTA covers
@@ -509,9 +248,19 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
     const float inv_d = 1.f / static_cast<float>(p.d_h);
     const int64_t row0 = static_cast<int64_t>(b) * p.T;
 
-    // per-token scalars: one warp per token, lanes split the tiles, fixed-order reduction
+    // per-token scalars: precomputed by gate_scalars_kernel when p.scal is set, else one warp
+    // per token reduces the tiles here
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    for (int i = warp; i < TC + HALO; i += kGateFastThreads / 32) {
+    if (p.scal != nullptr) {
+        for (int i = threadIdx.x; i < TC + HALO; i += kGateFastThreads) {
+            const int t = lo + i;
+            float2 sc = make_float2(0.f, 0.f);
+            if (t >= 0 && t < t1) sc = __ldg(p.scal + row0 + t);
+            s_g[i] = sc.x;
+            s_beta[i] = sc.y;
+        }
+    }
+    for (int i = warp; i < TC + HALO && p.scal == nullptr; i += kGateFastThreads / 32) {
         const int t = lo + i;
         float g = 0.f, beta = 0.f;
         if (t >= 0 && t < t1) {
@@ -617,7 +366,7 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
                 float acc = 0.f;
 #pragma unroll
                 for (int i = 0; i < KS; ++i) acc = fmaf(w[e][i], u[i][e], acc);
-                dl[e] = fmaf(g, vj[e], acc * fast_sigmoid(acc));
+                dl[e] = fmaf(g, vj[e], silu_fast(acc));
                 ob[e] = f32_to_bf16_bits(hv[e] + dl[e]);
             }
             const int64_t n = row0 + t;

@@ -53,6 +53,7 @@ def _plan(**kw):
     (dict(eps=0.0), E.ENGRAM_ERR_INVALID_ARG),
     (dict(conv_kernel=9), E.ENGRAM_ERR_UNSUPPORTED),
     (dict(heads_per_order=17), E.ENGRAM_ERR_UNSUPPORTED),
+    (dict(flags=0x2), E.ENGRAM_ERR_INVALID_ARG),                                # unknown flag bit
 ])
 def test_init_rejects_bad_configs(kw, code):
     with pytest.raises(E.EngramError) as ei:

@@ -203,7 +203,7 @@ Workspace layout(const engram_plan *plan, int64_t n_tok) {
     w.xr = off;   off = align256(off + sizeof(int32_t) * n_tok);
     w.idx = off;  off = align256(off + sizeof(uint32_t) * n_tok * H);
     w.m = off;    off = align256(off + sizeof(uint16_t) * n_tok * plan->mem_dim);
-    size_t v_bytes = sizeof(float) * n_tok * d_h;
+    size_t v_bytes = sizeof(uint16_t) * n_tok * d_h;
     if (use_fused_gate(plan, n_tok, false)) {
         const size_t fb = fused_vbuf_bytes(plan, n_tok);   // the fused kernel's v scratch reuses this region
         if (fb > v_bytes) v_bytes = fb;
@@ -282,7 +282,7 @@ int set_proj_smem_attr() {
 
 template <int BN>
 int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
-                int64_t n_tok, float *v, float4 *part, cudaStream_t stream, float *acc = nullptr,
+                int64_t n_tok, uint16_t *v, float4 *part, cudaStream_t stream, float *acc = nullptr,
                 int k_splits = 1, int kb_per_split = 0, bool run_reduce = true,
                 engram::ProjParams *params_out = nullptr) {
     const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim;
@@ -428,7 +428,7 @@ int launch_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *
 }
 
 engram::GateParams make_gate_params(const engram_plan *plan, const engram_weights *w, const uint16_t *h,
-                                    const float *v, const float4 *part, int n_tiles, int32_t B, int32_t T,
+                                    const uint16_t *v, const float4 *part, int n_tiles, int32_t B, int32_t T,
                                     uint16_t *conv_state, uint16_t *out, float *delta) {
     engram::GateParams p{};
     const int d_h = plan->cfg.hidden_dim;
@@ -454,7 +454,7 @@ engram::GateParams make_gate_params(const engram_plan *plan, const engram_weight
     return p;
 }
 
-int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const float *v,
+int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *v,
                      const float4 *part, int n_tiles, int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out,
                      float *delta, cudaStream_t stream, float2 *scal = nullptr) {
     engram::GateParams p{};
@@ -615,7 +615,7 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
         return launch_fused_gate(plan, w, h, m, B, T, out, delta, reinterpret_cast<float *>(ws + L.v), stream);
     }
     const ProjShape ps = proj_shape(plan, n_tok, true);
-    float *v = reinterpret_cast<float *>(ws + L.v);
+    uint16_t *v = reinterpret_cast<uint16_t *>(ws + L.v);
     float4 *part = reinterpret_cast<float4 *>(ws + L.part);
     float *acc = ps.k_splits > 1 ? reinterpret_cast<float *>(ws + L.acc) : nullptr;
     const int d_h = plan->cfg.hidden_dim;
@@ -954,7 +954,7 @@ int engram_gate_conv_noalloc(const engram_plan *plan, const engram_weights *w, c
     const int d_h = plan->cfg.hidden_dim;
     const int bn = choose_bn(d_h, n_tok);
     const int n_tiles = 2 * d_h / bn;
-    const size_t v_bytes = align256(sizeof(float) * static_cast<size_t>(n_tok) * d_h);
+    const size_t v_bytes = align256(sizeof(uint16_t) * static_cast<size_t>(n_tok) * d_h);
     const size_t part_bytes = align256(sizeof(float4) * static_cast<size_t>(n_tok) * n_tiles);
     if (v_bytes + part_bytes > ENGRAM_NOALLOC_SCRATCH_BYTES)
         return fail(ENGRAM_ERR_UNSUPPORTED,
@@ -963,7 +963,7 @@ int engram_gate_conv_noalloc(const engram_plan *plan, const engram_weights *w, c
     uint8_t *scratch = nullptr;
     if ((rc = noalloc_scratch(&scratch)) != ENGRAM_OK) return rc;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-    float *v = reinterpret_cast<float *>(scratch);
+    uint16_t *v = reinterpret_cast<uint16_t *>(scratch);
     float4 *part = reinterpret_cast<float4 *>(scratch + v_bytes);
     if (bn == 256) rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream);
     else if (bn == 128) rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream);

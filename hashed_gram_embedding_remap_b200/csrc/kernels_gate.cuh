@@ -18,7 +18,7 @@ namespace engram {
 
 struct GateParams {
     const uint16_t *h;        // [n_tok, d_h]
-    const float *v;           // [n_tok, d_h]
+    const uint16_t *v;        // [n_tok, d_h] bf16
     const float4 *part;       // [n_tok, n_tiles]
     const uint16_t *gamma_c;  // [d_h]
     const uint16_t *conv_w;   // [d_h, ksize]
@@ -109,8 +109,8 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
                 const int si = t - lo;
                 if (t >= 0) {
                     const int64_t n = static_cast<int64_t>(b) * p.T + t;
-                    const float4 v4 = *reinterpret_cast<const float4 *>(p.v + n * p.d_h + c);
-                    vv[0] = v4.x; vv[1] = v4.y; vv[2] = v4.z; vv[3] = v4.w;
+                    const uint2 v4 = *reinterpret_cast<const uint2 *>(p.v + n * p.d_h + c);
+                    vv[0] = bf16_lo(v4.x); vv[1] = bf16_hi(v4.x); vv[2] = bf16_lo(v4.y); vv[3] = bf16_hi(v4.y);
                     const float beta = s_beta[si];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) u[e] = beta * vv[e] * gc[e];
@@ -161,12 +161,12 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
                 uint2 o;
                 if (t >= 0) {
                     const int64_t n = static_cast<int64_t>(b) * p.T + t;
-                    const float4 v4 = *reinterpret_cast<const float4 *>(p.v + n * p.d_h + c);
+                    const uint2 v4 = *reinterpret_cast<const uint2 *>(p.v + n * p.d_h + c);
                     const float beta = s_beta[t - lo];
-                    const uint16_t u0 = f32_to_bf16_bits(beta * v4.x * gc[0]);
-                    const uint16_t u1 = f32_to_bf16_bits(beta * v4.y * gc[1]);
-                    const uint16_t u2 = f32_to_bf16_bits(beta * v4.z * gc[2]);
-                    const uint16_t u3 = f32_to_bf16_bits(beta * v4.w * gc[3]);
+                    const uint16_t u0 = f32_to_bf16_bits(beta * bf16_lo(v4.x) * gc[0]);
+                    const uint16_t u1 = f32_to_bf16_bits(beta * bf16_hi(v4.x) * gc[1]);
+                    const uint16_t u2 = f32_to_bf16_bits(beta * bf16_lo(v4.y) * gc[2]);
+                    const uint16_t u3 = f32_to_bf16_bits(beta * bf16_hi(v4.y) * gc[3]);
                     o.x = static_cast<uint32_t>(u0) | (static_cast<uint32_t>(u1) << 16);
                     o.y = static_cast<uint32_t>(u2) | (static_cast<uint32_t>(u3) << 16);
                 } else {
@@ -312,21 +312,18 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
     }
 #pragma unroll 1
     for (int r = 0; r < DIL; ++r) {
-        float2 vv[CH + KS - 1];
+        // raw bf16 pairs: v for positions in the call, the carried conv input u for positions
+        // before it (decode), zero otherwise; every load is issued before any is used
+        uint32_t vv[CH + KS - 1];
         uint32_t hh[CH];
 #pragma unroll
         for (int j = 0; j < CH + KS - 1; ++j) {
             const int t = lo + r + DIL * j;
-            if (t >= 0 && t < t1) {
-                vv[j] = __ldg(reinterpret_cast<const float2 *>(p.v + (row0 + t) * p.d_h + c));
-            } else if (t < 0 && p.conv_state != nullptr) {
-                // conv input carried from the previous call (already u, stored bf16)
-                const uint32_t sw = *reinterpret_cast<const uint32_t *>(
-                    p.conv_state + (static_cast<int64_t>(b) * HALO + HALO + t) * p.d_h + c);
-                vv[j] = make_float2(bf16_lo(sw), bf16_hi(sw));
-            } else {
-                vv[j] = make_float2(0.f, 0.f);
-            }
+            const bool in_call = t >= 0 && t < t1;
+            const bool carried = t < 0 && p.conv_state != nullptr;
+            const uint16_t *src = in_call ? p.v + (row0 + t) * p.d_h + c
+                                          : p.conv_state + (static_cast<int64_t>(b) * HALO + HALO + t) * p.d_h + c;
+            vv[j] = (in_call || carried) ? *reinterpret_cast<const uint32_t *>(src) : 0u;
         }
 #pragma unroll
         for (int j = 0; j < CH; ++j) {
@@ -340,7 +337,7 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
         for (int j = 0; j < CH + KS - 1; ++j) {
             const int si = r + DIL * j;            // index into s_g / s_beta
             const float beta = s_beta[si];
-            const float vj[2] = {vv[j].x, vv[j].y};
+            const float vj[2] = {bf16_lo(vv[j]), bf16_hi(vv[j])};
 #pragma unroll
             for (int i = KS - 1; i > 0; --i) {
                 u[i][0] = u[i - 1][0];
@@ -383,7 +380,8 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
             const int t = p.T - HALO + sl;
             uint32_t o;
             if (t >= 0) {
-                const float2 vt = __ldg(reinterpret_cast<const float2 *>(p.v + (row0 + t) * p.d_h + c));
+                const uint32_t vw = __ldg(reinterpret_cast<const uint32_t *>(p.v + (row0 + t) * p.d_h + c));
+                const float2 vt = make_float2(bf16_lo(vw), bf16_hi(vw));
                 const float beta = s_beta[t - lo];
                 o = static_cast<uint32_t>(f32_to_bf16_bits(beta * vt.x * gc[0])) |
                     (static_cast<uint32_t>(f32_to_bf16_bits(beta * vt.y * gc[1])) << 16);
@@ -448,7 +446,8 @@ __global__ void __launch_bounds__(kDecodeThreads) gate_conv_decode_kernel(const 
     if (active) {
 #pragma unroll
         for (int k = 0; k < S; ++k) st[k] = *reinterpret_cast<const uint32_t *>(state + k * p.d_h);
-        v = __ldg(reinterpret_cast<const float2 *>(p.v + static_cast<int64_t>(b) * p.d_h + c));
+        const uint32_t vw = __ldg(reinterpret_cast<const uint32_t *>(p.v + static_cast<int64_t>(b) * p.d_h + c));
+        v = make_float2(bf16_lo(vw), bf16_hi(vw));
         hw = __ldg(reinterpret_cast<const uint32_t *>(p.h + static_cast<int64_t>(b) * p.d_h + c));
         gw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_c + c));
         w0 = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + c * 4));

@@ -9,7 +9,7 @@
 // warps 2-5 drain the other accumulator with tcgen05.ld while the next unit's MMAs run.  The
 // epilogue never writes k~: for a key tile it reduces, per token, S0 = sum h^2,
 // S1 = sum h gamma_q gamma_k k~ and S2 = sum k~^2 over the tile's channels; for a value tile it
-// writes v (fp32) and S3 = sum v^2.  Split-K units write raw fp32 partial accumulators and
+// writes v (bf16; S3 = sum v^2 from the fp32 values).  Split-K units write raw fp32 partial accumulators and
 // splitk_reduce_kernel produces the same per-tile outputs.
 #pragma once
 #include <cstdint>
@@ -43,7 +43,7 @@ struct ProjParams {
     const uint16_t *h;         // [n_tok, d_h] bf16
     const uint16_t *gamma_q;   // [d_h]
     const uint16_t *gamma_k;   // [d_h]
-    float *v;                  // [n_tok, d_h] fp32 out
+    uint16_t *v;               // [n_tok, d_h] bf16 out (rounded from the fp32 accumulator)
     float4 *part;              // [n_tok, n_tiles] partial sums out
     int64_t n_tok;
     int32_t d_m, d_h;
@@ -59,6 +59,11 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
     return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+// two floats -> two bf16 (round to nearest even), lo in the low half
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
 }
 
 // Persistent: grid = min(#tiles, #SMs); CTA i takes tiles i, i + grid, ...  Tile t covers
@@ -231,15 +236,18 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                         }
                     }
                 } else {
-                    float4 *vp = reinterpret_cast<float4 *>(p.v + n * p.d_h + c0 + cc);
+                    // S3 from the fp32 accumulator; v itself is stored as bf16
+                    uint4 *vp = reinterpret_cast<uint4 *>(p.v + n * p.d_h + c0 + cc);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 x = make_float4(accv[4 * q], accv[4 * q + 1], accv[4 * q + 2], accv[4 * q + 3]);
-                        vp[q] = x;
-                        a0 = fmaf(x.x, x.x, a0);
-                        a0 = fmaf(x.y, x.y, a0);
-                        a0 = fmaf(x.z, x.z, a0);
-                        a0 = fmaf(x.w, x.w, a0);
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t wv[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float x0 = accv[8 * q + 2 * e], x1 = accv[8 * q + 2 * e + 1];
+                            a0 = fmaf(x0, x0, fmaf(x1, x1, a0));
+                            wv[e] = pack_bf16x2(x0, x1);
+                        }
+                        vp[q] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
                     }
                 }
             }
@@ -290,7 +298,7 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const __g
             a1 = fmaf(h0 * bf16_lo(qw) * bf16_lo(kw), x0, fmaf(h1 * bf16_hi(qw) * bf16_hi(kw), x1, a1));
             a2 = fmaf(x0, x0, fmaf(x1, x1, a2));
         } else {
-            *reinterpret_cast<float2 *>(p.v + n * p.d_h + c0 + j) = make_float2(x0, x1);
+            *reinterpret_cast<uint32_t *>(p.v + n * p.d_h + c0 + j) = pack_bf16x2(x0, x1);
             a0 = fmaf(x0, x0, fmaf(x1, x1, a0));
         }
     }

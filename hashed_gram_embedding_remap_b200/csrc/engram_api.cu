@@ -344,6 +344,7 @@ engram::HashParams make_hash_params(const engram_plan *plan, int32_t B, int32_t 
             const int h = oi * K + j;
             p.order[h] = c.orders[oi];
             p.prime[h] = static_cast<uint64_t>(c.table_rows[h]);
+            p.barrett[h] = static_cast<uint64_t>((static_cast<unsigned __int128>(1) << 64) / p.prime[h]);
             for (int i = 0; i < ENGRAM_MAX_ORDERS; ++i) p.mult[h][i] = plan->mult[h][i];
         }
     p.H = plan->num_tables;
@@ -364,7 +365,8 @@ int launch_lookup(const engram_plan *plan, const int32_t *ids, const int32_t *re
     p.hash = make_hash_params(plan, B, T);
     for (int h = 0; h < plan->num_tables; ++h) p.table[h] = tables[h];
     p.chunks_per_row = plan->cfg.row_dim / 8;
-    const int64_t warps = static_cast<int64_t>(B) * T * plan->num_tables;
+    p.warps_per_row = (p.chunks_per_row + engram::kLookupChunksPerWarp - 1) / engram::kLookupChunksPerWarp;
+    const int64_t warps = static_cast<int64_t>(B) * T * plan->num_tables * p.warps_per_row;
     const int threads = 256;
     const int64_t blocks = (warps * 32 + threads - 1) / threads;
     engram::lookup_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(ids, remap, history, xr_out,
@@ -375,23 +377,7 @@ int launch_lookup(const engram_plan *plan, const int32_t *ids, const int32_t *re
 
 int launch_hash(const engram_plan *plan, const int32_t *ids, const int32_t *remap, const int32_t *history,
                 int32_t B, int32_t T, uint32_t *idx, int32_t *xr_out, cudaStream_t stream) {
-    engram::HashParams p{};
-    const engram_config &c = plan->cfg;
-    const int K = c.heads_per_order;
-    for (int oi = 0; oi < c.num_orders; ++oi)
-        for (int j = 0; j < K; ++j) {
-            const int h = oi * K + j;
-            p.order[h] = c.orders[oi];
-            p.prime[h] = static_cast<uint64_t>(c.table_rows[h]);
-            for (int i = 0; i < ENGRAM_MAX_ORDERS; ++i) p.mult[h][i] = plan->mult[h][i];
-        }
-    p.H = plan->num_tables;
-    p.max_order = c.orders[c.num_orders - 1];
-    p.hist_len = plan->hist_len;
-    p.pad_id = c.pad_id;
-    p.vocab_in = c.vocab_in;
-    p.B = B;
-    p.T = T;
+    const engram::HashParams p = make_hash_params(plan, B, T);
     const int64_t n_tok = static_cast<int64_t>(B) * T;
     const int threads = 256;
     const unsigned blocks = static_cast<unsigned>((n_tok + threads - 1) / threads);
@@ -503,6 +489,14 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
             part, n_tok, n_tiles, p.n_key_tiles, d_h, p.eps, p.inv_sqrt_d, scal);
         ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_scalars_kernel launch");
         p.scal = scal;
+    }
+    if (fast && p.scal != nullptr) {
+        constexpr int kChain4 = 16;   // 48-token chunks, 4 channels per thread
+        dim3 grid4(static_cast<unsigned>((T + 3 * kChain4 - 1) / (3 * kChain4)), static_cast<unsigned>(B),
+                   static_cast<unsigned>((d_h / 4 + engram::kGate4Threads - 1) / engram::kGate4Threads));
+        engram::gate_conv_k4d3_c4_kernel<kChain4><<<grid4, engram::kGate4Threads, 0, stream>>>(p);
+        ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_conv_k4d3_c4_kernel launch");
+        return ENGRAM_OK;
     }
     if (fast) engram::gate_conv_k4d3_kernel<kChain><<<grid, threads, 0, stream>>>(p);
     else engram::gate_conv_kernel<<<grid, threads, smem, stream>>>(p);

@@ -394,6 +394,98 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
     }
 }
 
+// Prefill-only variant of gate_conv_k4d3_kernel with 4 channels per thread (8-byte bf16
+// loads, half the per-element address and predicate work) and 3*CH-token chunks.  Needs the
+// per-token scalars from gate_scalars_kernel.
+constexpr int kGate4Threads = 128;
+
+template <int CH>
+__global__ void __launch_bounds__(kGate4Threads) gate_conv_k4d3_c4_kernel(const __grid_constant__ GateParams p) {
+    constexpr int KS = 4, DIL = 3, HALO = (KS - 1) * DIL, TC = CH * DIL;
+    __shared__ float2 s_sc[TC + HALO];          // (g, beta) per token of [t0 - HALO, t1)
+    const int b = blockIdx.y;
+    const int t0 = blockIdx.x * TC;
+    if (t0 >= p.T) return;
+    const int t1 = min(p.T, t0 + TC);
+    const int lo = t0 - HALO;
+    const int64_t row0 = static_cast<int64_t>(b) * p.T;
+    for (int i = threadIdx.x; i < TC + HALO; i += kGate4Threads) {
+        const int t = lo + i;
+        s_sc[i] = (t >= 0 && t < t1) ? __ldg(p.scal + row0 + t) : make_float2(0.f, 0.f);
+    }
+    __syncthreads();
+    const int q = blockIdx.z * blockDim.x + threadIdx.x;
+    if (q >= p.d_h / 4) return;
+    const int c = q * 4;
+    float gc[4], w[4][KS];
+    {
+        const uint2 gw = __ldg(reinterpret_cast<const uint2 *>(p.gamma_c + c));
+        gc[0] = bf16_lo(gw.x); gc[1] = bf16_hi(gw.x); gc[2] = bf16_lo(gw.y); gc[3] = bf16_hi(gw.y);
+        const uint4 *wp = reinterpret_cast<const uint4 *>(p.conv_w + c * KS);   // 4 channels x 4 taps
+        const uint4 w01 = __ldg(wp), w23 = __ldg(wp + 1);
+        const uint32_t ww[8] = {w01.x, w01.y, w01.z, w01.w, w23.x, w23.y, w23.z, w23.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            w[e][0] = bf16_lo(ww[2 * e]); w[e][1] = bf16_hi(ww[2 * e]);
+            w[e][2] = bf16_lo(ww[2 * e + 1]); w[e][3] = bf16_hi(ww[2 * e + 1]);
+        }
+    }
+    const uint16_t *vbase = p.v + row0 * p.d_h + c;
+    const uint16_t *hbase = p.h + row0 * p.d_h + c;
+#pragma unroll 1
+    for (int r = 0; r < DIL; ++r) {
+        uint2 vv[CH + KS - 1];
+        uint2 hh[CH];
+#pragma unroll
+        for (int j = 0; j < CH + KS - 1; ++j) {
+            const int t = lo + r + DIL * j;
+            vv[j] = (t >= 0 && t < t1) ? __ldg(reinterpret_cast<const uint2 *>(vbase + static_cast<int64_t>(t) * p.d_h))
+                                       : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+            const int t = t0 + r + DIL * j;
+            hh[j] = t < t1 ? __ldg(reinterpret_cast<const uint2 *>(hbase + static_cast<int64_t>(t) * p.d_h))
+                           : make_uint2(0u, 0u);
+        }
+        float u[KS][4];
+#pragma unroll
+        for (int i = 0; i < KS; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) u[i][e] = 0.f;
+#pragma unroll
+        for (int j = 0; j < CH + KS - 1; ++j) {
+            const int si = r + DIL * j;
+            const float2 sc = s_sc[si];
+            const float vj[4] = {bf16_lo(vv[j].x), bf16_hi(vv[j].x), bf16_lo(vv[j].y), bf16_hi(vv[j].y)};
+#pragma unroll
+            for (int i = KS - 1; i > 0; --i)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) u[i][e] = u[i - 1][e];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) u[0][e] = sc.y * vj[e] * gc[e];
+            if (j < KS - 1) continue;
+            const int t = lo + si;
+            if (t >= t1) continue;
+            const uint2 hw = hh[j - (KS - 1)];
+            const float hv[4] = {bf16_lo(hw.x), bf16_hi(hw.x), bf16_lo(hw.y), bf16_hi(hw.y)};
+            float dl[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float acc = w[e][0] * u[0][e];
+#pragma unroll
+                for (int i = 1; i < KS; ++i) acc = fmaf(w[e][i], u[i][e], acc);
+                dl[e] = fmaf(sc.x, vj[e], silu_fast(acc));
+            }
+            const int64_t n = row0 + t;
+            *reinterpret_cast<uint2 *>(p.out + n * p.d_h + c) =
+                make_uint2(pack_bf16x2(hv[0] + dl[0], hv[1] + dl[1]), pack_bf16x2(hv[2] + dl[2], hv[3] + dl[3]));
+            if (p.delta != nullptr)
+                *reinterpret_cast<float4 *>(p.delta + n * p.d_h + c) = make_float4(dl[0], dl[1], dl[2], dl[3]);
+        }
+    }
+}
+
 // Decode step (T = 1) with a carried conv state, kernel 4 / dilation 3: the conv taps of the
 // new token read state slots 6, 3 and 0 (positions t-3, t-6, t-9); the new state is slots
 // 1..8 followed by u_t.  One CTA per (sequence, 512-channel slice); each thread loads all of

@@ -13,6 +13,7 @@ namespace engram {
 struct HashParams {
     uint64_t mult[ENGRAM_MAX_TABLES][ENGRAM_MAX_ORDERS];  // a_{o,j,i}, i = 0 is the current token
     uint64_t prime[ENGRAM_MAX_TABLES];
+    uint64_t barrett[ENGRAM_MAX_TABLES];                  // floor(2^64 / P_h)
     int32_t order[ENGRAM_MAX_TABLES];                     // n-gram order of table h
     int32_t H;
     int32_t max_order;
@@ -30,6 +31,17 @@ __device__ __forceinline__ uint64_t fmix64(uint64_t k) {
     k *= 0xC4CEB9FE1A85EC53ull;
     k ^= k >> 33;
     return k;
+}
+
+// s mod P for a 64-bit s and P < 2^32, exactly, by Barrett reduction: with M = floor(2^64 / P)
+// the estimate q = floor(s * M / 2^64) is at most 2 below floor(s / P), so the remainder
+// s - q P lies in [0, 3P) and at most two subtractions finish it.
+__device__ __forceinline__ uint32_t mod_prime(uint64_t s, uint64_t P, uint64_t M) {
+    const uint64_t q = __umul64hi(s, M);
+    uint64_t r = s - q * P;
+    if (r >= P) r -= P;
+    if (r >= P) r -= P;
+    return static_cast<uint32_t>(r);
 }
 
 // One thread per token.  Reads the token and the (max_order - 1) before it (remapping each
@@ -81,7 +93,7 @@ __global__ void __launch_bounds__(256) hash_kernel(const int32_t *__restrict__ i
 #pragma unroll
         for (int i = 0; i < ENGRAM_MAX_ORDERS; ++i)
             if (i < o) s ^= xp1[i] * p.mult[h][i];
-        row[h] = static_cast<uint32_t>(fmix64(s) % p.prime[h]);
+        row[h] = mod_prime(fmix64(s), p.prime[h], p.barrett[h]);
     }
 }
 
@@ -183,7 +195,9 @@ struct LookupParams {
     HashParams hash;
     const uint16_t *table[ENGRAM_MAX_TABLES];
     int32_t chunks_per_row;  // d_e / 8
+    int32_t warps_per_row;   // each warp copies up to kLookupChunksPerWarp chunks of a row
 };
+constexpr int kLookupChunksPerWarp = 64;
 
 __global__ void __launch_bounds__(256) lookup_kernel(const int32_t *__restrict__ ids,
                                                      const int32_t *__restrict__ remap,
@@ -192,11 +206,13 @@ __global__ void __launch_bounds__(256) lookup_kernel(const int32_t *__restrict__
                                                      const __grid_constant__ LookupParams p) {
     const HashParams &hp = p.hash;
     const int64_t n_tok = static_cast<int64_t>(hp.B) * hp.T;
-    const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+    const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x % 32;
-    const int64_t n = warp_id / hp.H;
+    const int64_t row_id = gw / p.warps_per_row;            // (token, table) row
+    const int part = static_cast<int>(gw - row_id * p.warps_per_row);
+    const int64_t n = row_id / hp.H;
     if (n >= n_tok) return;
-    const int h = static_cast<int>(warp_id - n * hp.H);
+    const int h = static_cast<int>(row_id - n * hp.H);
     uint32_t row = 0;
     if (lane == 0) {
         const int32_t b = static_cast<int32_t>(n / hp.T);
@@ -223,16 +239,26 @@ __global__ void __launch_bounds__(256) lookup_kernel(const int32_t *__restrict__
             } else {
                 x = hp.pad_id;
             }
-            if (i == 0 && h == 0 && xr_out != nullptr) xr_out[n] = x;
+            if (i == 0 && h == 0 && part == 0 && xr_out != nullptr) xr_out[n] = x;
             s ^= (static_cast<uint64_t>(static_cast<int64_t>(x)) + 1ull) * hp.mult[h][i];
         }
-        row = static_cast<uint32_t>(fmix64(s) % hp.prime[h]);
+        row = mod_prime(fmix64(s), hp.prime[h], hp.barrett[h]);
     }
     row = __shfl_sync(0xffffffffu, row, 0);
     const uint4 *src = reinterpret_cast<const uint4 *>(p.table[h]) + static_cast<int64_t>(row) * p.chunks_per_row;
     uint4 *dst = m + (n * hp.H + h) * p.chunks_per_row;
-#pragma unroll 4
-    for (int c = lane; c < p.chunks_per_row; c += 32) dst[c] = __ldg(src + c);
+    const int c_end = min(p.chunks_per_row, (part + 1) * kLookupChunksPerWarp);
+    uint4 val[kLookupChunksPerWarp / 32];
+#pragma unroll
+    for (int k = 0; k < kLookupChunksPerWarp / 32; ++k) {
+        const int c = part * kLookupChunksPerWarp + k * 32 + lane;
+        if (c < c_end) val[k] = __ldg(src + c);
+    }
+#pragma unroll
+    for (int k = 0; k < kLookupChunksPerWarp / 32; ++k) {
+        const int c = part * kLookupChunksPerWarp + k * 32 + lane;
+        if (c < c_end) dst[c] = val[k];
+    }
 }
 
 // ---------------------------------------------------------------- host-resident tables

@@ -182,20 +182,25 @@ def test_gate_conv_entry_matches_forward():
     assert torch.equal(out_fwd.view(torch.int16), out2.view(torch.int16))
 
 
-@pytest.mark.parametrize("geom", ["small", "splitk"])
+@pytest.mark.parametrize("geom", ["small", "splitk", "chunk4"])
 def test_decode_steps_match_oracle_and_update_state(geom):
+    """Consecutive calls carrying the hash history and conv state: one token per call
+    (one-token decode kernels, with and without split-K) and four tokens per call (the
+    chain kernel reading and rewriting the carried state)."""
     if geom == "small":
         wl = small_workload("dec", B=6, T=1, K=2, d_e=32, d_h=256, decode=True)
-    else:
+    elif geom == "splitk":
         wl = small_workload("dec_split", B=32, T=1, K=1, d_e=512, d_h=512, decode=True)
+    else:
+        wl = small_workload("dec_chunk", B=5, T=4, K=2, d_e=32, d_h=256, decode=True)
     di = DeviceInputs(wl)
     w = di.host_weights()
     tables = [synth.fill_bf16(wl.table_spec(h), (wl.primes[h], wl.d_e)) for h in range(wl.H)]
     hist = wl.history()
     state = to_host_u16(di.conv_state)
     for step in range(12):
-        ids_np = synth.zipf_ids(wl.vocab_in, 1.1, (wl.B, 1), 500 + step)
-        h_np = synth.fill_bf16(wl.h_spec(step), (wl.B, wl.d_h))
+        ids_np = synth.zipf_ids(wl.vocab_in, 1.1, (wl.B, wl.T), 500 + step)
+        h_np = synth.fill_bf16(wl.h_spec(step), (wl.B * wl.T, wl.d_h))
         di.ids = to_dev(ids_np)
         di.h = to_dev(h_np)
         di.forward()

@@ -425,7 +425,7 @@ def run_engram(args, wl, world, rank, local):
     # HBM view of the memory-bound kernels (gather and gate+conv)
     row_bytes = wl.H * wl.d_e * 2
     gather_bytes = n_tok * (row_bytes * 2 + wl.H * 4)            # rows read + m written + row ids
-    gate_bytes = n_tok * (wl.d_h * 2 * 3 + 8)                     # v (bf16) + h read, out written, scalars
+    gate_bytes = n_tok * (wl.d_h * 2 * 3 + 8)                     # v (fp16) + h read, out written, scalars
     hbm = {"gather_GBps": gather_bytes / (stage_ms["gather"] / 1e3) / 1e9,
            "gate_conv_GBps": gate_bytes / (stage_ms["gate_conv"] / 1e3) / 1e9,
            "peak_GBps": peaks["hbm"], "nominal_GBps": 8000.0}

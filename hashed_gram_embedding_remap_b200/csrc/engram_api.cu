@@ -485,7 +485,7 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
     if (fast && scal != nullptr && conv_state == nullptr) {
         // scalars once per token instead of once per (CTA, halo-extended chunk)
         const int64_t n_tok = static_cast<int64_t>(B) * T;
-        engram::gate_scalars_kernel<<<static_cast<unsigned>((n_tok * 32 + 255) / 256), 256, 0, stream>>>(
+        engram::gate_scalars_kernel<<<static_cast<unsigned>((n_tok * 8 + 255) / 256), 256, 0, stream>>>(
             part, n_tok, n_tiles, p.n_key_tiles, d_h, p.eps, p.inv_sqrt_d, scal);
         ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_scalars_kernel launch");
         p.scal = scal;

@@ -18,7 +18,7 @@ namespace engram {
 
 struct GateParams {
     const uint16_t *h;        // [n_tok, d_h]
-    const uint16_t *v;        // [n_tok, d_h] bf16
+    const uint16_t *v;        // [n_tok, d_h] fp16 (pack_v2 / v_lo / v_hi)
     const float4 *part;       // [n_tok, n_tiles]
     const uint16_t *gamma_c;  // [d_h]
     const uint16_t *conv_w;   // [d_h, ksize]
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
                 if (t >= 0) {
                     const int64_t n = static_cast<int64_t>(b) * p.T + t;
                     const uint2 v4 = *reinterpret_cast<const uint2 *>(p.v + n * p.d_h + c);
-                    vv[0] = bf16_lo(v4.x); vv[1] = bf16_hi(v4.x); vv[2] = bf16_lo(v4.y); vv[3] = bf16_hi(v4.y);
+                    vv[0] = v_lo(v4.x); vv[1] = v_hi(v4.x); vv[2] = v_lo(v4.y); vv[3] = v_hi(v4.y);
                     const float beta = s_beta[si];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) u[e] = beta * vv[e] * gc[e];
@@ -163,10 +163,10 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
                     const int64_t n = static_cast<int64_t>(b) * p.T + t;
                     const uint2 v4 = *reinterpret_cast<const uint2 *>(p.v + n * p.d_h + c);
                     const float beta = s_beta[t - lo];
-                    const uint16_t u0 = f32_to_bf16_bits(beta * bf16_lo(v4.x) * gc[0]);
-                    const uint16_t u1 = f32_to_bf16_bits(beta * bf16_hi(v4.x) * gc[1]);
-                    const uint16_t u2 = f32_to_bf16_bits(beta * bf16_lo(v4.y) * gc[2]);
-                    const uint16_t u3 = f32_to_bf16_bits(beta * bf16_hi(v4.y) * gc[3]);
+                    const uint16_t u0 = f32_to_bf16_bits(beta * v_lo(v4.x) * gc[0]);
+                    const uint16_t u1 = f32_to_bf16_bits(beta * v_hi(v4.x) * gc[1]);
+                    const uint16_t u2 = f32_to_bf16_bits(beta * v_lo(v4.y) * gc[2]);
+                    const uint16_t u3 = f32_to_bf16_bits(beta * v_hi(v4.y) * gc[3]);
                     o.x = static_cast<uint32_t>(u0) | (static_cast<uint32_t>(u1) << 16);
                     o.y = static_cast<uint32_t>(u2) | (static_cast<uint32_t>(u3) << 16);
                 } else {
@@ -179,34 +179,37 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
     }
 }
 
-// Per-token gate scalars from the projection partials: scal[n] = (g, g / rms_U).  One warp
-// per token; lanes split the tiles, fixed-order butterfly reduction.
+// Per-token gate scalars from the projection partials: scal[n] = (g, g / rms_U).  Eight
+// lanes per token take every eighth tile; a fixed-order butterfly over the eight lanes
+// finishes the sums (deterministic).
 __global__ void __launch_bounds__(256) gate_scalars_kernel(const float4 *__restrict__ part, int64_t n_tok,
                                                            int32_t n_tiles, int32_t n_key_tiles, int32_t d_h,
                                                            float eps, float inv_sqrt_d, float2 *__restrict__ scal) {
-    const int64_t n = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
-    const int lane = threadIdx.x % 32;
-    if (n >= n_tok) return;
-    const float4 *pp = part + n * n_tiles;
+    const int64_t gt = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t n = gt >> 3;
+    const int sub = static_cast<int>(gt & 7);
     float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-    for (int j = lane; j < n_tiles; j += 32) {
-        const float4 q = __ldg(pp + j);
-        if (j < n_key_tiles) {
-            s0 += q.x;
-            s1 += q.y;
-            s2 += q.z;
-        } else {
-            s3 += q.x;
+    if (n < n_tok) {
+        const float4 *pp = part + n * n_tiles;
+        for (int j = sub; j < n_tiles; j += 8) {
+            const float4 q = __ldg(pp + j);
+            if (j < n_key_tiles) {
+                s0 += q.x;
+                s1 += q.y;
+                s2 += q.z;
+            } else {
+                s3 += q.x;
+            }
         }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
+    for (int o = 4; o > 0; o >>= 1) {
         s0 += __shfl_xor_sync(0xffffffffu, s0, o);
         s1 += __shfl_xor_sync(0xffffffffu, s1, o);
         s2 += __shfl_xor_sync(0xffffffffu, s2, o);
         s3 += __shfl_xor_sync(0xffffffffu, s3, o);
     }
-    if (lane == 0) {
+    if (n < n_tok && sub == 0) {
         const float inv_d = 1.f / static_cast<float>(d_h);
         const float rms_h = sqrtf(s0 * inv_d + eps);
         const float rms_k = sqrtf(s2 * inv_d + eps);
@@ -337,18 +340,20 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
         for (int j = 0; j < CH + KS - 1; ++j) {
             const int si = r + DIL * j;            // index into s_g / s_beta
             const float beta = s_beta[si];
-            const float vj[2] = {bf16_lo(vv[j]), bf16_hi(vv[j])};
+            const bool in_seq = lo + si >= 0;
+            // positions in the call hold v (fp16); positions before it hold the carried u (bf16)
+            const float vj[2] = {in_seq ? v_lo(vv[j]) : 0.f, in_seq ? v_hi(vv[j]) : 0.f};
 #pragma unroll
             for (int i = KS - 1; i > 0; --i) {
                 u[i][0] = u[i - 1][0];
                 u[i][1] = u[i - 1][1];
             }
-            if (lo + si >= 0) {
+            if (in_seq) {
                 u[0][0] = beta * vj[0] * gc[0];
                 u[0][1] = beta * vj[1] * gc[1];
             } else {
-                u[0][0] = vj[0];
-                u[0][1] = vj[1];
+                u[0][0] = bf16_lo(vv[j]);
+                u[0][1] = bf16_hi(vv[j]);
             }
             if (j < KS - 1) continue;
             const int t = lo + si;
@@ -381,7 +386,7 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
             uint32_t o;
             if (t >= 0) {
                 const uint32_t vw = __ldg(reinterpret_cast<const uint32_t *>(p.v + (row0 + t) * p.d_h + c));
-                const float2 vt = make_float2(bf16_lo(vw), bf16_hi(vw));
+                const float2 vt = make_float2(v_lo(vw), v_hi(vw));
                 const float beta = s_beta[t - lo];
                 o = static_cast<uint32_t>(f32_to_bf16_bits(beta * vt.x * gc[0])) |
                     (static_cast<uint32_t>(f32_to_bf16_bits(beta * vt.y * gc[1])) << 16);
@@ -457,7 +462,7 @@ __global__ void __launch_bounds__(kGate4Threads) gate_conv_k4d3_c4_kernel(const 
         for (int j = 0; j < CH + KS - 1; ++j) {
             const int si = r + DIL * j;
             const float2 sc = s_sc[si];
-            const float vj[4] = {bf16_lo(vv[j].x), bf16_hi(vv[j].x), bf16_lo(vv[j].y), bf16_hi(vv[j].y)};
+            const float vj[4] = {v_lo(vv[j].x), v_hi(vv[j].x), v_lo(vv[j].y), v_hi(vv[j].y)};
 #pragma unroll
             for (int i = KS - 1; i > 0; --i)
 #pragma unroll
@@ -539,7 +544,7 @@ __global__ void __launch_bounds__(kDecodeThreads) gate_conv_decode_kernel(const 
 #pragma unroll
         for (int k = 0; k < S; ++k) st[k] = *reinterpret_cast<const uint32_t *>(state + k * p.d_h);
         const uint32_t vw = __ldg(reinterpret_cast<const uint32_t *>(p.v + static_cast<int64_t>(b) * p.d_h + c));
-        v = make_float2(bf16_lo(vw), bf16_hi(vw));
+        v = make_float2(v_lo(vw), v_hi(vw));
         hw = __ldg(reinterpret_cast<const uint32_t *>(p.h + static_cast<int64_t>(b) * p.d_h + c));
         gw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_c + c));
         w0 = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + c * 4));

@@ -9,12 +9,13 @@
 // warps 2-5 drain the other accumulator with tcgen05.ld while the next unit's MMAs run.  The
 // epilogue never writes k~: for a key tile it reduces, per token, S0 = sum h^2,
 // S1 = sum h gamma_q gamma_k k~ and S2 = sum k~^2 over the tile's channels; for a value tile it
-// writes v (bf16; S3 = sum v^2 from the fp32 values).  Split-K units write raw fp32 partial accumulators and
+// writes v (fp16; S3 = sum v^2 from the fp32 values).  Split-K units write raw fp32 partial accumulators and
 // splitk_reduce_kernel produces the same per-tile outputs.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "engram.h"
 #include "ptx.cuh"
@@ -43,7 +44,7 @@ struct ProjParams {
     const uint16_t *h;         // [n_tok, d_h] bf16
     const uint16_t *gamma_q;   // [d_h]
     const uint16_t *gamma_k;   // [d_h]
-    uint16_t *v;               // [n_tok, d_h] bf16 out (rounded from the fp32 accumulator)
+    uint16_t *v;               // [n_tok, d_h] fp16 out (rounded from the fp32 accumulator)
     float4 *part;              // [n_tok, n_tiles] partial sums out
     int64_t n_tok;
     int32_t d_m, d_h;
@@ -64,6 +65,20 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// Storage format of the value projection v between the projection and the gate kernels:
+// IEEE fp16 (11 significant bits; v is a projection of bf16 rows by bf16 weights, orders of
+// magnitude inside fp16's range).  Two values per 32-bit word, lo in the low half.
+__device__ __forceinline__ uint32_t pack_v2(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+__device__ __forceinline__ float v_lo(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu)));
+}
+__device__ __forceinline__ float v_hi(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
 }
 
 // Persistent: grid = min(#tiles, #SMs); CTA i takes tiles i, i + grid, ...  Tile t covers
@@ -236,7 +251,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                         }
                     }
                 } else {
-                    // S3 from the fp32 accumulator; v itself is stored as bf16
+                    // S3 from the fp32 accumulator; v itself is stored as fp16
                     uint4 *vp = reinterpret_cast<uint4 *>(p.v + n * p.d_h + c0 + cc);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -245,7 +260,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                         for (int e = 0; e < 4; ++e) {
                             const float x0 = accv[8 * q + 2 * e], x1 = accv[8 * q + 2 * e + 1];
                             a0 = fmaf(x0, x0, fmaf(x1, x1, a0));
-                            wv[e] = pack_bf16x2(x0, x1);
+                            wv[e] = pack_v2(x0, x1);
                         }
                         vp[q] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
                     }
@@ -298,7 +313,7 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const __g
             a1 = fmaf(h0 * bf16_lo(qw) * bf16_lo(kw), x0, fmaf(h1 * bf16_hi(qw) * bf16_hi(kw), x1, a1));
             a2 = fmaf(x0, x0, fmaf(x1, x1, a2));
         } else {
-            *reinterpret_cast<uint32_t *>(p.v + n * p.d_h + c0 + j) = pack_bf16x2(x0, x1);
+            *reinterpret_cast<uint32_t *>(p.v + n * p.d_h + c0 + j) = pack_v2(x0, x1);
             a0 = fmaf(x0, x0, fmaf(x1, x1, a0));
         }
     }

@@ -124,7 +124,7 @@ typedef struct engram_weights {
 int engram_init(const engram_config *cfg, engram_plan *plan);
 
 /* Bytes of device workspace engram_forward / engram_gate_conv need for n_tok = B*T tokens
- * (remapped ids, row ids, memory vectors, bf16 value projections, per-tile partial sums;
+ * (remapped ids, row ids, memory vectors, fp16 value projections, per-tile partial sums;
  * each region 256-byte aligned).  0 on an invalid plan. */
 size_t engram_workspace_size(const engram_plan *plan, int64_t n_tok);
 
@@ -192,7 +192,7 @@ int engram_gather_bounded(const engram_plan *plan, const uint32_t *idx, const ui
  * out: bf16 [B*T, d_h] = bf16_rne(h + Delta).  May not alias h.
  * delta_dbg: NULL, or fp32 [B*T, d_h] receiving Delta before the residual add.
  * The projections k~ = W_k m and v = W_v m run on the tcgen05 tensor cores (bf16 inputs,
- * fp32 accumulation; v is kept in bf16 between the projection and the gate, its norm is
+ * fp32 accumulation; v is kept in fp16 between the projection and the gate, its norm is
  * taken in fp32); norms, gate and conv run in fp32.
  * workspace: >= engram_workspace_size(plan, B*T) bytes, 256-byte aligned. */
 int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uint16_t *h,
@@ -224,10 +224,10 @@ int engram_forward(const engram_plan *plan, const engram_weights *w,
  * hosts that hand an operator only its inputs and outputs and own every device allocation
  * themselves (plugin and custom-op interfaces of inference servers, runtimes with a fixed
  * memory budget, code paths where the device-wide synchronisation of cudaMalloc/cudaFree is
- * not acceptable).  Its scratch (bf16 value projections and per-tile partial sums) lives in
+ * not acceptable).  Its scratch (fp16 value projections and per-tile partial sums) lives in
  * a statically sized array in the library's device data, ENGRAM_NOALLOC_SCRATCH_BYTES per
  * GPU, which every GPU that loads the library holds until the process exits.
- *  - Sizes: the call needs 2*B*T*d_h bytes for v (bf16) plus 16*B*T*(2*d_h/BN) bytes of
+ *  - Sizes: the call needs 2*B*T*d_h bytes for v (fp16) plus 16*B*T*(2*d_h/BN) bytes of
  *    partial sums (BN = 64, 128 or 256, the projection tile width), each rounded up to 256; a
  *    request that does not fit returns ENGRAM_ERR_UNSUPPORTED and launches nothing.  At
  *    d_h = 2560 that is about 5,000 tokens per call.

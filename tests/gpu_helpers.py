@@ -33,7 +33,8 @@ def to_host_u16(t: torch.Tensor) -> np.ndarray:
 class DeviceInputs:
     """All tensors of one workload on the device; tables filled on the GPU."""
 
-    def __init__(self, wl: synth.Workload, step: int = 0, device="cuda", tables=None, flags: int = 0):
+    def __init__(self, wl: synth.Workload, step: int = 0, device="cuda", tables=None, flags: int = 0,
+                 random_gammas: bool = False):
         fill_gpu.build()
         self.wl = wl
         self.ids_np = wl.ids(step)
@@ -48,6 +49,12 @@ class DeviceInputs:
         self.w_v = fill_gpu.filled((wl.d_h, wl.d_m), wl.wv_spec(), device)
         ones = torch.full((wl.d_h,), ONE, dtype=torch.int16, device=device).view(torch.bfloat16)
         self.gamma_q, self.gamma_k, self.gamma_c = ones.clone(), ones.clone(), ones.clone()
+        if random_gammas:
+            # three different gain vectors around 1 (the workloads use 1; these catch a
+            # swapped or dropped gain)
+            for i, g in enumerate((self.gamma_q, self.gamma_k, self.gamma_c)):
+                spec = synth.FillSpec(wl.seeds()["weights"], 200 + i, 0.3)
+                g.copy_((fill_gpu.filled((wl.d_h,), spec, device).float() + 1.0).to(torch.bfloat16))
         self.conv_w = fill_gpu.filled((wl.d_h, wl.conv_kernel), wl.conv_spec(), device)
         self.history = to_dev(wl.history(), device) if wl.decode else None
         self.conv_state = (fill_gpu.filled((wl.B, wl.state_len, wl.d_h), wl.state_spec(), device)

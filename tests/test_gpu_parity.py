@@ -152,6 +152,8 @@ PARITY_CASES = {
     # fewer units: separate projection (BN = 256) and gate/conv kernels
     "bn256_unfused": small_workload("bn256u", B=4, T=500, K=2, d_e=32, d_h=2560),      # 2000 tok
     "seq_shorter_than_halo": small_workload("short", B=40, T=7, K=2, d_e=16, d_h=128),
+    # gate kernel over several channel slices, two sequences with ragged 48-token chunks
+    "gate_3_slices": small_workload("g3s", B=2, T=301, K=2, d_e=24, d_h=1536),
     # decode-sized batches: the projection splits K across CTAs (partial accumulators + reduce)
     "splitk_64tok": small_workload("splitk64", B=64, T=1, K=1, d_e=512, d_h=512),          # 4 splits
     "splitk_ragged_k": small_workload("splitk200", B=100, T=2, K=1, d_e=360, d_h=512),     # d_m=720, 3 splits
@@ -168,6 +170,17 @@ def test_forward_matches_oracle(case):
     assert_delta_close(di.delta.cpu().numpy(), ref["delta"])
     assert_out_close(to_host_u16(di.out), ref["out"])
     assert E.engram_device_status(clear=True) == 0
+
+
+@pytest.mark.parametrize("case", ["ragged_k_bn64", "bn256_unfused", "splitk_64tok", "fused_seq_edges"])
+def test_forward_with_non_unit_gains(case):
+    wl = PARITY_CASES[case]
+    flags = E.ENGRAM_FLAG_FUSED_GATE if case.startswith("fused") else 0
+    di = DeviceInputs(wl, flags=flags, random_gammas=True).forward()
+    torch.cuda.synchronize()
+    ref = _oracle_full(wl, di)
+    assert_delta_close(di.delta.cpu().numpy(), ref["delta"])
+    assert_out_close(to_host_u16(di.out), ref["out"])
 
 
 def test_gate_conv_entry_matches_forward():
@@ -193,7 +206,7 @@ def test_decode_steps_match_oracle_and_update_state(geom):
         wl = small_workload("dec_split", B=32, T=1, K=1, d_e=512, d_h=512, decode=True)
     else:
         wl = small_workload("dec_chunk", B=5, T=4, K=2, d_e=32, d_h=256, decode=True)
-    di = DeviceInputs(wl)
+    di = DeviceInputs(wl, random_gammas=geom != "small")
     w = di.host_weights()
     tables = [synth.fill_bf16(wl.table_spec(h), (wl.primes[h], wl.d_e)) for h in range(wl.H)]
     hist = wl.history()

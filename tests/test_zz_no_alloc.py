@@ -68,7 +68,7 @@ def test_noalloc_matches_workspace_entry_two_calls(case):
 def test_noalloc_rejects_requests_beyond_its_scratch():
     wl = small_workload("noalloc_big", B=1, T=8, K=2, d_e=32, d_h=2560)
     plan = E.Plan.from_workload(wl)
-    # the bf16 value projections alone (2 bytes per channel and token) exceed the array here
+    # the fp16 value projections alone (2 bytes per channel and token) exceed the array here
     T = E.ENGRAM_NOALLOC_SCRATCH_BYTES // (2 * wl.d_h) + 1
     dummy = torch.empty(16, dtype=torch.bfloat16, device="cuda")
     w = E.Weights(dummy, dummy, dummy, dummy, dummy, dummy)

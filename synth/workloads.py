@@ -151,6 +151,7 @@ class Workload:
 P_C1 = (10007, 10009, 10037, 10039)
 P_1M = largest_prime_below(1_000_000)      # 999,983
 P_10M = largest_prime_below(10_000_000)    # 9,999,991
+P_20M = largest_prime_below(20_000_000)    # 19,999,999
 
 WORKLOADS = {
     "tiny": Workload(
@@ -184,6 +185,15 @@ WORKLOADS = {
         vocab_in=248_320, vocab_out=248_320, B=64, T=1, orders=(2, 3), K=1,
         primes=(P_10M,) * 2, d_e=2560, d_h=2560, identity_remap=True, decode=True,
         host_tables=True, ids_kind="uniform", zipf_s=1.3),
+    # the pages' own geometry: 8 two-gram + 8 three-gram heads, ~20M rows per table, 160
+    # values per row (16 x 20M x 160 = 51.2B parameters, ~102 GB): small rows spread over a
+    # huge table, the hardest case for DRAM efficiency of the row gather
+    "ngram16x20m": Workload(
+        name="ngram16x20m", index=5,
+        description="vocab 248,320 (no compression); 8x4096 Zipf(1.1); orders {2,3}, K=8; "
+                    "16 tables of 19,999,999 rows x 160 dims (102 GB); memory 2560; hidden 2560",
+        vocab_in=248_320, vocab_out=248_320, B=8, T=4096, orders=(2, 3), K=8,
+        primes=(P_20M,) * 16, d_e=160, d_h=2560, identity_remap=True),
 }
 
 

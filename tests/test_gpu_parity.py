@@ -295,3 +295,68 @@ def test_forward_replays_identically_in_a_cuda_graph():
         g.replay()
         torch.cuda.synchronize()
         assert torch.equal(di.out.view(torch.int16), eager.view(torch.int16))
+
+
+def _free_device():
+    import gc
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+def test_decode_step_on_full_95gib_tables_sampled():
+    """One decode step of 256 sequences on the full 2 x 9,999,991 x 2560 tables (row byte
+    offsets far above 2^32), checked on sampled sequences with their rows regenerated."""
+    wl = synth.get_workload("decode20m")
+    free, _ = torch.cuda.mem_get_info()
+    if free < wl.table_bytes + (4 << 30):
+        pytest.skip("not enough device memory for the 95.4 GiB tables")
+    try:
+        di = DeviceInputs(wl)
+        state_before = to_host_u16(di.conv_state)
+        hist_before = di.history.cpu().numpy()
+        di.forward()
+        torch.cuda.synchronize()
+        w = di.host_weights()
+        rng = np.random.default_rng(21)
+        seqs = np.sort(rng.choice(wl.B, 12, replace=False))
+        ids = di.ids_np[seqs]
+        idx = oracle.hash_ids(ids, wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id, history=hist_before[seqs])
+        assert idx.max() > (1 << 32) // (wl.d_e * 2)          # rows past the 4 GiB offset boundary
+        tables = [synth.fill_rows_bf16(wl.table_spec(h), wl.d_e, idx[:, h]) for h in range(wl.H)]
+        m = oracle.gather(np.tile(np.arange(len(seqs), dtype=np.uint32)[:, None], (1, wl.H)), tables)
+        h_rows = synth.fill_rows_bf16(wl.h_spec(0), wl.d_h, seqs)
+        ref = oracle.gate_conv(h_rows, m, w["Wk"], w["Wv"], w["gamma_q"], w["gamma_k"], w["gamma_c"],
+                               w["conv_w"], len(seqs), 1, dil=wl.conv_dilation, eps=wl.eps,
+                               conv_state=state_before[seqs], want_state=True)
+        assert_delta_close(di.delta.cpu().numpy()[seqs], ref["delta"])
+        assert_out_close(to_host_u16(di.out)[seqs], ref["out"])
+    finally:
+        di = None
+        _free_device()
+
+
+@pytest.mark.slow
+def test_forward_on_16x20m_tables_sampled_rows():
+    """The pages' own geometry (16 tables x 19,999,999 rows x 160, ~102 GB): the gathered
+    memory vectors on sampled tokens equal the regenerated rows bit for bit."""
+    wl = synth.get_workload("ngram16x20m")
+    free, _ = torch.cuda.mem_get_info()
+    if free < wl.table_bytes + (4 << 30):
+        pytest.skip("not enough device memory for the 102 GB tables")
+    try:
+        plan = E.Plan.from_workload(wl)
+        tables = [fill_gpu.filled((wl.primes[h], wl.d_e), wl.table_spec(h)) for h in range(wl.H)]
+        ids = wl.ids()
+        idx_np = _idx_oracle(wl, ids)
+        m = torch.empty((wl.n_tok, wl.d_m), dtype=torch.bfloat16, device="cuda")
+        E.engram_gather(plan, to_dev(idx_np.view(np.int32)), tables, m)
+        rng = np.random.default_rng(6)
+        sample = np.concatenate([[0, wl.n_tok - 1], rng.integers(0, wl.n_tok, 120)])
+        got = to_host_u16(m[torch.from_numpy(sample).cuda()]).reshape(len(sample), wl.H, wl.d_e)
+        for h in range(wl.H):
+            assert np.array_equal(got[:, h, :], synth.fill_rows_bf16(wl.table_spec(h), wl.d_e, idx_np[sample, h]))
+    finally:
+        tables = m = None
+        _free_device()

@@ -186,7 +186,12 @@ def oracle_sample(wl, n_tok_sample: int, seq: int = 0):
     remap = wl.remap()
     t_gen0 = time.perf_counter()
     idx_probe = oracle.hash_ids(remap[ids], wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id)
-    tables = [synth.fill_rows_bf16(wl.table_spec(h), wl.d_e, idx_probe[:, h]) for h in range(wl.H)]
+    if wl.table_dtype == "fp8":
+        tables = [synth.fill_rows_fp8(wl.table_spec(h), wl.d_e, idx_probe[:, h]) for h in range(wl.H)]
+        scales = [wl.table_scale(h) for h in range(wl.H)]
+    else:
+        tables = [synth.fill_rows_bf16(wl.table_spec(h), wl.d_e, idx_probe[:, h]) for h in range(wl.H)]
+        scales = None
     local_idx = np.tile(np.arange(T, dtype=np.uint32)[:, None], (1, wl.H))
     h = synth.fill_rows_bf16(wl.h_spec(0), wl.d_h, b * wl.T + np.arange(T))
     Wk = synth.fill_bf16(wl.wk_spec(), (wl.d_h, wl.d_m))
@@ -197,7 +202,7 @@ def oracle_sample(wl, n_tok_sample: int, seq: int = 0):
     t0 = time.perf_counter()
     xr = oracle.remap(ids, remap)
     idx = oracle.hash_ids(xr, wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id)
-    m = oracle.gather(local_idx, tables)      # compact tables hold exactly the rows idx names
+    m = oracle.gather(local_idx, tables, scales)   # compact tables hold exactly the rows idx names
     oracle.gate_conv(h, m, Wk, Wv, one, one, one, cw, 1, T, dil=wl.conv_dilation, eps=wl.eps)
     dt = time.perf_counter() - t0
     assert np.array_equal(idx, idx_probe)
@@ -238,7 +243,8 @@ def run_reference(args, wl, world, rank):
 def workload_config(wl, world):
     return {"workload": wl.name, "tokens_per_step_per_gpu": wl.n_tok, "B": wl.B, "T": wl.T,
             "orders": list(wl.orders), "K": wl.K, "H": wl.H, "table_rows": wl.primes[0], "d_e": wl.d_e,
-            "d_m": wl.d_m, "d_h": wl.d_h, "table_GiB": round(wl.table_bytes / 2 ** 30, 2),
+            "d_m": wl.d_m, "d_h": wl.d_h, "table_dtype": wl.table_dtype,
+            "table_GiB": round(wl.table_bytes / 2 ** 30, 2),
             "parallelism": f"replicas x{world}",
             "l2": "inputs larger than L2 (hidden states, memory vectors and tables each exceed 126 MB)"
             if wl.n_tok * wl.d_h * 2 > L2_BYTES else "inputs smaller than L2; L2 not flushed"}
@@ -258,7 +264,8 @@ def run_engram(args, wl, world, rank, local):
     if need > free:
         raise SystemExit(f"not enough device memory: need ~{need / 2**30:.1f} GiB, free {free / 2**30:.1f} GiB")
     # per-rank input: each rank draws its own batch (seed offset by rank)
-    tables = [fill_gpu.filled((wl.primes[h], wl.d_e), wl.table_spec(h), dev) for h in range(wl.H)]
+    fill = fill_gpu.filled_fp8 if wl.table_dtype == "fp8" else fill_gpu.filled
+    tables = [fill((wl.primes[h], wl.d_e), wl.table_spec(h), dev) for h in range(wl.H)]
     ids_np = wl.ids(step=rank)
     ids = torch.from_numpy(ids_np).to(dev)
     remap = None if wl.identity_remap else torch.from_numpy(wl.remap()).to(dev)
@@ -423,8 +430,8 @@ def run_engram(args, wl, world, rank, local):
                 "traffic": kernel_traffic("proj_kernel", wl.name), "peak_source": f"{peaks['source']} bf16 sustained",
                 "algorithmic_per_launch": flops}
     # HBM view of the memory-bound kernels (gather and gate+conv)
-    row_bytes = wl.H * wl.d_e * 2
-    gather_bytes = n_tok * (row_bytes * 2 + wl.H * 4)            # rows read + m written + row ids
+    row_bytes = wl.H * wl.d_e * wl.table_elem_bytes
+    gather_bytes = n_tok * (row_bytes + wl.H * wl.d_e * 2 + wl.H * 4)   # rows read + m written + row ids
     gate_bytes = n_tok * (wl.d_h * 2 * 3 + 8)                     # v (fp16) + h read, out written, scalars
     hbm = {"gather_GBps": gather_bytes / (stage_ms["gather"] / 1e3) / 1e9,
            "gate_conv_GBps": gate_bytes / (stage_ms["gate_conv"] / 1e3) / 1e9,
@@ -471,9 +478,10 @@ def run_hostpinned(args, wl, world, rank, local):
     comp = torch.cuda.current_stream()
     pref = torch.cuda.Stream(priority=-1)   # prefetch kernels get SMs ahead of the stand-in GEMM
     t0 = time.perf_counter()
-    bufs = [fill_gpu.HostMapped(wl.primes[h], wl.d_e) for h in range(wl.H)]
+    eb = wl.table_elem_bytes
+    bufs = [fill_gpu.HostMapped(wl.primes[h], wl.d_e, elem_bytes=eb) for h in range(wl.H)]
     for h, b in enumerate(bufs):
-        fill_gpu.fill_(b.tensor, wl.table_spec(h))
+        (fill_gpu.fill_fp8_ if eb == 1 else fill_gpu.fill_)(b.tensor, wl.table_spec(h))
     torch.cuda.synchronize()
     t_alloc = time.perf_counter() - t0
     tables = [b.tensor for b in bufs]
@@ -495,7 +503,8 @@ def run_hostpinned(args, wl, world, rank, local):
     out = torch.empty((B, wl.d_h), dtype=torch.bfloat16, device=dev)
     ws = E.alloc_workspace(plan, B, dev)
     idx = torch.empty((B, wl.H), dtype=torch.int32, device=dev)
-    staging = [torch.empty((B, wl.d_e), dtype=torch.bfloat16, device=dev) for _ in range(wl.H)]
+    tdt = torch.uint8 if eb == 1 else torch.bfloat16
+    staging = [torch.empty((B, wl.d_e), dtype=tdt, device=dev) for _ in range(wl.H)]
     sidx = torch.empty((B, wl.H), dtype=torch.int32, device=dev)
     uniq = torch.empty((wl.H, B), dtype=torch.int32, device=dev)
     nu = torch.empty((wl.H,), dtype=torch.int32, device=dev)
@@ -577,7 +586,7 @@ def run_hostpinned(args, wl, world, rank, local):
     torch.cuda.synchronize()
     gemm_ms = gs.elapsed_time(ge) / 50
     nu_h = nu.cpu().numpy()
-    uniq_bytes = int(nu_h.sum()) * wl.d_e * 2
+    uniq_bytes = int(nu_h.sum()) * wl.d_e * eb
     # host-link reference: pinned host -> device cudaMemcpyAsync, 1 GiB, best of 5
     hsrc = torch.empty(1 << 29, dtype=torch.int16).pin_memory()
     ddst = torch.empty(1 << 29, dtype=torch.int16, device=dev)
@@ -593,7 +602,7 @@ def run_hostpinned(args, wl, world, rank, local):
     # zero-copy staging throughput on a large batch (8192 tokens x H rows)
     big_n = 8192
     big_idx = torch.randint(0, min(wl.primes), (big_n, wl.H), dtype=torch.int32, device=dev)
-    big_stage = [torch.empty((big_n, wl.d_e), dtype=torch.bfloat16, device=dev) for _ in range(wl.H)]
+    big_stage = [torch.empty((big_n, wl.d_e), dtype=tdt, device=dev) for _ in range(wl.H)]
     big_sidx = torch.empty((big_n, wl.H), dtype=torch.int32, device=dev)
     big_uniq = torch.empty((wl.H, big_n), dtype=torch.int32, device=dev)
     big_nu = torch.empty((wl.H,), dtype=torch.int32, device=dev)
@@ -605,7 +614,7 @@ def run_hostpinned(args, wl, world, rank, local):
         E.engram_stage_rows(plan, big_idx, tables, big_stage, big_sidx, big_uniq, big_nu, stream=comp)
     b1.record(comp)
     torch.cuda.synchronize()
-    big_bytes = int(big_nu.cpu().numpy().sum()) * wl.d_e * 2
+    big_bytes = int(big_nu.cpu().numpy().sum()) * wl.d_e * eb
     big_gbps = big_bytes / (b0.elapsed_time(b1) / 5 / 1e3) / 1e9
     ovl_ms, ovl_clk = results["overlapped"]
     ser_ms, _ = results["serial"]
@@ -649,6 +658,8 @@ def main():
     ap.add_argument("--ids", choices=["uniform", "zipf"], default=None, help="id distribution (host-pinned workload)")
     ap.add_argument("--table-rows", type=int, default=0, help="override the table size (largest prime <= N)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--table-dtype", choices=["bf16", "fp8"], default="bf16",
+                    help="table element type: bf16 rows, or e4m3 codes with one scale per table")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -658,6 +669,8 @@ def main():
         p = synth.largest_prime_below(args.table_rows + 1) if synth.workloads.is_prime(args.table_rows) is False \
             else args.table_rows
         wl = wl.with_(primes=(p,) * wl.H, name=f"{wl.name}[rows={p}]")
+    if args.table_dtype == "fp8":
+        wl = wl.with_(table_dtype="fp8", name=f"{wl.name}-fp8")
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -8,7 +8,8 @@ from ._native import (  # noqa: F401
     ENGRAM_ERR_CUDA, ENGRAM_ERR_INVALID_ARG, ENGRAM_ERR_OOM, ENGRAM_ERR_TIMEOUT,
     ENGRAM_ERR_UNSUPPORTED, ENGRAM_FORWARD_STAGES, ENGRAM_OK, ENGRAM_STATUS_BAD_ROW,
     ENGRAM_STATUS_BAD_TOKEN, ENGRAM_STATUS_WAIT_TIMEOUT, ENGRAM_TABLES_DEVICE,
-    ENGRAM_TABLES_HOST_MAPPED, ENGRAM_NOALLOC_SCRATCH_BYTES, ENGRAM_FLAG_FUSED_GATE, EngramError, LIB_PATH, Plan, Weights, alloc_workspace,
+    ENGRAM_TABLES_HOST_MAPPED, ENGRAM_NOALLOC_SCRATCH_BYTES, ENGRAM_FLAG_FUSED_GATE, ENGRAM_TABLE_BF16,
+    ENGRAM_TABLE_FP8_E4M3, EngramError, LIB_PATH, Plan, Weights, alloc_workspace,
     engram_advance_history, engram_device_status, engram_forward, engram_gate_conv,
     engram_gate_conv_noalloc, engram_gather, engram_hash, engram_stage_rows, engram_remap, engram_workspace_size, last_error, lib, version,
 )

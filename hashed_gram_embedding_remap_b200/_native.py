@@ -31,6 +31,8 @@ ENGRAM_TABLES_DEVICE = 0
 ENGRAM_TABLES_HOST_MAPPED = 1
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
 ENGRAM_FLAG_FUSED_GATE = 0x1
+ENGRAM_TABLE_BF16 = 0
+ENGRAM_TABLE_FP8_E4M3 = 1
 
 _ERRNAMES = {-1: "ENGRAM_ERR_INVALID_ARG", -2: "ENGRAM_ERR_UNSUPPORTED", -3: "ENGRAM_ERR_CUDA",
              -4: "ENGRAM_ERR_OOM", -5: "ENGRAM_ERR_TIMEOUT"}
@@ -59,7 +61,9 @@ class engram_config(C.Structure):
         ("hash_seed", C.c_uint64),
         ("eps", C.c_float),
         ("flags", C.c_int32),
-        ("reserved", C.c_int32 * 6),
+        ("table_dtype", C.c_int32),
+        ("table_scale", C.c_float * ENGRAM_MAX_TABLES),
+        ("reserved", C.c_int32 * 5),
     ]
 
 
@@ -159,7 +163,8 @@ class Plan:
     def __init__(self, *, orders: Sequence[int], heads_per_order: int, table_rows: Sequence[int],
                  row_dim: int, hidden_dim: int, vocab_in: int, vocab_out: int, hash_seed: int,
                  eps: float = 1e-6, conv_kernel: int = 4, table_location: int = ENGRAM_TABLES_DEVICE,
-                 flags: int = 0):
+                 flags: int = 0, table_dtype: int = ENGRAM_TABLE_BF16,
+                 table_scale: Optional[Sequence[float]] = None):
         cfg = engram_config()
         cfg.num_orders = len(orders)
         for i, o in enumerate(orders):
@@ -178,6 +183,9 @@ class Plan:
         cfg.hash_seed = int(hash_seed) & 0xFFFFFFFFFFFFFFFF
         cfg.eps = float(eps)
         cfg.flags = int(flags)
+        cfg.table_dtype = int(table_dtype)
+        for i, sc in enumerate(table_scale or ()):
+            cfg.table_scale[i] = float(sc)
         self.cfg = cfg
         self.plan = engram_plan()
         _check(lib.engram_init(C.byref(cfg), C.byref(self.plan)))
@@ -185,10 +193,12 @@ class Plan:
     @classmethod
     def from_workload(cls, wl, **kw) -> "Plan":
         loc = ENGRAM_TABLES_HOST_MAPPED if kw.pop("host_tables", False) else ENGRAM_TABLES_DEVICE
+        fp8 = getattr(wl, "table_dtype", "bf16") == "fp8"
         return cls(orders=wl.orders, heads_per_order=wl.K, table_rows=wl.primes, row_dim=wl.d_e,
                    hidden_dim=wl.d_h, vocab_in=wl.vocab_in, vocab_out=wl.vocab_out,
                    hash_seed=wl.hash_seed, eps=wl.eps, conv_kernel=wl.conv_kernel,
-                   table_location=loc, **kw)
+                   table_location=loc, table_dtype=ENGRAM_TABLE_FP8_E4M3 if fp8 else ENGRAM_TABLE_BF16,
+                   table_scale=[float(wl.table_scale(h)) for h in range(wl.H)] if fp8 else None, **kw)
 
     @property
     def num_tables(self) -> int:
@@ -224,9 +234,16 @@ class Weights:
         return C.byref(self.struct)
 
 
-def _table_array(tables):
+def _table_array(tables, plan: Optional[Plan] = None):
+    """Pointer array of tables (tensors or raw addresses).  With a plan, tensors must hold the
+    plan's table element type: 2-byte bf16 patterns, or 1-byte e4m3 codes."""
+    want = None
+    if plan is not None:
+        want = 1 if plan.cfg.table_dtype == ENGRAM_TABLE_FP8_E4M3 else 2
     arr = (C.c_void_p * len(tables))()
     for i, t in enumerate(tables):
+        if not isinstance(t, int) and want is not None and t.element_size() != want:
+            raise ValueError(f"tables[{i}] has {t.element_size()}-byte elements; the plan's tables have {want}")
         arr[i] = t if isinstance(t, int) else t.data_ptr()
     return arr
 
@@ -259,7 +276,7 @@ def engram_advance_history(plan: Plan, ids_remapped: torch.Tensor, history: torc
 def engram_gather(plan: Plan, idx: torch.Tensor, tables, m: torch.Tensor, stream=None, rows_bound: int = 0):
     """rows_bound > 0: every table holds only that many rows (device staging buffers from
     engram_stage_rows); row ids at or beyond it read a zero row and raise the status bit."""
-    arr = _table_array(tables)
+    arr = _table_array(tables, plan)
     if rows_bound:
         _check(lib.engram_gather_bounded(plan, _ptr(idx, (torch.int32, torch.uint32), "idx"), arr, idx.shape[0],
                                          int(rows_bound), _ptr(m, _BF16, "m"), _stream(stream)))
@@ -274,7 +291,7 @@ def engram_stage_rows(plan: Plan, idx: torch.Tensor, tables, staging, staged_idx
     n_tok = idx.shape[0]
     cap = staging[0].shape[0]
     _check(lib.engram_stage_rows(plan, _ptr(idx, (torch.int32, torch.uint32), "idx"), n_tok,
-                                 _table_array(tables), _table_array(staging), cap,
+                                 _table_array(tables, plan), _table_array(staging, plan), cap,
                                  _ptr(staged_idx, (torch.int32, torch.uint32), "staged_idx"),
                                  _ptr(unique_rows, (torch.int32, torch.uint32), "unique_rows"),
                                  _ptr(n_unique, torch.int32, "n_unique"), _stream(stream)))
@@ -305,7 +322,7 @@ def engram_forward(plan: Plan, weights: Weights, tables, ids: torch.Tensor, h: t
                    history: Optional[torch.Tensor] = None, conv_state: Optional[torch.Tensor] = None,
                    delta_dbg: Optional[torch.Tensor] = None, stream=None, stage_events=None):
     B, T = ids.shape
-    arr = _table_array(tables)
+    arr = _table_array(tables, plan)
     ev = None
     if stage_events is not None:
         if len(stage_events) != ENGRAM_FORWARD_STAGES + 1:

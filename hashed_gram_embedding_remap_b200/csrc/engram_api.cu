@@ -113,6 +113,9 @@ struct Workspace {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+bool fp8_tables(const engram_plan *plan) { return plan->cfg.table_dtype == ENGRAM_TABLE_FP8_E4M3; }
+int table_elem_bytes(const engram_plan *plan) { return fp8_tables(plan) ? 1 : 2; }
+
 // Width of the projection's N tile: the widest of 256/128/64 that divides d_h and still
 // gives at least two waves of CTAs on the GPU.  ENGRAM_PROJ_TILE_N (64, 128 or 256) forces a
 // width (for tuning and tests); it is read once per process.
@@ -218,7 +221,7 @@ Workspace layout(const engram_plan *plan, int64_t n_tok) {
         w.staged_idx = off; off = align256(off + sizeof(uint32_t) * n_tok * H);
         w.unique = off;     off = align256(off + sizeof(uint32_t) * n_tok * H);
         w.n_unique = off;   off = align256(off + sizeof(int32_t) * H);
-        w.staging = off;    off = align256(off + sizeof(uint16_t) * n_tok * H * plan->cfg.row_dim);
+        w.staging = off;    off = align256(off + static_cast<size_t>(table_elem_bytes(plan)) * n_tok * H * plan->cfg.row_dim);
     }
     w.total = off;
     return w;
@@ -359,18 +362,22 @@ engram::HashParams make_hash_params(const engram_plan *plan, int32_t B, int32_t 
 
 // Fused remap + hash + gather, one warp per (token, table) row.
 int launch_lookup(const engram_plan *plan, const int32_t *ids, const int32_t *remap, const int32_t *history,
-                  int32_t B, int32_t T, const uint16_t *const *tables, int32_t *xr_out, uint16_t *m,
+                  int32_t B, int32_t T, const void *const *tables, int32_t *xr_out, uint16_t *m,
                   cudaStream_t stream) {
     engram::LookupParams p{};
     p.hash = make_hash_params(plan, B, T);
-    for (int h = 0; h < plan->num_tables; ++h) p.table[h] = tables[h];
+    for (int h = 0; h < plan->num_tables; ++h) {
+        p.table[h] = tables[h];
+        p.scale[h] = plan->cfg.table_scale[h];
+    }
     p.chunks_per_row = plan->cfg.row_dim / 8;
     p.warps_per_row = (p.chunks_per_row + engram::kLookupChunksPerWarp - 1) / engram::kLookupChunksPerWarp;
     const int64_t warps = static_cast<int64_t>(B) * T * plan->num_tables * p.warps_per_row;
     const int threads = 256;
     const int64_t blocks = (warps * 32 + threads - 1) / threads;
-    engram::lookup_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(ids, remap, history, xr_out,
-                                                                                reinterpret_cast<uint4 *>(m), p);
+    auto kern = fp8_tables(plan) ? engram::lookup_kernel<true> : engram::lookup_kernel<false>;
+    kern<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(ids, remap, history, xr_out,
+                                                                reinterpret_cast<uint4 *>(m), p);
     ENGRAM_CUDA_TRY(cudaGetLastError(), "lookup_kernel launch");
     return ENGRAM_OK;
 }
@@ -388,12 +395,13 @@ int launch_hash(const engram_plan *plan, const int32_t *ids, const int32_t *rema
 
 
 // rows_override > 0 bounds every table at that many rows (device staging buffers).
-int launch_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables, int64_t n_tok,
+int launch_gather(const engram_plan *plan, const uint32_t *idx, const void *const *tables, int64_t n_tok,
                   uint16_t *m, cudaStream_t stream, int64_t rows_override = 0) {
     engram::GatherParams p{};
     const int H = plan->num_tables;
     for (int h = 0; h < H; ++h) {
         p.table[h] = tables[h];
+        p.scale[h] = plan->cfg.table_scale[h];
         p.rows[h] = static_cast<uint64_t>(rows_override > 0 ? rows_override : plan->cfg.table_rows[h]);
     }
     p.H = H;
@@ -407,8 +415,8 @@ int launch_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;  // 8 x 256 threads resident per SM
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    engram::gather_kernel<kUnroll><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-        idx, reinterpret_cast<uint4 *>(m), p);
+    auto kern = fp8_tables(plan) ? engram::gather_kernel<kUnroll, true> : engram::gather_kernel<kUnroll, false>;
+    kern<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(idx, reinterpret_cast<uint4 *>(m), p);
     ENGRAM_CUDA_TRY(cudaGetLastError(), "gather_kernel launch");
     return ENGRAM_OK;
 }
@@ -504,8 +512,8 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
     return ENGRAM_OK;
 }
 
-int launch_stage(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, const uint16_t *const *tables,
-                 uint16_t *const *staging, int32_t capacity, uint32_t *staged_idx, uint32_t *unique_rows,
+int launch_stage(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, const void *const *tables,
+                 void *const *staging, int32_t capacity, uint32_t *staged_idx, uint32_t *unique_rows,
                  int32_t *n_unique, cudaStream_t stream) {
     const int H = plan->num_tables;
     int N = 1;
@@ -528,7 +536,7 @@ int launch_stage(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, co
     p.n_unique = n_unique;
     p.H = H;
     p.capacity = capacity;
-    p.chunks_per_row = plan->cfg.row_dim / 8;
+    p.chunks_per_row = plan->cfg.row_dim * table_elem_bytes(plan) / 16;   // rows copied as stored
     const int64_t total = static_cast<int64_t>(H) * n_tok * p.chunks_per_row;
     constexpr int kUnroll = 4;
     int64_t blocks = (total + 256 * kUnroll - 1) / (256 * kUnroll);
@@ -721,8 +729,21 @@ int engram_init(const engram_config *cfg, engram_plan *plan) {
     if (!(c.eps > 0.f) || !std::isfinite(c.eps)) return fail(ENGRAM_ERR_INVALID_ARG, "eps must be a positive finite number");
     if (c.table_location != ENGRAM_TABLES_DEVICE && c.table_location != ENGRAM_TABLES_HOST_MAPPED)
         return fail(ENGRAM_ERR_INVALID_ARG, "unknown table_location");
-    for (int i = 0; i < 6; ++i)
+    for (int i = 0; i < 5; ++i)
         if (c.reserved[i] != 0) return fail(ENGRAM_ERR_INVALID_ARG, "reserved fields must be zero");
+    if (c.table_dtype != ENGRAM_TABLE_BF16 && c.table_dtype != ENGRAM_TABLE_FP8_E4M3)
+        return fail(ENGRAM_ERR_INVALID_ARG, "unknown table_dtype %d", c.table_dtype);
+    for (int h = 0; h < ENGRAM_MAX_TABLES; ++h) {
+        const float sc = c.table_scale[h];
+        if (c.table_dtype == ENGRAM_TABLE_FP8_E4M3 && h < H) {
+            if (!(sc > 0.f) || !std::isfinite(sc))
+                return fail(ENGRAM_ERR_INVALID_ARG, "table_scale[%d] must be a positive finite number", h);
+        } else if (sc != 0.f) {
+            return fail(ENGRAM_ERR_INVALID_ARG, "table_scale[%d] must be 0 (bf16 tables or beyond the %d tables)", h, H);
+        }
+    }
+    if (c.table_dtype == ENGRAM_TABLE_FP8_E4M3 && c.row_dim % 16 != 0)
+        return fail(ENGRAM_ERR_UNSUPPORTED, "FP8 tables need row_dim % 16 == 0");
     if (c.flags & ~ENGRAM_FLAG_FUSED_GATE) return fail(ENGRAM_ERR_INVALID_ARG, "unknown flags 0x%x", c.flags);
 
     std::memset(plan, 0, sizeof *plan);
@@ -786,7 +807,7 @@ int engram_advance_history(const engram_plan *plan, const int32_t *ids_remapped,
     return ENGRAM_OK;
 }
 
-int engram_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables, int64_t n_tok,
+int engram_gather(const engram_plan *plan, const uint32_t *idx, const void *const *tables, int64_t n_tok,
                   uint16_t *m, engram_stream_t stream) {
     int rc;
     if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
@@ -801,7 +822,7 @@ int engram_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *
     return launch_gather(plan, idx, tables, n_tok, m, static_cast<cudaStream_t>(stream));
 }
 
-int engram_gather_bounded(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables,
+int engram_gather_bounded(const engram_plan *plan, const uint32_t *idx, const void *const *tables,
                           int64_t n_tok, int64_t rows, uint16_t *m, engram_stream_t stream) {
     int rc;
     if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
@@ -816,8 +837,8 @@ int engram_gather_bounded(const engram_plan *plan, const uint32_t *idx, const ui
     return launch_gather(plan, idx, tables, n_tok, m, static_cast<cudaStream_t>(stream), rows);
 }
 
-int engram_stage_rows(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, const uint16_t *const *tables,
-                      uint16_t *const *staging, int32_t capacity, uint32_t *staged_idx, uint32_t *unique_rows,
+int engram_stage_rows(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, const void *const *tables,
+                      void *const *staging, int32_t capacity, uint32_t *staged_idx, uint32_t *unique_rows,
                       int32_t *n_unique, engram_stream_t stream) {
     int rc;
     if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
@@ -859,7 +880,7 @@ int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
                           static_cast<cudaStream_t>(stream), nullptr);
 }
 
-int engram_forward(const engram_plan *plan, const engram_weights *w, const uint16_t *const *tables,
+int engram_forward(const engram_plan *plan, const engram_weights *w, const void *const *tables,
                    const int32_t *ids, const int32_t *remap, int32_t B, int32_t T, int32_t *history,
                    uint16_t *conv_state, const uint16_t *h, uint16_t *out, float *delta_dbg, void *workspace,
                    size_t workspace_bytes, engram_stream_t stream_, void *const *stage_events) {
@@ -908,9 +929,9 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const uint1
         // host-resident tables: fetch each distinct row of the batch once into HBM staging,
         // then gather from there (results are bit-identical to the HBM-resident path)
         const int H = plan->num_tables;
-        uint16_t *stage_ptr[ENGRAM_MAX_TABLES];
-        for (int h = 0; h < H; ++h)
-            stage_ptr[h] = reinterpret_cast<uint16_t *>(ws + L.staging) + static_cast<int64_t>(h) * n_tok * plan->cfg.row_dim;
+        void *stage_ptr[ENGRAM_MAX_TABLES];
+        const int64_t stage_bytes = n_tok * plan->cfg.row_dim * table_elem_bytes(plan);   // per table
+        for (int h = 0; h < H; ++h) stage_ptr[h] = ws + L.staging + static_cast<int64_t>(h) * stage_bytes;
         uint32_t *sidx = reinterpret_cast<uint32_t *>(ws + L.staged_idx);
         if ((rc = launch_stage(plan, idx, n_tok, tables, stage_ptr, static_cast<int32_t>(n_tok), sidx,
                                reinterpret_cast<uint32_t *>(ws + L.unique), reinterpret_cast<int32_t *>(ws + L.n_unique),

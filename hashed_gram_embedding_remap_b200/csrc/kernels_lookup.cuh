@@ -3,6 +3,8 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "engram.h"
 
@@ -127,19 +129,64 @@ __global__ void advance_history_kernel(const int32_t *__restrict__ xr, int32_t B
     }
 }
 
+// ---------------------------------------------------------------- FP8 (e4m3) tables
+// A table may hold e4m3 codes with one dequantisation scale per table; the gathered value is
+// the bf16 nearest to decode(code) * scale_h (ties to even), rounded once from the exact
+// product.  decode() is exact in fp16 (cvt.rn.f16x2.e4m3x2) and in fp32; the fp32 product
+// a*s is rounded, but fma(a, s, -a*s) recovers its error exactly, and a double rounding
+// (fp32, then bf16) can only go wrong when the fp32 product sits exactly on a bf16 midpoint,
+// where the sign of that error decides.
+
+// bf16 pattern of the correctly rounded product a * s (finite a, s; no underflow).
+__device__ __forceinline__ uint32_t bf16_of_product(float a, float s) {
+    const float hi = __fmul_rn(a, s);
+    const float lo = __fmaf_rn(a, s, -hi);
+    const uint32_t u = __float_as_uint(hi);
+    if ((u & 0xFFFFu) == 0x8000u && lo != 0.0f) return (lo > 0.0f) == (hi > 0.0f) ? (u >> 16) + 1u : (u >> 16);
+    if ((u & 0x7F800000u) == 0x7F800000u) return (u >> 16) | ((u & 0xFFFFu) ? 0x40u : 0u);  // inf / NaN
+    return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+}
+
+// Two e4m3 codes (low byte = first element) -> two dequantised bf16 packed in 32 bits.
+__device__ __forceinline__ uint32_t dequant_e4m3x2(uint32_t two_codes, float scale) {
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes), __NV_E4M3);
+    const float2 f = __half22float2(__half2(hr));
+    return bf16_of_product(f.x, scale) | (bf16_of_product(f.y, scale) << 16);
+}
+
+// Eight codes (8 bytes) -> eight bf16 (16 bytes).
+__device__ __forceinline__ uint4 dequant_e4m3x8(uint2 w, float scale) {
+    return make_uint4(dequant_e4m3x2(w.x & 0xFFFFu, scale), dequant_e4m3x2(w.x >> 16, scale),
+                      dequant_e4m3x2(w.y & 0xFFFFu, scale), dequant_e4m3x2(w.y >> 16, scale));
+}
+
 struct GatherParams {
-    const uint16_t *table[ENGRAM_MAX_TABLES];
+    const void *table[ENGRAM_MAX_TABLES];
     uint64_t rows[ENGRAM_MAX_TABLES];
+    float scale[ENGRAM_MAX_TABLES];  // FP8 tables only
     int32_t H;
-    int32_t chunks_per_row;  // d_e / 8  (16-byte chunks)
+    int32_t chunks_per_row;  // d_e / 8  (16-byte chunks of m)
     int32_t chunks_per_tok;  // H * d_e / 8
     int64_t n_tok;
 };
 
-// m[n, h*d_e + c] = table_h[idx[n, h], c], copied as 16-byte chunks.  Consecutive threads
-// take consecutive chunks of m, so stores are fully coalesced and each table row is read
-// as contiguous 16-byte pieces.  Each thread keeps UNROLL independent chunks in flight.
-template <int UNROLL>
+// One 16-byte chunk of m (8 values) from chunk c of row `row` of table h: 16 bytes of a bf16
+// table, or 8 bytes of an e4m3 table dequantised on the fly.
+template <bool FP8>
+__device__ __forceinline__ uint4 load_row_chunk(const void *table, float scale, uint32_t row, int32_t chunks_per_row,
+                                                int32_t c) {
+    const int64_t off = static_cast<int64_t>(row) * chunks_per_row + c;
+    if constexpr (FP8) {
+        return dequant_e4m3x8(__ldg(reinterpret_cast<const uint2 *>(table) + off), scale);
+    } else {
+        return __ldg(reinterpret_cast<const uint4 *>(table) + off);
+    }
+}
+
+// m[n, h*d_e + c] = table_h[idx[n, h], c], copied as 16-byte chunks of m.  Consecutive
+// threads take consecutive chunks of m, so stores are fully coalesced and each table row is
+// read as contiguous pieces.  Each thread keeps UNROLL independent chunks in flight.
+template <int UNROLL, bool FP8>
 __global__ void __launch_bounds__(256) gather_kernel(const uint32_t *__restrict__ idx, uint4 *__restrict__ m,
                                                      const __grid_constant__ GatherParams p) {
     const int64_t total = p.n_tok * p.chunks_per_tok;
@@ -170,9 +217,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint32_t *__restrict_
             val[u] = make_uint4(0, 0, 0, 0);
             if (i < total) {
                 if (row[u] < p.rows[hh[u]]) {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(p.table[hh[u]]) +
-                                       static_cast<int64_t>(row[u]) * p.chunks_per_row + cc[u];
-                    val[u] = __ldg(src);
+                    val[u] = load_row_chunk<FP8>(p.table[hh[u]], p.scale[hh[u]], row[u], p.chunks_per_row, cc[u]);
                 } else {
                     atomicOr(&g_engram_status, ENGRAM_STATUS_BAD_ROW);
                 }
@@ -193,12 +238,14 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint32_t *__restrict_
 // still written for the decode-history update).
 struct LookupParams {
     HashParams hash;
-    const uint16_t *table[ENGRAM_MAX_TABLES];
-    int32_t chunks_per_row;  // d_e / 8
+    const void *table[ENGRAM_MAX_TABLES];
+    float scale[ENGRAM_MAX_TABLES];  // FP8 tables only
+    int32_t chunks_per_row;  // d_e / 8 (16-byte chunks of m)
     int32_t warps_per_row;   // each warp copies up to kLookupChunksPerWarp chunks of a row
 };
 constexpr int kLookupChunksPerWarp = 64;
 
+template <bool FP8>
 __global__ void __launch_bounds__(256) lookup_kernel(const int32_t *__restrict__ ids,
                                                      const int32_t *__restrict__ remap,
                                                      const int32_t *__restrict__ history,
@@ -245,14 +292,13 @@ __global__ void __launch_bounds__(256) lookup_kernel(const int32_t *__restrict__
         row = mod_prime(fmix64(s), hp.prime[h], hp.barrett[h]);
     }
     row = __shfl_sync(0xffffffffu, row, 0);
-    const uint4 *src = reinterpret_cast<const uint4 *>(p.table[h]) + static_cast<int64_t>(row) * p.chunks_per_row;
     uint4 *dst = m + (n * hp.H + h) * p.chunks_per_row;
     const int c_end = min(p.chunks_per_row, (part + 1) * kLookupChunksPerWarp);
     uint4 val[kLookupChunksPerWarp / 32];
 #pragma unroll
     for (int k = 0; k < kLookupChunksPerWarp / 32; ++k) {
         const int c = part * kLookupChunksPerWarp + k * 32 + lane;
-        if (c < c_end) val[k] = __ldg(src + c);
+        if (c < c_end) val[k] = load_row_chunk<FP8>(p.table[h], p.scale[h], row, p.chunks_per_row, c);
     }
 #pragma unroll
     for (int k = 0; k < kLookupChunksPerWarp / 32; ++k) {
@@ -348,12 +394,12 @@ __global__ void __launch_bounds__(kDedupThreads) stage_dedup_kernel(const uint32
 }
 
 struct StageParams {
-    const uint16_t *table[ENGRAM_MAX_TABLES];  // host-mapped
-    uint16_t *staging[ENGRAM_MAX_TABLES];      // device, [capacity, d_e]
+    const void *table[ENGRAM_MAX_TABLES];  // host-mapped
+    void *staging[ENGRAM_MAX_TABLES];      // device, [capacity, d_e] of the table's element type
     uint64_t rows[ENGRAM_MAX_TABLES];
-    const uint32_t *unique_rows;               // [H, capacity]
-    const int32_t *n_unique;                   // [H]
-    int32_t H, capacity, chunks_per_row;
+    const uint32_t *unique_rows;           // [H, capacity]
+    const int32_t *n_unique;               // [H]
+    int32_t H, capacity, chunks_per_row;   // 16-byte chunks of a stored row (any element type)
 };
 
 template <int UNROLL>

@@ -66,6 +66,16 @@ enum engram_table_location {
     ENGRAM_TABLES_HOST_MAPPED = 1 /* tables in pinned, mapped host memory */
 };
 
+/* Element type of the n-gram tables.  The pages store bf16 rows; e4m3 rows with one
+ * dequantisation scale per table halve the table bytes (and the bytes a lookup reads).  An
+ * e4m3 value is dequantised into m as the bf16 nearest to decode(code) * table_scale[h]
+ * (ties to even, one rounding of the exact product); decode() is the OCP FP8 E4M3 format
+ * (bias 7, no infinities, codes 0x7F / 0xFF are NaN). */
+enum engram_table_dtype {
+    ENGRAM_TABLE_BF16 = 0,
+    ENGRAM_TABLE_FP8_E4M3 = 1
+};
+
 /* Static description of one lookup layer.  Filled by the caller, checked by engram_init. */
 typedef struct engram_config {
     int32_t num_orders;                   /* |O|, 1..ENGRAM_MAX_ORDERS */
@@ -84,7 +94,11 @@ typedef struct engram_config {
     uint64_t hash_seed;                   /* seeds the per-head hash multipliers */
     float eps;                            /* RMSNorm epsilon (> 0) */
     int32_t flags;                        /* ENGRAM_FLAG_* bits */
-    int32_t reserved[6];                  /* must be zero */
+    int32_t table_dtype;                  /* enum engram_table_dtype */
+    float table_scale[ENGRAM_MAX_TABLES]; /* FP8 tables: dequantisation scale of table h,
+                                             finite and > 0; must be 0 for bf16 tables and
+                                             beyond the H tables */
+    int32_t reserved[5];                  /* must be zero */
 } engram_config;
 
 /* engram_config.flags */
@@ -118,8 +132,9 @@ typedef struct engram_weights {
 } engram_weights;
 
 /* Validate `cfg` and fill `plan` (host only, no CUDA call).  Checks: orders, K, H <= 32,
- * primality of every table_rows[h] (deterministic Miller-Rabin), d_e % 8 == 0,
- * d_h % 64 == 0, pad_id == vocab_out, dilation == largest order, eps > 0, reserved == 0.
+ * primality of every table_rows[h] (deterministic Miller-Rabin), d_e % 8 == 0 (d_e % 16 == 0
+ * for FP8 tables), d_h % 64 == 0, pad_id == vocab_out, dilation == largest order, eps > 0,
+ * table scales, reserved == 0.
  * Derives the hash multipliers: a_{o,j,i} = SplitMix64(seed ^ (o<<16 ^ j<<8 ^ i)) | 1. */
 int engram_init(const engram_config *cfg, engram_plan *plan);
 
@@ -150,11 +165,13 @@ int engram_advance_history(const engram_plan *plan, const int32_t *ids_remapped,
                            int32_t T, int32_t *history, engram_stream_t stream);
 
 /* Step 3 [yktysq #2; zhichai §2.3]: m[n, h*d_e:(h+1)*d_e] = tables[h][idx[n, h], :].
- * tables: HOST array of H pointers, each to bf16 [table_rows[h], d_e] (device memory, or
- * pinned mapped host memory when cfg.table_location == ENGRAM_TABLES_HOST_MAPPED).
- * idx: uint32 [n_tok, H].  m: bf16 [n_tok, d_m].  Bit patterns are copied unchanged.
+ * tables: HOST array of H pointers, each to [table_rows[h], d_e] elements of
+ * cfg.table_dtype (bf16 patterns, or e4m3 codes), in device memory, or in pinned mapped
+ * host memory when cfg.table_location == ENGRAM_TABLES_HOST_MAPPED.
+ * idx: uint32 [n_tok, H].  m: bf16 [n_tok, d_m].  bf16 bit patterns are copied unchanged;
+ * e4m3 codes are dequantised (see engram_table_dtype).
  * A row id >= table_rows[h] yields a zero row and sets ENGRAM_STATUS_BAD_ROW. */
-int engram_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables,
+int engram_gather(const engram_plan *plan, const uint32_t *idx, const void *const *tables,
                   int64_t n_tok, uint16_t *m, engram_stream_t stream);
 
 /* Step 3 with host-resident tables (a7) [zhichai §2.3: the row ids are known as soon as the
@@ -165,7 +182,9 @@ int engram_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *
  *   staging[h][staged_idx[n, h], :] == tables[h][idx[n, h], :]   for every token n.
  * idx: uint32 [n_tok, H] (device).  tables: HOST array of H pointers to pinned, mapped
  * host memory (or device memory) [table_rows[h], d_e].  staging: HOST array of H device
- * pointers, each [capacity, d_e].  staged_idx: uint32 [n_tok, H] (device, out).
+ * pointers, each [capacity, d_e] of the tables' element type (rows are copied as stored:
+ * e4m3 codes stay e4m3 and are dequantised by the gather that reads the staging).
+ * staged_idx: uint32 [n_tok, H] (device, out).
  * unique_rows: uint32 [H, capacity] (device, out): the distinct row ids in increasing order.
  * n_unique: int32 [H] (device, out).  n_tok <= capacity, n_tok <= 8192.
  * The copy is done by a kernel reading the mapped host memory directly (zero-copy), many
@@ -174,14 +193,14 @@ int engram_gather(const engram_plan *plan, const uint32_t *idx, const uint16_t *
  * ENGRAM_TABLES_HOST_MAPPED and B*T <= 8192 (above that it gathers straight from the mapped
  * tables); results are bit-identical to HBM-resident tables. */
 int engram_stage_rows(const engram_plan *plan, const uint32_t *idx, int64_t n_tok,
-                      const uint16_t *const *tables, uint16_t *const *staging, int32_t capacity,
+                      const void *const *tables, void *const *staging, int32_t capacity,
                       uint32_t *staged_idx, uint32_t *unique_rows, int32_t *n_unique,
                       engram_stream_t stream);
 
 /* engram_gather over tables that all hold `rows` rows (e.g. the staging buffers filled by
  * engram_stage_rows, with staged_idx as idx).  Same layout and error behaviour as
  * engram_gather, with `rows` as every table's bound. */
-int engram_gather_bounded(const engram_plan *plan, const uint32_t *idx, const uint16_t *const *tables,
+int engram_gather_bounded(const engram_plan *plan, const uint32_t *idx, const void *const *tables,
                           int64_t n_tok, int64_t rows, uint16_t *m, engram_stream_t stream);
 
 /* Steps 4-6 [yktysq #3, #4; zhichai §2.3]: gate, conv, residual for B sequences of T tokens.
@@ -214,7 +233,7 @@ int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
  * sets kernel attributes), engram_forward / engram_gate_conv may be captured and replayed. */
 #define ENGRAM_FORWARD_STAGES 4 /* hash, gather, projections, gate+conv */
 int engram_forward(const engram_plan *plan, const engram_weights *w,
-                   const uint16_t *const *tables, const int32_t *ids, const int32_t *remap,
+                   const void *const *tables, const int32_t *ids, const int32_t *remap,
                    int32_t B, int32_t T, int32_t *history, uint16_t *conv_state,
                    const uint16_t *h, uint16_t *out, float *delta_dbg, void *workspace,
                    size_t workspace_bytes, engram_stream_t stream, void *const *stage_events);

@@ -78,6 +78,41 @@ uint16_t oracle_double_to_bf16(double x)
 }
 
 /* ------------------------------------------------------------------------------------------
+ * FP8 (e4m3) tables.  The pages store bf16 rows; the e4m3 variant with one dequantisation
+ * scale per table is an extension.  Reading taken: the value gathered into m is the bf16
+ * nearest to decode(code) * scale (ties to even), rounded once from the exact product.
+ * ------------------------------------------------------------------------------------------ */
+
+/* Value of an e4m3 code from the OCP 8-bit floating point (FP8 E4M3) definition: bit 7 sign,
+ * bits 6-3 exponent with bias 7, bits 2-0 mantissa; exponent field 0 encodes the subnormals
+ * m * 2^-9; S.1111.111 is NaN and there are no infinities. */
+double oracle_e4m3_to_double(uint8_t code)
+{
+    const int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* One dequantised element: a 4-bit significand times the 24-bit significand of `scale` is
+ * exact in double, so oracle_double_to_bf16 rounds the true product once.  NaN codes give the
+ * quiet NaN pattern 0x7FC0 (with the code's sign). */
+uint16_t oracle_dequant_e4m3(uint8_t code, float scale)
+{
+    const double v = oracle_e4m3_to_double(code);
+    if (isnan(v)) return (uint16_t)(0x7FC0u | ((code & 0x80u) ? 0x8000u : 0u));
+    return oracle_double_to_bf16(v * (double)scale);
+}
+
+/* A whole e4m3 table (n elements) to bf16 patterns. */
+void oracle_dequant_table(const uint8_t *codes, int64_t n, float scale, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_dequant_e4m3(codes[i], scale);
+}
+
+/* ------------------------------------------------------------------------------------------
  * Hash primitives (reading of the pages: they fix only "deterministic hash", "K independent
  * heads per order" and "prime-sized tables" [yktysq, component 2; zhichai §2.3].  The hash
  * taken here is: multiply-xor of the gram's ids with per-(order, head, position) odd 64-bit
@@ -197,6 +232,18 @@ void oracle_gather(const uint32_t *idx, int64_t n_tok, int32_t H,
             const uint16_t *row = tables[h] + (int64_t)idx[n * H + h] * d_e;
             for (int32_t c = 0; c < d_e; ++c)
                 m[(n * H + h) * d_e + c] = row[c];
+        }
+}
+
+/* Step 3 over e4m3 tables: m[n, h*d_e + c] = dequant(table_h[idx[n, h], c], scale[h]). */
+void oracle_gather_e4m3(const uint32_t *idx, int64_t n_tok, int32_t H, const uint8_t *const *tables,
+                        const float *scale, int32_t d_e, uint16_t *m)
+{
+    for (int64_t n = 0; n < n_tok; ++n)
+        for (int32_t h = 0; h < H; ++h) {
+            const uint8_t *row = tables[h] + (int64_t)idx[n * H + h] * d_e;
+            for (int32_t c = 0; c < d_e; ++c)
+                m[(n * H + h) * d_e + c] = oracle_dequant_e4m3(row[c], scale[h]);
         }
 }
 

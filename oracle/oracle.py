@@ -42,6 +42,14 @@ def lib():
         L.oracle_bf16_to_double.argtypes = [C.c_uint16]
         L.oracle_double_to_bf16.restype = C.c_uint16
         L.oracle_double_to_bf16.argtypes = [dbl]
+        L.oracle_e4m3_to_double.restype = dbl
+        L.oracle_e4m3_to_double.argtypes = [C.c_uint8]
+        L.oracle_dequant_e4m3.restype = C.c_uint16
+        L.oracle_dequant_e4m3.argtypes = [C.c_uint8, C.c_float]
+        L.oracle_dequant_table.restype = None
+        L.oracle_dequant_table.argtypes = [P, i64, C.c_float, P]
+        L.oracle_gather_e4m3.restype = None
+        L.oracle_gather_e4m3.argtypes = [P, i64, i32, P, P, i32, P]
         L.oracle_remap.restype = C.c_int
         L.oracle_remap.argtypes = [P, i64, P, i32, P]
         L.oracle_hash.restype = None
@@ -98,6 +106,22 @@ def double_to_bf16(x: float) -> int:
     return int(lib().oracle_double_to_bf16(float(x)))
 
 
+def e4m3_to_double(code: int) -> float:
+    return float(lib().oracle_e4m3_to_double(code & 0xFF))
+
+
+def dequant_e4m3(code: int, scale) -> int:
+    return int(lib().oracle_dequant_e4m3(code & 0xFF, float(np.float32(scale))))
+
+
+def dequant_table(codes: np.ndarray, scale) -> np.ndarray:
+    """e4m3 codes (any shape, uint8) -> bf16 patterns of the same shape."""
+    codes = _c(codes, np.uint8)
+    out = np.empty(codes.shape, dtype=np.uint16)
+    lib().oracle_dequant_table(_p(codes), codes.size, float(np.float32(scale)), _p(out))
+    return out
+
+
 # ---- steps -------------------------------------------------------------------------------
 def remap(ids: np.ndarray, table: np.ndarray) -> np.ndarray:
     ids = _c(ids, np.int32)
@@ -143,13 +167,22 @@ def _table_ptrs(tables):
     return arrs, ptrs
 
 
-def gather(idx: np.ndarray, tables) -> np.ndarray:
+def gather(idx: np.ndarray, tables, scales=None) -> np.ndarray:
+    """bf16 tables (uint16 patterns); or e4m3 tables (uint8 codes) with one scale per table."""
     idx = _c(idx, np.uint32)
     n_tok, H = idx.shape
-    arrs, ptrs = _table_ptrs(tables)
+    if scales is None:
+        arrs, ptrs = _table_ptrs(tables)
+        d_e = arrs[0].shape[1]
+        m = np.empty((n_tok, H * d_e), dtype=np.uint16)
+        lib().oracle_gather(_p(idx), n_tok, H, ptrs, d_e, _p(m))
+        return m
+    arrs = [_c(t, np.uint8) for t in tables]
+    ptrs = (C.c_void_p * len(arrs))(*[a.ctypes.data for a in arrs])
+    sc = _c([float(x) for x in scales], np.float32)
     d_e = arrs[0].shape[1]
     m = np.empty((n_tok, H * d_e), dtype=np.uint16)
-    lib().oracle_gather(_p(idx), n_tok, H, ptrs, d_e, _p(m))
+    lib().oracle_gather_e4m3(_p(idx), n_tok, H, ptrs, _p(sc), d_e, _p(m))
     return m
 
 
@@ -180,8 +213,12 @@ def gate_conv(h, m, Wk, Wv, gamma_q, gamma_k, gamma_c, conv_w, B: int, T: int,
 
 def forward(ids, remap_table, tables, h, Wk, Wv, gamma_q, gamma_k, gamma_c, conv_w, *,
             orders, K: int, primes, seed: int, pad_id: int, eps: float = 1e-6,
-            history=None, conv_state=None, decode_outputs: bool = False):
-    """All six steps.  Returns dict(out, delta, gate, idx[, state, history])."""
+            history=None, conv_state=None, decode_outputs: bool = False, table_scales=None):
+    """All six steps.  Returns dict(out, delta, gate, idx[, state, history]).
+    table_scales: None for bf16 tables, else one dequantisation scale per e4m3 table (the
+    tables are then uint8 codes, dequantised to bf16 before the lookup)."""
+    if table_scales is not None:
+        tables = [dequant_table(t, s) for t, s in zip(tables, table_scales)]
     ids = _c(ids, np.int32)
     B, T = ids.shape
     remap_table = _c(remap_table, np.int32)

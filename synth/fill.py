@@ -100,3 +100,69 @@ def fill_rows_bf16(spec: FillSpec, ncols: int, rows) -> np.ndarray:
     rows = np.asarray(rows, dtype=np.uint64).reshape(-1)
     e = rows[:, None] * np.uint64(ncols) + np.arange(ncols, dtype=np.uint64)[None, :]
     return _values_at(spec.key, spec.scale, e.reshape(-1)).reshape(rows.size, ncols)
+
+
+# ---------------------------------------------------------------------------------------
+# FP8 (e4m3) tables.  Element e is the Irwin-Hall integer n_e above, encoded as the e4m3
+# value nearest to n_e / 2^13 (ties to even, integer arithmetic only); the table's dequant
+# scale is sigma * 2^13 / sd, so that dequantised values are ~ N(0, sigma^2) again.  The GPU
+# generator in fill_gpu.cu runs the same integer steps.
+FP8_FRAC_BITS = 13
+
+
+def fp8_scale_for_sigma(sigma: float) -> np.float32:
+    return np.float32(sigma * (1 << FP8_FRAC_BITS) / IRWIN_HALL_SD)
+
+
+def encode_e4m3_int(n: np.ndarray) -> np.ndarray:
+    """e4m3 code of n / 2^13 for integers |n| < 2^17 (round to nearest even)."""
+    n = np.asarray(n, dtype=np.int64)
+    a = np.abs(n)
+    sign = (n < 0).astype(np.int64) << 7
+    code = np.zeros_like(a)
+    nz = a > 0
+    msb = np.zeros_like(a)
+    msb[nz] = np.floor(np.log2(a[nz])).astype(np.int64)
+    # guard against log2 rounding at exact powers of two
+    msb = np.where((a >> np.maximum(msb, 0)) >= 2, msb + 1, msb)
+    msb = np.where((a >> np.maximum(msb, 0)) == 0, msb - 1, msb)
+    e = msb - FP8_FRAC_BITS                      # a / 2^13 in [2^e, 2^(e+1))
+    normal = nz & (e >= -6)
+    # normal: keep 4 significant bits
+    sh = np.maximum(msb - 3, 0)
+    q = a >> sh
+    rem = a - (q << sh)
+    half = np.where(sh > 0, 1 << np.maximum(sh - 1, 0), 0)
+    up = (sh > 0) & ((rem > half) | ((rem == half) & ((q & 1) == 1)))
+    q = q + up
+    e_n = np.where(q == 16, e + 1, e)
+    q = np.where(q == 16, 8, q)
+    code_n = ((e_n + 7) << 3) | (q - 8)
+    # subnormal: value / 2^-9 = a / 16
+    qs = a >> 4
+    rs = a & 15
+    ups = (rs > 8) | ((rs == 8) & ((qs & 1) == 1))
+    code_s = qs + ups
+    code = np.where(normal, code_n, np.where(nz, code_s, 0))
+    return (code | np.where(nz, sign, 0)).astype(np.uint8)
+
+
+def _fp8_at(key: int, e: np.ndarray) -> np.ndarray:
+    with np.errstate(over="ignore"):
+        z = np.uint64(key) + e.astype(np.uint64) * GOLDEN + GOLDEN
+        r = _sm_mix(z)
+    mask = np.uint64(0xFFFF)
+    s = (r & mask) + ((r >> np.uint64(16)) & mask) + ((r >> np.uint64(32)) & mask) + (r >> np.uint64(48))
+    return encode_e4m3_int(s.astype(np.int64) - 131070)
+
+
+def fill_fp8(spec: FillSpec, shape) -> np.ndarray:
+    shape = tuple(int(x) for x in shape)
+    n = int(np.prod(shape))
+    return _fp8_at(spec.key, np.arange(n, dtype=np.uint64)).reshape(shape)
+
+
+def fill_rows_fp8(spec: FillSpec, ncols: int, rows) -> np.ndarray:
+    rows = np.asarray(rows, dtype=np.uint64).reshape(-1)
+    e = rows[:, None] * np.uint64(ncols) + np.arange(ncols, dtype=np.uint64)[None, :]
+    return _fp8_at(spec.key, e.reshape(-1)).reshape(rows.size, ncols)

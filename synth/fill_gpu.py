@@ -32,6 +32,8 @@ def _get():
         L = C.CDLL(_LIB)
         L.synth_fill_bf16.restype = C.c_int
         L.synth_fill_bf16.argtypes = [C.c_void_p, C.c_uint64, C.c_uint64, C.c_uint64, C.c_float, C.c_void_p]
+        L.synth_fill_fp8.restype = C.c_int
+        L.synth_fill_fp8.argtypes = [C.c_void_p, C.c_uint64, C.c_uint64, C.c_uint64, C.c_void_p]
         L.synth_host_alloc_mapped.restype = C.c_int
         L.synth_host_alloc_mapped.argtypes = [C.c_uint64, C.POINTER(C.c_void_p)]
         L.synth_host_free.restype = C.c_int
@@ -52,6 +54,22 @@ def fill_(t: torch.Tensor, spec: FillSpec, offset: int = 0, stream=None) -> torc
     return t
 
 
+def fill_fp8_(t: torch.Tensor, spec: FillSpec, stream=None) -> torch.Tensor:
+    """Fill a contiguous uint8 tensor (device or pinned-mapped) with e4m3 codes."""
+    assert t.is_contiguous() and t.element_size() == 1
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    rc = _get().synth_fill_fp8(C.c_void_p(t.data_ptr()), t.numel(), 0, spec.key, C.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise RuntimeError(f"synth_fill_fp8 failed with CUDA error {rc}")
+    return t
+
+
+def filled_fp8(shape, spec: FillSpec, device="cuda") -> torch.Tensor:
+    t = torch.empty(shape, dtype=torch.uint8, device=device)
+    return fill_fp8_(t, spec)
+
+
 def filled(shape, spec: FillSpec, device="cuda") -> torch.Tensor:
     t = torch.empty(shape, dtype=torch.bfloat16, device=device)
     return fill_(t, spec)
@@ -61,15 +79,19 @@ class HostMapped:
     """A pinned, device-mapped host buffer viewed as a CPU torch tensor of bf16 [rows, cols].
     Its data_ptr() is valid on the device too (unified addressing).  Freed by close()."""
 
-    def __init__(self, rows: int, cols: int):
+    def __init__(self, rows: int, cols: int, elem_bytes: int = 2):
         self.ptr = C.c_void_p()
-        nbytes = int(rows) * int(cols) * 2
+        nbytes = int(rows) * int(cols) * elem_bytes
         rc = _get().synth_host_alloc_mapped(nbytes, C.byref(self.ptr))
         if rc != 0 or not self.ptr.value:
             raise MemoryError(f"cudaHostAlloc({nbytes} bytes, mapped) failed with CUDA error {rc}")
         import numpy as np
-        arr = np.ctypeslib.as_array((C.c_int16 * (int(rows) * int(cols))).from_address(self.ptr.value))
-        self.tensor = torch.from_numpy(arr).view(torch.bfloat16).view(int(rows), int(cols))
+        if elem_bytes == 2:
+            arr = np.ctypeslib.as_array((C.c_int16 * (int(rows) * int(cols))).from_address(self.ptr.value))
+            self.tensor = torch.from_numpy(arr).view(torch.bfloat16).view(int(rows), int(cols))
+        else:
+            arr = np.ctypeslib.as_array((C.c_uint8 * (int(rows) * int(cols))).from_address(self.ptr.value))
+            self.tensor = torch.from_numpy(arr).view(int(rows), int(cols))
 
     def close(self):
         if self.ptr is not None and self.ptr.value:

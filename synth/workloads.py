@@ -12,7 +12,7 @@ from typing import Optional, Tuple
 
 import numpy as np
 
-from .fill import FillSpec
+from .fill import FillSpec, fp8_scale_for_sigma
 from .streams import zipf_ids, uniform_ids, remap_table, phrase_stream
 
 
@@ -66,6 +66,7 @@ class Workload:
     sigma_h: float = 1.0
     sigma_conv: float = 0.25
     index: int = 0
+    table_dtype: str = "bf16"  # bf16 | fp8 (e4m3 codes with one dequantisation scale per table)
 
     @property
     def H(self) -> int:
@@ -96,8 +97,12 @@ class Workload:
         return self.vocab_out
 
     @property
+    def table_elem_bytes(self) -> int:
+        return 1 if self.table_dtype == "fp8" else 2
+
+    @property
     def table_bytes(self) -> int:
-        return sum(self.primes) * self.d_e * 2
+        return sum(self.primes) * self.d_e * self.table_elem_bytes
 
     def seeds(self):
         c = self.index
@@ -106,6 +111,15 @@ class Workload:
     # ---- fill specs -------------------------------------------------------------------
     def table_spec(self, h: int) -> FillSpec:
         return FillSpec(self.seeds()["tables"], h, self.sigma_table)
+
+    def table_sigma(self, h: int) -> float:
+        """FP8 tables: table h is dequantised to ~N(0, sigma_h^2), sigma_h growing with h so that
+        every table has its own scale."""
+        return self.sigma_table * (1.0 + 0.125 * h)
+
+    def table_scale(self, h: int):
+        """Dequantisation scale of FP8 table h (float32)."""
+        return fp8_scale_for_sigma(self.table_sigma(h))
 
     def wk_spec(self) -> FillSpec:
         return FillSpec(self.seeds()["weights"], T_WK, self.sigma_w)

@@ -30,6 +30,25 @@ def to_host_u16(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+def host_tables(wl: synth.Workload):
+    """The workload's tables regenerated on the host: bf16 patterns, or e4m3 codes."""
+    fill = synth.fill_fp8 if wl.table_dtype == "fp8" else synth.fill_bf16
+    return [fill(wl.table_spec(h), (wl.primes[h], wl.d_e)) for h in range(wl.H)]
+
+
+def host_rows(wl: synth.Workload, h: int, rows) -> np.ndarray:
+    """Rows of table h as the gather must deliver them (bf16 patterns; e4m3 tables are
+    dequantised by the oracle)."""
+    if wl.table_dtype == "fp8":
+        import oracle
+        return oracle.dequant_table(synth.fill_rows_fp8(wl.table_spec(h), wl.d_e, rows), wl.table_scale(h))
+    return synth.fill_rows_bf16(wl.table_spec(h), wl.d_e, rows)
+
+
+def table_scales(wl: synth.Workload):
+    return [wl.table_scale(h) for h in range(wl.H)] if wl.table_dtype == "fp8" else None
+
+
 class DeviceInputs:
     """All tensors of one workload on the device; tables filled on the GPU."""
 
@@ -42,7 +61,8 @@ class DeviceInputs:
         self.ids = to_dev(self.ids_np, device)
         self.remap = to_dev(self.remap_np, device)
         if tables is None:
-            tables = [fill_gpu.filled((wl.primes[h], wl.d_e), wl.table_spec(h), device) for h in range(wl.H)]
+            fill = fill_gpu.filled_fp8 if wl.table_dtype == "fp8" else fill_gpu.filled
+            tables = [fill((wl.primes[h], wl.d_e), wl.table_spec(h), device) for h in range(wl.H)]
         self.tables = tables
         self.h = fill_gpu.filled((wl.n_tok, wl.d_h), wl.h_spec(step), device)
         self.w_k = fill_gpu.filled((wl.d_h, wl.d_m), wl.wk_spec(), device)

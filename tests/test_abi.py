@@ -54,6 +54,13 @@ def _plan(**kw):
     (dict(conv_kernel=9), E.ENGRAM_ERR_UNSUPPORTED),
     (dict(heads_per_order=17), E.ENGRAM_ERR_UNSUPPORTED),
     (dict(flags=0x2), E.ENGRAM_ERR_INVALID_ARG),                                # unknown flag bit
+    (dict(table_dtype=2), E.ENGRAM_ERR_INVALID_ARG),                            # unknown table dtype
+    (dict(table_dtype=1, table_scale=(0.1, 0.1, 0.1, 0.0)), E.ENGRAM_ERR_INVALID_ARG),   # zero scale
+    (dict(table_dtype=1, table_scale=(0.1, float("inf"), 0.1, 0.1)), E.ENGRAM_ERR_INVALID_ARG),
+    (dict(table_dtype=1, table_scale=(0.1, 0.1, 0.1, -0.1)), E.ENGRAM_ERR_INVALID_ARG),
+    (dict(table_dtype=1, table_scale=(0.1,) * 5), E.ENGRAM_ERR_INVALID_ARG),   # scale beyond H
+    (dict(table_dtype=0, table_scale=(0.1,)), E.ENGRAM_ERR_INVALID_ARG),       # scale on bf16
+    (dict(table_dtype=1, table_scale=(0.1,) * 4, row_dim=24), E.ENGRAM_ERR_UNSUPPORTED),
 ])
 def test_init_rejects_bad_configs(kw, code):
     with pytest.raises(E.EngramError) as ei:
@@ -67,6 +74,14 @@ def test_init_accepts_every_workload_and_derives_constants():
         assert p.num_tables == wl.H and p.mem_dim == wl.d_m
         assert p.hist_len == max(wl.orders) - 1 and p.state_len == 3 * max(wl.orders)
         assert E.engram_workspace_size(p, wl.n_tok) > 0
+        pf = E.Plan.from_workload(wl.with_(table_dtype="fp8"))
+        assert pf.cfg.table_dtype == E.ENGRAM_TABLE_FP8_E4M3
+        assert [pf.plan.cfg.table_scale[h] for h in range(wl.H)] == [float(wl.table_scale(h)) for h in range(wl.H)]
+        # host-mapped FP8 tables stage half the bytes of bf16 ones
+        hb = E.engram_workspace_size(E.Plan.from_workload(wl, host_tables=True), min(wl.n_tok, 4096))
+        hf = E.engram_workspace_size(E.Plan.from_workload(wl.with_(table_dtype="fp8"), host_tables=True),
+                                     min(wl.n_tok, 4096))
+        assert hf < hb
     p = _plan()
     assert E.engram_workspace_size(p, 1000) < E.engram_workspace_size(p, 2000)
     assert E.engram_workspace_size(p, 0) >= 0

@@ -13,7 +13,8 @@ import torch
 import hashed_gram_embedding_remap_b200 as E
 import oracle
 import synth
-from gpu_helpers import DeviceInputs, assert_delta_close, assert_out_close, to_dev, to_host_u16
+from gpu_helpers import (DeviceInputs, assert_delta_close, assert_out_close, host_tables, table_scales,
+                         to_dev, to_host_u16)
 from helpers import small_workload
 from synth import fill_gpu
 
@@ -130,11 +131,11 @@ def test_bad_ids_and_rows_raise_status_not_faults():
 # ------------------------------------------------------------------ steps 1-6
 def _oracle_full(wl, di):
     w = di.host_weights()
-    tables = [synth.fill_bf16(wl.table_spec(h), (wl.primes[h], wl.d_e)) for h in range(wl.H)]
+    tables = host_tables(wl)
     h = synth.fill_bf16(wl.h_spec(0), (wl.n_tok, wl.d_h))
-    kw = {}
+    kw = dict(table_scales=table_scales(wl))
     if wl.decode:
-        kw = dict(history=wl.history(), conv_state=to_host_u16(di.conv_state), decode_outputs=True)
+        kw.update(history=wl.history(), conv_state=to_host_u16(di.conv_state), decode_outputs=True)
     return oracle.forward(di.ids_np, di.remap_np, tables, h, w["Wk"], w["Wv"], w["gamma_q"],
                           w["gamma_k"], w["gamma_c"], w["conv_w"], orders=wl.orders, K=wl.K,
                           primes=wl.primes, seed=wl.hash_seed, pad_id=wl.pad_id, eps=wl.eps, **kw)

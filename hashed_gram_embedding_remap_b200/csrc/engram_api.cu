@@ -409,13 +409,31 @@ int launch_gather(const engram_plan *plan, const uint32_t *idx, const void *cons
     p.chunks_per_tok = H * p.chunks_per_row;
     p.n_tok = n_tok;
     const int64_t total = n_tok * p.chunks_per_tok;
-    constexpr int kUnroll = 4;
+    // independent chunks per thread: ENGRAM_GATHER_UNROLL (4 or 8) overrides, for tuning
+    static const int forced_unroll = [] {
+        const char *e = std::getenv("ENGRAM_GATHER_UNROLL");
+        const int v = e ? std::atoi(e) : 0;
+        return (v == 4 || v == 8) ? v : 0;
+    }();
+    const int unroll = forced_unroll ? forced_unroll : 4;
     const int threads = 256;
-    int64_t blocks = (total + threads * kUnroll - 1) / (threads * kUnroll);
+    int64_t blocks = (total + threads * unroll - 1) / (threads * unroll);
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;  // 8 x 256 threads resident per SM
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    auto kern = fp8_tables(plan) ? engram::gather_kernel<kUnroll, true> : engram::gather_kernel<kUnroll, false>;
+    p.div_row = engram::make_fastdiv(static_cast<uint32_t>(p.chunks_per_row));
+    p.div_tok = engram::make_fastdiv(static_cast<uint32_t>(p.chunks_per_tok));
+    const bool f8 = fp8_tables(plan);
+    // 32-bit chunk indices when the last index plus one grid stride per unrolled chunk fits
+    const bool idx32 = total + blocks * threads * (unroll + 1) < (int64_t(1) << 32);
+    using K = void (*)(const uint32_t *, uint4 *, const engram::GatherParams);
+    K kern;
+    if (idx32)
+        kern = unroll == 8 ? (f8 ? engram::gather_kernel<8, true, uint32_t> : engram::gather_kernel<8, false, uint32_t>)
+                           : (f8 ? engram::gather_kernel<4, true, uint32_t> : engram::gather_kernel<4, false, uint32_t>);
+    else
+        kern = unroll == 8 ? (f8 ? engram::gather_kernel<8, true, int64_t> : engram::gather_kernel<8, false, int64_t>)
+                           : (f8 ? engram::gather_kernel<4, true, int64_t> : engram::gather_kernel<4, false, int64_t>);
     kern<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(idx, reinterpret_cast<uint4 *>(m), p);
     ENGRAM_CUDA_TRY(cudaGetLastError(), "gather_kernel launch");
     return ENGRAM_OK;
@@ -736,8 +754,9 @@ int engram_init(const engram_config *cfg, engram_plan *plan) {
     for (int h = 0; h < ENGRAM_MAX_TABLES; ++h) {
         const float sc = c.table_scale[h];
         if (c.table_dtype == ENGRAM_TABLE_FP8_E4M3 && h < H) {
-            if (!(sc > 0.f) || !std::isfinite(sc))
-                return fail(ENGRAM_ERR_INVALID_ARG, "table_scale[%d] must be a positive finite number", h);
+            // products of codes (2^-9 .. 448) and scales in this range stay normal fp32 values
+            if (!(sc >= 0x1p-100f && sc <= 0x1p100f))
+                return fail(ENGRAM_ERR_INVALID_ARG, "table_scale[%d] must lie in [2^-100, 2^100]", h);
         } else if (sc != 0.f) {
             return fail(ENGRAM_ERR_INVALID_ARG, "table_scale[%d] must be 0 (bf16 tables or beyond the %d tables)", h, H);
         }

@@ -132,32 +132,57 @@ __global__ void advance_history_kernel(const int32_t *__restrict__ xr, int32_t B
 // ---------------------------------------------------------------- FP8 (e4m3) tables
 // A table may hold e4m3 codes with one dequantisation scale per table; the gathered value is
 // the bf16 nearest to decode(code) * scale_h (ties to even), rounded once from the exact
-// product.  decode() is exact in fp16 (cvt.rn.f16x2.e4m3x2) and in fp32; the fp32 product
-// a*s is rounded, but fma(a, s, -a*s) recovers its error exactly, and a double rounding
-// (fp32, then bf16) can only go wrong when the fp32 product sits exactly on a bf16 midpoint,
-// where the sign of that error decides.
+// product.  decode() is exact in fp16 (cvt.rn.f16x2.e4m3x2) and in fp32.  The product is
+// first rounded to odd at fp32 precision: truncated toward zero (mul.rz), with its last bit
+// set when the truncation was inexact (fma recovers the exact remainder).  Rounding a
+// round-to-odd value with p >= q + 2 bits to q bits is the correctly rounded q-bit result,
+// so one hardware RNE conversion to bf16 (24 >= 8 + 2) finishes it.  Scales are limited to
+// [2^-100, 2^100] on the host, so every product of a finite code is a normal fp32 value.
 
-// bf16 pattern of the correctly rounded product a * s (finite a, s; no underflow).
-__device__ __forceinline__ uint32_t bf16_of_product(float a, float s) {
-    const float hi = __fmul_rn(a, s);
-    const float lo = __fmaf_rn(a, s, -hi);
-    const uint32_t u = __float_as_uint(hi);
-    if ((u & 0xFFFFu) == 0x8000u && lo != 0.0f) return (lo > 0.0f) == (hi > 0.0f) ? (u >> 16) + 1u : (u >> 16);
-    if ((u & 0x7F800000u) == 0x7F800000u) return (u >> 16) | ((u & 0xFFFFu) ? 0x40u : 0u);  // inf / NaN
-    return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+// Round-to-odd fp32 pattern of a * s.
+__device__ __forceinline__ float product_round_to_odd(float a, float s) {
+    const float t = __fmul_rz(a, s);
+    const float r = __fmaf_rn(a, s, -t);
+    return __uint_as_float(__float_as_uint(t) | (r != 0.0f ? 1u : 0u));
 }
 
 // Two e4m3 codes (low byte = first element) -> two dequantised bf16 packed in 32 bits.
 __device__ __forceinline__ uint32_t dequant_e4m3x2(uint32_t two_codes, float scale) {
     const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes), __NV_E4M3);
     const float2 f = __half22float2(__half2(hr));
-    return bf16_of_product(f.x, scale) | (bf16_of_product(f.y, scale) << 16);
+    const __nv_bfloat162 b =
+        __floats2bfloat162_rn(product_round_to_odd(f.x, scale), product_round_to_odd(f.y, scale));
+    return *reinterpret_cast<const uint32_t *>(&b);
 }
 
 // Eight codes (8 bytes) -> eight bf16 (16 bytes).
 __device__ __forceinline__ uint4 dequant_e4m3x8(uint2 w, float scale) {
     return make_uint4(dequant_e4m3x2(w.x & 0xFFFFu, scale), dequant_e4m3x2(w.x >> 16, scale),
                       dequant_e4m3x2(w.y & 0xFFFFu, scale), dequant_e4m3x2(w.y >> 16, scale));
+}
+
+// Unsigned 32-bit division by a divisor fixed for a launch (Granlund and Montgomery,
+// "Division by Invariant Integers using Multiplication", PLDI 1994, the unsigned method of
+// section 4): with l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1,
+// n / d = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0), where t = mulhi(m, n).
+struct FastDivU32 {
+    uint32_t d, m, s1, s2;
+};
+
+inline FastDivU32 make_fastdiv(uint32_t d) {
+    uint32_t l = 0;
+    while (l < 32 && (1ull << l) < d) ++l;
+    FastDivU32 f;
+    f.d = d;
+    f.m = static_cast<uint32_t>(((1ull << 32) * ((1ull << l) - d)) / d + 1);
+    f.s1 = l < 1 ? l : 1;
+    f.s2 = l > 1 ? l - 1 : 0;
+    return f;
+}
+
+__device__ __forceinline__ uint32_t fastdiv(uint32_t n, const FastDivU32 &f) {
+    const uint32_t t = __umulhi(f.m, n);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
 }
 
 struct GatherParams {
@@ -168,56 +193,77 @@ struct GatherParams {
     int32_t chunks_per_row;  // d_e / 8  (16-byte chunks of m)
     int32_t chunks_per_tok;  // H * d_e / 8
     int64_t n_tok;
+    FastDivU32 div_row, div_tok;  // by chunks_per_row, chunks_per_tok (32-bit index launches)
 };
 
-// One 16-byte chunk of m (8 values) from chunk c of row `row` of table h: 16 bytes of a bf16
-// table, or 8 bytes of an e4m3 table dequantised on the fly.
+// The stored bytes behind one 16-byte chunk of m (8 values): 16 bytes of a bf16 row, or 8
+// bytes of an e4m3 row.  Loads and conversions are kept apart (all of a thread's loads are
+// issued before the first conversion), so that the conversions do not serialise the loads.
+template <bool FP8> struct RowChunk { using type = uint4; };
+template <> struct RowChunk<true> { using type = uint2; };
+
 template <bool FP8>
-__device__ __forceinline__ uint4 load_row_chunk(const void *table, float scale, uint32_t row, int32_t chunks_per_row,
-                                                int32_t c) {
+__device__ __forceinline__ typename RowChunk<FP8>::type load_row_chunk(const void *table, uint32_t row,
+                                                                       int32_t chunks_per_row, int32_t c) {
     const int64_t off = static_cast<int64_t>(row) * chunks_per_row + c;
-    if constexpr (FP8) {
-        return dequant_e4m3x8(__ldg(reinterpret_cast<const uint2 *>(table) + off), scale);
-    } else {
-        return __ldg(reinterpret_cast<const uint4 *>(table) + off);
-    }
+    return __ldg(reinterpret_cast<const typename RowChunk<FP8>::type *>(table) + off);
+}
+
+__device__ __forceinline__ uint4 chunk_to_m(uint4 raw, float) { return raw; }
+__device__ __forceinline__ uint4 chunk_to_m(uint2 raw, float scale) { return dequant_e4m3x8(raw, scale); }
+
+template <bool FP8>
+__device__ __forceinline__ typename RowChunk<FP8>::type zero_chunk() {
+    typename RowChunk<FP8>::type z;
+    memset(&z, 0, sizeof z);
+    return z;
 }
 
 // m[n, h*d_e + c] = table_h[idx[n, h], c], copied as 16-byte chunks of m.  Consecutive
 // threads take consecutive chunks of m, so stores are fully coalesced and each table row is
 // read as contiguous pieces.  Each thread keeps UNROLL independent chunks in flight.
-template <int UNROLL, bool FP8>
+// Idx = uint32_t when every chunk index of the launch (plus one grid stride) fits in 32 bits:
+// the chunk -> (token, table, column) split then runs on multiply-high divisions.
+template <int UNROLL, bool FP8, typename Idx>
 __global__ void __launch_bounds__(256) gather_kernel(const uint32_t *__restrict__ idx, uint4 *__restrict__ m,
                                                      const __grid_constant__ GatherParams p) {
-    const int64_t total = p.n_tok * p.chunks_per_tok;
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < total;
-         base += stride * UNROLL) {
+    const Idx total = static_cast<Idx>(p.n_tok * p.chunks_per_tok);
+    const Idx stride = static_cast<Idx>(gridDim.x) * blockDim.x;
+    for (Idx base = static_cast<Idx>(blockIdx.x) * blockDim.x + threadIdx.x; base < total; base += stride * UNROLL) {
         uint32_t row[UNROLL];
         int32_t hh[UNROLL], cc[UNROLL];
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
-            const int64_t i = base + u * stride;
+            const Idx i = base + u * stride;
             row[u] = 0xFFFFFFFFu;
             hh[u] = 0;
             cc[u] = 0;
             if (i < total) {
-                const int64_t n = i / p.chunks_per_tok;
-                const int32_t r = static_cast<int32_t>(i - n * p.chunks_per_tok);
-                const int32_t h = r / p.chunks_per_row;
+                int64_t n;
+                int32_t r, h;
+                if constexpr (sizeof(Idx) == 4) {
+                    const uint32_t n32 = fastdiv(i, p.div_tok);
+                    r = static_cast<int32_t>(i - n32 * p.div_tok.d);
+                    h = static_cast<int32_t>(fastdiv(static_cast<uint32_t>(r), p.div_row));
+                    n = n32;
+                } else {
+                    n = i / p.chunks_per_tok;
+                    r = static_cast<int32_t>(i - n * p.chunks_per_tok);
+                    h = r / p.chunks_per_row;
+                }
                 hh[u] = h;
                 cc[u] = r - h * p.chunks_per_row;
                 row[u] = __ldg(idx + n * p.H + h);
             }
         }
-        uint4 val[UNROLL];
+        typename RowChunk<FP8>::type val[UNROLL];
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
-            const int64_t i = base + u * stride;
-            val[u] = make_uint4(0, 0, 0, 0);
+            const Idx i = base + u * stride;
+            val[u] = zero_chunk<FP8>();
             if (i < total) {
                 if (row[u] < p.rows[hh[u]]) {
-                    val[u] = load_row_chunk<FP8>(p.table[hh[u]], p.scale[hh[u]], row[u], p.chunks_per_row, cc[u]);
+                    val[u] = load_row_chunk<FP8>(p.table[hh[u]], row[u], p.chunks_per_row, cc[u]);
                 } else {
                     atomicOr(&g_engram_status, ENGRAM_STATUS_BAD_ROW);
                 }
@@ -225,8 +271,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint32_t *__restrict_
         }
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
-            const int64_t i = base + u * stride;
-            if (i < total) m[i] = val[u];
+            const Idx i = base + u * stride;
+            if (i < total) m[i] = chunk_to_m(val[u], p.scale[hh[u]]);
         }
     }
 }
@@ -294,16 +340,17 @@ __global__ void __launch_bounds__(256) lookup_kernel(const int32_t *__restrict__
     row = __shfl_sync(0xffffffffu, row, 0);
     uint4 *dst = m + (n * hp.H + h) * p.chunks_per_row;
     const int c_end = min(p.chunks_per_row, (part + 1) * kLookupChunksPerWarp);
-    uint4 val[kLookupChunksPerWarp / 32];
+    typename RowChunk<FP8>::type val[kLookupChunksPerWarp / 32];
 #pragma unroll
     for (int k = 0; k < kLookupChunksPerWarp / 32; ++k) {
         const int c = part * kLookupChunksPerWarp + k * 32 + lane;
-        if (c < c_end) val[k] = load_row_chunk<FP8>(p.table[h], p.scale[h], row, p.chunks_per_row, c);
+        if (c < c_end) val[k] = load_row_chunk<FP8>(p.table[h], row, p.chunks_per_row, c);
     }
+    const float scale = p.scale[h];
 #pragma unroll
     for (int k = 0; k < kLookupChunksPerWarp / 32; ++k) {
         const int c = part * kLookupChunksPerWarp + k * 32 + lane;
-        if (c < c_end) dst[c] = val[k];
+        if (c < c_end) dst[c] = chunk_to_m(val[k], scale);
     }
 }
 

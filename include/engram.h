@@ -96,8 +96,8 @@ typedef struct engram_config {
     int32_t flags;                        /* ENGRAM_FLAG_* bits */
     int32_t table_dtype;                  /* enum engram_table_dtype */
     float table_scale[ENGRAM_MAX_TABLES]; /* FP8 tables: dequantisation scale of table h,
-                                             finite and > 0; must be 0 for bf16 tables and
-                                             beyond the H tables */
+                                             in [2^-100, 2^100]; must be 0 for bf16 tables
+                                             and beyond the H tables */
     int32_t reserved[5];                  /* must be zero */
 } engram_config;
 

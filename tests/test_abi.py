@@ -59,6 +59,8 @@ def _plan(**kw):
     (dict(table_dtype=1, table_scale=(0.1, float("inf"), 0.1, 0.1)), E.ENGRAM_ERR_INVALID_ARG),
     (dict(table_dtype=1, table_scale=(0.1, 0.1, 0.1, -0.1)), E.ENGRAM_ERR_INVALID_ARG),
     (dict(table_dtype=1, table_scale=(0.1,) * 5), E.ENGRAM_ERR_INVALID_ARG),   # scale beyond H
+    (dict(table_dtype=1, table_scale=(0.1, 2.0 ** -101, 0.1, 0.1)), E.ENGRAM_ERR_INVALID_ARG),  # products
+    (dict(table_dtype=1, table_scale=(0.1, 2.0 ** 101, 0.1, 0.1)), E.ENGRAM_ERR_INVALID_ARG),   # leave fp32
     (dict(table_dtype=0, table_scale=(0.1,)), E.ENGRAM_ERR_INVALID_ARG),       # scale on bf16
     (dict(table_dtype=1, table_scale=(0.1,) * 4, row_dim=24), E.ENGRAM_ERR_UNSUPPORTED),
 ])

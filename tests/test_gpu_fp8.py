@@ -46,16 +46,19 @@ def test_gpu_fp8_fill_matches_cpu_codes():
 
 
 def _midpoint_scales(count: int, seed: int = 5):
-    """Scales for which some code's binary32 product lands on a bf16 midpoint while the exact
-    product does not (the case where a plain fp32 multiply + round would be one ulp off)."""
+    """Scales for which some code's binary32 product -- rounded to nearest, or truncated --
+    lands exactly on a bf16 midpoint while the exact product does not: the cases where a
+    plain fp32 multiply then round, or a truncation without its sticky bit, is one ulp off."""
     rng = np.random.default_rng(seed)
     v = np.array([oracle.e4m3_to_double(c) for c in range(1, 0x7F)])
     out = []
     while len(out) < count:
         s = rng.uniform(0.001, 0.05, 20000).astype(np.float32)
-        prod = v[:, None] * s.astype(np.float64)[None, :]
-        p32 = prod.astype(np.float32)
-        hit = ((p32.view(np.uint32) & 0xFFFF) == 0x8000) & (p32.astype(np.float64) != prod)
+        prod = v[:, None] * s.astype(np.float64)[None, :]        # exact
+        rn = prod.astype(np.float32)
+        rz = np.where(np.abs(rn.astype(np.float64)) > np.abs(prod), np.nextafter(rn, np.float32(0)), rn)
+        inexact = rn.astype(np.float64) != prod
+        hit = inexact & (((rn.view(np.uint32) & 0xFFFF) == 0x8000) | ((rz.view(np.uint32) & 0xFFFF) == 0x8000))
         cols = np.unique(np.nonzero(hit)[1])
         out.extend(float(s[c]) for c in cols[: count - len(out)])
     return out

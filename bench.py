@@ -193,8 +193,10 @@ def oracle_sample(wl, n_tok_sample: int, seq: int = 0):
         tables = [synth.fill_rows_bf16(wl.table_spec(h), wl.d_e, idx_probe[:, h]) for h in range(wl.H)]
         scales = None
     local_idx = np.tile(np.arange(T, dtype=np.uint32)[:, None], (1, wl.H))
-    h = synth.fill_rows_bf16(wl.h_spec(0), wl.d_h, b * wl.T + np.arange(T))
-    Wk = synth.fill_bf16(wl.wk_spec(), (wl.d_h, wl.d_m))
+    M = wl.branches
+    hrows = ((b * wl.T + np.arange(T))[:, None] * M + np.arange(M)[None, :]).reshape(-1)
+    h = synth.fill_rows_bf16(wl.h_spec(0), wl.d_h, hrows).reshape(T, M, wl.d_h)
+    Wk = synth.fill_bf16(wl.wk_spec(), (M * wl.d_h, wl.d_m))
     Wv = synth.fill_bf16(wl.wv_spec(), (wl.d_h, wl.d_m))
     one = np.full(wl.d_h, 0x3F80, dtype=np.uint16)
     cw = synth.fill_bf16(wl.conv_spec(), (wl.d_h, wl.conv_kernel))
@@ -203,7 +205,9 @@ def oracle_sample(wl, n_tok_sample: int, seq: int = 0):
     xr = oracle.remap(ids, remap)
     idx = oracle.hash_ids(xr, wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id)
     m = oracle.gather(local_idx, tables, scales)   # compact tables hold exactly the rows idx names
-    oracle.gate_conv(h, m, Wk, Wv, one, one, one, cw, 1, T, dil=wl.conv_dilation, eps=wl.eps)
+    for br in range(M):      # the branches share m and W_v; each has its own h row and W_k
+        oracle.gate_conv(h[:, br], m, Wk[br * wl.d_h:(br + 1) * wl.d_h], Wv, one, one, one, cw, 1, T,
+                         dil=wl.conv_dilation, eps=wl.eps)
     dt = time.perf_counter() - t0
     assert np.array_equal(idx, idx_probe)
     return T, dt, t_gen
@@ -243,7 +247,7 @@ def run_reference(args, wl, world, rank):
 def workload_config(wl, world):
     return {"workload": wl.name, "tokens_per_step_per_gpu": wl.n_tok, "B": wl.B, "T": wl.T,
             "orders": list(wl.orders), "K": wl.K, "H": wl.H, "table_rows": wl.primes[0], "d_e": wl.d_e,
-            "d_m": wl.d_m, "d_h": wl.d_h, "table_dtype": wl.table_dtype,
+            "d_m": wl.d_m, "d_h": wl.d_h, "branches": wl.branches, "table_dtype": wl.table_dtype,
             "table_GiB": round(wl.table_bytes / 2 ** 30, 2),
             "parallelism": f"replicas x{world}",
             "l2": "inputs larger than L2 (hidden states, memory vectors and tables each exceed 126 MB)"
@@ -260,7 +264,8 @@ def run_engram(args, wl, world, rank, local):
     fill_gpu.build()
     stream = torch.cuda.current_stream()
     free, _ = torch.cuda.mem_get_info()
-    need = wl.table_bytes + 4 * wl.n_tok * (wl.d_h * 8 + wl.d_m * 2)
+    M = wl.branches
+    need = wl.table_bytes + 4 * wl.n_tok * (wl.d_h * 8 * M + wl.d_m * 2)
     if need > free:
         raise SystemExit(f"not enough device memory: need ~{need / 2**30:.1f} GiB, free {free / 2**30:.1f} GiB")
     # per-rank input: each rank draws its own batch (seed offset by rank)
@@ -269,16 +274,16 @@ def run_engram(args, wl, world, rank, local):
     ids_np = wl.ids(step=rank)
     ids = torch.from_numpy(ids_np).to(dev)
     remap = None if wl.identity_remap else torch.from_numpy(wl.remap()).to(dev)
-    h = fill_gpu.filled((wl.n_tok, wl.d_h), wl.h_spec(rank), dev)
-    wk = fill_gpu.filled((wl.d_h, wl.d_m), wl.wk_spec(), dev)
+    h = fill_gpu.filled((wl.h_rows, wl.d_h), wl.h_spec(rank), dev)       # [n_tok * M, d_h]
+    wk = fill_gpu.filled((M * wl.d_h, wl.d_m), wl.wk_spec(), dev)
     wv = fill_gpu.filled((wl.d_h, wl.d_m), wl.wv_spec(), dev)
     one = torch.full((wl.d_h,), 0x3F80, dtype=torch.int16, device=dev).view(torch.bfloat16)
     cw = fill_gpu.filled((wl.d_h, wl.conv_kernel), wl.conv_spec(), dev)
     history = torch.from_numpy(wl.history()).to(dev) if wl.decode else None
-    state = fill_gpu.filled((wl.B, wl.state_len, wl.d_h), wl.state_spec(), dev) if wl.decode else None
+    state = fill_gpu.filled((wl.B * M, wl.state_len, wl.d_h), wl.state_spec(), dev) if wl.decode else None
     plan = E.Plan.from_workload(wl)
     weights = E.Weights(wk, wv, one, one, one, cw)
-    out = torch.empty((wl.n_tok, wl.d_h), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((wl.h_rows, wl.d_h), dtype=torch.bfloat16, device=dev)
     ws = E.alloc_workspace(plan, wl.n_tok, dev)
     nstage = E.ENGRAM_FORWARD_STAGES + 1
 
@@ -353,9 +358,9 @@ def run_engram(args, wl, world, rank, local):
     if not args.no_e2e:
         nbuf = 2
         ids_host = torch.from_numpy(ids_np).pin_memory()
-        h_host = torch.empty((wl.n_tok, wl.d_h), dtype=torch.bfloat16).pin_memory()
+        h_host = torch.empty((wl.h_rows, wl.d_h), dtype=torch.bfloat16).pin_memory()
         h_host.copy_(h.cpu())
-        out_host = torch.empty((wl.n_tok, wl.d_h), dtype=torch.bfloat16).pin_memory()
+        out_host = torch.empty((wl.h_rows, wl.d_h), dtype=torch.bfloat16).pin_memory()
         ids_d = [torch.empty_like(ids) for _ in range(nbuf)]
         h_d = [torch.empty_like(h) for _ in range(nbuf)]
         out_d = [torch.empty_like(out) for _ in range(nbuf)]
@@ -422,7 +427,7 @@ def run_engram(args, wl, world, rank, local):
 
     peaks = load_peaks()
     n_tok = wl.n_tok
-    flops = 2.0 * n_tok * wl.d_m * 2 * wl.d_h
+    flops = 2.0 * n_tok * wl.d_m * (M + 1) * wl.d_h     # M key projections + the value projection
     proj_s = stage_ms["proj"] / 1e3
     tflops = flops / proj_s / 1e12
     roofline = {"bound": "tensor", "kernel": "proj_kernel (tcgen05 k/v projections + gate partials)",
@@ -432,7 +437,7 @@ def run_engram(args, wl, world, rank, local):
     # HBM view of the memory-bound kernels (gather and gate+conv)
     row_bytes = wl.H * wl.d_e * wl.table_elem_bytes
     gather_bytes = n_tok * (row_bytes + wl.H * wl.d_e * 2 + wl.H * 4)   # rows read + m written + row ids
-    gate_bytes = n_tok * (wl.d_h * 2 * 3 + 8)                     # v (fp16) + h read, out written, scalars
+    gate_bytes = n_tok * (wl.d_h * 2 + M * (wl.d_h * 2 * 2 + 8))   # v (fp16) once; h read, out written, scalars per branch
     hbm = {"gather_GBps": gather_bytes / (stage_ms["gather"] / 1e3) / 1e9,
            "gate_conv_GBps": gate_bytes / (stage_ms["gate_conv"] / 1e3) / 1e9,
            "peak_GBps": peaks["hbm"], "nominal_GBps": 8000.0}

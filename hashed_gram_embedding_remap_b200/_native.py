@@ -26,6 +26,7 @@ ENGRAM_STATUS_BAD_ROW = 0x2
 ENGRAM_STATUS_WAIT_TIMEOUT = 0x4
 ENGRAM_MAX_ORDERS = 4
 ENGRAM_MAX_TABLES = 32
+ENGRAM_MAX_BRANCHES = 8
 ENGRAM_FORWARD_STAGES = 4
 ENGRAM_TABLES_DEVICE = 0
 ENGRAM_TABLES_HOST_MAPPED = 1
@@ -63,7 +64,8 @@ class engram_config(C.Structure):
         ("flags", C.c_int32),
         ("table_dtype", C.c_int32),
         ("table_scale", C.c_float * ENGRAM_MAX_TABLES),
-        ("reserved", C.c_int32 * 5),
+        ("num_branches", C.c_int32),
+        ("reserved", C.c_int32 * 4),
     ]
 
 
@@ -76,7 +78,8 @@ class engram_plan(C.Structure):
         ("hist_len", C.c_int32),
         ("state_len", C.c_int32),
         ("magic", C.c_uint32),
-        ("reserved", C.c_int32 * 3),
+        ("num_branches", C.c_int32),
+        ("reserved", C.c_int32 * 2),
     ]
 
 
@@ -164,7 +167,7 @@ class Plan:
                  row_dim: int, hidden_dim: int, vocab_in: int, vocab_out: int, hash_seed: int,
                  eps: float = 1e-6, conv_kernel: int = 4, table_location: int = ENGRAM_TABLES_DEVICE,
                  flags: int = 0, table_dtype: int = ENGRAM_TABLE_BF16,
-                 table_scale: Optional[Sequence[float]] = None):
+                 table_scale: Optional[Sequence[float]] = None, num_branches: int = 1):
         cfg = engram_config()
         cfg.num_orders = len(orders)
         for i, o in enumerate(orders):
@@ -184,6 +187,7 @@ class Plan:
         cfg.eps = float(eps)
         cfg.flags = int(flags)
         cfg.table_dtype = int(table_dtype)
+        cfg.num_branches = int(num_branches)
         for i, sc in enumerate(table_scale or ()):
             cfg.table_scale[i] = float(sc)
         self.cfg = cfg
@@ -198,7 +202,8 @@ class Plan:
                    hidden_dim=wl.d_h, vocab_in=wl.vocab_in, vocab_out=wl.vocab_out,
                    hash_seed=wl.hash_seed, eps=wl.eps, conv_kernel=wl.conv_kernel,
                    table_location=loc, table_dtype=ENGRAM_TABLE_FP8_E4M3 if fp8 else ENGRAM_TABLE_BF16,
-                   table_scale=[float(wl.table_scale(h)) for h in range(wl.H)] if fp8 else None, **kw)
+                   table_scale=[float(wl.table_scale(h)) for h in range(wl.H)] if fp8 else None,
+                   num_branches=getattr(wl, "branches", 1), **kw)
 
     @property
     def num_tables(self) -> int:
@@ -207,6 +212,10 @@ class Plan:
     @property
     def mem_dim(self) -> int:
         return self.plan.mem_dim
+
+    @property
+    def num_branches(self) -> int:
+        return self.plan.num_branches
 
     @property
     def hist_len(self) -> int:
@@ -297,9 +306,19 @@ def engram_stage_rows(plan: Plan, idx: torch.Tensor, tables, staging, staged_idx
                                  _ptr(n_unique, torch.int32, "n_unique"), _stream(stream)))
 
 
+def _check_rows(plan: Plan, n_tok: int, **tensors):
+    """h / out / delta hold one d_h-wide row per (token, branch)."""
+    want = n_tok * plan.num_branches * plan.cfg.hidden_dim
+    for name, t in tensors.items():
+        if t is not None and t.numel() != want:
+            raise ValueError(f"{name} has {t.numel()} elements; {n_tok} tokens x {plan.num_branches} branches x "
+                             f"{plan.cfg.hidden_dim} need {want}")
+
+
 def engram_gate_conv(plan: Plan, weights: Weights, h: torch.Tensor, m: torch.Tensor, B: int, T: int,
                      out: torch.Tensor, workspace: torch.Tensor, conv_state: Optional[torch.Tensor] = None,
                      delta_dbg: Optional[torch.Tensor] = None, stream=None):
+    _check_rows(plan, B * T, h=h, out=out, delta_dbg=delta_dbg)
     _check(lib.engram_gate_conv(plan, weights, _ptr(h, _BF16, "h"), _ptr(m, _BF16, "m"), B, T,
                                 _ptr(conv_state, _BF16, "conv_state"), _ptr(out, _BF16, "out"),
                                 _ptr(delta_dbg, torch.float32, "delta_dbg"),
@@ -312,6 +331,7 @@ def engram_gate_conv_noalloc(plan: Plan, weights: Weights, h: torch.Tensor, m: t
                              delta_dbg: Optional[torch.Tensor] = None, stream=None):
     """engram_gate_conv without a workspace, for hosts that cannot allocate device memory
     (their scratch is the library's fixed per-GPU array of ENGRAM_NOALLOC_SCRATCH_BYTES)."""
+    _check_rows(plan, B * T, h=h, out=out, delta_dbg=delta_dbg)
     _check(lib.engram_gate_conv_noalloc(plan, weights, _ptr(h, _BF16, "h"), _ptr(m, _BF16, "m"), B, T,
                                         _ptr(conv_state, _BF16, "conv_state"), _ptr(out, _BF16, "out"),
                                         _ptr(delta_dbg, torch.float32, "delta_dbg"), _stream(stream)))
@@ -322,6 +342,7 @@ def engram_forward(plan: Plan, weights: Weights, tables, ids: torch.Tensor, h: t
                    history: Optional[torch.Tensor] = None, conv_state: Optional[torch.Tensor] = None,
                    delta_dbg: Optional[torch.Tensor] = None, stream=None, stage_events=None):
     B, T = ids.shape
+    _check_rows(plan, B * T, h=h, out=out, delta_dbg=delta_dbg)
     arr = _table_array(tables, plan)
     ev = None
     if stage_events is not None:

@@ -119,7 +119,7 @@ int table_elem_bytes(const engram_plan *plan) { return fp8_tables(plan) ? 1 : 2;
 // Width of the projection's N tile: the widest of 256/128/64 that divides d_h and still
 // gives at least two waves of CTAs on the GPU.  ENGRAM_PROJ_TILE_N (64, 128 or 256) forces a
 // width (for tuning and tests); it is read once per process.
-int choose_bn(int d_h, int64_t n_tok) {
+int choose_bn(int d_h, int64_t n_tok, int M) {
     static const int forced = [] {
         const char *e = std::getenv("ENGRAM_PROJ_TILE_N");
         const int v = e ? std::atoi(e) : 0;
@@ -130,7 +130,7 @@ int choose_bn(int d_h, int64_t n_tok) {
     const int cands[3] = {256, 128, 64};
     for (int bn : cands) {
         if (d_h % bn != 0) continue;
-        if (bn == 64 || m_tiles * (2 * d_h / bn) >= 2 * 148) return bn;
+        if (bn == 64 || m_tiles * ((M + 1) * d_h / bn) >= 2 * 148) return bn;
     }
     return 64;
 }
@@ -157,7 +157,8 @@ ProjShape proj_shape(const engram_plan *plan, int64_t n_tok, bool allow_split) {
             break;
         }
     }
-    const int64_t mn = m_tiles * (2 * d_h / wide);
+    const int M = plan->num_branches;
+    const int64_t mn = m_tiles * ((M + 1) * d_h / wide);
     // ENGRAM_PROJ_SPLITS (>= 1) forces the split count of decode-sized batches (tuning);
     // read once per process.
     static const int forced_splits = [] {
@@ -176,9 +177,9 @@ ProjShape proj_shape(const engram_plan *plan, int64_t n_tok, bool allow_split) {
         ps.kb_per_split = (ps.k_blocks + splits - 1) / splits;
         ps.k_splits = (ps.k_blocks + ps.kb_per_split - 1) / ps.kb_per_split;
     } else {
-        ps.bn = choose_bn(d_h, n_tok);
+        ps.bn = choose_bn(d_h, n_tok, M);
     }
-    ps.n_tiles = 2 * d_h / ps.bn;
+    ps.n_tiles = (M + 1) * d_h / ps.bn;
     return ps;
 }
 
@@ -214,8 +215,8 @@ Workspace layout(const engram_plan *plan, int64_t n_tok) {
     w.v = off;    off = align256(off + v_bytes);
     w.part = off; off = align256(off + sizeof(float4) * n_tok * n_tiles);
     w.acc = off;
-    if (ps.k_splits > 1) off = align256(off + sizeof(float) * ps.k_splits * n_tok * 2 * d_h);
-    w.scal = off; off = align256(off + sizeof(float2) * n_tok);
+    if (ps.k_splits > 1) off = align256(off + sizeof(float) * ps.k_splits * n_tok * ps.n_tiles * ps.bn);
+    w.scal = off; off = align256(off + sizeof(float2) * n_tok * plan->num_branches);
     w.staged = plan->cfg.table_location == ENGRAM_TABLES_HOST_MAPPED && n_tok <= engram::kStageMaxTok;
     if (w.staged) {
         w.staged_idx = off; off = align256(off + sizeof(uint32_t) * n_tok * H);
@@ -292,7 +293,8 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     CUtensorMap map_m, map_wk, map_wv;
     int rc;
     if ((rc = make_map_bf16(&map_m, m, static_cast<uint64_t>(n_tok), d_m, engram::kBM)) != ENGRAM_OK) return rc;
-    if ((rc = make_map_bf16(&map_wk, w->w_k, d_h, d_m, BN)) != ENGRAM_OK) return rc;
+    const int M = plan->num_branches;
+    if ((rc = make_map_bf16(&map_wk, w->w_k, static_cast<uint64_t>(M) * d_h, d_m, BN)) != ENGRAM_OK) return rc;
     if ((rc = make_map_bf16(&map_wv, w->w_v, d_h, d_m, BN)) != ENGRAM_OK) return rc;
     if ((rc = set_proj_smem_attr<BN>()) != ENGRAM_OK) return rc;
     engram::ProjParams p{};
@@ -304,7 +306,8 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     p.n_tok = n_tok;
     p.d_m = d_m;
     p.d_h = d_h;
-    p.n_tiles = 2 * d_h / BN;
+    p.n_tiles = (M + 1) * d_h / BN;
+    p.M = M;
     p.k_blocks = (d_m + engram::kBK - 1) / engram::kBK;
     p.m_tiles = static_cast<int32_t>((n_tok + engram::kBM - 1) / engram::kBM);
     p.k_splits = (acc != nullptr && k_splits > 1) ? k_splits : 1;
@@ -456,7 +459,8 @@ engram::GateParams make_gate_params(const engram_plan *plan, const engram_weight
     p.T = T;
     p.d_h = d_h;
     p.n_tiles = n_tiles;
-    p.n_key_tiles = n_tiles / 2;
+    p.M = plan->num_branches;
+    p.n_key_tiles = n_tiles / (p.M + 1);
     p.ksize = plan->cfg.conv_kernel;
     p.dil = plan->cfg.conv_dilation;
     p.state_len = plan->state_len;
@@ -483,18 +487,22 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
     p.T = T;
     p.d_h = d_h;
     p.n_tiles = n_tiles;
-    p.n_key_tiles = n_tiles / 2;
+    p.M = plan->num_branches;
+    p.n_key_tiles = n_tiles / (p.M + 1);
     p.ksize = plan->cfg.conv_kernel;
     p.dil = plan->cfg.conv_dilation;
     p.state_len = plan->state_len;
     constexpr int kChain = 12;   // outputs per residue chain in the k=4, dilation-3 fast path
-    const bool fast = p.ksize == 4 && p.dil == 3 && (conv_state == nullptr || T <= 3 * kChain);
+    const bool k4d3 = p.ksize == 4 && p.dil == 3;
+    // the single-branch kernels (decode, short stateful chains) serve M = 1; the generic
+    // kernel and the 4-channel prefill kernel serve every M
+    const bool fast = k4d3 && p.M == 1 && (conv_state == nullptr || T <= 3 * kChain);
     p.tok_chunk = fast ? 3 * kChain : (conv_state != nullptr ? T : 32);
     p.eps = plan->cfg.eps;
     p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(d_h));
     const int threads = fast ? engram::kGateFastThreads : engram::kGateThreads;
     const int per_thread = fast ? 2 : 4;   // channels per thread
-    const unsigned slices = static_cast<unsigned>((d_h / per_thread + threads - 1) / threads);
+    const unsigned slices = static_cast<unsigned>((d_h / per_thread + threads - 1) / threads) * p.M;
     const size_t smem = sizeof(float) * 2 * static_cast<size_t>(p.tok_chunk + p.state_len);
     if (smem > 48 * 1024) {
         ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::gate_conv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -508,17 +516,17 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
         return ENGRAM_OK;
     }
     dim3 grid(static_cast<unsigned>((T + p.tok_chunk - 1) / p.tok_chunk), static_cast<unsigned>(B), slices);
-    if (fast && scal != nullptr && conv_state == nullptr) {
-        // scalars once per token instead of once per (CTA, halo-extended chunk)
-        const int64_t n_tok = static_cast<int64_t>(B) * T;
-        engram::gate_scalars_kernel<<<static_cast<unsigned>((n_tok * 8 + 255) / 256), 256, 0, stream>>>(
-            part, n_tok, n_tiles, p.n_key_tiles, d_h, p.eps, p.inv_sqrt_d, scal);
+    if (k4d3 && scal != nullptr && conv_state == nullptr) {
+        // scalars once per (token, branch) instead of once per (CTA, halo-extended chunk)
+        const int64_t items = static_cast<int64_t>(B) * T * p.M;
+        engram::gate_scalars_kernel<<<static_cast<unsigned>((items * 8 + 255) / 256), 256, 0, stream>>>(
+            part, static_cast<int64_t>(B) * T, n_tiles, p.n_key_tiles, p.M, d_h, p.eps, p.inv_sqrt_d, scal);
         ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_scalars_kernel launch");
         p.scal = scal;
     }
-    if (fast && p.scal != nullptr) {
+    if (p.scal != nullptr) {
         constexpr int kChain4 = 16;   // 48-token chunks, 4 channels per thread
-        dim3 grid4(static_cast<unsigned>((T + 3 * kChain4 - 1) / (3 * kChain4)), static_cast<unsigned>(B),
+        dim3 grid4(static_cast<unsigned>((T + 3 * kChain4 - 1) / (3 * kChain4)) * p.M, static_cast<unsigned>(B),
                    static_cast<unsigned>((d_h / 4 + engram::kGate4Threads - 1) / engram::kGate4Threads));
         engram::gate_conv_k4d3_c4_kernel<kChain4><<<grid4, engram::kGate4Threads, 0, stream>>>(p);
         ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_conv_k4d3_c4_kernel launch");
@@ -640,7 +648,7 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
     float *acc = ps.k_splits > 1 ? reinterpret_cast<float *>(ws + L.acc) : nullptr;
     const int d_h = plan->cfg.hidden_dim;
     // one-token decode steps after a split-K projection: reduce + gate + conv in one kernel
-    const bool fused_decode = ps.k_splits > 1 && T == 1 && plan->cfg.conv_kernel == 4 &&
+    const bool fused_decode = ps.k_splits > 1 && T == 1 && plan->num_branches == 1 && plan->cfg.conv_kernel == 4 &&
                               plan->cfg.conv_dilation == 3 && d_h <= 2 * engram::kFusedDecodeThreads * engram::kFusedDecodeMaxPairs;
     engram::ProjParams pp{};
     int rc;
@@ -747,8 +755,13 @@ int engram_init(const engram_config *cfg, engram_plan *plan) {
     if (!(c.eps > 0.f) || !std::isfinite(c.eps)) return fail(ENGRAM_ERR_INVALID_ARG, "eps must be a positive finite number");
     if (c.table_location != ENGRAM_TABLES_DEVICE && c.table_location != ENGRAM_TABLES_HOST_MAPPED)
         return fail(ENGRAM_ERR_INVALID_ARG, "unknown table_location");
-    for (int i = 0; i < 5; ++i)
+    for (int i = 0; i < 4; ++i)
         if (c.reserved[i] != 0) return fail(ENGRAM_ERR_INVALID_ARG, "reserved fields must be zero");
+    const int M = c.num_branches == 0 ? 1 : c.num_branches;
+    if (M < 1 || M > ENGRAM_MAX_BRANCHES)
+        return fail(ENGRAM_ERR_UNSUPPORTED, "num_branches must be in 0..%d", ENGRAM_MAX_BRANCHES);
+    if (M > 1 && (c.flags & ENGRAM_FLAG_FUSED_GATE))
+        return fail(ENGRAM_ERR_UNSUPPORTED, "ENGRAM_FLAG_FUSED_GATE needs a single branch");
     if (c.table_dtype != ENGRAM_TABLE_BF16 && c.table_dtype != ENGRAM_TABLE_FP8_E4M3)
         return fail(ENGRAM_ERR_INVALID_ARG, "unknown table_dtype %d", c.table_dtype);
     for (int h = 0; h < ENGRAM_MAX_TABLES; ++h) {
@@ -775,6 +788,7 @@ int engram_init(const engram_config *cfg, engram_plan *plan) {
                 plan->mult[oi * c.heads_per_order + j][i] = splitmix64_first(key) | 1ull;
             }
     plan->num_tables = H;
+    plan->num_branches = M;
     plan->mem_dim = H * c.row_dim;
     plan->hist_len = c.orders[c.num_orders - 1] - 1;
     plan->state_len = (c.conv_kernel - 1) * c.conv_dilation;
@@ -986,8 +1000,8 @@ int engram_gate_conv_noalloc(const engram_plan *plan, const engram_weights *w, c
         return fail(ENGRAM_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
     if (conv_state && T > 16384) return fail(ENGRAM_ERR_UNSUPPORTED, "T above 16384 with a conv state");
     const int d_h = plan->cfg.hidden_dim;
-    const int bn = choose_bn(d_h, n_tok);
-    const int n_tiles = 2 * d_h / bn;
+    const int bn = choose_bn(d_h, n_tok, plan->num_branches);
+    const int n_tiles = (plan->num_branches + 1) * d_h / bn;
     const size_t v_bytes = align256(sizeof(uint16_t) * static_cast<size_t>(n_tok) * d_h);
     const size_t part_bytes = align256(sizeof(float4) * static_cast<size_t>(n_tok) * n_tiles);
     if (v_bytes + part_bytes > ENGRAM_NOALLOC_SCRATCH_BYTES)

@@ -17,18 +17,20 @@
 namespace engram {
 
 struct GateParams {
-    const uint16_t *h;        // [n_tok, d_h]
-    const uint16_t *v;        // [n_tok, d_h] fp16 (pack_v2 / v_lo / v_hi)
+    const uint16_t *h;        // [n_tok, M, d_h]
+    const uint16_t *v;        // [n_tok, d_h] fp16 (pack_v2 / v_lo / v_hi), shared by the branches
     const float4 *part;       // [n_tok, n_tiles]
     const uint16_t *gamma_c;  // [d_h]
     const uint16_t *conv_w;   // [d_h, ksize]
-    uint16_t *conv_state;     // [B, state_len, d_h] or null
-    uint16_t *out;            // [n_tok, d_h]
-    float *delta;             // [n_tok, d_h] or null
+    uint16_t *conv_state;     // [B, M, state_len, d_h] or null
+    uint16_t *out;            // [n_tok, M, d_h]
+    float *delta;             // [n_tok, M, d_h] or null
     int32_t B, T;
     int32_t d_h;
-    int32_t n_tiles;          // total tiles; the first n_key_tiles are key tiles
-    int32_t n_key_tiles;
+    int32_t n_tiles;          // (M + 1) * n_key_tiles: the key tiles of branch b are
+                              // [b * n_key_tiles, (b + 1) * n_key_tiles), then the value tiles
+    int32_t n_key_tiles;      // key tiles per branch
+    int32_t M;                // branches
     int32_t ksize, dil, state_len;
     int32_t tok_chunk;        // tokens per CTA (T when a conv state is carried)
     float eps;
@@ -44,11 +46,15 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
 
 constexpr int kGateThreads = 128;
 
-// Grid: (token chunks, B, channel slices of 4 * kGateThreads).  One thread per 4 channels.
-// Dynamic smem: 2 floats (g, g/rms_U) per token of [t0 - state_len, t1).
+// Grid: (token chunks, B, channel slices of 4 * kGateThreads x M branches, branch fastest).
+// One thread per 4 channels of one branch.  Dynamic smem: 2 floats (g, g/rms_U) per token of
+// [t0 - state_len, t1).
 __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_constant__ GateParams p) {
     extern __shared__ float s_scal[];   // [2][tok_chunk + state_len]
     const int b = blockIdx.y;
+    const int br = static_cast<int>(blockIdx.z % p.M);
+    const int slice = static_cast<int>(blockIdx.z / p.M);
+    const int64_t hrow = static_cast<int64_t>(p.M);   // rows of h / out per token
     const int t0 = blockIdx.x * p.tok_chunk;
     if (t0 >= p.T) return;
     const int t1 = min(p.T, t0 + p.tok_chunk);
@@ -65,13 +71,13 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
         if (t >= 0) {
             const float4 *pp = p.part + (static_cast<int64_t>(b) * p.T + t) * p.n_tiles;
             float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-            for (int j = 0; j < p.n_key_tiles; ++j) {
+            for (int j = br * p.n_key_tiles; j < (br + 1) * p.n_key_tiles; ++j) {
                 const float4 q = pp[j];
                 s0 += q.x;
                 s1 += q.y;
                 s2 += q.z;
             }
-            for (int j = p.n_key_tiles; j < p.n_tiles; ++j) s3 += pp[j].x;
+            for (int j = p.M * p.n_key_tiles; j < p.n_tiles; ++j) s3 += pp[j].x;
             const float rms_h = sqrtf(s0 * inv_d + p.eps);
             const float rms_k = sqrtf(s2 * inv_d + p.eps);
             g = sigmoidf_(s1 / (rms_h * rms_k) * p.inv_sqrt_d);
@@ -84,7 +90,8 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
     __syncthreads();
 
     const int nq = p.d_h / 4;
-    const int q = blockIdx.z * blockDim.x + threadIdx.x;
+    const int q = slice * blockDim.x + threadIdx.x;
+    const int64_t sbase = (static_cast<int64_t>(b) * p.M + br) * p.state_len;   // conv state rows of (b, br)
     if (q < nq) {
         const int c = q * 4;
         float gc[4], w[4][8];
@@ -116,7 +123,7 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
                     for (int e = 0; e < 4; ++e) u[e] = beta * vv[e] * gc[e];
                 } else if (p.conv_state != nullptr) {
                     const uint2 sw = *reinterpret_cast<const uint2 *>(
-                        p.conv_state + (static_cast<int64_t>(b) * p.state_len + p.state_len + t) * p.d_h + c);
+                        p.conv_state + (sbase + p.state_len + t) * p.d_h + c);
                     u[0] = bf16_lo(sw.x); u[1] = bf16_hi(sw.x); u[2] = bf16_lo(sw.y); u[3] = bf16_hi(sw.y);
                     vv[0] = vv[1] = vv[2] = vv[3] = 0.f;
                 } else {
@@ -131,8 +138,9 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
                 for (int e = 0; e < 4; ++e) hist[0][e] = u[e];
                 if (t < t0) continue;
                 const int64_t n = static_cast<int64_t>(b) * p.T + t;
+                const int64_t nr = n * hrow + br;   // row of (token, branch) in h / out / delta
                 const float g = s_g[si];
-                const uint2 hw = *reinterpret_cast<const uint2 *>(p.h + n * p.d_h + c);
+                const uint2 hw = *reinterpret_cast<const uint2 *>(p.h + nr * p.d_h + c);
                 const float hv[4] = {bf16_lo(hw.x), bf16_hi(hw.x), bf16_lo(hw.y), bf16_hi(hw.y)};
                 float dl[4];
                 uint16_t ob[4];
@@ -148,9 +156,9 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
                 uint2 o;
                 o.x = static_cast<uint32_t>(ob[0]) | (static_cast<uint32_t>(ob[1]) << 16);
                 o.y = static_cast<uint32_t>(ob[2]) | (static_cast<uint32_t>(ob[3]) << 16);
-                *reinterpret_cast<uint2 *>(p.out + n * p.d_h + c) = o;
+                *reinterpret_cast<uint2 *>(p.out + nr * p.d_h + c) = o;
                 if (p.delta != nullptr)
-                    *reinterpret_cast<float4 *>(p.delta + n * p.d_h + c) = make_float4(dl[0], dl[1], dl[2], dl[3]);
+                    *reinterpret_cast<float4 *>(p.delta + nr * p.d_h + c) = make_float4(dl[0], dl[1], dl[2], dl[3]);
             }
         }
         if (p.conv_state != nullptr) {
@@ -170,35 +178,38 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
                     o.x = static_cast<uint32_t>(u0) | (static_cast<uint32_t>(u1) << 16);
                     o.y = static_cast<uint32_t>(u2) | (static_cast<uint32_t>(u3) << 16);
                 } else {
-                    o = *reinterpret_cast<const uint2 *>(
-                        p.conv_state + (static_cast<int64_t>(b) * p.state_len + p.state_len + t) * p.d_h + c);
+                    o = *reinterpret_cast<const uint2 *>(p.conv_state + (sbase + p.state_len + t) * p.d_h + c);
                 }
-                *reinterpret_cast<uint2 *>(p.conv_state + (static_cast<int64_t>(b) * p.state_len + s) * p.d_h + c) = o;
+                *reinterpret_cast<uint2 *>(p.conv_state + (sbase + s) * p.d_h + c) = o;
             }
         }
     }
 }
 
-// Per-token gate scalars from the projection partials: scal[n] = (g, g / rms_U).  Eight
-// lanes per token take every eighth tile; a fixed-order butterfly over the eight lanes
-// finishes the sums (deterministic).
+// Per-(token, branch) gate scalars from the projection partials: scal[n*M + b] =
+// (g_b, g_b / rms(U_b)).  Eight lanes per (token, branch) take every eighth of the branch's
+// key tiles followed by the value tiles; a fixed-order butterfly over the eight lanes finishes
+// the sums (deterministic).
 __global__ void __launch_bounds__(256) gate_scalars_kernel(const float4 *__restrict__ part, int64_t n_tok,
-                                                           int32_t n_tiles, int32_t n_key_tiles, int32_t d_h,
-                                                           float eps, float inv_sqrt_d, float2 *__restrict__ scal) {
+                                                           int32_t n_tiles, int32_t n_key_tiles, int32_t M,
+                                                           int32_t d_h, float eps, float inv_sqrt_d,
+                                                           float2 *__restrict__ scal) {
     const int64_t gt = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t n = gt >> 3;
+    const int64_t item = gt >> 3;          // (token, branch)
     const int sub = static_cast<int>(gt & 7);
+    const int64_t n = item / M;
+    const int br = static_cast<int>(item - n * M);
     float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
     if (n < n_tok) {
         const float4 *pp = part + n * n_tiles;
-        for (int j = sub; j < n_tiles; j += 8) {
-            const float4 q = __ldg(pp + j);
+        for (int j = sub; j < 2 * n_key_tiles; j += 8) {
             if (j < n_key_tiles) {
+                const float4 q = __ldg(pp + br * n_key_tiles + j);
                 s0 += q.x;
                 s1 += q.y;
                 s2 += q.z;
             } else {
-                s3 += q.x;
+                s3 += __ldg(pp + M * n_key_tiles + (j - n_key_tiles)).x;
             }
         }
     }
@@ -214,7 +225,7 @@ __global__ void __launch_bounds__(256) gate_scalars_kernel(const float4 *__restr
         const float rms_h = sqrtf(s0 * inv_d + eps);
         const float rms_k = sqrtf(s2 * inv_d + eps);
         const float g = 1.f / (1.f + __expf(-(s1 / (rms_h * rms_k) * inv_sqrt_d)));
-        scal[n] = make_float2(g, g / sqrtf(g * g * s3 * inv_d + eps));
+        scal[item] = make_float2(g, g / sqrtf(g * g * s3 * inv_d + eps));
     }
 }
 
@@ -401,7 +412,9 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
 
 // Prefill-only variant of gate_conv_k4d3_kernel with 4 channels per thread (8-byte bf16
 // loads, half the per-element address and predicate work) and 3*CH-token chunks.  Needs the
-// per-token scalars from gate_scalars_kernel.
+// per-token scalars from gate_scalars_kernel.  Grid: (token chunks x M branches, branch
+// fastest so that the branches of a chunk read its shared v rows while they are in L2; B;
+// channel slices).
 constexpr int kGate4Threads = 128;
 
 template <int CH>
@@ -409,14 +422,16 @@ __global__ void __launch_bounds__(kGate4Threads) gate_conv_k4d3_c4_kernel(const 
     constexpr int KS = 4, DIL = 3, HALO = (KS - 1) * DIL, TC = CH * DIL;
     __shared__ float2 s_sc[TC + HALO];          // (g, beta) per token of [t0 - HALO, t1)
     const int b = blockIdx.y;
-    const int t0 = blockIdx.x * TC;
+    const int br = static_cast<int>(blockIdx.x % p.M);
+    const int t0 = static_cast<int>(blockIdx.x / p.M) * TC;
     if (t0 >= p.T) return;
     const int t1 = min(p.T, t0 + TC);
     const int lo = t0 - HALO;
     const int64_t row0 = static_cast<int64_t>(b) * p.T;
+    const int64_t hstride = static_cast<int64_t>(p.M) * p.d_h;   // h / out / delta token stride
     for (int i = threadIdx.x; i < TC + HALO; i += kGate4Threads) {
         const int t = lo + i;
-        s_sc[i] = (t >= 0 && t < t1) ? __ldg(p.scal + row0 + t) : make_float2(0.f, 0.f);
+        s_sc[i] = (t >= 0 && t < t1) ? __ldg(p.scal + (row0 + t) * p.M + br) : make_float2(0.f, 0.f);
     }
     __syncthreads();
     const int q = blockIdx.z * blockDim.x + threadIdx.x;
@@ -436,7 +451,7 @@ __global__ void __launch_bounds__(kGate4Threads) gate_conv_k4d3_c4_kernel(const 
         }
     }
     const uint16_t *vbase = p.v + row0 * p.d_h + c;
-    const uint16_t *hbase = p.h + row0 * p.d_h + c;
+    const uint16_t *hbase = p.h + (row0 * p.M + br) * p.d_h + c;
 #pragma unroll 1
     for (int r = 0; r < DIL; ++r) {
         uint2 vv[CH + KS - 1];
@@ -450,7 +465,7 @@ __global__ void __launch_bounds__(kGate4Threads) gate_conv_k4d3_c4_kernel(const 
 #pragma unroll
         for (int j = 0; j < CH; ++j) {
             const int t = t0 + r + DIL * j;
-            hh[j] = t < t1 ? __ldg(reinterpret_cast<const uint2 *>(hbase + static_cast<int64_t>(t) * p.d_h))
+            hh[j] = t < t1 ? __ldg(reinterpret_cast<const uint2 *>(hbase + static_cast<int64_t>(t) * hstride))
                            : make_uint2(0u, 0u);
         }
         float u[KS][4];
@@ -482,11 +497,11 @@ __global__ void __launch_bounds__(kGate4Threads) gate_conv_k4d3_c4_kernel(const 
                 for (int i = 1; i < KS; ++i) acc = fmaf(w[e][i], u[i][e], acc);
                 dl[e] = fmaf(sc.x, vj[e], silu_fast(acc));
             }
-            const int64_t n = row0 + t;
-            *reinterpret_cast<uint2 *>(p.out + n * p.d_h + c) =
+            const int64_t nr = (row0 + t) * p.M + br;   // row of (token, branch)
+            *reinterpret_cast<uint2 *>(p.out + nr * p.d_h + c) =
                 make_uint2(pack_bf16x2(hv[0] + dl[0], hv[1] + dl[1]), pack_bf16x2(hv[2] + dl[2], hv[3] + dl[3]));
             if (p.delta != nullptr)
-                *reinterpret_cast<float4 *>(p.delta + n * p.d_h + c) = make_float4(dl[0], dl[1], dl[2], dl[3]);
+                *reinterpret_cast<float4 *>(p.delta + nr * p.d_h + c) = make_float4(dl[0], dl[1], dl[2], dl[3]);
         }
     }
 }

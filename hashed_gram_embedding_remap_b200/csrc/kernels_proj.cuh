@@ -2,8 +2,9 @@
 // tcgen05 tensor cores, with the gate's per-token partial sums reduced in the epilogue.
 //
 // proj_kernel: persistent (grid = #SMs); CTA i takes work units i, i + grid, ...  A unit is
-// a 128-token x BN-channel tile of [k~ | v] (key tiles first), or for decode-sized batches a
-// K-slice of such a tile (split-K).  Warp 0 streams 128x64 tiles of m and BNx64 tiles of W
+// a 128-token x BN-channel tile of [k~_0 | .. | k~_{M-1} | v] (the key tiles of the M branches
+// first, branch-major, then the value tiles), or for decode-sized batches a K-slice of such a
+// tile (split-K).  Warp 0 streams 128x64 tiles of m and BNx64 tiles of W
 // with TMA (128-byte swizzle, no cluster multicast) through an S-stage shared-memory ring;
 // warp 1 owns TMEM and issues tcgen05.mma (M=128, N=BN, K=16) into one of two accumulators;
 // warps 2-5 drain the other accumulator with tcgen05.ld while the next unit's MMAs run.  The
@@ -41,19 +42,20 @@ struct ProjCfg {
 };
 
 struct ProjParams {
-    const uint16_t *h;         // [n_tok, d_h] bf16
+    const uint16_t *h;         // [n_tok, M, d_h] bf16
     const uint16_t *gamma_q;   // [d_h]
     const uint16_t *gamma_k;   // [d_h]
     uint16_t *v;               // [n_tok, d_h] fp16 out (rounded from the fp32 accumulator)
     float4 *part;              // [n_tok, n_tiles] partial sums out
     int64_t n_tok;
     int32_t d_m, d_h;
-    int32_t n_tiles;           // 2 * d_h / BN: key tiles first, then value tiles
+    int32_t n_tiles;           // (M + 1) * d_h / BN: key tiles (branch-major), then value tiles
+    int32_t M;                 // branches (key projections)
     int32_t k_blocks;          // ceil(d_m / kBK)
     int32_t m_tiles;           // ceil(n_tok / kBM)
     int32_t k_splits;          // > 1: split-K, raw fp32 partial accumulators go to acc_out
     int32_t kb_per_split;      // k-blocks per split
-    float *acc_out;            // [k_splits, n_tok, 2*d_h] when k_splits > 1
+    float *acc_out;            // [k_splits, n_tok, (M+1)*d_h] when k_splits > 1
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -108,7 +110,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     const int lane = threadIdx.x % 32;
     const int mn_tiles = p.m_tiles * p.n_tiles;
     const int total = mn_tiles * p.k_splits;   // work units: (k split, m tile, n tile), n fastest
-    const int key_tiles = p.d_h / BN;
+    const int key_tiles = p.M * (p.d_h / BN);   // all branches
+    const int kpb = p.d_h / BN;                 // key tiles per branch
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 const int mt = tmn / p.n_tiles, nt = tmn - mt * p.n_tiles;
                 const bool is_key = nt < key_tiles;
                 const CUtensorMap *map_w = is_key ? &map_wk : &map_wv;
-                const int c0 = (is_key ? nt : nt - key_tiles) * BN;
+                const int c0 = (is_key ? nt : nt - key_tiles) * BN;   // row of the stacked W_k, or of W_v
                 const int m0 = mt * kBM;
                 const int kb0 = ks * p.kb_per_split, kb1 = min(p.k_blocks, kb0 + p.kb_per_split);
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
@@ -209,7 +212,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             const int ks = t / mn_tiles, tmn = t - ks * mn_tiles;
             const int mt = tmn / p.n_tiles, nt = tmn - mt * p.n_tiles;
             const bool is_key = nt < key_tiles;
-            const int c0 = (is_key ? nt : nt - key_tiles) * BN;
+            const int br = is_key ? nt / kpb : 0;                       // branch of a key tile
+            const int c0 = (is_key ? nt - br * kpb : nt - key_tiles) * BN;   // channel within d_h
             const int64_t n = static_cast<int64_t>(mt) * kBM + row;
             const bool valid = n < p.n_tok;
             const uint32_t taddr = tmem_base + acc * BN + (static_cast<uint32_t>(sub * 32) << 16);
@@ -221,12 +225,12 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 if (p.k_splits > 1) {
                     // split-K: raw partial accumulator; splitk_reduce_kernel finishes the tile
                     float4 *ap = reinterpret_cast<float4 *>(
-                        p.acc_out + (static_cast<int64_t>(ks) * p.n_tok + n) * (2 * p.d_h) + nt * BN + cc);
+                        p.acc_out + (static_cast<int64_t>(ks) * p.n_tok + n) * (p.n_tiles * BN) + nt * BN + cc);
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
                         ap[q] = make_float4(accv[4 * q], accv[4 * q + 1], accv[4 * q + 2], accv[4 * q + 3]);
                 } else if (is_key) {
-                    const uint4 *hp = reinterpret_cast<const uint4 *>(p.h + n * p.d_h + c0 + cc);
+                    const uint4 *hp = reinterpret_cast<const uint4 *>(p.h + (n * p.M + br) * p.d_h + c0 + cc);
                     const uint4 *gq = reinterpret_cast<const uint4 *>(p.gamma_q + c0 + cc);
                     const uint4 *gk = reinterpret_cast<const uint4 *>(p.gamma_k + c0 + cc);
 #pragma unroll
@@ -291,13 +295,16 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const __g
     __shared__ float s_red[3][kReduceThreads / 32];
     const int nt = blockIdx.x;
     const int64_t n = blockIdx.y;
-    const int key_tiles = p.d_h / BN;
+    const int kpb = p.d_h / BN;
+    const int key_tiles = p.M * kpb;
     const bool is_key = nt < key_tiles;
-    const int c0 = (is_key ? nt : nt - key_tiles) * BN;
-    const int64_t stride_split = p.n_tok * (2 * p.d_h);
+    const int br = is_key ? nt / kpb : 0;
+    const int c0 = (is_key ? nt - br * kpb : nt - key_tiles) * BN;
+    const int64_t row_len = static_cast<int64_t>(p.n_tiles) * BN;
+    const int64_t stride_split = p.n_tok * row_len;
     float a0 = 0.f, a1 = 0.f, a2 = 0.f;
     for (int j = threadIdx.x * 2; j < BN; j += kReduceThreads * 2) {
-        const float *src = p.acc_out + n * (2 * p.d_h) + nt * BN + j;
+        const float *src = p.acc_out + n * row_len + nt * BN + j;
         float x0 = 0.f, x1 = 0.f;
         for (int ks = 0; ks < p.k_splits; ++ks) {
             const float2 q = __ldg(reinterpret_cast<const float2 *>(src + ks * stride_split));
@@ -305,7 +312,7 @@ __global__ void __launch_bounds__(kReduceThreads) splitk_reduce_kernel(const __g
             x1 += q.y;
         }
         if (is_key) {
-            const uint32_t hw = __ldg(reinterpret_cast<const uint32_t *>(p.h + n * p.d_h + c0 + j));
+            const uint32_t hw = __ldg(reinterpret_cast<const uint32_t *>(p.h + (n * p.M + br) * p.d_h + c0 + j));
             const uint32_t qw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_q + c0 + j));
             const uint32_t kw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_k + c0 + j));
             const float h0 = bf16_lo(hw), h1 = bf16_hi(hw);

@@ -58,6 +58,7 @@ extern "C" {
 #define ENGRAM_MAX_ORDERS 4
 #define ENGRAM_MAX_TABLES 32
 #define ENGRAM_MAX_HIST 3 /* largest order - 1 */
+#define ENGRAM_MAX_BRANCHES 8
 
 typedef void *engram_stream_t; /* cudaStream_t */
 
@@ -98,15 +99,30 @@ typedef struct engram_config {
     float table_scale[ENGRAM_MAX_TABLES]; /* FP8 tables: dequantisation scale of table h,
                                              in [2^-100, 2^100]; must be 0 for bf16 tables
                                              and beyond the H tables */
-    int32_t reserved[5];                  /* must be zero */
+    int32_t num_branches;                 /* M, 1..ENGRAM_MAX_BRANCHES (0 reads as 1): the
+                                             multi-branch form, see "Branches" below */
+    int32_t reserved[4];                  /* must be zero */
 } engram_config;
+
+/* Branches [yktysq #4: with a multi-branch residual stream the branches share one embedding
+ * table and one value projection, and each has its own key projection, so that every branch
+ * gates the memory differently; zhichai §2.2: the residual stream is widened to 4 branches].
+ * With M = num_branches > 1, for every branch b of token n:
+ *   k~_b = W_k^b m, v = W_v m (shared), g_b = sigmoid(RMSNorm(h_b).RMSNorm(k~_b) / sqrt(d_h)),
+ *   U_b = g_b v, Delta_b = U_b + SiLU(DWConv(RMSNorm(U_b))), out_b = h_b + Delta_b,
+ * with the gains and conv weights shared by the branches.  Layouts:
+ *   h, out, delta_dbg: [B*T, M, d_h] (branch b of token n is row n*M + b);
+ *   w_k: [M*d_h, d_m] (branch b's key projection is rows b*d_h .. b*d_h + d_h - 1);
+ *   conv_state: [B, M, state_len, d_h].
+ * M = 1 is the single-branch layer, with the layouts stated at each entry point. */
 
 /* engram_config.flags */
 #define ENGRAM_FLAG_FUSED_GATE 0x1 /* prefill with kernel 4 / dilation 3 and d_h % 256 == 0:
                                       run projections, gate and conv in ONE persistent kernel
                                       (the conv pass rides in the projection's epilogue warps).
                                       Results match the two-kernel path within tolerance; it is
-                                      opt-in because it is currently slower on B200. */
+                                      opt-in because it is currently slower on B200.  Single
+                                      branch only (num_branches <= 1). */
 
 /* Validated config plus derived constants.  Caller-owned, plain data: engram_init fills
  * it, every other call reads it.  Do not modify its fields. */
@@ -118,12 +134,13 @@ typedef struct engram_plan {
     int32_t hist_len;    /* largest order - 1 */
     int32_t state_len;   /* (conv_kernel - 1) * conv_dilation */
     uint32_t magic;
-    int32_t reserved[3];
+    int32_t num_branches; /* M >= 1 */
+    int32_t reserved[2];
 } engram_plan;
 
 /* Weights of the gate and conv (device pointers, bf16 patterns). */
 typedef struct engram_weights {
-    const uint16_t *w_k;     /* [d_h, d_m], row r = output channel r */
+    const uint16_t *w_k;     /* [M*d_h, d_m], row r = output channel r (M = 1: [d_h, d_m]) */
     const uint16_t *w_v;     /* [d_h, d_m] */
     const uint16_t *gamma_q; /* [d_h] RMSNorm gain of the query (hidden state) */
     const uint16_t *gamma_k; /* [d_h] RMSNorm gain of the key */

@@ -8,5 +8,5 @@ links or calls anything here, and nothing here calls the CUDA library.
 from .oracle import (  # noqa: F401
     build, lib, splitmix64, fmix64, hash_multiplier, hash_gram, bf16_to_double,
     double_to_bf16, remap, hash_ids, advance_history, gather, gate_conv, forward,
-    e4m3_to_double, dequant_e4m3, dequant_table,
+    e4m3_to_double, dequant_e4m3, dequant_table, forward_branches,
 )

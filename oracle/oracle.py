@@ -259,3 +259,42 @@ def forward(ids, remap_table, tables, h, Wk, Wv, gamma_q, gamma_k, gamma_c, conv
         res["state"] = st
         res["history"] = hist_out
     return res
+
+
+def forward_branches(ids, remap_table, tables, h, Wk, Wv, gamma_q, gamma_k, gamma_c, conv_w, *,
+                     orders, K: int, primes, seed: int, pad_id: int, eps: float = 1e-6,
+                     history=None, conv_state=None, decode_outputs: bool = False, table_scales=None):
+    """The multi-branch layer [yktysq, component 4: the branches share the embedding table and
+    the value projection, and each has its own key projection, so that each branch gates the
+    memory in its own way].  Every branch b is the single-branch layer on its own hidden state
+    h[:, b] and key projection Wk[b*d_h:(b+1)*d_h], with the same memory vector m, W_v, gains
+    and conv weights; its conv state (decode) is conv_state[:, b].
+
+    h: [B*T, M, d_h]; Wk: [M*d_h, d_m]; conv_state: None or [B, M, S, d_h].
+    Returns dict(out [B*T, M, d_h], delta, gate [B*T, M], idx[, state [B, M, S, d_h], history]).
+    """
+    ids = _c(ids, np.int32)
+    B, T = ids.shape
+    h = _c(h, np.uint16)
+    n, M, d_h = h.shape
+    Wk = _c(Wk, np.uint16)
+    assert Wk.shape[0] == M * d_h
+    dil = int(max(orders))
+    hist_len = dil - 1
+    xr = remap(ids, remap_table)
+    idx = hash_ids(xr, orders, K, primes, seed, pad_id, history=history)
+    m = gather(idx, tables, table_scales)
+    outs, deltas, gates, states = [], [], [], []
+    for b in range(M):
+        cs = None if conv_state is None else _c(conv_state, np.uint16)[:, b]
+        r = gate_conv(h[:, b], m, Wk[b * d_h:(b + 1) * d_h], Wv, gamma_q, gamma_k, gamma_c, conv_w, B, T,
+                      dil=dil, eps=eps, conv_state=cs, want_state=decode_outputs)
+        outs.append(r["out"])
+        deltas.append(r["delta"])
+        gates.append(r["gate"])
+        states.append(r["state"])
+    res = dict(out=np.stack(outs, axis=1), delta=np.stack(deltas, axis=1), gate=np.stack(gates, axis=1), idx=idx)
+    if decode_outputs:
+        res["state"] = np.stack(states, axis=1)
+        res["history"] = advance_history(xr, history, hist_len, pad_id)
+    return res

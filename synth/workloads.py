@@ -67,6 +67,7 @@ class Workload:
     sigma_conv: float = 0.25
     index: int = 0
     table_dtype: str = "bf16"  # bf16 | fp8 (e4m3 codes with one dequantisation scale per table)
+    branches: int = 1          # M: residual-stream branches, each with its own key projection
 
     @property
     def H(self) -> int:
@@ -79,6 +80,11 @@ class Workload:
     @property
     def n_tok(self) -> int:
         return self.B * self.T
+
+    @property
+    def h_rows(self) -> int:
+        """Rows of the hidden-state (and output) matrix: one per (token, branch)."""
+        return self.n_tok * self.branches
 
     @property
     def conv_dilation(self) -> int:
@@ -122,6 +128,7 @@ class Workload:
         return fp8_scale_for_sigma(self.table_sigma(h))
 
     def wk_spec(self) -> FillSpec:
+        """W_k as [branches * d_h, d_m] (the key projections of the branches stacked)."""
         return FillSpec(self.seeds()["weights"], T_WK, self.sigma_w)
 
     def wv_spec(self) -> FillSpec:
@@ -202,6 +209,14 @@ WORKLOADS = {
     # the pages' own geometry: 8 two-gram + 8 three-gram heads, ~20M rows per table, 160
     # values per row (16 x 20M x 160 = 51.2B parameters, ~102 GB): small rows spread over a
     # huge table, the hardest case for DRAM efficiency of the row gather
+    # the layer2560 workload on a 4-branch residual stream: tables, memory vectors and the
+    # value projection shared, one key projection per branch
+    "layer2560x4": Workload(
+        name="layer2560x4", index=6,
+        description="as layer2560 with 4 residual-stream branches (hidden states [32768, 4, 2560], "
+                    "4 key projections, shared value projection)",
+        vocab_in=128_000, vocab_out=98_560, B=8, T=4096, orders=(2, 3), K=8,
+        primes=(P_1M,) * 16, d_e=160, d_h=2560, branches=4),
     "ngram16x20m": Workload(
         name="ngram16x20m", index=5,
         description="vocab 248,320 (no compression); 8x4096 Zipf(1.1); orders {2,3}, K=8; "

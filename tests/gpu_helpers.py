@@ -64,8 +64,9 @@ class DeviceInputs:
             fill = fill_gpu.filled_fp8 if wl.table_dtype == "fp8" else fill_gpu.filled
             tables = [fill((wl.primes[h], wl.d_e), wl.table_spec(h), device) for h in range(wl.H)]
         self.tables = tables
-        self.h = fill_gpu.filled((wl.n_tok, wl.d_h), wl.h_spec(step), device)
-        self.w_k = fill_gpu.filled((wl.d_h, wl.d_m), wl.wk_spec(), device)
+        M = wl.branches
+        self.h = fill_gpu.filled((wl.h_rows, wl.d_h), wl.h_spec(step), device)
+        self.w_k = fill_gpu.filled((M * wl.d_h, wl.d_m), wl.wk_spec(), device)
         self.w_v = fill_gpu.filled((wl.d_h, wl.d_m), wl.wv_spec(), device)
         ones = torch.full((wl.d_h,), ONE, dtype=torch.int16, device=device).view(torch.bfloat16)
         self.gamma_q, self.gamma_k, self.gamma_c = ones.clone(), ones.clone(), ones.clone()
@@ -77,12 +78,14 @@ class DeviceInputs:
                 g.copy_((fill_gpu.filled((wl.d_h,), spec, device).float() + 1.0).to(torch.bfloat16))
         self.conv_w = fill_gpu.filled((wl.d_h, wl.conv_kernel), wl.conv_spec(), device)
         self.history = to_dev(wl.history(), device) if wl.decode else None
-        self.conv_state = (fill_gpu.filled((wl.B, wl.state_len, wl.d_h), wl.state_spec(), device)
-                           if wl.decode else None)
+        self.conv_state = (fill_gpu.filled((wl.B * M, wl.state_len, wl.d_h), wl.state_spec(), device)
+                           .view(wl.B, M, wl.state_len, wl.d_h) if wl.decode else None)
+        if self.conv_state is not None and M == 1:
+            self.conv_state = self.conv_state.view(wl.B, wl.state_len, wl.d_h)
         self.plan = E.Plan.from_workload(wl, flags=flags)
         self.weights = E.Weights(self.w_k, self.w_v, self.gamma_q, self.gamma_k, self.gamma_c, self.conv_w)
-        self.out = torch.empty((wl.n_tok, wl.d_h), dtype=torch.bfloat16, device=device)
-        self.delta = torch.empty((wl.n_tok, wl.d_h), dtype=torch.float32, device=device)
+        self.out = torch.empty((wl.h_rows, wl.d_h), dtype=torch.bfloat16, device=device)
+        self.delta = torch.empty((wl.h_rows, wl.d_h), dtype=torch.float32, device=device)
         self.ws = E.alloc_workspace(self.plan, wl.n_tok, device)
 
     def forward(self, delta=True, **kw):

@@ -23,19 +23,23 @@ def small_workload(name="small", *, B=2, T=40, orders=(2, 3), K=2, primes=None, 
 
 
 def make_inputs(wl: Workload, step: int = 0, tables=True):
-    """Host arrays for one call; bf16 tensors are uint16 bit patterns."""
+    """Host arrays for one call; bf16 tensors are uint16 bit patterns.  With M = wl.branches
+    > 1, h is [n_tok, M, d_h], Wk [M*d_h, d_m] and the conv state [B, M, S, d_h]."""
+    M = wl.branches
+    h = fill_bf16(wl.h_spec(step), (wl.h_rows, wl.d_h))
     d = dict(
         ids=wl.ids(step),
         remap=wl.remap(),
-        h=fill_bf16(wl.h_spec(step), (wl.n_tok, wl.d_h)),
-        Wk=fill_bf16(wl.wk_spec(), (wl.d_h, wl.d_m)),
+        h=h.reshape(wl.n_tok, M, wl.d_h) if M > 1 else h,
+        Wk=fill_bf16(wl.wk_spec(), (M * wl.d_h, wl.d_m)),
         Wv=fill_bf16(wl.wv_spec(), (wl.d_h, wl.d_m)),
         gamma_q=np.full(wl.d_h, ONE_BF16, dtype=np.uint16),
         gamma_k=np.full(wl.d_h, ONE_BF16, dtype=np.uint16),
         gamma_c=np.full(wl.d_h, ONE_BF16, dtype=np.uint16),
         conv_w=fill_bf16(wl.conv_spec(), (wl.d_h, wl.conv_kernel)),
         history=wl.history(),
-        conv_state=fill_bf16(wl.state_spec(), (wl.B, wl.state_len, wl.d_h)) if wl.decode else None,
+        conv_state=(fill_bf16(wl.state_spec(), (wl.B * M, wl.state_len, wl.d_h)).reshape(
+            (wl.B, M, wl.state_len, wl.d_h) if M > 1 else (wl.B, wl.state_len, wl.d_h)) if wl.decode else None),
     )
     if tables:
         d["tables"] = [fill_bf16(wl.table_spec(h), (wl.primes[h], wl.d_e)) for h in range(wl.H)]

@@ -63,6 +63,9 @@ def _plan(**kw):
     (dict(table_dtype=1, table_scale=(0.1, 2.0 ** 101, 0.1, 0.1)), E.ENGRAM_ERR_INVALID_ARG),   # leave fp32
     (dict(table_dtype=0, table_scale=(0.1,)), E.ENGRAM_ERR_INVALID_ARG),       # scale on bf16
     (dict(table_dtype=1, table_scale=(0.1,) * 4, row_dim=24), E.ENGRAM_ERR_UNSUPPORTED),
+    (dict(num_branches=9), E.ENGRAM_ERR_UNSUPPORTED),
+    (dict(num_branches=-1), E.ENGRAM_ERR_UNSUPPORTED),
+    (dict(num_branches=2, flags=E.ENGRAM_FLAG_FUSED_GATE), E.ENGRAM_ERR_UNSUPPORTED),
 ])
 def test_init_rejects_bad_configs(kw, code):
     with pytest.raises(E.EngramError) as ei:
@@ -138,3 +141,15 @@ def test_product_has_no_oracle_dependency():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(root, f), encoding="utf-8").read()
                 assert "import oracle" not in text and "from oracle" not in text and "liboracle" not in text
+
+
+def test_branches_default_and_workspace_growth():
+    assert _plan(num_branches=0).num_branches == 1      # a zeroed field reads as one branch
+    assert _plan().num_branches == 1
+    p1, p4 = _plan(num_branches=1), _plan(num_branches=4)
+    assert p4.num_branches == 4 and p4.mem_dim == p1.mem_dim
+    # more key tiles (partial sums) and per-branch gate scalars
+    assert E.engram_workspace_size(p4, 4096) > E.engram_workspace_size(p1, 4096)
+    wl = synth.get_workload("layer2560x4")
+    assert E.Plan.from_workload(wl).num_branches == 4 and wl.h_rows == 4 * wl.n_tok
+

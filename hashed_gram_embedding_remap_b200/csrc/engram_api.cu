@@ -525,10 +525,12 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
         p.scal = scal;
     }
     if (p.scal != nullptr) {
-        constexpr int kChain4 = 16;   // 48-token chunks, 4 channels per thread
-        dim3 grid4(static_cast<unsigned>((T + 3 * kChain4 - 1) / (3 * kChain4)) * p.M, static_cast<unsigned>(B),
-                   static_cast<unsigned>((d_h / 4 + engram::kGate4Threads - 1) / engram::kGate4Threads));
-        engram::gate_conv_k4d3_c4_kernel<kChain4><<<grid4, engram::kGate4Threads, 0, stream>>>(p);
+        // 36-token chunks (12 outputs per residue chain), 4 channels per thread, registers
+        // capped for 5 CTAs per SM: more resident warps hide more of the load latency
+        constexpr int kChain4 = 12;
+        const dim3 grid4(static_cast<unsigned>((T + 3 * kChain4 - 1) / (3 * kChain4)) * p.M, static_cast<unsigned>(B),
+                         static_cast<unsigned>((d_h / 4 + engram::kGate4Threads - 1) / engram::kGate4Threads));
+        engram::gate_conv_k4d3_c4_kernel<kChain4, engram::kGate4MinBlocks><<<grid4, engram::kGate4Threads, 0, stream>>>(p);
         ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_conv_k4d3_c4_kernel launch");
         return ENGRAM_OK;
     }

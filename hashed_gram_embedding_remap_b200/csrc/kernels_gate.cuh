@@ -410,15 +410,17 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
     }
 }
 
-// Prefill-only variant of gate_conv_k4d3_kernel with 4 channels per thread (8-byte bf16
-// loads, half the per-element address and predicate work) and 3*CH-token chunks.  Needs the
+// Prefill-only variant of gate_conv_k4d3_kernel with 4 channels per thread (8-byte loads,
+// half the per-element address and predicate work) and 3*CH-token chunks.  The kernel is
+// latency-bound: MINB caps the registers so that more CTAs stay resident.  Needs the
 // per-token scalars from gate_scalars_kernel.  Grid: (token chunks x M branches, branch
 // fastest so that the branches of a chunk read its shared v rows while they are in L2; B;
 // channel slices).
 constexpr int kGate4Threads = 128;
+constexpr int kGate4MinBlocks = 5;   // register cap for 5 resident CTAs per SM (96 registers)
 
-template <int CH>
-__global__ void __launch_bounds__(kGate4Threads) gate_conv_k4d3_c4_kernel(const __grid_constant__ GateParams p) {
+template <int CH, int MINB>
+__global__ void __launch_bounds__(kGate4Threads, MINB) gate_conv_k4d3_c4_kernel(const __grid_constant__ GateParams p) {
     constexpr int KS = 4, DIL = 3, HALO = (KS - 1) * DIL, TC = CH * DIL;
     __shared__ float2 s_sc[TC + HALO];          // (g, beta) per token of [t0 - HALO, t1)
     const int b = blockIdx.y;

@@ -525,13 +525,30 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
         p.scal = scal;
     }
     if (p.scal != nullptr) {
-        // 36-token chunks (12 outputs per residue chain), 4 channels per thread, registers
-        // capped for 5 CTAs per SM: more resident warps hide more of the load latency
-        constexpr int kChain4 = 12;
-        const dim3 grid4(static_cast<unsigned>((T + 3 * kChain4 - 1) / (3 * kChain4)) * p.M, static_cast<unsigned>(B),
-                         static_cast<unsigned>((d_h / 4 + engram::kGate4Threads - 1) / engram::kGate4Threads));
-        engram::gate_conv_k4d3_c4_kernel<kChain4, engram::kGate4MinBlocks><<<grid4, engram::kGate4Threads, 0, stream>>>(p);
-        ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_conv_k4d3_c4_kernel launch");
+        // streaming kernel: 9*G tokens per CTA, G chosen so that the last wave of CTAs is
+        // as full as possible
+        const int slices = (d_h / 4 + engram::kStreamThreads - 1) / engram::kStreamThreads;
+        const int64_t per_wave = static_cast<int64_t>(sm_count()) * engram::kStreamMinBlocks;
+        int best_g = 16;
+        double best_eff = -1.0;
+        for (int g : {16, 12, 8}) {
+            const int64_t ctas = static_cast<int64_t>((T + 9 * g - 1) / (9 * g)) * p.M * B * slices;
+            const double waves = static_cast<double>(ctas) / static_cast<double>(per_wave);
+            const double eff = waves / std::ceil(waves);
+            if (eff > best_eff + 0.05) {
+                best_eff = eff;
+                best_g = g;
+            }
+        }
+        const dim3 grid(static_cast<unsigned>((T + 9 * best_g - 1) / (9 * best_g)) * p.M * slices,
+                        static_cast<unsigned>(B));
+        using SK = void (*)(const engram::GateParams);
+        const bool dl = delta != nullptr;
+        const SK k = best_g == 16 ? (dl ? engram::gate_stream_kernel<16, true> : engram::gate_stream_kernel<16, false>)
+                   : best_g == 12 ? (dl ? engram::gate_stream_kernel<12, true> : engram::gate_stream_kernel<12, false>)
+                                  : (dl ? engram::gate_stream_kernel<8, true> : engram::gate_stream_kernel<8, false>);
+        k<<<grid, engram::kStreamThreads, 0, stream>>>(p);
+        ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_stream_kernel launch");
         return ENGRAM_OK;
     }
     if (fast) engram::gate_conv_k4d3_kernel<kChain><<<grid, threads, 0, stream>>>(p);

@@ -410,100 +410,125 @@ __global__ void __launch_bounds__(kGateFastThreads, 3) gate_conv_k4d3_kernel(con
     }
 }
 
-// Prefill-only variant of gate_conv_k4d3_kernel with 4 channels per thread (8-byte loads,
-// half the per-element address and predicate work) and 3*CH-token chunks.  The kernel is
-// latency-bound: MINB caps the registers so that more CTAs stay resident.  Needs the
-// per-token scalars from gate_scalars_kernel.  Grid: (token chunks x M branches, branch
-// fastest so that the branches of a chunk read its shared v rows while they are in L2; B;
-// channel slices).
-constexpr int kGate4Threads = 128;
-constexpr int kGate4MinBlocks = 5;   // register cap for 5 resident CTAs per SM (96 registers)
+// Prefill, kernel 4 / dilation 3, streaming form: a CTA owns 9*G consecutive tokens of one
+// (sequence, branch) and 512 channels (4 per thread); each thread walks its tokens in order.
+// Two 9-slot register rings replace a per-residue (t mod 3) decomposition: `ur` holds the
+// conv inputs u of the last 9 positions (slot = position mod 9, so the taps t-3, t-6, t-9 sit
+// in static slots of the unrolled loop), and the load ring holds (v, h) of the next 9
+// positions -- the slot of token t is refilled with token t+9 as soon as t has read it, so
+// every thread keeps 9 tokens of loads in flight instead of alternating load and compute
+// phases.  The first group of 9 is the conv halo before the chunk (conv inputs only).
+// Channel pairs go through the packed fp32x2 pipe (FFMA2 / FMUL2 / FADD2), about 8
+// instructions per element; gamma_c is folded into the conv taps (u' = beta v, taps
+// w_i gamma_c).  The kernel is issue- and latency-bound at 4 resident CTAs per SM (128
+// registers).  Needs the per-(token, branch) scalars of gate_scalars_kernel.
+constexpr int kStreamThreads = 128;
+constexpr int kStreamMinBlocks = 4;
 
-template <int CH, int MINB>
-__global__ void __launch_bounds__(kGate4Threads, MINB) gate_conv_k4d3_c4_kernel(const __grid_constant__ GateParams p) {
-    constexpr int KS = 4, DIL = 3, HALO = (KS - 1) * DIL, TC = CH * DIL;
-    __shared__ float2 s_sc[TC + HALO];          // (g, beta) per token of [t0 - HALO, t1)
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 half2_to_f2(uint32_t w) {
+    return __half22float2(*reinterpret_cast<const __half2 *>(&w));
+}
+__device__ __forceinline__ float2 bf162_to_f2(uint32_t w) { return make_float2(bf16_lo(w), bf16_hi(w)); }
+// x * sigmoid(x) = h + h * tanh(h), h = x / 2, per pair (hardware tanh approximation)
+__device__ __forceinline__ float2 silu2(float2 x) {
+    const float2 h = __fmul2_rn(x, f2(0.5f));
+    float2 t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t.x) : "f"(h.x));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t.y) : "f"(h.y));
+    return __ffma2_rn(h, t, h);
+}
+
+template <int G, bool DELTA>
+__global__ void __launch_bounds__(kStreamThreads, kStreamMinBlocks) gate_stream_kernel(const __grid_constant__ GateParams p) {
+    constexpr int R = 9;                       // ring length = conv halo (kernel 4, dilation 3)
+    constexpr int TC = R * G;                  // tokens per CTA
+    __shared__ float2 s_sc[TC + R];            // (g, beta) per token of [t0 - 9, t0 + TC)
+    // blockIdx.x = (chunk, branch, channel slice), slice fastest
+    const int n_slices = (p.d_h / 4 + kStreamThreads - 1) / kStreamThreads;
+    const int slice = static_cast<int>(blockIdx.x % n_slices);
+    const int bx = static_cast<int>(blockIdx.x / n_slices);
     const int b = blockIdx.y;
-    const int br = static_cast<int>(blockIdx.x % p.M);
-    const int t0 = static_cast<int>(blockIdx.x / p.M) * TC;
+    const int br = bx % p.M;
+    const int t0 = (bx / p.M) * TC;
     if (t0 >= p.T) return;
     const int t1 = min(p.T, t0 + TC);
-    const int lo = t0 - HALO;
+    const int lo = t0 - R;
     const int64_t row0 = static_cast<int64_t>(b) * p.T;
-    const int64_t hstride = static_cast<int64_t>(p.M) * p.d_h;   // h / out / delta token stride
-    for (int i = threadIdx.x; i < TC + HALO; i += kGate4Threads) {
+    for (int i = threadIdx.x; i < TC + R; i += kStreamThreads) {
         const int t = lo + i;
         s_sc[i] = (t >= 0 && t < t1) ? __ldg(p.scal + (row0 + t) * p.M + br) : make_float2(0.f, 0.f);
     }
     __syncthreads();
-    const int q = blockIdx.z * blockDim.x + threadIdx.x;
+    const int q = slice * kStreamThreads + threadIdx.x;
     if (q >= p.d_h / 4) return;
     const int c = q * 4;
-    float gc[4], w[4][KS];
-    {
-        const uint2 gw = __ldg(reinterpret_cast<const uint2 *>(p.gamma_c + c));
-        gc[0] = bf16_lo(gw.x); gc[1] = bf16_hi(gw.x); gc[2] = bf16_lo(gw.y); gc[3] = bf16_hi(gw.y);
-        const uint4 *wp = reinterpret_cast<const uint4 *>(p.conv_w + c * KS);   // 4 channels x 4 taps
-        const uint4 w01 = __ldg(wp), w23 = __ldg(wp + 1);
-        const uint32_t ww[8] = {w01.x, w01.y, w01.z, w01.w, w23.x, w23.y, w23.z, w23.w};
+    float2 w[4][2];   // [tap][channel pair] = conv tap x gamma_c
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            w[e][0] = bf16_lo(ww[2 * e]); w[e][1] = bf16_hi(ww[2 * e]);
-            w[e][2] = bf16_lo(ww[2 * e + 1]); w[e][3] = bf16_hi(ww[2 * e + 1]);
-        }
+    for (int k = 0; k < 2; ++k) {
+        const uint32_t gw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_c + c + 2 * k));
+        const uint4 ww = __ldg(reinterpret_cast<const uint4 *>(p.conv_w + (c + 2 * k) * 4));   // 2 channels x 4 taps
+        const float g0 = bf16_lo(gw), g1 = bf16_hi(gw);
+        w[0][k] = make_float2(bf16_lo(ww.x) * g0, bf16_lo(ww.z) * g1);
+        w[1][k] = make_float2(bf16_hi(ww.x) * g0, bf16_hi(ww.z) * g1);
+        w[2][k] = make_float2(bf16_lo(ww.y) * g0, bf16_lo(ww.w) * g1);
+        w[3][k] = make_float2(bf16_hi(ww.y) * g0, bf16_hi(ww.w) * g1);
     }
+    const int64_t hstride = static_cast<int64_t>(p.M) * p.d_h;   // h / out / delta token stride
     const uint16_t *vbase = p.v + row0 * p.d_h + c;
-    const uint16_t *hbase = p.h + (row0 * p.M + br) * p.d_h + c;
+    const int64_t hoff = (row0 * p.M + br) * p.d_h + c;
+    const uint16_t *hbase = p.h + hoff;
+    uint16_t *obase = p.out + hoff;
+
+    uint2 lv[R], lh[R];     // load ring: (v, h) of the token in each slot
+    float2 ur[R][2];        // conv-input ring: u' of the last 9 positions, slot = position mod 9
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+        const int t = lo + j;   // halo: conv inputs only
+        lv[j] = (t >= 0) ? __ldg(reinterpret_cast<const uint2 *>(vbase + static_cast<int64_t>(t) * p.d_h))
+                         : make_uint2(0u, 0u);
+        lh[j] = make_uint2(0u, 0u);
+        ur[j][0] = ur[j][1] = make_float2(0.f, 0.f);
+    }
 #pragma unroll 1
-    for (int r = 0; r < DIL; ++r) {
-        uint2 vv[CH + KS - 1];
-        uint2 hh[CH];
+    for (int gi = 0; gi <= G; ++gi) {
+        const int tb = lo + R * gi;
 #pragma unroll
-        for (int j = 0; j < CH + KS - 1; ++j) {
-            const int t = lo + r + DIL * j;
-            vv[j] = (t >= 0 && t < t1) ? __ldg(reinterpret_cast<const uint2 *>(vbase + static_cast<int64_t>(t) * p.d_h))
-                                       : make_uint2(0u, 0u);
-        }
-#pragma unroll
-        for (int j = 0; j < CH; ++j) {
-            const int t = t0 + r + DIL * j;
-            hh[j] = t < t1 ? __ldg(reinterpret_cast<const uint2 *>(hbase + static_cast<int64_t>(t) * hstride))
-                           : make_uint2(0u, 0u);
-        }
-        float u[KS][4];
-#pragma unroll
-        for (int i = 0; i < KS; ++i)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) u[i][e] = 0.f;
-#pragma unroll
-        for (int j = 0; j < CH + KS - 1; ++j) {
-            const int si = r + DIL * j;
-            const float2 sc = s_sc[si];
-            const float vj[4] = {v_lo(vv[j].x), v_hi(vv[j].x), v_lo(vv[j].y), v_hi(vv[j].y)};
-#pragma unroll
-            for (int i = KS - 1; i > 0; --i)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) u[i][e] = u[i - 1][e];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) u[0][e] = sc.y * vj[e] * gc[e];
-            if (j < KS - 1) continue;
-            const int t = lo + si;
-            if (t >= t1) continue;
-            const uint2 hw = hh[j - (KS - 1)];
-            const float hv[4] = {bf16_lo(hw.x), bf16_hi(hw.x), bf16_lo(hw.y), bf16_hi(hw.y)};
-            float dl[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                float acc = w[e][0] * u[0][e];
-#pragma unroll
-                for (int i = 1; i < KS; ++i) acc = fmaf(w[e][i], u[i][e], acc);
-                dl[e] = fmaf(sc.x, vj[e], silu_fast(acc));
+        for (int j = 0; j < R; ++j) {
+            const int t = tb + j;
+            const uint2 vw = lv[j], hw = lh[j];
+            // refill the slot with token t + 9 (the next group)
+            const int tn = t + R;
+            if (gi < G) {
+                lv[j] = (tn < t1) ? __ldg(reinterpret_cast<const uint2 *>(vbase + static_cast<int64_t>(tn) * p.d_h))
+                                  : make_uint2(0u, 0u);
+                lh[j] = (tn < t1) ? __ldg(reinterpret_cast<const uint2 *>(hbase + static_cast<int64_t>(tn) * hstride))
+                                  : make_uint2(0u, 0u);
             }
-            const int64_t nr = (row0 + t) * p.M + br;   // row of (token, branch)
-            *reinterpret_cast<uint2 *>(p.out + nr * p.d_h + c) =
-                make_uint2(pack_bf16x2(hv[0] + dl[0], hv[1] + dl[1]), pack_bf16x2(hv[2] + dl[2], hv[3] + dl[3]));
-            if (p.delta != nullptr)
-                *reinterpret_cast<float4 *>(p.delta + nr * p.d_h + c) = make_float4(dl[0], dl[1], dl[2], dl[3]);
+            const float2 sc = s_sc[t - lo];
+            const float2 vj[2] = {half2_to_f2(vw.x), half2_to_f2(vw.y)};
+            const float2 un[2] = {__fmul2_rn(f2(sc.y), vj[0]), __fmul2_rn(f2(sc.y), vj[1])};
+            if (gi > 0 && t < t1) {
+                const uint32_t hh[2] = {hw.x, hw.y};
+                float2 dl[2];
+                uint32_t ob[2];
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    float2 acc = __fmul2_rn(w[0][k], un[k]);
+                    acc = __ffma2_rn(w[1][k], ur[(j + 6) % R][k], acc);   // t - 3
+                    acc = __ffma2_rn(w[2][k], ur[(j + 3) % R][k], acc);   // t - 6
+                    acc = __ffma2_rn(w[3][k], ur[j][k], acc);             // t - 9
+                    dl[k] = __ffma2_rn(f2(sc.x), vj[k], silu2(acc));     // U + SiLU(conv)
+                    const float2 o = __fadd2_rn(bf162_to_f2(hh[k]), dl[k]);
+                    ob[k] = pack_bf16x2(o.x, o.y);
+                }
+                const int64_t off = static_cast<int64_t>(t) * hstride;
+                *reinterpret_cast<uint2 *>(obase + off) = make_uint2(ob[0], ob[1]);
+                if constexpr (DELTA)
+                    *reinterpret_cast<float4 *>(p.delta + hoff + off) = make_float4(dl[0].x, dl[0].y, dl[1].x, dl[1].y);
+            }
+            ur[j][0] = un[0];
+            ur[j][1] = un[1];
         }
     }
 }

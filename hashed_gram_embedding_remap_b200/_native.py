@@ -87,6 +87,15 @@ class engram_weights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("w_k", "w_v", "gamma_q", "gamma_k", "gamma_c", "conv_w")]
 
 
+class engram_row_cache(C.Structure):
+    _fields_ = [
+        ("data", C.c_void_p * ENGRAM_MAX_TABLES),
+        ("tags", C.c_void_p * ENGRAM_MAX_TABLES),
+        ("claim", C.c_void_p * ENGRAM_MAX_TABLES),
+        ("slots", C.c_int64),
+    ]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"CUDA library not built: {LIB_PATH} is missing "
@@ -102,6 +111,8 @@ def _load():
         "engram_gather": (C.c_int, [P, P, P, i64, P, P]),
         "engram_stage_rows": (C.c_int, [P, P, i64, P, P, i32, P, P, P, P]),
         "engram_gather_bounded": (C.c_int, [P, P, P, i64, i64, P, P]),
+        "engram_row_cache_reset": (C.c_int, [P, P, P]),
+        "engram_stage_rows_cached": (C.c_int, [P, P, i64, P, P, P, i32, P, P, P, P, P, P]),
         "engram_gate_conv": (C.c_int, [P, P, P, P, i32, i32, P, P, P, P, sz, P]),
         "engram_forward": (C.c_int, [P, P, P, P, P, i32, i32, P, P, P, P, P, P, sz, P, P]),
         "engram_gate_conv_noalloc": (C.c_int, [P, P, P, P, i32, i32, P, P, P, P]),
@@ -115,7 +126,7 @@ def _load():
         f.restype = res
         f.argtypes = args
     for name, cls in (("engram_config", engram_config), ("engram_plan", engram_plan),
-                      ("engram_weights", engram_weights)):
+                      ("engram_weights", engram_weights), ("engram_row_cache", engram_row_cache)):
         n = L.engram_sizeof(name.encode())
         if n != C.sizeof(cls):
             raise ImportError(f"ABI mismatch: sizeof({name}) is {n} in the library, {C.sizeof(cls)} here")
@@ -313,6 +324,51 @@ def _check_rows(plan: Plan, n_tok: int, **tensors):
         if t is not None and t.numel() != want:
             raise ValueError(f"{name} has {t.numel()} elements; {n_tok} tokens x {plan.num_branches} branches x "
                              f"{plan.cfg.hidden_dim} need {want}")
+
+
+class RowCache:
+    """Device buffers of an HBM row cache (engram_row_cache) for the plan's tables: per table
+    `slots` rows of the table element type, uint32 tags and claims.  Created empty."""
+
+    def __init__(self, plan: Plan, slots: int, device="cuda", stream=None):
+        if slots < 1 or slots & (slots - 1):
+            raise ValueError("slots must be a power of two")
+        elem = torch.uint8 if plan.cfg.table_dtype == ENGRAM_TABLE_FP8_E4M3 else torch.bfloat16
+        H, d_e = plan.num_tables, plan.cfg.row_dim
+        self.data = [torch.empty((slots, d_e), dtype=elem, device=device) for _ in range(H)]
+        self.tags = [torch.empty((slots,), dtype=torch.int32, device=device) for _ in range(H)]
+        self.claim = [torch.empty((slots,), dtype=torch.int32, device=device) for _ in range(H)]
+        self.struct = engram_row_cache()
+        for hh in range(H):
+            self.struct.data[hh] = self.data[hh].data_ptr()
+            self.struct.tags[hh] = self.tags[hh].data_ptr()
+            self.struct.claim[hh] = self.claim[hh].data_ptr()
+        self.struct.slots = int(slots)
+        self.plan = plan
+        self.reset(stream)
+
+    def reset(self, stream=None):
+        _check(lib.engram_row_cache_reset(self.plan, C.byref(self.struct), _stream(stream)))
+
+    @property
+    def _as_parameter_(self):
+        return C.byref(self.struct)
+
+
+def engram_stage_rows_cached(plan: Plan, idx: torch.Tensor, tables, cache: RowCache, staging,
+                             staged_idx: torch.Tensor, unique_rows: torch.Tensor, n_unique: torch.Tensor,
+                             row_flags: torch.Tensor, n_hits: torch.Tensor, stream=None):
+    """engram_stage_rows with the HBM row cache in front of the (host-mapped) tables; n_hits
+    accumulates the distinct rows served from the cache."""
+    n_tok = idx.shape[0]
+    cap = staging[0].shape[0]
+    _check(lib.engram_stage_rows_cached(plan, _ptr(idx, (torch.int32, torch.uint32), "idx"), n_tok,
+                                        _table_array(tables, plan), cache, _table_array(staging, plan), cap,
+                                        _ptr(staged_idx, (torch.int32, torch.uint32), "staged_idx"),
+                                        _ptr(unique_rows, (torch.int32, torch.uint32), "unique_rows"),
+                                        _ptr(n_unique, torch.int32, "n_unique"),
+                                        _ptr(row_flags, (torch.int32, torch.uint32), "row_flags"),
+                                        _ptr(n_hits, torch.int32, "n_hits"), _stream(stream)))
 
 
 def engram_gate_conv(plan: Plan, weights: Weights, h: torch.Tensor, m: torch.Tensor, B: int, T: int,

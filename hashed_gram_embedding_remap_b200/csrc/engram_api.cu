@@ -559,7 +559,8 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
 
 int launch_stage(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, const void *const *tables,
                  void *const *staging, int32_t capacity, uint32_t *staged_idx, uint32_t *unique_rows,
-                 int32_t *n_unique, cudaStream_t stream) {
+                 int32_t *n_unique, cudaStream_t stream, const engram_row_cache *cache = nullptr,
+                 uint32_t *row_flags = nullptr, int32_t *n_hits = nullptr) {
     const int H = plan->num_tables;
     int N = 1;
     while (N < n_tok) N <<= 1;
@@ -588,8 +589,46 @@ int launch_stage(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, co
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    engram::stage_copy_kernel<kUnroll><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "stage_copy_kernel launch");
+    if (cache == nullptr) {
+        engram::stage_copy_kernel<kUnroll><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+        ENGRAM_CUDA_TRY(cudaGetLastError(), "stage_copy_kernel launch");
+        return ENGRAM_OK;
+    }
+    engram::CacheParams cp{};
+    for (int h = 0; h < H; ++h) {
+        cp.data[h] = cache->data[h];
+        cp.tags[h] = cache->tags[h];
+        cp.claim[h] = cache->claim[h];
+        cp.rows[h] = static_cast<uint64_t>(plan->cfg.table_rows[h]);
+    }
+    cp.slot_mask = static_cast<uint64_t>(cache->slots) - 1;
+    cp.unique_rows = unique_rows;
+    cp.n_unique = n_unique;
+    cp.flags = row_flags;
+    cp.n_hits = n_hits;
+    cp.H = H;
+    cp.capacity = capacity;
+    const dim3 rgrid(static_cast<unsigned>((n_tok + 255) / 256), static_cast<unsigned>(H));
+    engram::cache_probe_kernel<<<rgrid, 256, 0, stream>>>(cp);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "cache_probe_kernel launch");
+    engram::cache_decide_kernel<<<rgrid, 256, 0, stream>>>(cp);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "cache_decide_kernel launch");
+    engram::cache_copy_kernel<kUnroll><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p, cp);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "cache_copy_kernel launch");
+    engram::cache_commit_kernel<<<rgrid, 256, 0, stream>>>(cp);
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "cache_commit_kernel launch");
+    return ENGRAM_OK;
+}
+
+int check_row_cache(const engram_plan *plan, const engram_row_cache *cache) {
+    if (cache == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "cache is NULL");
+    if (cache->slots < 1 || cache->slots > (int64_t(1) << 32) || (cache->slots & (cache->slots - 1)))
+        return fail(ENGRAM_ERR_INVALID_ARG, "cache slots must be a power of two in [1, 2^32]");
+    for (int h = 0; h < plan->num_tables; ++h) {
+        if (!cache->data[h] || !cache->tags[h] || !cache->claim[h])
+            return fail(ENGRAM_ERR_INVALID_ARG, "cache buffers of table %d are NULL", h);
+        if (!aligned16(cache->data[h])) return fail(ENGRAM_ERR_INVALID_ARG, "cache data of table %d not 16-byte aligned", h);
+    }
     return ENGRAM_OK;
 }
 
@@ -735,6 +774,7 @@ size_t engram_sizeof(const char *type_name) {
     if (std::strcmp(type_name, "engram_config") == 0) return sizeof(engram_config);
     if (std::strcmp(type_name, "engram_plan") == 0) return sizeof(engram_plan);
     if (std::strcmp(type_name, "engram_weights") == 0) return sizeof(engram_weights);
+    if (std::strcmp(type_name, "engram_row_cache") == 0) return sizeof(engram_row_cache);
     return 0;
 }
 
@@ -908,6 +948,43 @@ int engram_stage_rows(const engram_plan *plan, const uint32_t *idx, int64_t n_to
     }
     return launch_stage(plan, idx, n_tok, tables, staging, capacity, staged_idx, unique_rows, n_unique,
                         static_cast<cudaStream_t>(stream));
+}
+
+int engram_row_cache_reset(const engram_plan *plan, const engram_row_cache *cache, engram_stream_t stream) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if ((rc = check_row_cache(plan, cache)) != ENGRAM_OK) return rc;
+    for (int h = 0; h < plan->num_tables; ++h) {
+        int64_t blocks = (cache->slots + 255) / 256;
+        if (blocks > 148 * 16) blocks = 148 * 16;
+        engram::cache_reset_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+            cache->tags[h], cache->claim[h], cache->slots);
+        ENGRAM_CUDA_TRY(cudaGetLastError(), "cache_reset_kernel launch");
+    }
+    return ENGRAM_OK;
+}
+
+int engram_stage_rows_cached(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, const void *const *tables,
+                             const engram_row_cache *cache, void *const *staging, int32_t capacity,
+                             uint32_t *staged_idx, uint32_t *unique_rows, int32_t *n_unique, uint32_t *row_flags,
+                             int32_t *n_hits, engram_stream_t stream) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if (n_tok < 0) return fail(ENGRAM_ERR_INVALID_ARG, "n_tok must be >= 0");
+    if (n_tok == 0) return ENGRAM_OK;
+    if ((rc = check_row_cache(plan, cache)) != ENGRAM_OK) return rc;
+    if (n_tok > engram::kStageMaxTok)
+        return fail(ENGRAM_ERR_UNSUPPORTED, "engram_stage_rows_cached handles at most %d tokens per call", engram::kStageMaxTok);
+    if (capacity < n_tok) return fail(ENGRAM_ERR_INVALID_ARG, "capacity %d < n_tok %lld", capacity, (long long)n_tok);
+    if (!idx || !tables || !staging || !staged_idx || !unique_rows || !n_unique || !row_flags || !n_hits)
+        return fail(ENGRAM_ERR_INVALID_ARG, "NULL argument");
+    for (int h = 0; h < plan->num_tables; ++h) {
+        if (!tables[h] || !staging[h]) return fail(ENGRAM_ERR_INVALID_ARG, "tables[%d] or staging[%d] is NULL", h, h);
+        if (!aligned16(tables[h]) || !aligned16(staging[h]))
+            return fail(ENGRAM_ERR_INVALID_ARG, "tables[%d] / staging[%d] not 16-byte aligned", h, h);
+    }
+    return launch_stage(plan, idx, n_tok, tables, staging, capacity, staged_idx, unique_rows, n_unique,
+                        static_cast<cudaStream_t>(stream), cache, row_flags, n_hits);
 }
 
 int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,

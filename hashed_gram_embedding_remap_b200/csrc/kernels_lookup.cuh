@@ -489,3 +489,129 @@ __global__ void __launch_bounds__(256) stage_copy_kernel(const __grid_constant__
 }
 
 }  // namespace engram
+
+namespace engram {
+
+// ---------------------------------------------------------------- HBM cache of host-table rows
+// A direct-mapped cache per table in device memory sits in front of the host-resident
+// tables: slot(row) = row mod slots (row ids are already hash outputs, uniform mod P).
+// tags[slot] = row + 1 of the cached row (0 = empty); claim[slot] is per-call scratch that is
+// 0xFFFFFFFF between calls.  Per call, over the batch's distinct rows (from stage_dedup_kernel):
+//   probe:  hit = (tags[slot] == row + 1).  A hit pins its slot for this call
+//           (claim := 0); a miss bids for its slot (claim := min(claim, row + 1)).
+//   decide: a miss wins its slot iff claim[slot] == row + 1 (so no slot that is read this call
+//           is written this call, and at most one row is written into each slot).
+//   copy:   staging <- cache slot (hit) or host row (miss); a winner also writes the cache slot.
+//   commit: winners set tags[slot] = row + 1 (after their data is in place); every touched
+//           slot's claim goes back to 0xFFFFFFFF.
+// Staging always receives the exact row; the cache only decides where the bytes come from.
+struct CacheParams {
+    void *data[ENGRAM_MAX_TABLES];        // [slots, row bytes]
+    uint32_t *tags[ENGRAM_MAX_TABLES];    // [slots]
+    uint32_t *claim[ENGRAM_MAX_TABLES];   // [slots]
+    uint64_t slot_mask;                   // slots - 1 (slots a power of two)
+    uint64_t rows[ENGRAM_MAX_TABLES];     // table sizes: an out-of-range row never enters the cache
+    const uint32_t *unique_rows;          // [H, capacity]
+    const int32_t *n_unique;              // [H]
+    uint32_t *flags;                      // [H, capacity]: 1 = hit, 2 = miss that fills its slot, 0 = other miss
+    int32_t *n_hits;                      // [H]
+    int32_t H, capacity;
+};
+
+__global__ void cache_probe_kernel(const __grid_constant__ CacheParams p) {
+    const int h = blockIdx.y;
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= __ldg(p.n_unique + h)) return;
+    const uint32_t row = __ldg(p.unique_rows + static_cast<int64_t>(h) * p.capacity + s);
+    const uint64_t slot = row & p.slot_mask;
+    const bool hit = p.tags[h][slot] == row + 1u;   // only rows inside the table are ever tagged
+    if (hit) {
+        atomicMin(p.claim[h] + slot, 0u);
+        atomicAdd(p.n_hits + h, 1);
+    } else if (row < p.rows[h]) {
+        atomicMin(p.claim[h] + slot, row + 1u);
+    }
+    p.flags[static_cast<int64_t>(h) * p.capacity + s] = hit ? 1u : 0u;
+}
+
+__global__ void cache_decide_kernel(const __grid_constant__ CacheParams p) {
+    const int h = blockIdx.y;
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= __ldg(p.n_unique + h)) return;
+    const int64_t i = static_cast<int64_t>(h) * p.capacity + s;
+    if (p.flags[i] == 1u) return;
+    const uint32_t row = __ldg(p.unique_rows + i);
+    if (p.claim[h][row & p.slot_mask] == row + 1u) p.flags[i] = 2u;
+}
+
+__global__ void cache_commit_kernel(const __grid_constant__ CacheParams p) {
+    const int h = blockIdx.y;
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= __ldg(p.n_unique + h)) return;
+    const int64_t i = static_cast<int64_t>(h) * p.capacity + s;
+    const uint32_t row = __ldg(p.unique_rows + i);
+    const uint64_t slot = row & p.slot_mask;
+    if (p.flags[i] == 2u) p.tags[h][slot] = row + 1u;
+    p.claim[h][slot] = 0xFFFFFFFFu;
+}
+
+// Copy of the distinct rows into staging, from the cache (hits) or the host tables (misses);
+// a miss that won its slot also writes the cache.  16-byte chunks, many CTAs wide.
+template <int UNROLL>
+__global__ void __launch_bounds__(256) cache_copy_kernel(const __grid_constant__ StageParams sp,
+                                                         const __grid_constant__ CacheParams p) {
+    const int64_t per_table = static_cast<int64_t>(sp.capacity) * sp.chunks_per_row;
+    const int64_t total = per_table * sp.H;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < total;
+         base += stride * UNROLL) {
+        uint4 val[UNROLL];
+        int64_t dst[UNROLL], cdst[UNROLL];
+        int hh[UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            const int64_t i = base + u * stride;
+            dst[u] = -1;
+            cdst[u] = -1;
+            hh[u] = 0;
+            if (i < total) {
+                const int h = static_cast<int>(i / per_table);
+                const int64_t r = i - h * per_table;
+                const int32_t s = static_cast<int32_t>(r / sp.chunks_per_row);
+                const int32_t c = static_cast<int32_t>(r - static_cast<int64_t>(s) * sp.chunks_per_row);
+                if (s < __ldg(sp.n_unique + h)) {
+                    const int64_t k = static_cast<int64_t>(h) * sp.capacity + s;
+                    const uint32_t row = __ldg(sp.unique_rows + k);
+                    const uint32_t flag = p.flags[k];
+                    const uint64_t slot = row & p.slot_mask;
+                    hh[u] = h;
+                    dst[u] = r;
+                    if (flag == 1u) {
+                        val[u] = reinterpret_cast<const uint4 *>(p.data[h])[slot * sp.chunks_per_row + c];
+                    } else if (row < sp.rows[h]) {
+                        val[u] = reinterpret_cast<const uint4 *>(sp.table[h])[static_cast<int64_t>(row) * sp.chunks_per_row + c];
+                        if (flag == 2u) cdst[u] = static_cast<int64_t>(slot) * sp.chunks_per_row + c;
+                    } else {
+                        val[u] = make_uint4(0, 0, 0, 0);
+                        atomicOr(&g_engram_status, ENGRAM_STATUS_BAD_ROW);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            if (dst[u] >= 0) reinterpret_cast<uint4 *>(sp.staging[hh[u]])[dst[u]] = val[u];
+            if (cdst[u] >= 0) reinterpret_cast<uint4 *>(p.data[hh[u]])[cdst[u]] = val[u];
+        }
+    }
+}
+
+__global__ void cache_reset_kernel(uint32_t *tags, uint32_t *claim, int64_t slots) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < slots;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        tags[i] = 0u;
+        claim[i] = 0xFFFFFFFFu;
+    }
+}
+
+}  // namespace engram

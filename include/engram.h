@@ -214,6 +214,42 @@ int engram_stage_rows(const engram_plan *plan, const uint32_t *idx, int64_t n_to
                       uint32_t *staged_idx, uint32_t *unique_rows, int32_t *n_unique,
                       engram_stream_t stream);
 
+/* An HBM cache of host-table rows, in front of ENGRAM_TABLES_HOST_MAPPED tables [zhichai
+ * §2.3: n-gram frequencies are Zipf-like, so a few rows are read most of the time and can
+ * live in fast memory while the rest stays in host memory; the pages also report that real
+ * traffic shows little reuse across tokens, so the benefit depends on the stream].
+ * Direct-mapped, one per table: row r lives in slot r mod slots.  All buffers are DEVICE
+ * memory owned by the caller:
+ *   data[h]:  [slots, d_e] elements of the table type (bf16 patterns or e4m3 codes);
+ *   tags[h]:  uint32 [slots], row id + 1 of the row held in the slot, 0 = empty;
+ *   claim[h]: uint32 [slots], scratch that holds 0xFFFFFFFF between calls.
+ * engram_row_cache_reset() establishes that state (empty cache).  Contents are only ever
+ * changed by engram_stage_rows_cached on the caller's stream; calls that share a cache must
+ * be ordered on one stream. */
+typedef struct engram_row_cache {
+    void *data[ENGRAM_MAX_TABLES];
+    uint32_t *tags[ENGRAM_MAX_TABLES];
+    uint32_t *claim[ENGRAM_MAX_TABLES];
+    int64_t slots; /* power of two, 1 .. 2^32 */
+} engram_row_cache;
+
+/* Empty every table's cache (tags 0, claims 0xFFFFFFFF).  Asynchronous on `stream`. */
+int engram_row_cache_reset(const engram_plan *plan, const engram_row_cache *cache, engram_stream_t stream);
+
+/* engram_stage_rows with the row cache in front of the tables: the batch's distinct rows are
+ * copied into staging from the cache where it holds them and from the host tables otherwise;
+ * of the rows fetched from the host, each one that maps to a slot that no other distinct row
+ * of this call reads or bids for (ties: the smallest row id) is also written into the cache.
+ * staging, staged_idx, unique_rows and n_unique are exactly those of engram_stage_rows (the
+ * staged rows are bit-identical whatever the cache holds).
+ * row_flags: uint32 [H, capacity] device scratch.  n_hits: int32 [H] device, ACCUMULATES the
+ * number of distinct rows served from the cache (zero it to count one call). */
+int engram_stage_rows_cached(const engram_plan *plan, const uint32_t *idx, int64_t n_tok,
+                             const void *const *tables, const engram_row_cache *cache,
+                             void *const *staging, int32_t capacity, uint32_t *staged_idx,
+                             uint32_t *unique_rows, int32_t *n_unique, uint32_t *row_flags,
+                             int32_t *n_hits, engram_stream_t stream);
+
 /* engram_gather over tables that all hold `rows` rows (e.g. the staging buffers filled by
  * engram_stage_rows, with staged_idx as idx).  Same layout and error behaviour as
  * engram_gather, with `rows` as every table's bound. */
@@ -290,7 +326,8 @@ const char *engram_last_error(void);
 /* Library version, e.g. "0.1.0". */
 const char *engram_version(void);
 
-/* sizeof() of a public struct, by name ("engram_config", "engram_plan", "engram_weights"),
+/* sizeof() of a public struct, by name ("engram_config", "engram_plan", "engram_weights",
+ * "engram_row_cache"),
  * so that bindings in other languages can check their layout; 0 for an unknown name. */
 size_t engram_sizeof(const char *type_name);
 

@@ -31,7 +31,7 @@ def test_every_declared_symbol_is_exported():
 
 def test_struct_layouts_match_header():
     for name, cls in (("engram_config", _native.engram_config), ("engram_plan", _native.engram_plan),
-                      ("engram_weights", _native.engram_weights)):
+                      ("engram_weights", _native.engram_weights), ("engram_row_cache", _native.engram_row_cache)):
         assert E.lib.engram_sizeof(name.encode()) == C.sizeof(cls)
     assert E.lib.engram_sizeof(b"nope") == 0
 
@@ -152,4 +152,35 @@ def test_branches_default_and_workspace_growth():
     assert E.engram_workspace_size(p4, 4096) > E.engram_workspace_size(p1, 4096)
     wl = synth.get_workload("layer2560x4")
     assert E.Plan.from_workload(wl).num_branches == 4 and wl.h_rows == 4 * wl.n_tok
+
+
+def test_row_cache_arguments_rejected_on_host():
+    p = _plan()
+    c = _native.engram_row_cache()
+    for h in range(4):
+        c.data[h] = c.tags[h] = c.claim[h] = 256 * (h + 1)
+    for bad in (0, 3, 6, (1 << 32) + 1):
+        c.slots = bad
+        assert E.lib.engram_row_cache_reset(p, C.byref(c), None) == E.ENGRAM_ERR_INVALID_ARG
+        assert "power of two" in E.last_error()
+    c.slots = 64
+    c.tags[2] = 0
+    assert E.lib.engram_row_cache_reset(p, C.byref(c), None) == E.ENGRAM_ERR_INVALID_ARG
+    assert E.lib.engram_row_cache_reset(p, None, None) == E.ENGRAM_ERR_INVALID_ARG
+    # an empty batch is a no-op even without a device
+    assert E.lib.engram_stage_rows_cached(p, None, 0, None, None, None, 1, None, None, None, None, None,
+                                          None) == E.ENGRAM_OK
+
+
+def test_cache_model_policy():
+    """The host model used by the GPU cache tests: hits pin slots; the smallest row wins a
+    free slot; rows outside the table never enter."""
+    from cache_model import CacheModel
+    import numpy as np
+    m = CacheModel(1, 4, [100])
+    assert m.step(np.array([[1], [5], [9], [2]])) == [0]      # 1, 5, 9 share slot 1: 1 wins
+    assert m.tags[0].tolist() == [0, 2, 3, 0]
+    # 1 hits and pins slot 1 (5 may not replace it); 6 replaces 2 in slot 2; 101 is outside
+    assert m.step(np.array([[5], [1], [6], [101]])) == [1]
+    assert m.tags[0].tolist() == [0, 2, 7, 0]
 

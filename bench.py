@@ -514,6 +514,10 @@ def run_hostpinned(args, wl, world, rank, local):
     uniq = torch.empty((wl.H, B), dtype=torch.int32, device=dev)
     nu = torch.empty((wl.H,), dtype=torch.int32, device=dev)
     m = torch.empty((B, wl.d_m), dtype=torch.bfloat16, device=dev)
+    # optional HBM row cache in front of the host tables
+    cache = E.RowCache(plan, args.cache_slots, dev) if args.cache_slots else None
+    row_flags = torch.empty((wl.H, B), dtype=torch.int32, device=dev)
+    n_hits = torch.zeros((wl.H,), dtype=torch.int32, device=dev)
     ga = torch.randn(2560, 2560, device=dev, dtype=torch.bfloat16)
     gb = torch.randn(2560, 2560, device=dev, dtype=torch.bfloat16)
     gc_ = torch.empty(2560, 2560, device=dev, dtype=torch.bfloat16)
@@ -535,7 +539,11 @@ def run_hostpinned(args, wl, world, rank, local):
             if evs is not None:
                 evs[0].record(side)
             E.engram_hash(plan, x, idx, history=history, stream=side)
-            E.engram_stage_rows(plan, idx, tables, staging, sidx, uniq, nu, stream=side)
+            if cache is not None:
+                E.engram_stage_rows_cached(plan, idx, tables, cache, staging, sidx, uniq, nu, row_flags, n_hits,
+                                           stream=side)
+            else:
+                E.engram_stage_rows(plan, idx, tables, staging, sidx, uniq, nu, stream=side)
             if evs is not None:
                 evs[1].record(side)
         torch.matmul(ga, gb, out=gc_)              # stand-in for the layers before the lookup
@@ -568,6 +576,13 @@ def run_hostpinned(args, wl, world, rank, local):
         g = capture(overlap, name == "overlapped")
         g.replay()
         torch.cuda.synchronize()
+        if cache is not None:
+            # the upload replay above ran the timed steps' own ids: empty the cache and warm it
+            # on the warm-up steps only, so that the timed steps meet no row they inserted
+            cache.reset(comp)
+            for k in range(args.warmup):
+                one_step(k, False)
+            torch.cuda.synchronize()
         st, sp = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with ClockSampler(local) as clocks:
             c0 = time.perf_counter()
@@ -580,6 +595,25 @@ def run_hostpinned(args, wl, world, rank, local):
         del g
     prefetch_ms = statistics.mean(ev[k][0].elapsed_time(ev[k][1]) for k in range(K))
     tail_ms = statistics.mean(ev[k][2].elapsed_time(ev[k][3]) for k in range(K))
+    row_cache = None
+    if cache is not None:
+        # hit rate of the timed id stream under the timed protocol (cache emptied, warmed on the
+        # warm-up steps), stepped one by one with the distinct-row counts read back
+        cache.reset(comp)
+        for k in range(args.warmup):
+            one_step(k, False)
+        hits = distinct = 0
+        for k in range(K):
+            n_hits.zero_()
+            one_step(args.warmup + k, False)
+            torch.cuda.synchronize()
+            hits += int(n_hits.sum().item())
+            distinct += int(nu.sum().item())
+        row_cache = {"slots_per_table": args.cache_slots,
+                     "GB": round(wl.H * args.cache_slots * wl.d_e * eb / 1e9, 2),
+                     "hit_rate": hits / max(1, distinct),
+                     "distinct_rows_per_step": distinct / K,
+                     "host_bytes_per_step": (distinct - hits) / K * wl.d_e * eb}
     # GEMM alone, for the overlap figure
     gs, ge = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(5):
@@ -640,7 +674,8 @@ def run_hostpinned(args, wl, world, rank, local):
         "overlap": {"serial_ms_per_step": ser_ms, "overlapped_ms_per_step": ovl_ms, "gemm_ms": gemm_ms,
                     "prefetch_ms": prefetch_ms, "hidden_fraction": max(0.0, min(1.0, saved / max(1e-9, min(gemm_ms, prefetch_ms))))},
         "tail_ms": tail_ms, "table_setup_s": t_alloc, "clocks": ovl_clk,
-        "launch_mode": "one CUDA graph of the K timed steps", "gpu_launches": K * 7,
+        "launch_mode": "one CUDA graph of the K timed steps", "gpu_launches": K * (7 + (3 if cache is not None else 0)),
+        "row_cache": row_cache,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -663,6 +698,9 @@ def main():
     ap.add_argument("--ids", choices=["uniform", "zipf"], default=None, help="id distribution (host-pinned workload)")
     ap.add_argument("--table-rows", type=int, default=0, help="override the table size (largest prime <= N)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's sequences per step")
+    ap.add_argument("--cache-slots", type=int, default=0,
+                    help="host-resident tables: HBM row cache of this many slots per table (power of two; 0 = none)")
     ap.add_argument("--table-dtype", choices=["bf16", "fp8"], default="bf16",
                     help="table element type: bf16 rows, or e4m3 codes with one scale per table")
     args = ap.parse_args()
@@ -676,6 +714,10 @@ def main():
         wl = wl.with_(primes=(p,) * wl.H, name=f"{wl.name}[rows={p}]")
     if args.table_dtype == "fp8":
         wl = wl.with_(table_dtype="fp8", name=f"{wl.name}-fp8")
+    if args.batch:
+        wl = wl.with_(B=args.batch, name=f"{wl.name}[B={args.batch}]")
+    if args.cache_slots:
+        wl = wl.with_(name=f"{wl.name}[cache={args.cache_slots}]")
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -175,6 +175,19 @@ def barrier(world):
 
 # ---------------------------------------------------------------------------------------
 # CPU oracle on a bounded sample (the reference arm and the cpu_baseline object)
+def host_cpu() -> str:
+    """CPU model and logical core count of this host (for the CPU-baseline record)."""
+    model = "unknown CPU"
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return f"{model}, {os.cpu_count()} logical cores"
+
+
 def oracle_sample(wl, n_tok_sample: int, seq: int = 0):
     """Time the oracle's steps (remap, hash, gather, gate + conv + residual) on the first
     n_tok_sample tokens of sequence `seq`.  Table rows are regenerated from the seeded
@@ -230,8 +243,8 @@ def run_reference(args, wl, world, rank):
         times.append(dt)
         t_gen += tg
     tps = T * len(times) / sum(times)
-    sample = (f"{args.steps} samples of 1 sequence x {T} tokens of {wl.name}; fp64 scalar C, 1 thread; "
-              f"table-row regeneration ({t_gen:.2f} s total) not timed")
+    sample = (f"{args.steps} samples of 1 sequence x {T} tokens of {wl.name}; fp64 scalar C, 1 thread of "
+              f"{host_cpu()}; table-row regeneration ({t_gen:.2f} s total) not timed")
     line = {
         "impl": "reference", "metric": "engram_tokens_per_s", "value": tps, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -448,7 +461,7 @@ def run_engram(args, wl, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         T, dt, t_gen = oracle_sample(wl, args.cpu_baseline_tokens)
         cpu = {"value": T / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": f"1 sequence x {T} tokens of {wl.name}; fp64 scalar C, 1 thread; "
+               "sample": f"1 sequence x {T} tokens of {wl.name}; fp64 scalar C, 1 thread of {host_cpu()}; "
                          f"table-row regeneration ({t_gen:.2f} s) not timed"}
 
     value = n_tok * world * args.steps / (elapsed_ms / 1e3)

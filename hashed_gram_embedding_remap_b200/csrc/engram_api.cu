@@ -721,7 +721,13 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[1], stream), "cudaEventRecord");
     if (fused_decode) {
         const engram::GateParams gp = make_gate_params(plan, w, h, v, part, ps.n_tiles, B, T, conv_state, out, delta);
-        engram::decode_fused_kernel<<<static_cast<unsigned>(B), engram::kFusedDecodeThreads, 0, stream>>>(pp, gp);
+        using DK = void (*)(const engram::ProjParams, const engram::GateParams);
+        static const DK kernels[engram::kFusedDecodeMaxPairs] = {
+            engram::decode_fused_kernel<1>, engram::decode_fused_kernel<2>, engram::decode_fused_kernel<3>,
+            engram::decode_fused_kernel<4>, engram::decode_fused_kernel<5>, engram::decode_fused_kernel<6>,
+            engram::decode_fused_kernel<7>, engram::decode_fused_kernel<8>};
+        const int pairs = (d_h / 2 + engram::kFusedDecodeThreads - 1) / engram::kFusedDecodeThreads;
+        kernels[pairs - 1]<<<static_cast<unsigned>(B), engram::kFusedDecodeThreads, 0, stream>>>(pp, gp);
         ENGRAM_CUDA_TRY(cudaGetLastError(), "decode_fused_kernel launch");
         return ENGRAM_OK;
     }

@@ -618,11 +618,16 @@ __global__ void __launch_bounds__(kDecodeThreads) gate_conv_decode_kernel(const 
 // k_splits partial accumulators of its [k~ | v] row, reduces S0..S3 across the block, then
 // applies gate, conv (kernel 4, dilation 3, taps from the carried state or zeros), SiLU,
 // residual and the state shift.  Replaces splitk_reduce_kernel + the gate kernel for decode.
-constexpr int kFusedDecodeThreads = 512;
-constexpr int kFusedDecodeMaxPairs = 4;   // d_h <= 2 * 512 * 4 = 4096
+// P channel pairs per thread (d_h <= 2 * 256 * P): every load of the token -- split
+// accumulators, h, gains, conv taps, the 9 carried state slots -- is issued in one round
+// trip; P is the smallest that covers d_h, so the registers allow two CTAs per SM and a
+// decode batch of up to 2 x #SMs tokens runs in one wave.
+constexpr int kFusedDecodeThreads = 256;
+constexpr int kFusedDecodeMaxPairs = 8;   // d_h <= 2 * 256 * 8 = 4096
 
-__global__ void __launch_bounds__(kFusedDecodeThreads) decode_fused_kernel(const __grid_constant__ ProjParams pp,
-                                                                           const __grid_constant__ GateParams p) {
+template <int P>
+__global__ void __launch_bounds__(kFusedDecodeThreads, 2) decode_fused_kernel(const __grid_constant__ ProjParams pp,
+                                                                              const __grid_constant__ GateParams p) {
     constexpr int S = 9;
     __shared__ float s_red[4][kFusedDecodeThreads / 32];
     __shared__ float s_gb[2];
@@ -630,13 +635,13 @@ __global__ void __launch_bounds__(kFusedDecodeThreads) decode_fused_kernel(const
     const int d_h = p.d_h;
     const int64_t split_stride = pp.n_tok * (2 * d_h);
     const float *acc = pp.acc_out + static_cast<int64_t>(b) * (2 * d_h);
-    float2 v[kFusedDecodeMaxPairs];
-    uint32_t hv[kFusedDecodeMaxPairs], gw[kFusedDecodeMaxPairs], st[kFusedDecodeMaxPairs][S];
-    uint2 w0[kFusedDecodeMaxPairs], w1[kFusedDecodeMaxPairs];
+    float2 v[P];
+    uint32_t hv[P], gw[P], st[P][S];
+    uint2 w0[P], w1[P];
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     // one round trip: split accumulators, h, gains, conv weights and the carried state
 #pragma unroll
-    for (int k = 0; k < kFusedDecodeMaxPairs; ++k) {
+    for (int k = 0; k < P; ++k) {
         const int c = 2 * (threadIdx.x + k * kFusedDecodeThreads);
         v[k] = make_float2(0.f, 0.f);
         hv[k] = gw[k] = 0;
@@ -706,7 +711,7 @@ __global__ void __launch_bounds__(kFusedDecodeThreads) decode_fused_kernel(const
     __syncthreads();
     const float g = s_gb[0], beta = s_gb[1];
 #pragma unroll
-    for (int k = 0; k < kFusedDecodeMaxPairs; ++k) {
+    for (int k = 0; k < P; ++k) {
         const int c = 2 * (threadIdx.x + k * kFusedDecodeThreads);
         if (c >= d_h) continue;
         const float u0 = beta * v[k].x * bf16_lo(gw[k]), u1 = beta * v[k].y * bf16_hi(gw[k]);

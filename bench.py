@@ -456,6 +456,11 @@ def run_engram(args, wl, world, rank, local):
            "peak_GBps": peaks["hbm"], "nominal_GBps": 8000.0}
     hbm["gather_frac"] = hbm["gather_GBps"] / peaks["hbm"]
     hbm["gate_conv_frac"] = hbm["gate_conv_GBps"] / peaks["hbm"]
+    # the memory-bound part of the path taken together: gather + gate + conv
+    both_s = (stage_ms["gather"] + stage_ms["gate_conv"]) / 1e3
+    hbm["gather_gate_conv_GBps"] = (gather_bytes + gate_bytes) / both_s / 1e9
+    hbm["gather_gate_conv_frac"] = hbm["gather_gate_conv_GBps"] / peaks["hbm"]
+    hbm["gather_gate_conv_frac_nominal"] = hbm["gather_gate_conv_GBps"] / hbm["nominal_GBps"]
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

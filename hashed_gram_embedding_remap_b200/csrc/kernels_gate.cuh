@@ -636,16 +636,17 @@ __global__ void __launch_bounds__(kFusedDecodeThreads, 2) decode_fused_kernel(co
     const int64_t split_stride = pp.n_tok * (2 * d_h);
     const float *acc = pp.acc_out + static_cast<int64_t>(b) * (2 * d_h);
     float2 v[P];
-    uint32_t hv[P], gw[P], st[P][S];
-    uint2 w0[P], w1[P];
+    uint32_t hv[P], st[P][S];
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    // one round trip: split accumulators, h, gains, conv weights and the carried state
+    // the carried state and h first (independent of the splits), then the split accumulators
+    // one split at a time across all pairs: k_splits round trips in total.  The gains and
+    // conv taps (the same for every token, L2-resident) are read after the reduction.
+    float2 kt[P];
 #pragma unroll
     for (int k = 0; k < P; ++k) {
         const int c = 2 * (threadIdx.x + k * kFusedDecodeThreads);
-        v[k] = make_float2(0.f, 0.f);
-        hv[k] = gw[k] = 0;
-        w0[k] = w1[k] = make_uint2(0, 0);
+        v[k] = kt[k] = make_float2(0.f, 0.f);
+        hv[k] = 0;
 #pragma unroll
         for (int j = 0; j < S; ++j) st[k][j] = 0;
         if (c < d_h) {
@@ -654,28 +655,35 @@ __global__ void __launch_bounds__(kFusedDecodeThreads, 2) decode_fused_kernel(co
 #pragma unroll
                 for (int j = 0; j < S; ++j) st[k][j] = *reinterpret_cast<const uint32_t *>(state + j * d_h);
             }
-            gw[k] = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_c + c));
-            w0[k] = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + c * 4));
-            w1[k] = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + (c + 1) * 4));
-            float2 kt = make_float2(0.f, 0.f), vt = make_float2(0.f, 0.f);
-            for (int ks = 0; ks < pp.k_splits; ++ks) {
-                const float2 x = __ldg(reinterpret_cast<const float2 *>(acc + ks * split_stride + c));
-                const float2 y = __ldg(reinterpret_cast<const float2 *>(acc + ks * split_stride + d_h + c));
-                kt.x += x.x;
-                kt.y += x.y;
-                vt.x += y.x;
-                vt.y += y.y;
+            hv[k] = __ldg(reinterpret_cast<const uint32_t *>(pp.h + static_cast<int64_t>(b) * d_h + c));
+        }
+    }
+    for (int ks = 0; ks < pp.k_splits; ++ks) {
+        const float *src = acc + ks * split_stride;
+#pragma unroll
+        for (int k = 0; k < P; ++k) {
+            const int c = 2 * (threadIdx.x + k * kFusedDecodeThreads);
+            if (c < d_h) {
+                const float2 x = __ldg(reinterpret_cast<const float2 *>(src + c));
+                const float2 y = __ldg(reinterpret_cast<const float2 *>(src + d_h + c));
+                kt[k].x += x.x;
+                kt[k].y += x.y;
+                v[k].x += y.x;
+                v[k].y += y.y;
             }
-            const uint32_t hw = __ldg(reinterpret_cast<const uint32_t *>(pp.h + static_cast<int64_t>(b) * d_h + c));
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < P; ++k) {
+        const int c = 2 * (threadIdx.x + k * kFusedDecodeThreads);
+        if (c < d_h) {
             const uint32_t qw = __ldg(reinterpret_cast<const uint32_t *>(pp.gamma_q + c));
             const uint32_t kw = __ldg(reinterpret_cast<const uint32_t *>(pp.gamma_k + c));
-            const float h0 = bf16_lo(hw), h1 = bf16_hi(hw);
+            const float h0 = bf16_lo(hv[k]), h1 = bf16_hi(hv[k]);
             a0 = fmaf(h0, h0, fmaf(h1, h1, a0));
-            a1 = fmaf(h0 * bf16_lo(qw) * bf16_lo(kw), kt.x, fmaf(h1 * bf16_hi(qw) * bf16_hi(kw), kt.y, a1));
-            a2 = fmaf(kt.x, kt.x, fmaf(kt.y, kt.y, a2));
-            a3 = fmaf(vt.x, vt.x, fmaf(vt.y, vt.y, a3));
-            v[k] = vt;
-            hv[k] = hw;
+            a1 = fmaf(h0 * bf16_lo(qw) * bf16_lo(kw), kt[k].x, fmaf(h1 * bf16_hi(qw) * bf16_hi(kw), kt[k].y, a1));
+            a2 = fmaf(kt[k].x, kt[k].x, fmaf(kt[k].y, kt[k].y, a2));
+            a3 = fmaf(v[k].x, v[k].x, fmaf(v[k].y, v[k].y, a3));
         }
     }
 #pragma unroll
@@ -714,12 +722,15 @@ __global__ void __launch_bounds__(kFusedDecodeThreads, 2) decode_fused_kernel(co
     for (int k = 0; k < P; ++k) {
         const int c = 2 * (threadIdx.x + k * kFusedDecodeThreads);
         if (c >= d_h) continue;
-        const float u0 = beta * v[k].x * bf16_lo(gw[k]), u1 = beta * v[k].y * bf16_hi(gw[k]);
+        const uint32_t gwk = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_c + c));
+        const uint2 w0k = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + c * 4));
+        const uint2 w1k = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + (c + 1) * 4));
+        const float u0 = beta * v[k].x * bf16_lo(gwk), u1 = beta * v[k].y * bf16_hi(gwk);
         // taps: i = 0 current, 1 -> slot 6 (t-3), 2 -> slot 3 (t-6), 3 -> slot 0 (t-9)
-        const float c0 = fmaf(bf16_lo(w0[k].x), u0, fmaf(bf16_hi(w0[k].x), bf16_lo(st[k][6]),
-                         fmaf(bf16_lo(w0[k].y), bf16_lo(st[k][3]), bf16_hi(w0[k].y) * bf16_lo(st[k][0]))));
-        const float c1 = fmaf(bf16_lo(w1[k].x), u1, fmaf(bf16_hi(w1[k].x), bf16_hi(st[k][6]),
-                         fmaf(bf16_lo(w1[k].y), bf16_hi(st[k][3]), bf16_hi(w1[k].y) * bf16_hi(st[k][0]))));
+        const float c0 = fmaf(bf16_lo(w0k.x), u0, fmaf(bf16_hi(w0k.x), bf16_lo(st[k][6]),
+                         fmaf(bf16_lo(w0k.y), bf16_lo(st[k][3]), bf16_hi(w0k.y) * bf16_lo(st[k][0]))));
+        const float c1 = fmaf(bf16_lo(w1k.x), u1, fmaf(bf16_hi(w1k.x), bf16_hi(st[k][6]),
+                         fmaf(bf16_lo(w1k.y), bf16_hi(st[k][3]), bf16_hi(w1k.y) * bf16_hi(st[k][0]))));
         const float d0 = fmaf(g, v[k].x, c0 * fast_sigmoid(c0));
         const float d1 = fmaf(g, v[k].y, c1 * fast_sigmoid(c1));
         const uint32_t o = static_cast<uint32_t>(f32_to_bf16_bits(bf16_lo(hv[k]) + d0)) |

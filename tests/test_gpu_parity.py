@@ -196,15 +196,17 @@ def test_gate_conv_entry_matches_forward():
     assert torch.equal(out_fwd.view(torch.int16), out2.view(torch.int16))
 
 
-@pytest.mark.parametrize("geom", ["small", "splitk", "chunk4"])
+@pytest.mark.parametrize("geom", ["small", "splitk", "splitk_256seq", "chunk4"])
 def test_decode_steps_match_oracle_and_update_state(geom):
     """Consecutive calls carrying the hash history and conv state: one token per call
-    (one-token decode kernels, with and without split-K) and four tokens per call (the
-    chain kernel reading and rewriting the carried state)."""
+    (one-token decode kernels, with and without split-K, over one and two 128-token tiles)
+    and four tokens per call (the chain kernel reading and rewriting the carried state)."""
     if geom == "small":
         wl = small_workload("dec", B=6, T=1, K=2, d_e=32, d_h=256, decode=True)
     elif geom == "splitk":
         wl = small_workload("dec_split", B=32, T=1, K=1, d_e=512, d_h=512, decode=True)
+    elif geom == "splitk_256seq":
+        wl = small_workload("dec_256", B=256, T=1, K=1, d_e=512, d_h=512, decode=True)
     else:
         wl = small_workload("dec_chunk", B=5, T=4, K=2, d_e=32, d_h=256, decode=True)
     di = DeviceInputs(wl, random_gammas=geom != "small")

@@ -295,7 +295,8 @@ def run_engram(args, wl, world, rank, local):
     history = torch.from_numpy(wl.history()).to(dev) if wl.decode else None
     state = fill_gpu.filled((wl.B * M, wl.state_len, wl.d_h), wl.state_spec(), dev) if wl.decode else None
     plan = E.Plan.from_workload(wl)
-    weights = E.Weights(wk, wv, one, one, one, cw)
+    packed = E.pack_weights(plan, wk, wv) if args.packed else None
+    weights = E.Weights(wk, wv, one, one, one, cw, packed=packed)
     out = torch.empty((wl.h_rows, wl.d_h), dtype=torch.bfloat16, device=dev)
     ws = E.alloc_workspace(plan, wl.n_tok, dev)
     nstage = E.ENGRAM_FORWARD_STAGES + 1
@@ -522,7 +523,8 @@ def run_hostpinned(args, wl, world, rank, local):
     wv = fill_gpu.filled((wl.d_h, wl.d_m), wl.wv_spec(), dev)
     one = torch.full((wl.d_h,), 0x3F80, dtype=torch.int16, device=dev).view(torch.bfloat16)
     cw = fill_gpu.filled((wl.d_h, wl.conv_kernel), wl.conv_spec(), dev)
-    weights = E.Weights(wk, wv, one, one, one, cw)
+    packed = E.pack_weights(plan, wk, wv) if args.packed else None
+    weights = E.Weights(wk, wv, one, one, one, cw, packed=packed)
     out = torch.empty((B, wl.d_h), dtype=torch.bfloat16, device=dev)
     ws = E.alloc_workspace(plan, B, dev)
     idx = torch.empty((B, wl.H), dtype=torch.int32, device=dev)
@@ -717,6 +719,8 @@ def main():
     ap.add_argument("--table-rows", type=int, default=0, help="override the table size (largest prime <= N)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's sequences per step")
+    ap.add_argument("--packed", action="store_true",
+                    help="stream the projection weights from their packed copy (engram_pack_weights)")
     ap.add_argument("--cache-slots", type=int, default=0,
                     help="host-resident tables: HBM row cache of this many slots per table (power of two; 0 = none)")
     ap.add_argument("--table-dtype", choices=["bf16", "fp8"], default="bf16",
@@ -736,6 +740,8 @@ def main():
         wl = wl.with_(B=args.batch, name=f"{wl.name}[B={args.batch}]")
     if args.cache_slots:
         wl = wl.with_(name=f"{wl.name}[cache={args.cache_slots}]")
+    if args.packed:
+        wl = wl.with_(name=f"{wl.name}[packed]")
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

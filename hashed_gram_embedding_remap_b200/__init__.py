@@ -12,5 +12,6 @@ from ._native import (  # noqa: F401
     ENGRAM_TABLE_FP8_E4M3, EngramError, LIB_PATH, Plan, Weights, alloc_workspace,
     engram_advance_history, engram_device_status, engram_forward, engram_gate_conv,
     engram_gate_conv_noalloc, engram_gather, engram_hash, engram_stage_rows, engram_stage_rows_cached, RowCache,
+    pack_weights, engram_packed_weights_size,
     engram_remap, engram_workspace_size, last_error, lib, version,
 )

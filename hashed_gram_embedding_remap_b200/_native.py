@@ -84,7 +84,7 @@ class engram_plan(C.Structure):
 
 
 class engram_weights(C.Structure):
-    _fields_ = [(n, C.c_void_p) for n in ("w_k", "w_v", "gamma_q", "gamma_k", "gamma_c", "conv_w")]
+    _fields_ = [(n, C.c_void_p) for n in ("w_k", "w_v", "gamma_q", "gamma_k", "gamma_c", "conv_w", "w_packed")]
 
 
 class engram_row_cache(C.Structure):
@@ -112,6 +112,8 @@ def _load():
         "engram_stage_rows": (C.c_int, [P, P, i64, P, P, i32, P, P, P, P]),
         "engram_gather_bounded": (C.c_int, [P, P, P, i64, i64, P, P]),
         "engram_row_cache_reset": (C.c_int, [P, P, P]),
+        "engram_packed_weights_size": (sz, [P]),
+        "engram_pack_weights": (C.c_int, [P, P, P, P, sz, P]),
         "engram_stage_rows_cached": (C.c_int, [P, P, i64, P, P, P, i32, P, P, P, P, P, P]),
         "engram_gate_conv": (C.c_int, [P, P, P, P, i32, i32, P, P, P, P, sz, P]),
         "engram_forward": (C.c_int, [P, P, P, P, P, i32, i32, P, P, P, P, P, P, sz, P, P]),
@@ -242,16 +244,34 @@ class Plan:
 
 
 class Weights:
-    """Device tensors of the gate and conv, bundled as engram_weights."""
+    """Device tensors of the gate and conv, bundled as engram_weights.  `packed`: optional
+    copy of [W_k ; W_v] made by pack_weights (streamed by the projections instead)."""
 
-    def __init__(self, w_k, w_v, gamma_q, gamma_k, gamma_c, conv_w):
-        self.tensors = (w_k, w_v, gamma_q, gamma_k, gamma_c, conv_w)
+    def __init__(self, w_k, w_v, gamma_q, gamma_k, gamma_c, conv_w, packed=None):
+        self.tensors = (w_k, w_v, gamma_q, gamma_k, gamma_c, conv_w, packed)
         names = ("w_k", "w_v", "gamma_q", "gamma_k", "gamma_c", "conv_w")
-        self.struct = engram_weights(*[_ptr(t, _BF16, n) for t, n in zip(self.tensors, names)])
+        ptrs = [_ptr(t, _BF16, n) for t, n in zip(self.tensors[:6], names)]
+        ptrs.append(None if packed is None else _ptr(packed, None, "packed"))
+        self.struct = engram_weights(*ptrs)
 
     @property
     def _as_parameter_(self):
         return C.byref(self.struct)
+
+
+def engram_packed_weights_size(plan: Plan) -> int:
+    return int(lib.engram_packed_weights_size(plan))
+
+
+def pack_weights(plan: Plan, w_k: torch.Tensor, w_v: torch.Tensor, stream=None) -> torch.Tensor:
+    """The projection weights re-laid as pre-swizzled 256 x 64 tiles (engram_pack_weights)."""
+    n = engram_packed_weights_size(plan)
+    if n == 0:
+        raise EngramError(ENGRAM_ERR_UNSUPPORTED, "no packed form for this hidden size")
+    out = torch.empty(n, dtype=torch.uint8, device=w_k.device)
+    _check(lib.engram_pack_weights(plan, _ptr(w_k, _BF16, "w_k"), _ptr(w_v, _BF16, "w_v"),
+                                   _ptr(out, None, "packed"), n, _stream(stream)))
+    return out
 
 
 def _table_array(tables, plan: Optional[Plan] = None):

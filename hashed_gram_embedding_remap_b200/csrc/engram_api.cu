@@ -313,6 +313,7 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     p.k_splits = (acc != nullptr && k_splits > 1) ? k_splits : 1;
     p.kb_per_split = p.k_splits > 1 ? kb_per_split : p.k_blocks;
     p.acc_out = p.k_splits > 1 ? acc : nullptr;
+    p.w_packed = BN == 256 ? static_cast<const uint8_t *>(w->w_packed) : nullptr;
     const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles * p.k_splits;
     if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
     const int64_t sms = sm_count();
@@ -337,8 +338,20 @@ int validate_weights(const engram_plan *plan, const engram_weights *w) {
         if (ptrs[i] == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "weights.%s is NULL", names[i]);
         if (!aligned16(ptrs[i])) return fail(ENGRAM_ERR_INVALID_ARG, "weights.%s is not 16-byte aligned", names[i]);
     }
-    (void)plan;
+    if (w->w_packed != nullptr) {
+        if (plan->cfg.hidden_dim % 256 != 0)
+            return fail(ENGRAM_ERR_INVALID_ARG, "weights.w_packed given but hidden_dim %% 256 != 0 (no packed form)");
+        if (!aligned16(w->w_packed)) return fail(ENGRAM_ERR_INVALID_ARG, "weights.w_packed is not 16-byte aligned");
+    }
     return ENGRAM_OK;
+}
+
+size_t packed_weights_bytes(const engram_plan *plan) {
+    const int d_h = plan->cfg.hidden_dim;
+    if (d_h % 256 != 0) return 0;
+    const int64_t k_blocks = (plan->mem_dim + engram::kBK - 1) / engram::kBK;
+    const int64_t rows = static_cast<int64_t>(plan->num_branches + 1) * d_h;
+    return static_cast<size_t>(rows / 256 * k_blocks) * 32768u;
 }
 
 engram::HashParams make_hash_params(const engram_plan *plan, int32_t B, int32_t T) {
@@ -954,6 +967,31 @@ int engram_stage_rows(const engram_plan *plan, const uint32_t *idx, int64_t n_to
     }
     return launch_stage(plan, idx, n_tok, tables, staging, capacity, staged_idx, unique_rows, n_unique,
                         static_cast<cudaStream_t>(stream));
+}
+
+size_t engram_packed_weights_size(const engram_plan *plan) {
+    if (plan == nullptr || plan->magic != kPlanMagic) return 0;
+    return packed_weights_bytes(plan);
+}
+
+int engram_pack_weights(const engram_plan *plan, const uint16_t *w_k, const uint16_t *w_v, void *packed,
+                        size_t packed_bytes, engram_stream_t stream) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    const size_t need = packed_weights_bytes(plan);
+    if (need == 0) return fail(ENGRAM_ERR_UNSUPPORTED, "no packed form for hidden_dim %% 256 != 0");
+    if (!w_k || !w_v || !packed) return fail(ENGRAM_ERR_INVALID_ARG, "w_k, w_v and packed must be non-NULL");
+    if (!aligned16(w_k) || !aligned16(w_v) || !aligned16(packed))
+        return fail(ENGRAM_ERR_INVALID_ARG, "w_k, w_v and packed must be 16-byte aligned");
+    if (packed_bytes < need) return fail(ENGRAM_ERR_INVALID_ARG, "packed buffer too small: need %zu bytes", need);
+    const int64_t n_chunks = static_cast<int64_t>(need / 16);
+    int64_t blocks = (n_chunks + 255) / 256;
+    if (blocks > static_cast<int64_t>(sm_count()) * 16) blocks = static_cast<int64_t>(sm_count()) * 16;
+    engram::pack_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        w_k, w_v, static_cast<int64_t>(plan->num_branches) * plan->cfg.hidden_dim, plan->mem_dim,
+        (plan->mem_dim + engram::kBK - 1) / engram::kBK, n_chunks, static_cast<uint4 *>(packed));
+    ENGRAM_CUDA_TRY(cudaGetLastError(), "pack_weights_kernel launch");
+    return ENGRAM_OK;
 }
 
 int engram_row_cache_reset(const engram_plan *plan, const engram_row_cache *cache, engram_stream_t stream) {

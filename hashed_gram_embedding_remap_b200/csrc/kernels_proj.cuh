@@ -56,7 +56,32 @@ struct ProjParams {
     int32_t k_splits;          // > 1: split-K, raw fp32 partial accumulators go to acc_out
     int32_t kb_per_split;      // k-blocks per split
     float *acc_out;            // [k_splits, n_tok, (M+1)*d_h] when k_splits > 1
+    const uint8_t *w_packed;   // non-null: B tiles come as 32 KB pre-swizzled blocks (BN = 256)
 };
+
+// Packs [W_k ; W_v] into pre-swizzled 256 x 64 tiles (the layout engram_pack_weights
+// documents): one thread per 16-byte chunk of the packed copy.
+__global__ void pack_weights_kernel(const uint16_t *__restrict__ w_k, const uint16_t *__restrict__ w_v,
+                                    int64_t key_rows, int32_t d_m, int32_t k_blocks, int64_t n_chunks,
+                                    uint4 *__restrict__ packed) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_chunks;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t tile = i >> 11;                  // 2048 chunks of 16 B per 32 KB tile
+        const int within = static_cast<int>(i & 2047);
+        const int r = within >> 3, jp = within & 7;    // row in the tile, stored chunk position
+        const int j = jp ^ (r & 7);                    // source chunk (8 columns)
+        const int64_t t = tile / k_blocks;
+        const int b = static_cast<int>(tile - t * k_blocks);
+        const int64_t row = t * 256 + r;
+        const int col = b * 64 + j * 8;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (col < d_m) {
+            const uint16_t *src = row < key_rows ? w_k + row * d_m : w_v + (row - key_rows) * d_m;
+            val = __ldg(reinterpret_cast<const uint4 *>(src + col));
+        }
+        packed[i] = val;
+    }
+}
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -154,7 +179,12 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                     if (!mbar_wait(&empty_bar[s], ph ^ 1, &s_abort)) break;
                     mbar_arrive_expect_tx(&full_bar[s], Cfg::kStageBytes);
                     tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
-                    tma_load_2d(sB + s * Cfg::kBTile, map_w, &full_bar[s], kb * kBK, c0);
+                    if (BN == 256 && p.w_packed != nullptr)   // one linear 32 KB copy of the pre-swizzled tile
+                        bulk_load_1d(sB + s * Cfg::kBTile,
+                                     p.w_packed + (static_cast<int64_t>(nt) * p.k_blocks + kb) * Cfg::kBTile,
+                                     Cfg::kBTile, &full_bar[s]);
+                    else
+                        tma_load_2d(sB + s * Cfg::kBTile, map_w, &full_bar[s], kb * kBK, c0);
                     issued = it + 1;
                 }
             }

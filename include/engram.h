@@ -146,7 +146,23 @@ typedef struct engram_weights {
     const uint16_t *gamma_k; /* [d_h] RMSNorm gain of the key */
     const uint16_t *gamma_c; /* [d_h] RMSNorm gain of the conv input */
     const uint16_t *conv_w;  /* [d_h, conv_kernel]; tap i reads position t - i*dilation */
+    const void *w_packed;    /* NULL, or [W_k ; W_v] re-laid by engram_pack_weights from these same
+                                w_k / w_v; the projections then stream it instead (same results) */
 } engram_weights;
+
+/* Projection weights re-laid for streaming.  The projections read [W_k ; W_v] ((M+1)*d_h rows
+ * of d_m values) in tiles of 256 rows x 64 columns; in the row-major matrices each such tile
+ * is 256 separate 128-byte pieces 2*d_m bytes apart, which DRAM serves poorly when the
+ * weights do not stay in L2 (decode-sized batches stream all of them every step).  The packed
+ * copy stores every tile as one contiguous 32 KB block, already in the 128-byte-swizzled
+ * K-major shared-memory layout the tensor cores read, so each tile is fetched by one linear
+ * bulk copy.  Layout: tile (t, b) -- rows 256t..256t+255 of [W_k ; W_v], columns 64b..64b+63
+ * (zero beyond d_m) -- at byte (t * k_blocks + b) * 32768, k_blocks = ceil(d_m / 64); row r of
+ * the tile at r * 128; its 16-byte chunk j (columns 8j..8j+7) at chunk position j XOR (r mod 8).
+ * Only for d_h % 256 == 0 (otherwise the size is 0 and the row-major weights are used). */
+size_t engram_packed_weights_size(const engram_plan *plan);
+int engram_pack_weights(const engram_plan *plan, const uint16_t *w_k, const uint16_t *w_v, void *packed,
+                        size_t packed_bytes, engram_stream_t stream);
 
 /* Validate `cfg` and fill `plan` (host only, no CUDA call).  Checks: orders, K, H <= 32,
  * primality of every table_rows[h] (deterministic Miller-Rabin), d_e % 8 == 0 (d_e % 16 == 0

@@ -184,3 +184,22 @@ def test_cache_model_policy():
     assert m.step(np.array([[5], [1], [6], [101]])) == [1]
     assert m.tags[0].tolist() == [0, 2, 7, 0]
 
+
+def test_packed_weights_size_and_validation():
+    p = _plan()                                   # d_h 256, d_m 128: 2 row tiles x 2 k-blocks
+    assert E.engram_packed_weights_size(p) == 2 * 2 * 32768
+    assert E.engram_packed_weights_size(_plan(hidden_dim=384)) == 0
+    assert E.engram_packed_weights_size(_plan(num_branches=3)) == 4 * 2 * 32768
+    w = _native.engram_weights(*[C.c_void_p(256 * (i + 1)) for i in range(6)])
+    w.w_packed = 4096 + 8                         # misaligned
+    rc = E.lib.engram_gate_conv(p, C.byref(w), C.c_void_p(256), C.c_void_p(512), 1, 4, None,
+                                C.c_void_p(768), None, C.c_void_p(1024), 1 << 20, None)
+    assert rc == E.ENGRAM_ERR_INVALID_ARG and "w_packed" in E.last_error()
+    p384 = _plan(hidden_dim=384)
+    w.w_packed = 4096
+    rc = E.lib.engram_gate_conv(p384, C.byref(w), C.c_void_p(256), C.c_void_p(512), 1, 4, None,
+                                C.c_void_p(768), None, C.c_void_p(1024), 1 << 20, None)
+    assert rc == E.ENGRAM_ERR_INVALID_ARG and "packed" in E.last_error()
+    assert E.lib.engram_pack_weights(p384, C.c_void_p(256), C.c_void_p(512), C.c_void_p(768), 1 << 20,
+                                     None) == E.ENGRAM_ERR_UNSUPPORTED
+

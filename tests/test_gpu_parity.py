@@ -363,3 +363,80 @@ def test_forward_on_16x20m_tables_sampled_rows():
     finally:
         tables = m = None
         _free_device()
+
+
+@pytest.mark.slow
+def test_prefill_on_full_95gib_tables_sampled():
+    """32 x 8192 tokens (30% copied phrases) on the full 2 x 9,999,991 x 2560 tables, in the
+    benchmark's launch configuration, checked on sampled tokens (sequence starts, the edges of
+    128-token tiles and 144-token gate chunks, random) that the oracle computes one by one."""
+    wl = synth.get_workload("prefill20m")
+    free, _ = torch.cuda.mem_get_info()
+    if free < wl.table_bytes + (12 << 30):
+        pytest.skip("not enough device memory for the 95.4 GiB tables and the 262,144-token batch")
+    di = None
+    try:
+        di = DeviceInputs(wl).forward()
+        torch.cuda.synchronize()
+        w = di.host_weights()
+        rng = np.random.default_rng(31)
+        picks = [(0, 0), (0, 1), (0, 8), (0, 9), (5, 127), (5, 128), (9, 143), (9, 144), (31, wl.T - 1)]
+        picks += [(int(rng.integers(0, wl.B)), int(rng.integers(0, wl.T))) for _ in range(12)]
+        got_d, got_o = [], []
+        ref_d, ref_o = [], []
+        for b, t in picks:
+            n = b * wl.T + t
+            d_ref, o_ref = _window_oracle(wl, di, w, b, t)
+            got_d.append(di.delta[n].cpu().numpy())
+            got_o.append(to_host_u16(di.out[n]))
+            ref_d.append(d_ref)
+            ref_o.append(o_ref)
+        assert_delta_close(np.stack(got_d), np.stack(ref_d))
+        assert_out_close(np.stack(got_o), np.stack(ref_o))
+        assert E.engram_device_status(clear=True) == 0
+    finally:
+        di = None
+        _free_device()
+
+
+@pytest.mark.slow
+def test_decode_step_on_full_host_pinned_tables_sampled():
+    """One decode step of 64 sequences with the full 102 GB tables in pinned, mapped host
+    memory (distinct rows staged through HBM), checked on sampled sequences against the
+    oracle with the rows regenerated."""
+    import psutil
+    wl = synth.get_workload("hostpinned20m")
+    if psutil.virtual_memory().available < wl.table_bytes + (16 << 30):
+        pytest.skip("not enough host memory for 102 GB of pinned tables")
+    bufs = []
+    try:
+        for h in range(wl.H):
+            hm = fill_gpu.HostMapped(wl.primes[h], wl.d_e)
+            fill_gpu.fill_(hm.tensor, wl.table_spec(h))
+            bufs.append(hm)
+        torch.cuda.synchronize()
+        di = DeviceInputs(wl, tables=[b.tensor for b in bufs])
+        di.plan = E.Plan.from_workload(wl, host_tables=True)
+        di.ws = E.alloc_workspace(di.plan, wl.n_tok)
+        state_before = to_host_u16(di.conv_state)
+        hist_before = di.history.cpu().numpy()
+        di.forward()
+        torch.cuda.synchronize()
+        w = di.host_weights()
+        seqs = np.sort(np.random.default_rng(41).choice(wl.B, 10, replace=False))
+        ids = di.ids_np[seqs]
+        idx = oracle.hash_ids(ids, wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id, history=hist_before[seqs])
+        tables = [synth.fill_rows_bf16(wl.table_spec(h), wl.d_e, idx[:, h]) for h in range(wl.H)]
+        m = oracle.gather(np.tile(np.arange(len(seqs), dtype=np.uint32)[:, None], (1, wl.H)), tables)
+        h_rows = synth.fill_rows_bf16(wl.h_spec(0), wl.d_h, seqs)
+        ref = oracle.gate_conv(h_rows, m, w["Wk"], w["Wv"], w["gamma_q"], w["gamma_k"], w["gamma_c"],
+                               w["conv_w"], len(seqs), 1, dil=wl.conv_dilation, eps=wl.eps,
+                               conv_state=state_before[seqs], want_state=True)
+        assert_delta_close(di.delta.cpu().numpy()[seqs], ref["delta"])
+        assert_out_close(to_host_u16(di.out)[seqs], ref["out"])
+        assert E.engram_device_status(clear=True) == 0
+    finally:
+        di = None
+        for b in bufs:
+            b.close()
+        _free_device()

@@ -11,6 +11,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "engram.h"
 #include "kernels_gate.cuh"
@@ -112,6 +113,24 @@ struct Workspace {
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Launch with programmatic stream serialization: the kernel may start while the previous
+// kernel on the stream finishes (see pdl_wait / pdl_launch_dependents).
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 bool fp8_tables(const engram_plan *plan) { return plan->cfg.table_dtype == ENGRAM_TABLE_FP8_E4M3; }
 int table_elem_bytes(const engram_plan *plan) { return fp8_tables(plan) ? 1 : 2; }
@@ -318,9 +337,9 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
     const int64_t sms = sm_count();
     dim3 grid(static_cast<unsigned>(total < sms ? total : sms));
-    engram::proj_kernel<BN><<<grid, engram::kProjThreads, engram::ProjCfg<BN>::kSmemBytes, stream>>>(
-        map_m, map_wk, map_wv, p);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "proj_kernel launch");
+    ENGRAM_CUDA_TRY(launch_pdl(engram::proj_kernel<BN>, grid, dim3(engram::kProjThreads), engram::ProjCfg<BN>::kSmemBytes,
+                               stream, map_m, map_wk, map_wv, p),
+                    "proj_kernel launch");
     if (params_out) *params_out = p;
     if (p.k_splits > 1 && run_reduce) {
         engram::splitk_reduce_kernel<<<dim3(p.n_tiles, static_cast<unsigned>(n_tok)), engram::kReduceThreads, 0,
@@ -740,7 +759,9 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
             engram::decode_fused_kernel<4>, engram::decode_fused_kernel<5>, engram::decode_fused_kernel<6>,
             engram::decode_fused_kernel<7>, engram::decode_fused_kernel<8>};
         const int pairs = (d_h / 2 + engram::kFusedDecodeThreads - 1) / engram::kFusedDecodeThreads;
-        kernels[pairs - 1]<<<static_cast<unsigned>(B), engram::kFusedDecodeThreads, 0, stream>>>(pp, gp);
+        ENGRAM_CUDA_TRY(launch_pdl(kernels[pairs - 1], dim3(static_cast<unsigned>(B)), dim3(engram::kFusedDecodeThreads),
+                                   0, stream, pp, gp),
+                        "decode_fused_kernel launch");
         ENGRAM_CUDA_TRY(cudaGetLastError(), "decode_fused_kernel launch");
         return ENGRAM_OK;
     }

@@ -658,6 +658,7 @@ __global__ void __launch_bounds__(kFusedDecodeThreads, 2) decode_fused_kernel(co
             hv[k] = __ldg(reinterpret_cast<const uint32_t *>(pp.h + static_cast<int64_t>(b) * d_h + c));
         }
     }
+    pdl_wait();   // the split accumulators come from the projection kernel before this one
     for (int ks = 0; ks < pp.k_splits; ++ks) {
         const float *src = acc + ks * split_stride;
 #pragma unroll

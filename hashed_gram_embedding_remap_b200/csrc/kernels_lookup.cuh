@@ -8,6 +8,7 @@
 
 #include "engram.h"
 
+#include "ptx.cuh"
 #include "status.cuh"
 
 namespace engram {
@@ -297,6 +298,7 @@ __global__ void __launch_bounds__(256) lookup_kernel(const int32_t *__restrict__
                                                      const int32_t *__restrict__ history,
                                                      int32_t *__restrict__ xr_out, uint4 *__restrict__ m,
                                                      const __grid_constant__ LookupParams p) {
+    pdl_launch_dependents();   // the projection may start streaming its weights now
     const HashParams &hp = p.hash;
     const int64_t n_tok = static_cast<int64_t>(hp.B) * hp.T;
     const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;

@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(tempty_bar + NACC);
     __shared__ int s_abort;
 
+    pdl_launch_dependents();   // the kernel after this one may load its independent inputs now
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const int mn_tiles = p.m_tiles * p.n_tiles;
@@ -164,27 +165,54 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            int it = 0, issued = 0;
-            for (int t = blockIdx.x; t < total && !s_abort; t += gridDim.x) {
-                const int ks = t / mn_tiles, tmn = t - ks * mn_tiles;
-                const int mt = tmn / p.n_tiles, nt = tmn - mt * p.n_tiles;
+            // unit t -> (k split, m tile, n tile) and the weight tile it streams
+            auto unit = [&](int t, int &ks, int &mt, int &nt, int &kb0, int &kb1) {
+                ks = t / mn_tiles;
+                const int tmn = t - ks * mn_tiles;
+                mt = tmn / p.n_tiles;
+                nt = tmn - mt * p.n_tiles;
+                kb0 = ks * p.kb_per_split;
+                kb1 = min(p.k_blocks, kb0 + p.kb_per_split);
+            };
+            auto load_b = [&](int s, int nt, int kb) {
                 const bool is_key = nt < key_tiles;
-                const CUtensorMap *map_w = is_key ? &map_wk : &map_wv;
-                const int c0 = (is_key ? nt : nt - key_tiles) * BN;   // row of the stacked W_k, or of W_v
+                if (BN == 256 && p.w_packed != nullptr)   // one linear 32 KB copy of the pre-swizzled tile
+                    bulk_load_1d(sB + s * Cfg::kBTile, p.w_packed + (static_cast<int64_t>(nt) * p.k_blocks + kb) * Cfg::kBTile,
+                                 Cfg::kBTile, &full_bar[s]);
+                else   // row of the stacked W_k, or of W_v
+                    tma_load_2d(sB + s * Cfg::kBTile, is_key ? &map_wk : &map_wv, &full_bar[s], kb * kBK,
+                                (is_key ? nt : nt - key_tiles) * BN);
+            };
+            // The weight tiles of this CTA's first stages do not depend on the previous kernel on
+            // the stream: they are issued before waiting for it (programmatic dependent launch);
+            // the m tiles, which that kernel writes, follow the wait.
+            int pre = 0;
+            if (blockIdx.x < total) {
+                int ks, mt, nt, kb0, kb1;
+                unit(blockIdx.x, ks, mt, nt, kb0, kb1);
+                pre = min(S, kb1 - kb0);
+                for (int q = 0; q < pre; ++q) {   // fresh stages: nothing to wait for
+                    mbar_arrive_expect_tx(&full_bar[q], Cfg::kStageBytes);
+                    load_b(q, nt, kb0 + q);
+                }
+            }
+            pdl_wait();
+            int it = 0, issued = pre;
+            for (int t = blockIdx.x; t < total && !s_abort; t += gridDim.x) {
+                int ks, mt, nt, kb0, kb1;
+                unit(t, ks, mt, nt, kb0, kb1);
                 const int m0 = mt * kBM;
-                const int kb0 = ks * p.kb_per_split, kb1 = min(p.k_blocks, kb0 + p.kb_per_split);
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
+                    if (it < pre) {   // weight tile and byte count already issued
+                        tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
+                        continue;
+                    }
                     const uint32_t ph = (it / S) & 1;
                     if (!mbar_wait(&empty_bar[s], ph ^ 1, &s_abort)) break;
                     mbar_arrive_expect_tx(&full_bar[s], Cfg::kStageBytes);
                     tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
-                    if (BN == 256 && p.w_packed != nullptr)   // one linear 32 KB copy of the pre-swizzled tile
-                        bulk_load_1d(sB + s * Cfg::kBTile,
-                                     p.w_packed + (static_cast<int64_t>(nt) * p.k_blocks + kb) * Cfg::kBTile,
-                                     Cfg::kBTile, &full_bar[s]);
-                    else
-                        tma_load_2d(sB + s * Cfg::kBTile, map_w, &full_bar[s], kb * kBK, c0);
+                    load_b(s, nt, kb);
                     issued = it + 1;
                 }
             }

@@ -25,6 +25,17 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the previous
+// kernel on the stream is still running, once every CTA of that kernel has executed
+// pdl_launch_dependents() (or exited).  pdl_wait() blocks the calling thread until the
+// previous kernel has completed and its memory is visible; a thread must call it before it
+// touches anything that kernel writes.  Both are no-ops for a kernel launched without it.
+// A dependent kernel is only scheduled after all CTAs of the previous one are resident, so
+// the wait always ends.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

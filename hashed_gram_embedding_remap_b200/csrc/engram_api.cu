@@ -1140,8 +1140,9 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const void 
         return rc;
     if ((rc = rec(4)) != ENGRAM_OK) return rc;
     if (history != nullptr && plan->hist_len > 0) {
-        engram::advance_history_kernel<<<(B + 127) / 128, 128, 0, stream>>>(xr, B, T, history, plan->hist_len);
-        ENGRAM_CUDA_TRY(cudaGetLastError(), "advance_history_kernel launch");
+        ENGRAM_CUDA_TRY(launch_pdl(engram::advance_history_kernel, dim3((B + 127) / 128), dim3(128), 0, stream,
+                                   static_cast<const int32_t *>(xr), B, T, history, static_cast<int32_t>(plan->hist_len)),
+                        "advance_history_kernel launch");
     }
     return ENGRAM_OK;
 }

@@ -121,6 +121,7 @@ __global__ void remap_kernel(const int32_t *__restrict__ ids, int64_t n, const i
 // slots are rewritten in increasing order, each read slot lies at or after its target.
 __global__ void advance_history_kernel(const int32_t *__restrict__ xr, int32_t B, int32_t T,
                                        int32_t *history, int32_t hist_len) {
+    pdl_wait();   // launched early behind the gate kernel: xr and history belong to earlier kernels
     const int32_t b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= B) return;
     int32_t *hb = history + static_cast<int64_t>(b) * hist_len;

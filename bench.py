@@ -347,7 +347,7 @@ def run_engram(args, wl, world, rank, local):
     history = torch.from_numpy(wl.history()).to(dev) if wl.decode else None
     state = fill_gpu.filled((wl.B * M, wl.state_len, wl.d_h), wl.state_spec(), dev) if wl.decode else None
     plan = E.Plan.from_workload(wl)
-    packed = E.pack_weights(plan, wk, wv) if args.packed else None
+    packed = E.pack_weights(plan, wk, wv) if args.packed and E.engram_packed_weights_size(plan) else None
     weights = E.Weights(wk, wv, one, one, one, cw, packed=packed)
     out = torch.empty((wl.h_rows, wl.d_h), dtype=torch.bfloat16, device=dev)
     ws = E.alloc_workspace(plan, wl.n_tok, dev)
@@ -533,7 +533,7 @@ def run_engram(args, wl, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Zipf ids, counter-based bf16 tables/weights)",
-        "config": workload_config(wl, world),
+        "config": dict(workload_config(wl, world), weights="packed" if packed is not None else "row-major"),
         "stages_ms": stage_ms, "hbm": hbm, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * (E.ENGRAM_FORWARD_STAGES + (1 if wl.decode else 0)),
         "launch_mode": "eager" if args.eager else "one CUDA graph of the K timed steps (stage times from a "
@@ -580,7 +580,7 @@ def run_hostpinned(args, wl, world, rank, local):
     wv = fill_gpu.filled((wl.d_h, wl.d_m), wl.wv_spec(), dev)
     one = torch.full((wl.d_h,), 0x3F80, dtype=torch.int16, device=dev).view(torch.bfloat16)
     cw = fill_gpu.filled((wl.d_h, wl.conv_kernel), wl.conv_spec(), dev)
-    packed = E.pack_weights(plan, wk, wv) if args.packed else None
+    packed = E.pack_weights(plan, wk, wv) if args.packed and E.engram_packed_weights_size(plan) else None
     weights = E.Weights(wk, wv, one, one, one, cw, packed=packed)
     out = torch.empty((B, wl.d_h), dtype=torch.bfloat16, device=dev)
     ws = E.alloc_workspace(plan, B, dev)
@@ -778,8 +778,9 @@ def main():
     ap.add_argument("--table-rows", type=int, default=0, help="override the table size (largest prime <= N)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's sequences per step")
-    ap.add_argument("--packed", action="store_true",
-                    help="stream the projection weights from their packed copy (engram_pack_weights)")
+    ap.add_argument("--no-packed", dest="packed", action="store_false",
+                    help="stream the row-major projection weights instead of their packed copy "
+                         "(engram_pack_weights, made once before timing; used when d_h % 256 == 0)")
     ap.add_argument("--cache-slots", type=int, default=0,
                     help="host-resident tables: HBM row cache of this many slots per table (power of two; 0 = none)")
     ap.add_argument("--table-dtype", choices=["bf16", "fp8"], default="bf16",
@@ -799,8 +800,8 @@ def main():
         wl = wl.with_(B=args.batch, name=f"{wl.name}[B={args.batch}]")
     if args.cache_slots:
         wl = wl.with_(name=f"{wl.name}[cache={args.cache_slots}]")
-    if args.packed:
-        wl = wl.with_(name=f"{wl.name}[packed]")
+    if not args.packed:
+        wl = wl.with_(name=f"{wl.name}[row-major weights]")
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -229,6 +229,7 @@ __device__ __forceinline__ typename RowChunk<FP8>::type zero_chunk() {
 template <int UNROLL, bool FP8, typename Idx>
 __global__ void __launch_bounds__(256) gather_kernel(const uint32_t *__restrict__ idx, uint4 *__restrict__ m,
                                                      const __grid_constant__ GatherParams p) {
+    pdl_launch_dependents();   // the projection may prefetch its weight tiles while this drains
     const Idx total = static_cast<Idx>(p.n_tok * p.chunks_per_tok);
     const Idx stride = static_cast<Idx>(gridDim.x) * blockDim.x;
     for (Idx base = static_cast<Idx>(blockIdx.x) * blockDim.x + threadIdx.x; base < total; base += stride * UNROLL) {

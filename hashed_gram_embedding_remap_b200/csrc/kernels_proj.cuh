@@ -36,9 +36,14 @@ struct ProjCfg {
     static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
     static constexpr int kAccum = 2;                              // TMEM accumulators (double buffer)
     static constexpr int kTmemCols = kAccum * BN;                 // fp32 columns, power of two
-    // dynamic smem: [align pad][stages x A][stages x B][full, empty, tmem_full, tmem_empty][tmem addr]
+    // split-K epilogue: one 32 x 32 fp32 transpose tile per epilogue warp (rows padded to 36
+    // floats: 16-byte row starts, conflict-free quarter-warp phases)
+    static constexpr int kTrStride = 36;
+    static constexpr int kTrBytes = 4 * 32 * kTrStride * 4;
+    // dynamic smem: [align pad][stages x A][stages x B][transpose tiles]
+    //               [full, empty, tmem_full, tmem_empty][tmem addr]
     static constexpr int kBarBytes = (2 * kStages + 2 * kAccum) * 8;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 16;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kTrBytes + kBarBytes + 16;
 };
 
 struct ProjParams {
@@ -124,7 +129,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + S * Cfg::kATile;
-    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes);
+    float *s_tr = reinterpret_cast<float *>(smem + S * Cfg::kStageBytes);
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes + Cfg::kTrBytes);
     uint64_t *empty_bar = full_bar + S;
     uint64_t *tfull_bar = empty_bar + S;      // MMA -> epilogue, one per accumulator
     uint64_t *tempty_bar = tfull_bar + NACC;  // epilogue -> MMA, one per accumulator
@@ -279,15 +285,32 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             for (int cc = 0; cc < BN; cc += 32) {
                 float accv[32];
                 tmem_ld32(taddr + cc, accv);
-                if (!valid) continue;
                 if (p.k_splits > 1) {
-                    // split-K: raw partial accumulator; splitk_reduce_kernel finishes the tile
-                    float4 *ap = reinterpret_cast<float4 *>(
-                        p.acc_out + (static_cast<int64_t>(ks) * p.n_tok + n) * (p.n_tiles * BN) + nt * BN + cc);
+                    // split-K: raw partial accumulator; the reduction finishes the tile.  Each
+                    // lane holds 32 columns of its own row: the warp's 32 x 32 block goes through
+                    // shared memory so that every store instruction writes 4 whole 128-byte
+                    // row segments instead of 32 scattered 16-byte pieces.
+                    float *tr = s_tr + sub * (32 * Cfg::kTrStride);
+                    float4 *mine = reinterpret_cast<float4 *>(tr + lane * Cfg::kTrStride);
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
-                        ap[q] = make_float4(accv[4 * q], accv[4 * q + 1], accv[4 * q + 2], accv[4 * q + 3]);
-                } else if (is_key) {
+                        mine[q] = make_float4(accv[4 * q], accv[4 * q + 1], accv[4 * q + 2], accv[4 * q + 3]);
+                    __syncwarp();
+                    const int c4 = (lane & 7) * 4;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = i * 4 + (lane >> 3);                      // row within the warp's 32
+                        const int64_t nr = static_cast<int64_t>(mt) * kBM + sub * 32 + r;
+                        if (nr < p.n_tok)
+                            *reinterpret_cast<float4 *>(p.acc_out + (static_cast<int64_t>(ks) * p.n_tok + nr) *
+                                                                        (p.n_tiles * BN) + nt * BN + cc + c4) =
+                                *reinterpret_cast<const float4 *>(tr + r * Cfg::kTrStride + c4);
+                    }
+                    __syncwarp();   // the tile is rewritten by the next column block
+                    continue;
+                }
+                if (!valid) continue;
+                if (is_key) {
                     const uint4 *hp = reinterpret_cast<const uint4 *>(p.h + (n * p.M + br) * p.d_h + c0 + cc);
                     const uint4 *gq = reinterpret_cast<const uint4 *>(p.gamma_q + c0 + cc);
                     const uint4 *gk = reinterpret_cast<const uint4 *>(p.gamma_k + c0 + cc);

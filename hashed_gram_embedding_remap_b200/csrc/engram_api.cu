@@ -557,18 +557,19 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
         p.scal = scal;
     }
     if (p.scal != nullptr) {
-        // streaming kernel: 9*G tokens per CTA, G chosen so that the last wave of CTAs is
-        // as full as possible
+        // streaming kernel: 9*G tokens per CTA, each thread walking 9*(G+1) positions (the
+        // first 9 are the conv halo).  G minimises waves x (positions walked per CTA + a
+        // fixed per-CTA cost worth 36 positions): long sequences take the longest walk that
+        // fills the waves, short batches (few CTAs in all) a short one.
         const int slices = (d_h / 4 + engram::kStreamThreads - 1) / engram::kStreamThreads;
         const int64_t per_wave = static_cast<int64_t>(sm_count()) * engram::kStreamMinBlocks;
         int best_g = 16;
-        double best_eff = -1.0;
-        for (int g : {16, 12, 8}) {
+        int64_t best_cost = -1;
+        for (int g : {16, 8, 4, 1}) {
             const int64_t ctas = static_cast<int64_t>((T + 9 * g - 1) / (9 * g)) * p.M * B * slices;
-            const double waves = static_cast<double>(ctas) / static_cast<double>(per_wave);
-            const double eff = waves / std::ceil(waves);
-            if (eff > best_eff + 0.05) {
-                best_eff = eff;
+            const int64_t cost = ((ctas + per_wave - 1) / per_wave) * (9 * (g + 1) + 36);
+            if (best_cost < 0 || cost < best_cost) {
+                best_cost = cost;
                 best_g = g;
             }
         }
@@ -577,8 +578,9 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
         using SK = void (*)(const engram::GateParams);
         const bool dl = delta != nullptr;
         const SK k = best_g == 16 ? (dl ? engram::gate_stream_kernel<16, true> : engram::gate_stream_kernel<16, false>)
-                   : best_g == 12 ? (dl ? engram::gate_stream_kernel<12, true> : engram::gate_stream_kernel<12, false>)
-                                  : (dl ? engram::gate_stream_kernel<8, true> : engram::gate_stream_kernel<8, false>);
+                   : best_g == 8  ? (dl ? engram::gate_stream_kernel<8, true> : engram::gate_stream_kernel<8, false>)
+                   : best_g == 4  ? (dl ? engram::gate_stream_kernel<4, true> : engram::gate_stream_kernel<4, false>)
+                                  : (dl ? engram::gate_stream_kernel<1, true> : engram::gate_stream_kernel<1, false>);
         k<<<grid, engram::kStreamThreads, 0, stream>>>(p);
         ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_stream_kernel launch");
         return ENGRAM_OK;

@@ -155,9 +155,15 @@ PARITY_CASES = {
     "seq_shorter_than_halo": small_workload("short", B=40, T=7, K=2, d_e=16, d_h=128),
     # gate kernel over several channel slices, two sequences with ragged 48-token chunks
     "gate_3_slices": small_workload("g3s", B=2, T=301, K=2, d_e=24, d_h=1536),
+    # streaming gate kernel with 72-token CTAs (the longer walks serve the bench workloads;
+    # 36- and 9-token CTAs serve the small cases above); 6000 = 83 x 72 + 24: ragged last CTA
+    "gate_walk72": small_workload("gw72", B=4, T=6000, K=2, d_e=16, d_h=256),
     # decode-sized batches: the projection splits K across CTAs (partial accumulators + reduce)
     "splitk_64tok": small_workload("splitk64", B=64, T=1, K=1, d_e=512, d_h=512),          # 4 splits
     "splitk_ragged_k": small_workload("splitk200", B=100, T=2, K=1, d_e=360, d_h=512),     # d_m=720, 3 splits
+    # the 20M-row layer's widths (d_e = 2560, d_m = 5120, d_h = 2560) on 210 tokens: split-K
+    # over two 128-token tiles, the second ragged
+    "splitk_d2560": small_workload("splitk2560", B=3, T=70, K=1, d_e=2560, d_h=2560),
 }
 
 
@@ -196,17 +202,20 @@ def test_gate_conv_entry_matches_forward():
     assert torch.equal(out_fwd.view(torch.int16), out2.view(torch.int16))
 
 
-@pytest.mark.parametrize("geom", ["small", "splitk", "splitk_256seq", "chunk4"])
+@pytest.mark.parametrize("geom", ["small", "splitk", "splitk_256seq", "splitk_d2560", "chunk4"])
 def test_decode_steps_match_oracle_and_update_state(geom):
     """Consecutive calls carrying the hash history and conv state: one token per call
-    (one-token decode kernels, with and without split-K, over one and two 128-token tiles)
-    and four tokens per call (the chain kernel reading and rewriting the carried state)."""
+    (one-token decode kernels, with and without split-K, over one and two 128-token tiles,
+    also at the 20M-row layer's widths) and four tokens per call (the chain kernel reading
+    and rewriting the carried state)."""
     if geom == "small":
         wl = small_workload("dec", B=6, T=1, K=2, d_e=32, d_h=256, decode=True)
     elif geom == "splitk":
         wl = small_workload("dec_split", B=32, T=1, K=1, d_e=512, d_h=512, decode=True)
     elif geom == "splitk_256seq":
         wl = small_workload("dec_256", B=256, T=1, K=1, d_e=512, d_h=512, decode=True)
+    elif geom == "splitk_d2560":
+        wl = small_workload("dec_2560", B=200, T=1, K=1, d_e=2560, d_h=2560, decode=True)
     else:
         wl = small_workload("dec_chunk", B=5, T=4, K=2, d_e=32, d_h=256, decode=True)
     di = DeviceInputs(wl, random_gammas=geom != "small")
@@ -214,7 +223,7 @@ def test_decode_steps_match_oracle_and_update_state(geom):
     tables = [synth.fill_bf16(wl.table_spec(h), (wl.primes[h], wl.d_e)) for h in range(wl.H)]
     hist = wl.history()
     state = to_host_u16(di.conv_state)
-    for step in range(12):
+    for step in range(3 if geom == "splitk_d2560" else 12):
         ids_np = synth.zipf_ids(wl.vocab_in, 1.1, (wl.B, wl.T), 500 + step)
         h_np = synth.fill_bf16(wl.h_spec(step), (wl.B * wl.T, wl.d_h))
         di.ids = to_dev(ids_np)

@@ -543,8 +543,9 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
     }
     if (fast && conv_state != nullptr && T == 1) {
         const unsigned dslices = static_cast<unsigned>((d_h / 2 + engram::kDecodeThreads - 1) / engram::kDecodeThreads);
-        engram::gate_conv_decode_kernel<<<dim3(dslices, static_cast<unsigned>(B)), engram::kDecodeThreads, 0, stream>>>(p);
-        ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_conv_decode_kernel launch");
+        ENGRAM_CUDA_TRY(launch_pdl(engram::gate_conv_decode_kernel, dim3(dslices, static_cast<unsigned>(B)),
+                                   dim3(engram::kDecodeThreads), 0, stream, p),
+                        "gate_conv_decode_kernel launch");
         return ENGRAM_OK;
     }
     dim3 grid(static_cast<unsigned>((T + p.tok_chunk - 1) / p.tok_chunk), static_cast<unsigned>(B), slices);

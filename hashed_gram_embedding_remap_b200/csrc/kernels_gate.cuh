@@ -542,20 +542,39 @@ constexpr int kDecodeThreads = 256;
 __global__ void __launch_bounds__(kDecodeThreads) gate_conv_decode_kernel(const __grid_constant__ GateParams p) {
     constexpr int S = 9;
     __shared__ float s_gb[2];
+    pdl_launch_dependents();   // the history update may be scheduled now (it waits for this kernel)
     const int b = blockIdx.y;
     const float inv_d = 1.f / static_cast<float>(p.d_h);
+    // this thread's loads that do not depend on the projection first
+    const int q = blockIdx.x * blockDim.x + threadIdx.x;
+    const bool active = q < p.d_h / 2;
+    const int c = q * 2;
+    uint32_t st[S];
+    float2 v = make_float2(0.f, 0.f);
+    uint32_t hw = 0, gw = 0;
+    uint2 w0 = make_uint2(0, 0), w1 = make_uint2(0, 0);
+    uint16_t *state = p.conv_state + static_cast<int64_t>(b) * S * p.d_h + c;
+    if (active) {
+#pragma unroll
+        for (int k = 0; k < S; ++k) st[k] = *reinterpret_cast<const uint32_t *>(state + k * p.d_h);
+        hw = __ldg(reinterpret_cast<const uint32_t *>(p.h + static_cast<int64_t>(b) * p.d_h + c));
+        gw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_c + c));
+        w0 = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + c * 4));
+        w1 = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + (c + 1) * 4));
+    }
+    pdl_wait();   // v and the gate sums come from the projection kernel before this one
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
         const float4 *pp = p.part + static_cast<int64_t>(b) * p.n_tiles;
         float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
         for (int j = lane; j < p.n_tiles; j += 32) {
-            const float4 q = __ldg(pp + j);
+            const float4 e = __ldg(pp + j);
             if (j < p.n_key_tiles) {
-                s0 += q.x;
-                s1 += q.y;
-                s2 += q.z;
+                s0 += e.x;
+                s1 += e.y;
+                s2 += e.z;
             } else {
-                s3 += q.x;
+                s3 += e.x;
             }
         }
 #pragma unroll
@@ -573,24 +592,9 @@ __global__ void __launch_bounds__(kDecodeThreads) gate_conv_decode_kernel(const 
             s_gb[1] = g / sqrtf(g * g * s3 * inv_d + p.eps);
         }
     }
-    // issue this thread's loads while warp 0 reduces the scalars
-    const int q = blockIdx.x * blockDim.x + threadIdx.x;
-    const bool active = q < p.d_h / 2;
-    const int c = q * 2;
-    uint32_t st[S];
-    float2 v = make_float2(0.f, 0.f);
-    uint32_t hw = 0, gw = 0;
-    uint2 w0 = make_uint2(0, 0), w1 = make_uint2(0, 0);
-    uint16_t *state = p.conv_state + static_cast<int64_t>(b) * S * p.d_h + c;
     if (active) {
-#pragma unroll
-        for (int k = 0; k < S; ++k) st[k] = *reinterpret_cast<const uint32_t *>(state + k * p.d_h);
         const uint32_t vw = __ldg(reinterpret_cast<const uint32_t *>(p.v + static_cast<int64_t>(b) * p.d_h + c));
         v = make_float2(v_lo(vw), v_hi(vw));
-        hw = __ldg(reinterpret_cast<const uint32_t *>(p.h + static_cast<int64_t>(b) * p.d_h + c));
-        gw = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_c + c));
-        w0 = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + c * 4));
-        w1 = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + (c + 1) * 4));
     }
     __syncthreads();
     if (!active) return;

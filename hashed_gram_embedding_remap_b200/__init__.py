@@ -13,5 +13,5 @@ from ._native import (  # noqa: F401
     engram_advance_history, engram_device_status, engram_forward, engram_gate_conv,
     engram_gate_conv_noalloc, engram_gather, engram_hash, engram_stage_rows, engram_stage_rows_cached, RowCache,
     pack_weights, engram_packed_weights_size,
-    engram_remap, engram_workspace_size, last_error, lib, version,
+    engram_remap, engram_workspace_size, kernel_launches, last_error, lib, version,
 )

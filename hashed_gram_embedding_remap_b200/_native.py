@@ -122,6 +122,7 @@ def _load():
         "engram_last_error": (C.c_char_p, []),
         "engram_version": (C.c_char_p, []),
         "engram_sizeof": (sz, [C.c_char_p]),
+        "engram_kernel_launches": (C.c_uint64, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -144,6 +145,11 @@ def last_error() -> str:
 
 def version() -> str:
     return lib.engram_version().decode()
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched in this process so far (engram_kernel_launches)."""
+    return int(lib.engram_kernel_launches())
 
 
 def _check(rc: int):

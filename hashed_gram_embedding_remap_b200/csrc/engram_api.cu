@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -42,6 +43,16 @@ int cuda_fail(cudaError_t e, const char *what) {
     do {                                         \
         cudaError_t e_ = (expr);                 \
         if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+    } while (0)
+
+// Kernels launched by this library in this process (engram_kernel_launches).
+std::atomic<uint64_t> g_kernel_launches{0};
+
+// After a <<<...>>> launch: count it, then check that it was accepted.
+#define ENGRAM_LAUNCHED(what)                                                 \
+    do {                                                                      \
+        g_kernel_launches.fetch_add(1, std::memory_order_relaxed);            \
+        ENGRAM_CUDA_TRY(cudaGetLastError(), what);                            \
     } while (0)
 
 // ---------------------------------------------------------------- host-side integer helpers
@@ -129,7 +140,9 @@ cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    if (e == cudaSuccess) g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
+    return e;
 }
 
 bool fp8_tables(const engram_plan *plan) { return plan->cfg.table_dtype == ENGRAM_TABLE_FP8_E4M3; }
@@ -344,7 +357,7 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     if (p.k_splits > 1 && run_reduce) {
         engram::splitk_reduce_kernel<<<dim3(p.n_tiles, static_cast<unsigned>(n_tok)), engram::kReduceThreads, 0,
                                        stream>>>(p, BN);
-        ENGRAM_CUDA_TRY(cudaGetLastError(), "splitk_reduce_kernel launch");
+        ENGRAM_LAUNCHED("splitk_reduce_kernel launch");
     }
     return ENGRAM_OK;
 }
@@ -413,7 +426,7 @@ int launch_lookup(const engram_plan *plan, const int32_t *ids, const int32_t *re
     auto kern = fp8_tables(plan) ? engram::lookup_kernel<true> : engram::lookup_kernel<false>;
     kern<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(ids, remap, history, xr_out,
                                                                 reinterpret_cast<uint4 *>(m), p);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "lookup_kernel launch");
+    ENGRAM_LAUNCHED("lookup_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -424,7 +437,7 @@ int launch_hash(const engram_plan *plan, const int32_t *ids, const int32_t *rema
     const int threads = 256;
     const unsigned blocks = static_cast<unsigned>((n_tok + threads - 1) / threads);
     engram::hash_kernel<<<blocks, threads, 0, stream>>>(ids, remap, history, idx, xr_out, p);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "hash_kernel launch");
+    ENGRAM_LAUNCHED("hash_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -470,7 +483,7 @@ int launch_gather(const engram_plan *plan, const uint32_t *idx, const void *cons
         kern = unroll == 8 ? (f8 ? engram::gather_kernel<8, true, int64_t> : engram::gather_kernel<8, false, int64_t>)
                            : (f8 ? engram::gather_kernel<4, true, int64_t> : engram::gather_kernel<4, false, int64_t>);
     kern<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(idx, reinterpret_cast<uint4 *>(m), p);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "gather_kernel launch");
+    ENGRAM_LAUNCHED("gather_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -554,7 +567,7 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
         const int64_t items = static_cast<int64_t>(B) * T * p.M;
         engram::gate_scalars_kernel<<<static_cast<unsigned>((items * 8 + 255) / 256), 256, 0, stream>>>(
             part, static_cast<int64_t>(B) * T, n_tiles, p.n_key_tiles, p.M, d_h, p.eps, p.inv_sqrt_d, scal);
-        ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_scalars_kernel launch");
+        ENGRAM_LAUNCHED("gate_scalars_kernel launch");
         p.scal = scal;
     }
     if (p.scal != nullptr) {
@@ -583,12 +596,12 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
                    : best_g == 4  ? (dl ? engram::gate_stream_kernel<4, true> : engram::gate_stream_kernel<4, false>)
                                   : (dl ? engram::gate_stream_kernel<1, true> : engram::gate_stream_kernel<1, false>);
         k<<<grid, engram::kStreamThreads, 0, stream>>>(p);
-        ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_stream_kernel launch");
+        ENGRAM_LAUNCHED("gate_stream_kernel launch");
         return ENGRAM_OK;
     }
     if (fast) engram::gate_conv_k4d3_kernel<kChain><<<grid, threads, 0, stream>>>(p);
     else engram::gate_conv_kernel<<<grid, threads, smem, stream>>>(p);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "gate_conv_kernel launch");
+    ENGRAM_LAUNCHED("gate_conv_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -606,7 +619,7 @@ int launch_stage(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, co
                         "cudaFuncSetAttribute(stage_dedup_kernel)");
     engram::stage_dedup_kernel<<<H, engram::kDedupThreads, smem, stream>>>(
         idx, static_cast<int32_t>(n_tok), H, capacity, staged_idx, unique_rows, n_unique);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "stage_dedup_kernel launch");
+    ENGRAM_LAUNCHED("stage_dedup_kernel launch");
     engram::StageParams p{};
     for (int h = 0; h < H; ++h) {
         p.table[h] = tables[h];
@@ -626,7 +639,7 @@ int launch_stage(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, co
     if (blocks < 1) blocks = 1;
     if (cache == nullptr) {
         engram::stage_copy_kernel<kUnroll><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
-        ENGRAM_CUDA_TRY(cudaGetLastError(), "stage_copy_kernel launch");
+        ENGRAM_LAUNCHED("stage_copy_kernel launch");
         return ENGRAM_OK;
     }
     engram::CacheParams cp{};
@@ -645,13 +658,13 @@ int launch_stage(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, co
     cp.capacity = capacity;
     const dim3 rgrid(static_cast<unsigned>((n_tok + 255) / 256), static_cast<unsigned>(H));
     engram::cache_probe_kernel<<<rgrid, 256, 0, stream>>>(cp);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "cache_probe_kernel launch");
+    ENGRAM_LAUNCHED("cache_probe_kernel launch");
     engram::cache_decide_kernel<<<rgrid, 256, 0, stream>>>(cp);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "cache_decide_kernel launch");
+    ENGRAM_LAUNCHED("cache_decide_kernel launch");
     engram::cache_copy_kernel<kUnroll><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p, cp);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "cache_copy_kernel launch");
+    ENGRAM_LAUNCHED("cache_copy_kernel launch");
     engram::cache_commit_kernel<<<rgrid, 256, 0, stream>>>(cp);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "cache_commit_kernel launch");
+    ENGRAM_LAUNCHED("cache_commit_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -710,7 +723,7 @@ int launch_fused_gate(const engram_plan *plan, const engram_weights *w, const ui
     const unsigned grid = static_cast<unsigned>(p.n_units < sms ? p.n_units : sms);
     engram::fused_proj_gate_kernel<256><<<grid, engram::kFusedThreads, engram::FusedCfg<256>::kSmemBytes, stream>>>(
         map_m, map_wk, map_wv, p);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "fused_proj_gate_kernel launch");
+    ENGRAM_LAUNCHED("fused_proj_gate_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -915,7 +928,7 @@ int engram_remap(const engram_plan *plan, const int32_t *ids, int64_t n, const i
     if (blocks > 65535LL * 16) blocks = 65535LL * 16;
     engram::remap_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
         ids, n, remap, plan->cfg.vocab_in, plan->cfg.pad_id, out);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "remap_kernel launch");
+    ENGRAM_LAUNCHED("remap_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -938,7 +951,7 @@ int engram_advance_history(const engram_plan *plan, const int32_t *ids_remapped,
     if (!history || (T > 0 && !ids_remapped)) return fail(ENGRAM_ERR_INVALID_ARG, "history and ids must be non-NULL");
     engram::advance_history_kernel<<<(B + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(
         ids_remapped, B, T, history, plan->hist_len);
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "advance_history_kernel launch");
+    ENGRAM_LAUNCHED("advance_history_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -1014,7 +1027,7 @@ int engram_pack_weights(const engram_plan *plan, const uint16_t *w_k, const uint
     engram::pack_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         w_k, w_v, static_cast<int64_t>(plan->num_branches) * plan->cfg.hidden_dim, plan->mem_dim,
         (plan->mem_dim + engram::kBK - 1) / engram::kBK, n_chunks, static_cast<uint4 *>(packed));
-    ENGRAM_CUDA_TRY(cudaGetLastError(), "pack_weights_kernel launch");
+    ENGRAM_LAUNCHED("pack_weights_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -1027,7 +1040,7 @@ int engram_row_cache_reset(const engram_plan *plan, const engram_row_cache *cach
         if (blocks > 148 * 16) blocks = 148 * 16;
         engram::cache_reset_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
             cache->tags[h], cache->claim[h], cache->slots);
-        ENGRAM_CUDA_TRY(cudaGetLastError(), "cache_reset_kernel launch");
+        ENGRAM_LAUNCHED("cache_reset_kernel launch");
     }
     return ENGRAM_OK;
 }
@@ -1184,6 +1197,8 @@ int engram_gate_conv_noalloc(const engram_plan *plan, const engram_weights *w, c
     if (rc != ENGRAM_OK) return rc;
     return launch_gate_conv(plan, w, h, v, part, n_tiles, B, T, conv_state, out, delta_dbg, stream);
 }
+
+uint64_t engram_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }
 
 int engram_device_status(uint32_t *status, int clear) {
     if (!status) return fail(ENGRAM_ERR_INVALID_ARG, "status is NULL");

@@ -342,6 +342,12 @@ const char *engram_last_error(void);
 /* Library version, e.g. "0.1.0". */
 const char *engram_version(void);
 
+/* Number of kernels this library has launched in this process so far (all host threads and
+ * devices; a launch is counted once the CUDA runtime has accepted it, whether it runs eagerly
+ * or is recorded into a CUDA graph being captured).  A diagnostic: read it before and after
+ * a call to learn how many kernels that call launches. */
+uint64_t engram_kernel_launches(void);
+
 /* sizeof() of a public struct, by name ("engram_config", "engram_plan", "engram_weights",
  * "engram_row_cache"),
  * so that bindings in other languages can check their layout; 0 for an unknown name. */

@@ -102,6 +102,7 @@ def test_hash_multipliers_are_odd_and_seeded():
 def test_invalid_calls_fail_on_host_without_launching():
     lib = E.lib
     p = _plan()
+    launches0 = E.kernel_launches()
     # uninitialised plan
     bad = _native.engram_plan()
     assert lib.engram_hash(C.byref(bad), None, 1, 1, None, None, None) == E.ENGRAM_ERR_INVALID_ARG
@@ -122,6 +123,8 @@ def test_invalid_calls_fail_on_host_without_launching():
     assert lib.engram_hash(p, None, 0, 5, None, None, None) == E.ENGRAM_OK
     assert lib.engram_gather(p, None, None, 0, None, None) == E.ENGRAM_OK
     assert lib.engram_remap(p, None, 0, None, None, None) == E.ENGRAM_OK
+    # nothing above reached a kernel launch: the library's own launch count is unchanged
+    assert E.kernel_launches() == launches0
 
 
 def test_workspace_too_small_is_rejected():

@@ -179,6 +179,24 @@ def test_forward_matches_oracle(case):
     assert E.engram_device_status(clear=True) == 0
 
 
+def test_kernel_launch_count_per_call():
+    """The library's launch counter (bench.py's gpu_launches): a prefill call on the two-stage
+    gate path launches remap + hash, gather, projection, gate scalars and the streaming gate
+    kernel; the same call twice counts the same; a call rejected on the host counts nothing."""
+    wl = PARITY_CASES["bn128"]                  # 9,554 tokens x 4 tables: the separate hash and gather
+    di = DeviceInputs(wl).forward()
+    torch.cuda.synchronize()
+    n0 = E.kernel_launches()
+    di.forward()
+    n1 = E.kernel_launches()
+    di.forward()
+    n2 = E.kernel_launches()
+    assert n1 - n0 == 5 and n2 - n1 == 5
+    with pytest.raises(E.EngramError):
+        E.engram_forward(di.plan, di.weights, di.tables, di.ids, di.h, di.out, di.ws[:16])   # workspace too small
+    assert E.kernel_launches() == n2
+
+
 @pytest.mark.parametrize("case", ["ragged_k_bn64", "bn256_unfused", "splitk_64tok", "fused_seq_edges"])
 def test_forward_with_non_unit_gains(case):
     wl = PARITY_CASES[case]

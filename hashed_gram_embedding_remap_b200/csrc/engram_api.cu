@@ -302,14 +302,14 @@ int sm_count() {
     return n;
 }
 
-template <int BN>
+template <int BN, bool SPLIT>
 int set_proj_smem_attr() {
     // Per device: the attribute is a property of the function on the current device.
     static bool done[64] = {};
     int dev = 0;
     ENGRAM_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
     if (dev < 64 && done[dev]) return ENGRAM_OK;
-    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::proj_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::proj_kernel<BN, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          engram::ProjCfg<BN>::kSmemBytes),
                     "cudaFuncSetAttribute(proj_kernel)");
     if (dev < 64) done[dev] = true;
@@ -328,7 +328,8 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     const int M = plan->num_branches;
     if ((rc = make_map_bf16(&map_wk, w->w_k, static_cast<uint64_t>(M) * d_h, d_m, BN)) != ENGRAM_OK) return rc;
     if ((rc = make_map_bf16(&map_wv, w->w_v, d_h, d_m, BN)) != ENGRAM_OK) return rc;
-    if ((rc = set_proj_smem_attr<BN>()) != ENGRAM_OK) return rc;
+    const bool split = acc != nullptr && k_splits > 1;
+    if ((rc = split ? set_proj_smem_attr<BN, true>() : set_proj_smem_attr<BN, false>()) != ENGRAM_OK) return rc;
     engram::ProjParams p{};
     p.h = h;
     p.gamma_q = w->gamma_q;
@@ -350,8 +351,9 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
     const int64_t sms = sm_count();
     dim3 grid(static_cast<unsigned>(total < sms ? total : sms));
-    ENGRAM_CUDA_TRY(launch_pdl(engram::proj_kernel<BN>, grid, dim3(engram::kProjThreads), engram::ProjCfg<BN>::kSmemBytes,
-                               stream, map_m, map_wk, map_wv, p),
+    ENGRAM_CUDA_TRY(launch_pdl(split ? engram::proj_kernel<BN, true> : engram::proj_kernel<BN, false>, grid,
+                               dim3(engram::kProjThreads), engram::ProjCfg<BN>::kSmemBytes, stream, map_m, map_wk,
+                               map_wv, p),
                     "proj_kernel launch");
     if (params_out) *params_out = p;
     if (p.k_splits > 1 && run_reduce) {

@@ -118,7 +118,9 @@ __device__ __forceinline__ float v_hi(uint32_t w) {
 // one time share a few 128-token blocks of m (re-read from L2) and stream all of W.
 // Roles: warp 0 = TMA producer, warp 1 = TMEM owner + MMA issuer, warps 2-5 = epilogue.
 // Two TMEM accumulators: the epilogue drains tile i while the MMAs of tile i+1 run.
-template <int BN>
+// SPLIT: compiled for split-K work units (p.k_splits > 1, raw partial accumulators out) or
+// for whole-K tiles only, so that neither epilogue costs the other registers.
+template <int BN, bool SPLIT>
 __global__ void __launch_bounds__(kProjThreads, 1)
     proj_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ CUtensorMap map_wk,
                 const __grid_constant__ CUtensorMap map_wv, const __grid_constant__ ProjParams p) {
@@ -285,7 +287,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             for (int cc = 0; cc < BN; cc += 32) {
                 float accv[32];
                 tmem_ld32(taddr + cc, accv);
-                if (p.k_splits > 1) {
+                if constexpr (SPLIT) {
                     // split-K: raw partial accumulator; the reduction finishes the tile.  Each
                     // lane holds 32 columns of its own row: the warp's 32 x 32 block goes through
                     // shared memory so that every store instruction writes 4 whole 128-byte
@@ -355,7 +357,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty_bar[acc]);
-            if (valid && p.k_splits == 1) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
+            if constexpr (!SPLIT) {
+                if (valid) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
+            }
         }
     }
     tc_fence_before();

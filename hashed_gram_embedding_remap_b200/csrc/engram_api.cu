@@ -740,9 +740,13 @@ cudaError_t record_stage_event(void *ev, cudaStream_t stream) {
     return cudaEventRecord(static_cast<cudaEvent_t>(ev), stream);
 }
 
+// history / xr (engram_forward's decode steps): when the step ends in decode_fused_kernel, that
+// kernel also advances the hash history and *history_done is set; otherwise the caller does.
 int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                    int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out, float *delta, uint8_t *ws,
-                   cudaStream_t stream, void *const *events) {
+                   cudaStream_t stream, void *const *events, int32_t *history = nullptr,
+                   const int32_t *xr = nullptr, bool *history_done = nullptr) {
+    if (history_done) *history_done = false;
     const int64_t n_tok = static_cast<int64_t>(B) * T;
     const Workspace L = layout(plan, n_tok);
     if (use_fused_gate(plan, n_tok, conv_state != nullptr)) {
@@ -770,7 +774,12 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
     if (rc != ENGRAM_OK) return rc;
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[1], stream), "cudaEventRecord");
     if (fused_decode) {
-        const engram::GateParams gp = make_gate_params(plan, w, h, v, part, ps.n_tiles, B, T, conv_state, out, delta);
+        engram::GateParams gp = make_gate_params(plan, w, h, v, part, ps.n_tiles, B, T, conv_state, out, delta);
+        if (history != nullptr && xr != nullptr && plan->hist_len > 0) {
+            gp.history = history;
+            gp.xr = xr;
+            gp.hist_len = plan->hist_len;
+        }
         using DK = void (*)(const engram::ProjParams, const engram::GateParams);
         static const DK kernels[engram::kFusedDecodeMaxPairs] = {
             engram::decode_fused_kernel<1>, engram::decode_fused_kernel<2>, engram::decode_fused_kernel<3>,
@@ -781,6 +790,7 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
                                    0, stream, pp, gp),
                         "decode_fused_kernel launch");
         ENGRAM_CUDA_TRY(cudaGetLastError(), "decode_fused_kernel launch");
+        if (history_done) *history_done = gp.history != nullptr;
         return ENGRAM_OK;
     }
     return launch_gate_conv(plan, w, h, v, part, ps.n_tiles, B, T, conv_state, out, delta, stream,
@@ -1153,11 +1163,12 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const void 
     } else if ((rc = launch_gather(plan, idx, tables, n_tok, m, stream)) != ENGRAM_OK) {
         return rc;
     }
+    bool history_done = false;
     if ((rc = gate_conv_impl(plan, w, h, m, B, T, conv_state, out, delta_dbg, ws, stream,
-                             stage_events ? stage_events + 2 : nullptr)) != ENGRAM_OK)
+                             stage_events ? stage_events + 2 : nullptr, history, xr, &history_done)) != ENGRAM_OK)
         return rc;
     if ((rc = rec(4)) != ENGRAM_OK) return rc;
-    if (history != nullptr && plan->hist_len > 0) {
+    if (history != nullptr && plan->hist_len > 0 && !history_done) {
         ENGRAM_CUDA_TRY(launch_pdl(engram::advance_history_kernel, dim3((B + 127) / 128), dim3(128), 0, stream,
                                    static_cast<const int32_t *>(xr), B, T, history, static_cast<int32_t>(plan->hist_len)),
                         "advance_history_kernel launch");

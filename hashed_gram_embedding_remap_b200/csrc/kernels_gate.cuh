@@ -36,6 +36,9 @@ struct GateParams {
     float eps;
     float inv_sqrt_d;
     const float2 *scal;       // [n_tok] (g, beta) from gate_scalars_kernel, or null
+    int32_t *history;         // decode_fused_kernel: [B, hist_len] hash history to advance, or null
+    const int32_t *xr;        // with history: [B] remapped ids of this step
+    int32_t hist_len;
 };
 
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + __expf(-z)); }
@@ -664,6 +667,13 @@ __global__ void __launch_bounds__(kFusedDecodeThreads, 2) decode_fused_kernel(co
         }
     }
     pdl_wait();   // the split accumulators come from the projection kernel before this one
+    if (p.history != nullptr && threadIdx.x == 0) {
+        // the step's hash history update (T = 1): drop the oldest id, append this step's.
+        // The lookup that read the history finished before the projection did.
+        int32_t *hb = p.history + static_cast<int64_t>(b) * p.hist_len;
+        for (int s = 0; s + 1 < p.hist_len; ++s) hb[s] = hb[s + 1];
+        hb[p.hist_len - 1] = p.xr[b];
+    }
     for (int ks = 0; ks < pp.k_splits; ++ks) {
         const float *src = acc + ks * split_stride;
 #pragma unroll

@@ -293,8 +293,8 @@ int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
  * when `history` is given.  Kernels per call: prefill batches launch remap + hash, gather,
  * projection, gate scalars and the streaming gate + conv kernel (5); batches of at most
  * 16,384 (token, table) rows on HBM-resident tables fuse remap + hash + gather into one
- * kernel; one-token decode steps whose projection splits K finish the split sums, gate and
- * conv in one kernel (lookup, projection, fused gate, history update: 4).
+ * kernel; one-token decode steps whose projection splits K finish the split sums, gate,
+ * conv and the history update in one kernel (lookup, projection, that kernel: 3).
  * engram_kernel_launches() counts them.
  * ids: int32 [B, T] raw token ids.  remap: int32 [vocab_in], or NULL when ids are already
  * in the compressed vocabulary.  history / conv_state: NULL for prefill, or the decode state

@@ -2,10 +2,11 @@
 """Throughput of the hashed n-gram embedding lookup on B200 (one JSON line on rank 0).
 
 A step is one pass of the whole path -- remap + hash, gather, projections, gate + conv +
-residual -- over one batch of the workload (default: the Engram layer at hidden 2560,
-8 x 4096 tokens, 16 tables of 999,983 rows x 160).  Inputs are resident in HBM when the
-timed region starts; the e2e figure repeats the measurement through the same public call
-with the inputs copied from pinned host memory and the output copied back every step.
+residual -- over one batch of the workload (default: prefill on the 20M-row tables,
+32 x 8192 tokens, 2 tables of 9,999,991 rows x 2560 bf16 = 95.4 GiB in HBM).  Inputs are
+resident in HBM when the timed region starts; the e2e figure repeats the measurement
+through the same public call with the inputs copied from pinned host memory and the output
+copied back every step.
 
 Multi-GPU (torchrun): every rank runs its own replica on its own batch (the lookup has no
 cross-token exchange), so scaling is weak; time is the max over ranks.
@@ -300,7 +301,10 @@ def run_reference(args, wl, world, rank):
     line = {
         "impl": "reference", "metric": "engram_tokens_per_s", "value": tps, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": wl.n_tok / tps * 1e3,
+        # a step of this arm is one measured round of samples (procs x T tokens), not the
+        # workload's whole batch; the time one whole batch would take is extrapolated apart
+        "ms_per_step": 1e3 * sum(times) / args.steps, "tokens_per_step": procs * T,
+        "ms_per_workload_batch_extrapolated": wl.n_tok / tps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(wl, world),
         "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": procs, "kind": "oracle", "sample": sample},
@@ -309,14 +313,18 @@ def run_reference(args, wl, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(wl, world):
-    return {"workload": wl.name, "tokens_per_step_per_gpu": wl.n_tok, "B": wl.B, "T": wl.T,
-            "orders": list(wl.orders), "K": wl.K, "H": wl.H, "table_rows": wl.primes[0], "d_e": wl.d_e,
-            "d_m": wl.d_m, "d_h": wl.d_h, "branches": wl.branches, "table_dtype": wl.table_dtype,
-            "table_GiB": round(wl.table_bytes / 2 ** 30, 2),
-            "parallelism": f"replicas x{world}",
-            "l2": "inputs larger than L2 (hidden states, memory vectors and tables each exceed 126 MB)"
-            if l2_exceeded(wl) else "L2 flushed between timed steps (252 MiB write, outside the per-step events)"}
+def workload_config(wl, world, ids_kind=None):
+    """The workload's description, identical in both arms' lines."""
+    c = {"workload": wl.name, "tokens_per_step_per_gpu": wl.n_tok, "B": wl.B, "T": wl.T,
+         "orders": list(wl.orders), "K": wl.K, "H": wl.H, "table_rows": wl.primes[0], "d_e": wl.d_e,
+         "d_m": wl.d_m, "d_h": wl.d_h, "branches": wl.branches, "table_dtype": wl.table_dtype,
+         "table_GiB": round(wl.table_bytes / 2 ** 30, 2),
+         "parallelism": f"replicas x{world}",
+         "l2": "inputs larger than L2 (hidden states and tables each exceed 126 MB)"
+         if l2_exceeded(wl) else "L2 flushed between timed steps (252 MiB write, outside the per-step events)"}
+    if wl.host_tables:
+        c.update(tables="pinned mapped host memory", ids=ids_kind or wl.ids_kind)
+    return c
 
 
 def l2_exceeded(wl) -> bool:
@@ -352,12 +360,25 @@ def run_engram(args, wl, world, rank, local):
     cw = fill_gpu.filled((wl.d_h, wl.conv_kernel), wl.conv_spec(), dev)
     history = torch.from_numpy(wl.history()).to(dev) if wl.decode else None
     state = fill_gpu.filled((wl.B * M, wl.state_len, wl.d_h), wl.state_spec(), dev) if wl.decode else None
-    plan = E.Plan.from_workload(wl)
+    plan = E.Plan.from_workload(wl, flags=(E.ENGRAM_FLAG_SEPARATE_GATHER if args.separate_gather else 0)
+                                | (E.ENGRAM_FLAG_SINGLE_CTA_MMA if args.single_cta_mma else 0))
+    path = E.engram_forward_path(plan, wl.B, wl.T)
+    gather_in_proj = bool(path & E.ENGRAM_PATH_GATHER_IN_PROJ)
     packed = E.pack_weights(plan, wk, wv) if args.packed and E.engram_packed_weights_size(plan) else None
     weights = E.Weights(wk, wv, one, one, one, cw, packed=packed)
     out = torch.empty((wl.h_rows, wl.d_h), dtype=torch.bfloat16, device=dev)
     ws = E.alloc_workspace(plan, wl.n_tok, dev)
     nstage = E.ENGRAM_FORWARD_STAGES + 1
+
+    # Row ids of the batch (the library's own remap + hash, untimed): distinct rows per
+    # table for the byte count of the HBM roofline
+    xr = ids
+    if remap is not None:
+        xr = torch.empty_like(ids)
+        E.engram_remap(plan, ids, remap, xr)
+    idx = torch.empty((wl.n_tok, wl.H), dtype=torch.int32, device=dev)
+    E.engram_hash(plan, xr, idx, history=history)
+    distinct_rows = sum(int(torch.unique(idx[:, t]).numel()) for t in range(wl.H))
 
     def step(evs=None):
         E.engram_forward(plan, weights, tables, ids, h, out, ws, remap=remap, history=history,
@@ -446,9 +467,27 @@ def run_engram(args, wl, world, rank, local):
     stage_names = ["hash", "gather", "proj", "gate_conv"]
     stage_ms = {n: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
                 for i, n in enumerate(stage_names)}
+    if gather_in_proj:   # the projection reads the rows itself: there is no gather stage
+        del stage_ms["gather"]
     status = E.engram_device_status(clear=True)
     if status:
         raise SystemExit(f"device status {status:#x} after the timed region")
+
+    # The separate gather kernel on the same row ids (what the path costs when m is
+    # materialised), timed alone for the HBM accounting below; not part of a step here.
+    sep_gather_ms = None
+    if gather_in_proj and not args.no_separate_gather_timing:
+        m_buf = torch.empty((wl.n_tok, wl.d_m), dtype=torch.bfloat16, device=dev)
+        E.engram_gather(plan, idx, tables, m_buf, stream=stream)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        g0.record(stream)
+        for _ in range(reps):
+            E.engram_gather(plan, idx, tables, m_buf, stream=stream)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        sep_gather_ms = g0.elapsed_time(g1) / reps
+        del m_buf
 
     # ---- e2e: inputs from pinned host memory, result back to pinned host memory.
     # Every step copies its ids and hidden states host->device and its output device->host.
@@ -549,31 +588,67 @@ def run_engram(args, wl, world, rank, local):
     flops = 2.0 * n_tok * wl.d_m * (M + 1) * wl.d_h     # M key projections + the value projection
     proj_s = stage_ms["proj"] / 1e3
     tflops = flops / proj_s / 1e12
-    roofline = {"bound": "tensor", "kernel": "proj_kernel (tcgen05 k/v projections + gate partials)",
-                "achieved": tflops, "peak": peaks["bf16_sus"], "unit": "TFLOP/s", "frac": tflops / peaks["bf16_sus"],
-                "traffic": kernel_traffic("proj_kernel", wl.name), "peak_source": f"{peaks['source']} bf16 sustained",
+    # A timed region of at most a second is a burst for the tensor pipe (clocks have not yet
+    # settled under the power cap): the denominator is the measured burst bf16 rate; longer
+    # regions use the sustained one.
+    timed_s = elapsed_ms / 1e3
+    burst = timed_s <= 1.0
+    peak_tf = peaks["bf16"] if burst else peaks["bf16_sus"]
+    pair = bool(path & E.ENGRAM_PATH_PAIR_MMA)
+    roofline = {"bound": "tensor",
+                "kernel": ("proj_pair_kernel (cta_group::2 " if pair else "proj_kernel (")
+                          + "tcgen05 k/v projections + gate partials"
+                          + (", rows gathered into its A tiles)" if gather_in_proj else ")"),
+                "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s", "frac": tflops / peak_tf,
+                "frac_of_sustained": tflops / peaks["bf16_sus"],
+                "traffic": kernel_traffic("proj_kernel", wl.name),
+                "peak_source": f"{peaks['source']} bf16 {'burst' if burst else 'sustained'} "
+                               f"(timed region {timed_s:.2f} s)",
                 "algorithmic_per_launch": flops}
-    # HBM view of the memory-bound kernels (gather and gate+conv)
-    row_bytes = wl.H * wl.d_e * wl.table_elem_bytes
-    gather_bytes = n_tok * (row_bytes + wl.H * wl.d_e * 2 + wl.H * 4)   # rows read + m written + row ids
-    gate_bytes = n_tok * (wl.d_h * 2 + M * (wl.d_h * 2 * 2 + 8))   # v (fp16) once; h read, out written, scalars per branch
-    hbm = {"gather_GBps": gather_bytes / (stage_ms["gather"] / 1e3) / 1e9,
-           "gate_conv_GBps": gate_bytes / (stage_ms["gate_conv"] / 1e3) / 1e9,
-           "peak_GBps": peaks["hbm"], "nominal_GBps": 8000.0}
-    hbm["gather_frac"] = hbm["gather_GBps"] / peaks["hbm"]
+    # HBM view of the memory-bound part of the path.  Algorithmic bytes per step (the
+    # method's own, no intermediates): each distinct table row once, hidden states read,
+    # outputs written, token ids read; beside them the same with every token's rows.
+    row_b = wl.d_e * wl.table_elem_bytes
+    hout = n_tok * M * wl.d_h * 2 * 2
+    alg_distinct = distinct_rows * row_b + hout + n_tok * 4
+    alg_tokrows = n_tok * wl.H * row_b + hout + n_tok * 4
+    gate_bytes = n_tok * (wl.d_h * 2 + M * (wl.d_h * 2 * 2 + 8))   # v (fp16) once; h read, out written, scalars
+    hbm = {"peak_GBps": peaks["hbm"], "nominal_GBps": 8000.0,
+           "distinct_rows_per_step": distinct_rows, "token_rows_per_step": n_tok * wl.H,
+           "algorithmic_bytes_distinct_rows": alg_distinct, "algorithmic_bytes_token_rows": alg_tokrows,
+           "gate_conv_GBps": gate_bytes / (stage_ms["gate_conv"] / 1e3) / 1e9}
     hbm["gate_conv_frac"] = hbm["gate_conv_GBps"] / peaks["hbm"]
-    # the memory-bound part of the path taken together: gather + gate + conv
-    both_s = (stage_ms["gather"] + stage_ms["gate_conv"]) / 1e3
-    hbm["gather_gate_conv_GBps"] = (gather_bytes + gate_bytes) / both_s / 1e9
-    hbm["gather_gate_conv_frac"] = hbm["gather_gate_conv_GBps"] / peaks["hbm"]
-    hbm["gather_gate_conv_frac_nominal"] = hbm["gather_gate_conv_GBps"] / hbm["nominal_GBps"]
+    path_ms = stage_ms["hash"] + stage_ms.get("gather", 0.0) + stage_ms["gate_conv"]
+    hbm["path_ms"] = path_ms
+    hbm["path_frac"] = alg_distinct / (path_ms / 1e3) / 1e9 / peaks["hbm"]
+    hbm["path_frac_token_rows"] = alg_tokrows / (path_ms / 1e3) / 1e9 / peaks["hbm"]
+    hbm["path_frac_nominal"] = alg_distinct / (path_ms / 1e3) / 1e9 / hbm["nominal_GBps"]
+    if gather_in_proj:
+        hbm["path_note"] = ("path_ms = hash + gate_conv: the rows are read by the projection kernel's "
+                            "gather warps, overlapped with its tensor-core work, so no stage of its own "
+                            "remains for them")
+        if sep_gather_ms is not None:
+            # the same bytes over the stages with the separate gather kernel in the path
+            sep_ms = path_ms + sep_gather_ms
+            hbm["separate_gather_ms"] = sep_gather_ms
+            hbm["path_frac_with_separate_gather"] = alg_distinct / (sep_ms / 1e3) / 1e9 / peaks["hbm"]
+    else:
+        gather_bytes = n_tok * (wl.H * row_b + wl.d_m * 2 + wl.H * 4)   # rows read + m written + row ids
+        hbm["gather_GBps"] = gather_bytes / (stage_ms["gather"] / 1e3) / 1e9
+        hbm["gather_frac"] = hbm["gather_GBps"] / peaks["hbm"]
+    # bytes the path's own kernels move, intermediates included (m written and read back
+    # when materialised, v written by the projection and read by the gate kernel)
+    moved = gate_bytes + (0 if gather_in_proj else n_tok * (wl.H * row_b + wl.d_m * 2 + wl.H * 4))
+    hbm["incl_intermediates_GBps"] = moved / (path_ms / 1e3) / 1e9
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        T1, dt1, _ = oracle_sample(wl, args.cpu_baseline_tokens // 4)    # one core, for the record
+        # tokens per worker scaled to the per-token work (about 20 s of CPU time per worker)
+        cpu_tok = max(32, int(args.cpu_baseline_tokens * (2 * 2560 * 2560) / (wl.d_m * wl.d_h * (M + 1))))
+        T1, dt1, _ = oracle_sample(wl, max(8, cpu_tok // 4))    # one core, for the record
         procs = oracle_procs(args, wl)
         pool = OraclePool(procs, wl)
-        toks, dt = pool.round(wl, args.cpu_baseline_tokens)
+        toks, dt = pool.round(wl, cpu_tok)
         pool.close()
         cpu = {"value": toks / dt, "unit": "tokens/s", "cores": procs, "kind": "oracle",
                "sample": f"{procs} samples of 1 sequence x {toks // procs} tokens of {wl.name}, one per process, "
@@ -586,7 +661,10 @@ def run_engram(args, wl, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Zipf ids, counter-based bf16 tables/weights)",
-        "config": dict(workload_config(wl, world), weights="packed" if packed is not None else "row-major"),
+        "config": workload_config(wl, world),
+        "weights_layout": "packed" if packed is not None else "row-major",
+        "path": {"gather_in_projection": gather_in_proj, "pair_mma": bool(path & E.ENGRAM_PATH_PAIR_MMA),
+                 "path_bits": path},
         "stages_ms": stage_ms, "hbm": hbm, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * launches_per_step,
         "launch_mode": "eager" if args.eager else "one CUDA graph of the K timed steps (stage times from a "
@@ -809,8 +887,7 @@ def run_hostpinned(args, wl, world, rank, local):
         "metric": "engram_tokens_per_s", "value": B / (ovl_ms / 1e3), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": ovl_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": f"synthetic; ids {kind}",
-        "config": dict(workload_config(wl, world), tables="pinned mapped host memory",
-                       host_tables_GB=round(wl.table_bytes / 1e9, 1), ids=kind),
+        "config": workload_config(wl, world, ids_kind=kind),
         "step_includes": "hash + distinct-row staging from host (side stream) || 2560^3 bf16 GEMM stand-in; "
                          "then gather + projections + gate/conv + history update",
         "host_link": {"bound": "host-link", "staged_rows_per_step": int(nu_h.sum()),
@@ -833,10 +910,16 @@ def run_hostpinned(args, wl, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["engram", "reference"], default="engram")
-    ap.add_argument("--workload", default="layer2560", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="prefill20m", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--separate-gather", action="store_true",
+                    help="materialise m with the separate gather kernel (ENGRAM_FLAG_SEPARATE_GATHER)")
+    ap.add_argument("--single-cta-mma", action="store_true",
+                    help="never pair CTAs for the projection's MMAs (ENGRAM_FLAG_SINGLE_CTA_MMA)")
+    ap.add_argument("--no-separate-gather-timing", action="store_true",
+                    help="skip timing the separate gather kernel beside the row-gathering projection")
     ap.add_argument("--oracle-tokens", type=int, default=128)
     ap.add_argument("--cpu-baseline-tokens", type=int, default=768)
     ap.add_argument("--oracle-procs", type=int, default=0,
@@ -864,6 +947,8 @@ def main():
         p = synth.largest_prime_below(args.table_rows + 1) if synth.workloads.is_prime(args.table_rows) is False \
             else args.table_rows
         wl = wl.with_(primes=(p,) * wl.H, name=f"{wl.name}[rows={p}]")
+    if args.ids:
+        wl = wl.with_(ids_kind=args.ids)
     if args.table_dtype == "fp8":
         wl = wl.with_(table_dtype="fp8", name=f"{wl.name}-fp8")
     if args.batch:

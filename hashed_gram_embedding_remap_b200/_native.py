@@ -19,7 +19,6 @@ ENGRAM_OK = 0
 ENGRAM_ERR_INVALID_ARG = -1
 ENGRAM_ERR_UNSUPPORTED = -2
 ENGRAM_ERR_CUDA = -3
-ENGRAM_ERR_OOM = -4
 ENGRAM_ERR_TIMEOUT = -5
 ENGRAM_STATUS_BAD_TOKEN = 0x1
 ENGRAM_STATUS_BAD_ROW = 0x2
@@ -31,12 +30,18 @@ ENGRAM_FORWARD_STAGES = 4
 ENGRAM_TABLES_DEVICE = 0
 ENGRAM_TABLES_HOST_MAPPED = 1
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
-ENGRAM_FLAG_FUSED_GATE = 0x1
+ENGRAM_FLAG_SEPARATE_GATHER = 0x2
+ENGRAM_FLAG_SINGLE_CTA_MMA = 0x4
+ENGRAM_PATH_FUSED_LOOKUP = 0x1
+ENGRAM_PATH_STAGED_ROWS = 0x2
+ENGRAM_PATH_GATHER_IN_PROJ = 0x4
+ENGRAM_PATH_SPLIT_K = 0x8
+ENGRAM_PATH_PAIR_MMA = 0x10
 ENGRAM_TABLE_BF16 = 0
 ENGRAM_TABLE_FP8_E4M3 = 1
 
 _ERRNAMES = {-1: "ENGRAM_ERR_INVALID_ARG", -2: "ENGRAM_ERR_UNSUPPORTED", -3: "ENGRAM_ERR_CUDA",
-             -4: "ENGRAM_ERR_OOM", -5: "ENGRAM_ERR_TIMEOUT"}
+             -5: "ENGRAM_ERR_TIMEOUT"}
 
 
 class EngramError(RuntimeError):
@@ -119,6 +124,9 @@ def _load():
         "engram_forward": (C.c_int, [P, P, P, P, P, i32, i32, P, P, P, P, P, P, sz, P, P]),
         "engram_gate_conv_noalloc": (C.c_int, [P, P, P, P, i32, i32, P, P, P, P]),
         "engram_device_status": (C.c_int, [P, C.c_int]),
+        "engram_forward_path": (C.c_int, [P, i32, i32, P]),
+        "engram_synchronize": (C.c_int, [P]),
+        "engram_selftest_wait_timeout": (C.c_int, [P, P, P, P, i64, P, sz, C.c_uint64, P]),
         "engram_last_error": (C.c_char_p, []),
         "engram_version": (C.c_char_p, []),
         "engram_sizeof": (sz, [C.c_char_p]),
@@ -443,6 +451,29 @@ def engram_device_status(clear: bool = True) -> int:
     s = C.c_uint32(0)
     _check(lib.engram_device_status(C.byref(s), int(clear)))
     return int(s.value)
+
+
+def engram_forward_path(plan: Plan, B: int, T: int) -> int:
+    """ENGRAM_PATH_* bits: which kernels engram_forward runs for B sequences of T tokens."""
+    bits = C.c_uint32(0)
+    _check(lib.engram_forward_path(plan, int(B), int(T), C.byref(bits)))
+    return int(bits.value)
+
+
+def engram_synchronize(stream=None):
+    """Wait for the stream; raises EngramError(ENGRAM_ERR_TIMEOUT) if a bounded wait inside a
+    kernel gave up since the device status word was last cleared."""
+    _check(lib.engram_synchronize(_stream(stream)))
+
+
+def engram_selftest_wait_timeout(plan: Plan, weights: Weights, h: torch.Tensor, m: torch.Tensor,
+                                 workspace: torch.Tensor, wait_limit_ns: int, stream=None):
+    """Run the projection with its loads stalled so that every bounded wait runs out after
+    wait_limit_ns (the failure path of engram_selftest_wait_timeout)."""
+    _check(lib.engram_selftest_wait_timeout(plan, weights, _ptr(h, _BF16, "h"), _ptr(m, _BF16, "m"), m.shape[0],
+                                            _ptr(workspace, None, "workspace"),
+                                            workspace.numel() * workspace.element_size(), int(wait_limit_ns),
+                                            _stream(stream)))
 
 
 def alloc_workspace(plan: Plan, n_tok: int, device="cuda") -> torch.Tensor:

@@ -16,8 +16,8 @@
 
 #include "engram.h"
 #include "kernels_gate.cuh"
-#include "kernels_fused.cuh"
 #include "kernels_lookup.cuh"
+#include "kernels_proj_pair.cuh"
 #include "ptx.cuh"
 
 namespace {
@@ -215,18 +215,36 @@ ProjShape proj_shape(const engram_plan *plan, int64_t n_tok, bool allow_split) {
     return ps;
 }
 
-// With ENGRAM_FLAG_FUSED_GATE, prefill with the pages' conv shape runs projections, gate
-// and conv in one kernel (fused_proj_gate_kernel).
-bool use_fused_gate(const engram_plan *plan, int64_t n_tok, bool has_state) {
-    if (!(plan->cfg.flags & ENGRAM_FLAG_FUSED_GATE) || has_state || n_tok <= 0) return false;
-    if (plan->cfg.conv_kernel != 4 || plan->cfg.conv_dilation != 3) return false;
-    return plan->cfg.hidden_dim % 256 == 0;
+// The projection of whole-K tiles runs on CTA pairs (proj_pair_kernel, 256 x 256 units) when
+// d_h is a multiple of 256 and there are at least two units per pair of SMs.
+bool use_pair_mma(const engram_plan *plan, int64_t n_tok, const ProjShape &ps) {
+    if (ps.k_splits != 1 || plan->cfg.hidden_dim % engram::kPairBN != 0) return false;
+    if (plan->cfg.flags & ENGRAM_FLAG_SINGLE_CTA_MMA) return false;
+    const int64_t units = (n_tok + engram::kPairRows - 1) / engram::kPairRows *
+                          ((plan->num_branches + 1) * plan->cfg.hidden_dim / engram::kPairBN);
+    return units >= 148;
 }
 
-size_t fused_vbuf_bytes(const engram_plan *plan, int64_t n_tok) {
-    const int64_t units = (n_tok + engram::kFusedRows - 1) / engram::kFusedRows;
-    const int64_t ctas = units < 148 ? units : 148;
-    return sizeof(float) * static_cast<size_t>(ctas) * 2 * engram::kBM * plan->cfg.hidden_dim;
+// Which kernels engram_forward runs for a batch of n_tok tokens (engram_forward_path).
+struct ForwardPath {
+    bool fused_lookup;    // remap + hash + gather in one kernel (decode-sized, HBM tables)
+    bool staged;          // host-mapped tables: the batch's distinct rows are staged into HBM
+    bool gather_in_proj;  // the projection gathers the rows into its A tiles (m never written)
+    bool pair;            // the projection's MMAs span CTA pairs
+    ProjShape ps;
+};
+
+ForwardPath forward_path(const engram_plan *plan, int64_t n_tok) {
+    ForwardPath f{};
+    f.ps = proj_shape(plan, n_tok, true);
+    f.staged = plan->cfg.table_location == ENGRAM_TABLES_HOST_MAPPED && n_tok <= engram::kStageMaxTok;
+    f.fused_lookup = !f.staged && plan->cfg.table_location == ENGRAM_TABLES_DEVICE &&
+                     n_tok * plan->num_tables <= kFusedLookupMaxRows;
+    f.gather_in_proj = !f.fused_lookup && !f.staged && plan->cfg.table_location == ENGRAM_TABLES_DEVICE &&
+                       plan->cfg.table_dtype == ENGRAM_TABLE_BF16 && f.ps.k_splits == 1 &&
+                       !(plan->cfg.flags & ENGRAM_FLAG_SEPARATE_GATHER);
+    f.pair = use_pair_mma(plan, n_tok, f.ps);
+    return f;
 }
 
 Workspace layout(const engram_plan *plan, int64_t n_tok) {
@@ -238,18 +256,15 @@ Workspace layout(const engram_plan *plan, int64_t n_tok) {
     size_t off = 0;
     w.xr = off;   off = align256(off + sizeof(int32_t) * n_tok);
     w.idx = off;  off = align256(off + sizeof(uint32_t) * n_tok * H);
-    w.m = off;    off = align256(off + sizeof(uint16_t) * n_tok * plan->mem_dim);
-    size_t v_bytes = sizeof(uint16_t) * n_tok * d_h;
-    if (use_fused_gate(plan, n_tok, false)) {
-        const size_t fb = fused_vbuf_bytes(plan, n_tok);   // the fused kernel's v scratch reuses this region
-        if (fb > v_bytes) v_bytes = fb;
-    }
+    w.m = off;    // m is only materialised when the projection does not gather the rows itself
+    if (!forward_path(plan, n_tok).gather_in_proj) off = align256(off + sizeof(uint16_t) * n_tok * plan->mem_dim);
+    const size_t v_bytes = sizeof(uint16_t) * n_tok * d_h;
     w.v = off;    off = align256(off + v_bytes);
     w.part = off; off = align256(off + sizeof(float4) * n_tok * n_tiles);
     w.acc = off;
     if (ps.k_splits > 1) off = align256(off + sizeof(float) * ps.k_splits * n_tok * ps.n_tiles * ps.bn);
     w.scal = off; off = align256(off + sizeof(float2) * n_tok * plan->num_branches);
-    w.staged = plan->cfg.table_location == ENGRAM_TABLES_HOST_MAPPED && n_tok <= engram::kStageMaxTok;
+    w.staged = forward_path(plan, n_tok).staged;
     if (w.staged) {
         w.staged_idx = off; off = align256(off + sizeof(uint32_t) * n_tok * H);
         w.unique = off;     off = align256(off + sizeof(uint32_t) * n_tok * H);
@@ -302,34 +317,55 @@ int sm_count() {
     return n;
 }
 
-template <int BN, bool SPLIT>
+template <int BN, bool SPLIT, bool GATHER>
 int set_proj_smem_attr() {
     // Per device: the attribute is a property of the function on the current device.
     static bool done[64] = {};
     int dev = 0;
     ENGRAM_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
     if (dev < 64 && done[dev]) return ENGRAM_OK;
-    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::proj_kernel<BN, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::proj_kernel<BN, SPLIT, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          engram::ProjCfg<BN>::kSmemBytes),
                     "cudaFuncSetAttribute(proj_kernel)");
     if (dev < 64) done[dev] = true;
     return ENGRAM_OK;
 }
 
+// Where the projection's A tiles come from when m is not materialised: the row ids of step 2
+// and the (bf16, HBM-resident) tables.
+struct GatherSrc {
+    const uint32_t *idx;          // [n_tok, H]
+    const void *const *tables;    // host array of H device pointers
+};
+
+// Test hooks of the projection: a shorter bound on every pipeline wait, and a stalled
+// pipeline (no loads issued) that makes the first wait run out.
+struct ProjTest {
+    uint64_t wait_limit_ns = 0;
+    int stall = 0;
+};
+
 template <int BN>
 int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                 int64_t n_tok, uint16_t *v, float4 *part, cudaStream_t stream, float *acc = nullptr,
                 int k_splits = 1, int kb_per_split = 0, bool run_reduce = true,
-                engram::ProjParams *params_out = nullptr) {
+                engram::ProjParams *params_out = nullptr, const GatherSrc *gs = nullptr,
+                const ProjTest &test = ProjTest()) {
     const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim;
     CUtensorMap map_m, map_wk, map_wv;
     int rc;
-    if ((rc = make_map_bf16(&map_m, m, static_cast<uint64_t>(n_tok), d_m, engram::kBM)) != ENGRAM_OK) return rc;
     const int M = plan->num_branches;
     if ((rc = make_map_bf16(&map_wk, w->w_k, static_cast<uint64_t>(M) * d_h, d_m, BN)) != ENGRAM_OK) return rc;
     if ((rc = make_map_bf16(&map_wv, w->w_v, d_h, d_m, BN)) != ENGRAM_OK) return rc;
+    if (gs != nullptr)
+        map_m = map_wk;   // unused: the A tiles are gathered from the tables
+    else if ((rc = make_map_bf16(&map_m, m, static_cast<uint64_t>(n_tok), d_m, engram::kBM)) != ENGRAM_OK)
+        return rc;
     const bool split = acc != nullptr && k_splits > 1;
-    if ((rc = split ? set_proj_smem_attr<BN, true>() : set_proj_smem_attr<BN, false>()) != ENGRAM_OK) return rc;
+    if (split && gs != nullptr) return fail(ENGRAM_ERR_UNSUPPORTED, "row gather with a split-K projection");
+    if ((rc = split ? set_proj_smem_attr<BN, true, false>()
+                    : gs ? set_proj_smem_attr<BN, false, true>() : set_proj_smem_attr<BN, false, false>()) != ENGRAM_OK)
+        return rc;
     engram::ProjParams p{};
     p.h = h;
     p.gamma_q = w->gamma_q;
@@ -347,12 +383,25 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     p.kb_per_split = p.k_splits > 1 ? kb_per_split : p.k_blocks;
     p.acc_out = p.k_splits > 1 ? acc : nullptr;
     p.w_packed = BN == 256 ? static_cast<const uint8_t *>(w->w_packed) : nullptr;
+    if (gs != nullptr) {
+        p.idx = gs->idx;
+        p.H = plan->num_tables;
+        p.d_e = plan->cfg.row_dim;
+        for (int t = 0; t < p.H; ++t) {
+            p.tab[t] = static_cast<const uint16_t *>(gs->tables[t]);
+            p.tab_rows[t] = static_cast<uint32_t>(plan->cfg.table_rows[t]);
+        }
+    }
+    p.wait_limit_ns = test.wait_limit_ns;
+    p.stall = test.stall;
     const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles * p.k_splits;
     if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
     const int64_t sms = sm_count();
     dim3 grid(static_cast<unsigned>(total < sms ? total : sms));
-    ENGRAM_CUDA_TRY(launch_pdl(split ? engram::proj_kernel<BN, true> : engram::proj_kernel<BN, false>, grid,
-                               dim3(engram::kProjThreads), engram::ProjCfg<BN>::kSmemBytes, stream, map_m, map_wk,
+    auto kernel = split ? engram::proj_kernel<BN, true, false>
+                        : gs ? engram::proj_kernel<BN, false, true> : engram::proj_kernel<BN, false, false>;
+    const int threads = engram::kProjThreads + (gs ? engram::kGatherThreads : 0);
+    ENGRAM_CUDA_TRY(launch_pdl(kernel, grid, dim3(threads), engram::ProjCfg<BN>::kSmemBytes, stream, map_m, map_wk,
                                map_wv, p),
                     "proj_kernel launch");
     if (params_out) *params_out = p;
@@ -361,6 +410,101 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
                                        stream>>>(p, BN);
         ENGRAM_LAUNCHED("splitk_reduce_kernel launch");
     }
+    return ENGRAM_OK;
+}
+
+template <bool GATHER>
+int set_pair_smem_attr() {
+    static bool done[64] = {};
+    int dev = 0;
+    ENGRAM_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev < 64 && done[dev]) return ENGRAM_OK;
+    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::proj_pair_kernel<GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         engram::PairCfg::kSmemBytes),
+                    "cudaFuncSetAttribute(proj_pair_kernel)");
+    if (dev < 64) done[dev] = true;
+    return ENGRAM_OK;
+}
+
+// CTA pairs that can be resident at once (one CTA per SM; a pair needs two SMs of one GPC).
+template <bool GATHER>
+int max_pairs(int *out) {
+    static int cached[64] = {};
+    int dev = 0;
+    ENGRAM_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev < 64 && cached[dev]) {
+        *out = cached[dev];
+        return ENGRAM_OK;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 74);
+    cfg.blockDim = dim3(engram::kProjThreads + (GATHER ? engram::kGatherThreads : 0));
+    cfg.dynamicSmemBytes = engram::PairCfg::kSmemBytes;
+    int n = 0;
+    ENGRAM_CUDA_TRY(cudaOccupancyMaxActiveClusters(&n, engram::proj_pair_kernel<GATHER>, &cfg),
+                    "cudaOccupancyMaxActiveClusters(proj_pair_kernel)");
+    if (n < 1) return fail(ENGRAM_ERR_CUDA, "no CTA pair of the projection fits on this device");
+    if (dev < 64) cached[dev] = n;
+    *out = n;
+    return ENGRAM_OK;
+}
+
+// Whole-K projection on CTA pairs: 256-token x 256-channel units (see kernels_proj_pair.cuh).
+int launch_proj_pair(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
+                     int64_t n_tok, uint16_t *v, float4 *part, cudaStream_t stream, const GatherSrc *gs) {
+    const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim, M = plan->num_branches;
+    constexpr int BN = engram::kPairBN;
+    CUtensorMap map_m, map_wk, map_wv;
+    int rc;
+    if ((rc = make_map_bf16(&map_wk, w->w_k, static_cast<uint64_t>(M) * d_h, d_m, BN / 2)) != ENGRAM_OK) return rc;
+    if ((rc = make_map_bf16(&map_wv, w->w_v, d_h, d_m, BN / 2)) != ENGRAM_OK) return rc;
+    if (gs != nullptr)
+        map_m = map_wk;   // unused: the A tiles are gathered from the tables
+    else if ((rc = make_map_bf16(&map_m, m, static_cast<uint64_t>(n_tok), d_m, engram::kBM)) != ENGRAM_OK)
+        return rc;
+    if ((rc = gs ? set_pair_smem_attr<true>() : set_pair_smem_attr<false>()) != ENGRAM_OK) return rc;
+    int pairs = 0;
+    if ((rc = gs ? max_pairs<true>(&pairs) : max_pairs<false>(&pairs)) != ENGRAM_OK) return rc;
+    engram::ProjParams p{};
+    p.h = h;
+    p.gamma_q = w->gamma_q;
+    p.gamma_k = w->gamma_k;
+    p.v = v;
+    p.part = part;
+    p.n_tok = n_tok;
+    p.d_m = d_m;
+    p.d_h = d_h;
+    p.n_tiles = (M + 1) * d_h / BN;
+    p.M = M;
+    p.k_blocks = (d_m + engram::kBK - 1) / engram::kBK;
+    p.m_tiles = static_cast<int32_t>((n_tok + engram::kPairRows - 1) / engram::kPairRows);
+    p.k_splits = 1;
+    p.kb_per_split = p.k_blocks;
+    p.w_packed = static_cast<const uint8_t *>(w->w_packed);
+    if (gs != nullptr) {
+        p.idx = gs->idx;
+        p.H = plan->num_tables;
+        p.d_e = plan->cfg.row_dim;
+        for (int t = 0; t < p.H; ++t) {
+            p.tab[t] = static_cast<const uint16_t *>(gs->tables[t]);
+            p.tab_rows[t] = static_cast<uint32_t>(plan->cfg.table_rows[t]);
+        }
+    }
+    const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+    if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
+    // ENGRAM_PROJ_PAIRS (>= 1) caps the number of CTA pairs (tuning); read once per process.
+    static const int forced_pairs = [] {
+        const char *e = std::getenv("ENGRAM_PROJ_PAIRS");
+        const int v = e ? std::atoi(e) : 0;
+        return v > 0 ? v : 0;
+    }();
+    if (forced_pairs && forced_pairs < pairs) pairs = forced_pairs;
+    const int64_t npairs = total < pairs ? total : pairs;
+    auto kernel = gs ? engram::proj_pair_kernel<true> : engram::proj_pair_kernel<false>;
+    const int threads = engram::kProjThreads + (gs ? engram::kGatherThreads : 0);
+    ENGRAM_CUDA_TRY(launch_pdl(kernel, dim3(static_cast<unsigned>(2 * npairs)), dim3(threads),
+                               engram::PairCfg::kSmemBytes, stream, map_m, map_wk, map_wv, p),
+                    "proj_pair_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -682,53 +826,6 @@ int check_row_cache(const engram_plan *plan, const engram_row_cache *cache) {
     return ENGRAM_OK;
 }
 
-int set_fused_smem_attr() {
-    static bool done[64] = {};
-    int dev = 0;
-    ENGRAM_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
-    if (dev < 64 && done[dev]) return ENGRAM_OK;
-    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::fused_proj_gate_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         engram::FusedCfg<256>::kSmemBytes),
-                    "cudaFuncSetAttribute(fused_proj_gate_kernel)");
-    if (dev < 64) done[dev] = true;
-    return ENGRAM_OK;
-}
-
-int launch_fused_gate(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
-                      int32_t B, int32_t T, uint16_t *out, float *delta, float *vbuf, cudaStream_t stream) {
-    const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim;
-    const int64_t n_tok = static_cast<int64_t>(B) * T;
-    CUtensorMap map_m, map_wk, map_wv;
-    int rc;
-    if ((rc = make_map_bf16(&map_m, m, static_cast<uint64_t>(n_tok), d_m, engram::kBM)) != ENGRAM_OK) return rc;
-    if ((rc = make_map_bf16(&map_wk, w->w_k, d_h, d_m, 256)) != ENGRAM_OK) return rc;
-    if ((rc = make_map_bf16(&map_wv, w->w_v, d_h, d_m, 256)) != ENGRAM_OK) return rc;
-    if ((rc = set_fused_smem_attr()) != ENGRAM_OK) return rc;
-    engram::FusedParams p{};
-    p.h = h;
-    p.gamma_q = w->gamma_q;
-    p.gamma_k = w->gamma_k;
-    p.gamma_c = w->gamma_c;
-    p.conv_w = w->conv_w;
-    p.out = out;
-    p.delta = delta;
-    p.vbuf = vbuf;
-    p.n_tok = n_tok;
-    p.T = T;
-    p.d_m = d_m;
-    p.d_h = d_h;
-    p.k_blocks = (d_m + engram::kBK - 1) / engram::kBK;
-    p.n_units = static_cast<int32_t>((n_tok + engram::kFusedRows - 1) / engram::kFusedRows);
-    p.eps = plan->cfg.eps;
-    p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(d_h));
-    const int sms = sm_count();
-    const unsigned grid = static_cast<unsigned>(p.n_units < sms ? p.n_units : sms);
-    engram::fused_proj_gate_kernel<256><<<grid, engram::kFusedThreads, engram::FusedCfg<256>::kSmemBytes, stream>>>(
-        map_m, map_wk, map_wv, p);
-    ENGRAM_LAUNCHED("fused_proj_gate_kernel launch");
-    return ENGRAM_OK;
-}
-
 // Stage events are profiling hooks.  Under stream capture they must become event-record
 // nodes of the graph (cudaEventRecordExternal) so that they can be timed after a replay.
 cudaError_t record_stage_event(void *ev, cudaStream_t stream) {
@@ -742,18 +839,14 @@ cudaError_t record_stage_event(void *ev, cudaStream_t stream) {
 
 // history / xr (engram_forward's decode steps): when the step ends in decode_fused_kernel, that
 // kernel also advances the hash history and *history_done is set; otherwise the caller does.
+// gs: the projection gathers its A tiles from the tables (m unused; whole-K tiles only).
 int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                    int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out, float *delta, uint8_t *ws,
                    cudaStream_t stream, void *const *events, int32_t *history = nullptr,
-                   const int32_t *xr = nullptr, bool *history_done = nullptr) {
+                   const int32_t *xr = nullptr, bool *history_done = nullptr, const GatherSrc *gs = nullptr) {
     if (history_done) *history_done = false;
     const int64_t n_tok = static_cast<int64_t>(B) * T;
     const Workspace L = layout(plan, n_tok);
-    if (use_fused_gate(plan, n_tok, conv_state != nullptr)) {
-        if (events) ENGRAM_CUDA_TRY(record_stage_event(events[0], stream), "cudaEventRecord");
-        if (events) ENGRAM_CUDA_TRY(record_stage_event(events[1], stream), "cudaEventRecord");
-        return launch_fused_gate(plan, w, h, m, B, T, out, delta, reinterpret_cast<float *>(ws + L.v), stream);
-    }
     const ProjShape ps = proj_shape(plan, n_tok, true);
     uint16_t *v = reinterpret_cast<uint16_t *>(ws + L.v);
     float4 *part = reinterpret_cast<float4 *>(ws + L.part);
@@ -765,12 +858,16 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
     engram::ProjParams pp{};
     int rc;
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[0], stream), "cudaEventRecord");
-    if (ps.bn == 256)
-        rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
+    const bool pair = use_pair_mma(plan, n_tok, ps);
+    const int n_tiles = pair ? (plan->num_branches + 1) * d_h / engram::kPairBN : ps.n_tiles;
+    if (pair)
+        rc = launch_proj_pair(plan, w, h, m, n_tok, v, part, stream, gs);
+    else if (ps.bn == 256)
+        rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp, gs);
     else if (ps.bn == 128)
-        rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
+        rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp, gs);
     else
-        rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
+        rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp, gs);
     if (rc != ENGRAM_OK) return rc;
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[1], stream), "cudaEventRecord");
     if (fused_decode) {
@@ -793,7 +890,7 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
         if (history_done) *history_done = gp.history != nullptr;
         return ENGRAM_OK;
     }
-    return launch_gate_conv(plan, w, h, v, part, ps.n_tiles, B, T, conv_state, out, delta, stream,
+    return launch_gate_conv(plan, w, h, v, part, n_tiles, B, T, conv_state, out, delta, stream,
                             reinterpret_cast<float2 *>(ws + L.scal));
 }
 
@@ -808,23 +905,15 @@ int check_bt(int32_t B, int32_t T) {
 // ---------------------------------------------------------------- no-allocation variant
 // Scratch for engram_gate_conv_noalloc: one array per device in the library's static device
 // data.  Host code may not pass the symbol itself to a kernel (on the host it only names a
-// shadow variable); the device address is looked up once per device below.
+// shadow variable); its device address is looked up below.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[ENGRAM_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_noalloc_mutex;
-uint8_t *g_noalloc_ptr[64] = {};
-
+// Looked up on every call, with the caller's device current: a host-side lookup that
+// allocates nothing, and stays right if the context (and the module with it) is recreated.
 int noalloc_scratch(uint8_t **out) {
-    int dev = 0;
-    ENGRAM_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
-    if (dev < 0 || dev >= 64) return fail(ENGRAM_ERR_UNSUPPORTED, "device ordinal %d above 63", dev);
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_ptr[dev] == nullptr) {
-        void *p = nullptr;
-        ENGRAM_CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(no-alloc scratch)");
-        g_noalloc_ptr[dev] = static_cast<uint8_t *>(p);
-    }
-    *out = g_noalloc_ptr[dev];
+    void *p = nullptr;
+    ENGRAM_CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(no-alloc scratch)");
+    *out = static_cast<uint8_t *>(p);
     return ENGRAM_OK;
 }
 
@@ -887,8 +976,6 @@ int engram_init(const engram_config *cfg, engram_plan *plan) {
     const int M = c.num_branches == 0 ? 1 : c.num_branches;
     if (M < 1 || M > ENGRAM_MAX_BRANCHES)
         return fail(ENGRAM_ERR_UNSUPPORTED, "num_branches must be in 0..%d", ENGRAM_MAX_BRANCHES);
-    if (M > 1 && (c.flags & ENGRAM_FLAG_FUSED_GATE))
-        return fail(ENGRAM_ERR_UNSUPPORTED, "ENGRAM_FLAG_FUSED_GATE needs a single branch");
     if (c.table_dtype != ENGRAM_TABLE_BF16 && c.table_dtype != ENGRAM_TABLE_FP8_E4M3)
         return fail(ENGRAM_ERR_INVALID_ARG, "unknown table_dtype %d", c.table_dtype);
     for (int h = 0; h < ENGRAM_MAX_TABLES; ++h) {
@@ -903,7 +990,7 @@ int engram_init(const engram_config *cfg, engram_plan *plan) {
     }
     if (c.table_dtype == ENGRAM_TABLE_FP8_E4M3 && c.row_dim % 16 != 0)
         return fail(ENGRAM_ERR_UNSUPPORTED, "FP8 tables need row_dim % 16 == 0");
-    if (c.flags & ~ENGRAM_FLAG_FUSED_GATE) return fail(ENGRAM_ERR_INVALID_ARG, "unknown flags 0x%x", c.flags);
+    if (c.flags & ~(ENGRAM_FLAG_SEPARATE_GATHER | ENGRAM_FLAG_SINGLE_CTA_MMA)) return fail(ENGRAM_ERR_INVALID_ARG, "unknown flags 0x%x", c.flags);
 
     std::memset(plan, 0, sizeof *plan);
     plan->cfg = c;
@@ -1134,9 +1221,10 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const void 
         return ENGRAM_OK;
     };
     // Decode-sized batches on HBM-resident tables: remap + hash + gather in one kernel (the
-    // row ids stay in registers).  Larger batches: the hash kernel, then the wide gather.
-    const bool fused_lookup = !L.staged && plan->cfg.table_location == ENGRAM_TABLES_DEVICE &&
-                              n_tok * plan->num_tables <= kFusedLookupMaxRows;
+    // row ids stay in registers).  Larger batches: the hash kernel, then either the
+    // projection gathers the rows into its tiles itself, or the wide gather writes m.
+    const ForwardPath fp = forward_path(plan, n_tok);
+    const bool fused_lookup = fp.fused_lookup;
     if ((rc = rec(0)) != ENGRAM_OK) return rc;
     if (fused_lookup) {
         if ((rc = rec(1)) != ENGRAM_OK) return rc;
@@ -1160,12 +1248,14 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const void 
                                stream)) != ENGRAM_OK)
             return rc;
         if ((rc = launch_gather(plan, sidx, stage_ptr, n_tok, m, stream, n_tok)) != ENGRAM_OK) return rc;
-    } else if ((rc = launch_gather(plan, idx, tables, n_tok, m, stream)) != ENGRAM_OK) {
+    } else if (!fp.gather_in_proj && (rc = launch_gather(plan, idx, tables, n_tok, m, stream)) != ENGRAM_OK) {
         return rc;
     }
     bool history_done = false;
-    if ((rc = gate_conv_impl(plan, w, h, m, B, T, conv_state, out, delta_dbg, ws, stream,
-                             stage_events ? stage_events + 2 : nullptr, history, xr, &history_done)) != ENGRAM_OK)
+    const GatherSrc gsrc{idx, tables};
+    if ((rc = gate_conv_impl(plan, w, h, fp.gather_in_proj ? nullptr : m, B, T, conv_state, out, delta_dbg, ws,
+                             stream, stage_events ? stage_events + 2 : nullptr, history, xr, &history_done,
+                             fp.gather_in_proj ? &gsrc : nullptr)) != ENGRAM_OK)
         return rc;
     if ((rc = rec(4)) != ENGRAM_OK) return rc;
     if (history != nullptr && plan->hist_len > 0 && !history_done) {
@@ -1209,6 +1299,56 @@ int engram_gate_conv_noalloc(const engram_plan *plan, const engram_weights *w, c
     else rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream);
     if (rc != ENGRAM_OK) return rc;
     return launch_gate_conv(plan, w, h, v, part, n_tiles, B, T, conv_state, out, delta_dbg, stream);
+}
+
+int engram_forward_path(const engram_plan *plan, int32_t B, int32_t T, uint32_t *path) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if ((rc = check_bt(B, T)) != ENGRAM_OK) return rc;
+    if (path == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "path is NULL");
+    const int64_t n_tok = static_cast<int64_t>(B) * T;
+    const ForwardPath fp = forward_path(plan, n_tok);
+    uint32_t bits = 0;
+    if (fp.fused_lookup) bits |= ENGRAM_PATH_FUSED_LOOKUP;
+    if (fp.staged) bits |= ENGRAM_PATH_STAGED_ROWS;
+    if (fp.gather_in_proj) bits |= ENGRAM_PATH_GATHER_IN_PROJ;
+    if (fp.ps.k_splits > 1) bits |= ENGRAM_PATH_SPLIT_K;
+    if (fp.pair) bits |= ENGRAM_PATH_PAIR_MMA;
+    *path = bits;
+    return ENGRAM_OK;
+}
+
+int engram_synchronize(engram_stream_t stream) {
+    ENGRAM_CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "cudaStreamSynchronize");
+    uint32_t s = 0;
+    ENGRAM_CUDA_TRY(cudaMemcpyFromSymbol(&s, g_engram_status, sizeof s), "cudaMemcpyFromSymbol");
+    if (s & ENGRAM_STATUS_WAIT_TIMEOUT)
+        return fail(ENGRAM_ERR_TIMEOUT, "a pipeline wait inside a kernel gave up (device status 0x%x)", s);
+    return ENGRAM_OK;
+}
+
+int engram_selftest_wait_timeout(const engram_plan *plan, const engram_weights *w, const uint16_t *h,
+                                 const uint16_t *m, int64_t n_tok, void *workspace, size_t workspace_bytes,
+                                 uint64_t wait_limit_ns, engram_stream_t stream) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if ((rc = validate_weights(plan, w)) != ENGRAM_OK) return rc;
+    if (n_tok < 1 || n_tok > (int64_t(1) << 31)) return fail(ENGRAM_ERR_INVALID_ARG, "n_tok must be in 1..2^31");
+    if (wait_limit_ns < 1000 || wait_limit_ns > 1000000000ull)
+        return fail(ENGRAM_ERR_INVALID_ARG, "wait_limit_ns must be in [1 us, 1 s]");
+    if (!h || !m || !aligned16(h) || !aligned16(m))
+        return fail(ENGRAM_ERR_INVALID_ARG, "h and m must be non-NULL and 16-byte aligned");
+    const Workspace L = layout(plan, n_tok);
+    if (!workspace || workspace_bytes < L.total)
+        return fail(ENGRAM_ERR_INVALID_ARG, "workspace too small: need %zu bytes", L.total);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint16_t *v = reinterpret_cast<uint16_t *>(ws + L.v);
+    float4 *part = reinterpret_cast<float4 *>(ws + L.part);
+    ProjTest test;
+    test.wait_limit_ns = wait_limit_ns;
+    test.stall = 1;
+    return launch_proj<64>(plan, w, h, m, n_tok, v, part, static_cast<cudaStream_t>(stream), nullptr, 1, 0, false,
+                           nullptr, nullptr, test);
 }
 
 uint64_t engram_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }

@@ -638,7 +638,9 @@ __global__ void __launch_bounds__(kFusedDecodeThreads, 2) decode_fused_kernel(co
     constexpr int S = 9;
     __shared__ float s_red[4][kFusedDecodeThreads / 32];
     __shared__ float s_gb[2];
-    pdl_launch_dependents();   // the history update may be scheduled now (it waits for this kernel)
+    // dependents (the next step's kernels) may be scheduled now; the hash history, when given,
+    // is advanced below by this kernel itself, after pdl_wait
+    pdl_launch_dependents();
     const int b = blockIdx.x;
     const int d_h = p.d_h;
     const int64_t split_stride = pp.n_tok * (2 * d_h);

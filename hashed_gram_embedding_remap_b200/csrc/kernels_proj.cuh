@@ -27,6 +27,8 @@ constexpr int kBM = 128;          // tokens per tile (UMMA M)
 constexpr int kBK = 64;           // K elements per stage: one 128-byte swizzle row
 constexpr int kUmmaK = 16;        // K per tcgen05.mma for 16-bit inputs
 constexpr int kProjThreads = 192; // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
+constexpr int kGatherThreads = 128; // row-gather mode: warps 6-9 fill the A tiles from the tables
+constexpr int kGatherRows = kBM * (kBK * 2 / 16) / kGatherThreads;   // tile rows per gather thread (8)
 
 template <int BN>
 struct ProjCfg {
@@ -40,6 +42,7 @@ struct ProjCfg {
     // floats: 16-byte row starts, conflict-free quarter-warp phases)
     static constexpr int kTrStride = 36;
     static constexpr int kTrBytes = 4 * 32 * kTrStride * 4;
+    static_assert(kTrBytes >= kBM * ENGRAM_MAX_TABLES * 4, "row-gather mode keeps a tile's row ids there");
     // dynamic smem: [align pad][stages x A][stages x B][transpose tiles]
     //               [full, empty, tmem_full, tmem_empty][tmem addr]
     static constexpr int kBarBytes = (2 * kStages + 2 * kAccum) * 8;
@@ -62,6 +65,14 @@ struct ProjParams {
     int32_t kb_per_split;      // k-blocks per split
     float *acc_out;            // [k_splits, n_tok, (M+1)*d_h] when k_splits > 1
     const uint8_t *w_packed;   // non-null: B tiles come as 32 KB pre-swizzled blocks (BN = 256)
+    // row-gather mode (GATHER): the A tiles are the tables' rows named by idx, not a tile of m
+    const uint32_t *idx;                   // [n_tok, H] row ids
+    const uint16_t *tab[ENGRAM_MAX_TABLES];  // bf16 tables [tab_rows[h], d_e]
+    uint32_t tab_rows[ENGRAM_MAX_TABLES];
+    int32_t H, d_e;
+    uint64_t wait_limit_ns;    // bound of every pipeline wait (0: ENGRAM_WAIT_TIMEOUT_NS)
+    int32_t stall;             // self-test of the bounded waits: issue no loads at all, so that
+                               // the first wait for a stage runs out and the kernel unwinds
 };
 
 // Packs [W_k ; W_v] into pre-swizzled 256 x 64 tiles (the layout engram_pack_weights
@@ -113,6 +124,158 @@ __device__ __forceinline__ float v_hi(uint32_t w) {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
 }
 
+// Whole-K epilogue of one 32-column chunk of a token's accumulator row: for a key tile the
+// gate's partial sums S0 = sum h^2, S1 = sum h gamma_q gamma_k k~, S2 = sum k~^2 over the
+// chunk's channels; for a value tile the fp16 store of v and S3 = sum v^2 (in a0).
+__device__ __forceinline__ void epilogue_chunk(const ProjParams &p, const float (&accv)[32], int64_t n, int br,
+                                               int ch, bool is_key, float &a0, float &a1, float &a2) {
+    if (is_key) {
+        const uint4 *hp = reinterpret_cast<const uint4 *>(p.h + (n * p.M + br) * p.d_h + ch);
+        const uint4 *gq = reinterpret_cast<const uint4 *>(p.gamma_q + ch);
+        const uint4 *gk = reinterpret_cast<const uint4 *>(p.gamma_k + ch);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 hw = __ldg(hp + q), qw = __ldg(gq + q), kw = __ldg(gk + q);
+            const uint32_t h4[4] = {hw.x, hw.y, hw.z, hw.w};
+            const uint32_t q4[4] = {qw.x, qw.y, qw.z, qw.w};
+            const uint32_t k4[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = q * 8 + e * 2;
+                const float h0 = bf16_lo(h4[e]), h1 = bf16_hi(h4[e]);
+                const float g0 = bf16_lo(q4[e]) * bf16_lo(k4[e]);
+                const float g1 = bf16_hi(q4[e]) * bf16_hi(k4[e]);
+                const float k0 = accv[j], k1 = accv[j + 1];
+                a0 = fmaf(h0, h0, a0);
+                a0 = fmaf(h1, h1, a0);
+                a1 = fmaf(h0 * g0, k0, a1);
+                a1 = fmaf(h1 * g1, k1, a1);
+                a2 = fmaf(k0, k0, a2);
+                a2 = fmaf(k1, k1, a2);
+            }
+        }
+    } else {
+        // S3 from the fp32 accumulator; v itself is stored as fp16
+        uint4 *vp = reinterpret_cast<uint4 *>(p.v + n * p.d_h + ch);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float x0 = accv[8 * q + 2 * e], x1 = accv[8 * q + 2 * e + 1];
+                a0 = fmaf(x0, x0, fmaf(x1, x1, a0));
+                wv[e] = pack_v2(x0, x1);
+            }
+            vp[q] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+    }
+}
+
+// L2 prefetch of `bytes` (a multiple of 16, 16-byte aligned) at `src`: no data reaches the SM.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void gather_bar_sync() {   // the gather warps only (named barrier 1)
+    asm volatile("bar.sync 1, %0;" ::"n"(kGatherThreads) : "memory");
+}
+constexpr uint32_t kNoRow = 0xFFFFFFFFu;   // sIdx entry of a token past n_tok or a bad row id
+
+// Row-gather producer (kGatherThreads threads): fills the A tile of every stage from the
+// tables.  Work unit t (t = t0, t0 + tstep, ... < total; whole K) covers tile rows
+// [(t / n_tiles) * unit_rows + row_off, +kBM).  At the start of a unit the gather warps copy
+// the unit's row ids [kBM, H] into shared memory (sIdx) and ask L2 to prefetch every row the
+// unit will read (the CTA whose unit is the tile's first channel slice only: the other
+// slices' CTAs read the same rows at about the same time), so the k-blocks after the first
+// few find their rows in L2.  Thread g then
+// fills the 16-byte piece j = g % 8 of tile rows r0 + 16i (r0 = g / 8, i < 8) of every stage;
+// all those rows share r mod 8 = r0 mod 8, hence one 128-byte-swizzle position.  Column c of
+// the memory vector lies in table c / d_e at column c % d_e (the concatenation of step 3).
+// Lane 0 of each warp waits for the stage to be free; each thread's completion is one
+// arrival on the stage's full barrier (cp.async.mbarrier.arrive.noinc), which is what makes
+// the copies visible to the tensor cores that read the stage.  Rows past n_tok,
+// bad row ids and columns past d_m are zero-filled.  Returns after its copies have landed.
+template <int S, int ATILE>
+__device__ __forceinline__ void gather_a_tiles(const ProjParams &p, uint8_t *sA, uint32_t *sIdx, uint64_t *full_bar,
+                                               uint64_t *empty_bar, volatile int *abort_flag, uint64_t lim,
+                                               int g, int t0, int tstep, int total, int unit_rows, int row_off) {
+    const int j = g & 7;
+    const int r0 = g >> 3;
+    const int lane = g & 31;
+    const uint32_t off0 = static_cast<uint32_t>(r0 * (kBK * 2) + ((j ^ (r0 & 7)) << 4));
+    constexpr uint32_t kRowStep = (kGatherThreads / 8) * kBK * 2;   // 16 rows of 128 bytes
+    const int H = p.H;
+    const uint32_t row_bytes = static_cast<uint32_t>(p.d_e) * 2;
+    int it = 0;
+    bool stop = false;
+    for (int t = t0; t < total && !stop; t += tstep) {
+        const int64_t m0 = static_cast<int64_t>(t / p.n_tiles) * unit_rows + row_off;
+        // ---- the unit's row ids into shared memory, and its rows on their way into L2
+        gather_bar_sync();   // every gather thread is done with the previous unit's ids
+        if (g == 0 && t + tstep < total) {   // the next unit's row ids, into L2 ahead of time
+            const int64_t m1 = static_cast<int64_t>((t + tstep) / p.n_tiles) * unit_rows + row_off;
+            const int64_t rows = min(static_cast<int64_t>(kBM), p.n_tok - m1);
+            const uint32_t bytes = static_cast<uint32_t>(rows * H * 4) & ~15u;   // whole 16-byte pieces inside idx
+            if (rows > 0 && bytes > 0) prefetch_l2_bulk(p.idx + m1 * H, bytes);
+        }
+        const bool prefetch_rows = t % p.n_tiles == 0;
+        // kBM * H entries, kGatherThreads apart: eight independent loads in flight per round
+        for (int e0 = g; e0 < kBM * H; e0 += 8 * kGatherThreads) {
+            uint32_t rid[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + u * kGatherThreads;
+                const int64_t n = m0 + e / H;
+                rid[u] = (e < kBM * H && n < p.n_tok) ? __ldg(p.idx + m0 * H + e) : kNoRow;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + u * kGatherThreads;
+                if (e >= kBM * H) break;
+                const int h = e % H;
+                if (rid[u] != kNoRow) {
+                    if (rid[u] >= p.tab_rows[h]) {
+                        atomicOr(&g_engram_status, ENGRAM_STATUS_BAD_ROW);
+                        rid[u] = kNoRow;
+                    } else if (prefetch_rows) {
+                        prefetch_l2_bulk(p.tab[h] + static_cast<int64_t>(rid[u]) * p.d_e, row_bytes);
+                    }
+                }
+                sIdx[e] = rid[u];
+            }
+        }
+        gather_bar_sync();
+        // ---- the unit's k-blocks
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+            const int s = it % S;
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(&empty_bar[s], ((it / S) & 1) ^ 1, abort_flag, lim);
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                stop = true;
+                break;
+            }
+            const uint32_t dst = smem_u32(sA + s * ATILE) + off0;
+            const int col = kb * kBK + j * 8;
+            if (col < p.d_m) {
+                const int h = col / p.d_e;
+                const uint16_t *base = p.tab[h] + (col - h * p.d_e);
+#pragma unroll
+                for (int i = 0; i < kGatherRows; ++i) {
+                    const uint32_t rid = sIdx[(r0 + 16 * i) * H + h];
+                    const bool valid = rid != kNoRow;
+                    cp_async_16(dst + i * kRowStep, valid ? base + static_cast<int64_t>(rid) * p.d_e : base,
+                                valid ? 16u : 0u);
+                }
+            } else {   // columns beyond d_m (ragged last k-block): zeros
+#pragma unroll
+                for (int i = 0; i < kGatherRows; ++i) cp_async_16(dst + i * kRowStep, p.tab[0], 0u);
+            }
+            cp_async_arrive_noinc(&full_bar[s]);
+        }
+    }
+    cp_async_wait_all();   // nothing may still land in shared memory after the CTA ends
+}
+
 // Persistent: grid = min(#tiles, #SMs); CTA i takes tiles i, i + grid, ...  Tile t covers
 // tokens [128*(t / n_tiles), +128) and channel slice t % n_tiles, so the CTAs running at
 // one time share a few 128-token blocks of m (re-read from L2) and stream all of W.
@@ -120,8 +283,14 @@ __device__ __forceinline__ float v_hi(uint32_t w) {
 // Two TMEM accumulators: the epilogue drains tile i while the MMAs of tile i+1 run.
 // SPLIT: compiled for split-K work units (p.k_splits > 1, raw partial accumulators out) or
 // for whole-K tiles only, so that neither epilogue costs the other registers.
-template <int BN, bool SPLIT>
-__global__ void __launch_bounds__(kProjThreads, 1)
+// GATHER (whole-K tiles only): m is never materialised.  Warps 6-9 build each 128 x 64 A
+// tile from the tables themselves -- token n's columns [64kb, 64kb+64) are 16-byte pieces of
+// the rows idx[n, h] names (column c lies in table c / d_e at column c % d_e, the
+// concatenation of step 3) -- with cp.async into the same 128-byte-swizzled layout the TMA
+// would write; each thread's completion is one arrival on the stage's full barrier.  Warp 0
+// then streams only the weight tiles.
+template <int BN, bool SPLIT, bool GATHER>
+__global__ void __launch_bounds__(kProjThreads + (GATHER ? kGatherThreads : 0), 1)
     proj_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ CUtensorMap map_wk,
                 const __grid_constant__ CUtensorMap map_wv, const __grid_constant__ ProjParams p) {
     using Cfg = ProjCfg<BN>;
@@ -139,7 +308,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(tempty_bar + NACC);
     __shared__ int s_abort;
 
+    static_assert(!(SPLIT && GATHER), "the row-gather mode runs whole-K tiles only");
     pdl_launch_dependents();   // the kernel after this one may load its independent inputs now
+    const uint64_t lim = p.wait_limit_ns ? p.wait_limit_ns : ENGRAM_WAIT_TIMEOUT_NS;
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const int mn_tiles = p.m_tiles * p.n_tiles;
@@ -150,7 +321,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     if (threadIdx.x == 0) {
         s_abort = 0;
         for (int s = 0; s < S; ++s) {
-            mbar_init(&full_bar[s], 1);
+            mbar_init(&full_bar[s], GATHER ? 1 + kGatherThreads : 1);
             mbar_init(&empty_bar[s], 1);
         }
         for (int a = 0; a < NACC; ++a) {
@@ -171,8 +342,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
 
+    constexpr uint32_t kTxBytes = GATHER ? Cfg::kBTile : Cfg::kStageBytes;   // TMA bytes per stage
     if (warp == 0) {
-        if (lane == 0) {
+        if (lane == 0 && !p.stall) {
             // unit t -> (k split, m tile, n tile) and the weight tile it streams
             auto unit = [&](int t, int &ks, int &mt, int &nt, int &kb0, int &kb1) {
                 ks = t / mn_tiles;
@@ -200,7 +372,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 unit(blockIdx.x, ks, mt, nt, kb0, kb1);
                 pre = min(S, kb1 - kb0);
                 for (int q = 0; q < pre; ++q) {   // fresh stages: nothing to wait for
-                    mbar_arrive_expect_tx(&full_bar[q], Cfg::kStageBytes);
+                    mbar_arrive_expect_tx(&full_bar[q], kTxBytes);
                     load_b(q, nt, kb0 + q);
                 }
             }
@@ -213,13 +385,13 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     if (it < pre) {   // weight tile and byte count already issued
-                        tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
+                        if constexpr (!GATHER) tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
                         continue;
                     }
                     const uint32_t ph = (it / S) & 1;
-                    if (!mbar_wait(&empty_bar[s], ph ^ 1, &s_abort)) break;
-                    mbar_arrive_expect_tx(&full_bar[s], Cfg::kStageBytes);
-                    tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
+                    if (!mbar_wait(&empty_bar[s], ph ^ 1, &s_abort, lim)) break;
+                    mbar_arrive_expect_tx(&full_bar[s], kTxBytes);
+                    if constexpr (!GATHER) tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
                     load_b(s, nt, kb);
                     issued = it + 1;
                 }
@@ -228,7 +400,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 // Every issued copy must land before the CTA's shared memory is released.
                 volatile int never = 0;
                 for (int k = issued - S > 0 ? issued - S : 0; k < issued; ++k)
-                    if (!mbar_wait(&full_bar[k % S], (k / S) & 1, &never)) break;
+                    if (!mbar_wait(&full_bar[k % S], (k / S) & 1, &never, lim)) break;
             }
         }
     } else if (warp == 1) {
@@ -238,7 +410,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             for (int t = blockIdx.x; t < total && !s_abort; t += gridDim.x, ++li) {
                 const int acc = li % NACC;
                 const uint32_t use = li / NACC;
-                if (!mbar_wait(&tempty_bar[acc], (use & 1) ^ 1, &s_abort)) break;
+                if (!mbar_wait(&tempty_bar[acc], (use & 1) ^ 1, &s_abort, lim)) break;
                 tc_fence_after();
                 const uint32_t dst = tmem_base + acc * BN;
                 const int ks = t / mn_tiles;
@@ -247,7 +419,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1;
-                    if (!mbar_wait(&full_bar[s], ph, &s_abort)) { ok = false; break; }
+                    if (!mbar_wait(&full_bar[s], ph, &s_abort, lim)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t adesc = sdesc_kmajor_sw128(sA + s * Cfg::kATile);
                     const uint64_t bdesc = sdesc_kmajor_sw128(sB + s * Cfg::kBTile);
@@ -265,7 +437,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 for (int a = 0; a < NACC; ++a) mbar_arrive(&tfull_bar[a]);   // release waiting epilogue warps
             }
         }
-    } else {
+    } else if (warp < kProjThreads / 32) {
         // ---------------------------------------------------------------- epilogue
         const int sub = warp & 3;                      // TMEM lane quarter this warp may access
         const int row = sub * 32 + lane;
@@ -273,7 +445,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++li) {
             const int acc = li % NACC;
             const uint32_t use = li / NACC;
-            if (!mbar_wait(&tfull_bar[acc], use & 1, &s_abort) || s_abort) break;
+            if (!mbar_wait(&tfull_bar[acc], use & 1, &s_abort, lim) || s_abort) break;
             tc_fence_after();
             const int ks = t / mn_tiles, tmn = t - ks * mn_tiles;
             const int mt = tmn / p.n_tiles, nt = tmn - mt * p.n_tiles;
@@ -311,47 +483,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                     __syncwarp();   // the tile is rewritten by the next column block
                     continue;
                 }
-                if (!valid) continue;
-                if (is_key) {
-                    const uint4 *hp = reinterpret_cast<const uint4 *>(p.h + (n * p.M + br) * p.d_h + c0 + cc);
-                    const uint4 *gq = reinterpret_cast<const uint4 *>(p.gamma_q + c0 + cc);
-                    const uint4 *gk = reinterpret_cast<const uint4 *>(p.gamma_k + c0 + cc);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 hw = __ldg(hp + q), qw = __ldg(gq + q), kw = __ldg(gk + q);
-                        const uint32_t h4[4] = {hw.x, hw.y, hw.z, hw.w};
-                        const uint32_t q4[4] = {qw.x, qw.y, qw.z, qw.w};
-                        const uint32_t k4[4] = {kw.x, kw.y, kw.z, kw.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = q * 8 + e * 2;
-                            const float h0 = bf16_lo(h4[e]), h1 = bf16_hi(h4[e]);
-                            const float g0 = bf16_lo(q4[e]) * bf16_lo(k4[e]);
-                            const float g1 = bf16_hi(q4[e]) * bf16_hi(k4[e]);
-                            const float k0 = accv[j], k1 = accv[j + 1];
-                            a0 = fmaf(h0, h0, a0);
-                            a0 = fmaf(h1, h1, a0);
-                            a1 = fmaf(h0 * g0, k0, a1);
-                            a1 = fmaf(h1 * g1, k1, a1);
-                            a2 = fmaf(k0, k0, a2);
-                            a2 = fmaf(k1, k1, a2);
-                        }
-                    }
-                } else {
-                    // S3 from the fp32 accumulator; v itself is stored as fp16
-                    uint4 *vp = reinterpret_cast<uint4 *>(p.v + n * p.d_h + c0 + cc);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t wv[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float x0 = accv[8 * q + 2 * e], x1 = accv[8 * q + 2 * e + 1];
-                            a0 = fmaf(x0, x0, fmaf(x1, x1, a0));
-                            wv[e] = pack_v2(x0, x1);
-                        }
-                        vp[q] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                    }
-                }
+                if (valid) epilogue_chunk(p, accv, n, br, c0 + cc, is_key, a0, a1, a2);
             }
             // the accumulator has been read: hand it back to the MMA warp
             tc_fence_before();
@@ -360,6 +492,14 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             if constexpr (!SPLIT) {
                 if (valid) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
             }
+        }
+    } else if constexpr (GATHER) {
+        // ---------------------------------------------------------------- A-tile row gather
+        if (!p.stall) {
+            pdl_wait();   // the row ids come from the kernel before this one
+            // the row ids live in the split-K transpose region, unused by whole-K tiles
+            gather_a_tiles<S, Cfg::kATile>(p, sA, reinterpret_cast<uint32_t *>(s_tr), full_bar, empty_bar, &s_abort,
+                                           lim, threadIdx.x - kProjThreads, blockIdx.x, gridDim.x, total, kBM, 0);
         }
     }
     tc_fence_before();

@@ -46,8 +46,8 @@ extern "C" {
 #define ENGRAM_ERR_INVALID_ARG (-1) /* null / misaligned pointer, bad size, dim mismatch */
 #define ENGRAM_ERR_UNSUPPORTED (-2) /* valid but not handled: d_e % 8, order outside 1..4, ... */
 #define ENGRAM_ERR_CUDA (-3)        /* a CUDA runtime call failed; see engram_last_error() */
-#define ENGRAM_ERR_OOM (-4)         /* not enough device memory for the request */
-#define ENGRAM_ERR_TIMEOUT (-5)     /* a bounded device-side wait gave up */
+#define ENGRAM_ERR_TIMEOUT (-5)     /* a bounded device-side wait gave up (engram_synchronize);
+                                       -4 is not used */
 
 /* bits of the per-device status word (engram_device_status) */
 #define ENGRAM_STATUS_BAD_TOKEN 0x1u    /* a token id was outside [0, vocab_in) */
@@ -117,12 +117,14 @@ typedef struct engram_config {
  * M = 1 is the single-branch layer, with the layouts stated at each entry point. */
 
 /* engram_config.flags */
-#define ENGRAM_FLAG_FUSED_GATE 0x1 /* prefill with kernel 4 / dilation 3 and d_h % 256 == 0:
-                                      run projections, gate and conv in ONE persistent kernel
-                                      (the conv pass rides in the projection's epilogue warps).
-                                      Results match the two-kernel path within tolerance; it is
-                                      opt-in because it is currently slower on B200.  Single
-                                      branch only (num_branches <= 1). */
+#define ENGRAM_FLAG_SEPARATE_GATHER 0x2 /* engram_forward gathers the rows into m with the
+                                           separate gather kernel even where the projection
+                                           could gather them straight into its tiles (see
+                                           engram_forward_path); results are bit-identical
+                                           either way.  Bit 0x1 is retired and rejected. */
+#define ENGRAM_FLAG_SINGLE_CTA_MMA 0x4  /* never pair CTAs for the projection's MMAs (see
+                                           ENGRAM_PATH_PAIR_MMA); results are bit-identical
+                                           either way. */
 
 /* Validated config plus derived constants.  Caller-owned, plain data: engram_init fills
  * it, every other call reads it.  Do not modify its fields. */
@@ -290,11 +292,14 @@ int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
 
 /* Steps 1-6 chained: remap + hash (one kernel), gather, projections with the gate's partial
  * reductions fused in their epilogue, then gate + conv + residual, then the history update
- * when `history` is given.  Kernels per call: prefill batches launch remap + hash, gather,
- * projection, gate scalars and the streaming gate + conv kernel (5); batches of at most
- * 16,384 (token, table) rows on HBM-resident tables fuse remap + hash + gather into one
- * kernel; one-token decode steps whose projection splits K finish the split sums, gate,
- * conv and the history update in one kernel (lookup, projection, that kernel: 3).
+ * when `history` is given.  Kernels per call (engram_forward_path tells which apply): prefill
+ * batches on bf16 HBM-resident tables launch remap + hash, the projection -- which gathers
+ * each token's rows into its tiles itself -- gate scalars and the streaming gate + conv
+ * kernel (4); with e4m3 or host-mapped tables, or ENGRAM_FLAG_SEPARATE_GATHER, a gather
+ * kernel writes m first (5); batches of at most 16,384 (token, table) rows on HBM-resident
+ * tables fuse remap + hash + gather into one kernel; one-token decode steps whose
+ * projection splits K finish the split sums, gate, conv and the history update in one
+ * kernel (lookup, projection, that kernel: 3).
  * engram_kernel_launches() counts them.
  * ids: int32 [B, T] raw token ids.  remap: int32 [vocab_in], or NULL when ids are already
  * in the compressed vocabulary.  history / conv_state: NULL for prefill, or the decode state
@@ -305,7 +310,7 @@ int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
  * be timed per stage.
  * CUDA graphs: after one eager call on a device (which resolves the tensor-map encoder and
  * sets kernel attributes), engram_forward / engram_gate_conv may be captured and replayed. */
-#define ENGRAM_FORWARD_STAGES 4 /* hash, gather, projections, gate+conv */
+#define ENGRAM_FORWARD_STAGES 4 /* hash, gather (empty when the projection gathers), projections, gate+conv */
 int engram_forward(const engram_plan *plan, const engram_weights *w,
                    const void *const *tables, const int32_t *ids, const int32_t *remap,
                    int32_t B, int32_t T, int32_t *history, uint16_t *conv_state,
@@ -324,9 +329,10 @@ int engram_forward(const engram_plan *plan, const engram_weights *w,
  *    partial sums (BN = 64, 128 or 256, the projection tile width), each rounded up to 256; a
  *    request that does not fit returns ENGRAM_ERR_UNSUPPORTED and launches nothing.  At
  *    d_h = 2560 that is about 5,000 tokens per call.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call before any
- *    stream capture.  No call allocates or frees memory.
+ *  - Every call looks up the array's device address (cudaGetSymbolAddress, a host-side
+ *    lookup) with the caller's device current; the first call on a device may load the
+ *    library's device code there, so make it before any stream capture.  No call allocates
+ *    or frees memory.
  *  - Every call on a device shares the one array and leaves its contents behind.  No part of
  *    it needs clearing: each element a call reads is written earlier in the same call.
  *    Calls that overlap on the GPU (other streams, other host threads) race on the array
@@ -336,6 +342,49 @@ int engram_forward(const engram_plan *plan, const engram_weights *w,
 int engram_gate_conv_noalloc(const engram_plan *plan, const engram_weights *w, const uint16_t *h,
                              const uint16_t *m, int32_t B, int32_t T, uint16_t *conv_state,
                              uint16_t *out, float *delta_dbg, engram_stream_t stream);
+
+/* The kernels engram_forward runs for a batch of B sequences of T tokens, as ENGRAM_PATH_*
+ * bits in *path (host only, no CUDA call).  A diagnostic for tests and benchmarks:
+ *   FUSED_LOOKUP   remap + hash + gather in one kernel (at most 16,384 (token, table) rows,
+ *                  HBM-resident tables); m is written by it;
+ *   STAGED_ROWS    host-mapped tables: the batch's distinct rows are staged into HBM first;
+ *   GATHER_IN_PROJ the projection gathers each token's rows straight from the tables into
+ *                  its shared-memory tiles (bf16 HBM-resident tables, whole-K projection
+ *                  tiles, ENGRAM_FLAG_SEPARATE_GATHER not set): m is never written, and the
+ *                  workspace holds no m;
+ *   SPLIT_K        the projection splits K across CTAs (decode-sized batches);
+ *   PAIR_MMA       the projection runs on pairs of CTAs (a thread-block cluster of two), each
+ *                  tensor-core MMA spanning both: 256-token x 256-channel tiles, each CTA
+ *                  holding half of every operand tile (d_h % 256 == 0, whole-K tiles, at
+ *                  least 148 tiles, ENGRAM_FLAG_SINGLE_CTA_MMA not set); the workspace's
+ *                  partial sums then have (M+1)*d_h/256 columns per token.
+ * Otherwise the hash kernel writes the row ids and the separate gather kernel writes m. */
+#define ENGRAM_PATH_FUSED_LOOKUP 0x1u
+#define ENGRAM_PATH_STAGED_ROWS 0x2u
+#define ENGRAM_PATH_GATHER_IN_PROJ 0x4u
+#define ENGRAM_PATH_SPLIT_K 0x8u
+#define ENGRAM_PATH_PAIR_MMA 0x10u
+int engram_forward_path(const engram_plan *plan, int32_t B, int32_t T, uint32_t *path);
+
+/* Wait for `stream` and report what the device found: ENGRAM_ERR_TIMEOUT if a pipeline wait
+ * inside one of this library's kernels on the current device gave up since the status word
+ * was last cleared (the kernel then abandoned its work and returned, so its outputs are
+ * undefined, but the device stays usable); ENGRAM_ERR_CUDA if the stream reports a CUDA
+ * error; ENGRAM_OK otherwise.  Does not clear the status word (engram_device_status does). */
+int engram_synchronize(engram_stream_t stream);
+
+/* Self-test of the bounded waits (no counterpart in the pages: it checks this library's
+ * failure handling).  Runs the projection kernel of engram_gate_conv over n_tok tokens with
+ * its producer stalled -- no tile is ever loaded -- and every pipeline wait bounded by
+ * wait_limit_ns (1 us .. 1 s) instead of the built-in 2 s.  Each CTA's first wait for a stage
+ * runs out, raises ENGRAM_STATUS_WAIT_TIMEOUT, and the CTA unwinds: its other roles stop
+ * waiting, its tensor memory is released and it exits.  engram_synchronize(stream) then
+ * returns ENGRAM_ERR_TIMEOUT.  Arguments as engram_gate_conv (h, m: bf16 [n_tok, d_h] and
+ * [n_tok, d_m], never read; workspace >= engram_workspace_size(plan, n_tok)).  Clear the
+ * status word afterwards with engram_device_status(&s, 1). */
+int engram_selftest_wait_timeout(const engram_plan *plan, const engram_weights *w, const uint16_t *h,
+                                 const uint16_t *m, int64_t n_tok, void *workspace, size_t workspace_bytes,
+                                 uint64_t wait_limit_ns, engram_stream_t stream);
 
 /* Read (and optionally clear) the status word of the current device.  Synchronises the
  * device.  *status receives the OR of ENGRAM_STATUS_* bits since the last clear. */

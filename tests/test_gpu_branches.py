@@ -10,7 +10,8 @@ import torch
 import hashed_gram_embedding_remap_b200 as E
 import oracle
 import synth
-from gpu_helpers import DeviceInputs, assert_delta_close, assert_out_close, host_tables, table_scales, to_dev, to_host_u16
+from gpu_helpers import (DeviceInputs, assert_bf16_within_ulp, assert_delta_close, assert_out_close, host_tables,
+                         table_scales, to_dev, to_host_u16)
 from helpers import small_workload
 
 pytestmark = pytest.mark.gpu
@@ -74,8 +75,7 @@ def test_branch_decode_steps_carry_per_branch_state(geom):
         assert_delta_close(di.delta.cpu().numpy().reshape(-1, M, wl.d_h), ref["delta"])
         assert_out_close(to_host_u16(di.out).reshape(-1, M, wl.d_h), ref["out"])
         assert np.array_equal(di.history.cpu().numpy(), ref["history"])
-        got_state = synth.bf16_to_float(to_host_u16(di.conv_state))
-        assert np.abs(got_state - synth.bf16_to_float(ref["state"])).max() <= 2.0 ** -5 + 1e-7
+        assert_bf16_within_ulp(to_host_u16(di.conv_state), ref["state"])
         hist, state = ref["history"], to_host_u16(di.conv_state)
 
 

@@ -6,8 +6,8 @@ some runtimes run under a fixed memory budget or cannot afford the device-wide
 synchronisation of cudaMalloc/cudaFree.  For them the library keeps the scratch of the
 projection + gate/conv step in a fixed per-GPU array inside its own device data.  This
 test calls that entry point through the C ABI twice in a row and checks each result
-against the workspace entry point, within the tolerance the parity tests use.  It lives in
-its own file so that pytest collects it last.
+against the workspace entry point and against the CPU oracle, within the tolerance the
+parity tests use.  It lives in its own file so that pytest collects it last.
 """
 from __future__ import annotations
 
@@ -19,8 +19,8 @@ import torch
 
 import hashed_gram_embedding_remap_b200 as E
 import oracle
-import synth
-from gpu_helpers import DeviceInputs, assert_delta_close, assert_out_close, to_dev, to_host_u16
+from gpu_helpers import (DeviceInputs, assert_bf16_within_ulp, assert_delta_close, assert_out_close, to_dev,
+                         to_host_u16)
 from helpers import small_workload
 
 pytestmark = pytest.mark.gpu
@@ -32,6 +32,15 @@ def _memory_vectors(wl, di):
     m = torch.empty((wl.n_tok, wl.d_m), dtype=torch.bfloat16, device="cuda")
     E.engram_gather(di.plan, to_dev(idx.view(np.int32)), di.tables, m)
     return m
+
+
+def _oracle(wl, di, m, state0):
+    """The oracle's steps 4-6 on the same memory vectors, hidden states and conv state."""
+    w = di.host_weights()
+    return oracle.gate_conv(to_host_u16(di.h), to_host_u16(m), w["Wk"], w["Wv"], w["gamma_q"], w["gamma_k"],
+                            w["gamma_c"], w["conv_w"], wl.B, wl.T, dil=wl.conv_dilation, eps=wl.eps,
+                            conv_state=None if state0 is None else to_host_u16(state0),
+                            want_state=state0 is not None)
 
 
 @pytest.mark.parametrize("case", ["prefill", "decode"])
@@ -51,6 +60,7 @@ def test_noalloc_matches_workspace_entry_two_calls(case):
                        delta_dbg=ref_delta)
     torch.cuda.synchronize()
     ref_o, ref_d = to_host_u16(ref_out), ref_delta.cpu().numpy()
+    orc = _oracle(wl, di, m, state0)
 
     for call in range(2):
         out = torch.full_like(di.out, 7.0)
@@ -61,9 +71,11 @@ def test_noalloc_matches_workspace_entry_two_calls(case):
         torch.cuda.synchronize()
         assert_delta_close(delta.cpu().numpy(), ref_d)
         assert_out_close(to_host_u16(out), ref_o)
+        assert_delta_close(delta.cpu().numpy(), orc["delta"])
+        assert_out_close(to_host_u16(out), orc["out"])
         if state is not None:
-            diff = np.abs(synth.bf16_to_float(to_host_u16(state)) - synth.bf16_to_float(to_host_u16(ref_state)))
-            assert diff.max() <= 2.0 ** -5
+            assert_bf16_within_ulp(to_host_u16(state), to_host_u16(ref_state))
+            assert_bf16_within_ulp(to_host_u16(state), orc["state"])
     assert E.engram_device_status(clear=True) == 0
 
 

@@ -360,10 +360,8 @@ def run_engram(args, wl, world, rank, local):
     cw = fill_gpu.filled((wl.d_h, wl.conv_kernel), wl.conv_spec(), dev)
     history = torch.from_numpy(wl.history()).to(dev) if wl.decode else None
     state = fill_gpu.filled((wl.B * M, wl.state_len, wl.d_h), wl.state_spec(), dev) if wl.decode else None
-    plan = E.Plan.from_workload(wl, flags=(E.ENGRAM_FLAG_SEPARATE_GATHER if args.separate_gather else 0)
-                                | (E.ENGRAM_FLAG_SINGLE_CTA_MMA if args.single_cta_mma else 0))
+    plan = E.Plan.from_workload(wl, flags=E.ENGRAM_FLAG_SINGLE_CTA_MMA if args.single_cta_mma else 0)
     path = E.engram_forward_path(plan, wl.B, wl.T)
-    gather_in_proj = bool(path & E.ENGRAM_PATH_GATHER_IN_PROJ)
     packed = E.pack_weights(plan, wk, wv) if args.packed and E.engram_packed_weights_size(plan) else None
     weights = E.Weights(wk, wv, one, one, one, cw, packed=packed)
     out = torch.empty((wl.h_rows, wl.d_h), dtype=torch.bfloat16, device=dev)
@@ -467,27 +465,9 @@ def run_engram(args, wl, world, rank, local):
     stage_names = ["hash", "gather", "proj", "gate_conv"]
     stage_ms = {n: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
                 for i, n in enumerate(stage_names)}
-    if gather_in_proj:   # the projection reads the rows itself: there is no gather stage
-        del stage_ms["gather"]
     status = E.engram_device_status(clear=True)
     if status:
         raise SystemExit(f"device status {status:#x} after the timed region")
-
-    # The separate gather kernel on the same row ids (what the path costs when m is
-    # materialised), timed alone for the HBM accounting below; not part of a step here.
-    sep_gather_ms = None
-    if gather_in_proj and not args.no_separate_gather_timing:
-        m_buf = torch.empty((wl.n_tok, wl.d_m), dtype=torch.bfloat16, device=dev)
-        E.engram_gather(plan, idx, tables, m_buf, stream=stream)
-        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 5
-        g0.record(stream)
-        for _ in range(reps):
-            E.engram_gather(plan, idx, tables, m_buf, stream=stream)
-        g1.record(stream)
-        torch.cuda.synchronize()
-        sep_gather_ms = g0.elapsed_time(g1) / reps
-        del m_buf
 
     # ---- e2e: inputs from pinned host memory, result back to pinned host memory.
     # Every step copies its ids and hidden states host->device and its output device->host.
@@ -597,8 +577,7 @@ def run_engram(args, wl, world, rank, local):
     pair = bool(path & E.ENGRAM_PATH_PAIR_MMA)
     roofline = {"bound": "tensor",
                 "kernel": ("proj_pair_kernel (cta_group::2 " if pair else "proj_kernel (")
-                          + "tcgen05 k/v projections + gate partials"
-                          + (", rows gathered into its A tiles)" if gather_in_proj else ")"),
+                          + "tcgen05 k/v projections + gate partials)",
                 "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s", "frac": tflops / peak_tf,
                 "frac_of_sustained": tflops / peaks["bf16_sus"],
                 "traffic": kernel_traffic("proj_kernel", wl.name),
@@ -618,28 +597,20 @@ def run_engram(args, wl, world, rank, local):
            "algorithmic_bytes_distinct_rows": alg_distinct, "algorithmic_bytes_token_rows": alg_tokrows,
            "gate_conv_GBps": gate_bytes / (stage_ms["gate_conv"] / 1e3) / 1e9}
     hbm["gate_conv_frac"] = hbm["gate_conv_GBps"] / peaks["hbm"]
-    path_ms = stage_ms["hash"] + stage_ms.get("gather", 0.0) + stage_ms["gate_conv"]
+    gather_bytes = n_tok * (wl.H * row_b + wl.d_m * 2 + wl.H * 4)   # rows read + m written + row ids
+    hbm["gather_GBps"] = gather_bytes / (max(1e-6, stage_ms["gather"]) / 1e3) / 1e9
+    hbm["gather_frac"] = hbm["gather_GBps"] / peaks["hbm"]
+    # the path outside the projection: hash + gather + gate/conv, over the method's bytes (every
+    # distinct row once, h, out, ids), and beside that with every token's rows
+    path_ms = stage_ms["hash"] + stage_ms["gather"] + stage_ms["gate_conv"]
     hbm["path_ms"] = path_ms
     hbm["path_frac"] = alg_distinct / (path_ms / 1e3) / 1e9 / peaks["hbm"]
     hbm["path_frac_token_rows"] = alg_tokrows / (path_ms / 1e3) / 1e9 / peaks["hbm"]
     hbm["path_frac_nominal"] = alg_distinct / (path_ms / 1e3) / 1e9 / hbm["nominal_GBps"]
-    if gather_in_proj:
-        hbm["path_note"] = ("path_ms = hash + gate_conv: the rows are read by the projection kernel's "
-                            "gather warps, overlapped with its tensor-core work, so no stage of its own "
-                            "remains for them")
-        if sep_gather_ms is not None:
-            # the same bytes over the stages with the separate gather kernel in the path
-            sep_ms = path_ms + sep_gather_ms
-            hbm["separate_gather_ms"] = sep_gather_ms
-            hbm["path_frac_with_separate_gather"] = alg_distinct / (sep_ms / 1e3) / 1e9 / peaks["hbm"]
-    else:
-        gather_bytes = n_tok * (wl.H * row_b + wl.d_m * 2 + wl.H * 4)   # rows read + m written + row ids
-        hbm["gather_GBps"] = gather_bytes / (stage_ms["gather"] / 1e3) / 1e9
-        hbm["gather_frac"] = hbm["gather_GBps"] / peaks["hbm"]
-    # bytes the path's own kernels move, intermediates included (m written and read back
-    # when materialised, v written by the projection and read by the gate kernel)
-    moved = gate_bytes + (0 if gather_in_proj else n_tok * (wl.H * row_b + wl.d_m * 2 + wl.H * 4))
-    hbm["incl_intermediates_GBps"] = moved / (path_ms / 1e3) / 1e9
+    # bytes these kernels move, their intermediates included (m written by the gather and read
+    # back by the projection, v written by the projection and read by the gate kernel)
+    hbm["incl_intermediates_GBps"] = (gather_bytes + gate_bytes) / (path_ms / 1e3) / 1e9
+    hbm["incl_intermediates_frac"] = hbm["incl_intermediates_GBps"] / peaks["hbm"]
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -663,8 +634,7 @@ def run_engram(args, wl, world, rank, local):
         "data": "synthetic (seeded Zipf ids, counter-based bf16 tables/weights)",
         "config": workload_config(wl, world),
         "weights_layout": "packed" if packed is not None else "row-major",
-        "path": {"gather_in_projection": gather_in_proj, "pair_mma": bool(path & E.ENGRAM_PATH_PAIR_MMA),
-                 "path_bits": path},
+        "path": {"pair_mma": bool(path & E.ENGRAM_PATH_PAIR_MMA), "path_bits": path},
         "stages_ms": stage_ms, "hbm": hbm, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * launches_per_step,
         "launch_mode": "eager" if args.eager else "one CUDA graph of the K timed steps (stage times from a "
@@ -758,12 +728,13 @@ def run_hostpinned(args, wl, world, rank, local):
         with torch.cuda.stream(side):
             if evs is not None:
                 evs[0].record(side)
-            E.engram_hash(plan, x, idx, history=history, stream=side)
             if cache is not None:
+                E.engram_hash(plan, x, idx, history=history, stream=side)
                 E.engram_stage_rows_cached(plan, idx, tables, cache, staging, sidx, uniq, nu, row_flags, n_hits,
                                            stream=side)
-            else:
-                E.engram_stage_rows(plan, idx, tables, staging, sidx, uniq, nu, stream=side)
+            else:   # hash + in-batch dedup + host-link copy (one kernel for a decode step)
+                E.engram_stage_rows_from_ids(plan, x, tables, staging, idx, sidx, uniq, nu, history=history,
+                                             stream=side)
             if evs is not None:
                 evs[1].record(side)
         torch.matmul(ga, gb, out=gc_)              # stand-in for the layers before the lookup
@@ -888,7 +859,8 @@ def run_hostpinned(args, wl, world, rank, local):
         "steps": K, "warmup": args.warmup, "ms_per_step": ovl_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": f"synthetic; ids {kind}",
         "config": workload_config(wl, world, ids_kind=kind),
-        "step_includes": "hash + distinct-row staging from host (side stream) || 2560^3 bf16 GEMM stand-in; "
+        "step_includes": "hash + distinct-row staging from host (side stream; one kernel without a row cache) "
+                         "|| 2560^3 bf16 GEMM stand-in; "
                          "then gather + projections + gate/conv + history update",
         "host_link": {"bound": "host-link", "staged_rows_per_step": int(nu_h.sum()),
                       "staged_bytes_per_step": uniq_bytes, "prefetch_ms": prefetch_ms,
@@ -914,12 +886,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["engram", "reference"], default="engram")
     ap.add_argument("--workload", default="prefill20m", choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--separate-gather", action="store_true",
-                    help="materialise m with the separate gather kernel (ENGRAM_FLAG_SEPARATE_GATHER)")
     ap.add_argument("--single-cta-mma", action="store_true",
                     help="never pair CTAs for the projection's MMAs (ENGRAM_FLAG_SINGLE_CTA_MMA)")
-    ap.add_argument("--no-separate-gather-timing", action="store_true",
-                    help="skip timing the separate gather kernel beside the row-gathering projection")
     ap.add_argument("--oracle-tokens", type=int, default=128)
     ap.add_argument("--cpu-baseline-tokens", type=int, default=768)
     ap.add_argument("--oracle-procs", type=int, default=0,

@@ -30,11 +30,9 @@ ENGRAM_FORWARD_STAGES = 4
 ENGRAM_TABLES_DEVICE = 0
 ENGRAM_TABLES_HOST_MAPPED = 1
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
-ENGRAM_FLAG_SEPARATE_GATHER = 0x2
 ENGRAM_FLAG_SINGLE_CTA_MMA = 0x4
 ENGRAM_PATH_FUSED_LOOKUP = 0x1
 ENGRAM_PATH_STAGED_ROWS = 0x2
-ENGRAM_PATH_GATHER_IN_PROJ = 0x4
 ENGRAM_PATH_SPLIT_K = 0x8
 ENGRAM_PATH_PAIR_MMA = 0x10
 ENGRAM_TABLE_BF16 = 0
@@ -115,6 +113,7 @@ def _load():
         "engram_advance_history": (C.c_int, [P, P, i32, i32, P, P]),
         "engram_gather": (C.c_int, [P, P, P, i64, P, P]),
         "engram_stage_rows": (C.c_int, [P, P, i64, P, P, i32, P, P, P, P]),
+        "engram_stage_rows_from_ids": (C.c_int, [P, P, P, i32, i32, P, P, P, i32, P, P, P, P, P]),
         "engram_gather_bounded": (C.c_int, [P, P, P, i64, i64, P, P]),
         "engram_row_cache_reset": (C.c_int, [P, P, P]),
         "engram_packed_weights_size": (sz, [P]),
@@ -349,6 +348,23 @@ def engram_stage_rows(plan: Plan, idx: torch.Tensor, tables, staging, staged_idx
                                  _ptr(staged_idx, (torch.int32, torch.uint32), "staged_idx"),
                                  _ptr(unique_rows, (torch.int32, torch.uint32), "unique_rows"),
                                  _ptr(n_unique, torch.int32, "n_unique"), _stream(stream)))
+
+
+def engram_stage_rows_from_ids(plan: Plan, ids: torch.Tensor, tables, staging, idx: torch.Tensor,
+                               staged_idx: torch.Tensor, unique_rows: torch.Tensor, n_unique: torch.Tensor,
+                               remap: Optional[torch.Tensor] = None, history: Optional[torch.Tensor] = None,
+                               stream=None):
+    """Hash the ids (into idx) and stage the batch's distinct rows from the (host-mapped)
+    tables, in one kernel for decode-sized batches."""
+    B, T = ids.shape
+    cap = staging[0].shape[0]
+    _check(lib.engram_stage_rows_from_ids(plan, _ptr(ids, torch.int32, "ids"), _ptr(remap, torch.int32, "remap"),
+                                          B, T, _ptr(history, torch.int32, "history"), _table_array(tables, plan),
+                                          _table_array(staging, plan), cap,
+                                          _ptr(idx, (torch.int32, torch.uint32), "idx"),
+                                          _ptr(staged_idx, (torch.int32, torch.uint32), "staged_idx"),
+                                          _ptr(unique_rows, (torch.int32, torch.uint32), "unique_rows"),
+                                          _ptr(n_unique, torch.int32, "n_unique"), _stream(stream)))
 
 
 def _check_rows(plan: Plan, n_tok: int, **tensors):

@@ -229,7 +229,6 @@ bool use_pair_mma(const engram_plan *plan, int64_t n_tok, const ProjShape &ps) {
 struct ForwardPath {
     bool fused_lookup;    // remap + hash + gather in one kernel (decode-sized, HBM tables)
     bool staged;          // host-mapped tables: the batch's distinct rows are staged into HBM
-    bool gather_in_proj;  // the projection gathers the rows into its A tiles (m never written)
     bool pair;            // the projection's MMAs span CTA pairs
     ProjShape ps;
 };
@@ -240,9 +239,6 @@ ForwardPath forward_path(const engram_plan *plan, int64_t n_tok) {
     f.staged = plan->cfg.table_location == ENGRAM_TABLES_HOST_MAPPED && n_tok <= engram::kStageMaxTok;
     f.fused_lookup = !f.staged && plan->cfg.table_location == ENGRAM_TABLES_DEVICE &&
                      n_tok * plan->num_tables <= kFusedLookupMaxRows;
-    f.gather_in_proj = !f.fused_lookup && !f.staged && plan->cfg.table_location == ENGRAM_TABLES_DEVICE &&
-                       plan->cfg.table_dtype == ENGRAM_TABLE_BF16 && f.ps.k_splits == 1 &&
-                       !(plan->cfg.flags & ENGRAM_FLAG_SEPARATE_GATHER);
     f.pair = use_pair_mma(plan, n_tok, f.ps);
     return f;
 }
@@ -256,8 +252,7 @@ Workspace layout(const engram_plan *plan, int64_t n_tok) {
     size_t off = 0;
     w.xr = off;   off = align256(off + sizeof(int32_t) * n_tok);
     w.idx = off;  off = align256(off + sizeof(uint32_t) * n_tok * H);
-    w.m = off;    // m is only materialised when the projection does not gather the rows itself
-    if (!forward_path(plan, n_tok).gather_in_proj) off = align256(off + sizeof(uint16_t) * n_tok * plan->mem_dim);
+    w.m = off;    off = align256(off + sizeof(uint16_t) * n_tok * plan->mem_dim);
     const size_t v_bytes = sizeof(uint16_t) * n_tok * d_h;
     w.v = off;    off = align256(off + v_bytes);
     w.part = off; off = align256(off + sizeof(float4) * n_tok * n_tiles);
@@ -317,26 +312,19 @@ int sm_count() {
     return n;
 }
 
-template <int BN, bool SPLIT, bool GATHER>
+template <int BN, bool SPLIT>
 int set_proj_smem_attr() {
     // Per device: the attribute is a property of the function on the current device.
     static bool done[64] = {};
     int dev = 0;
     ENGRAM_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
     if (dev < 64 && done[dev]) return ENGRAM_OK;
-    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::proj_kernel<BN, SPLIT, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::proj_kernel<BN, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          engram::ProjCfg<BN>::kSmemBytes),
                     "cudaFuncSetAttribute(proj_kernel)");
     if (dev < 64) done[dev] = true;
     return ENGRAM_OK;
 }
-
-// Where the projection's A tiles come from when m is not materialised: the row ids of step 2
-// and the (bf16, HBM-resident) tables.
-struct GatherSrc {
-    const uint32_t *idx;          // [n_tok, H]
-    const void *const *tables;    // host array of H device pointers
-};
 
 // Test hooks of the projection: a shorter bound on every pipeline wait, and a stalled
 // pipeline (no loads issued) that makes the first wait run out.
@@ -349,23 +337,16 @@ template <int BN>
 int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                 int64_t n_tok, uint16_t *v, float4 *part, cudaStream_t stream, float *acc = nullptr,
                 int k_splits = 1, int kb_per_split = 0, bool run_reduce = true,
-                engram::ProjParams *params_out = nullptr, const GatherSrc *gs = nullptr,
-                const ProjTest &test = ProjTest()) {
+                engram::ProjParams *params_out = nullptr, const ProjTest &test = ProjTest()) {
     const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim;
     CUtensorMap map_m, map_wk, map_wv;
     int rc;
     const int M = plan->num_branches;
     if ((rc = make_map_bf16(&map_wk, w->w_k, static_cast<uint64_t>(M) * d_h, d_m, BN)) != ENGRAM_OK) return rc;
     if ((rc = make_map_bf16(&map_wv, w->w_v, d_h, d_m, BN)) != ENGRAM_OK) return rc;
-    if (gs != nullptr)
-        map_m = map_wk;   // unused: the A tiles are gathered from the tables
-    else if ((rc = make_map_bf16(&map_m, m, static_cast<uint64_t>(n_tok), d_m, engram::kBM)) != ENGRAM_OK)
-        return rc;
+    if ((rc = make_map_bf16(&map_m, m, static_cast<uint64_t>(n_tok), d_m, engram::kBM)) != ENGRAM_OK) return rc;
     const bool split = acc != nullptr && k_splits > 1;
-    if (split && gs != nullptr) return fail(ENGRAM_ERR_UNSUPPORTED, "row gather with a split-K projection");
-    if ((rc = split ? set_proj_smem_attr<BN, true, false>()
-                    : gs ? set_proj_smem_attr<BN, false, true>() : set_proj_smem_attr<BN, false, false>()) != ENGRAM_OK)
-        return rc;
+    if ((rc = split ? set_proj_smem_attr<BN, true>() : set_proj_smem_attr<BN, false>()) != ENGRAM_OK) return rc;
     engram::ProjParams p{};
     p.h = h;
     p.gamma_q = w->gamma_q;
@@ -383,25 +364,14 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     p.kb_per_split = p.k_splits > 1 ? kb_per_split : p.k_blocks;
     p.acc_out = p.k_splits > 1 ? acc : nullptr;
     p.w_packed = BN == 256 ? static_cast<const uint8_t *>(w->w_packed) : nullptr;
-    if (gs != nullptr) {
-        p.idx = gs->idx;
-        p.H = plan->num_tables;
-        p.d_e = plan->cfg.row_dim;
-        for (int t = 0; t < p.H; ++t) {
-            p.tab[t] = static_cast<const uint16_t *>(gs->tables[t]);
-            p.tab_rows[t] = static_cast<uint32_t>(plan->cfg.table_rows[t]);
-        }
-    }
     p.wait_limit_ns = test.wait_limit_ns;
     p.stall = test.stall;
     const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles * p.k_splits;
     if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
     const int64_t sms = sm_count();
     dim3 grid(static_cast<unsigned>(total < sms ? total : sms));
-    auto kernel = split ? engram::proj_kernel<BN, true, false>
-                        : gs ? engram::proj_kernel<BN, false, true> : engram::proj_kernel<BN, false, false>;
-    const int threads = engram::kProjThreads + (gs ? engram::kGatherThreads : 0);
-    ENGRAM_CUDA_TRY(launch_pdl(kernel, grid, dim3(threads), engram::ProjCfg<BN>::kSmemBytes, stream, map_m, map_wk,
+    ENGRAM_CUDA_TRY(launch_pdl(split ? engram::proj_kernel<BN, true> : engram::proj_kernel<BN, false>, grid,
+                               dim3(engram::kProjThreads), engram::ProjCfg<BN>::kSmemBytes, stream, map_m, map_wk,
                                map_wv, p),
                     "proj_kernel launch");
     if (params_out) *params_out = p;
@@ -413,13 +383,12 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     return ENGRAM_OK;
 }
 
-template <bool GATHER>
 int set_pair_smem_attr() {
     static bool done[64] = {};
     int dev = 0;
     ENGRAM_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
     if (dev < 64 && done[dev]) return ENGRAM_OK;
-    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::proj_pair_kernel<GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::proj_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          engram::PairCfg::kSmemBytes),
                     "cudaFuncSetAttribute(proj_pair_kernel)");
     if (dev < 64) done[dev] = true;
@@ -427,7 +396,6 @@ int set_pair_smem_attr() {
 }
 
 // CTA pairs that can be resident at once (one CTA per SM; a pair needs two SMs of one GPC).
-template <bool GATHER>
 int max_pairs(int *out) {
     static int cached[64] = {};
     int dev = 0;
@@ -438,10 +406,10 @@ int max_pairs(int *out) {
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 74);
-    cfg.blockDim = dim3(engram::kProjThreads + (GATHER ? engram::kGatherThreads : 0));
+    cfg.blockDim = dim3(engram::kProjThreads);
     cfg.dynamicSmemBytes = engram::PairCfg::kSmemBytes;
     int n = 0;
-    ENGRAM_CUDA_TRY(cudaOccupancyMaxActiveClusters(&n, engram::proj_pair_kernel<GATHER>, &cfg),
+    ENGRAM_CUDA_TRY(cudaOccupancyMaxActiveClusters(&n, engram::proj_pair_kernel, &cfg),
                     "cudaOccupancyMaxActiveClusters(proj_pair_kernel)");
     if (n < 1) return fail(ENGRAM_ERR_CUDA, "no CTA pair of the projection fits on this device");
     if (dev < 64) cached[dev] = n;
@@ -451,20 +419,35 @@ int max_pairs(int *out) {
 
 // Whole-K projection on CTA pairs: 256-token x 256-channel units (see kernels_proj_pair.cuh).
 int launch_proj_pair(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
-                     int64_t n_tok, uint16_t *v, float4 *part, cudaStream_t stream, const GatherSrc *gs) {
+                     int64_t n_tok, uint16_t *v, float4 *part, cudaStream_t stream) {
     const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim, M = plan->num_branches;
     constexpr int BN = engram::kPairBN;
     CUtensorMap map_m, map_wk, map_wv;
     int rc;
-    if ((rc = make_map_bf16(&map_wk, w->w_k, static_cast<uint64_t>(M) * d_h, d_m, BN / 2)) != ENGRAM_OK) return rc;
-    if ((rc = make_map_bf16(&map_wv, w->w_v, d_h, d_m, BN / 2)) != ENGRAM_OK) return rc;
-    if (gs != nullptr)
-        map_m = map_wk;   // unused: the A tiles are gathered from the tables
-    else if ((rc = make_map_bf16(&map_m, m, static_cast<uint64_t>(n_tok), d_m, engram::kBM)) != ENGRAM_OK)
-        return rc;
-    if ((rc = gs ? set_pair_smem_attr<true>() : set_pair_smem_attr<false>()) != ENGRAM_OK) return rc;
+    if (w->w_packed != nullptr) {
+        // the packed tiles as rows of 64 columns, already in the tensor cores' layout: boxes of
+        // 128 rows copied as they are (no swizzle)
+        auto enc = get_encode_fn();
+        if (enc == nullptr) return fail(ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+        const uint64_t k_blocks = (d_m + engram::kBK - 1) / engram::kBK;
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(engram::kBK),
+                              static_cast<cuuint64_t>((M + 1) * d_h / BN) * k_blocks * BN};
+        cuuint64_t strides[1] = {engram::kBK * 2};
+        cuuint32_t box[2] = {static_cast<cuuint32_t>(engram::kBK), BN / 2};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(&map_wk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(w->w_packed), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(ENGRAM_ERR_CUDA, "cuTensorMapEncodeTiled(packed weights) failed (%d)", static_cast<int>(r));
+        map_wv = map_wk;
+    } else {
+        if ((rc = make_map_bf16(&map_wk, w->w_k, static_cast<uint64_t>(M) * d_h, d_m, BN / 2)) != ENGRAM_OK) return rc;
+        if ((rc = make_map_bf16(&map_wv, w->w_v, d_h, d_m, BN / 2)) != ENGRAM_OK) return rc;
+    }
+    if ((rc = make_map_bf16(&map_m, m, static_cast<uint64_t>(n_tok), d_m, engram::kBM)) != ENGRAM_OK) return rc;
+    if ((rc = set_pair_smem_attr()) != ENGRAM_OK) return rc;
     int pairs = 0;
-    if ((rc = gs ? max_pairs<true>(&pairs) : max_pairs<false>(&pairs)) != ENGRAM_OK) return rc;
+    if ((rc = max_pairs(&pairs)) != ENGRAM_OK) return rc;
     engram::ProjParams p{};
     p.h = h;
     p.gamma_q = w->gamma_q;
@@ -481,15 +464,6 @@ int launch_proj_pair(const engram_plan *plan, const engram_weights *w, const uin
     p.k_splits = 1;
     p.kb_per_split = p.k_blocks;
     p.w_packed = static_cast<const uint8_t *>(w->w_packed);
-    if (gs != nullptr) {
-        p.idx = gs->idx;
-        p.H = plan->num_tables;
-        p.d_e = plan->cfg.row_dim;
-        for (int t = 0; t < p.H; ++t) {
-            p.tab[t] = static_cast<const uint16_t *>(gs->tables[t]);
-            p.tab_rows[t] = static_cast<uint32_t>(plan->cfg.table_rows[t]);
-        }
-    }
     const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
     if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
     // ENGRAM_PROJ_PAIRS (>= 1) caps the number of CTA pairs (tuning); read once per process.
@@ -500,10 +474,8 @@ int launch_proj_pair(const engram_plan *plan, const engram_weights *w, const uin
     }();
     if (forced_pairs && forced_pairs < pairs) pairs = forced_pairs;
     const int64_t npairs = total < pairs ? total : pairs;
-    auto kernel = gs ? engram::proj_pair_kernel<true> : engram::proj_pair_kernel<false>;
-    const int threads = engram::kProjThreads + (gs ? engram::kGatherThreads : 0);
-    ENGRAM_CUDA_TRY(launch_pdl(kernel, dim3(static_cast<unsigned>(2 * npairs)), dim3(threads),
-                               engram::PairCfg::kSmemBytes, stream, map_m, map_wk, map_wv, p),
+    ENGRAM_CUDA_TRY(launch_pdl(engram::proj_pair_kernel, dim3(static_cast<unsigned>(2 * npairs)),
+                               dim3(engram::kProjThreads), engram::PairCfg::kSmemBytes, stream, map_m, map_wk, map_wv, p),
                     "proj_pair_kernel launch");
     return ENGRAM_OK;
 }
@@ -814,6 +786,35 @@ int launch_stage(const engram_plan *plan, const uint32_t *idx, int64_t n_tok, co
     return ENGRAM_OK;
 }
 
+// Remap + hash + dedup + copy of host-table rows in one kernel (batches of at most
+// kStageSmallRows (token, table) rows); xr: remapped ids out, or NULL.
+int launch_stage_small(const engram_plan *plan, const int32_t *ids, const int32_t *remap, const int32_t *history,
+                       int32_t B, int32_t T, const void *const *tables, void *const *staging, int32_t capacity,
+                       uint32_t *idx, int32_t *xr, uint32_t *staged_idx, uint32_t *unique_rows, int32_t *n_unique,
+                       cudaStream_t stream) {
+    const int H = plan->num_tables;
+    const engram::HashParams hp = make_hash_params(plan, B, T);
+    engram::StageParams sp{};
+    for (int h = 0; h < H; ++h) {
+        sp.table[h] = tables[h];
+        sp.staging[h] = staging[h];
+        sp.rows[h] = static_cast<uint64_t>(plan->cfg.table_rows[h]);
+    }
+    sp.H = H;
+    sp.capacity = capacity;
+    sp.chunks_per_row = plan->cfg.row_dim * table_elem_bytes(plan) / 16;
+    const int64_t total = static_cast<int64_t>(H) * B * T * sp.chunks_per_row;
+    constexpr int kUnroll = 2;
+    int64_t blocks = (total + engram::kStageSmallThreads * kUnroll - 1) / (engram::kStageSmallThreads * kUnroll);
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 2;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    engram::stage_small_kernel<kUnroll><<<static_cast<unsigned>(blocks), engram::kStageSmallThreads, 0, stream>>>(
+        ids, remap, history, idx, xr, staged_idx, unique_rows, n_unique, hp, sp);
+    ENGRAM_LAUNCHED("stage_small_kernel launch");
+    return ENGRAM_OK;
+}
+
 int check_row_cache(const engram_plan *plan, const engram_row_cache *cache) {
     if (cache == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "cache is NULL");
     if (cache->slots < 1 || cache->slots > (int64_t(1) << 32) || (cache->slots & (cache->slots - 1)))
@@ -839,11 +840,10 @@ cudaError_t record_stage_event(void *ev, cudaStream_t stream) {
 
 // history / xr (engram_forward's decode steps): when the step ends in decode_fused_kernel, that
 // kernel also advances the hash history and *history_done is set; otherwise the caller does.
-// gs: the projection gathers its A tiles from the tables (m unused; whole-K tiles only).
 int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                    int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out, float *delta, uint8_t *ws,
                    cudaStream_t stream, void *const *events, int32_t *history = nullptr,
-                   const int32_t *xr = nullptr, bool *history_done = nullptr, const GatherSrc *gs = nullptr) {
+                   const int32_t *xr = nullptr, bool *history_done = nullptr) {
     if (history_done) *history_done = false;
     const int64_t n_tok = static_cast<int64_t>(B) * T;
     const Workspace L = layout(plan, n_tok);
@@ -861,13 +861,13 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
     const bool pair = use_pair_mma(plan, n_tok, ps);
     const int n_tiles = pair ? (plan->num_branches + 1) * d_h / engram::kPairBN : ps.n_tiles;
     if (pair)
-        rc = launch_proj_pair(plan, w, h, m, n_tok, v, part, stream, gs);
+        rc = launch_proj_pair(plan, w, h, m, n_tok, v, part, stream);
     else if (ps.bn == 256)
-        rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp, gs);
+        rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
     else if (ps.bn == 128)
-        rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp, gs);
+        rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
     else
-        rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp, gs);
+        rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
     if (rc != ENGRAM_OK) return rc;
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[1], stream), "cudaEventRecord");
     if (fused_decode) {
@@ -990,7 +990,7 @@ int engram_init(const engram_config *cfg, engram_plan *plan) {
     }
     if (c.table_dtype == ENGRAM_TABLE_FP8_E4M3 && c.row_dim % 16 != 0)
         return fail(ENGRAM_ERR_UNSUPPORTED, "FP8 tables need row_dim % 16 == 0");
-    if (c.flags & ~(ENGRAM_FLAG_SEPARATE_GATHER | ENGRAM_FLAG_SINGLE_CTA_MMA)) return fail(ENGRAM_ERR_INVALID_ARG, "unknown flags 0x%x", c.flags);
+    if (c.flags & ~ENGRAM_FLAG_SINGLE_CTA_MMA) return fail(ENGRAM_ERR_INVALID_ARG, "unknown flags 0x%x", c.flags);
 
     std::memset(plan, 0, sizeof *plan);
     plan->cfg = c;
@@ -1103,6 +1103,34 @@ int engram_stage_rows(const engram_plan *plan, const uint32_t *idx, int64_t n_to
     }
     return launch_stage(plan, idx, n_tok, tables, staging, capacity, staged_idx, unique_rows, n_unique,
                         static_cast<cudaStream_t>(stream));
+}
+
+int engram_stage_rows_from_ids(const engram_plan *plan, const int32_t *ids, const int32_t *remap, int32_t B,
+                               int32_t T, const int32_t *history, const void *const *tables, void *const *staging,
+                               int32_t capacity, uint32_t *idx, uint32_t *staged_idx, uint32_t *unique_rows,
+                               int32_t *n_unique, engram_stream_t stream_) {
+    int rc;
+    if ((rc = check_plan(plan)) != ENGRAM_OK) return rc;
+    if ((rc = check_bt(B, T)) != ENGRAM_OK) return rc;
+    const int64_t n_tok = static_cast<int64_t>(B) * T;
+    if (n_tok == 0) return ENGRAM_OK;
+    if (n_tok > engram::kStageMaxTok)
+        return fail(ENGRAM_ERR_UNSUPPORTED, "engram_stage_rows_from_ids handles at most %d tokens per call",
+                    engram::kStageMaxTok);
+    if (capacity < n_tok) return fail(ENGRAM_ERR_INVALID_ARG, "capacity %d < n_tok %lld", capacity, (long long)n_tok);
+    if (!ids || !idx || !tables || !staging || !staged_idx || !unique_rows || !n_unique)
+        return fail(ENGRAM_ERR_INVALID_ARG, "NULL argument");
+    for (int h = 0; h < plan->num_tables; ++h) {
+        if (!tables[h] || !staging[h]) return fail(ENGRAM_ERR_INVALID_ARG, "tables[%d] or staging[%d] is NULL", h, h);
+        if (!aligned16(tables[h]) || !aligned16(staging[h]))
+            return fail(ENGRAM_ERR_INVALID_ARG, "tables[%d] / staging[%d] not 16-byte aligned", h, h);
+    }
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (n_tok * plan->num_tables <= engram::kStageSmallRows)
+        return launch_stage_small(plan, ids, remap, history, B, T, tables, staging, capacity, idx, nullptr,
+                                  staged_idx, unique_rows, n_unique, stream);
+    if ((rc = launch_hash(plan, ids, remap, history, B, T, idx, nullptr, stream)) != ENGRAM_OK) return rc;
+    return launch_stage(plan, idx, n_tok, tables, staging, capacity, staged_idx, unique_rows, n_unique, stream);
 }
 
 size_t engram_packed_weights_size(const engram_plan *plan) {
@@ -1221,14 +1249,25 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const void 
         return ENGRAM_OK;
     };
     // Decode-sized batches on HBM-resident tables: remap + hash + gather in one kernel (the
-    // row ids stay in registers).  Larger batches: the hash kernel, then either the
-    // projection gathers the rows into its tiles itself, or the wide gather writes m.
+    // row ids stay in registers).  Larger batches: the hash kernel, then the wide gather.
     const ForwardPath fp = forward_path(plan, n_tok);
     const bool fused_lookup = fp.fused_lookup;
     if ((rc = rec(0)) != ENGRAM_OK) return rc;
+    const bool stage_small = L.staged && n_tok * plan->num_tables <= engram::kStageSmallRows;
     if (fused_lookup) {
         if ((rc = rec(1)) != ENGRAM_OK) return rc;
         if ((rc = launch_lookup(plan, ids, remap, history, B, T, tables, xr, m, stream)) != ENGRAM_OK) return rc;
+    } else if (stage_small) {
+        // host-resident tables, decode-sized batch: hash + dedup + staging copy in one kernel
+        const int64_t stage_bytes = n_tok * plan->cfg.row_dim * table_elem_bytes(plan);   // per table
+        void *stage_ptr[ENGRAM_MAX_TABLES];
+        for (int hh = 0; hh < plan->num_tables; ++hh) stage_ptr[hh] = ws + L.staging + static_cast<int64_t>(hh) * stage_bytes;
+        if ((rc = launch_stage_small(plan, ids, remap, history, B, T, tables, stage_ptr, static_cast<int32_t>(n_tok),
+                                     idx, xr, reinterpret_cast<uint32_t *>(ws + L.staged_idx),
+                                     reinterpret_cast<uint32_t *>(ws + L.unique),
+                                     reinterpret_cast<int32_t *>(ws + L.n_unique), stream)) != ENGRAM_OK)
+            return rc;
+        if ((rc = rec(1)) != ENGRAM_OK) return rc;
     } else {
         if ((rc = launch_hash(plan, ids, remap, history, B, T, idx, xr, stream)) != ENGRAM_OK) return rc;
         if ((rc = rec(1)) != ENGRAM_OK) return rc;
@@ -1243,19 +1282,18 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const void 
         const int64_t stage_bytes = n_tok * plan->cfg.row_dim * table_elem_bytes(plan);   // per table
         for (int h = 0; h < H; ++h) stage_ptr[h] = ws + L.staging + static_cast<int64_t>(h) * stage_bytes;
         uint32_t *sidx = reinterpret_cast<uint32_t *>(ws + L.staged_idx);
-        if ((rc = launch_stage(plan, idx, n_tok, tables, stage_ptr, static_cast<int32_t>(n_tok), sidx,
+        if (!stage_small &&
+            (rc = launch_stage(plan, idx, n_tok, tables, stage_ptr, static_cast<int32_t>(n_tok), sidx,
                                reinterpret_cast<uint32_t *>(ws + L.unique), reinterpret_cast<int32_t *>(ws + L.n_unique),
                                stream)) != ENGRAM_OK)
             return rc;
         if ((rc = launch_gather(plan, sidx, stage_ptr, n_tok, m, stream, n_tok)) != ENGRAM_OK) return rc;
-    } else if (!fp.gather_in_proj && (rc = launch_gather(plan, idx, tables, n_tok, m, stream)) != ENGRAM_OK) {
+    } else if ((rc = launch_gather(plan, idx, tables, n_tok, m, stream)) != ENGRAM_OK) {
         return rc;
     }
     bool history_done = false;
-    const GatherSrc gsrc{idx, tables};
-    if ((rc = gate_conv_impl(plan, w, h, fp.gather_in_proj ? nullptr : m, B, T, conv_state, out, delta_dbg, ws,
-                             stream, stage_events ? stage_events + 2 : nullptr, history, xr, &history_done,
-                             fp.gather_in_proj ? &gsrc : nullptr)) != ENGRAM_OK)
+    if ((rc = gate_conv_impl(plan, w, h, m, B, T, conv_state, out, delta_dbg, ws, stream,
+                             stage_events ? stage_events + 2 : nullptr, history, xr, &history_done)) != ENGRAM_OK)
         return rc;
     if ((rc = rec(4)) != ENGRAM_OK) return rc;
     if (history != nullptr && plan->hist_len > 0 && !history_done) {
@@ -1311,7 +1349,6 @@ int engram_forward_path(const engram_plan *plan, int32_t B, int32_t T, uint32_t 
     uint32_t bits = 0;
     if (fp.fused_lookup) bits |= ENGRAM_PATH_FUSED_LOOKUP;
     if (fp.staged) bits |= ENGRAM_PATH_STAGED_ROWS;
-    if (fp.gather_in_proj) bits |= ENGRAM_PATH_GATHER_IN_PROJ;
     if (fp.ps.k_splits > 1) bits |= ENGRAM_PATH_SPLIT_K;
     if (fp.pair) bits |= ENGRAM_PATH_PAIR_MMA;
     *path = bits;
@@ -1348,7 +1385,7 @@ int engram_selftest_wait_timeout(const engram_plan *plan, const engram_weights *
     test.wait_limit_ns = wait_limit_ns;
     test.stall = 1;
     return launch_proj<64>(plan, w, h, m, n_tok, v, part, static_cast<cudaStream_t>(stream), nullptr, 1, 0, false,
-                           nullptr, nullptr, test);
+                           nullptr, test);
 }
 
 uint64_t engram_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }

@@ -47,19 +47,12 @@ __device__ __forceinline__ uint32_t mod_prime(uint64_t s, uint64_t P, uint64_t M
     return static_cast<uint32_t>(r);
 }
 
-// One thread per token.  Reads the token and the (max_order - 1) before it (remapping each
-// through `remap` when given), then for every table h forms the gram of its order and writes
-// idx[n, h] = fmix64(XOR_i (x'_{t-i} + 1) * a_{h,i}) mod P_h.
-// Token ids outside [0, vocab_in) read as the pad id and raise ENGRAM_STATUS_BAD_TOKEN.
-__global__ void __launch_bounds__(256) hash_kernel(const int32_t *__restrict__ ids,
-                                                   const int32_t *__restrict__ remap,
-                                                   const int32_t *__restrict__ history,
-                                                   uint32_t *__restrict__ idx,
-                                                   int32_t *__restrict__ xr_out,
-                                                   const __grid_constant__ HashParams p) {
-    const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t n_tok = static_cast<int64_t>(p.B) * p.T;
-    if (n >= n_tok) return;
+// The row ids of token n for every table: row[h] = fmix64(XOR_i (x'_{t-i} + 1) * a_{h,i}) mod
+// P_h, reading the token and the (max_order - 1) before it (through `remap` when given; the
+// history, then the pad id, before the sequence start).  xr_out[n] = x'_t when given.
+__device__ __forceinline__ void hash_token(const int32_t *__restrict__ ids, const int32_t *__restrict__ remap,
+                                           const int32_t *__restrict__ history, uint32_t *row,
+                                           int32_t *__restrict__ xr_out, const HashParams &p, int64_t n) {
     const int32_t b = static_cast<int32_t>(n / p.T);
     const int32_t t = static_cast<int32_t>(n - static_cast<int64_t>(b) * p.T);
 
@@ -89,7 +82,6 @@ __global__ void __launch_bounds__(256) hash_kernel(const int32_t *__restrict__ i
         if (i == 0 && xr_out != nullptr) xr_out[n] = x;
         xp1[i] = static_cast<uint64_t>(static_cast<int64_t>(x)) + 1ull;
     }
-    uint32_t *row = idx + n * p.H;
     for (int h = 0; h < p.H; ++h) {
         const int o = p.order[h];
         uint64_t s = 0;
@@ -98,6 +90,22 @@ __global__ void __launch_bounds__(256) hash_kernel(const int32_t *__restrict__ i
             if (i < o) s ^= xp1[i] * p.mult[h][i];
         row[h] = mod_prime(fmix64(s), p.prime[h], p.barrett[h]);
     }
+}
+
+// One thread per token.  Reads the token and the (max_order - 1) before it (remapping each
+// through `remap` when given), then for every table h forms the gram of its order and writes
+// idx[n, h] = fmix64(XOR_i (x'_{t-i} + 1) * a_{h,i}) mod P_h.
+// Token ids outside [0, vocab_in) read as the pad id and raise ENGRAM_STATUS_BAD_TOKEN.
+__global__ void __launch_bounds__(256) hash_kernel(const int32_t *__restrict__ ids,
+                                                   const int32_t *__restrict__ remap,
+                                                   const int32_t *__restrict__ history,
+                                                   uint32_t *__restrict__ idx,
+                                                   int32_t *__restrict__ xr_out,
+                                                   const __grid_constant__ HashParams p) {
+    const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t n_tok = static_cast<int64_t>(p.B) * p.T;
+    if (n >= n_tok) return;
+    hash_token(ids, remap, history, idx + n * p.H, xr_out, p, n);
 }
 
 // Plain remap (step 1 on its own).
@@ -489,6 +497,110 @@ __global__ void __launch_bounds__(256) stage_copy_kernel(const __grid_constant__
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u)
             if (dst[u] >= 0) reinterpret_cast<uint4 *>(p.staging[hh[u]])[dst[u]] = val[u];
+    }
+}
+
+// Small batches (at most kStageSmallRows (token, table) rows): remap + hash, in-batch dedup
+// and the copy of the distinct rows in ONE kernel, so that a decode step's prefetch from host
+// memory pays one launch and one dependent chain instead of three.  Every CTA hashes the whole
+// batch and dedups it in shared memory itself (a few hundred rows: cheaper than a second
+// launch), then copies its share of the distinct rows' 16-byte chunks; CTA 0 alone writes the
+// row ids, the slots and the distinct-row lists.  Results are those of hash_kernel,
+// stage_dedup_kernel and stage_copy_kernel: the same slots (distinct rows numbered in
+// increasing order per table) and the same staged bytes.
+constexpr int kStageSmallRows = 256;
+constexpr int kStageSmallThreads = 256;
+static_assert(kStageSmallRows % kStageSmallThreads == 0, "rows per thread");
+
+template <int UNROLL>
+__global__ void __launch_bounds__(kStageSmallThreads) stage_small_kernel(
+    const int32_t *__restrict__ ids, const int32_t *__restrict__ remap, const int32_t *__restrict__ history,
+    uint32_t *__restrict__ idx_out, int32_t *__restrict__ xr_out, uint32_t *__restrict__ staged_idx,
+    uint32_t *__restrict__ unique_rows, int32_t *__restrict__ n_unique, const __grid_constant__ HashParams hp,
+    const __grid_constant__ StageParams sp) {
+    __shared__ uint32_t s_row[kStageSmallRows];    // [n_tok, H] row ids
+    __shared__ uint32_t s_slot[kStageSmallRows];   // slot of each (token, table)
+    __shared__ uint32_t s_uniq[kStageSmallRows];   // [H][n_tok] distinct rows, increasing
+    __shared__ int32_t s_nu[ENGRAM_MAX_TABLES];
+    const int H = hp.H;
+    const int n_tok = hp.B * hp.T;
+    const int rows = n_tok * H;
+    const bool writer = blockIdx.x == 0;
+    if (threadIdx.x < H) s_nu[threadIdx.x] = 0;
+    for (int n = threadIdx.x; n < n_tok; n += blockDim.x)
+        hash_token(ids, remap, history, s_row + n * H, writer ? xr_out : nullptr, hp, n);
+    __syncthreads();
+    // a (token, table) row is a head if no earlier token of the table has the same row id
+    // (s_slot holds the flag for now) ...
+    for (int e = threadIdx.x; e < rows; e += blockDim.x) {
+        const int h = e % H;
+        const uint32_t r = s_row[e];
+        uint32_t head = 1;
+        for (int m = 0; m < e / H; ++m) head &= s_row[m * H + h] != r;
+        s_slot[e] = head;
+    }
+    __syncthreads();
+    // ... and its slot is the number of heads of the table with a smaller row id
+    uint32_t slot[kStageSmallRows / kStageSmallThreads];
+    for (int e = threadIdx.x, k = 0; e < rows; e += blockDim.x, ++k) {
+        const int h = e % H;
+        const uint32_t r = s_row[e];
+        uint32_t below = 0;
+        for (int m = 0; m < n_tok; ++m) below += s_slot[m * H + h] & static_cast<uint32_t>(s_row[m * H + h] < r);
+        slot[k] = below;
+        if (s_slot[e]) {
+            s_uniq[h * n_tok + below] = r;
+            atomicAdd(&s_nu[h], 1);
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x, k = 0; e < rows; e += blockDim.x, ++k) s_slot[e] = slot[k];
+    __syncthreads();
+    if (writer) {
+        for (int e = threadIdx.x; e < rows; e += blockDim.x) {
+            idx_out[e] = s_row[e];
+            staged_idx[e] = s_slot[e];
+        }
+        for (int h = 0; h < H; ++h)
+            for (int i = threadIdx.x; i < s_nu[h]; i += blockDim.x)
+                unique_rows[static_cast<int64_t>(h) * sp.capacity + i] = s_uniq[h * n_tok + i];
+        if (threadIdx.x < H) n_unique[threadIdx.x] = s_nu[threadIdx.x];
+    }
+    // copy the distinct rows: chunk c of slot s of table h, grid-wide
+    const int64_t per_table = static_cast<int64_t>(n_tok) * sp.chunks_per_row;
+    const int64_t total = per_table * H;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < total;
+         base += stride * UNROLL) {
+        uint4 val[UNROLL];
+        int64_t dst[UNROLL];
+        int hh[UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            const int64_t i = base + u * stride;
+            dst[u] = -1;
+            hh[u] = 0;
+            if (i < total) {
+                const int h = static_cast<int>(i / per_table);
+                const int64_t r = i - h * per_table;
+                const int32_t sl = static_cast<int32_t>(r / sp.chunks_per_row);
+                const int32_t c = static_cast<int32_t>(r - static_cast<int64_t>(sl) * sp.chunks_per_row);
+                if (sl < s_nu[h]) {
+                    const uint32_t row = s_uniq[h * n_tok + sl];
+                    hh[u] = h;
+                    dst[u] = r;
+                    if (row < sp.rows[h]) {
+                        val[u] = reinterpret_cast<const uint4 *>(sp.table[h])[static_cast<int64_t>(row) * sp.chunks_per_row + c];
+                    } else {
+                        val[u] = make_uint4(0, 0, 0, 0);
+                        atomicOr(&g_engram_status, ENGRAM_STATUS_BAD_ROW);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u)
+            if (dst[u] >= 0) reinterpret_cast<uint4 *>(sp.staging[hh[u]])[dst[u]] = val[u];
     }
 }
 

@@ -27,8 +27,6 @@ constexpr int kBM = 128;          // tokens per tile (UMMA M)
 constexpr int kBK = 64;           // K elements per stage: one 128-byte swizzle row
 constexpr int kUmmaK = 16;        // K per tcgen05.mma for 16-bit inputs
 constexpr int kProjThreads = 192; // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
-constexpr int kGatherThreads = 128; // row-gather mode: warps 6-9 fill the A tiles from the tables
-constexpr int kGatherRows = kBM * (kBK * 2 / 16) / kGatherThreads;   // tile rows per gather thread (8)
 
 template <int BN>
 struct ProjCfg {
@@ -42,7 +40,6 @@ struct ProjCfg {
     // floats: 16-byte row starts, conflict-free quarter-warp phases)
     static constexpr int kTrStride = 36;
     static constexpr int kTrBytes = 4 * 32 * kTrStride * 4;
-    static_assert(kTrBytes >= kBM * ENGRAM_MAX_TABLES * 4, "row-gather mode keeps a tile's row ids there");
     // dynamic smem: [align pad][stages x A][stages x B][transpose tiles]
     //               [full, empty, tmem_full, tmem_empty][tmem addr]
     static constexpr int kBarBytes = (2 * kStages + 2 * kAccum) * 8;
@@ -65,11 +62,6 @@ struct ProjParams {
     int32_t kb_per_split;      // k-blocks per split
     float *acc_out;            // [k_splits, n_tok, (M+1)*d_h] when k_splits > 1
     const uint8_t *w_packed;   // non-null: B tiles come as 32 KB pre-swizzled blocks (BN = 256)
-    // row-gather mode (GATHER): the A tiles are the tables' rows named by idx, not a tile of m
-    const uint32_t *idx;                   // [n_tok, H] row ids
-    const uint16_t *tab[ENGRAM_MAX_TABLES];  // bf16 tables [tab_rows[h], d_e]
-    uint32_t tab_rows[ENGRAM_MAX_TABLES];
-    int32_t H, d_e;
     uint64_t wait_limit_ns;    // bound of every pipeline wait (0: ENGRAM_WAIT_TIMEOUT_NS)
     int32_t stall;             // self-test of the bounded waits: issue no loads at all, so that
                                // the first wait for a stage runs out and the kernel unwinds
@@ -171,111 +163,6 @@ __device__ __forceinline__ void epilogue_chunk(const ProjParams &p, const float 
     }
 }
 
-// L2 prefetch of `bytes` (a multiple of 16, 16-byte aligned) at `src`: no data reaches the SM.
-__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void gather_bar_sync() {   // the gather warps only (named barrier 1)
-    asm volatile("bar.sync 1, %0;" ::"n"(kGatherThreads) : "memory");
-}
-constexpr uint32_t kNoRow = 0xFFFFFFFFu;   // sIdx entry of a token past n_tok or a bad row id
-
-// Row-gather producer (kGatherThreads threads): fills the A tile of every stage from the
-// tables.  Work unit t (t = t0, t0 + tstep, ... < total; whole K) covers tile rows
-// [(t / n_tiles) * unit_rows + row_off, +kBM).  At the start of a unit the gather warps copy
-// the unit's row ids [kBM, H] into shared memory (sIdx) and ask L2 to prefetch every row the
-// unit will read (the CTA whose unit is the tile's first channel slice only: the other
-// slices' CTAs read the same rows at about the same time), so the k-blocks after the first
-// few find their rows in L2.  Thread g then
-// fills the 16-byte piece j = g % 8 of tile rows r0 + 16i (r0 = g / 8, i < 8) of every stage;
-// all those rows share r mod 8 = r0 mod 8, hence one 128-byte-swizzle position.  Column c of
-// the memory vector lies in table c / d_e at column c % d_e (the concatenation of step 3).
-// Lane 0 of each warp waits for the stage to be free; each thread's completion is one
-// arrival on the stage's full barrier (cp.async.mbarrier.arrive.noinc), which is what makes
-// the copies visible to the tensor cores that read the stage.  Rows past n_tok,
-// bad row ids and columns past d_m are zero-filled.  Returns after its copies have landed.
-template <int S, int ATILE>
-__device__ __forceinline__ void gather_a_tiles(const ProjParams &p, uint8_t *sA, uint32_t *sIdx, uint64_t *full_bar,
-                                               uint64_t *empty_bar, volatile int *abort_flag, uint64_t lim,
-                                               int g, int t0, int tstep, int total, int unit_rows, int row_off) {
-    const int j = g & 7;
-    const int r0 = g >> 3;
-    const int lane = g & 31;
-    const uint32_t off0 = static_cast<uint32_t>(r0 * (kBK * 2) + ((j ^ (r0 & 7)) << 4));
-    constexpr uint32_t kRowStep = (kGatherThreads / 8) * kBK * 2;   // 16 rows of 128 bytes
-    const int H = p.H;
-    const uint32_t row_bytes = static_cast<uint32_t>(p.d_e) * 2;
-    int it = 0;
-    bool stop = false;
-    for (int t = t0; t < total && !stop; t += tstep) {
-        const int64_t m0 = static_cast<int64_t>(t / p.n_tiles) * unit_rows + row_off;
-        // ---- the unit's row ids into shared memory, and its rows on their way into L2
-        gather_bar_sync();   // every gather thread is done with the previous unit's ids
-        if (g == 0 && t + tstep < total) {   // the next unit's row ids, into L2 ahead of time
-            const int64_t m1 = static_cast<int64_t>((t + tstep) / p.n_tiles) * unit_rows + row_off;
-            const int64_t rows = min(static_cast<int64_t>(kBM), p.n_tok - m1);
-            const uint32_t bytes = static_cast<uint32_t>(rows * H * 4) & ~15u;   // whole 16-byte pieces inside idx
-            if (rows > 0 && bytes > 0) prefetch_l2_bulk(p.idx + m1 * H, bytes);
-        }
-        const bool prefetch_rows = t % p.n_tiles == 0;
-        // kBM * H entries, kGatherThreads apart: eight independent loads in flight per round
-        for (int e0 = g; e0 < kBM * H; e0 += 8 * kGatherThreads) {
-            uint32_t rid[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int e = e0 + u * kGatherThreads;
-                const int64_t n = m0 + e / H;
-                rid[u] = (e < kBM * H && n < p.n_tok) ? __ldg(p.idx + m0 * H + e) : kNoRow;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int e = e0 + u * kGatherThreads;
-                if (e >= kBM * H) break;
-                const int h = e % H;
-                if (rid[u] != kNoRow) {
-                    if (rid[u] >= p.tab_rows[h]) {
-                        atomicOr(&g_engram_status, ENGRAM_STATUS_BAD_ROW);
-                        rid[u] = kNoRow;
-                    } else if (prefetch_rows) {
-                        prefetch_l2_bulk(p.tab[h] + static_cast<int64_t>(rid[u]) * p.d_e, row_bytes);
-                    }
-                }
-                sIdx[e] = rid[u];
-            }
-        }
-        gather_bar_sync();
-        // ---- the unit's k-blocks
-        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
-            const int s = it % S;
-            bool ok = true;
-            if (lane == 0) ok = mbar_wait(&empty_bar[s], ((it / S) & 1) ^ 1, abort_flag, lim);
-            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
-                stop = true;
-                break;
-            }
-            const uint32_t dst = smem_u32(sA + s * ATILE) + off0;
-            const int col = kb * kBK + j * 8;
-            if (col < p.d_m) {
-                const int h = col / p.d_e;
-                const uint16_t *base = p.tab[h] + (col - h * p.d_e);
-#pragma unroll
-                for (int i = 0; i < kGatherRows; ++i) {
-                    const uint32_t rid = sIdx[(r0 + 16 * i) * H + h];
-                    const bool valid = rid != kNoRow;
-                    cp_async_16(dst + i * kRowStep, valid ? base + static_cast<int64_t>(rid) * p.d_e : base,
-                                valid ? 16u : 0u);
-                }
-            } else {   // columns beyond d_m (ragged last k-block): zeros
-#pragma unroll
-                for (int i = 0; i < kGatherRows; ++i) cp_async_16(dst + i * kRowStep, p.tab[0], 0u);
-            }
-            cp_async_arrive_noinc(&full_bar[s]);
-        }
-    }
-    cp_async_wait_all();   // nothing may still land in shared memory after the CTA ends
-}
-
 // Persistent: grid = min(#tiles, #SMs); CTA i takes tiles i, i + grid, ...  Tile t covers
 // tokens [128*(t / n_tiles), +128) and channel slice t % n_tiles, so the CTAs running at
 // one time share a few 128-token blocks of m (re-read from L2) and stream all of W.
@@ -283,14 +170,8 @@ __device__ __forceinline__ void gather_a_tiles(const ProjParams &p, uint8_t *sA,
 // Two TMEM accumulators: the epilogue drains tile i while the MMAs of tile i+1 run.
 // SPLIT: compiled for split-K work units (p.k_splits > 1, raw partial accumulators out) or
 // for whole-K tiles only, so that neither epilogue costs the other registers.
-// GATHER (whole-K tiles only): m is never materialised.  Warps 6-9 build each 128 x 64 A
-// tile from the tables themselves -- token n's columns [64kb, 64kb+64) are 16-byte pieces of
-// the rows idx[n, h] names (column c lies in table c / d_e at column c % d_e, the
-// concatenation of step 3) -- with cp.async into the same 128-byte-swizzled layout the TMA
-// would write; each thread's completion is one arrival on the stage's full barrier.  Warp 0
-// then streams only the weight tiles.
-template <int BN, bool SPLIT, bool GATHER>
-__global__ void __launch_bounds__(kProjThreads + (GATHER ? kGatherThreads : 0), 1)
+template <int BN, bool SPLIT>
+__global__ void __launch_bounds__(kProjThreads, 1)
     proj_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ CUtensorMap map_wk,
                 const __grid_constant__ CUtensorMap map_wv, const __grid_constant__ ProjParams p) {
     using Cfg = ProjCfg<BN>;
@@ -308,7 +189,6 @@ __global__ void __launch_bounds__(kProjThreads + (GATHER ? kGatherThreads : 0), 
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(tempty_bar + NACC);
     __shared__ int s_abort;
 
-    static_assert(!(SPLIT && GATHER), "the row-gather mode runs whole-K tiles only");
     pdl_launch_dependents();   // the kernel after this one may load its independent inputs now
     const uint64_t lim = p.wait_limit_ns ? p.wait_limit_ns : ENGRAM_WAIT_TIMEOUT_NS;
     const int warp = threadIdx.x / 32;
@@ -321,7 +201,7 @@ __global__ void __launch_bounds__(kProjThreads + (GATHER ? kGatherThreads : 0), 
     if (threadIdx.x == 0) {
         s_abort = 0;
         for (int s = 0; s < S; ++s) {
-            mbar_init(&full_bar[s], GATHER ? 1 + kGatherThreads : 1);
+            mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
         for (int a = 0; a < NACC; ++a) {
@@ -342,7 +222,7 @@ __global__ void __launch_bounds__(kProjThreads + (GATHER ? kGatherThreads : 0), 
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
 
-    constexpr uint32_t kTxBytes = GATHER ? Cfg::kBTile : Cfg::kStageBytes;   // TMA bytes per stage
+    constexpr uint32_t kTxBytes = Cfg::kStageBytes;   // TMA bytes per stage: A + B
     if (warp == 0) {
         if (lane == 0 && !p.stall) {
             // unit t -> (k split, m tile, n tile) and the weight tile it streams
@@ -385,13 +265,13 @@ __global__ void __launch_bounds__(kProjThreads + (GATHER ? kGatherThreads : 0), 
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     if (it < pre) {   // weight tile and byte count already issued
-                        if constexpr (!GATHER) tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
+                        tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
                         continue;
                     }
                     const uint32_t ph = (it / S) & 1;
                     if (!mbar_wait(&empty_bar[s], ph ^ 1, &s_abort, lim)) break;
                     mbar_arrive_expect_tx(&full_bar[s], kTxBytes);
-                    if constexpr (!GATHER) tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
+                    tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
                     load_b(s, nt, kb);
                     issued = it + 1;
                 }
@@ -437,7 +317,7 @@ __global__ void __launch_bounds__(kProjThreads + (GATHER ? kGatherThreads : 0), 
                 for (int a = 0; a < NACC; ++a) mbar_arrive(&tfull_bar[a]);   // release waiting epilogue warps
             }
         }
-    } else if (warp < kProjThreads / 32) {
+    } else {
         // ---------------------------------------------------------------- epilogue
         const int sub = warp & 3;                      // TMEM lane quarter this warp may access
         const int row = sub * 32 + lane;
@@ -492,14 +372,6 @@ __global__ void __launch_bounds__(kProjThreads + (GATHER ? kGatherThreads : 0), 
             if constexpr (!SPLIT) {
                 if (valid) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
             }
-        }
-    } else if constexpr (GATHER) {
-        // ---------------------------------------------------------------- A-tile row gather
-        if (!p.stall) {
-            pdl_wait();   // the row ids come from the kernel before this one
-            // the row ids live in the split-K transpose region, unused by whole-K tiles
-            gather_a_tiles<S, Cfg::kATile>(p, sA, reinterpret_cast<uint32_t *>(s_tr), full_bar, empty_bar, &s_abort,
-                                           lim, threadIdx.x - kProjThreads, blockIdx.x, gridDim.x, total, kBM, 0);
         }
     }
     tc_fence_before();

@@ -7,14 +7,14 @@
 // half the MMA work), so the tensor cores read half the B bytes per flop and the stage ring
 // holds six k-blocks instead of four.
 //
-// Roles in each CTA: warp 0 lane 0 loads its CTA's tiles (TMA / bulk copies onto its own full
-// barrier, no multicast); warp 1 lane 0 of the even CTA waits for both CTAs' stages and
-// issues the MMAs, committing stage and accumulator releases to the barriers of both CTAs
-// (tcgen05.commit with a CTA mask: an arrival, not a data multicast); warp 1 lane 0 of the
-// odd CTA forwards its CTA's stage completions to the even CTA's full barrier; warps 2-5 drain
-// their CTA's accumulator rows (the epilogue of proj_kernel) and hand the accumulator back to
-// the even CTA; in row-gather mode warps 6-9 build the CTA's A tiles from the tables.  Every
-// wait is bounded; the CTAs leave only together (cluster barrier), after the last MMA.
+// Roles in each CTA: warp 0 lane 0 loads its CTA's tiles into its own shared memory with the
+// cta_group::2 TMA forms, whose bytes are counted on the EVEN CTA's full barrier (no
+// multicast; the even CTA's expect_tx covers both halves); warp 1 lane 0 of the even CTA
+// waits for the stage and issues the MMAs, committing stage and accumulator releases to the
+// barriers of both CTAs (tcgen05.commit with a CTA mask: an arrival, not a data multicast);
+// warps 2-5 drain their CTA's accumulator rows (the epilogue of proj_kernel) and hand the
+// accumulator back to the even CTA.  Every wait is bounded; the CTAs leave only together
+// (cluster barrier), after the last MMA.
 #pragma once
 #include "kernels_proj.cuh"
 
@@ -30,11 +30,10 @@ struct PairCfg {
     static constexpr int kStages = 6;
     static constexpr int kAccum = 2;
     static constexpr int kTmemCols = kAccum * kPairBN;        // 512: all of tensor memory
-    // dynamic smem: [align pad][stages x A][stages x B][row ids of a tile (row-gather mode)]
-    //               [full, empty, tmem_full, tmem_empty, drain][tmem addr]
-    static constexpr int kIdxBytes = kBM * ENGRAM_MAX_TABLES * 4;
+    // dynamic smem: [align pad][stages x A][stages x B][full, empty, tmem_full, tmem_empty,
+    //               drain][tmem addr]
     static constexpr int kBarBytes = (2 * kStages + 2 * kAccum + 1) * 8;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kIdxBytes + kBarBytes + 16;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 16;
 };
 
 __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
@@ -42,8 +41,10 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v
 }
 
 // p.m_tiles counts 256-token tiles; p.n_tiles = (M + 1) * d_h / 256; whole-K units only.
-template <bool GATHER>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads + (GATHER ? kGatherThreads : 0), 1)
+// map_wk / map_wv: the row-major weights (boxes of 128 rows), or with packed weights map_wk
+// spans the packed copy as [tiles * k_blocks * 256 rows, 64 columns] (boxes of 128 rows, no
+// swizzle: the bytes are already in the tensor cores' layout) and map_wv is unused.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads, 1)
     proj_pair_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ CUtensorMap map_wk,
                      const __grid_constant__ CUtensorMap map_wv, const __grid_constant__ ProjParams p) {
     using Cfg = PairCfg;
@@ -54,8 +55,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads + (GATH
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + S * Cfg::kATile;
-    uint32_t *sIdx = reinterpret_cast<uint32_t *>(smem + S * Cfg::kStageBytes);
-    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes + Cfg::kIdxBytes);
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes);
     uint64_t *empty_bar = full_bar + S;
     uint64_t *tfull_bar = empty_bar + S;      // MMA -> epilogue of both CTAs
     uint64_t *tempty_bar = tfull_bar + NACC;  // epilogues of both CTAs -> MMA (even CTA's copy)
@@ -77,8 +77,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads + (GATH
     if (threadIdx.x == 0) {
         s_abort = 0;
         for (int s = 0; s < S; ++s) {
-            // own loads' expect_tx arrival, own gather threads, and (even CTA) the partner's forward
-            mbar_init(&full_bar[s], 1 + (GATHER ? kGatherThreads : 0) + (rank == 0 ? 1 : 0));
+            mbar_init(&full_bar[s], 1);    // even CTA: its producer's expect_tx arrival (both halves' bytes)
             mbar_init(&empty_bar[s], 1);
         }
         for (int a = 0; a < NACC; ++a) {
@@ -99,20 +98,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads + (GATH
     cluster_sync();   // both CTAs' barriers initialised, tensor memory allocated
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
-    constexpr uint32_t kTxBytes = GATHER ? Cfg::kBTile : Cfg::kStageBytes;
+    constexpr uint32_t kTxBytes = 2 * Cfg::kStageBytes;   // both CTAs' A and B halves, on the even CTA's barrier
+    const uint32_t full_cluster = mapa_shared(full_bar, 0);
 
     if (warp == 0) {
         if (lane == 0 && !p.stall) {
             auto load_b = [&](int s, int nt, int kb) {
                 if (p.w_packed != nullptr)   // this CTA's 128 rows of the pre-swizzled 256 x 64 tile: 16 KB
-                    bulk_load_1d(sB + s * Cfg::kBTile,
-                                 p.w_packed + (static_cast<int64_t>(nt) * p.k_blocks + kb) * (2 * Cfg::kBTile) +
-                                     rank * Cfg::kBTile,
-                                 Cfg::kBTile, &full_bar[s]);
+                    tma_load_2d_pair(sB + s * Cfg::kBTile, &map_wk, full_cluster + s * 8, 0,
+                                     (nt * p.k_blocks + kb) * BN + static_cast<int>(rank) * (BN / 2));
                 else {
                     const bool is_key = nt < key_tiles;
-                    tma_load_2d(sB + s * Cfg::kBTile, is_key ? &map_wk : &map_wv, &full_bar[s], kb * kBK,
-                                (is_key ? nt : nt - key_tiles) * BN + static_cast<int>(rank) * (BN / 2));
+                    tma_load_2d_pair(sB + s * Cfg::kBTile, is_key ? &map_wk : &map_wv, full_cluster + s * 8, kb * kBK,
+                                     (is_key ? nt : nt - key_tiles) * BN + static_cast<int>(rank) * (BN / 2));
                 }
             };
             int pre = 0;
@@ -120,7 +118,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads + (GATH
                 const int nt0 = pair % p.n_tiles;
                 pre = min(S, p.k_blocks);
                 for (int q = 0; q < pre; ++q) {
-                    mbar_arrive_expect_tx(&full_bar[q], kTxBytes);
+                    if (rank == 0) mbar_arrive_expect_tx(&full_bar[q], kTxBytes);
                     load_b(q, nt0, q);
                 }
             }
@@ -132,17 +130,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads + (GATH
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int s = it % S;
                     if (it < pre) {
-                        if constexpr (!GATHER) tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
+                        tma_load_2d_pair(sA + s * Cfg::kATile, &map_m, full_cluster + s * 8, kb * kBK, m0);
                         continue;
                     }
                     if (!mbar_wait(&empty_bar[s], ((it / S) & 1) ^ 1, &s_abort, lim)) break;
-                    mbar_arrive_expect_tx(&full_bar[s], kTxBytes);
-                    if constexpr (!GATHER) tma_load_2d(sA + s * Cfg::kATile, &map_m, &full_bar[s], kb * kBK, m0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], kTxBytes);
+                    tma_load_2d_pair(sA + s * Cfg::kATile, &map_m, full_cluster + s * 8, kb * kBK, m0);
                     load_b(s, nt, kb);
                     issued = it + 1;
                 }
             }
-            if (s_abort) {   // every issued copy lands before the CTA's shared memory is released
+            if (s_abort && rank == 0) {   // every issued copy lands before shared memory is released
                 volatile int never = 0;
                 for (int k = issued - S > 0 ? issued - S : 0; k < issued; ++k)
                     if (!mbar_wait(&full_bar[k % S], (k / S) & 1, &never, lim)) break;
@@ -163,7 +161,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads + (GATH
                 bool ok = true;
                 for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
                     const int s = it % S;
-                    if (!mbar_wait_cluster(&full_bar[s], (it / S) & 1, &s_abort, lim)) { ok = false; break; }
+                    if (!mbar_wait(&full_bar[s], (it / S) & 1, &s_abort, lim)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t adesc = sdesc_kmajor_sw128(sA + s * Cfg::kATile);
                     const uint64_t bdesc = sdesc_kmajor_sw128(sB + s * Cfg::kBTile);
@@ -191,20 +189,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads + (GATH
                     mbar_arrive_cluster(mapa_shared(&tfull_bar[a], 1));
                 }
             }
-        } else if (lane == 0) {
-            // ------------------------------------------------------------ stage forwarding (odd CTA)
-            const uint32_t leader_full = mapa_shared(full_bar, 0);
-            int it = 0;
-            bool stop = false;
-            for (int t = pair; t < total && !stop; t += npairs) {
-                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
-                    const int s = it % S;
-                    if (!mbar_wait(&full_bar[s], (it / S) & 1, &s_abort, lim)) { stop = true; break; }
-                    mbar_arrive_cluster(leader_full + s * 8);
-                }
-            }
         }
-    } else if (warp < kProjThreads / 32) {
+    } else {
         // ---------------------------------------------------------------- epilogue
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
@@ -213,7 +199,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads + (GATH
         for (int t = pair; t < total; t += npairs, ++li) {
             const int acc = li % NACC;
             const uint32_t use = li / NACC;
-            if (!mbar_wait_cluster(&tfull_bar[acc], use & 1, &s_abort, lim) || s_abort) break;
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait_cluster(&tfull_bar[acc], use & 1, &s_abort, lim) && !s_abort;
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             tc_fence_after();
             const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
             const bool is_key = nt < key_tiles;
@@ -232,14 +220,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads + (GATH
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_tempty + acc * 8);   // to the even CTA's copy
             if (valid) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
-        }
-    } else if constexpr (GATHER) {
-        // ---------------------------------------------------------------- A-tile row gather
-        if (!p.stall) {
-            pdl_wait();
-            gather_a_tiles<S, Cfg::kATile>(p, sA, sIdx, full_bar, empty_bar, &s_abort, lim,
-                                           threadIdx.x - kProjThreads, pair, npairs, total, kPairRows,
-                                           static_cast<int>(rank) * kBM);
         }
     }
     tc_fence_before();

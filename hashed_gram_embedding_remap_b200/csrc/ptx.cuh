@@ -86,27 +86,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
-// Same, with cluster-scope acquire: for barriers that threads of the other CTA of a cluster
-// arrive on (their writes become visible to the waiting thread).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+// Non-blocking test of a phase with cluster-scope acquire: for barriers that the other CTA of
+// a cluster completes (remote arrivals, multicast commits), whose waiters are polled rather
+// than suspended in try_wait.
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }
+// Polling wait for such barriers, bounded like mbar_wait.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                                   uint64_t limit_ns) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (mbar_test_wait_cluster(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
 #pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait_cluster(bar, parity)) return true;
+        for (int i = 0; i < 64; ++i)
+            if (mbar_test_wait_cluster(bar, parity)) return true;
         if (*abort_flag) return false;
         if (global_timer_ns() - t0 > limit_ns) {
             atomicOr(&g_engram_status, 0x4u);
@@ -153,6 +155,17 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// CTA-pair forms (cta_group::2): the copy lands in this CTA's shared memory and its bytes are
+// counted on the mbarrier at `bar_cluster` (a shared::cluster address: the even CTA's barrier,
+// so that one barrier sees both CTAs' halves of a stage).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster, int x,
+                                                 int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+        : "memory");
+}
 // 1-D bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from global
 // into this CTA's shared memory, completion signalled on `bar` as bytes.  No multicast.
 __device__ __forceinline__ void bulk_load_1d(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {

@@ -117,14 +117,9 @@ typedef struct engram_config {
  * M = 1 is the single-branch layer, with the layouts stated at each entry point. */
 
 /* engram_config.flags */
-#define ENGRAM_FLAG_SEPARATE_GATHER 0x2 /* engram_forward gathers the rows into m with the
-                                           separate gather kernel even where the projection
-                                           could gather them straight into its tiles (see
-                                           engram_forward_path); results are bit-identical
-                                           either way.  Bit 0x1 is retired and rejected. */
-#define ENGRAM_FLAG_SINGLE_CTA_MMA 0x4  /* never pair CTAs for the projection's MMAs (see
-                                           ENGRAM_PATH_PAIR_MMA); results are bit-identical
-                                           either way. */
+#define ENGRAM_FLAG_SINGLE_CTA_MMA 0x4 /* never pair CTAs for the projection's MMAs (see
+                                          ENGRAM_PATH_PAIR_MMA); results are bit-identical either
+                                          way.  Bits 0x1 and 0x2 are retired and rejected. */
 
 /* Validated config plus derived constants.  Caller-owned, plain data: engram_init fills
  * it, every other call reads it.  Do not modify its fields. */
@@ -232,6 +227,20 @@ int engram_stage_rows(const engram_plan *plan, const uint32_t *idx, int64_t n_to
                       uint32_t *staged_idx, uint32_t *unique_rows, int32_t *n_unique,
                       engram_stream_t stream);
 
+/* Steps 1-2 and the staging of engram_stage_rows in one call: idx = engram_hash of the
+ * (remapped) ids -- ids, remap, B, T and history as in engram_forward and engram_hash --
+ * then the batch's distinct rows staged exactly as engram_stage_rows stages them (same
+ * staged_idx, unique_rows, n_unique and staging contents).  idx: uint32 [B*T, H] (device,
+ * out).  Batches of at most 256 (token, table) rows (a decode step) run as ONE kernel that
+ * hashes, dedups in shared memory and copies from the host tables, so the prefetch of a step
+ * pays one launch; larger batches run the hash kernel, then engram_stage_rows' kernels.
+ * B*T <= 8192, capacity >= B*T.  engram_forward takes the one-kernel path itself for
+ * decode-sized batches on ENGRAM_TABLES_HOST_MAPPED tables. */
+int engram_stage_rows_from_ids(const engram_plan *plan, const int32_t *ids, const int32_t *remap, int32_t B,
+                               int32_t T, const int32_t *history, const void *const *tables, void *const *staging,
+                               int32_t capacity, uint32_t *idx, uint32_t *staged_idx, uint32_t *unique_rows,
+                               int32_t *n_unique, engram_stream_t stream);
+
 /* An HBM cache of host-table rows, in front of ENGRAM_TABLES_HOST_MAPPED tables [zhichai
  * §2.3: n-gram frequencies are Zipf-like, so a few rows are read most of the time and can
  * live in fast memory while the rest stays in host memory; the pages also report that real
@@ -293,13 +302,12 @@ int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
 /* Steps 1-6 chained: remap + hash (one kernel), gather, projections with the gate's partial
  * reductions fused in their epilogue, then gate + conv + residual, then the history update
  * when `history` is given.  Kernels per call (engram_forward_path tells which apply): prefill
- * batches on bf16 HBM-resident tables launch remap + hash, the projection -- which gathers
- * each token's rows into its tiles itself -- gate scalars and the streaming gate + conv
- * kernel (4); with e4m3 or host-mapped tables, or ENGRAM_FLAG_SEPARATE_GATHER, a gather
- * kernel writes m first (5); batches of at most 16,384 (token, table) rows on HBM-resident
- * tables fuse remap + hash + gather into one kernel; one-token decode steps whose
- * projection splits K finish the split sums, gate, conv and the history update in one
- * kernel (lookup, projection, that kernel: 3).
+ * batches launch remap + hash, gather, projection, gate scalars and the streaming gate + conv
+ * kernel (5); batches of at most 16,384 (token, table) rows on HBM-resident tables fuse
+ * remap + hash + gather into one kernel; decode-sized batches on host-mapped tables fuse
+ * remap + hash + dedup + staging into one; one-token decode steps whose projection splits K
+ * finish the split sums, gate, conv and the history update in one kernel (lookup,
+ * projection, that kernel: 3).
  * engram_kernel_launches() counts them.
  * ids: int32 [B, T] raw token ids.  remap: int32 [vocab_in], or NULL when ids are already
  * in the compressed vocabulary.  history / conv_state: NULL for prefill, or the decode state
@@ -310,7 +318,7 @@ int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
  * be timed per stage.
  * CUDA graphs: after one eager call on a device (which resolves the tensor-map encoder and
  * sets kernel attributes), engram_forward / engram_gate_conv may be captured and replayed. */
-#define ENGRAM_FORWARD_STAGES 4 /* hash, gather (empty when the projection gathers), projections, gate+conv */
+#define ENGRAM_FORWARD_STAGES 4 /* hash, gather, projections, gate+conv */
 int engram_forward(const engram_plan *plan, const engram_weights *w,
                    const void *const *tables, const int32_t *ids, const int32_t *remap,
                    int32_t B, int32_t T, int32_t *history, uint16_t *conv_state,
@@ -348,20 +356,15 @@ int engram_gate_conv_noalloc(const engram_plan *plan, const engram_weights *w, c
  *   FUSED_LOOKUP   remap + hash + gather in one kernel (at most 16,384 (token, table) rows,
  *                  HBM-resident tables); m is written by it;
  *   STAGED_ROWS    host-mapped tables: the batch's distinct rows are staged into HBM first;
- *   GATHER_IN_PROJ the projection gathers each token's rows straight from the tables into
- *                  its shared-memory tiles (bf16 HBM-resident tables, whole-K projection
- *                  tiles, ENGRAM_FLAG_SEPARATE_GATHER not set): m is never written, and the
- *                  workspace holds no m;
  *   SPLIT_K        the projection splits K across CTAs (decode-sized batches);
  *   PAIR_MMA       the projection runs on pairs of CTAs (a thread-block cluster of two), each
  *                  tensor-core MMA spanning both: 256-token x 256-channel tiles, each CTA
  *                  holding half of every operand tile (d_h % 256 == 0, whole-K tiles, at
  *                  least 148 tiles, ENGRAM_FLAG_SINGLE_CTA_MMA not set); the workspace's
  *                  partial sums then have (M+1)*d_h/256 columns per token.
- * Otherwise the hash kernel writes the row ids and the separate gather kernel writes m. */
+ * Otherwise the hash kernel writes the row ids and the gather kernel writes m. */
 #define ENGRAM_PATH_FUSED_LOOKUP 0x1u
 #define ENGRAM_PATH_STAGED_ROWS 0x2u
-#define ENGRAM_PATH_GATHER_IN_PROJ 0x4u
 #define ENGRAM_PATH_SPLIT_K 0x8u
 #define ENGRAM_PATH_PAIR_MMA 0x10u
 int engram_forward_path(const engram_plan *plan, int32_t B, int32_t T, uint32_t *path);

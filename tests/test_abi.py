@@ -53,7 +53,8 @@ def _plan(**kw):
     (dict(eps=0.0), E.ENGRAM_ERR_INVALID_ARG),
     (dict(conv_kernel=9), E.ENGRAM_ERR_UNSUPPORTED),
     (dict(heads_per_order=17), E.ENGRAM_ERR_UNSUPPORTED),
-    (dict(flags=0x1), E.ENGRAM_ERR_INVALID_ARG),                                # retired flag bit
+    (dict(flags=0x1), E.ENGRAM_ERR_INVALID_ARG),                                # retired flag bits
+    (dict(flags=0x2), E.ENGRAM_ERR_INVALID_ARG),
     (dict(flags=0x8), E.ENGRAM_ERR_INVALID_ARG),                                # unknown flag bit
     (dict(table_dtype=2), E.ENGRAM_ERR_INVALID_ARG),                            # unknown table dtype
     (dict(table_dtype=1, table_scale=(0.1, 0.1, 0.1, 0.0)), E.ENGRAM_ERR_INVALID_ARG),   # zero scale
@@ -211,32 +212,24 @@ def test_packed_weights_size_and_validation():
 def test_forward_path_selection():
     """engram_forward_path (host only): which kernels a forward call runs."""
     P = E.engram_forward_path
-    G, PAIR = E.ENGRAM_PATH_GATHER_IN_PROJ, E.ENGRAM_PATH_PAIR_MMA
-    lay = synth.get_workload("layer2560")
-    p = E.Plan.from_workload(lay)
-    # prefill on bf16 HBM tables: the projection (on CTA pairs) gathers the rows itself, and
-    # the workspace holds no m
-    assert P(p, lay.B, lay.T) == G | PAIR
-    sep = E.Plan.from_workload(lay, flags=E.ENGRAM_FLAG_SEPARATE_GATHER)
-    assert P(sep, lay.B, lay.T) == PAIR
-    assert E.engram_workspace_size(sep, lay.n_tok) - E.engram_workspace_size(p, lay.n_tok) >= lay.n_tok * lay.d_m * 2
-    single = E.Plan.from_workload(lay, flags=E.ENGRAM_FLAG_SINGLE_CTA_MMA)
-    assert P(single, lay.B, lay.T) == G
-    # too few 256 x 256 units for the pairs, or d_h not a multiple of 256
-    assert P(p, 1, 1100) == G
+    PAIR = E.ENGRAM_PATH_PAIR_MMA
+    for name in ("prefill20m", "layer2560"):
+        wl = synth.get_workload(name)
+        # prefill: hash kernel, gather kernel, projection on CTA pairs (d_h % 256 == 0, enough tiles)
+        assert P(E.Plan.from_workload(wl), wl.B, wl.T) == PAIR
+        assert P(E.Plan.from_workload(wl, flags=E.ENGRAM_FLAG_SINGLE_CTA_MMA), wl.B, wl.T) == 0
+        assert P(E.Plan.from_workload(wl.with_(table_dtype="fp8")), wl.B, wl.T) == PAIR
+    p16 = _plan(heads_per_order=8, table_rows=[10007] * 16, row_dim=64, hidden_dim=2560)
+    assert P(p16, 1, 1100) == 0            # 5 x 20 tiles: too few for the pairs
     assert not P(_plan(hidden_dim=384), 8, 4096) & PAIR
-    # e4m3 tables are dequantised by the gather kernel
-    assert P(E.Plan.from_workload(lay.with_(table_dtype="fp8")), lay.B, lay.T) == PAIR
     # decode-sized batches: one lookup kernel, split-K projection
     dec = synth.get_workload("decode20m")
     assert P(E.Plan.from_workload(dec), dec.B, 1) == E.ENGRAM_PATH_FUSED_LOOKUP | E.ENGRAM_PATH_SPLIT_K
     # host-mapped tables: distinct rows staged into HBM first
     hp = synth.get_workload("hostpinned20m")
     assert P(E.Plan.from_workload(hp, host_tables=True), hp.B, 1) & E.ENGRAM_PATH_STAGED_ROWS
-    pre = synth.get_workload("prefill20m")
-    assert P(E.Plan.from_workload(pre), pre.B, pre.T) == G | PAIR
     with pytest.raises(E.EngramError):
-        P(p, -1, 4)
+        P(p16, -1, 4)
 
 
 def test_selftest_and_synchronize_validate_on_host():

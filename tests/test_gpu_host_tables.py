@@ -67,3 +67,48 @@ def test_host_tables_bit_identical_to_device_tables(B, T):
     assert E.engram_device_status(clear=True) == 0
     for b in bufs:
         b.close()
+
+
+@pytest.mark.parametrize("B,T,history", [(64, 1, True), (1, 200, False), (40, 8, True)])
+def test_stage_rows_from_ids_matches_hash_then_stage(B, T, history):
+    """engram_stage_rows_from_ids (one kernel up to 256 (token, table) rows: 64 x 1 with a hash
+    history and 1 x 200; the hash kernel + staging kernels above it: 40 x 8) stages exactly
+    what engram_hash followed by engram_stage_rows stages: row ids, slots, distinct-row lists,
+    counts and the staged bytes."""
+    wl = small_workload("stage_ids", B=B, T=T, K=1, d_e=64, d_h=128, primes=(1009, 1013), ids_kind="zipf",
+                        zipf_s=1.3, decode=history)
+    plan = E.Plan.from_workload(wl, host_tables=True)
+    bufs = _host_tables(wl)
+    tables = [b.tensor for b in bufs]
+    ids = to_dev(wl.ids())
+    remap = to_dev(wl.remap())
+    hist = to_dev(wl.history()) if history else None
+    n = wl.n_tok
+
+    def buffers():
+        return ([torch.full((n, wl.d_e), 7.0, dtype=torch.bfloat16, device="cuda") for _ in range(wl.H)],
+                torch.full((n, wl.H), -1, dtype=torch.int32, device="cuda"),
+                torch.full((n, wl.H), -1, dtype=torch.int32, device="cuda"),
+                torch.full((wl.H, n), -1, dtype=torch.int32, device="cuda"),
+                torch.full((wl.H,), -1, dtype=torch.int32, device="cuda"))
+
+    st_a, idx_a, sidx_a, uq_a, nu_a = buffers()
+    E.engram_stage_rows_from_ids(plan, ids, tables, st_a, idx_a, sidx_a, uq_a, nu_a, remap=remap, history=hist)
+    st_b, idx_b, sidx_b, uq_b, nu_b = buffers()
+    xr = torch.empty_like(ids)
+    E.engram_remap(plan, ids, remap, xr)
+    E.engram_hash(plan, xr, idx_b, history=hist)
+    E.engram_stage_rows(plan, idx_b, tables, st_b, sidx_b, uq_b, nu_b)
+    torch.cuda.synchronize()
+    assert torch.equal(idx_a, idx_b) and torch.equal(sidx_a, sidx_b) and torch.equal(nu_a, nu_b)
+    for h in range(wl.H):
+        k = int(nu_a[h])
+        assert torch.equal(uq_a[h, :k], uq_b[h, :k])
+        assert torch.equal(st_a[h][:k].view(torch.int16), st_b[h][:k].view(torch.int16))
+    # and the row ids are the oracle's
+    ref = oracle.hash_ids(wl.remap()[wl.ids()], wl.orders, wl.K, wl.primes, wl.hash_seed, wl.pad_id,
+                          history=wl.history() if history else None)
+    assert np.array_equal(idx_a.cpu().numpy().view(np.uint32), ref)
+    assert E.engram_device_status(clear=True) == 0
+    for b in bufs:
+        b.close()

@@ -177,71 +177,32 @@ def test_forward_matches_oracle(case):
     assert E.engram_device_status(clear=True) == 0
 
 
-# Batches above 16,384 (token, table) rows, where the projection gathers the rows itself.
-GATHER_IN_PROJ_CASES = {
-    "bn128": PARITY_CASES["bn128"],
-    "bn256": PARITY_CASES["bn256"],
-    "seq_edges": PARITY_CASES["seq_edges"],
-    "gate_walk72": PARITY_CASES["gate_walk72"],
-    # d_e = 40: 64-column k-blocks straddle tables at 16-byte granularity; d_m = 240: the
-    # last k-block is ragged (zero columns); BN = 128
-    "ragged_k_d40": small_workload("gip_rk", B=3, T=2001, K=3, d_e=40, d_h=384),
-    # BN = 64 (d_h = 192), one table per order, ragged token tail
-    "bn64_d48": small_workload("gip_64", B=7, T=1301, K=1, d_e=48, d_h=192),
-    # the 20M-row layer's widths: d_e = 2560 (40 k-blocks per table), d_m = 5120, d_h = 2560
-    "d2560": small_workload("gip_2560", B=3, T=3001, K=1, d_e=2560, d_h=2560),
-}
-
-
-@pytest.mark.parametrize("case", list(GATHER_IN_PROJ_CASES) + ["d2560_packed"])
-def test_gather_in_projection_bit_identical_to_separate_gather(case):
-    """The projection reading its A tiles straight from the tables (cp.async row gather)
-    computes exactly what it computes from the materialised m: Delta and out bit for bit.
-    The cases cover d_e = 16..2560 (k-blocks straddling tables), ragged K, ragged token
-    tails and every projection tile width.  (The parity cases above with more than 16,384
-    (token, table) rows take this path too and are checked against the oracle.)"""
-    packed = case.endswith("_packed")
-    wl = GATHER_IN_PROJ_CASES[case.replace("_packed", "")]
-    a = DeviceInputs(wl)
-    assert E.engram_forward_path(a.plan, wl.B, wl.T) & ~E.ENGRAM_PATH_PAIR_MMA == E.ENGRAM_PATH_GATHER_IN_PROJ
-    if packed:   # weight tiles as one linear bulk copy each (the benchmark's layout)
-        a.weights = E.Weights(a.w_k, a.w_v, a.gamma_q, a.gamma_k, a.gamma_c, a.conv_w,
-                              packed=E.pack_weights(a.plan, a.w_k, a.w_v))
-    a.forward()
-    b = DeviceInputs(wl, tables=a.tables, flags=E.ENGRAM_FLAG_SEPARATE_GATHER)
-    assert E.engram_forward_path(b.plan, wl.B, wl.T) & ~E.ENGRAM_PATH_PAIR_MMA == 0
-    b.forward()
-    torch.cuda.synchronize()
-    assert torch.equal(a.delta, b.delta)
-    assert torch.equal(a.out.view(torch.int16), b.out.view(torch.int16))
-    assert E.engram_device_status(clear=True) == 0
-
-
 PAIR_CASES = {
     "bn256": PARITY_CASES["bn256"],                  # d_h 512: 4 channel slices, 38 x 4 units
     "gate_walk72": PARITY_CASES["gate_walk72"],      # d_h 256, 24,000 tokens
-    "d2560": GATHER_IN_PROJ_CASES["d2560"],          # 9,003 tokens: the last tile's odd CTA holds no token
+    # the 20M-row layer's widths: d_e = 2560 (40 k-blocks per table), d_m = 5120, d_h = 2560;
+    # 9,003 tokens: the last tile's odd CTA holds no token
+    "d2560": small_workload("pair_2560", B=3, T=3001, K=1, d_e=2560, d_h=2560),
+    "bn256_d64": small_workload("pair_256", B=48, T=211, K=2, d_e=64, d_h=512),
     # three branches: key slices of three W_k, then the value slices
     "branches3": small_workload("pair_b3", B=3, T=3001, K=1, d_e=64, d_h=512, branches=3),
+    "d2560_b2": small_workload("pair_2560b", B=2, T=4500, K=1, d_e=2560, d_h=2560, branches=2),
 }
 
 
-@pytest.mark.parametrize("mode", ["gather", "separate_gather", "packed"])
+@pytest.mark.parametrize("packed", [False, True])
 @pytest.mark.parametrize("case", list(PAIR_CASES))
-def test_pair_mma_bit_identical_to_single_cta(case, mode):
+def test_pair_mma_bit_identical_to_single_cta(case, packed):
     """The projection on CTA pairs (cta_group::2 MMAs, 256 x 256 units) computes exactly what
     the single-CTA kernel computes: Delta, out (and so v and the gate partial sums) bit for
-    bit, with the rows gathered in the projection, with m materialised, and with the packed
-    weight tiles (each CTA bulk-copying its 128-row half)."""
+    bit, with row-major weights and with the packed weight tiles (each CTA loading its 128-row
+    half)."""
     wl = PAIR_CASES[case]
-    flags = E.ENGRAM_FLAG_SEPARATE_GATHER if mode == "separate_gather" else 0
-    a = DeviceInputs(wl, flags=flags, random_gammas=True)
-    path = E.engram_forward_path(a.plan, wl.B, wl.T)
-    assert path & E.ENGRAM_PATH_PAIR_MMA
-    assert bool(path & E.ENGRAM_PATH_GATHER_IN_PROJ) == (mode != "separate_gather")
-    b = DeviceInputs(wl, tables=a.tables, flags=flags | E.ENGRAM_FLAG_SINGLE_CTA_MMA, random_gammas=True)
+    a = DeviceInputs(wl, random_gammas=True)
+    assert E.engram_forward_path(a.plan, wl.B, wl.T) & E.ENGRAM_PATH_PAIR_MMA
+    b = DeviceInputs(wl, tables=a.tables, flags=E.ENGRAM_FLAG_SINGLE_CTA_MMA, random_gammas=True)
     assert not E.engram_forward_path(b.plan, wl.B, wl.T) & E.ENGRAM_PATH_PAIR_MMA
-    if mode == "packed":
+    if packed:
         for d in (a, b):
             d.weights = E.Weights(d.w_k, d.w_v, d.gamma_q, d.gamma_k, d.gamma_c, d.conv_w,
                                   packed=E.pack_weights(d.plan, d.w_k, d.w_v))
@@ -255,21 +216,19 @@ def test_pair_mma_bit_identical_to_single_cta(case, mode):
 
 def test_kernel_launch_count_per_call():
     """The library's launch counter (bench.py's gpu_launches): a prefill call launches remap +
-    hash, the projection (gathering the rows itself), gate scalars and the streaming gate
-    kernel (4); with the separate gather, 5; a one-token split-K decode step with hash history
-    and conv state launches the lookup, the projection and the fused reduce + gate + conv +
-    history kernel (3); the same call twice counts the same; a call rejected on the host
-    counts nothing."""
-    wl = PARITY_CASES["bn128"]                  # 9,554 tokens x 4 tables
-    for flags, want in ((0, 4), (E.ENGRAM_FLAG_SEPARATE_GATHER, 5)):
-        di = DeviceInputs(wl, flags=flags).forward()
-        torch.cuda.synchronize()
-        n0 = E.kernel_launches()
-        di.forward()
-        n1 = E.kernel_launches()
-        di.forward()
-        n2 = E.kernel_launches()
-        assert n1 - n0 == want and n2 - n1 == want
+    hash, gather, projection, gate scalars and the streaming gate kernel (5); a one-token
+    split-K decode step with hash history and conv state launches the lookup, the projection
+    and the fused reduce + gate + conv + history kernel (3); the same call twice counts the
+    same; a call rejected on the host counts nothing."""
+    wl = PARITY_CASES["bn128"]                  # 9,554 tokens x 4 tables: the separate hash and gather
+    di = DeviceInputs(wl).forward()
+    torch.cuda.synchronize()
+    n0 = E.kernel_launches()
+    di.forward()
+    n1 = E.kernel_launches()
+    di.forward()
+    n2 = E.kernel_launches()
+    assert n1 - n0 == 5 and n2 - n1 == 5
     with pytest.raises(E.EngramError):
         E.engram_forward(di.plan, di.weights, di.tables, di.ids, di.h, di.out, di.ws[:16])   # workspace too small
     assert E.kernel_launches() == n2

@@ -172,6 +172,7 @@ int choose_bn(int d_h, int64_t n_tok, int M) {
 // the weights; the split-K partial accumulators are finished by splitk_reduce_kernel.
 struct ProjShape {
     int bn, n_tiles, k_blocks, k_splits, kb_per_split;
+    bool pair;   // CTA pairs (proj_pair_kernel): 256-token x 256-channel units
 };
 
 ProjShape proj_shape(const engram_plan *plan, int64_t n_tok, bool allow_split) {
@@ -211,18 +212,28 @@ ProjShape proj_shape(const engram_plan *plan, int64_t n_tok, bool allow_split) {
     } else {
         ps.bn = choose_bn(d_h, n_tok, M);
     }
+    // CTA pairs for d_h % 256 == 0: whole-K units when there are at least two waves of them;
+    // K split across pairs when even one wave of units would leave pairs idle (decode-sized
+    // batches), like the single-CTA split above but with each weight tile read by one pair
+    if (d_h % engram::kPairBN == 0 && !(plan->cfg.flags & ENGRAM_FLAG_SINGLE_CTA_MMA)) {
+        const int64_t mn2 = (n_tok + engram::kPairRows - 1) / engram::kPairRows * ((M + 1) * d_h / engram::kPairBN);
+        int sp = 0;
+        if (mn2 >= sms) {
+            sp = 1;
+        } else if (allow_split && mn2 > 0 && mn2 < sms / 2) {
+            sp = forced_splits ? forced_splits : static_cast<int>((sms / 2) / mn2);
+            if (sp > ps.k_blocks / 4) sp = ps.k_blocks / 4;
+            if (sp < 2) sp = 0;
+        }
+        if (sp > 0) {
+            ps.pair = true;
+            ps.bn = engram::kPairBN;
+            ps.kb_per_split = (ps.k_blocks + sp - 1) / sp;
+            ps.k_splits = (ps.k_blocks + ps.kb_per_split - 1) / ps.kb_per_split;
+        }
+    }
     ps.n_tiles = (M + 1) * d_h / ps.bn;
     return ps;
-}
-
-// The projection of whole-K tiles runs on CTA pairs (proj_pair_kernel, 256 x 256 units) when
-// d_h is a multiple of 256 and there are at least two units per pair of SMs.
-bool use_pair_mma(const engram_plan *plan, int64_t n_tok, const ProjShape &ps) {
-    if (ps.k_splits != 1 || plan->cfg.hidden_dim % engram::kPairBN != 0) return false;
-    if (plan->cfg.flags & ENGRAM_FLAG_SINGLE_CTA_MMA) return false;
-    const int64_t units = (n_tok + engram::kPairRows - 1) / engram::kPairRows *
-                          ((plan->num_branches + 1) * plan->cfg.hidden_dim / engram::kPairBN);
-    return units >= 148;
 }
 
 // Which kernels engram_forward runs for a batch of n_tok tokens (engram_forward_path).
@@ -239,7 +250,7 @@ ForwardPath forward_path(const engram_plan *plan, int64_t n_tok) {
     f.staged = plan->cfg.table_location == ENGRAM_TABLES_HOST_MAPPED && n_tok <= engram::kStageMaxTok;
     f.fused_lookup = !f.staged && plan->cfg.table_location == ENGRAM_TABLES_DEVICE &&
                      n_tok * plan->num_tables <= kFusedLookupMaxRows;
-    f.pair = use_pair_mma(plan, n_tok, f.ps);
+    f.pair = f.ps.pair;
     return f;
 }
 
@@ -383,12 +394,13 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     return ENGRAM_OK;
 }
 
+template <bool SPLIT>
 int set_pair_smem_attr() {
     static bool done[64] = {};
     int dev = 0;
     ENGRAM_CUDA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
     if (dev < 64 && done[dev]) return ENGRAM_OK;
-    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::proj_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    ENGRAM_CUDA_TRY(cudaFuncSetAttribute(engram::proj_pair_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          engram::PairCfg::kSmemBytes),
                     "cudaFuncSetAttribute(proj_pair_kernel)");
     if (dev < 64) done[dev] = true;
@@ -396,6 +408,7 @@ int set_pair_smem_attr() {
 }
 
 // CTA pairs that can be resident at once (one CTA per SM; a pair needs two SMs of one GPC).
+template <bool SPLIT>
 int max_pairs(int *out) {
     static int cached[64] = {};
     int dev = 0;
@@ -409,7 +422,7 @@ int max_pairs(int *out) {
     cfg.blockDim = dim3(engram::kProjThreads);
     cfg.dynamicSmemBytes = engram::PairCfg::kSmemBytes;
     int n = 0;
-    ENGRAM_CUDA_TRY(cudaOccupancyMaxActiveClusters(&n, engram::proj_pair_kernel, &cfg),
+    ENGRAM_CUDA_TRY(cudaOccupancyMaxActiveClusters(&n, engram::proj_pair_kernel<SPLIT>, &cfg),
                     "cudaOccupancyMaxActiveClusters(proj_pair_kernel)");
     if (n < 1) return fail(ENGRAM_ERR_CUDA, "no CTA pair of the projection fits on this device");
     if (dev < 64) cached[dev] = n;
@@ -417,9 +430,12 @@ int max_pairs(int *out) {
     return ENGRAM_OK;
 }
 
-// Whole-K projection on CTA pairs: 256-token x 256-channel units (see kernels_proj_pair.cuh).
+// Projection on CTA pairs: 256-token x 256-channel units (see kernels_proj_pair.cuh); with
+// k_splits > 1, K-split units writing raw partial accumulators to acc (finished like the
+// single-CTA split).
 int launch_proj_pair(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
-                     int64_t n_tok, uint16_t *v, float4 *part, cudaStream_t stream) {
+                     int64_t n_tok, uint16_t *v, float4 *part, cudaStream_t stream, float *acc, int k_splits,
+                     int kb_per_split, bool run_reduce, engram::ProjParams *params_out) {
     const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim, M = plan->num_branches;
     constexpr int BN = engram::kPairBN;
     CUtensorMap map_m, map_wk, map_wv;
@@ -445,9 +461,10 @@ int launch_proj_pair(const engram_plan *plan, const engram_weights *w, const uin
         if ((rc = make_map_bf16(&map_wv, w->w_v, d_h, d_m, BN / 2)) != ENGRAM_OK) return rc;
     }
     if ((rc = make_map_bf16(&map_m, m, static_cast<uint64_t>(n_tok), d_m, engram::kBM)) != ENGRAM_OK) return rc;
-    if ((rc = set_pair_smem_attr()) != ENGRAM_OK) return rc;
+    const bool split = acc != nullptr && k_splits > 1;
+    if ((rc = split ? set_pair_smem_attr<true>() : set_pair_smem_attr<false>()) != ENGRAM_OK) return rc;
     int pairs = 0;
-    if ((rc = max_pairs(&pairs)) != ENGRAM_OK) return rc;
+    if ((rc = split ? max_pairs<true>(&pairs) : max_pairs<false>(&pairs)) != ENGRAM_OK) return rc;
     engram::ProjParams p{};
     p.h = h;
     p.gamma_q = w->gamma_q;
@@ -461,10 +478,11 @@ int launch_proj_pair(const engram_plan *plan, const engram_weights *w, const uin
     p.M = M;
     p.k_blocks = (d_m + engram::kBK - 1) / engram::kBK;
     p.m_tiles = static_cast<int32_t>((n_tok + engram::kPairRows - 1) / engram::kPairRows);
-    p.k_splits = 1;
-    p.kb_per_split = p.k_blocks;
+    p.k_splits = split ? k_splits : 1;
+    p.kb_per_split = split ? kb_per_split : p.k_blocks;
+    p.acc_out = split ? acc : nullptr;
     p.w_packed = static_cast<const uint8_t *>(w->w_packed);
-    const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+    const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles * p.k_splits;
     if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
     // ENGRAM_PROJ_PAIRS (>= 1) caps the number of CTA pairs (tuning); read once per process.
     static const int forced_pairs = [] {
@@ -474,9 +492,16 @@ int launch_proj_pair(const engram_plan *plan, const engram_weights *w, const uin
     }();
     if (forced_pairs && forced_pairs < pairs) pairs = forced_pairs;
     const int64_t npairs = total < pairs ? total : pairs;
-    ENGRAM_CUDA_TRY(launch_pdl(engram::proj_pair_kernel, dim3(static_cast<unsigned>(2 * npairs)),
-                               dim3(engram::kProjThreads), engram::PairCfg::kSmemBytes, stream, map_m, map_wk, map_wv, p),
+    ENGRAM_CUDA_TRY(launch_pdl(split ? engram::proj_pair_kernel<true> : engram::proj_pair_kernel<false>,
+                               dim3(static_cast<unsigned>(2 * npairs)), dim3(engram::kProjThreads),
+                               engram::PairCfg::kSmemBytes, stream, map_m, map_wk, map_wv, p),
                     "proj_pair_kernel launch");
+    if (params_out) *params_out = p;
+    if (split && run_reduce) {
+        engram::splitk_reduce_kernel<<<dim3(p.n_tiles, static_cast<unsigned>(n_tok)), engram::kReduceThreads, 0,
+                                       stream>>>(p, BN);
+        ENGRAM_LAUNCHED("splitk_reduce_kernel launch");
+    }
     return ENGRAM_OK;
 }
 
@@ -803,10 +828,12 @@ int launch_stage_small(const engram_plan *plan, const int32_t *ids, const int32_
     sp.H = H;
     sp.capacity = capacity;
     sp.chunks_per_row = plan->cfg.row_dim * table_elem_bytes(plan) / 16;
+    // few CTAs with many 16-byte reads in flight each (8 per thread): enough to cover the host
+    // link's latency, while leaving the SMs to whatever the prefetch overlaps with
     const int64_t total = static_cast<int64_t>(H) * B * T * sp.chunks_per_row;
-    constexpr int kUnroll = 2;
+    constexpr int kUnroll = 8;
     int64_t blocks = (total + engram::kStageSmallThreads * kUnroll - 1) / (engram::kStageSmallThreads * kUnroll);
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 2;
+    const int64_t cap = static_cast<int64_t>(sm_count());
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     engram::stage_small_kernel<kUnroll><<<static_cast<unsigned>(blocks), engram::kStageSmallThreads, 0, stream>>>(
@@ -858,10 +885,10 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
     engram::ProjParams pp{};
     int rc;
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[0], stream), "cudaEventRecord");
-    const bool pair = use_pair_mma(plan, n_tok, ps);
-    const int n_tiles = pair ? (plan->num_branches + 1) * d_h / engram::kPairBN : ps.n_tiles;
-    if (pair)
-        rc = launch_proj_pair(plan, w, h, m, n_tok, v, part, stream);
+    const int n_tiles = ps.n_tiles;
+    if (ps.pair)
+        rc = launch_proj_pair(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode,
+                              &pp);
     else if (ps.bn == 256)
         rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
     else if (ps.bn == 128)

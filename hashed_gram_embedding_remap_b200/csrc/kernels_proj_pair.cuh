@@ -30,20 +30,26 @@ struct PairCfg {
     static constexpr int kStages = 6;
     static constexpr int kAccum = 2;
     static constexpr int kTmemCols = kAccum * kPairBN;        // 512: all of tensor memory
-    // dynamic smem: [align pad][stages x A][stages x B][full, empty, tmem_full, tmem_empty,
-    //               drain][tmem addr]
+    // dynamic smem: [align pad][stages x A][stages x B][split-K transpose tiles][full, empty,
+    //               tmem_full, tmem_empty, drain][tmem addr]
     static constexpr int kBarBytes = (2 * kStages + 2 * kAccum + 1) * 8;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 16;
+    static constexpr int kTrStride = 36;                          // split-K transpose (as ProjCfg)
+    static constexpr int kTrBytes = 4 * 32 * kTrStride * 4;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kTrBytes + kBarBytes + 16;
 };
 
 __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
-// p.m_tiles counts 256-token tiles; p.n_tiles = (M + 1) * d_h / 256; whole-K units only.
+// p.m_tiles counts 256-token tiles; p.n_tiles = (M + 1) * d_h / 256.  SPLIT: units are
+// (k split, 256-token tile, 256-channel slice), n fastest, and their raw fp32 partial
+// accumulators go to p.acc_out exactly as proj_kernel's split-K units write them (the rows of
+// each CTA through a per-warp shared-memory transpose), to be finished by the same kernels.
 // map_wk / map_wv: the row-major weights (boxes of 128 rows), or with packed weights map_wk
 // spans the packed copy as [tiles * k_blocks * 256 rows, 64 columns] (boxes of 128 rows, no
 // swizzle: the bytes are already in the tensor cores' layout) and map_wv is unused.
+template <bool SPLIT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads, 1)
     proj_pair_kernel(const __grid_constant__ CUtensorMap map_m, const __grid_constant__ CUtensorMap map_wk,
                      const __grid_constant__ CUtensorMap map_wv, const __grid_constant__ ProjParams p) {
@@ -55,7 +61,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + S * Cfg::kATile;
-    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes);
+    float *s_tr = reinterpret_cast<float *>(smem + S * Cfg::kStageBytes);
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + S * Cfg::kStageBytes + Cfg::kTrBytes);
     uint64_t *empty_bar = full_bar + S;
     uint64_t *tfull_bar = empty_bar + S;      // MMA -> epilogue of both CTAs
     uint64_t *tempty_bar = tfull_bar + NACC;  // epilogues of both CTAs -> MMA (even CTA's copy)
@@ -70,7 +77,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads, 1)
     const uint32_t rank = cluster_ctarank();   // 0: issues the MMAs; 1: its partner
     const int pair = blockIdx.x >> 1;
     const int npairs = gridDim.x >> 1;
-    const int total = p.m_tiles * p.n_tiles;   // units: (256-token tile, 256-channel slice), n fastest
+    const int mn_tiles = p.m_tiles * p.n_tiles;
+    const int total = mn_tiles * p.k_splits;   // units: (k split, 256-token tile, 256-channel slice), n fastest
+    // unit t -> (k split, 256-token tile, channel slice) and its k-block range
+    auto unit = [&](int t, int &ks, int &mt, int &nt, int &kb0, int &kb1) {
+        ks = t / mn_tiles;
+        const int tmn = t - ks * mn_tiles;
+        mt = tmn / p.n_tiles;
+        nt = tmn - mt * p.n_tiles;
+        kb0 = ks * p.kb_per_split;
+        kb1 = min(p.k_blocks, kb0 + p.kb_per_split);
+    };
     const int key_tiles = p.M * (p.d_h / BN);
     const int kpb = p.d_h / BN;
 
@@ -115,19 +132,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads, 1)
             };
             int pre = 0;
             if (pair < total) {   // weight tiles of the first stages: independent of the previous kernel
-                const int nt0 = pair % p.n_tiles;
-                pre = min(S, p.k_blocks);
+                int ks, mt, nt, kb0, kb1;
+                unit(pair, ks, mt, nt, kb0, kb1);
+                pre = min(S, kb1 - kb0);
                 for (int q = 0; q < pre; ++q) {
                     if (rank == 0) mbar_arrive_expect_tx(&full_bar[q], kTxBytes);
-                    load_b(q, nt0, q);
+                    load_b(q, nt, kb0 + q);
                 }
             }
             pdl_wait();
             int it = 0, issued = pre;
             for (int t = pair; t < total && !s_abort; t += npairs) {
-                const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
+                int ks, mt, nt, kb0, kb1;
+                unit(t, ks, mt, nt, kb0, kb1);
                 const int m0 = mt * kPairRows + static_cast<int>(rank) * kBM;
-                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     if (it < pre) {
                         tma_load_2d_pair(sA + s * Cfg::kATile, &map_m, full_cluster + s * 8, kb * kBK, m0);
@@ -158,8 +177,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads, 1)
                 if (!mbar_wait_cluster(&tempty_bar[acc], (use & 1) ^ 1, &s_abort, lim)) break;
                 tc_fence_after();
                 const uint32_t dst = tmem_base + acc * BN;
+                int ks, mt, nt, kb0, kb1;
+                unit(t, ks, mt, nt, kb0, kb1);
                 bool ok = true;
-                for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     if (!mbar_wait(&full_bar[s], (it / S) & 1, &s_abort, lim)) { ok = false; break; }
                     tc_fence_after();
@@ -168,7 +189,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads, 1)
 #pragma unroll
                     for (int k = 0; k < kBK / kUmmaK; ++k) {
                         const uint64_t koff = static_cast<uint64_t>((k * kUmmaK * 2) >> 4);
-                        umma_bf16_ss_pair(dst, adesc + koff, bdesc + koff, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                        umma_bf16_ss_pair(dst, adesc + koff, bdesc + koff, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
                     }
                     issued_any = true;
                     umma_commit_pair(&empty_bar[s], 0x3);   // frees stage s in both CTAs
@@ -203,23 +224,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads, 1)
             if (lane == 0) ok = mbar_wait_cluster(&tfull_bar[acc], use & 1, &s_abort, lim) && !s_abort;
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             tc_fence_after();
-            const int mt = t / p.n_tiles, nt = t - mt * p.n_tiles;
+            int ks, mt, nt, kb0, kb1;
+            unit(t, ks, mt, nt, kb0, kb1);
             const bool is_key = nt < key_tiles;
             const int br = is_key ? nt / kpb : 0;
             const int c0 = (is_key ? nt - br * kpb : nt - key_tiles) * BN;
-            const int64_t n = static_cast<int64_t>(mt) * kPairRows + static_cast<int>(rank) * kBM + row;
+            const int64_t rows0 = static_cast<int64_t>(mt) * kPairRows + static_cast<int>(rank) * kBM;
+            const int64_t n = rows0 + row;
             const bool valid = n < p.n_tok;
             const uint32_t taddr = tmem_base + acc * BN + (static_cast<uint32_t>(sub * 32) << 16);
             float a0 = 0.f, a1 = 0.f, a2 = 0.f;
             for (int cc = 0; cc < BN; cc += 32) {
                 float accv[32];
                 tmem_ld32(taddr + cc, accv);
+                if constexpr (SPLIT) {
+                    // raw partial accumulator, stored through the warp's 32 x 32 transpose tile so
+                    // that each store instruction writes whole 128-byte row segments
+                    float *tr = s_tr + sub * (32 * Cfg::kTrStride);
+                    float4 *mine = reinterpret_cast<float4 *>(tr + lane * Cfg::kTrStride);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        mine[q] = make_float4(accv[4 * q], accv[4 * q + 1], accv[4 * q + 2], accv[4 * q + 3]);
+                    __syncwarp();
+                    const int c4 = (lane & 7) * 4;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = i * 4 + (lane >> 3);
+                        const int64_t nr = rows0 + sub * 32 + r;
+                        if (nr < p.n_tok)
+                            *reinterpret_cast<float4 *>(p.acc_out + (static_cast<int64_t>(ks) * p.n_tok + nr) *
+                                                                        (p.n_tiles * BN) + nt * BN + cc + c4) =
+                                *reinterpret_cast<const float4 *>(tr + r * Cfg::kTrStride + c4);
+                    }
+                    __syncwarp();
+                    continue;
+                }
                 if (valid) epilogue_chunk(p, accv, n, br, c0 + cc, is_key, a0, a1, a2);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_tempty + acc * 8);   // to the even CTA's copy
-            if (valid) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
+            if constexpr (!SPLIT) {
+                if (valid) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
+            }
         }
     }
     tc_fence_before();

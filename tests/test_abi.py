@@ -224,7 +224,9 @@ def test_forward_path_selection():
     assert not P(_plan(hidden_dim=384), 8, 4096) & PAIR
     # decode-sized batches: one lookup kernel, split-K projection
     dec = synth.get_workload("decode20m")
-    assert P(E.Plan.from_workload(dec), dec.B, 1) == E.ENGRAM_PATH_FUSED_LOOKUP | E.ENGRAM_PATH_SPLIT_K
+    assert P(E.Plan.from_workload(dec), dec.B, 1) == E.ENGRAM_PATH_FUSED_LOOKUP | E.ENGRAM_PATH_SPLIT_K | PAIR
+    assert (P(E.Plan.from_workload(dec, flags=E.ENGRAM_FLAG_SINGLE_CTA_MMA), dec.B, 1)
+            == E.ENGRAM_PATH_FUSED_LOOKUP | E.ENGRAM_PATH_SPLIT_K)
     # host-mapped tables: distinct rows staged into HBM first
     hp = synth.get_workload("hostpinned20m")
     assert P(E.Plan.from_workload(hp, host_tables=True), hp.B, 1) & E.ENGRAM_PATH_STAGED_ROWS

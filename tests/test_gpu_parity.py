@@ -214,6 +214,31 @@ def test_pair_mma_bit_identical_to_single_cta(case, packed):
     assert E.engram_device_status(clear=True) == 0
 
 
+@pytest.mark.parametrize("B,d_h", [(256, 2560), (96, 512)])
+def test_pair_split_k_decode_bit_identical_to_single_cta(B, d_h):
+    """One-token decode steps whose projection splits K: on CTA pairs (256-token units, each
+    weight tile read by one pair) the partial accumulators, and so Delta, out, the conv state
+    and the hash history, equal the single-CTA kernel's bit for bit when both split K the same
+    number of ways."""
+    wl = small_workload("pair_dec", B=B, T=1, K=1, d_e=d_h, d_h=d_h, decode=True)
+    a = DeviceInputs(wl, random_gammas=True)
+    b = DeviceInputs(wl, tables=a.tables, flags=E.ENGRAM_FLAG_SINGLE_CTA_MMA, random_gammas=True)
+    pa, pb = E.engram_forward_path(a.plan, wl.B, 1), E.engram_forward_path(b.plan, wl.B, 1)
+    assert pa & E.ENGRAM_PATH_PAIR_MMA and pa & E.ENGRAM_PATH_SPLIT_K
+    assert not pb & E.ENGRAM_PATH_PAIR_MMA and pb & E.ENGRAM_PATH_SPLIT_K
+    for step in range(3):
+        ids = to_dev(synth.zipf_ids(wl.vocab_in, 1.1, (wl.B, 1), 700 + step))
+        a.ids = b.ids = ids
+        a.forward()
+        b.forward()
+        torch.cuda.synchronize()
+        assert torch.equal(a.delta, b.delta)
+        assert torch.equal(a.out.view(torch.int16), b.out.view(torch.int16))
+        assert torch.equal(a.conv_state.view(torch.int16), b.conv_state.view(torch.int16))
+        assert torch.equal(a.history, b.history)
+    assert E.engram_device_status(clear=True) == 0
+
+
 def test_kernel_launch_count_per_call():
     """The library's launch counter (bench.py's gpu_launches): a prefill call launches remap +
     hash, gather, projection, gate scalars and the streaming gate kernel (5); a one-token
@@ -234,7 +259,8 @@ def test_kernel_launch_count_per_call():
     assert E.kernel_launches() == n2
     dec = small_workload("dec_split", B=32, T=1, K=1, d_e=512, d_h=512, decode=True)
     dd = DeviceInputs(dec)
-    assert E.engram_forward_path(dd.plan, dec.B, 1) == E.ENGRAM_PATH_FUSED_LOOKUP | E.ENGRAM_PATH_SPLIT_K
+    assert E.engram_forward_path(dd.plan, dec.B, 1) & (E.ENGRAM_PATH_FUSED_LOOKUP | E.ENGRAM_PATH_SPLIT_K) == (
+        E.ENGRAM_PATH_FUSED_LOOKUP | E.ENGRAM_PATH_SPLIT_K)
     dd.forward()
     torch.cuda.synchronize()
     n0 = E.kernel_launches()

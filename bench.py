@@ -39,7 +39,7 @@ L2_BYTES = 126 * 2 ** 20
 def kernel_traffic(kernel: str, workload: str):
     """DRAM bytes per launch of `kernel` on `workload` from the committed ncu summary
     (profiles/traffic.json), or None when that summary was taken on a different version of
-    the kernel's source file than the one built here."""
+    the kernel's source files than the ones built here."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
@@ -47,9 +47,10 @@ def kernel_traffic(kernel: str, workload: str):
     entry = json.load(open(p)).get(kernel, {}).get(workload)
     if not entry:
         return None
-    src = os.path.join(ROOT, entry["source"])
-    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != entry["source_sha256"]:
-        return None
+    for rel, digest in entry["sources"].items():
+        src = os.path.join(ROOT, rel)
+        if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != digest:
+            return None
     return entry["dram_bytes_per_launch"]
 
 
@@ -580,7 +581,7 @@ def run_engram(args, wl, world, rank, local):
                           + "tcgen05 k/v projections + gate partials)",
                 "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s", "frac": tflops / peak_tf,
                 "frac_of_sustained": tflops / peaks["bf16_sus"],
-                "traffic": kernel_traffic("proj_kernel", wl.name),
+                "traffic": kernel_traffic("proj_pair_kernel" if pair else "proj_kernel", wl.name),
                 "peak_source": f"{peaks['source']} bf16 {'burst' if burst else 'sustained'} "
                                f"(timed region {timed_s:.2f} s)",
                 "algorithmic_per_launch": flops}

@@ -828,12 +828,20 @@ int launch_stage_small(const engram_plan *plan, const int32_t *ids, const int32_
     sp.H = H;
     sp.capacity = capacity;
     sp.chunks_per_row = plan->cfg.row_dim * table_elem_bytes(plan) / 16;
-    // few CTAs with many 16-byte reads in flight each (8 per thread): enough to cover the host
-    // link's latency, while leaving the SMs to whatever the prefetch overlaps with
+    // few CTAs with many 16-byte reads in flight each (16 per thread, 64 KB per CTA): enough to
+    // cover the host link's latency, while leaving the SMs to whatever the prefetch overlaps
+    // with (measured on a 64-token step over a 2560^3 GEMM: 8 CTAs hide the most; 16 or more
+    // shorten the prefetch a little but slow what it overlaps).  ENGRAM_STAGE_CTAS (>= 1)
+    // overrides the CTA count (tuning); read once per process.
+    static const int forced_ctas = [] {
+        const char *e = std::getenv("ENGRAM_STAGE_CTAS");
+        const int v = e ? std::atoi(e) : 0;
+        return v > 0 ? v : 0;
+    }();
     const int64_t total = static_cast<int64_t>(H) * B * T * sp.chunks_per_row;
-    constexpr int kUnroll = 8;
+    constexpr int kUnroll = 16;
     int64_t blocks = (total + engram::kStageSmallThreads * kUnroll - 1) / (engram::kStageSmallThreads * kUnroll);
-    const int64_t cap = static_cast<int64_t>(sm_count());
+    const int64_t cap = forced_ctas ? forced_ctas : 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     engram::stage_small_kernel<kUnroll><<<static_cast<unsigned>(blocks), engram::kStageSmallThreads, 0, stream>>>(

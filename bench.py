@@ -335,6 +335,80 @@ def l2_exceeded(wl) -> bool:
 
 
 # ---------------------------------------------------------------------------------------
+def measure_decode_steps(E, fill_gpu, plan, weights, tables, wl_dec, steps, warmup, stream, dev):
+    """One-token decode steps (wl_dec's batch, hash history and conv state carried from step to
+    step) through engram_forward on already-resident tables; L2 flushed between steps (outside
+    each step's events).  Returns per-step time, the CUDA-event stage breakdown and launches."""
+    B = wl_dec.B
+    hist = torch.from_numpy(wl_dec.history()).to(dev)
+    state = fill_gpu.filled((B, wl_dec.state_len, wl_dec.d_h), wl_dec.state_spec(), dev)
+    ids_all = torch.from_numpy(synth.zipf_ids(wl_dec.vocab_in, wl_dec.zipf_s, (warmup + steps, B, 1),
+                                              wl_dec.seeds()["ids"])).to(dev)
+    h = fill_gpu.filled((B, wl_dec.d_h), wl_dec.h_spec(0), dev)
+    out = torch.empty((B, wl_dec.d_h), dtype=torch.bfloat16, device=dev)
+    ws = E.alloc_workspace(plan, B, dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+    nst = E.ENGRAM_FORWARD_STAGES + 1
+
+    def step(k, evs=None):
+        E.engram_forward(plan, weights, tables, ids_all[k], h, out, ws, history=hist, conv_state=state,
+                         stream=stream, stage_events=evs)
+
+    for k in range(warmup):
+        step(k)
+    torch.cuda.synchronize()
+    n0 = E.kernel_launches()
+    step(0)
+    torch.cuda.synchronize()
+    launches = E.kernel_launches() - n0
+    # the K steps as one CUDA graph, as the main measurement does (no host launch gaps); a
+    # second graph of the same steps carries the per-stage events
+    se = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+          for _ in range(steps)]
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nst)] for _ in range(steps)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    for a, b in se:
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+
+    def capture(with_events):
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+            cs = torch.cuda.current_stream()
+            for k in range(steps):
+                flush.fill_(k)
+                if not with_events:
+                    se[k][0].record(cs)
+                E.engram_forward(plan, weights, tables, ids_all[warmup + k], h, out, ws, history=hist,
+                                 conv_state=state, stream=cs, stage_events=evs[k] if with_events else None)
+                if not with_events:
+                    se[k][1].record(cs)
+        stream.wait_stream(cap)
+        torch.cuda.synchronize()
+        return g
+
+    g_time, g_ev = capture(False), capture(True)
+    g_time.replay()   # upload
+    torch.cuda.synchronize()
+    g_time.replay()
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in se)
+    g_ev.replay()
+    torch.cuda.synchronize()
+    names = ["hash", "gather", "proj", "gate_conv"]
+    stages = {n: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(steps))
+              for i, n in enumerate(names)}
+    if E.engram_device_status(clear=True):
+        raise SystemExit("device status raised during the decode steps")
+    return {"ms_per_step": ms, "us_per_step": ms * 1e3, "tokens_per_s": B / (ms / 1e3), "stages_ms": stages,
+            "gpu_launches_per_step": launches, "path_bits": E.engram_forward_path(plan, B, 1)}
+
+
 def run_engram(args, wl, world, rank, local):
     import hashed_gram_embedding_remap_b200 as E
     from synth import fill_gpu
@@ -642,6 +716,15 @@ def run_engram(args, wl, world, rank, local):
                                                   "second replay of the same steps with event nodes)",
         "clocks": clocks.summary(t_host0, t_host1),
     }
+    # The decode workload's steps on the same resident tables (decode20m and prefill20m share
+    # the table geometry, the hash and the weights' shapes; only the seeded contents differ),
+    # so that one bench run also reports the decode step time.
+    if wl.name == "prefill20m" and not args.no_decode_steps:
+        wl_dec = synth.get_workload("decode20m")
+        dec = measure_decode_steps(E, fill_gpu, plan, weights, tables, wl_dec, max(args.steps, 20),
+                                   max(args.warmup, 3), stream, dev)
+        dec["workload"] = "decode20m shapes (256 sequences x 1 token, history and conv state) on the prefill20m tables"
+        line["decode_steps"] = dec
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -887,6 +970,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["engram", "reference"], default="engram")
     ap.add_argument("--workload", default="prefill20m", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-decode-steps", action="store_true",
+                    help="prefill20m: skip timing decode20m's steps on the same tables after the main line")
     ap.add_argument("--single-cta-mma", action="store_true",
                     help="never pair CTAs for the projection's MMAs (ENGRAM_FLAG_SINGLE_CTA_MMA)")
     ap.add_argument("--oracle-tokens", type=int, default=128)

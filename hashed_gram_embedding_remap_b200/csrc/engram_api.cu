@@ -889,7 +889,8 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
     const int d_h = plan->cfg.hidden_dim;
     // one-token decode steps after a split-K projection: reduce + gate + conv in one kernel
     const bool fused_decode = ps.k_splits > 1 && T == 1 && plan->num_branches == 1 && plan->cfg.conv_kernel == 4 &&
-                              plan->cfg.conv_dilation == 3 && d_h <= 2 * engram::kFusedDecodeThreads * engram::kFusedDecodeMaxPairs;
+                              plan->cfg.conv_dilation == 3 && d_h <= 8 * engram::kFusedDecodeMaxThreads &&
+                              d_h % 256 == 0;   // d_h / 8 threads: whole warps
     engram::ProjParams pp{};
     int rc;
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[0], stream), "cudaEventRecord");
@@ -912,14 +913,9 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
             gp.xr = xr;
             gp.hist_len = plan->hist_len;
         }
-        using DK = void (*)(const engram::ProjParams, const engram::GateParams);
-        static const DK kernels[engram::kFusedDecodeMaxPairs] = {
-            engram::decode_fused_kernel<1>, engram::decode_fused_kernel<2>, engram::decode_fused_kernel<3>,
-            engram::decode_fused_kernel<4>, engram::decode_fused_kernel<5>, engram::decode_fused_kernel<6>,
-            engram::decode_fused_kernel<7>, engram::decode_fused_kernel<8>};
-        const int pairs = (d_h / 2 + engram::kFusedDecodeThreads - 1) / engram::kFusedDecodeThreads;
-        ENGRAM_CUDA_TRY(launch_pdl(kernels[pairs - 1], dim3(static_cast<unsigned>(B)), dim3(engram::kFusedDecodeThreads),
-                                   0, stream, pp, gp),
+        ENGRAM_CUDA_TRY(launch_pdl(d_h <= 8 * 320 ? engram::decode_fused_kernel<320>
+                                                  : engram::decode_fused_kernel<engram::kFusedDecodeMaxThreads>,
+                                   dim3(static_cast<unsigned>(B)), dim3(d_h / 8), 0, stream, pp, gp),
                         "decode_fused_kernel launch");
         ENGRAM_CUDA_TRY(cudaGetLastError(), "decode_fused_kernel launch");
         if (history_done) *history_done = gp.history != nullptr;

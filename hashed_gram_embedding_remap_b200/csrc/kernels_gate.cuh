@@ -442,6 +442,77 @@ __device__ __forceinline__ float2 silu2(float2 x) {
     return __ffma2_rn(h, t, h);
 }
 
+// One thread's walk over its CTA's tokens (see gate_stream_kernel).  FULL: the CTA's chunk is
+// whole (t1 == t0 + 9G), so no token of the walk needs a bounds check.  Each load and store
+// address advances by a fixed stride per token instead of being recomputed.
+template <int G, bool DELTA, bool FULL>
+__device__ __forceinline__ void gate_stream_walk(const GateParams &p, const float2 *s_sc, const float2 (&w)[4][2],
+                                                 const uint16_t *vbase, const uint16_t *hbase, uint16_t *obase,
+                                                 float *dbase, int lo, int t0, int t1) {
+    constexpr int R = 9;
+    const int64_t vstride = p.d_h;                               // elements per token of v
+    const int64_t hstride = static_cast<int64_t>(p.M) * p.d_h;   // h / out / delta token stride
+    uint2 lv[R], lh[R];     // load ring: (v, h) of the token in each slot
+    float2 ur[R][2];        // conv-input ring: u' of the last 9 positions, slot = position mod 9
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+        const int t = lo + j;   // halo: conv inputs only
+        lv[j] = (t >= 0) ? __ldg(reinterpret_cast<const uint2 *>(vbase + static_cast<int64_t>(t) * vstride))
+                         : make_uint2(0u, 0u);
+        lh[j] = make_uint2(0u, 0u);
+        ur[j][0] = ur[j][1] = make_float2(0.f, 0.f);
+    }
+    // next tokens to load: t0 (the first output token) onwards
+    const uint16_t *vp = vbase + static_cast<int64_t>(t0) * vstride;
+    const uint16_t *hp = hbase + static_cast<int64_t>(t0) * hstride;
+    uint16_t *op = obase + static_cast<int64_t>(t0) * hstride;
+    float *dp = DELTA ? dbase + static_cast<int64_t>(t0) * hstride : nullptr;
+#pragma unroll 1
+    for (int gi = 0; gi <= G; ++gi) {
+        const int tb = lo + R * gi;
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+            const int t = tb + j;
+            const uint2 vw = lv[j], hw = lh[j];
+            // refill the slot with token t + 9 (the next group)
+            if (gi < G) {
+                const bool in = FULL || t + R < t1;
+                lv[j] = in ? __ldg(reinterpret_cast<const uint2 *>(vp)) : make_uint2(0u, 0u);
+                lh[j] = in ? __ldg(reinterpret_cast<const uint2 *>(hp)) : make_uint2(0u, 0u);
+                vp += vstride;
+                hp += hstride;
+            }
+            const float2 sc = s_sc[t - lo];
+            const float2 vj[2] = {half2_to_f2(vw.x), half2_to_f2(vw.y)};
+            const float2 un[2] = {__fmul2_rn(f2(sc.y), vj[0]), __fmul2_rn(f2(sc.y), vj[1])};
+            if (gi > 0) {
+                if (FULL || t < t1) {
+                    const uint32_t hh[2] = {hw.x, hw.y};
+                    float2 dl[2];
+                    uint32_t ob[2];
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        float2 acc = __fmul2_rn(w[0][k], un[k]);
+                        acc = __ffma2_rn(w[1][k], ur[(j + 6) % R][k], acc);   // t - 3
+                        acc = __ffma2_rn(w[2][k], ur[(j + 3) % R][k], acc);   // t - 6
+                        acc = __ffma2_rn(w[3][k], ur[j][k], acc);             // t - 9
+                        dl[k] = __ffma2_rn(f2(sc.x), vj[k], silu2(acc));     // U + SiLU(conv)
+                        const float2 o = __fadd2_rn(bf162_to_f2(hh[k]), dl[k]);
+                        ob[k] = pack_bf16x2(o.x, o.y);
+                    }
+                    *reinterpret_cast<uint2 *>(op) = make_uint2(ob[0], ob[1]);
+                    if constexpr (DELTA)
+                        *reinterpret_cast<float4 *>(dp) = make_float4(dl[0].x, dl[0].y, dl[1].x, dl[1].y);
+                }
+                op += hstride;
+                if constexpr (DELTA) dp += hstride;
+            }
+            ur[j][0] = un[0];
+            ur[j][1] = un[1];
+        }
+    }
+}
+
 template <int G, bool DELTA>
 __global__ void __launch_bounds__(kStreamThreads, kStreamMinBlocks) gate_stream_kernel(const __grid_constant__ GateParams p) {
     constexpr int R = 9;                       // ring length = conv halo (kernel 4, dilation 3)
@@ -477,63 +548,13 @@ __global__ void __launch_bounds__(kStreamThreads, kStreamMinBlocks) gate_stream_
         w[2][k] = make_float2(bf16_lo(ww.y) * g0, bf16_lo(ww.w) * g1);
         w[3][k] = make_float2(bf16_hi(ww.y) * g0, bf16_hi(ww.w) * g1);
     }
-    const int64_t hstride = static_cast<int64_t>(p.M) * p.d_h;   // h / out / delta token stride
     const uint16_t *vbase = p.v + row0 * p.d_h + c;
     const int64_t hoff = (row0 * p.M + br) * p.d_h + c;
-    const uint16_t *hbase = p.h + hoff;
-    uint16_t *obase = p.out + hoff;
-
-    uint2 lv[R], lh[R];     // load ring: (v, h) of the token in each slot
-    float2 ur[R][2];        // conv-input ring: u' of the last 9 positions, slot = position mod 9
-#pragma unroll
-    for (int j = 0; j < R; ++j) {
-        const int t = lo + j;   // halo: conv inputs only
-        lv[j] = (t >= 0) ? __ldg(reinterpret_cast<const uint2 *>(vbase + static_cast<int64_t>(t) * p.d_h))
-                         : make_uint2(0u, 0u);
-        lh[j] = make_uint2(0u, 0u);
-        ur[j][0] = ur[j][1] = make_float2(0.f, 0.f);
-    }
-#pragma unroll 1
-    for (int gi = 0; gi <= G; ++gi) {
-        const int tb = lo + R * gi;
-#pragma unroll
-        for (int j = 0; j < R; ++j) {
-            const int t = tb + j;
-            const uint2 vw = lv[j], hw = lh[j];
-            // refill the slot with token t + 9 (the next group)
-            const int tn = t + R;
-            if (gi < G) {
-                lv[j] = (tn < t1) ? __ldg(reinterpret_cast<const uint2 *>(vbase + static_cast<int64_t>(tn) * p.d_h))
-                                  : make_uint2(0u, 0u);
-                lh[j] = (tn < t1) ? __ldg(reinterpret_cast<const uint2 *>(hbase + static_cast<int64_t>(tn) * hstride))
-                                  : make_uint2(0u, 0u);
-            }
-            const float2 sc = s_sc[t - lo];
-            const float2 vj[2] = {half2_to_f2(vw.x), half2_to_f2(vw.y)};
-            const float2 un[2] = {__fmul2_rn(f2(sc.y), vj[0]), __fmul2_rn(f2(sc.y), vj[1])};
-            if (gi > 0 && t < t1) {
-                const uint32_t hh[2] = {hw.x, hw.y};
-                float2 dl[2];
-                uint32_t ob[2];
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    float2 acc = __fmul2_rn(w[0][k], un[k]);
-                    acc = __ffma2_rn(w[1][k], ur[(j + 6) % R][k], acc);   // t - 3
-                    acc = __ffma2_rn(w[2][k], ur[(j + 3) % R][k], acc);   // t - 6
-                    acc = __ffma2_rn(w[3][k], ur[j][k], acc);             // t - 9
-                    dl[k] = __ffma2_rn(f2(sc.x), vj[k], silu2(acc));     // U + SiLU(conv)
-                    const float2 o = __fadd2_rn(bf162_to_f2(hh[k]), dl[k]);
-                    ob[k] = pack_bf16x2(o.x, o.y);
-                }
-                const int64_t off = static_cast<int64_t>(t) * hstride;
-                *reinterpret_cast<uint2 *>(obase + off) = make_uint2(ob[0], ob[1]);
-                if constexpr (DELTA)
-                    *reinterpret_cast<float4 *>(p.delta + hoff + off) = make_float4(dl[0].x, dl[0].y, dl[1].x, dl[1].y);
-            }
-            ur[j][0] = un[0];
-            ur[j][1] = un[1];
-        }
-    }
+    float *dbase = DELTA ? p.delta + hoff : nullptr;
+    if (t1 - t0 == TC)
+        gate_stream_walk<G, DELTA, true>(p, s_sc, w, vbase, p.h + hoff, p.out + hoff, dbase, lo, t0, t1);
+    else
+        gate_stream_walk<G, DELTA, false>(p, s_sc, w, vbase, p.h + hoff, p.out + hoff, dbase, lo, t0, t1);
 }
 
 // Decode step (T = 1) with a carried conv state, kernel 4 / dilation 3: the conv taps of the
@@ -624,50 +645,42 @@ __global__ void __launch_bounds__(kDecodeThreads) gate_conv_decode_kernel(const 
 // Decode step (T = 1) after a split-K projection, fully fused: one CTA per token sums the
 // k_splits partial accumulators of its [k~ | v] row, reduces S0..S3 across the block, then
 // applies gate, conv (kernel 4, dilation 3, taps from the carried state or zeros), SiLU,
-// residual and the state shift.  Replaces splitk_reduce_kernel + the gate kernel for decode.
-// P channel pairs per thread (d_h <= 2 * 256 * P): every load of the token -- split
-// accumulators, h, gains, conv taps, the 9 carried state slots -- is issued in one round
-// trip; P is the smallest that covers d_h, so the registers allow two CTAs per SM and a
-// decode batch of up to 2 x #SMs tokens runs in one wave.
-constexpr int kFusedDecodeThreads = 256;
-constexpr int kFusedDecodeMaxPairs = 8;   // d_h <= 2 * 256 * 8 = 4096
+// residual and the state shift, and advances the token's hash history.  Replaces
+// splitk_reduce_kernel + the gate kernel for decode.  d_h / 8 threads, 8 consecutive channels
+// each, so that every access is 16 bytes wide (the 9 carried state slots, h, the gains, the
+// taps, out and the new state as bf16 x 8; the split accumulators as fp32 x 4): about 25 wide
+// loads per thread in one round trip, instead of ~80 narrow ones, which the load queues
+// throttled.
+constexpr int kFusedDecodeMaxThreads = 512;   // d_h <= 8 * 512 = 4096
+// MAXT: the largest block this instantiation runs; 320 (d_h <= 2560) keeps two CTAs per SM
+// (<= 102 registers), so a 256-sequence decode step runs in one wave.
 
-template <int P>
-__global__ void __launch_bounds__(kFusedDecodeThreads, 2) decode_fused_kernel(const __grid_constant__ ProjParams pp,
-                                                                              const __grid_constant__ GateParams p) {
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &w, float (&f)[8]) {
+    f[0] = bf16_lo(w.x); f[1] = bf16_hi(w.x); f[2] = bf16_lo(w.y); f[3] = bf16_hi(w.y);
+    f[4] = bf16_lo(w.z); f[5] = bf16_hi(w.z); f[6] = bf16_lo(w.w); f[7] = bf16_hi(w.w);
+}
+
+template <int MAXT>
+__global__ void __launch_bounds__(MAXT, MAXT <= 320 ? 2 : 1) decode_fused_kernel(const __grid_constant__ ProjParams pp,
+                                                                                const __grid_constant__ GateParams p) {
     constexpr int S = 9;
-    __shared__ float s_red[4][kFusedDecodeThreads / 32];
+    __shared__ float s_red[4][MAXT / 32];
     __shared__ float s_gb[2];
     // dependents (the next step's kernels) may be scheduled now; the hash history, when given,
     // is advanced below by this kernel itself, after pdl_wait
     pdl_launch_dependents();
     const int b = blockIdx.x;
     const int d_h = p.d_h;
+    const int c = threadIdx.x * 8;   // blockDim.x == d_h / 8, a multiple of 32
     const int64_t split_stride = pp.n_tok * (2 * d_h);
-    const float *acc = pp.acc_out + static_cast<int64_t>(b) * (2 * d_h);
-    float2 v[P];
-    uint32_t hv[P], st[P][S];
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    // the carried state and h first (independent of the splits), then the split accumulators
-    // one split at a time across all pairs: k_splits round trips in total.  The gains and
-    // conv taps (the same for every token, L2-resident) are read after the reduction.
-    float2 kt[P];
+    const float *acc = pp.acc_out + static_cast<int64_t>(b) * (2 * d_h) + c;
+    // the carried state and h first (independent of the splits)
+    uint4 st[S];
+    uint16_t *state = p.conv_state != nullptr ? p.conv_state + static_cast<int64_t>(b) * S * d_h + c : nullptr;
 #pragma unroll
-    for (int k = 0; k < P; ++k) {
-        const int c = 2 * (threadIdx.x + k * kFusedDecodeThreads);
-        v[k] = kt[k] = make_float2(0.f, 0.f);
-        hv[k] = 0;
-#pragma unroll
-        for (int j = 0; j < S; ++j) st[k][j] = 0;
-        if (c < d_h) {
-            if (p.conv_state != nullptr) {
-                const uint16_t *state = p.conv_state + static_cast<int64_t>(b) * S * d_h + c;
-#pragma unroll
-                for (int j = 0; j < S; ++j) st[k][j] = *reinterpret_cast<const uint32_t *>(state + j * d_h);
-            }
-            hv[k] = __ldg(reinterpret_cast<const uint32_t *>(pp.h + static_cast<int64_t>(b) * d_h + c));
-        }
-    }
+    for (int j = 0; j < S; ++j)
+        st[j] = state != nullptr ? *reinterpret_cast<const uint4 *>(state + j * d_h) : make_uint4(0, 0, 0, 0);
+    const uint4 hw = __ldg(reinterpret_cast<const uint4 *>(pp.h + static_cast<int64_t>(b) * d_h + c));
     pdl_wait();   // the split accumulators come from the projection kernel before this one
     if (p.history != nullptr && threadIdx.x == 0) {
         // the step's hash history update (T = 1): drop the oldest id, append this step's.
@@ -676,33 +689,29 @@ __global__ void __launch_bounds__(kFusedDecodeThreads, 2) decode_fused_kernel(co
         for (int s = 0; s + 1 < p.hist_len; ++s) hb[s] = hb[s + 1];
         hb[p.hist_len - 1] = p.xr[b];
     }
+    float kt[8], v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) kt[e] = v[e] = 0.f;
     for (int ks = 0; ks < pp.k_splits; ++ks) {
-        const float *src = acc + ks * split_stride;
-#pragma unroll
-        for (int k = 0; k < P; ++k) {
-            const int c = 2 * (threadIdx.x + k * kFusedDecodeThreads);
-            if (c < d_h) {
-                const float2 x = __ldg(reinterpret_cast<const float2 *>(src + c));
-                const float2 y = __ldg(reinterpret_cast<const float2 *>(src + d_h + c));
-                kt[k].x += x.x;
-                kt[k].y += x.y;
-                v[k].x += y.x;
-                v[k].y += y.y;
-            }
-        }
+        const float4 *src = reinterpret_cast<const float4 *>(acc + ks * split_stride);
+        const float4 k0 = __ldg(src), k1 = __ldg(src + 1);
+        const float4 v0 = __ldg(src + d_h / 4), v1 = __ldg(src + d_h / 4 + 1);
+        kt[0] += k0.x; kt[1] += k0.y; kt[2] += k0.z; kt[3] += k0.w;
+        kt[4] += k1.x; kt[5] += k1.y; kt[6] += k1.z; kt[7] += k1.w;
+        v[0] += v0.x; v[1] += v0.y; v[2] += v0.z; v[3] += v0.w;
+        v[4] += v1.x; v[5] += v1.y; v[6] += v1.z; v[7] += v1.w;
     }
+    float hf[8], gq[8], gk[8];
+    bf16x8_to_f32(hw, hf);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(pp.gamma_q + c)), gq);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(pp.gamma_k + c)), gk);
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-    for (int k = 0; k < P; ++k) {
-        const int c = 2 * (threadIdx.x + k * kFusedDecodeThreads);
-        if (c < d_h) {
-            const uint32_t qw = __ldg(reinterpret_cast<const uint32_t *>(pp.gamma_q + c));
-            const uint32_t kw = __ldg(reinterpret_cast<const uint32_t *>(pp.gamma_k + c));
-            const float h0 = bf16_lo(hv[k]), h1 = bf16_hi(hv[k]);
-            a0 = fmaf(h0, h0, fmaf(h1, h1, a0));
-            a1 = fmaf(h0 * bf16_lo(qw) * bf16_lo(kw), kt[k].x, fmaf(h1 * bf16_hi(qw) * bf16_hi(kw), kt[k].y, a1));
-            a2 = fmaf(kt[k].x, kt[k].x, fmaf(kt[k].y, kt[k].y, a2));
-            a3 = fmaf(v[k].x, v[k].x, fmaf(v[k].y, v[k].y, a3));
-        }
+    for (int e = 0; e < 8; ++e) {
+        a0 = fmaf(hf[e], hf[e], a0);
+        a1 = fmaf(hf[e] * gq[e] * gk[e], kt[e], a1);
+        a2 = fmaf(kt[e], kt[e], a2);
+        a3 = fmaf(v[e], v[e], a3);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -721,7 +730,7 @@ __global__ void __launch_bounds__(kFusedDecodeThreads, 2) decode_fused_kernel(co
     __syncthreads();
     if (threadIdx.x == 0) {
         float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-        for (int w = 0; w < kFusedDecodeThreads / 32; ++w) {
+        for (int w = 0; w < static_cast<int>(blockDim.x / 32); ++w) {
             s0 += s_red[0][w];
             s1 += s_red[1][w];
             s2 += s_red[2][w];
@@ -736,33 +745,43 @@ __global__ void __launch_bounds__(kFusedDecodeThreads, 2) decode_fused_kernel(co
     }
     __syncthreads();
     const float g = s_gb[0], beta = s_gb[1];
+    float gc[8], s6[8], s3f[8], s0f[8];
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(p.gamma_c + c)), gc);
+    bf16x8_to_f32(st[6], s6);    // position t-3
+    bf16x8_to_f32(st[3], s3f);   // t-6
+    bf16x8_to_f32(st[0], s0f);   // t-9
+    const uint4 *wp = reinterpret_cast<const uint4 *>(p.conv_w + c * 4);   // 8 channels x 4 taps
+    float u[8], d[8];
 #pragma unroll
-    for (int k = 0; k < P; ++k) {
-        const int c = 2 * (threadIdx.x + k * kFusedDecodeThreads);
-        if (c >= d_h) continue;
-        const uint32_t gwk = __ldg(reinterpret_cast<const uint32_t *>(p.gamma_c + c));
-        const uint2 w0k = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + c * 4));
-        const uint2 w1k = __ldg(reinterpret_cast<const uint2 *>(p.conv_w + (c + 1) * 4));
-        const float u0 = beta * v[k].x * bf16_lo(gwk), u1 = beta * v[k].y * bf16_hi(gwk);
-        // taps: i = 0 current, 1 -> slot 6 (t-3), 2 -> slot 3 (t-6), 3 -> slot 0 (t-9)
-        const float c0 = fmaf(bf16_lo(w0k.x), u0, fmaf(bf16_hi(w0k.x), bf16_lo(st[k][6]),
-                         fmaf(bf16_lo(w0k.y), bf16_lo(st[k][3]), bf16_hi(w0k.y) * bf16_lo(st[k][0]))));
-        const float c1 = fmaf(bf16_lo(w1k.x), u1, fmaf(bf16_hi(w1k.x), bf16_hi(st[k][6]),
-                         fmaf(bf16_lo(w1k.y), bf16_hi(st[k][3]), bf16_hi(w1k.y) * bf16_hi(st[k][0]))));
-        const float d0 = fmaf(g, v[k].x, c0 * fast_sigmoid(c0));
-        const float d1 = fmaf(g, v[k].y, c1 * fast_sigmoid(c1));
-        const uint32_t o = static_cast<uint32_t>(f32_to_bf16_bits(bf16_lo(hv[k]) + d0)) |
-                           (static_cast<uint32_t>(f32_to_bf16_bits(bf16_hi(hv[k]) + d1)) << 16);
-        *reinterpret_cast<uint32_t *>(p.out + static_cast<int64_t>(b) * d_h + c) = o;
-        if (p.delta != nullptr)
-            *reinterpret_cast<float2 *>(p.delta + static_cast<int64_t>(b) * d_h + c) = make_float2(d0, d1);
-        if (p.conv_state != nullptr) {
-            uint16_t *state = p.conv_state + static_cast<int64_t>(b) * S * d_h + c;
+    for (int q = 0; q < 4; ++q) {   // channel pairs
+        const uint4 ww = __ldg(wp + q);   // taps of channels c + 2q (x, y) and c + 2q + 1 (z, w)
+        const float w0[4] = {bf16_lo(ww.x), bf16_hi(ww.x), bf16_lo(ww.y), bf16_hi(ww.y)};
+        const float w1[4] = {bf16_lo(ww.z), bf16_hi(ww.z), bf16_lo(ww.w), bf16_hi(ww.w)};
 #pragma unroll
-            for (int j = 0; j < S - 1; ++j) *reinterpret_cast<uint32_t *>(state + j * d_h) = st[k][j + 1];
-            *reinterpret_cast<uint32_t *>(state + (S - 1) * d_h) =
-                static_cast<uint32_t>(f32_to_bf16_bits(u0)) | (static_cast<uint32_t>(f32_to_bf16_bits(u1)) << 16);
+        for (int e2 = 0; e2 < 2; ++e2) {
+            const int e = 2 * q + e2;
+            const float *w = e2 == 0 ? w0 : w1;
+            u[e] = beta * v[e] * gc[e];
+            const float cv = fmaf(w[0], u[e], fmaf(w[1], s6[e], fmaf(w[2], s3f[e], w[3] * s0f[e])));
+            d[e] = fmaf(g, v[e], cv * fast_sigmoid(cv));
         }
+    }
+    uint4 o;
+    o.x = pack_bf16x2(hf[0] + d[0], hf[1] + d[1]);
+    o.y = pack_bf16x2(hf[2] + d[2], hf[3] + d[3]);
+    o.z = pack_bf16x2(hf[4] + d[4], hf[5] + d[5]);
+    o.w = pack_bf16x2(hf[6] + d[6], hf[7] + d[7]);
+    *reinterpret_cast<uint4 *>(p.out + static_cast<int64_t>(b) * d_h + c) = o;
+    if (p.delta != nullptr) {
+        float4 *dp = reinterpret_cast<float4 *>(p.delta + static_cast<int64_t>(b) * d_h + c);
+        dp[0] = make_float4(d[0], d[1], d[2], d[3]);
+        dp[1] = make_float4(d[4], d[5], d[6], d[7]);
+    }
+    if (state != nullptr) {
+#pragma unroll
+        for (int j = 0; j < S - 1; ++j) *reinterpret_cast<uint4 *>(state + j * d_h) = st[j + 1];
+        *reinterpret_cast<uint4 *>(state + (S - 1) * d_h) =
+            make_uint4(pack_bf16x2(u[0], u[1]), pack_bf16x2(u[2], u[3]), pack_bf16x2(u[4], u[5]), pack_bf16x2(u[6], u[7]));
     }
 }
 

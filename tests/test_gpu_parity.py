@@ -291,7 +291,7 @@ def test_gate_conv_entry_matches_forward():
     assert torch.equal(out_fwd.view(torch.int16), out2.view(torch.int16))
 
 
-@pytest.mark.parametrize("geom", ["small", "splitk", "splitk_256seq", "splitk_d2560", "chunk4"])
+@pytest.mark.parametrize("geom", ["small", "splitk", "splitk_256seq", "splitk_d2560", "splitk_d384", "chunk4"])
 def test_decode_steps_match_oracle_and_update_state(geom):
     """Consecutive calls carrying the hash history and conv state: one token per call
     (one-token decode kernels, with and without split-K, over one and two 128-token tiles,
@@ -303,6 +303,8 @@ def test_decode_steps_match_oracle_and_update_state(geom):
         wl = small_workload("dec_split", B=32, T=1, K=1, d_e=512, d_h=512, decode=True)
     elif geom == "splitk_256seq":
         wl = small_workload("dec_256", B=256, T=1, K=1, d_e=512, d_h=512, decode=True)
+    elif geom == "splitk_d384":   # split K, d_h not a multiple of 256: split reduce + decode gate kernels
+        wl = small_workload("dec_384", B=64, T=1, K=1, d_e=512, d_h=384, decode=True)
     elif geom == "splitk_d2560":
         wl = small_workload("dec_2560", B=200, T=1, K=1, d_e=2560, d_h=2560, decode=True)
     else:

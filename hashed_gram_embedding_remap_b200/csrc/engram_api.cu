@@ -125,11 +125,15 @@ struct Workspace {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Launch with programmatic stream serialization: the kernel may start while the previous
-// kernel on the stream finishes (see pdl_wait / pdl_launch_dependents).
+// Launch with programmatic stream serialization (pdl = true): the kernel may start while the
+// previous kernel on the stream finishes (see pdl_wait / pdl_launch_dependents).  Only a
+// kernel whose predecessor belongs to the same entry-point call is launched that way: the
+// kernels before pdl_wait read inputs (weights, conv state, h) that an earlier call's kernels
+// may still be writing if they were let run alongside, so the first kernel of each call
+// waits for everything before it.
 template <typename... Params, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                       Args &&...args) {
+cudaError_t launch_ex(bool pdl, void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                      Args &&...args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -139,10 +143,16 @@ cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t 
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 1 : 0;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
     if (e == cudaSuccess) g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
     return e;
+}
+
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args) {
+    return launch_ex(true, kernel, grid, block, smem, stream, std::forward<Args>(args)...);
 }
 
 bool fp8_tables(const engram_plan *plan) { return plan->cfg.table_dtype == ENGRAM_TABLE_FP8_E4M3; }
@@ -348,7 +358,7 @@ template <int BN>
 int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                 int64_t n_tok, uint16_t *v, float4 *part, cudaStream_t stream, float *acc = nullptr,
                 int k_splits = 1, int kb_per_split = 0, bool run_reduce = true,
-                engram::ProjParams *params_out = nullptr, const ProjTest &test = ProjTest()) {
+                engram::ProjParams *params_out = nullptr, const ProjTest &test = ProjTest(), bool pdl = true) {
     const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim;
     CUtensorMap map_m, map_wk, map_wv;
     int rc;
@@ -381,7 +391,7 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
     const int64_t sms = sm_count();
     dim3 grid(static_cast<unsigned>(total < sms ? total : sms));
-    ENGRAM_CUDA_TRY(launch_pdl(split ? engram::proj_kernel<BN, true> : engram::proj_kernel<BN, false>, grid,
+    ENGRAM_CUDA_TRY(launch_ex(pdl, split ? engram::proj_kernel<BN, true> : engram::proj_kernel<BN, false>, grid,
                                dim3(engram::kProjThreads), engram::ProjCfg<BN>::kSmemBytes, stream, map_m, map_wk,
                                map_wv, p),
                     "proj_kernel launch");
@@ -435,7 +445,7 @@ int max_pairs(int *out) {
 // single-CTA split).
 int launch_proj_pair(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                      int64_t n_tok, uint16_t *v, float4 *part, cudaStream_t stream, float *acc, int k_splits,
-                     int kb_per_split, bool run_reduce, engram::ProjParams *params_out) {
+                     int kb_per_split, bool run_reduce, engram::ProjParams *params_out, bool pdl) {
     const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim, M = plan->num_branches;
     constexpr int BN = engram::kPairBN;
     CUtensorMap map_m, map_wk, map_wv;
@@ -492,7 +502,7 @@ int launch_proj_pair(const engram_plan *plan, const engram_weights *w, const uin
     }();
     if (forced_pairs && forced_pairs < pairs) pairs = forced_pairs;
     const int64_t npairs = total < pairs ? total : pairs;
-    ENGRAM_CUDA_TRY(launch_pdl(split ? engram::proj_pair_kernel<true> : engram::proj_pair_kernel<false>,
+    ENGRAM_CUDA_TRY(launch_ex(pdl, split ? engram::proj_pair_kernel<true> : engram::proj_pair_kernel<false>,
                                dim3(static_cast<unsigned>(2 * npairs)), dim3(engram::kProjThreads),
                                engram::PairCfg::kSmemBytes, stream, map_m, map_wk, map_wv, p),
                     "proj_pair_kernel launch");
@@ -875,9 +885,11 @@ cudaError_t record_stage_event(void *ev, cudaStream_t stream) {
 
 // history / xr (engram_forward's decode steps): when the step ends in decode_fused_kernel, that
 // kernel also advances the hash history and *history_done is set; otherwise the caller does.
+// in_call: the kernel before the projection belongs to the same entry-point call (engram_forward),
+// so the projection may overlap it (launch_ex).
 int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                    int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out, float *delta, uint8_t *ws,
-                   cudaStream_t stream, void *const *events, int32_t *history = nullptr,
+                   cudaStream_t stream, void *const *events, bool in_call, int32_t *history = nullptr,
                    const int32_t *xr = nullptr, bool *history_done = nullptr) {
     if (history_done) *history_done = false;
     const int64_t n_tok = static_cast<int64_t>(B) * T;
@@ -897,13 +909,16 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
     const int n_tiles = ps.n_tiles;
     if (ps.pair)
         rc = launch_proj_pair(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode,
-                              &pp);
+                              &pp, in_call);
     else if (ps.bn == 256)
-        rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
+        rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp,
+                              ProjTest(), in_call);
     else if (ps.bn == 128)
-        rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
+        rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp,
+                              ProjTest(), in_call);
     else
-        rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp);
+        rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp,
+                              ProjTest(), in_call);
     if (rc != ENGRAM_OK) return rc;
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[1], stream), "cudaEventRecord");
     if (fused_decode) {
@@ -1245,7 +1260,7 @@ int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
         return fail(ENGRAM_ERR_INVALID_ARG, "workspace too small: need %zu bytes", need);
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(ENGRAM_ERR_INVALID_ARG, "workspace not 256-byte aligned");
     return gate_conv_impl(plan, w, h, m, B, T, conv_state, out, delta_dbg, static_cast<uint8_t *>(workspace),
-                          static_cast<cudaStream_t>(stream), nullptr);
+                          static_cast<cudaStream_t>(stream), nullptr, false);
 }
 
 int engram_forward(const engram_plan *plan, const engram_weights *w, const void *const *tables,
@@ -1324,7 +1339,7 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const void 
     }
     bool history_done = false;
     if ((rc = gate_conv_impl(plan, w, h, m, B, T, conv_state, out, delta_dbg, ws, stream,
-                             stage_events ? stage_events + 2 : nullptr, history, xr, &history_done)) != ENGRAM_OK)
+                             stage_events ? stage_events + 2 : nullptr, true, history, xr, &history_done)) != ENGRAM_OK)
         return rc;
     if ((rc = rec(4)) != ENGRAM_OK) return rc;
     if (history != nullptr && plan->hist_len > 0 && !history_done) {
@@ -1363,9 +1378,10 @@ int engram_gate_conv_noalloc(const engram_plan *plan, const engram_weights *w, c
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     uint16_t *v = reinterpret_cast<uint16_t *>(scratch);
     float4 *part = reinterpret_cast<float4 *>(scratch + v_bytes);
-    if (bn == 256) rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream);
-    else if (bn == 128) rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream);
-    else rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream);
+    // the first kernel of the call: no overlap with the caller's earlier kernels (launch_ex)
+    if (bn == 256) rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream, nullptr, 1, 0, true, nullptr, ProjTest(), false);
+    else if (bn == 128) rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream, nullptr, 1, 0, true, nullptr, ProjTest(), false);
+    else rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream, nullptr, 1, 0, true, nullptr, ProjTest(), false);
     if (rc != ENGRAM_OK) return rc;
     return launch_gate_conv(plan, w, h, v, part, n_tiles, B, T, conv_state, out, delta_dbg, stream);
 }
@@ -1416,7 +1432,7 @@ int engram_selftest_wait_timeout(const engram_plan *plan, const engram_weights *
     test.wait_limit_ns = wait_limit_ns;
     test.stall = 1;
     return launch_proj<64>(plan, w, h, m, n_tok, v, part, static_cast<cudaStream_t>(stream), nullptr, 1, 0, false,
-                           nullptr, test);
+                           nullptr, test, false);
 }
 
 uint64_t engram_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }

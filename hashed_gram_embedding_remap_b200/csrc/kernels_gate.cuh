@@ -674,13 +674,29 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 320 ? 2 : 1) decode_fused_kernel
     const int c = threadIdx.x * 8;   // blockDim.x == d_h / 8, a multiple of 32
     const int64_t split_stride = pp.n_tok * (2 * d_h);
     const float *acc = pp.acc_out + static_cast<int64_t>(b) * (2 * d_h) + c;
-    // the carried state and h first (independent of the splits)
-    uint4 st[S];
+    // Everything that does not depend on the projection first: the carried state, h, the
+    // gains and the conv taps.  The state shift (slot j <- slot j + 1 for j < 8) needs only
+    // the old state, so it is stored here too; only the three conv taps (slots 6, 3, 0 =
+    // positions t-3, t-6, t-9) stay in registers across the wait.
+    uint4 tap6 = make_uint4(0, 0, 0, 0), tap3 = tap6, tap0 = tap6;
     uint16_t *state = p.conv_state != nullptr ? p.conv_state + static_cast<int64_t>(b) * S * d_h + c : nullptr;
+    if (state != nullptr) {
+        uint4 st[S];
 #pragma unroll
-    for (int j = 0; j < S; ++j)
-        st[j] = state != nullptr ? *reinterpret_cast<const uint4 *>(state + j * d_h) : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < S; ++j) st[j] = *reinterpret_cast<const uint4 *>(state + j * d_h);
+        tap6 = st[6];
+        tap3 = st[3];
+        tap0 = st[0];
+#pragma unroll
+        for (int j = 0; j < S - 1; ++j) *reinterpret_cast<uint4 *>(state + j * d_h) = st[j + 1];
+    }
     const uint4 hw = __ldg(reinterpret_cast<const uint4 *>(pp.h + static_cast<int64_t>(b) * d_h + c));
+    const uint4 gqw = __ldg(reinterpret_cast<const uint4 *>(pp.gamma_q + c));
+    const uint4 gkw = __ldg(reinterpret_cast<const uint4 *>(pp.gamma_k + c));
+    const uint4 gcw = __ldg(reinterpret_cast<const uint4 *>(p.gamma_c + c));
+    uint4 ww[4];   // conv taps: ww[q] holds channel c + 2q (x, y) and channel c + 2q + 1 (z, w)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) ww[q] = __ldg(reinterpret_cast<const uint4 *>(p.conv_w + c * 4) + q);
     pdl_wait();   // the split accumulators come from the projection kernel before this one
     if (p.history != nullptr && threadIdx.x == 0) {
         // the step's hash history update (T = 1): drop the oldest id, append this step's.
@@ -701,17 +717,20 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 320 ? 2 : 1) decode_fused_kernel
         v[0] += v0.x; v[1] += v0.y; v[2] += v0.z; v[3] += v0.w;
         v[4] += v1.x; v[5] += v1.y; v[6] += v1.z; v[7] += v1.w;
     }
-    float hf[8], gq[8], gk[8];
+    float hf[8];
     bf16x8_to_f32(hw, hf);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(pp.gamma_q + c)), gq);
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(pp.gamma_k + c)), gk);
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    {
+        float gq[8], gk[8];
+        bf16x8_to_f32(gqw, gq);
+        bf16x8_to_f32(gkw, gk);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        a0 = fmaf(hf[e], hf[e], a0);
-        a1 = fmaf(hf[e] * gq[e] * gk[e], kt[e], a1);
-        a2 = fmaf(kt[e], kt[e], a2);
-        a3 = fmaf(v[e], v[e], a3);
+        for (int e = 0; e < 8; ++e) {
+            a0 = fmaf(hf[e], hf[e], a0);
+            a1 = fmaf(hf[e] * gq[e] * gk[e], kt[e], a1);
+            a2 = fmaf(kt[e], kt[e], a2);
+            a3 = fmaf(v[e], v[e], a3);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -746,17 +765,15 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 320 ? 2 : 1) decode_fused_kernel
     __syncthreads();
     const float g = s_gb[0], beta = s_gb[1];
     float gc[8], s6[8], s3f[8], s0f[8];
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(p.gamma_c + c)), gc);
-    bf16x8_to_f32(st[6], s6);    // position t-3
-    bf16x8_to_f32(st[3], s3f);   // t-6
-    bf16x8_to_f32(st[0], s0f);   // t-9
-    const uint4 *wp = reinterpret_cast<const uint4 *>(p.conv_w + c * 4);   // 8 channels x 4 taps
+    bf16x8_to_f32(gcw, gc);
+    bf16x8_to_f32(tap6, s6);    // position t-3
+    bf16x8_to_f32(tap3, s3f);   // t-6
+    bf16x8_to_f32(tap0, s0f);   // t-9
     float u[8], d[8];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {   // channel pairs
-        const uint4 ww = __ldg(wp + q);   // taps of channels c + 2q (x, y) and c + 2q + 1 (z, w)
-        const float w0[4] = {bf16_lo(ww.x), bf16_hi(ww.x), bf16_lo(ww.y), bf16_hi(ww.y)};
-        const float w1[4] = {bf16_lo(ww.z), bf16_hi(ww.z), bf16_lo(ww.w), bf16_hi(ww.w)};
+        const float w0[4] = {bf16_lo(ww[q].x), bf16_hi(ww[q].x), bf16_lo(ww[q].y), bf16_hi(ww[q].y)};
+        const float w1[4] = {bf16_lo(ww[q].z), bf16_hi(ww[q].z), bf16_lo(ww[q].w), bf16_hi(ww[q].w)};
 #pragma unroll
         for (int e2 = 0; e2 < 2; ++e2) {
             const int e = 2 * q + e2;
@@ -777,12 +794,9 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 320 ? 2 : 1) decode_fused_kernel
         dp[0] = make_float4(d[0], d[1], d[2], d[3]);
         dp[1] = make_float4(d[4], d[5], d[6], d[7]);
     }
-    if (state != nullptr) {
-#pragma unroll
-        for (int j = 0; j < S - 1; ++j) *reinterpret_cast<uint4 *>(state + j * d_h) = st[j + 1];
+    if (state != nullptr)   // the new slot 8: this token's conv input (slots 0..7 were shifted above)
         *reinterpret_cast<uint4 *>(state + (S - 1) * d_h) =
             make_uint4(pack_bf16x2(u[0], u[1]), pack_bf16x2(u[2], u[3]), pack_bf16x2(u[4], u[5]), pack_bf16x2(u[6], u[7]));
-    }
 }
 
 }  // namespace engram

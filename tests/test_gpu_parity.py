@@ -333,6 +333,49 @@ def test_decode_steps_match_oracle_and_update_state(geom):
         hist, state = ref["history"], to_host_u16(di.conv_state)
 
 
+@pytest.mark.parametrize("geom", ["fused_d2560", "decode_kernel_d384"])
+def test_gate_conv_decode_steps_queued_back_to_back(geom):
+    """engram_gate_conv decode steps queued on one stream with nothing between them, the conv
+    state carried from call to call: every step's output and the final state equal those of
+    the same steps run one at a time.  (The decode kernels read and shift the carried state
+    before they wait for the projection, so a call's first kernel must not overlap the
+    previous call's last one.)"""
+    if geom == "fused_d2560":   # split-K projection + decode_fused_kernel
+        wl = small_workload("dec_q2560", B=200, T=1, K=1, d_e=2560, d_h=2560, decode=True)
+    else:                       # split-K reduce + gate_conv_decode_kernel
+        wl = small_workload("dec_q384", B=64, T=1, K=1, d_e=512, d_h=384, decode=True)
+    di = DeviceInputs(wl, random_gammas=True)
+    steps = 6
+    ms, hs = [], []
+    for step in range(steps):
+        ids_np = synth.zipf_ids(wl.vocab_in, 1.1, (wl.B, wl.T), 900 + step)
+        idx = _idx_oracle(wl, ids_np)
+        m = torch.empty((wl.n_tok, wl.d_m), dtype=torch.bfloat16, device="cuda")
+        E.engram_gather(di.plan, to_dev(idx.view(np.int32)), di.tables, m)
+        ms.append(m)
+        hs.append(to_dev(synth.fill_bf16(wl.h_spec(step), (wl.B * wl.T, wl.d_h))))
+    state0 = di.conv_state.clone()
+    torch.cuda.synchronize()
+
+    def run(sync_each):
+        state = state0.clone()
+        outs = [torch.empty_like(di.out) for _ in range(steps)]
+        torch.cuda.synchronize()
+        for k in range(steps):
+            E.engram_gate_conv(di.plan, di.weights, hs[k], ms[k], wl.B, wl.T, outs[k], di.ws, conv_state=state)
+            if sync_each:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        return outs, state
+
+    outs_a, state_a = run(True)
+    outs_b, state_b = run(False)
+    for k in range(steps):
+        assert torch.equal(outs_a[k].view(torch.int16), outs_b[k].view(torch.int16)), k
+    assert torch.equal(state_a.view(torch.int16), state_b.view(torch.int16))
+    assert E.engram_device_status(clear=True) == 0
+
+
 def _window_oracle(wl, di, w, b, t):
     """Oracle for token (b, t) on a window of at most 1 + state_len tokens, with the rows it
     needs regenerated from the seeded generator (the tables are never materialised)."""

@@ -17,6 +17,7 @@
 #include "engram.h"
 #include "kernels_gate.cuh"
 #include "kernels_lookup.cuh"
+#include "kernels_order.cuh"
 #include "kernels_proj_pair.cuh"
 #include "ptx.cuh"
 
@@ -116,9 +117,11 @@ int check_plan(const engram_plan *plan) {
 
 // ---------------------------------------------------------------- workspace layout
 constexpr int64_t kFusedLookupMaxRows = 16384;   // (token, table) rows handled by lookup_kernel
+constexpr int64_t kRowOrderMinRows = 65536;      // (token, table) rows from which the gather runs in row order
 struct Workspace {
     size_t xr, idx, m, v, part, acc, scal;
     size_t staged_idx, unique, n_unique, staging;  // host-resident tables only
+    size_t order_count, order_cursor, order;       // row-ordered gather only
     bool staged;                                   // rows go through device staging
     size_t total;
 };
@@ -251,6 +254,7 @@ struct ForwardPath {
     bool fused_lookup;    // remap + hash + gather in one kernel (decode-sized, HBM tables)
     bool staged;          // host-mapped tables: the batch's distinct rows are staged into HBM
     bool pair;            // the projection's MMAs span CTA pairs
+    bool row_order;       // the gather walks the rows grouped by row id (kernels_order.cuh)
     ProjShape ps;
 };
 
@@ -261,6 +265,12 @@ ForwardPath forward_path(const engram_plan *plan, int64_t n_tok) {
     f.fused_lookup = !f.staged && plan->cfg.table_location == ENGRAM_TABLES_DEVICE &&
                      n_tok * plan->num_tables <= kFusedLookupMaxRows;
     f.pair = f.ps.pair;
+    // row order (opt-in): HBM tables through the hash + gather path, enough rows for the list to pay,
+    // and 32-bit list items and chunk indices (with slack for the grid stride)
+    const int64_t rows = n_tok * plan->num_tables;
+    f.row_order = !f.staged && !f.fused_lookup && plan->cfg.table_location == ENGRAM_TABLES_DEVICE &&
+                  (plan->cfg.flags & ENGRAM_FLAG_ROW_ORDER_GATHER) && rows >= kRowOrderMinRows &&
+                  rows * (plan->cfg.row_dim / 8) < (int64_t(1) << 31);
     return f;
 }
 
@@ -280,7 +290,13 @@ Workspace layout(const engram_plan *plan, int64_t n_tok) {
     w.acc = off;
     if (ps.k_splits > 1) off = align256(off + sizeof(float) * ps.k_splits * n_tok * ps.n_tiles * ps.bn);
     w.scal = off; off = align256(off + sizeof(float2) * n_tok * plan->num_branches);
-    w.staged = forward_path(plan, n_tok).staged;
+    const ForwardPath fp = forward_path(plan, n_tok);
+    w.staged = fp.staged;
+    if (fp.row_order) {
+        w.order_count = off;  off = align256(off + sizeof(uint32_t) * H * engram::kOrderBuckets);
+        w.order_cursor = off; off = align256(off + sizeof(uint32_t) * H * engram::kOrderBuckets);
+        w.order = off;        off = align256(off + sizeof(uint2) * n_tok * H);
+    }
     if (w.staged) {
         w.staged_idx = off; off = align256(off + sizeof(uint32_t) * n_tok * H);
         w.unique = off;     off = align256(off + sizeof(uint32_t) * n_tok * H);
@@ -637,6 +653,57 @@ int launch_gather(const engram_plan *plan, const uint32_t *idx, const void *cons
                            : (f8 ? engram::gather_kernel<4, true, int64_t> : engram::gather_kernel<4, false, int64_t>);
     kern<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(idx, reinterpret_cast<uint4 *>(m), p);
     ENGRAM_LAUNCHED("gather_kernel launch");
+    return ENGRAM_OK;
+}
+
+// The gather in row order (kernels_order.cuh): count the batch's (token, table) rows per
+// bucket, scan the counts, list the rows bucket by bucket, then copy them.  count / cursor:
+// H * kOrderBuckets words each; order: n_tok * H entries.  HBM-resident tables only.
+int launch_gather_ordered(const engram_plan *plan, const uint32_t *idx, const void *const *tables, int64_t n_tok,
+                          uint16_t *m, uint32_t *count, uint32_t *cursor, uint2 *order, cudaStream_t stream) {
+    const int H = plan->num_tables;
+    const int64_t items = n_tok * H;
+    engram::OrderParams op{};
+    op.H = H;
+    op.n_items = items;
+    for (int h = 0; h < H; ++h) {
+        // bucket = row >> shift: the table's rows spread over at most kOrderBuckets buckets
+        int bits = 0;
+        while (bits < 32 && (uint64_t(1) << bits) < static_cast<uint64_t>(plan->cfg.table_rows[h])) ++bits;
+        op.shift[h] = bits > engram::kOrderBucketsLog2 ? bits - engram::kOrderBucketsLog2 : 0;
+    }
+    const int nb = H * engram::kOrderBuckets;
+    ENGRAM_CUDA_TRY(cudaMemsetAsync(count, 0, sizeof(uint32_t) * nb, stream), "cudaMemsetAsync(order counts)");
+    const unsigned blocks = static_cast<unsigned>((items + engram::kOrderThreads - 1) / engram::kOrderThreads);
+    engram::order_count_kernel<<<blocks, engram::kOrderThreads, 0, stream>>>(idx, count, op);
+    ENGRAM_LAUNCHED("order_count_kernel launch");
+    engram::order_scan_kernel<<<1, engram::kOrderScanThreads, 0, stream>>>(count, cursor, nb);
+    ENGRAM_LAUNCHED("order_scan_kernel launch");
+    engram::order_scatter_kernel<<<blocks, engram::kOrderThreads, 0, stream>>>(idx, cursor, order, op);
+    ENGRAM_LAUNCHED("order_scatter_kernel launch");
+
+    engram::GatherParams p{};
+    for (int h = 0; h < H; ++h) {
+        p.table[h] = tables[h];
+        p.scale[h] = plan->cfg.table_scale[h];
+        p.rows[h] = static_cast<uint64_t>(plan->cfg.table_rows[h]);
+    }
+    p.H = H;
+    p.chunks_per_row = plan->cfg.row_dim / 8;
+    p.chunks_per_tok = H * p.chunks_per_row;
+    p.n_tok = n_tok;
+    p.div_row = engram::make_fastdiv(static_cast<uint32_t>(p.chunks_per_row));
+    p.div_h = engram::make_fastdiv(static_cast<uint32_t>(H));
+    const int64_t total = n_tok * p.chunks_per_tok;   // < 2^31 (forward_path)
+    constexpr int unroll = 4;
+    const int threads = 256;
+    int64_t gblocks = (total + threads * unroll - 1) / (threads * unroll);
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;  // 8 x 256 threads resident per SM
+    if (gblocks > cap) gblocks = cap;
+    if (gblocks < 1) gblocks = 1;
+    auto kern = fp8_tables(plan) ? engram::gather_ordered_kernel<unroll, true> : engram::gather_ordered_kernel<unroll, false>;
+    kern<<<static_cast<unsigned>(gblocks), threads, 0, stream>>>(order, reinterpret_cast<uint4 *>(m), p);
+    ENGRAM_LAUNCHED("gather_ordered_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -1036,7 +1103,8 @@ int engram_init(const engram_config *cfg, engram_plan *plan) {
     }
     if (c.table_dtype == ENGRAM_TABLE_FP8_E4M3 && c.row_dim % 16 != 0)
         return fail(ENGRAM_ERR_UNSUPPORTED, "FP8 tables need row_dim % 16 == 0");
-    if (c.flags & ~ENGRAM_FLAG_SINGLE_CTA_MMA) return fail(ENGRAM_ERR_INVALID_ARG, "unknown flags 0x%x", c.flags);
+    if (c.flags & ~(ENGRAM_FLAG_SINGLE_CTA_MMA | ENGRAM_FLAG_ROW_ORDER_GATHER))
+        return fail(ENGRAM_ERR_INVALID_ARG, "unknown flags 0x%x", c.flags);
 
     std::memset(plan, 0, sizeof *plan);
     plan->cfg = c;
@@ -1334,6 +1402,11 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const void 
                                stream)) != ENGRAM_OK)
             return rc;
         if ((rc = launch_gather(plan, sidx, stage_ptr, n_tok, m, stream, n_tok)) != ENGRAM_OK) return rc;
+    } else if (fp.row_order) {
+        if ((rc = launch_gather_ordered(plan, idx, tables, n_tok, m, reinterpret_cast<uint32_t *>(ws + L.order_count),
+                                        reinterpret_cast<uint32_t *>(ws + L.order_cursor),
+                                        reinterpret_cast<uint2 *>(ws + L.order), stream)) != ENGRAM_OK)
+            return rc;
     } else if ((rc = launch_gather(plan, idx, tables, n_tok, m, stream)) != ENGRAM_OK) {
         return rc;
     }
@@ -1398,6 +1471,7 @@ int engram_forward_path(const engram_plan *plan, int32_t B, int32_t T, uint32_t 
     if (fp.staged) bits |= ENGRAM_PATH_STAGED_ROWS;
     if (fp.ps.k_splits > 1) bits |= ENGRAM_PATH_SPLIT_K;
     if (fp.pair) bits |= ENGRAM_PATH_PAIR_MMA;
+    if (fp.row_order) bits |= ENGRAM_PATH_ROW_ORDER;
     *path = bits;
     return ENGRAM_OK;
 }

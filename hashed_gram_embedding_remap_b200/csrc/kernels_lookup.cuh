@@ -204,6 +204,7 @@ struct GatherParams {
     int32_t chunks_per_tok;  // H * d_e / 8
     int64_t n_tok;
     FastDivU32 div_row, div_tok;  // by chunks_per_row, chunks_per_tok (32-bit index launches)
+    FastDivU32 div_h;             // by H (row-ordered gather: list item -> table)
 };
 
 // The stored bytes behind one 16-byte chunk of m (8 values): 16 bytes of a bf16 row, or 8

@@ -120,6 +120,9 @@ typedef struct engram_config {
 #define ENGRAM_FLAG_SINGLE_CTA_MMA 0x4 /* never pair CTAs for the projection's MMAs (see
                                           ENGRAM_PATH_PAIR_MMA); results are bit-identical either
                                           way.  Bits 0x1 and 0x2 are retired and rejected. */
+#define ENGRAM_FLAG_ROW_ORDER_GATHER 0x8 /* gather large batches grouped by row id: in-batch
+                                            dedup of the HBM reads (see ENGRAM_PATH_ROW_ORDER);
+                                            results are bit-identical either way */
 
 /* Validated config plus derived constants.  Caller-owned, plain data: engram_init fills
  * it, every other call reads it.  Do not modify its fields. */
@@ -303,7 +306,8 @@ int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
  * reductions fused in their epilogue, then gate + conv + residual, then the history update
  * when `history` is given.  Kernels per call (engram_forward_path tells which apply): prefill
  * batches launch remap + hash, gather, projection, gate scalars and the streaming gate + conv
- * kernel (5); batches of at most 16,384 (token, table) rows on HBM-resident tables fuse
+ * kernel (5), and with ENGRAM_PATH_ROW_ORDER three more ahead of the gather (count rows per
+ * bucket, scan, list; 8); batches of at most 16,384 (token, table) rows on HBM-resident tables fuse
  * remap + hash + gather into one kernel; decode-sized batches on host-mapped tables fuse
  * remap + hash + dedup + staging into one; one-token decode steps whose projection splits K
  * finish the split sums, gate, conv and the history update in one kernel (lookup,
@@ -359,14 +363,25 @@ int engram_gate_conv_noalloc(const engram_plan *plan, const engram_weights *w, c
  *   SPLIT_K        the projection splits K across CTAs (decode-sized batches);
  *   PAIR_MMA       the projection runs on pairs of CTAs (a thread-block cluster of two), each
  *                  tensor-core MMA spanning both: 256-token x 256-channel tiles, each CTA
- *                  holding half of every operand tile (d_h % 256 == 0, whole-K tiles, at
- *                  least 148 tiles, ENGRAM_FLAG_SINGLE_CTA_MMA not set); the workspace's
- *                  partial sums then have (M+1)*d_h/256 columns per token.
- * Otherwise the hash kernel writes the row ids and the gather kernel writes m. */
+ *                  holding half of every operand tile (d_h % 256 == 0 and
+ *                  ENGRAM_FLAG_SINGLE_CTA_MMA not set; whole-K tiles when there are at least
+ *                  148 of them, K split across pairs when fewer than 74 would leave pairs
+ *                  idle); the workspace's partial sums then have (M+1)*d_h/256 columns per
+ *                  token;
+ *   ROW_ORDER      the gather walks the batch's (token, table) rows grouped by row id (buckets
+ *                  of neighbouring rows, table by table) instead of in token order, so that
+ *                  every repeat of a row in the batch follows its first read while the row is
+ *                  still in L2: DRAM reads each distinct row about once (in-batch dedup of the
+ *                  HBM reads; m is bit-identical).  ENGRAM_FLAG_ROW_ORDER_GATHER set,
+ *                  HBM-resident tables, the hash + gather path, at least 65,536 rows per
+ *                  call.  Opt-in: m is then written in row order, as scattered slices, and on
+ *                  B200 that costs more write bandwidth than the saved reads.
+ * Otherwise the hash kernel writes the row ids and the gather kernel writes m in token order. */
 #define ENGRAM_PATH_FUSED_LOOKUP 0x1u
 #define ENGRAM_PATH_STAGED_ROWS 0x2u
 #define ENGRAM_PATH_SPLIT_K 0x8u
 #define ENGRAM_PATH_PAIR_MMA 0x10u
+#define ENGRAM_PATH_ROW_ORDER 0x20u
 int engram_forward_path(const engram_plan *plan, int32_t B, int32_t T, uint32_t *path);
 
 /* Wait for `stream` and report what the device found: ENGRAM_ERR_TIMEOUT if a pipeline wait

@@ -55,7 +55,7 @@ def _plan(**kw):
     (dict(heads_per_order=17), E.ENGRAM_ERR_UNSUPPORTED),
     (dict(flags=0x1), E.ENGRAM_ERR_INVALID_ARG),                                # retired flag bits
     (dict(flags=0x2), E.ENGRAM_ERR_INVALID_ARG),
-    (dict(flags=0x8), E.ENGRAM_ERR_INVALID_ARG),                                # unknown flag bit
+    (dict(flags=0x10), E.ENGRAM_ERR_INVALID_ARG),                               # unknown flag bit
     (dict(table_dtype=2), E.ENGRAM_ERR_INVALID_ARG),                            # unknown table dtype
     (dict(table_dtype=1, table_scale=(0.1, 0.1, 0.1, 0.0)), E.ENGRAM_ERR_INVALID_ARG),   # zero scale
     (dict(table_dtype=1, table_scale=(0.1, float("inf"), 0.1, 0.1)), E.ENGRAM_ERR_INVALID_ARG),
@@ -213,14 +213,21 @@ def test_forward_path_selection():
     """engram_forward_path (host only): which kernels a forward call runs."""
     P = E.engram_forward_path
     PAIR = E.ENGRAM_PATH_PAIR_MMA
+    ROW = E.ENGRAM_PATH_ROW_ORDER
+    RO = E.ENGRAM_FLAG_ROW_ORDER_GATHER
     for name in ("prefill20m", "layer2560"):
         wl = synth.get_workload(name)
-        # prefill: hash kernel, gather kernel, projection on CTA pairs (d_h % 256 == 0, enough tiles)
+        # prefill: hash kernel, gather kernel (token order), projection on CTA pairs
+        # (d_h % 256 == 0, enough tiles)
         assert P(E.Plan.from_workload(wl), wl.B, wl.T) == PAIR
         assert P(E.Plan.from_workload(wl, flags=E.ENGRAM_FLAG_SINGLE_CTA_MMA), wl.B, wl.T) == 0
+        assert P(E.Plan.from_workload(wl, flags=RO), wl.B, wl.T) == PAIR | ROW   # 524,288 rows
         assert P(E.Plan.from_workload(wl.with_(table_dtype="fp8")), wl.B, wl.T) == PAIR
     p16 = _plan(heads_per_order=8, table_rows=[10007] * 16, row_dim=64, hidden_dim=2560)
     assert P(p16, 1, 1100) == 0            # 5 x 20 tiles: too few for the pairs
+    p16r = _plan(heads_per_order=8, table_rows=[10007] * 16, row_dim=64, hidden_dim=2560, flags=RO)
+    assert P(p16r, 1, 4096) == PAIR | ROW   # 65,536 rows: row order from here when asked for
+    assert P(p16r, 1, 4095) == PAIR
     assert not P(_plan(hidden_dim=384), 8, 4096) & PAIR
     # decode-sized batches: one lookup kernel, split-K projection
     dec = synth.get_workload("decode20m")
@@ -230,6 +237,10 @@ def test_forward_path_selection():
     # host-mapped tables: distinct rows staged into HBM first
     hp = synth.get_workload("hostpinned20m")
     assert P(E.Plan.from_workload(hp, host_tables=True), hp.B, 1) & E.ENGRAM_PATH_STAGED_ROWS
+    # host tables never take the row-ordered HBM gather (their rows are staged and deduplicated)
+    assert P(E.Plan.from_workload(hp, host_tables=True, flags=RO), 64, 128) & (E.ENGRAM_PATH_STAGED_ROWS | ROW) == (
+        E.ENGRAM_PATH_STAGED_ROWS)
+    assert not P(E.Plan.from_workload(hp, host_tables=True, flags=RO), 64, 8192) & ROW
     with pytest.raises(E.EngramError):
         P(p16, -1, 4)
 

@@ -214,6 +214,39 @@ def test_pair_mma_bit_identical_to_single_cta(case, packed):
     assert E.engram_device_status(clear=True) == 0
 
 
+ROW_ORDER_CASES = {
+    # 24,000 tokens x 4 tables of ~1,000 rows: most rows repeat many times
+    "walk72": PARITY_CASES["gate_walk72"],
+    # the 16-table layer's widths (d_e = 160: 20 chunks per row), ~100,000-row tables: 3,126
+    # buckets per table; 4,200 tokens = 67,200 rows, just above the row-order threshold
+    "h16_d160": small_workload("ro16", B=2, T=2100, K=8, d_e=160, d_h=256,
+                               primes=tuple(synth.largest_prime_below(100003 + 40 * h) for h in range(16))),
+    # e4m3 tables with their per-table scales
+    "fp8": small_workload("ro8", B=2, T=9000, K=2, d_e=32, d_h=256, table_dtype="fp8"),
+    # the 20M-row layer's row width (d_e = 2560, 320 chunks per row), two tables
+    "d2560": small_workload("ro2560", B=2, T=16500, K=1, d_e=2560, d_h=256, primes=(100003, 100019)),
+}
+
+
+@pytest.mark.parametrize("case", list(ROW_ORDER_CASES))
+def test_row_order_gather_bit_identical_to_token_order(case):
+    """In-batch dedup of the HBM reads: the gather walking the batch's rows grouped by row id
+    (ENGRAM_PATH_ROW_ORDER) gives the same m as the gather in token order, hence the same
+    Delta and out bit for bit."""
+    wl = ROW_ORDER_CASES[case]
+    a = DeviceInputs(wl, flags=E.ENGRAM_FLAG_ROW_ORDER_GATHER, random_gammas=True)
+    assert E.engram_forward_path(a.plan, wl.B, wl.T) & E.ENGRAM_PATH_ROW_ORDER
+    b = DeviceInputs(wl, tables=a.tables, random_gammas=True)
+    assert not E.engram_forward_path(b.plan, wl.B, wl.T) & E.ENGRAM_PATH_ROW_ORDER
+    for _ in range(2):   # the list is rebuilt on every call
+        a.forward()
+        b.forward()
+        torch.cuda.synchronize()
+        assert torch.equal(a.delta, b.delta)
+        assert torch.equal(a.out.view(torch.int16), b.out.view(torch.int16))
+    assert E.engram_device_status(clear=True) == 0
+
+
 @pytest.mark.parametrize("B,d_h", [(256, 2560), (96, 512)])
 def test_pair_split_k_decode_bit_identical_to_single_cta(B, d_h):
     """One-token decode steps whose projection splits K: on CTA pairs (256-token units, each

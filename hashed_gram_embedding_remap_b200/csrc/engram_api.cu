@@ -122,17 +122,11 @@ struct Workspace {
     size_t xr, idx, m, v, part, acc, scal;
     size_t staged_idx, unique, n_unique, staging;  // host-resident tables only
     size_t order_count, order_cursor, order;       // row-ordered gather only
-    size_t row_done;                               // projection epilogue's 32-token group counts
     bool staged;                                   // rows go through device staging
     size_t total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-
-// 32-token group counters of the projection epilogue: one per group of every (whole, possibly
-// partly empty) 256-token tile, so that the single-CTA (128-row) and pair (256-row) tiles both
-// stay inside
-int64_t row_done_words(int64_t n_tok) { return (n_tok + 255) / 256 * 8; }
 
 // Launch with programmatic stream serialization (pdl = true): the kernel may start while the
 // previous kernel on the stream finishes (see pdl_wait / pdl_launch_dependents).  Only a
@@ -296,7 +290,6 @@ Workspace layout(const engram_plan *plan, int64_t n_tok) {
     w.acc = off;
     if (ps.k_splits > 1) off = align256(off + sizeof(float) * ps.k_splits * n_tok * ps.n_tiles * ps.bn);
     w.scal = off; off = align256(off + sizeof(float2) * n_tok * plan->num_branches);
-    w.row_done = off; off = align256(off + sizeof(uint32_t) * row_done_words(n_tok));
     const ForwardPath fp = forward_path(plan, n_tok);
     w.staged = fp.staged;
     if (fp.row_order) {
@@ -377,19 +370,11 @@ struct ProjTest {
     int stall = 0;
 };
 
-// Gate scalars finished in the projection's epilogue (ProjParams::scal_out): row_done must be
-// zero when the projection starts.
-struct ProjScal {
-    float2 *scal;
-    uint32_t *row_done;
-};
-
 template <int BN>
 int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                 int64_t n_tok, uint16_t *v, float4 *part, cudaStream_t stream, float *acc = nullptr,
                 int k_splits = 1, int kb_per_split = 0, bool run_reduce = true,
-                engram::ProjParams *params_out = nullptr, const ProjTest &test = ProjTest(), bool pdl = true,
-                const ProjScal *fin = nullptr) {
+                engram::ProjParams *params_out = nullptr, const ProjTest &test = ProjTest(), bool pdl = true) {
     const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim;
     CUtensorMap map_m, map_wk, map_wv;
     int rc;
@@ -418,12 +403,6 @@ int launch_proj(const engram_plan *plan, const engram_weights *w, const uint16_t
     p.w_packed = BN == 256 ? static_cast<const uint8_t *>(w->w_packed) : nullptr;
     p.wait_limit_ns = test.wait_limit_ns;
     p.stall = test.stall;
-    if (fin != nullptr && p.k_splits == 1) {
-        p.scal_out = fin->scal;
-        p.row_done = fin->row_done;
-        p.eps = plan->cfg.eps;
-        p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(d_h));
-    }
     const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles * p.k_splits;
     if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
     const int64_t sms = sm_count();
@@ -482,8 +461,7 @@ int max_pairs(int *out) {
 // single-CTA split).
 int launch_proj_pair(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                      int64_t n_tok, uint16_t *v, float4 *part, cudaStream_t stream, float *acc, int k_splits,
-                     int kb_per_split, bool run_reduce, engram::ProjParams *params_out, bool pdl,
-                     const ProjScal *fin = nullptr) {
+                     int kb_per_split, bool run_reduce, engram::ProjParams *params_out, bool pdl) {
     const int d_m = plan->mem_dim, d_h = plan->cfg.hidden_dim, M = plan->num_branches;
     constexpr int BN = engram::kPairBN;
     CUtensorMap map_m, map_wk, map_wv;
@@ -530,12 +508,6 @@ int launch_proj_pair(const engram_plan *plan, const engram_weights *w, const uin
     p.kb_per_split = split ? kb_per_split : p.k_blocks;
     p.acc_out = split ? acc : nullptr;
     p.w_packed = static_cast<const uint8_t *>(w->w_packed);
-    if (fin != nullptr && !split) {
-        p.scal_out = fin->scal;
-        p.row_done = fin->row_done;
-        p.eps = plan->cfg.eps;
-        p.inv_sqrt_d = 1.0f / std::sqrt(static_cast<float>(d_h));
-    }
     const int64_t total = static_cast<int64_t>(p.m_tiles) * p.n_tiles * p.k_splits;
     if (total > 0x7FFFFFFF) return fail(ENGRAM_ERR_UNSUPPORTED, "too many projection tiles");
     // ENGRAM_PROJ_PAIRS (>= 1) caps the number of CTA pairs (tuning); read once per process.
@@ -768,7 +740,7 @@ engram::GateParams make_gate_params(const engram_plan *plan, const engram_weight
 
 int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *v,
                      const float4 *part, int n_tiles, int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out,
-                     float *delta, cudaStream_t stream, float2 *scal = nullptr, bool scal_ready = false) {
+                     float *delta, cudaStream_t stream, float2 *scal = nullptr) {
     engram::GateParams p{};
     const int d_h = plan->cfg.hidden_dim;
     p.h = h;
@@ -813,9 +785,7 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
         return ENGRAM_OK;
     }
     dim3 grid(static_cast<unsigned>((T + p.tok_chunk - 1) / p.tok_chunk), static_cast<unsigned>(B), slices);
-    if (k4d3 && scal != nullptr && conv_state == nullptr && scal_ready) {
-        p.scal = scal;   // finished in the projection's epilogue
-    } else if (k4d3 && scal != nullptr && conv_state == nullptr) {
+    if (k4d3 && scal != nullptr && conv_state == nullptr) {
         // scalars once per (token, branch) instead of once per (CTA, halo-extended chunk)
         const int64_t items = static_cast<int64_t>(B) * T * p.M;
         // programmatic launches (the projection before them belongs to the same call)
@@ -986,16 +956,8 @@ cudaError_t record_stage_event(void *ev, cudaStream_t stream) {
 
 // history / xr (engram_forward's decode steps): when the step ends in decode_fused_kernel, that
 // kernel also advances the hash history and *history_done is set; otherwise the caller does.
-// A whole-K projection ahead of the streaming gate kernel (kernel 4, dilation 3, no carried
-// state) finishes the gate scalars in its epilogue, counting finished units in the
-// workspace's row_done, which must be zero when the projection starts.
-bool proj_finishes_scalars(const engram_plan *plan, const ProjShape &ps, const uint16_t *conv_state) {
-    return ps.k_splits == 1 && plan->cfg.conv_kernel == 4 && plan->cfg.conv_dilation == 3 && conv_state == nullptr;
-}
-
 // in_call: the kernel before the projection belongs to the same entry-point call (engram_forward),
-// so the projection may overlap it (launch_ex), and the call zeroed row_done before its first
-// kernel; otherwise it is zeroed here, ahead of the projection.
+// so the projection may overlap it (launch_ex).
 int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint16_t *h, const uint16_t *m,
                    int32_t B, int32_t T, uint16_t *conv_state, uint16_t *out, float *delta, uint8_t *ws,
                    cudaStream_t stream, void *const *events, bool in_call, int32_t *history = nullptr,
@@ -1004,11 +966,6 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
     const int64_t n_tok = static_cast<int64_t>(B) * T;
     const Workspace L = layout(plan, n_tok);
     const ProjShape ps = proj_shape(plan, n_tok, true);
-    const bool fin_scal = proj_finishes_scalars(plan, ps, conv_state);
-    const ProjScal fin{reinterpret_cast<float2 *>(ws + L.scal), reinterpret_cast<uint32_t *>(ws + L.row_done)};
-    if (fin_scal && !in_call)
-        ENGRAM_CUDA_TRY(cudaMemsetAsync(fin.row_done, 0, sizeof(uint32_t) * row_done_words(n_tok), stream),
-                        "cudaMemsetAsync(row_done)");
     uint16_t *v = reinterpret_cast<uint16_t *>(ws + L.v);
     float4 *part = reinterpret_cast<float4 *>(ws + L.part);
     float *acc = ps.k_splits > 1 ? reinterpret_cast<float *>(ws + L.acc) : nullptr;
@@ -1023,16 +980,16 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
     const int n_tiles = ps.n_tiles;
     if (ps.pair)
         rc = launch_proj_pair(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode,
-                              &pp, in_call, fin_scal ? &fin : nullptr);
+                              &pp, in_call);
     else if (ps.bn == 256)
         rc = launch_proj<256>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp,
-                              ProjTest(), in_call, fin_scal ? &fin : nullptr);
+                              ProjTest(), in_call);
     else if (ps.bn == 128)
         rc = launch_proj<128>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp,
-                              ProjTest(), in_call, fin_scal ? &fin : nullptr);
+                              ProjTest(), in_call);
     else
         rc = launch_proj<64>(plan, w, h, m, n_tok, v, part, stream, acc, ps.k_splits, ps.kb_per_split, !fused_decode, &pp,
-                              ProjTest(), in_call, fin_scal ? &fin : nullptr);
+                              ProjTest(), in_call);
     if (rc != ENGRAM_OK) return rc;
     if (events) ENGRAM_CUDA_TRY(record_stage_event(events[1], stream), "cudaEventRecord");
     if (fused_decode) {
@@ -1050,7 +1007,8 @@ int gate_conv_impl(const engram_plan *plan, const engram_weights *w, const uint1
         if (history_done) *history_done = gp.history != nullptr;
         return ENGRAM_OK;
     }
-    return launch_gate_conv(plan, w, h, v, part, n_tiles, B, T, conv_state, out, delta, stream, fin.scal, fin_scal);
+    return launch_gate_conv(plan, w, h, v, part, n_tiles, B, T, conv_state, out, delta, stream,
+                            reinterpret_cast<float2 *>(ws + L.scal));
 }
 
 int check_bt(int32_t B, int32_t T) {
@@ -1413,11 +1371,6 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const void 
     const ForwardPath fp = forward_path(plan, n_tok);
     const bool fused_lookup = fp.fused_lookup;
     if ((rc = rec(0)) != ENGRAM_OK) return rc;
-    // the projection's group counts (proj_finishes_scalars) are zeroed ahead of the call's
-    // first kernel, so that no copy node sits between the gather and the projection
-    if (proj_finishes_scalars(plan, fp.ps, conv_state))
-        ENGRAM_CUDA_TRY(cudaMemsetAsync(ws + L.row_done, 0, sizeof(uint32_t) * row_done_words(n_tok), stream),
-                        "cudaMemsetAsync(row_done)");
     const bool stage_small = L.staged && n_tok * plan->num_tables <= engram::kStageSmallRows;
     if (fused_lookup) {
         if ((rc = rec(1)) != ENGRAM_OK) return rc;

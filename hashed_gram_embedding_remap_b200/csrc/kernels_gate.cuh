@@ -190,20 +190,48 @@ __global__ void __launch_bounds__(kGateThreads) gate_conv_kernel(const __grid_co
 }
 
 // Per-(token, branch) gate scalars from the projection partials: scal[n*M + b] =
-// (g_b, g_b / rms(U_b)), one thread per (token, branch), in gate_scalars_of's fixed order.
-// Whole-K projections finish the scalars in their own epilogue (finish_scalars_if_last); this
-// kernel serves the split-K path, after the split reduction.
+// (g_b, g_b / rms(U_b)).  Eight lanes per (token, branch) take every eighth of the branch's
+// key tiles followed by the value tiles; a fixed-order butterfly over the eight lanes finishes
+// the sums (deterministic).
 __global__ void __launch_bounds__(256) gate_scalars_kernel(const float4 *__restrict__ part, int64_t n_tok,
                                                            int32_t n_tiles, int32_t n_key_tiles, int32_t M,
                                                            int32_t d_h, float eps, float inv_sqrt_d,
                                                            float2 *__restrict__ scal) {
     pdl_launch_dependents();   // the gate kernel may load its conv taps now
     pdl_wait();                // the partial sums come from the projection before this kernel
-    const int64_t item = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;   // (token, branch)
-    if (item >= n_tok * M) return;
+    const int64_t gt = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t item = gt >> 3;          // (token, branch)
+    const int sub = static_cast<int>(gt & 7);
     const int64_t n = item / M;
     const int br = static_cast<int>(item - n * M);
-    scal[item] = gate_scalars_of(part + n * n_tiles, n_key_tiles, M, br, d_h, eps, inv_sqrt_d);
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    if (n < n_tok) {
+        const float4 *pp = part + n * n_tiles;
+        for (int j = sub; j < 2 * n_key_tiles; j += 8) {
+            if (j < n_key_tiles) {
+                const float4 q = __ldg(pp + br * n_key_tiles + j);
+                s0 += q.x;
+                s1 += q.y;
+                s2 += q.z;
+            } else {
+                s3 += __ldg(pp + M * n_key_tiles + (j - n_key_tiles)).x;
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) {
+        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+        s3 += __shfl_xor_sync(0xffffffffu, s3, o);
+    }
+    if (n < n_tok && sub == 0) {
+        const float inv_d = 1.f / static_cast<float>(d_h);
+        const float rms_h = sqrtf(s0 * inv_d + eps);
+        const float rms_k = sqrtf(s2 * inv_d + eps);
+        const float g = 1.f / (1.f + __expf(-(s1 / (rms_h * rms_k) * inv_sqrt_d)));
+        scal[item] = make_float2(g, g / sqrtf(g * g * s3 * inv_d + eps));
+    }
 }
 
 // x * sigmoid(x) = h + h * tanh(h) with h = x / 2, on the hardware tanh approximation
@@ -652,9 +680,8 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 320 ? 2 : 1) decode_fused_kernel
     const int c = threadIdx.x * 8;   // blockDim.x == d_h / 8, a multiple of 32
     const int64_t split_stride = pp.n_tok * (2 * d_h);
     const float *acc = pp.acc_out + static_cast<int64_t>(b) * (2 * d_h) + c;
-    // Everything that does not depend on the projection first: the carried state and the
-    // gate's gains (h goes with the split sums; gamma_c and the conv taps are loaded after
-    // them, which need the registers).  The state shift (slot j <- slot j + 1 for j < 8) needs only
+    // Everything that does not depend on the projection first: the carried state, h, the
+    // gains and the conv taps.  The state shift (slot j <- slot j + 1 for j < 8) needs only
     // the old state, so it is stored here too; only the three conv taps (slots 6, 3, 0 =
     // positions t-3, t-6, t-9) stay in registers across the wait.
     uint4 tap6 = make_uint4(0, 0, 0, 0), tap3 = tap6, tap0 = tap6;
@@ -669,8 +696,13 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 320 ? 2 : 1) decode_fused_kernel
 #pragma unroll
         for (int j = 0; j < S - 1; ++j) *reinterpret_cast<uint4 *>(state + j * d_h) = st[j + 1];
     }
+    const uint4 hw = __ldg(reinterpret_cast<const uint4 *>(pp.h + static_cast<int64_t>(b) * d_h + c));
     const uint4 gqw = __ldg(reinterpret_cast<const uint4 *>(pp.gamma_q + c));
     const uint4 gkw = __ldg(reinterpret_cast<const uint4 *>(pp.gamma_k + c));
+    const uint4 gcw = __ldg(reinterpret_cast<const uint4 *>(p.gamma_c + c));
+    uint4 ww[4];   // conv taps: ww[q] holds channel c + 2q (x, y) and channel c + 2q + 1 (z, w)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) ww[q] = __ldg(reinterpret_cast<const uint4 *>(p.conv_w + c * 4) + q);
     pdl_wait();   // the split accumulators come from the projection kernel before this one
     if (p.history != nullptr && threadIdx.x == 0) {
         // the step's hash history update (T = 1): drop the oldest id, append this step's.
@@ -679,13 +711,9 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 320 ? 2 : 1) decode_fused_kernel
         for (int s = 0; s + 1 < p.hist_len; ++s) hb[s] = hb[s + 1];
         hb[p.hist_len - 1] = p.xr[b];
     }
-    // h with the split sums (one round trip; holding it across the wait would cost registers)
-    const uint4 hw = __ldg(reinterpret_cast<const uint4 *>(pp.h + static_cast<int64_t>(b) * d_h + c));
     float kt[8], v[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) kt[e] = v[e] = 0.f;
-    // the splits summed in split order (unrolled so that their loads issue together)
-#pragma unroll 3
     for (int ks = 0; ks < pp.k_splits; ++ks) {
         const float4 *src = reinterpret_cast<const float4 *>(acc + ks * split_stride);
         const float4 k0 = __ldg(src), k1 = __ldg(src + 1);
@@ -741,10 +769,6 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 320 ? 2 : 1) decode_fused_kernel
         s_gb[1] = g / sqrtf(g * g * s3 * inv_d + p.eps);
     }
     __syncthreads();
-    const uint4 gcw = __ldg(reinterpret_cast<const uint4 *>(p.gamma_c + c));
-    uint4 ww[4];   // conv taps: ww[q] holds channel c + 2q (x, y) and channel c + 2q + 1 (z, w)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) ww[q] = __ldg(reinterpret_cast<const uint4 *>(p.conv_w + c * 4) + q);
     const float g = s_gb[0], beta = s_gb[1];
     float gc[8], s6[8], s3f[8], s0f[8];
     bf16x8_to_f32(gcw, gc);

@@ -65,67 +65,7 @@ struct ProjParams {
     uint64_t wait_limit_ns;    // bound of every pipeline wait (0: ENGRAM_WAIT_TIMEOUT_NS)
     int32_t stall;             // self-test of the bounded waits: issue no loads at all, so that
                                // the first wait for a stage runs out and the kernel unwinds
-    // Whole-K units only: when scal_out is set, the warp that writes the last of the n_tiles
-    // partial sums of a 32-token group (counted in row_done, zeroed before the launch) also
-    // finishes that group's gate scalars (g, g / rms(U)) per (token, branch) into scal_out.
-    float2 *scal_out;          // [n_tok, M] or null
-    uint32_t *row_done;        // one per 32-token group of every 256-token tile: [ceil(n_tok / 256) * 8]
-    float eps, inv_sqrt_d;
 };
-
-// The gate's scalars of (token, branch) from the token's per-tile partial sums `pp`
-// (key tiles branch-major, then the value tiles): S0 = sum h^2, S1 = sum h gamma_q gamma_k k~,
-// S2 = sum k~^2 over the branch's key tiles and S3 = sum v^2 over the value tiles, each as
-// eight interleaved sums (tiles j, j + 8, ...) folded (0 + 4, 2 + 6) + (1 + 5, 3 + 7): one fixed
-// order wherever it runs.  Then g = sigmoid(S1 / (rms(h) rms(k~)) / sqrt(d_h)) and
-// beta = g / rms(g v) = 1 / rms(U) scaled by g.  Read through L2 (written by other CTAs).
-__device__ __forceinline__ float2 gate_scalars_of(const float4 *pp, int n_key_tiles, int M, int br, int d_h,
-                                                  float eps, float inv_sqrt_d) {
-    float s0[8], s1[8], s2[8], s3[8];
-#pragma unroll
-    for (int l = 0; l < 8; ++l) s0[l] = s1[l] = s2[l] = s3[l] = 0.f;
-#pragma unroll
-    for (int l = 0; l < 8; ++l) {
-        for (int j = l; j < 2 * n_key_tiles; j += 8) {
-            if (j < n_key_tiles) {
-                const float4 q = __ldcg(pp + br * n_key_tiles + j);
-                s0[l] += q.x;
-                s1[l] += q.y;
-                s2[l] += q.z;
-            } else {
-                s3[l] += __ldcg(pp + M * n_key_tiles + (j - n_key_tiles)).x;
-            }
-        }
-    }
-    const float S0 = ((s0[0] + s0[4]) + (s0[2] + s0[6])) + ((s0[1] + s0[5]) + (s0[3] + s0[7]));
-    const float S1 = ((s1[0] + s1[4]) + (s1[2] + s1[6])) + ((s1[1] + s1[5]) + (s1[3] + s1[7]));
-    const float S2 = ((s2[0] + s2[4]) + (s2[2] + s2[6])) + ((s2[1] + s2[5]) + (s2[3] + s2[7]));
-    const float S3 = ((s3[0] + s3[4]) + (s3[2] + s3[6])) + ((s3[1] + s3[5]) + (s3[3] + s3[7]));
-    const float inv_d = 1.f / static_cast<float>(d_h);
-    const float rms_h = sqrtf(S0 * inv_d + eps);
-    const float rms_k = sqrtf(S2 * inv_d + eps);
-    const float g = 1.f / (1.f + __expf(-(S1 / (rms_h * rms_k) * inv_sqrt_d)));
-    return make_float2(g, g / sqrtf(g * g * S3 * inv_d + eps));
-}
-
-// Epilogue tail of a whole-K unit, per warp, after its lanes stored their tokens' partial
-// sums: count the unit into the 32-token group's row_done; the warp that brings the count to
-// n_tiles (all units of the group written) finishes the group's gate scalars.  BN: the tile
-// width the partial sums were taken over.
-__device__ __forceinline__ void finish_scalars_if_last(const ProjParams &p, int64_t group, int lane, int BN) {
-    __threadfence();   // this lane's partial sums, device-wide, before the count
-    __syncwarp();
-    uint32_t last = 0;
-    if (lane == 0) last = atomicAdd(p.row_done + group, 1u) == static_cast<uint32_t>(p.n_tiles - 1);
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (!last) return;
-    __threadfence();   // every unit's partial sums of the group are visible from here
-    const int64_t n = group * 32 + lane;
-    if (n >= p.n_tok) return;
-    const int kpb = p.d_h / BN;
-    for (int br = 0; br < p.M; ++br)
-        p.scal_out[n * p.M + br] = gate_scalars_of(p.part + n * p.n_tiles, kpb, p.M, br, p.d_h, p.eps, p.inv_sqrt_d);
-}
 
 // Packs [W_k ; W_v] into pre-swizzled 256 x 64 tiles (the layout engram_pack_weights
 // documents): one thread per 16-byte chunk of the packed copy.
@@ -431,8 +371,6 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             if (lane == 0) mbar_arrive(&tempty_bar[acc]);
             if constexpr (!SPLIT) {
                 if (valid) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
-                if (p.scal_out != nullptr)
-                    finish_scalars_if_last(p, (static_cast<int64_t>(mt) * kBM + sub * 32) / 32, lane, BN);
             }
         }
     }

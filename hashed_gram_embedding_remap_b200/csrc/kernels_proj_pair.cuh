@@ -266,7 +266,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kProjThreads, 1)
             if (lane == 0) mbar_arrive_cluster(leader_tempty + acc * 8);   // to the even CTA's copy
             if constexpr (!SPLIT) {
                 if (valid) p.part[n * p.n_tiles + nt] = make_float4(a0, a1, a2, 0.f);
-                if (p.scal_out != nullptr) finish_scalars_if_last(p, (rows0 + sub * 32) / 32, lane, BN);
             }
         }
     }

@@ -305,11 +305,9 @@ int engram_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
 /* Steps 1-6 chained: remap + hash (one kernel), gather, projections with the gate's partial
  * reductions fused in their epilogue, then gate + conv + residual, then the history update
  * when `history` is given.  Kernels per call (engram_forward_path tells which apply): prefill
- * batches launch remap + hash, gather, projection (whose epilogue also finishes the gate's
- * per-token scalars) and the streaming gate + conv kernel (4), and with ENGRAM_PATH_ROW_ORDER
- * three more ahead of the gather (count rows per bucket, scan, list; 7); split-K prefill
- * batches add the split reduction and a gate-scalar kernel; batches of at most 16,384
- * (token, table) rows on HBM-resident tables fuse
+ * batches launch remap + hash, gather, projection, gate scalars and the streaming gate + conv
+ * kernel (5), and with ENGRAM_PATH_ROW_ORDER three more ahead of the gather (count rows per
+ * bucket, scan, list; 8); batches of at most 16,384 (token, table) rows on HBM-resident tables fuse
  * remap + hash + gather into one kernel; decode-sized batches on host-mapped tables fuse
  * remap + hash + dedup + staging into one; one-token decode steps whose projection splits K
  * finish the split sums, gate, conv and the history update in one kernel (lookup,

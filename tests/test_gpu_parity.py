@@ -274,7 +274,7 @@ def test_pair_split_k_decode_bit_identical_to_single_cta(B, d_h):
 
 def test_kernel_launch_count_per_call():
     """The library's launch counter (bench.py's gpu_launches): a prefill call launches remap +
-    hash, gather, projection (finishing the gate scalars) and the streaming gate kernel (4); a one-token
+    hash, gather, projection, gate scalars and the streaming gate kernel (5); a one-token
     split-K decode step with hash history and conv state launches the lookup, the projection
     and the fused reduce + gate + conv + history kernel (3); the same call twice counts the
     same; a call rejected on the host counts nothing."""
@@ -286,7 +286,7 @@ def test_kernel_launch_count_per_call():
     n1 = E.kernel_launches()
     di.forward()
     n2 = E.kernel_launches()
-    assert n1 - n0 == 4 and n2 - n1 == 4
+    assert n1 - n0 == 5 and n2 - n1 == 5
     with pytest.raises(E.EngramError):
         E.engram_forward(di.plan, di.weights, di.tables, di.ids, di.h, di.out, di.ws[:16])   # workspace too small
     assert E.kernel_launches() == n2

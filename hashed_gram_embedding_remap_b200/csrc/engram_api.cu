@@ -612,10 +612,8 @@ int launch_hash(const engram_plan *plan, const int32_t *ids, const int32_t *rema
 
 
 // rows_override > 0 bounds every table at that many rows (device staging buffers).
-// pdl: a programmatic launch, for a gather whose row ids come from an earlier kernel of the
-// same call (engram_forward)
 int launch_gather(const engram_plan *plan, const uint32_t *idx, const void *const *tables, int64_t n_tok,
-                  uint16_t *m, cudaStream_t stream, int64_t rows_override = 0, bool pdl = false) {
+                  uint16_t *m, cudaStream_t stream, int64_t rows_override = 0) {
     engram::GatherParams p{};
     const int H = plan->num_tables;
     for (int h = 0; h < H; ++h) {
@@ -653,9 +651,8 @@ int launch_gather(const engram_plan *plan, const uint32_t *idx, const void *cons
     else
         kern = unroll == 8 ? (f8 ? engram::gather_kernel<8, true, int64_t> : engram::gather_kernel<8, false, int64_t>)
                            : (f8 ? engram::gather_kernel<4, true, int64_t> : engram::gather_kernel<4, false, int64_t>);
-    ENGRAM_CUDA_TRY(launch_ex(pdl, kern, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream, idx,
-                              reinterpret_cast<uint4 *>(m), p),
-                    "gather_kernel launch");
+    kern<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(idx, reinterpret_cast<uint4 *>(m), p);
+    ENGRAM_LAUNCHED("gather_kernel launch");
     return ENGRAM_OK;
 }
 
@@ -788,11 +785,9 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
     if (k4d3 && scal != nullptr && conv_state == nullptr) {
         // scalars once per (token, branch) instead of once per (CTA, halo-extended chunk)
         const int64_t items = static_cast<int64_t>(B) * T * p.M;
-        // programmatic launches (the projection before them belongs to the same call)
-        ENGRAM_CUDA_TRY(launch_pdl(engram::gate_scalars_kernel, dim3(static_cast<unsigned>((items * 8 + 255) / 256)),
-                                   dim3(256), 0, stream, static_cast<const float4 *>(part), static_cast<int64_t>(B) * T,
-                                   n_tiles, p.n_key_tiles, p.M, d_h, p.eps, p.inv_sqrt_d, scal),
-                        "gate_scalars_kernel launch");
+        engram::gate_scalars_kernel<<<static_cast<unsigned>((items * 8 + 255) / 256), 256, 0, stream>>>(
+            part, static_cast<int64_t>(B) * T, n_tiles, p.n_key_tiles, p.M, d_h, p.eps, p.inv_sqrt_d, scal);
+        ENGRAM_LAUNCHED("gate_scalars_kernel launch");
         p.scal = scal;
     }
     if (p.scal != nullptr) {
@@ -820,7 +815,8 @@ int launch_gate_conv(const engram_plan *plan, const engram_weights *w, const uin
                    : best_g == 8  ? (dl ? engram::gate_stream_kernel<8, true> : engram::gate_stream_kernel<8, false>)
                    : best_g == 4  ? (dl ? engram::gate_stream_kernel<4, true> : engram::gate_stream_kernel<4, false>)
                                   : (dl ? engram::gate_stream_kernel<1, true> : engram::gate_stream_kernel<1, false>);
-        ENGRAM_CUDA_TRY(launch_pdl(k, grid, dim3(engram::kStreamThreads), 0, stream, p), "gate_stream_kernel launch");
+        k<<<grid, engram::kStreamThreads, 0, stream>>>(p);
+        ENGRAM_LAUNCHED("gate_stream_kernel launch");
         return ENGRAM_OK;
     }
     if (fast) engram::gate_conv_k4d3_kernel<kChain><<<grid, threads, 0, stream>>>(p);
@@ -1405,13 +1401,13 @@ int engram_forward(const engram_plan *plan, const engram_weights *w, const void 
                                reinterpret_cast<uint32_t *>(ws + L.unique), reinterpret_cast<int32_t *>(ws + L.n_unique),
                                stream)) != ENGRAM_OK)
             return rc;
-        if ((rc = launch_gather(plan, sidx, stage_ptr, n_tok, m, stream, n_tok, true)) != ENGRAM_OK) return rc;
+        if ((rc = launch_gather(plan, sidx, stage_ptr, n_tok, m, stream, n_tok)) != ENGRAM_OK) return rc;
     } else if (fp.row_order) {
         if ((rc = launch_gather_ordered(plan, idx, tables, n_tok, m, reinterpret_cast<uint32_t *>(ws + L.order_count),
                                         reinterpret_cast<uint32_t *>(ws + L.order_cursor),
                                         reinterpret_cast<uint2 *>(ws + L.order), stream)) != ENGRAM_OK)
             return rc;
-    } else if ((rc = launch_gather(plan, idx, tables, n_tok, m, stream, 0, true)) != ENGRAM_OK) {
+    } else if ((rc = launch_gather(plan, idx, tables, n_tok, m, stream)) != ENGRAM_OK) {
         return rc;
     }
     bool history_done = false;

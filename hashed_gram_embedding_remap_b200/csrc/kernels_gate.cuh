@@ -197,8 +197,6 @@ __global__ void __launch_bounds__(256) gate_scalars_kernel(const float4 *__restr
                                                            int32_t n_tiles, int32_t n_key_tiles, int32_t M,
                                                            int32_t d_h, float eps, float inv_sqrt_d,
                                                            float2 *__restrict__ scal) {
-    pdl_launch_dependents();   // the gate kernel may load its conv taps now
-    pdl_wait();                // the partial sums come from the projection before this kernel
     const int64_t gt = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t item = gt >> 3;          // (token, branch)
     const int sub = static_cast<int>(gt & 7);
@@ -531,11 +529,14 @@ __global__ void __launch_bounds__(kStreamThreads, kStreamMinBlocks) gate_stream_
     const int t1 = min(p.T, t0 + TC);
     const int lo = t0 - R;
     const int64_t row0 = static_cast<int64_t>(b) * p.T;
+    for (int i = threadIdx.x; i < TC + R; i += kStreamThreads) {
+        const int t = lo + i;
+        s_sc[i] = (t >= 0 && t < t1) ? __ldg(p.scal + (row0 + t) * p.M + br) : make_float2(0.f, 0.f);
+    }
+    __syncthreads();
     const int q = slice * kStreamThreads + threadIdx.x;
-    const bool active = q < p.d_h / 4;
-    const int c = active ? q * 4 : 0;
-    // the conv taps and gains do not depend on the kernels before this one: loaded before the
-    // wait (programmatic launch behind the scalars kernel)
+    if (q >= p.d_h / 4) return;
+    const int c = q * 4;
     float2 w[4][2];   // [tap][channel pair] = conv tap x gamma_c
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -547,13 +548,6 @@ __global__ void __launch_bounds__(kStreamThreads, kStreamMinBlocks) gate_stream_
         w[2][k] = make_float2(bf16_lo(ww.y) * g0, bf16_lo(ww.w) * g1);
         w[3][k] = make_float2(bf16_hi(ww.y) * g0, bf16_hi(ww.w) * g1);
     }
-    pdl_wait();   // the gate scalars and v come from the kernels before this one
-    for (int i = threadIdx.x; i < TC + R; i += kStreamThreads) {
-        const int t = lo + i;
-        s_sc[i] = (t >= 0 && t < t1) ? __ldg(p.scal + (row0 + t) * p.M + br) : make_float2(0.f, 0.f);
-    }
-    __syncthreads();
-    if (!active) return;
     const uint16_t *vbase = p.v + row0 * p.d_h + c;
     const int64_t hoff = (row0 * p.M + br) * p.d_h + c;
     float *dbase = DELTA ? p.delta + hoff : nullptr;

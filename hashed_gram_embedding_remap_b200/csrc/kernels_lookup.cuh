@@ -102,7 +102,6 @@ __global__ void __launch_bounds__(256) hash_kernel(const int32_t *__restrict__ i
                                                    uint32_t *__restrict__ idx,
                                                    int32_t *__restrict__ xr_out,
                                                    const __grid_constant__ HashParams p) {
-    pdl_launch_dependents();   // the gather may be scheduled now (it waits for this kernel)
     const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t n_tok = static_cast<int64_t>(p.B) * p.T;
     if (n >= n_tok) return;
@@ -240,7 +239,6 @@ template <int UNROLL, bool FP8, typename Idx>
 __global__ void __launch_bounds__(256) gather_kernel(const uint32_t *__restrict__ idx, uint4 *__restrict__ m,
                                                      const __grid_constant__ GatherParams p) {
     pdl_launch_dependents();   // the projection may prefetch its weight tiles while this drains
-    pdl_wait();                // the row ids come from the hash kernel before this one
     const Idx total = static_cast<Idx>(p.n_tok * p.chunks_per_tok);
     const Idx stride = static_cast<Idx>(gridDim.x) * blockDim.x;
     for (Idx base = static_cast<Idx>(blockIdx.x) * blockDim.x + threadIdx.x; base < total; base += stride * UNROLL) {

@@ -905,9 +905,9 @@ int launch_stage_small(const engram_plan *plan, const int32_t *ids, const int32_
     sp.H = H;
     sp.capacity = capacity;
     sp.chunks_per_row = plan->cfg.row_dim * table_elem_bytes(plan) / 16;
-    // few CTAs with many 16-byte reads in flight each (16 per thread, 64 KB per CTA): enough to
+    // few CTAs, one warp per distinct row (a row's reads all in flight at once): enough to
     // cover the host link's latency, while leaving the SMs to whatever the prefetch overlaps
-    // with (measured on a 64-token step over a 2560^3 GEMM: 8 CTAs hide the most; 16 or more
+    // with (measured on a 64-token step over a 2560^3 GEMM: 8 CTAs hide the most; more
     // shorten the prefetch a little but slow what it overlaps).  ENGRAM_STAGE_CTAS (>= 1)
     // overrides the CTA count (tuning); read once per process.
     static const int forced_ctas = [] {
@@ -915,13 +915,13 @@ int launch_stage_small(const engram_plan *plan, const int32_t *ids, const int32_
         const int v = e ? std::atoi(e) : 0;
         return v > 0 ? v : 0;
     }();
-    const int64_t total = static_cast<int64_t>(H) * B * T * sp.chunks_per_row;
-    constexpr int kUnroll = 16;
-    int64_t blocks = (total + engram::kStageSmallThreads * kUnroll - 1) / (engram::kStageSmallThreads * kUnroll);
+    const int64_t rows = static_cast<int64_t>(H) * B * T;   // distinct rows at most
+    constexpr int warps = engram::kStageSmallThreads / 32;
+    int64_t blocks = (rows + warps - 1) / warps;
     const int64_t cap = forced_ctas ? forced_ctas : 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    engram::stage_small_kernel<kUnroll><<<static_cast<unsigned>(blocks), engram::kStageSmallThreads, 0, stream>>>(
+    engram::stage_small_kernel<<<static_cast<unsigned>(blocks), engram::kStageSmallThreads, 0, stream>>>(
         ids, remap, history, idx, xr, staged_idx, unique_rows, n_unique, hp, sp);
     ENGRAM_LAUNCHED("stage_small_kernel launch");
     return ENGRAM_OK;

@@ -510,10 +510,9 @@ __global__ void __launch_bounds__(256) stage_copy_kernel(const __grid_constant__
 // stage_dedup_kernel and stage_copy_kernel: the same slots (distinct rows numbered in
 // increasing order per table) and the same staged bytes.
 constexpr int kStageSmallRows = 256;
-constexpr int kStageSmallThreads = 256;
-static_assert(kStageSmallRows % kStageSmallThreads == 0, "rows per thread");
+constexpr int kStageSmallThreads = 512;   // 16 warps: with 8 CTAs, one warp per distinct row of a 64 x 2 step
+constexpr int kStageChunksPerLane = 16;   // loads in flight per lane and row (rows of up to 8 KB in one pass)
 
-template <int UNROLL>
 __global__ void __launch_bounds__(kStageSmallThreads) stage_small_kernel(
     const int32_t *__restrict__ ids, const int32_t *__restrict__ remap, const int32_t *__restrict__ history,
     uint32_t *__restrict__ idx_out, int32_t *__restrict__ xr_out, uint32_t *__restrict__ staged_idx,
@@ -542,7 +541,7 @@ __global__ void __launch_bounds__(kStageSmallThreads) stage_small_kernel(
     }
     __syncthreads();
     // ... and its slot is the number of heads of the table with a smaller row id
-    uint32_t slot[kStageSmallRows / kStageSmallThreads];
+    uint32_t slot[(kStageSmallRows + kStageSmallThreads - 1) / kStageSmallThreads];
     for (int e = threadIdx.x, k = 0; e < rows; e += blockDim.x, ++k) {
         const int h = e % H;
         const uint32_t r = s_row[e];
@@ -567,41 +566,39 @@ __global__ void __launch_bounds__(kStageSmallThreads) stage_small_kernel(
                 unique_rows[static_cast<int64_t>(h) * sp.capacity + i] = s_uniq[h * n_tok + i];
         if (threadIdx.x < H) n_unique[threadIdx.x] = s_nu[threadIdx.x];
     }
-    // copy the distinct rows: chunk c of slot s of table h, grid-wide
-    const int64_t per_table = static_cast<int64_t>(n_tok) * sp.chunks_per_row;
-    const int64_t total = per_table * H;
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < total;
-         base += stride * UNROLL) {
-        uint4 val[UNROLL];
-        int64_t dst[UNROLL];
-        int hh[UNROLL];
+    // copy the distinct rows (table by table, slot order), one warp per row: lane l takes
+    // chunks l, l + 32, ... of its row, all of them in flight at once, so that a row costs one
+    // round trip over the host link; 32-bit index arithmetic only
+    const int lane = threadIdx.x & 31;
+    const int gw = static_cast<int>(blockIdx.x) * (kStageSmallThreads / 32) + static_cast<int>(threadIdx.x >> 5);
+    const int nw = static_cast<int>(gridDim.x) * (kStageSmallThreads / 32);
+    int n_rows = 0;
+    for (int h = 0; h < H; ++h) n_rows += s_nu[h];
+    const int cpr = sp.chunks_per_row;
+    for (int q = gw; q < n_rows; q += nw) {
+        int h = 0, sl = q;
+        while (sl >= s_nu[h]) {
+            sl -= s_nu[h];
+            ++h;
+        }
+        const uint32_t row = s_uniq[h * n_tok + sl];
+        const bool ok = row < sp.rows[h];
+        if (!ok && lane == 0) atomicOr(&g_engram_status, ENGRAM_STATUS_BAD_ROW);
+        const uint4 *src = reinterpret_cast<const uint4 *>(sp.table[h]) + static_cast<int64_t>(ok ? row : 0u) * cpr;
+        uint4 *dst = reinterpret_cast<uint4 *>(sp.staging[h]) + static_cast<int64_t>(sl) * cpr;
+        for (int c0 = 0; c0 < cpr; c0 += 32 * kStageChunksPerLane) {
+            uint4 val[kStageChunksPerLane];
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const int64_t i = base + u * stride;
-            dst[u] = -1;
-            hh[u] = 0;
-            if (i < total) {
-                const int h = static_cast<int>(i / per_table);
-                const int64_t r = i - h * per_table;
-                const int32_t sl = static_cast<int32_t>(r / sp.chunks_per_row);
-                const int32_t c = static_cast<int32_t>(r - static_cast<int64_t>(sl) * sp.chunks_per_row);
-                if (sl < s_nu[h]) {
-                    const uint32_t row = s_uniq[h * n_tok + sl];
-                    hh[u] = h;
-                    dst[u] = r;
-                    if (row < sp.rows[h]) {
-                        val[u] = reinterpret_cast<const uint4 *>(sp.table[h])[static_cast<int64_t>(row) * sp.chunks_per_row + c];
-                    } else {
-                        val[u] = make_uint4(0, 0, 0, 0);
-                        atomicOr(&g_engram_status, ENGRAM_STATUS_BAD_ROW);
-                    }
-                }
+            for (int u = 0; u < kStageChunksPerLane; ++u) {
+                const int c = c0 + u * 32 + lane;
+                val[u] = (ok && c < cpr) ? src[c] : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kStageChunksPerLane; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c < cpr) dst[c] = val[u];
             }
         }
-#pragma unroll
-        for (int u = 0; u < UNROLL; ++u)
-            if (dst[u] >= 0) reinterpret_cast<uint4 *>(sp.staging[hh[u]])[dst[u]] = val[u];
     }
 }
 

@@ -436,7 +436,8 @@ def run_engram(args, wl, world, rank, local):
     history = torch.from_numpy(wl.history()).to(dev) if wl.decode else None
     state = fill_gpu.filled((wl.B * M, wl.state_len, wl.d_h), wl.state_spec(), dev) if wl.decode else None
     flags = (E.ENGRAM_FLAG_SINGLE_CTA_MMA if args.single_cta_mma else 0) | (
-        E.ENGRAM_FLAG_ROW_ORDER_GATHER if args.row_order_gather else 0)
+        E.ENGRAM_FLAG_ROW_ORDER_GATHER if args.row_order_gather else 0) | (
+        E.ENGRAM_FLAG_BULK_GATHER if args.bulk_gather else 0)
     plan = E.Plan.from_workload(wl, flags=flags)
     path = E.engram_forward_path(plan, wl.B, wl.T)
     packed = E.pack_weights(plan, wk, wv) if args.packed and E.engram_packed_weights_size(plan) else None
@@ -712,7 +713,7 @@ def run_engram(args, wl, world, rank, local):
         "config": workload_config(wl, world),
         "weights_layout": "packed" if packed is not None else "row-major",
         "path": {"pair_mma": bool(path & E.ENGRAM_PATH_PAIR_MMA), "row_order_gather": bool(path & E.ENGRAM_PATH_ROW_ORDER),
-                 "path_bits": path},
+                 "bulk_gather": bool(path & E.ENGRAM_PATH_BULK_GATHER), "path_bits": path},
         "stages_ms": stage_ms, "hbm": hbm, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * launches_per_step,
         "launch_mode": "eager" if args.eager else "one CUDA graph of the K timed steps (stage times from a "
@@ -980,6 +981,8 @@ def main():
     ap.add_argument("--row-order-gather", action="store_true",
                     help="gather the rows grouped by row id: in-batch dedup of the HBM reads "
                          "(ENGRAM_FLAG_ROW_ORDER_GATHER)")
+    ap.add_argument("--bulk-gather", action="store_true",
+                    help="gather bf16 rows with bulk copies staged in shared memory (ENGRAM_FLAG_BULK_GATHER)")
     ap.add_argument("--oracle-tokens", type=int, default=128)
     ap.add_argument("--cpu-baseline-tokens", type=int, default=768)
     ap.add_argument("--oracle-procs", type=int, default=0,

@@ -32,11 +32,13 @@ ENGRAM_TABLES_HOST_MAPPED = 1
 ENGRAM_NOALLOC_SCRATCH_BYTES = 32 << 20
 ENGRAM_FLAG_SINGLE_CTA_MMA = 0x4
 ENGRAM_FLAG_ROW_ORDER_GATHER = 0x8
+ENGRAM_FLAG_BULK_GATHER = 0x10
 ENGRAM_PATH_FUSED_LOOKUP = 0x1
 ENGRAM_PATH_STAGED_ROWS = 0x2
 ENGRAM_PATH_SPLIT_K = 0x8
 ENGRAM_PATH_PAIR_MMA = 0x10
 ENGRAM_PATH_ROW_ORDER = 0x20
+ENGRAM_PATH_BULK_GATHER = 0x40
 ENGRAM_TABLE_BF16 = 0
 ENGRAM_TABLE_FP8_E4M3 = 1
 

@@ -161,6 +161,15 @@ cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t 
 bool fp8_tables(const engram_plan *plan) { return plan->cfg.table_dtype == ENGRAM_TABLE_FP8_E4M3; }
 int table_elem_bytes(const engram_plan *plan) { return fp8_tables(plan) ? 1 : 2; }
 
+// The gather as bulk copies staged in shared memory (ENGRAM_FLAG_BULK_GATHER): bf16 rows of at
+// most 8 KB (a ring of 8, or 32 rows under 2 KB, per one-warp CTA: at most 64 KB), list items
+// below 2^31.
+bool bulk_gather(const engram_plan *plan, int64_t n_tok) {
+    const int64_t row_bytes = static_cast<int64_t>(plan->cfg.row_dim) * 2;
+    return (plan->cfg.flags & ENGRAM_FLAG_BULK_GATHER) && !fp8_tables(plan) &&
+           n_tok * plan->num_tables < (int64_t(1) << 31) && row_bytes * (row_bytes >= 2048 ? 8 : 32) <= 64 * 1024;
+}
+
 // Width of the projection's N tile: the widest of 256/128/64 that divides d_h and still
 // gives at least two waves of CTAs on the GPU.  ENGRAM_PROJ_TILE_N (64, 128 or 256) forces a
 // width (for tuning and tests); it is read once per process.
@@ -626,6 +635,32 @@ int launch_gather(const engram_plan *plan, const uint32_t *idx, const void *cons
     p.chunks_per_tok = H * p.chunks_per_row;
     p.n_tok = n_tok;
     const int64_t total = n_tok * p.chunks_per_tok;
+    p.div_h = engram::make_fastdiv(static_cast<uint32_t>(H));
+    // ENGRAM_FLAG_BULK_GATHER (bf16 rows): bulk copies staged in shared memory
+    // (gather_bulk_kernel); otherwise, and for FP8 rows (dequantised on the way), the register
+    // gather below
+    if (bulk_gather(plan, n_tok)) {
+        const int64_t row_bytes = static_cast<int64_t>(p.chunks_per_row) * 16;
+        const int64_t items = n_tok * H;
+        const bool wide = row_bytes >= 2048;
+        using BK = void (*)(const uint32_t *, uint8_t *, const engram::GatherParams, int64_t);
+        const BK kern = wide ? engram::gather_bulk_kernel<8, 4> : engram::gather_bulk_kernel<32, 16>;
+        const int slots = wide ? 8 : 32;
+        const size_t smem = static_cast<size_t>(slots) * row_bytes;
+        ENGRAM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
+                        "cudaFuncSetAttribute(gather_bulk_kernel)");
+        int per_sm = 0;
+        ENGRAM_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32, smem),
+                        "cudaOccupancyMaxActiveBlocksPerMultiprocessor(gather_bulk_kernel)");
+        if (per_sm < 1) per_sm = 1;
+        int64_t grid = static_cast<int64_t>(sm_count()) * per_sm;
+        if (grid > items) grid = items;
+        const int64_t per_cta = (items + grid - 1) / grid;
+        grid = (items + per_cta - 1) / per_cta;
+        kern<<<static_cast<unsigned>(grid), 32, smem, stream>>>(idx, reinterpret_cast<uint8_t *>(m), p, per_cta);
+        ENGRAM_LAUNCHED("gather_bulk_kernel launch");
+        return ENGRAM_OK;
+    }
     // independent chunks per thread: ENGRAM_GATHER_UNROLL (4 or 8) overrides, for tuning
     static const int forced_unroll = [] {
         const char *e = std::getenv("ENGRAM_GATHER_UNROLL");
@@ -1103,7 +1138,7 @@ int engram_init(const engram_config *cfg, engram_plan *plan) {
     }
     if (c.table_dtype == ENGRAM_TABLE_FP8_E4M3 && c.row_dim % 16 != 0)
         return fail(ENGRAM_ERR_UNSUPPORTED, "FP8 tables need row_dim % 16 == 0");
-    if (c.flags & ~(ENGRAM_FLAG_SINGLE_CTA_MMA | ENGRAM_FLAG_ROW_ORDER_GATHER))
+    if (c.flags & ~(ENGRAM_FLAG_SINGLE_CTA_MMA | ENGRAM_FLAG_ROW_ORDER_GATHER | ENGRAM_FLAG_BULK_GATHER))
         return fail(ENGRAM_ERR_INVALID_ARG, "unknown flags 0x%x", c.flags);
 
     std::memset(plan, 0, sizeof *plan);
@@ -1472,6 +1507,7 @@ int engram_forward_path(const engram_plan *plan, int32_t B, int32_t T, uint32_t 
     if (fp.ps.k_splits > 1) bits |= ENGRAM_PATH_SPLIT_K;
     if (fp.pair) bits |= ENGRAM_PATH_PAIR_MMA;
     if (fp.row_order) bits |= ENGRAM_PATH_ROW_ORDER;
+    if (!fp.fused_lookup && !fp.row_order && bulk_gather(plan, n_tok)) bits |= ENGRAM_PATH_BULK_GATHER;
     *path = bits;
     return ENGRAM_OK;
 }

@@ -289,6 +289,83 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint32_t *__restrict_
     }
 }
 
+// m[n, h*d_e : (h+1)*d_e] = table_h[idx[n, h]] for bf16 rows, as bulk (TMA) copies staged in
+// shared memory: list item i = n * H + h is the i-th row-sized piece of m, so a CTA that takes
+// the consecutive items [c0, c1) fills one contiguous stretch of m.  One warp per CTA: the lanes
+// fetch the row ids 32 at a time, lane 0 issues a bulk load of each row into a ring of S slots
+// (bytes counted on the slot's mbarrier) and, L items behind, a bulk store of the landed row
+// into m; before a slot is refilled, the store that read it has finished reading (bulk
+// async-group wait).  No per-chunk index arithmetic, no register staging: the rows move
+// global -> shared -> global in one instruction each.  Rows beyond the table are written as
+// zeros and flagged (ENGRAM_STATUS_BAD_ROW); every wait is bounded.
+template <int S, int L>
+__global__ void __launch_bounds__(32) gather_bulk_kernel(const uint32_t *__restrict__ idx, uint8_t *__restrict__ m,
+                                                        const __grid_constant__ GatherParams p, int64_t per_cta) {
+    static_assert(L >= 1 && L < S, "lag");
+    extern __shared__ __align__(128) uint8_t g_smem[];
+    __shared__ uint64_t full[S];
+    __shared__ int s_abort;
+    pdl_launch_dependents();   // the projection may prefetch its weight tiles while this drains
+    const int lane = threadIdx.x;
+    const uint32_t rb = static_cast<uint32_t>(p.chunks_per_row) * 16u;   // row bytes
+    const int64_t n_items = p.n_tok * p.H;
+    const int64_t c0 = static_cast<int64_t>(blockIdx.x) * per_cta;
+    const int64_t c1 = min(n_items, c0 + per_cta);
+    if (c0 >= c1) return;
+    const int count = static_cast<int>(c1 - c0);
+    if (lane == 0) {
+        s_abort = 0;
+        for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    int issued = 0;       // lane 0: items whose slot was filled or armed so far
+    uint32_t batch = 0;   // lane l: row id of item c0 + 32 * (k / 32) + l
+    for (int k = 0; k < count + L; ++k) {
+        if (k < count) {
+            if ((k & 31) == 0) {
+                const int64_t it = c0 + k + lane;
+                batch = it < c1 ? __ldg(idx + it) : 0u;
+            }
+            const uint32_t row = __shfl_sync(0xffffffffu, batch, k & 31);
+            if (lane == 0 && !s_abort) {
+                const int s = k % S;
+                uint8_t *slot = g_smem + static_cast<int64_t>(s) * rb;
+                if (k >= S) bulk_wait_group_read<S - L - 1>();   // the store of item k - S has read the slot
+                const uint32_t i = static_cast<uint32_t>(c0 + k);
+                const uint32_t h = i - fastdiv(i, p.div_h) * p.div_h.d;
+                if (row < p.rows[h]) {
+                    mbar_arrive_expect_tx(&full[s], rb);
+                    bulk_load_1d(slot, static_cast<const uint8_t *>(p.table[h]) + static_cast<int64_t>(row) * rb, rb,
+                                 &full[s]);
+                } else {
+                    atomicOr(&g_engram_status, ENGRAM_STATUS_BAD_ROW);
+                    for (uint32_t o = 0; o < rb; o += 16) *reinterpret_cast<uint4 *>(slot + o) = make_uint4(0, 0, 0, 0);
+                    fence_proxy_async_smem();
+                    mbar_arrive(&full[s]);
+                }
+                issued = k + 1;
+            }
+        }
+        const int j = k - L;
+        if (lane == 0 && j >= 0 && j < count && !s_abort) {
+            const int s = j % S;
+            if (mbar_wait(&full[s], (j / S) & 1, &s_abort)) {
+                bulk_store_1d(m + (c0 + j) * rb, g_smem + static_cast<int64_t>(s) * rb, rb);
+                bulk_commit_group();
+            }
+        }
+    }
+    if (lane == 0) {
+        if (s_abort) {   // every issued load lands before the shared memory is released
+            volatile int never = 0;
+            for (int k = issued > S ? issued - S : 0; k < issued; ++k)
+                if (!mbar_wait(&full[k % S], (k / S) & 1, &never)) break;
+        }
+        bulk_wait_group_all();
+    }
+}
+
 // Steps 1-3 fused for device-resident tables: one warp per (token, table) row.  Lane 0
 // remaps the gram's ids and hashes them (same arithmetic as hash_kernel), the row id is
 // broadcast to the warp, and the 32 lanes copy the row into m as 16-byte chunks.  Used by

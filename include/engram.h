@@ -123,6 +123,9 @@ typedef struct engram_config {
 #define ENGRAM_FLAG_ROW_ORDER_GATHER 0x8 /* gather large batches grouped by row id: in-batch
                                             dedup of the HBM reads (see ENGRAM_PATH_ROW_ORDER);
                                             results are bit-identical either way */
+#define ENGRAM_FLAG_BULK_GATHER 0x10 /* gather bf16 rows (at most 8 KB) with bulk copies staged
+                                        in shared memory (see ENGRAM_PATH_BULK_GATHER), in
+                                        engram_gather and engram_forward; bit-identical */
 
 /* Validated config plus derived constants.  Caller-owned, plain data: engram_init fills
  * it, every other call reads it.  Do not modify its fields. */
@@ -375,13 +378,20 @@ int engram_gate_conv_noalloc(const engram_plan *plan, const engram_weights *w, c
  *                  HBM reads; m is bit-identical).  ENGRAM_FLAG_ROW_ORDER_GATHER set,
  *                  HBM-resident tables, the hash + gather path, at least 65,536 rows per
  *                  call.  Opt-in: m is then written in row order, as scattered slices, and on
- *                  B200 that costs more write bandwidth than the saved reads.
+ *                  B200 that costs more write bandwidth than the saved reads;
+ *   BULK_GATHER    the gather (in token order) moves each row global -> shared -> global with
+ *                  one bulk copy each way (TMA engine; a ring of rows per one-warp CTA, each
+ *                  CTA filling one contiguous stretch of m) instead of 16-byte register copies.
+ *                  ENGRAM_FLAG_BULK_GATHER set, bf16 rows of at most 8 KB, the hash + gather
+ *                  path.  Opt-in: on B200 the register gather keeps more bytes in flight per
+ *                  SM and is faster.
  * Otherwise the hash kernel writes the row ids and the gather kernel writes m in token order. */
 #define ENGRAM_PATH_FUSED_LOOKUP 0x1u
 #define ENGRAM_PATH_STAGED_ROWS 0x2u
 #define ENGRAM_PATH_SPLIT_K 0x8u
 #define ENGRAM_PATH_PAIR_MMA 0x10u
 #define ENGRAM_PATH_ROW_ORDER 0x20u
+#define ENGRAM_PATH_BULK_GATHER 0x40u
 int engram_forward_path(const engram_plan *plan, int32_t B, int32_t T, uint32_t *path);
 
 /* Wait for `stream` and report what the device found: ENGRAM_ERR_TIMEOUT if a pipeline wait

@@ -55,7 +55,7 @@ def _plan(**kw):
     (dict(heads_per_order=17), E.ENGRAM_ERR_UNSUPPORTED),
     (dict(flags=0x1), E.ENGRAM_ERR_INVALID_ARG),                                # retired flag bits
     (dict(flags=0x2), E.ENGRAM_ERR_INVALID_ARG),
-    (dict(flags=0x10), E.ENGRAM_ERR_INVALID_ARG),                               # unknown flag bit
+    (dict(flags=0x20), E.ENGRAM_ERR_INVALID_ARG),                               # unknown flag bit
     (dict(table_dtype=2), E.ENGRAM_ERR_INVALID_ARG),                            # unknown table dtype
     (dict(table_dtype=1, table_scale=(0.1, 0.1, 0.1, 0.0)), E.ENGRAM_ERR_INVALID_ARG),   # zero scale
     (dict(table_dtype=1, table_scale=(0.1, float("inf"), 0.1, 0.1)), E.ENGRAM_ERR_INVALID_ARG),
@@ -228,6 +228,15 @@ def test_forward_path_selection():
     p16r = _plan(heads_per_order=8, table_rows=[10007] * 16, row_dim=64, hidden_dim=2560, flags=RO)
     assert P(p16r, 1, 4096) == PAIR | ROW   # 65,536 rows: row order from here when asked for
     assert P(p16r, 1, 4095) == PAIR
+    # the bulk-copy gather, when asked for, on the hash + gather path only (not with row order,
+    # not with the fused decode lookup, not for FP8 rows)
+    BG = E.ENGRAM_FLAG_BULK_GATHER
+    pf = synth.get_workload("prefill20m")
+    assert P(E.Plan.from_workload(pf, flags=BG), pf.B, pf.T) == PAIR | E.ENGRAM_PATH_BULK_GATHER
+    assert P(E.Plan.from_workload(pf, flags=BG | RO), pf.B, pf.T) == PAIR | ROW
+    assert not P(E.Plan.from_workload(pf.with_(table_dtype="fp8"), flags=BG), pf.B, pf.T) & E.ENGRAM_PATH_BULK_GATHER
+    dec = synth.get_workload("decode20m")
+    assert not P(E.Plan.from_workload(dec, flags=BG), dec.B, 1) & E.ENGRAM_PATH_BULK_GATHER
     assert not P(_plan(hidden_dim=384), 8, 4096) & PAIR
     # decode-sized batches: one lookup kernel, split-K projection
     dec = synth.get_workload("decode20m")

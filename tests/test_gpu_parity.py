@@ -82,10 +82,18 @@ def test_hash_brute_force_small_vocab():
 
 
 # ------------------------------------------------------------------ step 3
-@pytest.mark.parametrize("K,d_e", [(2, 32), (3, 40), (8, 160)])
-def test_gather_bit_exact(K, d_e):
-    wl = small_workload(K=K, d_e=d_e, B=3, T=97)
-    plan = E.Plan.from_workload(wl)
+@pytest.mark.parametrize("bulk", [False, True])
+@pytest.mark.parametrize("K,d_e,B,T", [(2, 32, 3, 97), (3, 40, 3, 97), (8, 160, 3, 97), (1, 1024, 3, 97),
+                                       (1, 2560, 3, 97), (1, 2560, 8, 1000)])
+def test_gather_bit_exact(K, d_e, B, T, bulk):
+    """The register gather and the bulk-copy gather (ENGRAM_FLAG_BULK_GATHER: a 32-row ring per
+    one-warp CTA for rows under 2 KB, an 8-row ring for 1,024 and 2,560 columns, the second
+    the 20M-row geometry) against the oracle; 16,000 rows of 2,560 columns take 22 rows per
+    CTA, so the ring wraps."""
+    wl = small_workload(K=K, d_e=d_e, B=B, T=T)
+    plan = E.Plan.from_workload(wl, flags=E.ENGRAM_FLAG_BULK_GATHER if bulk else 0)
+    if bulk:
+        assert E.engram_forward_path(plan, B, T) & E.ENGRAM_PATH_BULK_GATHER or B * T * wl.H <= 16384
     tables_np = [synth.fill_bf16(wl.table_spec(h), (wl.primes[h], d_e)) for h in range(wl.H)]
     tables = [to_dev(t) for t in tables_np]
     idx_np = _idx_oracle(wl, wl.ids())
@@ -125,6 +133,22 @@ def test_bad_ids_and_rows_raise_status_not_faults():
     assert E.engram_device_status(clear=True) & E.ENGRAM_STATUS_BAD_ROW
     mh = to_host_u16(m).reshape(4, wl.H, wl.d_e)
     assert (mh[1, 2] == 0).all() and not (mh[0, 2] == 0).all()
+    assert E.engram_device_status(clear=True) == 0
+    # the bulk-copy gather (ENGRAM_FLAG_BULK_GATHER, 2,560-column rows): a row beyond the table
+    # is written as zeros and flagged, the other rows land
+    wb = small_workload(B=1, T=16, K=1, d_e=2560)
+    pb = E.Plan.from_workload(wb, flags=E.ENGRAM_FLAG_BULK_GATHER)
+    tb = [to_dev(synth.fill_bf16(wb.table_spec(h), (wb.primes[h], wb.d_e))) for h in range(wb.H)]
+    ib = torch.zeros((5, wb.H), dtype=torch.int32, device="cuda")
+    ib[3, 1] = wb.primes[1] + 7
+    ib[2, 0] = 5
+    mb = torch.full((5, wb.d_m), 3.0, dtype=torch.bfloat16, device="cuda")
+    E.engram_gather(pb, ib, tb, mb)
+    assert E.engram_device_status(clear=True) & E.ENGRAM_STATUS_BAD_ROW
+    mbh = to_host_u16(mb).reshape(5, wb.H, wb.d_e)
+    assert (mbh[3, 1] == 0).all()
+    assert np.array_equal(mbh[2, 0], synth.fill_rows_bf16(wb.table_spec(0), wb.d_e, np.array([5]))[0])
+    assert np.array_equal(mbh[4, 1], synth.fill_rows_bf16(wb.table_spec(1), wb.d_e, np.array([0]))[0])
     assert E.engram_device_status(clear=True) == 0
 
 

@@ -166,13 +166,6 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
         : "memory");
 }
-// Ask L2 to fetch one box of a 2-D tensor (no data reaches shared memory, nothing to wait for).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(x), "r"(y)
-                 : "memory");
-}
 
 // 1-D bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from global
 // into this CTA's shared memory, completion signalled on `bar` as bytes.  No multicast.

@@ -708,6 +708,8 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 320 ? 2 : 1) decode_fused_kernel
     float kt[8], v[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) kt[e] = v[e] = 0.f;
+    // in split order; unrolled by three so that the loads of three splits issue together
+#pragma unroll 3
     for (int ks = 0; ks < pp.k_splits; ++ks) {
         const float4 *src = reinterpret_cast<const float4 *>(acc + ks * split_stride);
         const float4 k0 = __ldg(src), k1 = __ldg(src + 1);

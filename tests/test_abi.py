@@ -29,6 +29,27 @@ def test_every_declared_symbol_is_exported():
         assert hasattr(lib, n), f"{n} declared in engram.h but not exported"
 
 
+def test_binding_constants_match_header():
+    """Every ENGRAM_* value the binding defines is the header's (status codes, flags, path
+    bits, limits): parsed from the #define lines, evaluated as plain integers."""
+    src = open(HEADER).read()
+    defs = {}
+    for name, val in re.findall(r"^#define (ENGRAM_[A-Z0-9_]+) +([^/\n]+)", src, flags=re.M):
+        v = val.strip().replace("u", "")
+        if re.fullmatch(r"[-+()0-9xa-fA-F <]+", v):
+            defs[name] = eval(v)   # integer literals, shifts and parentheses only
+    assert len(defs) >= 20
+    checked = 0
+    for name, v in defs.items():
+        if hasattr(_native, name):
+            assert getattr(_native, name) == v, name
+            checked += 1
+    assert checked >= 20
+    for name in ("ENGRAM_FLAG_ROW_ORDER_GATHER", "ENGRAM_FLAG_BULK_GATHER", "ENGRAM_PATH_ROW_ORDER",
+                 "ENGRAM_PATH_BULK_GATHER", "ENGRAM_PATH_PAIR_MMA"):
+        assert name in defs and hasattr(_native, name), name
+
+
 def test_struct_layouts_match_header():
     for name, cls in (("engram_config", _native.engram_config), ("engram_plan", _native.engram_plan),
                       ("engram_weights", _native.engram_weights), ("engram_row_cache", _native.engram_row_cache)):
